@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Throughput of the MoE-layer forward on B200, as one JSON line.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one moe_forward over one batch (route, permute, grouped GEMM 1/3 +
+SwiGLU, grouped GEMM 2, combine, statistics) of the named workload, default
+the Mixtral-8x7B-shaped prefill layer (T=4096, d=4096, E=8, d_ff=14336,
+top-2, bf16). Inputs are seeded synthetic tensors resident in HBM; between
+timed steps a 512 MiB buffer is written to flush L2 (the 2.8 GB of expert
+weights exceed L2 anyway). Steps are timed with CUDA events on the launching
+stream and summed; the job time is the max over ranks. With N > 1 every rank
+is an independent data-parallel replica over its own tokens (weak scaling)
+and the per-expert statistics are summed over ranks with one NCCL
+all-reduce per step.
+
+Also reported: end to end through host buffers (pinned H2D copy of x, the
+forward, D2H of the output, all inside the timed region), a per-stage
+breakdown, the roofline of the dominant kernel (grouped GEMM 1/3 + SwiGLU)
+against the measured bf16 peak, SM clocks sampled during the timed region,
+and (rank 0, N = 1) the CPU oracle timed on a bounded token sample.
+--impl reference times the CPU oracle alone (this build's reference arm).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_62_b200 import inputs  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s & TFLOP/s vs bf16 peak; small-batch decode HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+GEMM_SRC = os.path.join(ROOT, "mixture_experts_layer_62_b200", "csrc", "gemm_sm100.cu")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops_per_step(cfg, rows=None):
+    """Algorithmic FLOPs: 2 T k 3 d d_ff (routed) + 2 T d E (router) + shared."""
+    T, d, dff, E, k, dfs = cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg["d_ff_shared"]
+    R = T * k if rows is None else rows
+    return 2.0 * R * 3 * d * dff + 2.0 * T * d * E + 2.0 * T * 3 * d * dfs
+
+
+def up_flops(cfg, rows):
+    return 2.0 * rows * cfg["d"] * 2 * cfg["d_ff"] + 2.0 * cfg["T"] * cfg["d"] * 2 * cfg["d_ff_shared"]
+
+
+def down_flops(cfg, rows):
+    return 2.0 * rows * cfg["d_ff"] * cfg["d"] + 2.0 * cfg["T"] * cfg["d_ff_shared"] * cfg["d"]
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.2)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[3:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_index_for(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it still
+    describes the current kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as fh:
+        d = json.load(fh)
+    src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
+    ent = d.get(kernel, {}).get(workload)
+    if not ent or ent.get("source_sha256") != src_hash:
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_sample(cfg, L, n_tokens, seed=0):
+    """Time the CPU oracle: routing of all tokens plus the expert math of a
+    seeded sample of n_tokens tokens. Weights are copied to host numpy
+    before the clock starts."""
+    from oracle import moe_oracle as O
+    x = L["x"].float().cpu().numpy()
+    W_r = L["W_r"].float().cpu().numpy()
+    bias = None if L["bias"] is None else L["bias"].float().cpu().numpy()
+    rng = np.random.default_rng(seed)
+    tokens = np.sort(rng.choice(cfg["T"], size=min(n_tokens, cfg["T"]), replace=False))
+    W1 = {e: L["W1"][e].float().cpu().numpy() for e in range(cfg["E"])}
+    W3 = {e: L["W3"][e].float().cpu().numpy() for e in range(cfg["E"])}
+    W2 = {e: L["W2"][e].float().cpu().numpy() for e in range(cfg["E"])}
+    sh = {}
+    if cfg["d_ff_shared"]:
+        sh = {n: L[n].float().cpu().numpy() for n in ("Ws1", "Ws3", "Ws2")}
+    t0 = time.perf_counter()
+    O.moe_forward(x, W_r, W1, W3, W2, cfg["k"], cfg["cf"], bias, cfg["bias_mode"],
+                  sh.get("Ws1"), sh.get("Ws3"), sh.get("Ws2"), tokens=tokens)
+    dt = time.perf_counter() - t0
+    return len(tokens), dt
+
+
+def run_reference(args, cfg, rank):
+    """The reference arm: the CPU oracle as it stands, on a bounded sample of
+    the workload per step; rank 0 only."""
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=dev)
+    n = args.ref_sample
+    for i in range(args.warmup):
+        oracle_sample(cfg, L, n, seed=1000 + i)
+    total_tok, total_t = 0, 0.0
+    for i in range(args.steps):
+        nt, dt = oracle_sample(cfg, L, n, seed=i)
+        total_tok += nt
+        total_t += dt
+    value = total_tok / total_t
+    cores = blas_threads()
+    sample = f"per step: routing of all {cfg['T']} tokens + expert math of {n} seeded random tokens"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(cfg, args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(cfg, args):
+    return {"workload": args.workload, "T_per_gpu": cfg["T"], "d": cfg["d"], "d_ff": cfg["d_ff"], "E": cfg["E"],
+            "k": cfg["k"], "capacity_factor": cfg["cf"], "bias_mode": cfg["bias_mode"],
+            "d_ff_shared": cfg["d_ff_shared"], "global_batch_tokens": cfg["T"] * args.gpus,
+            "parallelism": f"dp{args.gpus} replicas" if args.gpus > 1 else "single GPU",
+            "l2": "512 MiB buffer written between timed steps (weights 2.8 GB also exceed L2)"}
+
+
+def launches_per_forward(cfg):
+    # transpose W_r, logits (SIMT or tensor-core), select, scan, permute+gather,
+    # grouped GEMM 1/3, grouped GEMM 2, combine
+    return 8 if cfg["T"] > 0 else 1
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_prefill")
+    ap.add_argument("--cpu-sample", type=int, default=256, help="tokens of the timed CPU-oracle sample")
+    ap.add_argument("--ref-sample", type=int, default=16, help="tokens per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("--gpus N > 1 must be launched with torch.distributed.run (one rank per GPU)")
+    cfg = inputs.workload(args.workload)
+
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import mixture_experts_layer_62_b200 as moe
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    # each rank: its own tokens (seed = rank), the same weights (seed 0)
+    L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=dev)
+    if rank > 0:
+        x_r, _, _ = inputs.make_routing_inputs(cfg, seed=rank)
+        L["x"] = x_r
+    L = {k_: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k_, v in L.items()}
+    p = moe.problem(cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg["cf"], cfg["dtype"], cfg["bias_mode"],
+                    cfg["d_ff_shared"])
+    layer = moe.MoELayer(p, L["W_r"], L["W1"], L["W3"], L["W2"], bias=L["bias"], Ws1=L["Ws1"], Ws3=L["Ws3"],
+                         Ws2=L["Ws2"])
+    x = L["x"]
+    E = cfg["E"]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    gstats = torch.zeros(2 * E, dtype=torch.float64, device=dev)
+
+    def step():
+        layer(x)
+        if world > 1:
+            # global load statistics: counts and sum of probabilities over ranks
+            cnt = layer.stats[32:32 + 4 * E].view(torch.int32).to(torch.float64)
+            psum = layer.stats[32 + 8 * E:32 + 12 * E].view(torch.float32).to(torch.float64) * cfg["T"]
+            torch.cat([cnt, psum], out=gstats)
+            dist.all_reduce(gstats)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- device-timed steps ----
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    sampler = ClockSampler(gpu_index_for(local_rank))
+    sampler.start()
+    torch.cuda.synchronize(dev)
+    barrier()
+    evs = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    job_ms = float(t.item())
+    st = layer.read_stats()
+    if st.status != moe.MOE_OK:
+        raise SystemExit(f"device status {st.status}: {moe.error_string(st.status)}")
+    tokens_total = cfg["T"] * world * args.steps
+    value = tokens_total / (job_ms / 1e3)
+    ms_per_step = job_ms / args.steps
+    rows = st.rows
+    tflops = flops_per_step(cfg, rows) * world * args.steps / (job_ms / 1e3) / 1e12
+
+    # ---- end to end through host buffers ----
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty((cfg["T"], cfg["d"]), dtype=x.dtype).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(3):
+        x_dev.copy_(x_host, non_blocking=True)
+        out = layer(x_dev)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_evs = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        out = layer(x_dev)
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e2e_evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = tokens_total / (float(t.item()) / 1e3)
+    nbytes = x.numel() * x.element_size()
+
+    # ---- per-stage breakdown (stage entry points, events between) ----
+    stages = breakdown(moe, p, cfg, L, dev, stream, flush, iters=max(3, min(10, args.steps)))
+
+    peaks, peak_src = load_peaks()
+    up_ms = stages["expert_up"]
+    achieved = up_flops(cfg, rows) / (up_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    down_ms = stages["expert_down"]
+    roofline = {"bound": "tensor", "kernel": "tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{peak_src} bf16 burst",
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
+                "traffic": traffic_for("tc_grouped_gemm_swiglu", args.workload),
+                "flops_per_launch": up_flops(cfg, rows), "ms_per_launch": up_ms,
+                "down_proj": {"achieved": down_flops(cfg, rows) / (down_ms / 1e3) / 1e12, "ms_per_launch": down_ms}}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg["dtype"] == "bf16" else "f32", "data": "synthetic",
+        "config": config_of(cfg, args), "tflops": tflops,
+        "tflops_frac_of_peak": tflops / peak,
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
+                "d2h_bytes_per_step": nbytes},
+        "gpu_launches": launches_per_forward(cfg) * args.steps,
+        "clocks": clocks,
+        "stages_ms": stages,
+        "routing": {"rows": rows, "dropped": st.dropped, "l_aux": st.l_aux, "max_over_mean": st.max_over_mean},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, dt = oracle_sample(cfg, L, args.cpu_sample)
+        line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"routing of all {cfg['T']} tokens + expert math of {n} seeded random "
+                                          f"tokens ({dt:.1f} s)"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def breakdown(moe, p, cfg, L, dev, stream, flush, iters):
+    """Average device time of each stage, each launched through its own entry point."""
+    T, d, dff, E, k, dfs = cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg["d_ff_shared"]
+    dt = L["x"].dtype
+    ws = moe.alloc_workspace(p, dev)
+    st = moe.alloc_stats(E, dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gate = torch.empty((T, k), dtype=torch.float32, device=dev)
+    pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+    indptr = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    row_token = torch.empty((T * k,), dtype=torch.int32, device=dev)
+    xp = torch.empty((T * k, d), dtype=dt, device=dev)
+    h = torch.empty((T * k, dff), dtype=dt, device=dev)
+    o = torch.empty((T * k, d), dtype=dt, device=dev)
+    hs = torch.empty((T, dfs), dtype=dt, device=dev) if dfs else None
+    s = torch.empty((T, d), dtype=dt, device=dev) if dfs else None
+    out = torch.empty((T, d), dtype=dt, device=dev)
+    names = ["route", "permute", "expert_up", "expert_down", "combine"]
+    acc = {n: 0.0 for n in names}
+
+    def run(record):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        evs[0].record(stream)
+        moe.route(p, L["x"], L["W_r"], idx, gate, st, ws, bias=L["bias"])
+        evs[1].record(stream)
+        moe.permute(p, L["x"], idx, pos, indptr, row_token, xp, st, ws)
+        evs[2].record(stream)
+        moe.expert_up(p, xp, indptr, L["W1"], L["W3"], h, ws, x=L["x"], Ws1=L["Ws1"], Ws3=L["Ws3"], hs=hs)
+        evs[3].record(stream)
+        moe.expert_down(p, h, indptr, L["W2"], o, ws, hs=hs, Ws2=L["Ws2"], s=s)
+        evs[4].record(stream)
+        moe.combine(p, o, pos, gate, out, s=s)
+        evs[5].record(stream)
+        return evs
+
+    for _ in range(2):
+        run(False)
+    allev = []
+    for _ in range(iters):
+        flush.fill_(1)
+        allev.append(run(True))
+    torch.cuda.synchronize(dev)
+    for evs in allev:
+        for i, n in enumerate(names):
+            acc[n] += evs[i].elapsed_time(evs[i + 1])
+    return {n: acc[n] / iters for n in names}
+
+
+if __name__ == "__main__":
+    main()

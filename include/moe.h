@@ -1,0 +1,224 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) forward pass of one sparse
+ * Mixture-of-Experts layer.
+ *
+ * The pass (citations name the source page and its section):
+ *   1. router logits z = W_r^T x            ("Week 2 Day 2: Mixture of Experts", §1.3)
+ *   2. top-k of a selection key, optionally z + b or softmax(z) + b; gates are
+ *      the softmax over the k selected raw logits   (same page §1.3, §4.2;
+ *      "Stanford CS336 Lecture 04", §2.3.3c)
+ *   3. expert histogram, expert-major prefix sum, capacity truncation and
+ *      permutation of token rows       ("Lecture 21 · LLM: Mixture-of-Experts", §3.3, §3.5)
+ *   4. grouped GEMM over E SwiGLU experts, Z = GroupGemm(data, indptr, weights)
+ *                                       (Lecture 21, §3.3; Week 2 Day 2, §2.1)
+ *   5. un-permute and gate-weighted sum (Lecture 21, §3.2 step 4), plus an
+ *      always-on shared expert           (Week 2 Day 2, §4.1)
+ *   6. load statistics f, P, L_aux = E sum f P (Week 2 Day 2, §3.2)
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *    16-byte aligned. The library allocates no device memory and keeps no
+ *    per-call state; scratch lives in a caller-provided workspace.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*, NULL
+ *    = legacy default stream). Results, including the status word of the
+ *    statistics block, are valid after the stream is synchronised.
+ *  - Return value: MOE_OK, or an MOE_ERR_* code for a host-side rejection
+ *    (nothing was launched) or a launch failure. Device-side failures (a
+ *    bounded wait that ran out) are reported in moe_stats.status.
+ *  - Element type of activations and expert weights: MOE_DTYPE_BF16 (bf16
+ *    storage, fp32 accumulation, tcgen05 tensor cores) or MOE_DTYPE_F32
+ *    (fp32 storage and arithmetic on CUDA cores). Router math is fp32 for
+ *    both; gates and the bias are fp32.
+ *  - Inputs are assumed finite; NaN handling is unspecified.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- error codes ------------------------------------------------------- */
+#define MOE_OK              0
+#define MOE_ERR_INVALID_ARG 1  /* null pointer, bad size, k<1, k>E, misaligned pointer */
+#define MOE_ERR_UNSUPPORTED 2  /* shape/dtype combination this build does not run */
+#define MOE_ERR_WORKSPACE   3  /* workspace missing or smaller than moe_workspace_size() */
+#define MOE_ERR_CUDA        4  /* a CUDA launch or driver call failed */
+#define MOE_ERR_TIMEOUT     5  /* device status only: a bounded wait gave up */
+
+/* ---- enums -------------------------------------------------------------- */
+#define MOE_DTYPE_F32  0
+#define MOE_DTYPE_BF16 1
+
+/* Selection key of the top-k (gates always use the raw logits z):
+ * NONE : key = z                       (Week 2 Day 2, §1.3)
+ * LOGIT: key = z + b                   (Week 2 Day 2, §4.2; tutorial route())
+ * PROB : key = softmax(z) + b          (CS336 Lecture 04, §2.3.3c)          */
+#define MOE_BIAS_NONE  0
+#define MOE_BIAS_LOGIT 1
+#define MOE_BIAS_PROB  2
+
+/* Limits of this build. */
+#define MOE_MAX_E 512
+#define MOE_MAX_K 16
+
+/* ---- problem description ----------------------------------------------- */
+typedef struct moe_problem {
+    int32_t T;                /* tokens (rows of x), >= 0                                 */
+    int32_t d;                /* model width                                              */
+    int32_t d_ff;             /* hidden width of a routed expert                          */
+    int32_t E;                /* routed experts, 1..MOE_MAX_E                             */
+    int32_t k;                /* experts per token, 1..min(E, MOE_MAX_K)                  */
+    float   capacity_factor;  /* C = ceil(cf*T*k/E) pairs per expert; <= 0: no limit     */
+    int32_t dtype;            /* MOE_DTYPE_*                                              */
+    int32_t bias_mode;        /* MOE_BIAS_*                                               */
+    int32_t d_ff_shared;      /* hidden width of the always-on shared expert, 0 = none    */
+} moe_problem;
+
+/* ---- statistics block (device memory, moe_stats_size(E) bytes) ----------
+ * A fixed header followed by four per-expert arrays:
+ *     int32_t counts[E]  pairs routed to e before capacity (c_e)
+ *     int32_t kept[E]    pairs kept after capacity
+ *     float   P[E]       mean full-softmax router probability of e
+ *     float   f[E]       c_e / (T k)
+ * L_aux = E * sum_e f_e P_e (the coefficient alpha is left to the caller;
+ * uniform routing gives 1). Reductions run in a fixed order, so repeated
+ * calls on the same inputs give bit-identical statistics.               */
+typedef struct moe_stats {
+    int32_t status;        /* MOE_OK, or MOE_ERR_TIMEOUT from a device-side bounded wait */
+    int32_t capacity;      /* C, or -1 when unlimited                                     */
+    int32_t rows;          /* R = sum_e kept_e (rows of the permuted buffer)             */
+    int32_t dropped;       /* sum_e (c_e - kept_e)                                        */
+    int32_t max_count;     /* max_e c_e                                                   */
+    float   l_aux;         /* E * sum_e f_e P_e                                           */
+    float   max_over_mean; /* max_e c_e / (T k / E)                                       */
+    int32_t reserved;
+} moe_stats;
+
+#define MOE_STATS_COUNTS(base, E) ((int32_t*)((char*)(base) + sizeof(moe_stats)))
+#define MOE_STATS_KEPT(base, E)   ((int32_t*)((char*)(base) + sizeof(moe_stats)) + (E))
+#define MOE_STATS_P(base, E)      ((float*)((int32_t*)((char*)(base) + sizeof(moe_stats)) + 2 * (E)))
+#define MOE_STATS_F(base, E)      ((float*)((int32_t*)((char*)(base) + sizeof(moe_stats)) + 3 * (E)))
+
+/* Bytes of the statistics block for E experts. */
+size_t moe_stats_size(int32_t E);
+
+/* ---- workspace ---------------------------------------------------------
+ * Scratch of moe_forward and of the stage entry points. The caller allocates
+ * moe_workspace_size(p) bytes of device memory (256-byte aligned) and keeps
+ * it alive until the stream has finished the call. Its contents need no
+ * initialisation. moe_workspace_layout() gives byte offsets of the
+ * intermediates that moe_forward leaves in it, for inspection:           */
+typedef struct moe_workspace_layout_t {
+    size_t idx;        /* int32 [T, k]  selected experts, descending key            */
+    size_t gate;       /* fp32  [T, k]  gates                                         */
+    size_t pos;        /* int32 [T, k]  permuted row of (t, j), -1 = dropped          */
+    size_t indptr;     /* int32 [E+1]   CSR row offsets over kept rows                */
+    size_t row_token;  /* int32 [T*k]   token of each permuted row (first R valid)    */
+    size_t logits;     /* fp32  [T, E]  router logits                                 */
+    size_t xp;         /* dtype [T*k, d]      permuted activations (first R rows)     */
+    size_t h;          /* dtype [T*k, d_ff]   SwiGLU hidden rows                      */
+    size_t o;          /* dtype [T*k, d]      expert outputs, permuted order          */
+    size_t hs;         /* dtype [T, d_ff_shared]  shared-expert hidden rows           */
+    size_t s;          /* dtype [T, d]        shared-expert output                    */
+    size_t total;      /* = moe_workspace_size(p)                                    */
+} moe_workspace_layout_t;
+
+size_t moe_workspace_size(const moe_problem* p);
+int    moe_workspace_layout(const moe_problem* p, moe_workspace_layout_t* out);
+
+/* ---- the whole layer ----------------------------------------------------
+ * moe_forward: out[t] = sum_{j<k, kept} gate[t,j] * FFN_{idx[t,j]}(x[t]) + FFN_shared(x[t]).
+ *   x     [T, d]          dtype
+ *   W_r   [d, E]          dtype (z = W_r^T x, Week 2 Day 2 §1.3)
+ *   bias  [E]             fp32, required unless bias_mode == MOE_BIAS_NONE
+ *   W1,W3 [E, d_ff, d]    dtype (nn.Linear layout: out x in)
+ *   W2    [E, d, d_ff]    dtype
+ *   Ws1,Ws3 [d_ff_shared, d], Ws2 [d, d_ff_shared]  dtype; NULL when d_ff_shared == 0
+ *   out   [T, d]          dtype, written fully (a fully dropped token gets 0)
+ *   stats moe_stats_size(E) bytes of device memory, written fully
+ * bf16 also requires d % 64 == 0, d_ff % 64 == 0, d_ff_shared % 64 == 0;
+ * f32 requires d % 4 == 0 and d_ff % 4 == 0. Otherwise MOE_ERR_UNSUPPORTED. */
+int moe_forward(const moe_problem* p,
+                const void* x, const void* W_r, const float* bias,
+                const void* W1, const void* W3, const void* W2,
+                const void* Ws1, const void* Ws3, const void* Ws2,
+                void* out, void* stats,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- stage entry points (the same kernels moe_forward launches) --------- */
+
+/* Router: logits (fp32, accumulated in fp32), selection key, top-k with the
+ * lowest index winning ties, gates, and the statistics counts/P/f/L_aux
+ * (kept/rows/dropped assume the capacity of p).
+ * logits [T, E] fp32 may be NULL. idx [T, k] int32, gate [T, k] fp32. */
+int moe_route(const moe_problem* p, const void* x, const void* W_r, const float* bias,
+              int32_t* idx, float* gate, float* logits, void* stats,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Routing from given fp32 logits [T, E] (selection, gates, statistics). */
+int moe_route_from_logits(const moe_problem* p, const float* logits, const float* bias,
+                          int32_t* idx, float* gate, void* stats,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Permutation (Lecture 21 §3.3 and §3.5): per-expert histogram, expert-major
+ * exclusive scan, rank of each pair in token order, capacity truncation,
+ * and gather of token rows: xp[pos[t,j]] = x[t] for kept pairs.
+ *   idx [T, k] int32 in; pos [T, k], indptr [E+1], row_token [T*k] int32 out;
+ *   xp [T*k, d] dtype out (rows >= R untouched).
+ * stats receives counts/kept/capacity/rows/dropped/max_count; P, f and
+ * l_aux are left as they are. */
+int moe_permute(const moe_problem* p, const void* x, const int32_t* idx,
+                int32_t* pos, int32_t* indptr, int32_t* row_token, void* xp, void* stats,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Expert FFNs over the permuted rows (Lecture 21 §3.3, Z = GroupGemm(data,
+ * indptr, weights)): for every expert e and row r in [indptr[e], indptr[e+1]):
+ *   o[r] = W2_e (SiLU(W1_e xp[r]) * (W3_e xp[r]))
+ * and, when d_ff_shared > 0, s[t] = Ws2 (SiLU(Ws1 x[t]) * (Ws3 x[t])).
+ *   xp [T*k, d], o [T*k, d] (rows >= indptr[E] untouched), x [T, d], s [T, d].
+ * indptr is read on the device; the host never waits for it; its entries must
+ * be non-decreasing with indptr[0] = 0 and indptr[E] <= T*k.
+ * stats (may be NULL): only the status word is written (MOE_OK, or
+ * MOE_ERR_TIMEOUT if a bounded wait of the tensor-core kernel gave up). */
+int moe_experts(const moe_problem* p, const void* xp, const int32_t* indptr,
+                const void* W1, const void* W3, const void* W2,
+                const void* x, const void* Ws1, const void* Ws3, const void* Ws2,
+                void* o, void* s, void* stats,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* The two halves of moe_experts, for per-stage timing and inspection:
+ *   moe_expert_up:   h[r] = SiLU(W1_e xp[r]) * (W3_e xp[r])      h  [T*k, d_ff]
+ *                    hs[t] = SiLU(Ws1 x[t]) * (Ws3 x[t])          hs [T, d_ff_shared]
+ *   moe_expert_down: o[r] = W2_e h[r];  s[t] = Ws2 hs[t]          o [T*k, d], s [T, d]
+ * Same indptr rules and workspace as moe_experts (the tile schedule is
+ * rebuilt from indptr by each call). */
+int moe_expert_up(const moe_problem* p, const void* xp, const int32_t* indptr,
+                  const void* W1, const void* W3, const void* x, const void* Ws1, const void* Ws3,
+                  void* h, void* hs, void* stats,
+                  void* workspace, size_t workspace_bytes, void* stream);
+int moe_expert_down(const moe_problem* p, const void* h, const int32_t* indptr, const void* W2,
+                    const void* hs, const void* Ws2, void* o, void* s, void* stats,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Un-permute and mix (Lecture 21 §3.2 step 4): for every token, in slot order
+ *   out[t] = sum_{j<k, pos[t,j] >= 0} gate[t,j] * o[pos[t,j]]  (+ s[t] if s != NULL)
+ * accumulated in fp32 and rounded once; no atomics. */
+int moe_combine(const moe_problem* p, const void* o, const int32_t* pos, const float* gate,
+                const void* s, void* out, void* stream);
+
+/* Human-readable text of an MOE_* code (static storage). */
+const char* moe_error_string(int code);
+
+/* Number of streaming multiprocessors the library sizes persistent grids for
+ * on the current device, or -1 on error. */
+int moe_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,517 @@
+// C ABI of the MoE-layer library: argument checks, workspace layout and the
+// launch sequence of the forward pass (route -> scan -> permute/gather ->
+// grouped GEMM 1/3 + SwiGLU -> grouped GEMM 2 -> combine). Every launch is
+// asynchronous on the caller's stream; the host never waits on the device.
+#include <cmath>
+
+#include "common.cuh"
+
+namespace moe {
+
+Layout make_layout(const moe_problem& p) {
+    const size_t T = p.T > 0 ? (size_t)p.T : 0, k = (size_t)p.k, E = (size_t)p.E;
+    const size_t d = (size_t)p.d, dff = (size_t)p.d_ff, dfs = (size_t)(p.d_ff_shared > 0 ? p.d_ff_shared : 0);
+    const size_t eb = elem_bytes(p.dtype);
+    const size_t NB = (T + kChunk - 1) / kChunk;
+    Layout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + (bytes > 0 ? bytes : 1), 256);
+        return o;
+    };
+    L.idx = take(T * k * 4);
+    L.gate = take(T * k * 4);
+    L.pos = take(T * k * 4);
+    L.indptr = take((E + 1) * 4);
+    L.row_token = take(T * k * 4);
+    L.logits = take(T * E * 4);
+    L.wrt = take(E * d * eb);
+    L.blockcnt = take(E * NB * 4);
+    L.blockoff = take(E * NB * 4);
+    L.blockpsum = take(NB * E * 4);
+    L.tiles13 = take((E + 2) * 4);
+    L.tiles2 = take((E + 2) * 4);
+    L.xp = take(T * k * d * eb);
+    L.h = take(T * k * dff * eb);
+    L.o = take(T * k * d * eb);
+    L.hs = take(T * dfs * eb);
+    L.s = take(dfs ? T * d * eb : 0);
+    L.total = off;
+    return L;
+}
+
+int device_sm_count() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+int check_problem(const moe_problem* p) {
+    if (p == nullptr) return MOE_ERR_INVALID_ARG;
+    if (p->T < 0 || p->d <= 0 || p->d_ff <= 0 || p->E < 1 || p->E > MOE_MAX_E || p->k < 1 ||
+        p->k > p->E || p->k > MOE_MAX_K || p->d_ff_shared < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (p->dtype != MOE_DTYPE_F32 && p->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+    if (p->bias_mode < MOE_BIAS_NONE || p->bias_mode > MOE_BIAS_PROB) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(p->capacity_factor)) return MOE_ERR_INVALID_ARG;
+    const long long rows = (long long)p->T * p->k;
+    if (rows * (long long)(p->d > p->d_ff ? p->d : p->d_ff) >= (1LL << 40) || rows >= (1LL << 30))
+        return MOE_ERR_UNSUPPORTED;
+    if (p->dtype == MOE_DTYPE_BF16) {
+        if (p->d % 64 || p->d_ff % 64 || p->d_ff_shared % 64) return MOE_ERR_UNSUPPORTED;
+    } else {
+        if (p->d % 8 || p->d_ff % 4 || p->d_ff_shared % 4) return MOE_ERR_UNSUPPORTED;
+    }
+    return MOE_OK;
+}
+
+// C = ceil(cf * T * k / E), computed in double from the float factor; -1 = none.
+int capacity_of(const moe_problem* p) {
+    double cf = (double)p->capacity_factor;
+    if (!(cf > 0.0)) return -1;
+    double c = std::ceil(cf * (double)p->T * (double)p->k / (double)p->E);
+    if (c > 2147483647.0) return -1;
+    return (int)c;
+}
+
+#define CK(expr)                                   \
+    do {                                           \
+        if ((expr) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+
+char* wsp(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
+
+// Router: logits (fp32) for all tokens into `logits`.
+int run_logits(const moe_problem* p, const void* x, const void* W_r, float* logits, const Layout& L,
+               void* ws, int32_t* status, cudaStream_t st) {
+    void* wrt = wsp(ws, L.wrt);
+    CK(launch_transpose_wr(p->dtype, W_r, wrt, p->d, p->E, st));
+    if (p->dtype == MOE_DTYPE_BF16 && p->E >= 64 && p->E % 32 == 0) {
+        // wide routers (e.g. 256 experts) are a real GEMM: tensor cores, fp32 out
+        TcArgs a = {};
+        a.mode = TC_F32OUT;
+        a.indptr = nullptr;
+        a.tiles = nullptr;
+        a.static_rows = p->T;
+        a.E = 1;
+        a.has_shared = 0;
+        a.T = p->T;
+        a.A[0] = x; a.a_rows[0] = p->T;
+        a.B[0][0] = wrt; a.B[0][1] = wrt; a.b_rows[0] = p->E; a.b_total_rows[0] = p->E;
+        a.N[0] = p->E; a.K[0] = p->d;
+        a.out[0] = logits;
+        a.status = status;
+        CK(launch_tc_gemm(a, st));
+    } else {
+        CK(launch_logits_simt(p->dtype, x, wrt, logits, p->T, p->d, p->E, st));
+    }
+    return MOE_OK;
+}
+
+// Grouped GEMM 1/3 with the SwiGLU epilogue (and the shared expert's).
+int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13, const void* W1,
+           const void* W3, const void* x, const void* Ws1, const void* Ws3, void* h, void* hs, int32_t* status,
+           cudaStream_t st) {
+    const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
+    const int rows = p->T * p->k;
+    if (p->dtype == MOE_DTYPE_BF16) {
+        TcArgs a = {};
+        a.mode = TC_SWIGLU;
+        a.indptr = indptr; a.tiles = tiles13;
+        a.E = p->E; a.has_shared = has_shared; a.T = p->T;
+        a.A[0] = xp; a.a_rows[0] = rows; a.A[1] = has_shared ? x : nullptr; a.a_rows[1] = p->T;
+        a.B[0][0] = W1; a.B[0][1] = W3; a.b_rows[0] = p->d_ff; a.b_total_rows[0] = p->E * p->d_ff;
+        a.B[1][0] = Ws1; a.B[1][1] = Ws3; a.b_rows[1] = p->d_ff_shared; a.b_total_rows[1] = p->d_ff_shared;
+        a.N[0] = p->d_ff; a.N[1] = p->d_ff_shared;
+        a.K[0] = p->d; a.K[1] = p->d;
+        a.out[0] = h; a.out[1] = hs;
+        a.status = status;
+        CK(launch_tc_gemm(a, st));
+    } else {
+        GroupedArgs a = {};
+        a.indptr = indptr; a.tiles = tiles13;
+        a.E = p->E; a.has_shared = has_shared; a.T = p->T;
+        a.A[0] = xp; a.a_rows[0] = rows; a.A[1] = x; a.a_rows[1] = p->T;
+        a.B[0][0] = W1; a.B[0][1] = W3; a.B[1][0] = Ws1; a.B[1][1] = Ws3;
+        a.N[0] = p->d_ff; a.N[1] = p->d_ff_shared;
+        a.K[0] = p->d; a.K[1] = p->d;
+        a.out[0] = h; a.out[1] = hs;
+        a.status = status;
+        CK(launch_simt_gemm(true, a, st));
+    }
+    return MOE_OK;
+}
+
+// Grouped GEMM 2 (down projection, and the shared expert's).
+int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const int32_t* tiles2, const void* W2,
+             const void* hs, const void* Ws2, void* o, void* s, int32_t* status, cudaStream_t st) {
+    const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
+    const int rows = p->T * p->k;
+    if (p->dtype == MOE_DTYPE_BF16) {
+        TcArgs b = {};
+        b.mode = TC_PLAIN;
+        b.indptr = indptr; b.tiles = tiles2;
+        b.E = p->E; b.has_shared = has_shared; b.T = p->T;
+        b.A[0] = h; b.a_rows[0] = rows; b.A[1] = has_shared ? hs : nullptr; b.a_rows[1] = p->T;
+        b.B[0][0] = W2; b.B[0][1] = W2; b.b_rows[0] = p->d; b.b_total_rows[0] = p->E * p->d;
+        b.B[1][0] = Ws2; b.B[1][1] = Ws2; b.b_rows[1] = p->d; b.b_total_rows[1] = p->d;
+        b.N[0] = p->d; b.N[1] = p->d;
+        b.K[0] = p->d_ff; b.K[1] = p->d_ff_shared;
+        b.out[0] = o; b.out[1] = s;
+        b.status = status;
+        CK(launch_tc_gemm(b, st));
+    } else {
+        GroupedArgs b = {};
+        b.indptr = indptr; b.tiles = tiles2;
+        b.E = p->E; b.has_shared = has_shared; b.T = p->T;
+        b.A[0] = h; b.a_rows[0] = rows; b.A[1] = hs; b.a_rows[1] = p->T;
+        b.B[0][0] = W2; b.B[0][1] = nullptr; b.B[1][0] = Ws2; b.B[1][1] = nullptr;
+        b.N[0] = p->d; b.N[1] = p->d;
+        b.K[0] = p->d_ff; b.K[1] = p->d_ff_shared;
+        b.out[0] = o; b.out[1] = s;
+        b.status = status;
+        CK(launch_simt_gemm(false, b, st));
+    }
+    return MOE_OK;
+}
+
+int run_experts(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13,
+                const int32_t* tiles2, const void* W1, const void* W3, const void* W2, const void* x,
+                const void* Ws1, const void* Ws3, const void* Ws2, void* h, void* hs, void* o, void* s,
+                int32_t* status, cudaStream_t st) {
+    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st);
+    if (rc != MOE_OK) return rc;
+    return run_down(p, h, indptr, tiles2, W2, hs, Ws2, o, s, status, st);
+}
+
+void schedule_sizes(const moe_problem* p, int& tile_m, int& nt13, int& nt2, int& nt13s, int& nt2s) {
+    if (p->dtype == MOE_DTYPE_BF16) {
+        tile_m = kTcTileM;
+        int c13 = tc_out_cols_per_tile(TC_SWIGLU), c2 = tc_out_cols_per_tile(TC_PLAIN);
+        nt13 = ceil_div(p->d_ff, c13);
+        nt2 = ceil_div(p->d, c2);
+        nt13s = ceil_div(p->d_ff_shared, c13);
+        nt2s = nt2;
+    } else {
+        tile_m = kSimtTileM;
+        nt13 = ceil_div(p->d_ff, kSimtTileN);
+        nt2 = ceil_div(p->d, kSimtTileN);
+        nt13s = ceil_div(p->d_ff_shared, kSimtTileN);
+        nt2s = nt2;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_stats_size(int32_t E) { return sizeof(moe_stats) + 16u * (size_t)(E > 0 ? E : 0); }
+
+size_t moe_workspace_size(const moe_problem* p) {
+    if (check_problem(p) != MOE_OK) return 0;
+    return make_layout(*p).total;
+}
+
+int moe_workspace_layout(const moe_problem* p, moe_workspace_layout_t* out) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    if (out == nullptr) return MOE_ERR_INVALID_ARG;
+    Layout L = make_layout(*p);
+    out->idx = L.idx; out->gate = L.gate; out->pos = L.pos; out->indptr = L.indptr;
+    out->row_token = L.row_token; out->logits = L.logits; out->xp = L.xp; out->h = L.h;
+    out->o = L.o; out->hs = L.hs; out->s = L.s; out->total = L.total;
+    return MOE_OK;
+}
+
+int moe_device_sm_count(void) { return device_sm_count(); }
+
+const char* moe_error_string(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_CUDA: return "CUDA launch or driver error";
+        case MOE_ERR_TIMEOUT: return "device-side bounded wait timed out";
+        default: return "unknown error";
+    }
+}
+
+int moe_forward(const moe_problem* p, const void* x, const void* W_r, const float* bias, const void* W1,
+                const void* W3, const void* W2, const void* Ws1, const void* Ws3, const void* Ws2, void* out,
+                void* stats, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    const bool shared = p->d_ff_shared > 0;
+    if (!x || !W_r || !W1 || !W3 || !W2 || !out || !stats) return MOE_ERR_INVALID_ARG;
+    if (p->bias_mode != MOE_BIAS_NONE && !bias) return MOE_ERR_INVALID_ARG;
+    if (shared && (!Ws1 || !Ws3 || !Ws2)) return MOE_ERR_INVALID_ARG;
+    for (const void* q : {x, W_r, W1, W3, W2, (const void*)out, (const void*)stats})
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (shared)
+        for (const void* q : {Ws1, Ws3, Ws2})
+            if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(*p);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int C = capacity_of(p);
+    int32_t* status = static_cast<int32_t*>(stats);
+    if (p->T == 0) {
+        CK(launch_zero_stats(stats, p->E, C, st));
+        return MOE_OK;
+    }
+    CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    float* logits = reinterpret_cast<float*>(wsp(workspace, L.logits));
+    int32_t* idx = reinterpret_cast<int32_t*>(wsp(workspace, L.idx));
+    float* gate = reinterpret_cast<float*>(wsp(workspace, L.gate));
+    int32_t* pos = reinterpret_cast<int32_t*>(wsp(workspace, L.pos));
+    int32_t* indptr = reinterpret_cast<int32_t*>(wsp(workspace, L.indptr));
+    int32_t* row_token = reinterpret_cast<int32_t*>(wsp(workspace, L.row_token));
+    int32_t* blockcnt = reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
+    int32_t* blockoff = reinterpret_cast<int32_t*>(wsp(workspace, L.blockoff));
+    float* blockpsum = reinterpret_cast<float*>(wsp(workspace, L.blockpsum));
+    int32_t* tiles13 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles13));
+    int32_t* tiles2 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles2));
+
+    rc = run_logits(p, x, W_r, logits, L, workspace, status, st);
+    if (rc != MOE_OK) return rc;
+    CK(launch_select(logits, bias, p->bias_mode, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum, st));
+    ScanArgs sa = {};
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
+    sa.blockcnt = blockcnt; sa.blockoff = blockoff; sa.blockpsum = blockpsum;
+    sa.indptr = indptr; sa.stats = stats;
+    sa.tiles13 = tiles13; sa.tiles2 = tiles2; sa.has_shared = shared ? 1 : 0;
+    schedule_sizes(p, sa.tile_m, sa.ntiles13, sa.ntiles2, sa.ntiles13_shared, sa.ntiles2_shared);
+    CK(launch_scan(sa, st));
+    void* xp = wsp(workspace, L.xp);
+    CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, C, pos, row_token, xp,
+                             st));
+    void* h = wsp(workspace, L.h);
+    void* o = wsp(workspace, L.o);
+    void* hs = shared ? wsp(workspace, L.hs) : nullptr;
+    void* s = shared ? wsp(workspace, L.s) : nullptr;
+    rc = run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st);
+    if (rc != MOE_OK) return rc;
+    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st));
+    return MOE_OK;
+}
+
+int moe_route(const moe_problem* p, const void* x, const void* W_r, const float* bias, int32_t* idx, float* gate,
+              float* logits, void* stats, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    if (!x || !W_r || !idx || !gate || !stats) return MOE_ERR_INVALID_ARG;
+    if (p->bias_mode != MOE_BIAS_NONE && !bias) return MOE_ERR_INVALID_ARG;
+    for (const void* q : {x, W_r, (const void*)stats})
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (logits && !aligned16(logits)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(*p);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int C = capacity_of(p);
+    if (p->T == 0) {
+        CK(launch_zero_stats(stats, p->E, C, st));
+        return MOE_OK;
+    }
+    int32_t* status = static_cast<int32_t*>(stats);
+    CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    float* lg = logits ? logits : reinterpret_cast<float*>(wsp(workspace, L.logits));
+    rc = run_logits(p, x, W_r, lg, L, workspace, status, st);
+    if (rc != MOE_OK) return rc;
+    int32_t* blockcnt = reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
+    float* blockpsum = reinterpret_cast<float*>(wsp(workspace, L.blockpsum));
+    CK(launch_select(lg, bias, p->bias_mode, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum, st));
+    ScanArgs sa = {};
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
+    sa.blockcnt = blockcnt; sa.blockoff = reinterpret_cast<int32_t*>(wsp(workspace, L.blockoff));
+    sa.blockpsum = blockpsum;
+    sa.indptr = reinterpret_cast<int32_t*>(wsp(workspace, L.indptr));
+    sa.stats = stats;
+    CK(launch_scan(sa, st));
+    return MOE_OK;
+}
+
+int moe_route_from_logits(const moe_problem* p, const float* logits, const float* bias, int32_t* idx, float* gate,
+                          void* stats, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    if (!logits || !idx || !gate || !stats) return MOE_ERR_INVALID_ARG;
+    if (p->bias_mode != MOE_BIAS_NONE && !bias) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(stats)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(*p);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int C = capacity_of(p);
+    if (p->T == 0) {
+        CK(launch_zero_stats(stats, p->E, C, st));
+        return MOE_OK;
+    }
+    CK(cudaMemsetAsync(stats, 0, sizeof(int32_t), st));
+    int32_t* blockcnt = reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
+    float* blockpsum = reinterpret_cast<float*>(wsp(workspace, L.blockpsum));
+    CK(launch_select(logits, bias, p->bias_mode, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum, st));
+    ScanArgs sa = {};
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
+    sa.blockcnt = blockcnt; sa.blockoff = reinterpret_cast<int32_t*>(wsp(workspace, L.blockoff));
+    sa.blockpsum = blockpsum;
+    sa.indptr = reinterpret_cast<int32_t*>(wsp(workspace, L.indptr));
+    sa.stats = stats;
+    CK(launch_scan(sa, st));
+    return MOE_OK;
+}
+
+int moe_permute(const moe_problem* p, const void* x, const int32_t* idx, int32_t* pos, int32_t* indptr,
+                int32_t* row_token, void* xp, void* stats, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    if (!idx || !pos || !indptr || !stats) return MOE_ERR_INVALID_ARG;
+    if (xp && (!x || !aligned16(x) || !aligned16(xp))) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(stats)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(*p);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int C = capacity_of(p);
+    if (p->T == 0) {
+        CK(launch_zero_stats(stats, p->E, C, st));
+        CK(cudaMemsetAsync(indptr, 0, sizeof(int32_t) * (size_t)(p->E + 1), st));
+        return MOE_OK;
+    }
+    CK(cudaMemsetAsync(stats, 0, sizeof(int32_t), st));
+    int32_t* blockcnt = reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
+    int32_t* blockoff = reinterpret_cast<int32_t*>(wsp(workspace, L.blockoff));
+    CK(launch_hist(idx, p->T, p->k, p->E, blockcnt, st));
+    ScanArgs sa = {};
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
+    sa.blockcnt = blockcnt; sa.blockoff = blockoff; sa.blockpsum = nullptr;
+    sa.indptr = indptr; sa.stats = stats;
+    CK(launch_scan(sa, st));
+    CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, C, pos, row_token, xp,
+                             st));
+    return MOE_OK;
+}
+
+int moe_experts(const moe_problem* p, const void* xp, const int32_t* indptr, const void* W1, const void* W3,
+                const void* W2, const void* x, const void* Ws1, const void* Ws3, const void* Ws2, void* o, void* s,
+                void* stats, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    const bool shared = p->d_ff_shared > 0;
+    if (!xp || !indptr || !W1 || !W3 || !W2 || !o) return MOE_ERR_INVALID_ARG;
+    if (shared && (!x || !Ws1 || !Ws3 || !Ws2 || !s)) return MOE_ERR_INVALID_ARG;
+    for (const void* q : {xp, W1, W3, W2, (const void*)o})
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (shared)
+        for (const void* q : {x, Ws1, Ws3, Ws2, (const void*)s})
+            if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(*p);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    if (p->T == 0) return MOE_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = stats ? static_cast<int32_t*>(stats)
+                            : reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
+    CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    int32_t* tiles13 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles13));
+    int32_t* tiles2 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles2));
+    int tile_m, nt13, nt2, nt13s, nt2s;
+    schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
+    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2, st));
+    void* h = wsp(workspace, L.h);
+    void* hs = shared ? wsp(workspace, L.hs) : nullptr;
+    return run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st);
+}
+
+// Shared prologue of the expert-stage entry points: checks, status reset and
+// the tile schedules built from indptr.
+static int expert_stage_setup(const moe_problem* p, void* stats, void* workspace, size_t workspace_bytes,
+                              cudaStream_t st, int32_t** status, int32_t** tiles13, int32_t** tiles2) {
+    const Layout L = make_layout(*p);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    *status = stats ? static_cast<int32_t*>(stats) : reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
+    *tiles13 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles13));
+    *tiles2 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles2));
+    return MOE_OK;
+}
+
+int moe_expert_up(const moe_problem* p, const void* xp, const int32_t* indptr, const void* W1, const void* W3,
+                  const void* x, const void* Ws1, const void* Ws3, void* h, void* hs, void* stats, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    const bool shared = p->d_ff_shared > 0;
+    if (!xp || !indptr || !W1 || !W3 || !h) return MOE_ERR_INVALID_ARG;
+    if (shared && (!x || !Ws1 || !Ws3 || !hs)) return MOE_ERR_INVALID_ARG;
+    for (const void* q : {xp, W1, W3, (const void*)h})
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (shared)
+        for (const void* q : {x, Ws1, Ws3, (const void*)hs})
+            if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t *status, *tiles13, *tiles2;
+    rc = expert_stage_setup(p, stats, workspace, workspace_bytes, st, &status, &tiles13, &tiles2);
+    if (rc != MOE_OK) return rc;
+    if (p->T == 0) return MOE_OK;
+    CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    int tile_m, nt13, nt2, nt13s, nt2s;
+    schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
+    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2, st));
+    return run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, shared ? hs : nullptr, status, st);
+}
+
+int moe_expert_down(const moe_problem* p, const void* h, const int32_t* indptr, const void* W2, const void* hs,
+                    const void* Ws2, void* o, void* s, void* stats, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    const bool shared = p->d_ff_shared > 0;
+    if (!h || !indptr || !W2 || !o) return MOE_ERR_INVALID_ARG;
+    if (shared && (!hs || !Ws2 || !s)) return MOE_ERR_INVALID_ARG;
+    for (const void* q : {h, W2, (const void*)o})
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (shared)
+        for (const void* q : {hs, Ws2, (const void*)s})
+            if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t *status, *tiles13, *tiles2;
+    rc = expert_stage_setup(p, stats, workspace, workspace_bytes, st, &status, &tiles13, &tiles2);
+    if (rc != MOE_OK) return rc;
+    if (p->T == 0) return MOE_OK;
+    CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    int tile_m, nt13, nt2, nt13s, nt2s;
+    schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
+    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2, st));
+    return run_down(p, h, indptr, tiles2, W2, shared ? hs : nullptr, Ws2, o, shared ? s : nullptr, status, st);
+}
+
+int moe_combine(const moe_problem* p, const void* o, const int32_t* pos, const float* gate, const void* s, void* out,
+                void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    if (!o || !pos || !gate || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(o) || !aligned16(out) || (s && !aligned16(s))) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st));
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+// Internal declarations shared by the kernels of the MoE-layer library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Tokens per permutation chunk: the histogram, the rank computation and the
+// gather all work on chunks of this many consecutive tokens.
+constexpr int kChunk = 32;
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline size_t elem_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+
+// Byte offsets of everything the library keeps in the caller's workspace.
+struct Layout {
+    size_t idx, gate, pos, indptr, row_token, logits, wrt;
+    size_t blockcnt, blockoff, blockpsum, tiles13, tiles2;
+    size_t xp, h, o, hs, s;
+    size_t total;
+};
+Layout make_layout(const moe_problem& p);
+
+// Kernel launchers (each returns cudaGetLastError() of its launches).
+cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, int E, cudaStream_t st);
+cudaError_t launch_logits_simt(int dtype, const void* x, const void* wrt, float* logits,
+                               int T, int d, int E, cudaStream_t st);
+cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
+                          int32_t* idx, float* gate, int32_t* blockcnt, float* blockpsum,
+                          cudaStream_t st);
+cudaError_t launch_hist(const int32_t* idx, int T, int k, int E, int32_t* blockcnt, cudaStream_t st);
+
+// Scan over per-chunk expert counts: per-expert totals, capacity, indptr,
+// chunk rank bases, statistics and (optionally) the tile schedules of the
+// two grouped GEMMs.
+struct ScanArgs {
+    int T, k, E, capacity;       // capacity < 0: unlimited
+    const int32_t* blockcnt;     // [E][NB]
+    int32_t* blockoff;           // [E][NB]
+    const float* blockpsum;      // [NB][E] or null (then P, f, l_aux untouched)
+    int32_t* indptr;             // [E+1]
+    void* stats;                 // moe_stats block
+    // tile schedules (null pointers: skipped)
+    int32_t* tiles13; int32_t* tiles2;
+    int tile_m, ntiles13, ntiles2, ntiles13_shared, ntiles2_shared, has_shared;
+};
+cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st);
+cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
+                            int ntiles13, int ntiles2, int ntiles13_shared, int ntiles2_shared,
+                            int32_t* tiles13, int32_t* tiles2, cudaStream_t st);
+cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
+                                  const int32_t* blockoff, const int32_t* indptr,
+                                  int T, int d, int E, int k, int capacity,
+                                  int32_t* pos, int32_t* row_token, void* xp, cudaStream_t st);
+cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const float* gate,
+                           const void* s, void* out, int T, int d, int k, cudaStream_t st);
+cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st);
+
+// fp32 grouped GEMM on CUDA cores (the fp32 path). Tile 64 x 64.
+constexpr int kSimtTileM = 64;
+constexpr int kSimtTileN = 64;
+struct GroupedArgs {
+    const int32_t* indptr;   // routed row offsets [E+1] (device)
+    const int32_t* tiles;    // cumulative tile counts [G+1] (device)
+    int E, has_shared, T;    // group E (if present) covers rows [0, T)
+    const void* A[2];        // routed A rows [*, K0], shared A rows [T, K1]
+    int a_rows[2];           // allocated rows of each A buffer
+    const void* B[2][2];     // [kind][0/1]: SWIGLU uses W1/W3, PLAIN uses [kind][0]
+    int N[2], K[2];          // output columns and reduction length per kind
+    void* out[2];            // [*, N0] and [T, N1]
+    int32_t* status;
+};
+cudaError_t launch_simt_gemm(bool swiglu, const GroupedArgs& a, cudaStream_t st);
+
+// bf16 grouped GEMM on tcgen05 tensor cores (sm_100a). Tile 128 x 256.
+constexpr int kTcTileM = 128;
+int tc_out_cols_per_tile(int mode);   // 128 for SWIGLU, 256 otherwise
+enum TcMode { TC_SWIGLU = 0, TC_PLAIN = 1, TC_F32OUT = 2 };
+struct TcArgs {
+    int mode;
+    const int32_t* indptr;   // null: one static group of `static_rows` rows
+    const int32_t* tiles;    // null with indptr == null
+    int static_rows;
+    int E, has_shared, T;
+    const void* A[2]; int a_rows[2];
+    const void* B[2][2]; int b_rows[2];   // rows of one expert's matrix in B
+    int b_total_rows[2];                  // rows of the whole B buffer
+    int N[2], K[2];
+    void* out[2];
+    int32_t* status;
+    long long timeout_ns;
+};
+cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
+
+int device_sm_count();
+
+}  // namespace moe

@@ -1,0 +1,526 @@
+// bf16 grouped GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Z = GroupGemm(data, indptr, weights) ("Lecture 21 · LLM: Mixture-of-Experts"
+// §3.3): group e multiplies the rows [indptr[e], indptr[e+1]) of the permuted
+// activations by expert e's weight matrix; one kernel runs every group
+// (§3.7: one kernel for all experts matters most when experts are small).
+// Modes:
+//   SWIGLU  D tile = [Xp W1_e^T | Xp W3_e^T] for 128 output columns; the
+//           epilogue writes H = SiLU(a) * b in bf16 ("Week 2 Day 2" §2.1).
+//   PLAIN   D tile = Xp W_e^T for 256 output columns, written as bf16.
+//   F32OUT  as PLAIN, written as fp32 (router logits).
+//
+// Design:
+//  * persistent grid (one CTA per SM), static tile list: tile ids are laid
+//    out group by group, and inside a group the 128-row M blocks vary
+//    fastest, so CTAs that run at the same time share one weight tile (read
+//    from HBM once, the others hit L2) and a group's activation rows stay in
+//    L2 across its N blocks;
+//  * warp 0: one thread issues TMA loads (A 128x64, B 2 x 128x64, 128-byte
+//    swizzle) into a 4-stage ring guarded by full/empty mbarriers;
+//  * warp 1: one thread issues tcgen05.mma (M=128, N=256, K=16, bf16 in,
+//    fp32 accumulate) into one of two TMEM accumulators (2 x 256 columns)
+//    and commits stage releases and accumulator completion to mbarriers;
+//  * warps 2-5: epilogue, tcgen05.ld of their 32 TMEM lanes, row masking of
+//    the ragged tail of a group, conversion and 16-byte stores; the next
+//    tile's MMAs run into the other accumulator meanwhile.
+//  * every mbarrier wait is bounded by a wall-clock limit; on expiry the CTA
+//    records MOE_ERR_TIMEOUT, drains its in-flight TMA and MMA work, frees
+//    TMEM and returns.
+// No cluster multicast anywhere: every CTA fetches its own tiles.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                       // 64 bf16 = 128 bytes = one swizzle row
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KB
+constexpr int B_HALF_BYTES = 128 * BK * 2;   // 16 KB
+constexpr int B_BYTES = 2 * B_HALF_BYTES;    // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int NUM_THREADS = 192;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+// ---- PTX wrappers -----------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane; the wait is in the
+// same statement so no register is read before the load has landed.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), descriptor
+// version 1, tile base 1024-byte aligned (base offset 0).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(1) << 16;              // leading byte offset (ignored for SW128 K-major)
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;      // stride byte offset
+    d |= static_cast<uint64_t>(1) << 46;              // version
+    d |= static_cast<uint64_t>(2) << 61;              // SWIZZLE_128B
+    return d;
+}
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, both K-major.
+constexpr uint32_t make_idesc(int M, int N) {
+    return (1u << 4)      // D format fp32
+         | (1u << 7)      // A format bf16
+         | (1u << 10)     // B format bf16
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+struct KParams {
+    const int32_t* indptr;
+    const int32_t* tiles;
+    int static_rows;
+    int E, has_shared, T;
+    int b_rows[2];
+    int N[2], K[2];
+    void* out[2];
+    int32_t* status;
+    long long timeout_ns;
+};
+
+struct Tile {
+    int kind, g, rows, row0, m_blk, n_blk, num_kb;
+};
+
+__device__ __forceinline__ int total_tiles(const KParams& p, int cols_per_tile) {
+    if (p.indptr == nullptr)
+        return ((p.static_rows + BM - 1) / BM) * ((p.N[0] + cols_per_tile - 1) / cols_per_tile);
+    return p.tiles[p.E + p.has_shared];
+}
+
+__device__ __forceinline__ Tile decode_tile(const KParams& p, int tile) {
+    Tile t;
+    if (p.indptr == nullptr) {
+        t.kind = 0; t.g = 0; t.rows = p.static_rows; t.row0 = 0;
+    } else {
+        int lo = 0, hi = p.E + p.has_shared;   // tiles[lo] <= tile < tiles[hi]
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (p.tiles[mid] <= tile) lo = mid; else hi = mid;
+        }
+        t.g = lo;
+        t.kind = lo >= p.E ? 1 : 0;
+        t.rows = t.kind ? p.T : p.indptr[lo + 1] - p.indptr[lo];
+        t.row0 = t.kind ? 0 : p.indptr[lo];
+        tile -= p.tiles[lo];
+    }
+    const int mt = (t.rows + BM - 1) / BM;
+    t.n_blk = tile / mt;
+    t.m_blk = tile % mt;
+    t.num_kb = (p.K[t.kind] + BK - 1) / BK;
+    return t;
+}
+
+struct SharedCtl {
+    uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// Wait for phase `parity` of `bar`; false if the CTA aborted or the limit ran out.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, SharedCtl* ctl,
+                                             const KParams& p) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) return false;
+        if (global_timer_ns() - t0 > static_cast<uint64_t>(p.timeout_ns)) {
+            *reinterpret_cast<volatile int*>(&ctl->abort_flag) = 1;
+            atomicExch(p.status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+// Drain wait used on the abort path: ignores the abort flag, still bounded.
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, const KParams& p) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > static_cast<uint64_t>(p.timeout_ns)) {
+            atomicExch(p.status, MOE_ERR_TIMEOUT);
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ float silu(float a) { return a / (1.f + __expf(-a)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                const __grid_constant__ CUtensorMap tmB00, const __grid_constant__ CUtensorMap tmB01,
+                const __grid_constant__ CUtensorMap tmB10, const __grid_constant__ CUtensorMap tmB11,
+                const KParams p) {
+    constexpr int COLS_PER_TILE = MODE == TC_SWIGLU ? 128 : 256;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SharedCtl* ctl = reinterpret_cast<SharedCtl*>(smem + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&ctl->tfull[a], 1);
+            mbar_init(&ctl->tempty[a], 4);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort_flag = 0;
+        fence_mbar_init();
+        prefetch_map(&tmA0); prefetch_map(&tmA1);
+        prefetch_map(&tmB00); prefetch_map(&tmB01);
+        prefetch_map(&tmB10); prefetch_map(&tmB11);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&ctl->tmem_base)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+    const int total = total_tiles(p, COLS_PER_TILE);
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_mask = 0, issued_ph = 0;
+            bool aborted = false;
+            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+                const Tile t = decode_tile(p, tile);
+                const CUtensorMap* ma = t.kind ? &tmA1 : &tmA0;
+                const CUtensorMap* mb0 = t.kind ? &tmB10 : &tmB00;
+                const CUtensorMap* mb1 = t.kind ? &tmB11 : &tmB01;
+                const int arow = t.row0 + t.m_blk * BM;
+                const int eoff = t.kind ? 0 : t.g * p.b_rows[0];
+                int brow0, brow1;
+                const CUtensorMap *mlo, *mhi;
+                if (MODE == TC_SWIGLU) {
+                    brow0 = eoff + t.n_blk * 128; brow1 = brow0; mlo = mb0; mhi = mb1;
+                } else {
+                    brow0 = eoff + t.n_blk * 256; brow1 = brow0 + 128; mlo = mb0; mhi = mb0;
+                }
+                for (int kb = 0; kb < t.num_kb; ++kb) {
+                    if (!wait_bounded(&ctl->empty[s], ph ^ 1u, ctl, p)) { aborted = true; break; }
+                    const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+                    mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
+                    tma_load_2d(sa, ma, &ctl->full[s], kb * BK, arow);
+                    tma_load_2d(sa + A_BYTES, mlo, &ctl->full[s], kb * BK, brow0);
+                    tma_load_2d(sa + A_BYTES + B_HALF_BYTES, mhi, &ctl->full[s], kb * BK, brow1);
+                    issued_mask |= 1u << s;
+                    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (aborted) {
+                // let every load this thread started land before the CTA exits
+                for (int st = 0; st < STAGES; ++st)
+                    if ((issued_mask >> st) & 1u) wait_drain(&ctl->full[st], (issued_ph >> st) & 1u, p);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc(BM, 256);
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t aph = 0;
+            bool aborted = false, issued_any = false;
+            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
+                const Tile t = decode_tile(p, tile);
+                if (!wait_bounded(&ctl->tempty[acc], aph ^ 1u, ctl, p)) { aborted = true; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
+                for (int kb = 0; kb < t.num_kb; ++kb) {
+                    if (!wait_bounded(&ctl->full[s], ph, ctl, p)) { aborted = true; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+                    const uint64_t adesc = sw128_desc(sa);
+                    const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc_mma(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    issued_any = true;
+                    tc_commit(&ctl->empty[s]);
+                    if (++s == STAGES) { s = 0; ph ^= 1u; }
+                }
+                if (aborted) break;
+                tc_commit(&ctl->tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) aph ^= 1u;
+            }
+            if (aborted && issued_any) {
+                // all MMAs of this thread must finish before TMEM is freed
+                tc_commit(&ctl->drain);
+                wait_drain(&ctl->drain, 0, p);
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int r = q * 32 + lane;            // accumulator row of this thread
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile(p, tile);
+            if (!wait_bounded(&ctl->tfull[acc], aph, ctl, p)) break;
+            tc_fence_after();
+            const int grow = t.m_blk * BM + r;
+            const bool valid = grow < t.rows;
+            const size_t orow = static_cast<size_t>(t.row0) + static_cast<size_t>(grow);
+            const int N = p.N[t.kind];
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                static_cast<uint32_t>(acc * ACC_COLS);
+            if (MODE == TC_SWIGLU) {
+                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 32) {
+                    uint32_t gv[32], uv[32];
+                    tmem_ld32(tb + c, gv);
+                    tmem_ld32(tb + 128 + c, uv);
+                    const int col = t.n_blk * 128 + c;
+                    if (valid && col < N) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
+                            float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
+                            packed[i] = pack_bf16(silu(g0) * u0, silu(g1) * u1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    }
+                }
+            } else if (MODE == TC_PLAIN) {
+                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tb + c, v);
+                    const int col = t.n_blk * 256 + c;
+                    if (valid && col < N) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            packed[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                        uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    }
+                }
+            } else {
+                float* out = static_cast<float*>(p.out[t.kind]) + orow * N;
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tb + c, v);
+                    const int col = t.n_blk * 256 + c;
+                    if (valid && col < N) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) aph ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ---- host side --------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encode() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// 2-D bf16 map over a [rows, cols] row-major matrix, box 64 columns x 128 rows,
+// 128-byte swizzle; reads outside the matrix return zeros.
+bool make_map(CUtensorMap* m, const void* base, int rows, int cols) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {BK, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const TcArgs& a, const KParams& kp, const CUtensorMap (&maps)[6], cudaStream_t st) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(tc_grouped_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    int grid = device_sm_count();
+    if (grid <= 0) return cudaErrorInvalidDevice;
+    tc_grouped_gemm<MODE><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                                maps[5], kp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int tc_out_cols_per_tile(int mode) { return mode == TC_SWIGLU ? 128 : 256; }
+
+cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
+    if (!get_encode()) return cudaErrorNotSupported;
+    CUtensorMap maps[6];
+    // A maps: [rows, K]; B maps: [total rows, K]. Unused slots reuse slot 0.
+    const int has1 = a.has_shared && a.A[1] != nullptr;
+    if (!make_map(&maps[0], a.A[0], a.a_rows[0], a.K[0])) return cudaErrorInvalidValue;
+    if (!make_map(&maps[1], has1 ? a.A[1] : a.A[0], has1 ? a.a_rows[1] : a.a_rows[0], has1 ? a.K[1] : a.K[0]))
+        return cudaErrorInvalidValue;
+    if (!make_map(&maps[2], a.B[0][0], a.b_total_rows[0], a.K[0])) return cudaErrorInvalidValue;
+    const void* b01 = a.mode == TC_SWIGLU ? a.B[0][1] : a.B[0][0];
+    if (!make_map(&maps[3], b01, a.b_total_rows[0], a.K[0])) return cudaErrorInvalidValue;
+    if (has1) {
+        if (!make_map(&maps[4], a.B[1][0], a.b_total_rows[1], a.K[1])) return cudaErrorInvalidValue;
+        const void* b11 = a.mode == TC_SWIGLU ? a.B[1][1] : a.B[1][0];
+        if (!make_map(&maps[5], b11, a.b_total_rows[1], a.K[1])) return cudaErrorInvalidValue;
+    } else {
+        maps[4] = maps[2];
+        maps[5] = maps[3];
+    }
+    KParams kp;
+    kp.indptr = a.indptr;
+    kp.tiles = a.tiles;
+    kp.static_rows = a.static_rows;
+    kp.E = a.E;
+    kp.has_shared = has1;
+    kp.T = a.T;
+    kp.b_rows[0] = a.b_rows[0]; kp.b_rows[1] = a.b_rows[1];
+    kp.N[0] = a.N[0]; kp.N[1] = a.N[1];
+    kp.K[0] = a.K[0]; kp.K[1] = a.K[1];
+    kp.out[0] = a.out[0]; kp.out[1] = a.out[1];
+    kp.status = a.status;
+    kp.timeout_ns = a.timeout_ns > 0 ? a.timeout_ns : 2000000000LL;
+    switch (a.mode) {
+        case TC_SWIGLU: return launch_mode<TC_SWIGLU>(a, kp, maps, st);
+        case TC_PLAIN: return launch_mode<TC_PLAIN>(a, kp, maps, st);
+        default: return launch_mode<TC_F32OUT>(a, kp, maps, st);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,284 @@
+// Permutation of token rows by expert ("Lecture 21 · LLM: Mixture-of-Experts"
+// §3.3: the N x E selection mask flattened expert-major, an exclusive prefix
+// sum giving every selected pair its destination row, indptr from the same
+// scan; §3.5: capacity C = ceil(k N / E x cf), overflow pairs dropped).
+//
+// The mask is never materialised. Per chunk of kChunk tokens the router (or
+// hist_kernel) counts pairs per expert; one block scans those counts in
+// expert-major order (e outer, chunk inner), which is the order of the
+// flattened mask; a pair's rank inside its expert is the scan value of its
+// chunk plus the number of earlier pairs of the same expert in the chunk.
+// No atomics decide any position, so the permutation is deterministic and
+// ranks follow token order.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kScanThreads = 1024;
+
+// Exclusive block-wide scan of one int per thread; returns the block total.
+__device__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int nw = blockDim.x >> 5;
+        int w = lane < nw ? warp_tot[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int n = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += n;
+        }
+        if (lane < nw) warp_tot[lane] = wi - w;   // exclusive warp offsets
+        if (lane == 31) warp_tot[32] = wi;
+    }
+    __syncthreads();
+    int excl = warp_tot[warp] + incl - v;
+    total = warp_tot[32];
+    __syncthreads();
+    return excl;
+}
+
+// Tile schedule of a grouped GEMM: tiles[g] = sum_{g' < g} mtiles(g') * ntiles(g').
+__device__ void build_schedule(const int* rows, int G, int E, int tile_m, int nt, int nt_shared,
+                               int32_t* tiles, int* warp_tot) {
+    int carry = 0;
+    for (int base = 0; base < G; base += blockDim.x) {
+        int g = base + threadIdx.x;
+        int v = 0;
+        if (g < G) v = ((rows[g] + tile_m - 1) / tile_m) * (g < E ? nt : nt_shared);
+        int tot;
+        int ex = block_exclusive_scan(v, warp_tot, tot);
+        if (g < G) tiles[g] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0) tiles[G] = carry;
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) {
+    __shared__ int warp_tot[33];
+    __shared__ int start[MOE_MAX_E + 1];
+    __shared__ int kept_s[MOE_MAX_E + 1];
+    __shared__ float fP[MOE_MAX_E];
+    const int E = a.E;
+    const long long n = (long long)E * NB;
+
+    // 1. global exclusive scan of blockcnt (expert-major), written to blockoff
+    {
+        const long long per = (n + kScanThreads - 1) / kScanThreads;
+        const long long lo = min(n, per * threadIdx.x), hi = min(n, lo + per);
+        int local = 0;
+        for (long long i = lo; i < hi; ++i) local += a.blockcnt[i];
+        int tot;
+        int run = block_exclusive_scan(local, warp_tot, tot);
+        for (long long i = lo; i < hi; ++i) {
+            int c = a.blockcnt[i];
+            a.blockoff[i] = run;
+            if (i % NB == 0) start[i / NB] = run;
+            run += c;
+        }
+        if (threadIdx.x == 0) start[E] = tot;
+    }
+    __syncthreads();
+    // 2. make the chunk bases relative to their expert's first pair
+    for (long long i = threadIdx.x; i < n; i += kScanThreads) a.blockoff[i] -= start[i / NB];
+
+    // 3. counts, capacity, kept and indptr over kept rows
+    int c = 0, kp = 0;
+    const int e = threadIdx.x;
+    if (e < E) {
+        c = start[e + 1] - start[e];
+        kp = a.capacity < 0 ? c : min(c, a.capacity);
+    }
+    int tot_kept;
+    int ex = block_exclusive_scan(e < E ? kp : 0, warp_tot, tot_kept);
+    if (e < E) {
+        a.indptr[e] = ex;
+        kept_s[e] = kp;
+    }
+    if (threadIdx.x == 0) a.indptr[E] = tot_kept;
+
+    moe_stats* st = (moe_stats*)a.stats;
+    int32_t* counts = MOE_STATS_COUNTS(a.stats, E);
+    int32_t* kept = MOE_STATS_KEPT(a.stats, E);
+    float* P = MOE_STATS_P(a.stats, E);
+    float* f = MOE_STATS_F(a.stats, E);
+    if (e < E) {
+        counts[e] = c;
+        kept[e] = kp;
+    }
+
+    // 4. P_e = mean router probability: one warp per expert, fixed order
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (a.blockpsum != nullptr) {
+        for (int ee = warp; ee < E; ee += kScanThreads / 32) {
+            float acc = 0.f;
+            for (int b = lane; b < NB; b += 32) acc += a.blockpsum[(size_t)b * E + ee];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) {
+                float Pe = a.T > 0 ? acc / (float)a.T : 0.f;
+                float fe = a.T > 0 ? (float)(start[ee + 1] - start[ee]) / ((float)a.T * (float)a.k) : 0.f;
+                P[ee] = Pe;
+                f[ee] = fe;
+                fP[ee] = fe * Pe;
+            }
+        }
+    }
+    __syncthreads();
+    // 5. header: fixed-order sums in one thread
+    if (threadIdx.x == 0) {
+        int dropped = 0, maxc = 0;
+        for (int ee = 0; ee < E; ++ee) {
+            int ce = start[ee + 1] - start[ee];
+            dropped += ce - kept_s[ee];
+            maxc = max(maxc, ce);
+        }
+        st->status = MOE_OK;
+        st->capacity = a.capacity;
+        st->rows = tot_kept;
+        st->dropped = dropped;
+        st->max_count = maxc;
+        float mean = a.T > 0 ? (float)a.T * (float)a.k / (float)E : 0.f;
+        st->max_over_mean = mean > 0.f ? (float)maxc / mean : 0.f;
+        if (a.blockpsum != nullptr) {
+            float s = 0.f;
+            for (int ee = 0; ee < E; ++ee) s += fP[ee];
+            st->l_aux = (float)E * s;
+        }
+        st->reserved = 0;
+    }
+    // 6. tile schedules of the grouped GEMMs
+    if (a.tiles13 != nullptr) {
+        __shared__ int rows[MOE_MAX_E + 1];
+        if (threadIdx.x < E) rows[threadIdx.x] = kept_s[threadIdx.x];
+        if (threadIdx.x == 0) rows[E] = a.T;
+        __syncthreads();
+        const int G = E + a.has_shared;
+        build_schedule(rows, G, E, a.tile_m, a.ntiles13, a.ntiles13_shared, a.tiles13, warp_tot);
+        __syncthreads();
+        build_schedule(rows, G, E, a.tile_m, a.ntiles2, a.ntiles2_shared, a.tiles2, warp_tot);
+    }
+}
+
+cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st) {
+    int NB = ceil_div(a.T, kChunk);
+    scan_kernel<<<1, kScanThreads, 0, st>>>(a, NB);
+    return cudaGetLastError();
+}
+
+// Tile schedule from a given indptr (the standalone expert stage).
+__global__ void __launch_bounds__(kScanThreads)
+schedule_kernel(const int32_t* __restrict__ indptr, int E, int T, int has_shared, int tile_m,
+                int nt13, int nt2, int nt13s, int nt2s, int32_t* tiles13, int32_t* tiles2) {
+    __shared__ int warp_tot[33];
+    __shared__ int rows[MOE_MAX_E + 1];
+    for (int g = threadIdx.x; g < E; g += blockDim.x) rows[g] = indptr[g + 1] - indptr[g];
+    if (threadIdx.x == 0) rows[E] = T;
+    __syncthreads();
+    const int G = E + has_shared;
+    build_schedule(rows, G, E, tile_m, nt13, nt13s, tiles13, warp_tot);
+    __syncthreads();
+    build_schedule(rows, G, E, tile_m, nt2, nt2s, tiles2, warp_tot);
+}
+
+cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
+                            int ntiles13, int ntiles2, int ntiles13_shared, int ntiles2_shared,
+                            int32_t* tiles13, int32_t* tiles2, cudaStream_t st) {
+    schedule_kernel<<<1, kScanThreads, 0, st>>>(indptr, E, T, has_shared, tile_m, ntiles13, ntiles2,
+                                                ntiles13_shared, ntiles2_shared, tiles13, tiles2);
+    return cudaGetLastError();
+}
+
+// Ranks, destinations and the row gather. One block per chunk.
+// Gather: xp[pos[t, j]] = x[t] for every kept pair, 16-byte vectors; each
+// source vector is read once and written to all of the token's kept rows.
+__global__ void __launch_bounds__(256)
+permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
+                      const int32_t* __restrict__ blockoff, const int32_t* __restrict__ indptr,
+                      int Tn, int nvec, int E, int k, int capacity,
+                      int32_t* __restrict__ pos, int32_t* __restrict__ row_token,
+                      uint4* __restrict__ xp) {
+    __shared__ int sidx[kChunk][MOE_MAX_K];
+    __shared__ int spos[kChunk][MOE_MAX_K];
+    const int chunk = blockIdx.x, NB = gridDim.x;
+    const int t0 = chunk * kChunk;
+    const int ntok = min(kChunk, Tn - t0);
+    for (int i = threadIdx.x; i < ntok * k; i += blockDim.x)
+        sidx[i / k][i % k] = idx[(size_t)t0 * k + i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < ntok * k; i += blockDim.x) {
+        const int q = i / k, j = i % k;
+        const int e = sidx[q][j];
+        if (e < 0 || e >= E) {   // not an expert: the pair takes no row
+            spos[q][j] = -1;
+            pos[(size_t)(t0 + q) * k + j] = -1;
+            continue;
+        }
+        int before = 0;
+        for (int q2 = 0; q2 < q; ++q2)
+            for (int j2 = 0; j2 < k; ++j2) before += (sidx[q2][j2] == e);
+        const int rank = blockoff[(size_t)e * NB + chunk] + before;
+        int p = -1;
+        if (capacity < 0 || rank < capacity) p = indptr[e] + rank;
+        spos[q][j] = p;
+        pos[(size_t)(t0 + q) * k + j] = p;
+        if (p >= 0 && row_token != nullptr) row_token[p] = t0 + q;
+    }
+    __syncthreads();
+    if (xp == nullptr) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int q = warp; q < ntok; q += blockDim.x >> 5) {
+        const uint4* src = x + (size_t)(t0 + q) * nvec;
+        int dst[MOE_MAX_K];
+        int nd = 0;
+        for (int j = 0; j < k; ++j)
+            if (spos[q][j] >= 0) dst[nd++] = spos[q][j];
+        if (nd == 0) continue;
+        for (int v = lane; v < nvec; v += 32) {
+            uint4 val = src[v];
+            for (int j = 0; j < nd; ++j) xp[(size_t)dst[j] * nvec + v] = val;
+        }
+    }
+}
+
+cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
+                                  const int32_t* blockoff, const int32_t* indptr,
+                                  int T, int d, int E, int k, int capacity,
+                                  int32_t* pos, int32_t* row_token, void* xp, cudaStream_t st) {
+    int NB = ceil_div(T, kChunk);
+    if (NB == 0) return cudaSuccess;
+    int nvec = (int)((size_t)d * elem_bytes(dtype) / 16);
+    permute_gather_kernel<<<NB, 256, 0, st>>>((const uint4*)x, idx, blockoff, indptr, T, nvec, E, k,
+                                              capacity, pos, row_token, (uint4*)xp);
+    return cudaGetLastError();
+}
+
+// Statistics for T == 0 (nothing routed).
+__global__ void zero_stats_kernel(void* stats, int E, int capacity) {
+    moe_stats* st = (moe_stats*)stats;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        MOE_STATS_COUNTS(stats, E)[e] = 0;
+        MOE_STATS_KEPT(stats, E)[e] = 0;
+        MOE_STATS_P(stats, E)[e] = 0.f;
+        MOE_STATS_F(stats, E)[e] = 0.f;
+    }
+    if (threadIdx.x == 0) {
+        st->status = MOE_OK; st->capacity = capacity; st->rows = 0; st->dropped = 0;
+        st->max_count = 0; st->l_aux = 0.f; st->max_over_mean = 0.f; st->reserved = 0;
+    }
+}
+
+cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st) {
+    zero_stats_kernel<<<1, 256, 0, st>>>(stats, E, capacity);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,280 @@
+// Router: logits z = W_r^T x, selection key, top-k, gates and the per-chunk
+// partial statistics.
+//
+// "Week 2 Day 2: Mixture of Experts" §1.3 (z = W_r^T x, T = TopK(z, k),
+// g_i = exp(z_i) / sum_{j in T} exp(z_j)), §4.2 (selection on z + b, gates from
+// the raw z), §3.2 (f_i and P_i of the balance loss); "Stanford CS336 Lecture
+// 04" §2.3.3c (bias added to the softmax score). Router arithmetic is fp32
+// ("Lecture 21 · LLM: Mixture-of-Experts" §7.1: the router runs in fp32).
+#include "common.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ float ld_f(const float* p) { return *p; }
+__device__ __forceinline__ float ld_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// ---- W_r [d, E] -> W_r^T [E, d] ------------------------------------------
+template <typename T>
+__global__ void transpose_kernel(const T* __restrict__ in, T* __restrict__ out, int d, int E) {
+    __shared__ T tile[32][33];
+    int i0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        int i = i0 + r, e = e0 + threadIdx.x;
+        if (i < d && e < E) tile[r][threadIdx.x] = in[(size_t)i * E + e];
+    }
+    __syncthreads();
+    for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+        int e = e0 + r, i = i0 + threadIdx.x;
+        if (i < d && e < E) out[(size_t)e * d + i] = tile[threadIdx.x][r];
+    }
+}
+
+cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, int E, cudaStream_t st) {
+    dim3 grid(ceil_div(d, 32), ceil_div(E, 32)), block(32, 8);
+    if (dtype == MOE_DTYPE_BF16)
+        transpose_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
+            (const __nv_bfloat16*)W_r, (__nv_bfloat16*)wrt, d, E);
+    else
+        transpose_kernel<float><<<grid, block, 0, st>>>((const float*)W_r, (float*)wrt, d, E);
+    return cudaGetLastError();
+}
+
+// ---- logits on CUDA cores: one thread per (token, expert) ----------------
+// Eight partial sums over i mod 8 (fixed assignment), combined by a fixed
+// tree: the same inputs always give the same bits.
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    float4 a = *reinterpret_cast<const float4*>(p);
+    float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x; v[2 * i + 1] = f.y;
+    }
+}
+
+template <typename T>
+__global__ void logits_kernel(const T* __restrict__ x, const T* __restrict__ wrt,
+                              float* __restrict__ logits, int Tn, int d, int E) {
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long long)Tn * E) return;
+    int t = (int)(gid / E), e = (int)(gid % E);
+    const T* xr = x + (size_t)t * d;
+    const T* wr = wrt + (size_t)e * d;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < d; i += 8) {
+        float xv[8], wv[8];
+        load8(xr + i, xv);
+        load8(wr + i, wv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = fmaf(xv[j], wv[j], acc[j]);
+    }
+    float z = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    logits[gid] = z;
+}
+
+cudaError_t launch_logits_simt(int dtype, const void* x, const void* wrt, float* logits,
+                               int T, int d, int E, cudaStream_t st) {
+    long long n = (long long)T * E;
+    if (n == 0) return cudaSuccess;
+    int block = 256;
+    unsigned grid = (unsigned)((n + block - 1) / block);
+    if (dtype == MOE_DTYPE_BF16)
+        logits_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
+            (const __nv_bfloat16*)x, (const __nv_bfloat16*)wrt, logits, T, d, E);
+    else
+        logits_kernel<float><<<grid, block, 0, st>>>((const float*)x, (const float*)wrt, logits, T, d, E);
+    return cudaGetLastError();
+}
+
+// ---- selection: softmax, key, top-k, gates, chunk statistics -------------
+// Grid: one block per chunk of kChunk tokens; 8 warps, 4 tokens per warp.
+// Lane l holds experts e = l + 32 i, i < EPL. Every warp reduction is an xor
+// butterfly, so all lanes end with the same bits and the order is fixed.
+constexpr int kSelWarps = 8;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(kSelWarps * 32)
+select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int bias_mode,
+              int Tn, int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+              int32_t* __restrict__ blockcnt, float* __restrict__ blockpsum) {
+    __shared__ int cnt[MOE_MAX_E];
+    __shared__ float ps[kSelWarps][MOE_MAX_E];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunk = blockIdx.x, NB = gridDim.x;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+
+    float b[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        int e = lane + 32 * i;
+        b[i] = (bias_mode != MOE_BIAS_NONE && e < E) ? bias[e] : 0.f;
+    }
+    float psum[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) psum[i] = 0.f;
+
+    constexpr int kTokPerWarp = kChunk / kSelWarps;
+    for (int q = 0; q < kTokPerWarp; ++q) {
+        const int t = chunk * kChunk + warp * kTokPerWarp + q;
+        if (t >= Tn) break;
+        float z[EPL], key[EPL];
+        const float* zr = logits + (size_t)t * E;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            int e = lane + 32 * i;
+            z[i] = e < E ? zr[e] : -INFINITY;
+        }
+        // full softmax over all E raw logits (for P and the PROB key)
+        float m = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) m = fmaxf(m, z[i]);
+        m = warp_max(m);
+        float ex[EPL], s = 0.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            int e = lane + 32 * i;
+            ex[i] = e < E ? expf(z[i] - m) : 0.f;
+            s += ex[i];
+        }
+        s = warp_sum(s);
+        const float inv_s = 1.f / s;
+        unsigned valid = 0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            int e = lane + 32 * i;
+            float p = ex[i] * inv_s;
+            if (e < E) {
+                psum[i] += p;
+                valid |= 1u << i;
+            }
+            key[i] = bias_mode == MOE_BIAS_NONE ? z[i]
+                   : bias_mode == MOE_BIAS_LOGIT ? z[i] + b[i]
+                   : p + b[i];
+        }
+        // top-k: k rounds of a warp arg-max over (key desc, index asc)
+        unsigned taken = 0;
+        float zsel[MOE_MAX_K];
+        int esel[MOE_MAX_K];
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) {
+            if (j < k) {
+                float bk = -INFINITY, bz = 0.f;
+                int be = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) {
+                    bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
+                    if (ok && (key[i] > bk || be == 0x7fffffff)) {
+                        bk = key[i]; be = lane + 32 * i; bz = z[i];
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
+                    int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                    float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+                    bool better = (oe != 0x7fffffff) &&
+                                  (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
+                    if (better) { bk = ok_; be = oe; bz = oz; }
+                }
+                if ((be & 31) == lane) taken |= 1u << (be >> 5);
+                zsel[j] = bz;
+                esel[j] = be;
+            }
+        }
+        // gates: softmax over the selected raw logits, slot order
+        float zm = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) zm = fmaxf(zm, zsel[j]);
+        float gs = 0.f, ge[MOE_MAX_K];
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) {
+            if (j < k) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
+        }
+        const float inv_g = 1.f / gs;
+        if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < MOE_MAX_K; ++j) {
+                if (j < k) {
+                    idx_out[(size_t)t * k + j] = esel[j];
+                    gate_out[(size_t)t * k + j] = ge[j] * inv_g;
+                    atomicAdd(&cnt[esel[j]], 1);   // integer: order does not matter
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        int e = lane + 32 * i;
+        if (e < E) ps[warp][e] = psum[i];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float acc = 0.f;
+        for (int w = 0; w < kSelWarps; ++w) acc += ps[w][e];   // fixed order over warps
+        blockpsum[(size_t)chunk * E + e] = acc;
+        blockcnt[(size_t)e * NB + chunk] = cnt[e];
+    }
+}
+
+cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
+                          int32_t* idx, float* gate, int32_t* blockcnt, float* blockpsum,
+                          cudaStream_t st) {
+    int NB = ceil_div(T, kChunk);
+    if (NB == 0) return cudaSuccess;
+    dim3 grid(NB), block(kSelWarps * 32);
+    int epl = ceil_div(E, 32);
+    if (epl <= 1)
+        select_kernel<1><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+    else if (epl <= 2)
+        select_kernel<2><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+    else if (epl <= 4)
+        select_kernel<4><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+    else if (epl <= 8)
+        select_kernel<8><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+    else
+        select_kernel<16><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+    return cudaGetLastError();
+}
+
+// ---- per-chunk histogram of given selections (standalone permutation) ----
+__global__ void hist_kernel(const int32_t* __restrict__ idx, int Tn, int k, int E,
+                            int32_t* __restrict__ blockcnt) {
+    __shared__ int cnt[MOE_MAX_E];
+    const int chunk = blockIdx.x, NB = gridDim.x;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    const int t0 = chunk * kChunk;
+    const int n = min(kChunk, Tn - t0) * k;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        int e = idx[(size_t)t0 * k + i];
+        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) blockcnt[(size_t)e * NB + chunk] = cnt[e];
+}
+
+cudaError_t launch_hist(const int32_t* idx, int T, int k, int E, int32_t* blockcnt, cudaStream_t st) {
+    int NB = ceil_div(T, kChunk);
+    if (NB == 0) return cudaSuccess;
+    hist_kernel<<<NB, 256, 0, st>>>(idx, T, k, E, blockcnt);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -389,6 +389,29 @@ def moe_forward(x, W_r, W1, W3, W2, k, capacity_factor=0.0, bias=None,
     return ForwardResult(routing=routing, perm=perm, stats=stats, y=y, tokens=tokens)
 
 
+def unpermute_combine(O_rows, pos, gate, S=None):
+    """Un-permute and mix: y_t = sum_{j < k, pos[t,j] >= 0} g_{t,j} O[pos[t,j]]
+    in slot order, plus the shared-expert row S_t when given.
+
+    [CMU 15-779 L21] §3.2 step 4 (restore token order, weight by the gates);
+    [CME295 W2D2] §4.1 (the shared expert is added for every token).
+    O_rows: [R, d] expert outputs in permuted order; pos, gate: [T, k].
+    """
+    O_rows = np.asarray(O_rows, dtype=np.float64)
+    pos = np.asarray(pos)
+    gate = np.asarray(gate, dtype=np.float64)
+    T, k = pos.shape
+    d = O_rows.shape[1] if O_rows.ndim == 2 else (np.asarray(S).shape[1] if S is not None else 0)
+    y = np.zeros((T, d), dtype=np.float64)
+    for t in range(T):
+        for j in range(k):
+            if pos[t, j] >= 0:
+                y[t] = y[t] + gate[t, j] * O_rows[pos[t, j]]
+    if S is not None:
+        y = y + np.asarray(S, dtype=np.float64)
+    return y
+
+
 # --------------------------------------------------------------------------
 # Closed forms the notes print
 # --------------------------------------------------------------------------

@@ -1,0 +1,129 @@
+"""The C-ABI library: it loads, exports every function include/moe.h declares,
+and rejects bad arguments on the host before launching anything (CPU only)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mixture_experts_layer_62_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:int|size_t|const\s+char\s*\*)\s+(moe_\w+)\s*\(", src, flags=re.M)
+    assert names, "no declarations parsed"
+    return sorted(set(names))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = moe.lib
+    names = declared_functions()
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in moe.h but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(moe_\w+)", out))
+    assert set(names) <= exported
+    # nothing exported under the moe_ prefix that the header does not declare
+    assert exported <= set(names), exported - set(names)
+
+
+def test_error_strings():
+    assert moe.error_string(0) == "ok"
+    for code in range(1, 6):
+        assert moe.error_string(code) not in ("ok", "unknown error")
+    assert moe.error_string(99) == "unknown error"
+
+
+def test_stats_size_matches_header_layout():
+    assert moe.stats_size(8) == 32 + 16 * 8
+    assert moe.stats_size(256) == 32 + 16 * 256
+
+
+def test_workspace_layout_is_aligned_and_ordered():
+    for p in (moe.problem(4096, 4096, 14336, 8, 2), moe.problem(8192, 7168, 2048, 256, 8, d_ff_shared=2048),
+              moe.problem(1, 128, 256, 8, 2, dtype="f32"), moe.problem(0, 64, 64, 4, 1)):
+        lay = moe.workspace_layout(p)
+        offs = [lay[n] for n in ("idx", "gate", "pos", "indptr", "row_token", "logits", "xp", "h", "o", "hs", "s")]
+        assert all(o % 256 == 0 for o in offs)
+        assert offs == sorted(offs)
+        assert lay["total"] == moe.workspace_size(p) >= offs[-1]
+    # permuted buffers hold T*k rows
+    p = moe.problem(4096, 4096, 14336, 8, 2)
+    lay = moe.workspace_layout(p)
+    assert lay["h"] - lay["xp"] >= 4096 * 2 * 4096 * 2
+    assert lay["o"] - lay["h"] >= 4096 * 2 * 14336 * 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=16, d=64, d_ff=64, E=4, k=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=16, d=64, d_ff=64, E=4, k=5), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=16, d=64, d_ff=64, E=600, k=2), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=16, d=64, d_ff=64, E=32, k=17), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=-1, d=64, d_ff=64, E=4, k=2), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=16, d=96, d_ff=64, E=4, k=2), moe.MOE_ERR_UNSUPPORTED),        # bf16 needs d % 64 == 0
+    (dict(T=16, d=64, d_ff=96, E=4, k=2), moe.MOE_ERR_UNSUPPORTED),
+    (dict(T=16, d=64, d_ff=64, E=4, k=2, d_ff_shared=32), moe.MOE_ERR_UNSUPPORTED),
+    (dict(T=16, d=12, d_ff=64, E=4, k=2, dtype="f32"), moe.MOE_ERR_UNSUPPORTED),  # f32 needs d % 8
+])
+def test_problem_validation(kw, code):
+    p = moe.problem(**kw)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any launch
+    rc = moe.lib.moe_forward(ctypes.byref(p), *([fake] * 11), fake, 1 << 30, None)
+    assert rc == code
+    assert moe.lib.moe_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_bad_bias_mode_and_dtype_rejected():
+    p = moe.problem(16, 64, 64, 4, 2)
+    p.bias_mode = 7
+    fake = ctypes.c_void_p(1 << 20)
+    assert moe.lib.moe_forward(ctypes.byref(p), *([fake] * 11), fake, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    p = moe.problem(16, 64, 64, 4, 2)
+    p.dtype = 5
+    assert moe.lib.moe_forward(ctypes.byref(p), *([fake] * 11), fake, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = moe.problem(16, 64, 64, 4, 2)
+    fake = ctypes.c_void_p(1 << 20)
+    args = [fake] * 11
+    args[0] = None                                       # x missing
+    assert moe.lib.moe_forward(ctypes.byref(p), *args, fake, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    args = [fake] * 11
+    args[3] = ctypes.c_void_p((1 << 20) + 8)             # W1 not 16-byte aligned
+    assert moe.lib.moe_forward(ctypes.byref(p), *args, fake, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    # bias required when a bias mode is set
+    p = moe.problem(16, 64, 64, 4, 2, bias_mode=moe.BIAS_LOGIT)
+    args = [fake] * 11
+    args[2] = None
+    assert moe.lib.moe_forward(ctypes.byref(p), *args, fake, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    # shared expert weights required when d_ff_shared > 0
+    p = moe.problem(16, 64, 64, 4, 2, d_ff_shared=64)
+    args = [fake] * 11
+    args[7] = None
+    assert moe.lib.moe_forward(ctypes.byref(p), *args, fake, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_small_or_missing_workspace_rejected():
+    p = moe.problem(16, 64, 64, 4, 2)
+    need = moe.workspace_size(p)
+    fake = ctypes.c_void_p(1 << 20)
+    assert moe.lib.moe_forward(ctypes.byref(p), *([fake] * 11), fake, need - 1, None) == moe.MOE_ERR_WORKSPACE
+    assert moe.lib.moe_forward(ctypes.byref(p), *([fake] * 11), None, need, None) == moe.MOE_ERR_WORKSPACE
+    misaligned = ctypes.c_void_p((1 << 20) + 16)
+    assert moe.lib.moe_forward(ctypes.byref(p), *([fake] * 11), misaligned, need, None) == moe.MOE_ERR_WORKSPACE
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    p = moe.problem(4, 64, 64, 4, 2)
+    t = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        moe.combine(p, t, t, t, t)

@@ -1,0 +1,434 @@
+"""GPU parity of every stage of the CUDA path against the CPU oracle.
+
+Stage by stage (same inputs on both sides):
+  route from given logits   indices bit-exact (NONE / LOGIT keys are formed
+                            in fp32 on both sides), gates to fp32 rounding
+  permutation               pos, indptr, row_token, counts, kept bit-exact,
+                            gathered rows bit-exact
+  expert GEMMs              per-row relative error under the bf16 bar
+  combine                   to fp32 / bf16 rounding
+End to end: small shapes over all tokens, the full-size workloads on sampled
+tokens (routing over all tokens), determinism, and stage composition.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_62_b200 as moe
+from mixture_experts_layer_62_b200 import inputs
+from oracle import moe_oracle as O
+from parity_util import (MARGIN, TOL_BF16, TOL_F32, TOL_LAUX, LazyExperts, gpu_forward, key_margin, np32,
+                         oracle_weights, problem_of, to_device, token_rel_err)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _dt(name):
+    return torch.bfloat16 if name == "bf16" else torch.float32
+
+
+# --------------------------------------------------------------------------
+# routing from given logits
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,k,mode", [
+    (1000, 8, 2, 0), (777, 8, 2, 1), (300, 64, 8, 0), (513, 256, 8, 1), (64, 256, 8, 0),
+    (40, 5, 5, 0), (33, 1, 1, 0), (1, 8, 2, 1), (95, 512, 16, 0), (200, 32, 1, 1),
+])
+def test_route_from_logits_bit_exact(T, E, k, mode):
+    rng = np.random.default_rng(T * 31 + E)
+    z = rng.standard_normal((T, E)).astype(np.float32) * 2
+    if E >= 3:
+        z[::7, 1:3] = z[::7, 0:1]           # exact ties: the lower index must win
+    bias = rng.uniform(-0.5, 0.5, E).astype(np.float32) if mode else None
+    p = moe.problem(T, 64, 64, E, k, 0.0, "bf16", mode)
+    ws = moe.alloc_workspace(p, DEV)
+    st = moe.alloc_stats(E, DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gate = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    moe.route_from_logits(p, torch.from_numpy(z).to(DEV), idx, gate, st, ws,
+                          bias=None if bias is None else torch.from_numpy(bias).to(DEV))
+    torch.cuda.synchronize()
+    r = O.route(z, k, bias, mode, key_dtype=np.float32)
+    assert np.array_equal(idx.cpu().numpy(), r.idx)
+    assert np.allclose(gate.cpu().numpy(), r.gate, rtol=2e-6, atol=1e-7)
+    s = moe.read_stats(st, E)
+    perm = O.permute(r.idx, E)
+    ls = O.load_stats(perm, r.probs, T, k, None)
+    assert s.status == moe.MOE_OK
+    assert s.counts == ls.counts.tolist()
+    assert np.allclose(s.P, ls.P, rtol=1e-5, atol=1e-7)
+    assert s.l_aux == pytest.approx(ls.l_aux, rel=TOL_LAUX)
+    assert s.rows == T * k and s.dropped == 0 and s.capacity == -1
+
+
+@pytest.mark.parametrize("T,E,k", [(500, 64, 8), (257, 256, 8), (100, 16, 4)])
+def test_route_from_logits_prob_bias(T, E, k):
+    # key = softmax(z) + b: the softmax is formed with each side's exp, so the
+    # comparison excludes rows whose k-th / (k+1)-th key gap is within rounding
+    rng = np.random.default_rng(E + k)
+    z = rng.standard_normal((T, E)).astype(np.float32)
+    bias = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    p = moe.problem(T, 64, 64, E, k, 0.0, "bf16", moe.BIAS_PROB)
+    ws = moe.alloc_workspace(p, DEV)
+    st = moe.alloc_stats(E, DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gate = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    moe.route_from_logits(p, torch.from_numpy(z).to(DEV), idx, gate, st, ws, bias=torch.from_numpy(bias).to(DEV))
+    torch.cuda.synchronize()
+    r = O.route(z, k, bias, O.BIAS_PROB)
+    key = O.selection_key(z, bias, O.BIAS_PROB)
+    m = key_margin(key, k)
+    ok = m > 1e-6
+    g_idx = idx.cpu().numpy()
+    assert ok.mean() > 0.95
+    assert np.array_equal(g_idx[ok], r.idx[ok])
+    # near-tie rows: the GPU's set must still be a valid top-k within rounding
+    kth = -np.sort(-key, axis=1)[:, k - 1]
+    for t in np.nonzero(~ok)[0]:
+        assert (key[t, g_idx[t]] >= kth[t] - 1e-6).all()
+    assert np.allclose(gate.cpu().numpy()[ok], r.gate[ok], rtol=2e-6, atol=1e-7)
+
+
+# --------------------------------------------------------------------------
+# permutation
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,k,cf,dtype", [
+    (1000, 8, 2, 0.0, "bf16"), (1000, 8, 2, 0.6, "bf16"), (31, 4, 2, 0.5, "f32"), (1, 8, 2, 0.0, "bf16"),
+    (2049, 256, 8, 1.0, "bf16"), (300, 64, 8, 0.3, "f32"), (64, 3, 3, 0.9, "bf16"), (4096, 8, 2, 1.25, "bf16"),
+])
+def test_permute_bit_exact(T, E, k, cf, dtype):
+    rng = np.random.default_rng(T + E * 7)
+    z = rng.standard_normal((T, E))
+    z[:, 0] += 1.0                                    # skew toward expert 0 so capacity bites
+    idx_np = O.topk_lowest_index(z, k)
+    d = 128 if dtype == "bf16" else 64
+    x = torch.randn((T, d), dtype=torch.float32).to(_dt(dtype)).to(DEV)
+    p = moe.problem(T, d, 64, E, k, cf, dtype)
+    ws = moe.alloc_workspace(p, DEV)
+    st = moe.alloc_stats(E, DEV)
+    idx = torch.from_numpy(idx_np.astype(np.int32)).to(DEV)
+    pos = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    indptr = torch.empty((E + 1,), dtype=torch.int32, device=DEV)
+    row_token = torch.full((T * k,), -7, dtype=torch.int32, device=DEV)
+    xp = torch.zeros((T * k, d), dtype=_dt(dtype), device=DEV)
+    moe.permute(p, x, idx, pos, indptr, row_token, xp, st, ws)
+    torch.cuda.synchronize()
+    C = O.capacity(cf, T, k, E)
+    perm = O.permute(idx_np, E, C)
+    assert np.array_equal(pos.cpu().numpy(), perm.pos)
+    assert np.array_equal(indptr.cpu().numpy(), perm.indptr)
+    R = int(perm.indptr[-1])
+    assert np.array_equal(row_token.cpu().numpy()[:R], perm.row_token)
+    s = moe.read_stats(st, E)
+    assert s.counts == perm.counts.tolist() and s.kept == perm.kept.tolist()
+    assert s.rows == R and s.dropped == int((perm.counts - perm.kept).sum())
+    assert s.capacity == (-1 if C is None else C)
+    # gathered rows are bit copies of their token rows
+    assert torch.equal(xp[:R].cpu(), x.cpu()[torch.from_numpy(perm.row_token)])
+
+
+# --------------------------------------------------------------------------
+# expert GEMMs (tcgen05 for bf16, CUDA cores for fp32)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,d,d_ff,counts,shared,T", [
+    ("bf16", 512, 384, [0, 130, 1, 257], 128, 100),          # empty group, ragged tails, 8 k-blocks
+    ("bf16", 256, 128, [128, 128, 128], 0, 64),              # exact tiles
+    ("bf16", 1024, 256, [300], 0, 10),                       # 16 k-blocks: ring wraps 4 times
+    ("bf16", 128, 512, [5, 0, 0, 700, 3], 192, 257),         # shared width != routed width
+    ("f32", 128, 256, [0, 70, 1, 129], 64, 50),
+])
+def test_experts_stage(dtype, d, d_ff, counts, shared, T):
+    E = len(counts)
+    k = 2
+    Tt = max(T, (sum(counts) + k - 1) // k)
+    rows = Tt * k
+    assert sum(counts) <= rows
+    g = torch.Generator().manual_seed(d + d_ff)
+    dt = _dt(dtype)
+    xp = torch.randn((rows, d), generator=g).to(dt)
+    W1 = (torch.randn((E, d_ff, d), generator=g) / math.sqrt(d)).to(dt)
+    W3 = (torch.randn((E, d_ff, d), generator=g) / math.sqrt(d)).to(dt)
+    W2 = (torch.randn((E, d, d_ff), generator=g) / math.sqrt(d_ff)).to(dt)
+    x = torch.randn((Tt, d), generator=g).to(dt)
+    sh = {}
+    if shared:
+        sh = dict(Ws1=(torch.randn((shared, d), generator=g) / math.sqrt(d)).to(dt),
+                  Ws3=(torch.randn((shared, d), generator=g) / math.sqrt(d)).to(dt),
+                  Ws2=(torch.randn((d, shared), generator=g) / math.sqrt(shared)).to(dt))
+    indptr_np = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    p = moe.problem(Tt, d, d_ff, E, k, 0.0, dtype, 0, shared)
+    ws = moe.alloc_workspace(p, DEV)
+    st = moe.alloc_stats(E, DEV)
+    o = torch.full((rows, d), float("nan"), dtype=dt, device=DEV)
+    s = torch.empty((Tt, d), dtype=dt, device=DEV) if shared else None
+    moe.experts(p, xp.to(DEV), torch.from_numpy(indptr_np).to(DEV), W1.to(DEV), W3.to(DEV), W2.to(DEV), o, ws,
+                x=x.to(DEV), s=s, stats=st, **{n: v.to(DEV) for n, v in sh.items()})
+    torch.cuda.synchronize()
+    assert moe.read_stats(st, E).status == moe.MOE_OK
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    on = o.float().cpu().numpy()
+    for e in range(E):
+        lo, hi = indptr_np[e], indptr_np[e + 1]
+        if hi == lo:
+            continue
+        ref = O.swiglu_expert(xp[lo:hi].float().numpy(), W1[e].float().numpy(), W3[e].float().numpy(),
+                              W2[e].float().numpy())
+        rel, _ = token_rel_err(on[lo:hi], ref)
+        assert rel < tol, (e, rel)
+    # rows past the last group are never written
+    R = indptr_np[-1]
+    if R < rows:
+        assert torch.isnan(o[R:].float()).all()
+    if shared:
+        ref = O.swiglu_expert(x.float().numpy(), sh["Ws1"].float().numpy(), sh["Ws3"].float().numpy(),
+                              sh["Ws2"].float().numpy())
+        rel, _ = token_rel_err(s.float().cpu().numpy(), ref)
+        assert rel < tol
+
+
+# --------------------------------------------------------------------------
+# combine
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,T,d,k,shared", [("bf16", 300, 256, 2, False), ("f32", 77, 64, 3, True),
+                                                 ("bf16", 65, 7168, 8, True)])
+def test_combine(dtype, T, d, k, shared):
+    rng = np.random.default_rng(T + d)
+    R = T * k
+    perm_rows = rng.permutation(R)
+    pos = perm_rows.reshape(T, k).astype(np.int32)
+    pos[rng.random((T, k)) < 0.2] = -1
+    pos[3] = -1                                           # a fully dropped token
+    gate = rng.random((T, k)).astype(np.float32)
+    dt = _dt(dtype)
+    O_rows = torch.randn((R, d)).to(dt)
+    S = torch.randn((T, d)).to(dt) if shared else None
+    p = moe.problem(T, d, 64, 8, k, 0.0, dtype)
+    out = torch.empty((T, d), dtype=dt, device=DEV)
+    moe.combine(p, O_rows.to(DEV), torch.from_numpy(pos).to(DEV), torch.from_numpy(gate).to(DEV), out,
+                s=None if S is None else S.to(DEV))
+    torch.cuda.synchronize()
+    ref = O.unpermute_combine(O_rows.float().numpy(), pos, gate, None if S is None else S.float().numpy())
+    got = out.float().cpu().numpy()
+    if dtype == "bf16":
+        assert np.allclose(got, ref, rtol=2 ** -8, atol=1e-6)
+    else:
+        assert np.allclose(got, ref, rtol=1e-6, atol=1e-6)
+    if not shared:
+        assert np.abs(got[3]).max() == 0.0
+
+
+# --------------------------------------------------------------------------
+# end to end, small shapes, all tokens
+# --------------------------------------------------------------------------
+
+SMALL = [
+    dict(T=300, d=256, d_ff=384, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    dict(T=130, d=128, d_ff=128, E=64, k=8, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=128),
+    dict(T=1000, d=256, d_ff=256, E=8, k=2, cf=0.6, dtype="bf16", bias_mode=1, d_ff_shared=0),
+    dict(T=33, d=128, d_ff=128, E=1, k=1, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    dict(T=50, d=128, d_ff=192, E=4, k=4, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    dict(T=1, d=512, d_ff=256, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    dict(T=64, d=256, d_ff=128, E=256, k=8, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=256),
+    dict(T=257, d=64, d_ff=128, E=6, k=3, cf=0.25, dtype="f32", bias_mode=1, d_ff_shared=64),
+]
+
+
+def _small_layer(cfg, seed):
+    g = torch.Generator().manual_seed(seed)
+    dt = _dt(cfg["dtype"])
+    T, d, dff, E, dfs = cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["d_ff_shared"]
+    L = dict(x=torch.randn((T, d), generator=g).to(dt),
+             W_r=(torch.randn((d, E), generator=g) / math.sqrt(d)).to(dt),
+             W1=(torch.randn((E, dff, d), generator=g) / math.sqrt(d)).to(dt),
+             W3=(torch.randn((E, dff, d), generator=g) / math.sqrt(d)).to(dt),
+             W2=(torch.randn((E, d, dff), generator=g) / math.sqrt(dff)).to(dt),
+             bias=None, Ws1=None, Ws3=None, Ws2=None)
+    if cfg["bias_mode"] == 1:
+        L["bias"] = torch.linspace(1.0, -1.0, E)
+    elif cfg["bias_mode"] == 2:
+        L["bias"] = torch.rand((E,), generator=g) * 0.2 - 0.1
+    if dfs:
+        L["Ws1"] = (torch.randn((dfs, d), generator=g) / math.sqrt(d)).to(dt)
+        L["Ws3"] = (torch.randn((dfs, d), generator=g) / math.sqrt(d)).to(dt)
+        L["Ws2"] = (torch.randn((d, dfs), generator=g) / math.sqrt(dfs)).to(dt)
+    return L
+
+
+def _check_forward(cfg, L_cpu, tokens=None, check_own_routing=True):
+    """Run the CUDA forward and compare with the oracle; returns the errors."""
+    L = to_device(L_cpu)
+    p, out, st, ws = gpu_forward(cfg, L)
+    T, k, E = cfg["T"], cfg["k"], cfg["E"]
+    s = moe.read_stats(st, E)
+    assert s.status == moe.MOE_OK
+    logits = moe.workspace_view(ws, p, "logits").cpu().numpy()
+    g_idx = moe.workspace_view(ws, p, "idx").cpu().numpy()
+    g_pos = moe.workspace_view(ws, p, "pos").cpu().numpy()
+    x_np = np32(L_cpu["x"])
+    bias = None if L_cpu["bias"] is None else L_cpu["bias"].float().numpy()
+    W = oracle_weights(L_cpu)
+    # (1) oracle consuming the GPU's logits: routing, drops, outputs
+    exact_key = cfg["bias_mode"] != O.BIAS_PROB
+    res = O.moe_forward(x_np, None, W["W1"], W["W3"], W["W2"], k, cfg["cf"], bias, cfg["bias_mode"],
+                        W["Ws1"], W["Ws3"], W["Ws2"], logits=logits, tokens=tokens,
+                        key_dtype=np.float32 if exact_key else np.float64)
+    if exact_key:
+        assert np.array_equal(g_idx, res.routing.idx)
+        assert np.array_equal(g_pos, res.perm.pos)
+        assert s.counts == res.stats.counts.tolist()
+        assert s.kept == res.stats.kept.tolist()
+        assert s.dropped == res.stats.dropped
+        good = np.ones(T, dtype=bool)
+    else:
+        m = key_margin(res.routing.key, k)
+        good = m > 1e-6
+        assert np.array_equal(g_idx[good], res.routing.idx[good])
+        assert cfg["cf"] <= 0, "PROB-key parity with capacity needs a drop-set argument"
+    assert s.l_aux == pytest.approx(res.stats.l_aux, rel=TOL_LAUX)
+    toks = res.tokens
+    sel = good[toks]
+    got = out.float().cpu().numpy()[toks]
+    rel, zmax = token_rel_err(got[sel], res.y[sel])
+    tol = TOL_BF16 if cfg["dtype"] == "bf16" else TOL_F32
+    assert rel < tol, rel
+    assert zmax == 0.0
+    # (2) the oracle's own fp64 logits: indices equal away from near-ties
+    if check_own_routing:
+        z64 = O.router_logits(x_np, np32(L_cpu["W_r"]))
+        assert np.abs(z64 - logits).max() < 1e-3 * max(1.0, np.abs(z64).max())
+        key64 = O.selection_key(z64, bias, cfg["bias_mode"])
+        own = O.topk_lowest_index(key64, k)
+        far = key_margin(key64, k) >= MARGIN
+        assert np.array_equal(g_idx[far], own[far])
+    return rel
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=[f"T{c['T']}_E{c['E']}_k{c['k']}_{c['dtype']}_b{c['bias_mode']}"
+                                            f"_cf{c['cf']}_s{c['d_ff_shared']}" for c in SMALL])
+def test_forward_small(cfg):
+    _check_forward(cfg, _small_layer(cfg, cfg["T"] + cfg["E"]))
+
+
+def test_forward_zero_tokens():
+    cfg = dict(T=0, d=128, d_ff=128, E=8, k=2, cf=1.0, dtype="bf16", bias_mode=0, d_ff_shared=0)
+    p = problem_of(cfg)
+    ws = moe.alloc_workspace(p, DEV)
+    st = moe.alloc_stats(8, DEV)
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
+    W = torch.zeros((8, 128, 128), dtype=torch.bfloat16, device=DEV)
+    W_r = torch.zeros((128, 8), dtype=torch.bfloat16, device=DEV)
+    out = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
+    # zero-size tensors may carry a null pointer: pass a 16-byte aligned stand-in
+    x = torch.empty((1, 128), dtype=torch.bfloat16, device=DEV)
+    out = torch.empty((1, 128), dtype=torch.bfloat16, device=DEV)
+    moe.forward(p, x, W_r, W, W, W, out, st, ws)
+    torch.cuda.synchronize()
+    s = moe.read_stats(st, 8)
+    assert s.status == 0 and s.rows == 0 and s.counts == [0] * 8 and s.l_aux == 0.0
+
+
+def test_forward_toy_fp32_full():
+    cfg = inputs.workload("toy_fp32")
+    L = inputs.make_layer(cfg, seed=0)
+    rel = _check_forward(cfg, L)
+    assert rel < TOL_F32
+
+
+# --------------------------------------------------------------------------
+# determinism and stage composition
+# --------------------------------------------------------------------------
+
+def test_forward_is_deterministic():
+    cfg = dict(T=1000, d=256, d_ff=256, E=8, k=2, cf=0.6, dtype="bf16", bias_mode=1, d_ff_shared=128)
+    L = to_device(_small_layer(cfg, 5))
+    _, out1, st1, _ = gpu_forward(cfg, L)
+    _, out2, st2, _ = gpu_forward(cfg, L)
+    assert torch.equal(out1, out2)
+    assert torch.equal(st1, st2)
+
+
+def test_stages_compose_to_forward():
+    cfg = dict(T=500, d=256, d_ff=384, E=16, k=4, cf=0.8, dtype="bf16", bias_mode=1, d_ff_shared=128)
+    L = to_device(_small_layer(cfg, 9))
+    p, out, st, ws = gpu_forward(cfg, L)
+    T, d, E, k = cfg["T"], cfg["d"], cfg["E"], cfg["k"]
+    ws2 = moe.alloc_workspace(p, DEV)
+    st2 = moe.alloc_stats(E, DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gate = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    logits = torch.empty((T, E), dtype=torch.float32, device=DEV)
+    moe.route(p, L["x"], L["W_r"], idx, gate, st2, ws2, bias=L["bias"], logits=logits)
+    pos = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    indptr = torch.empty((E + 1,), dtype=torch.int32, device=DEV)
+    row_token = torch.empty((T * k,), dtype=torch.int32, device=DEV)
+    xp = torch.empty((T * k, d), dtype=torch.bfloat16, device=DEV)
+    moe.permute(p, L["x"], idx, pos, indptr, row_token, xp, st2, ws2)
+    o = torch.empty((T * k, d), dtype=torch.bfloat16, device=DEV)
+    s = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    moe.experts(p, xp, indptr, L["W1"], L["W3"], L["W2"], o, ws2, x=L["x"], Ws1=L["Ws1"], Ws3=L["Ws3"],
+                Ws2=L["Ws2"], s=s)
+    out2 = torch.empty_like(out)
+    moe.combine(p, o, pos, gate, out2, s=s)
+    torch.cuda.synchronize()
+    assert torch.equal(moe.workspace_view(ws, p, "idx"), idx)
+    assert torch.equal(moe.workspace_view(ws, p, "pos"), pos)
+    assert torch.equal(out, out2)
+
+
+# --------------------------------------------------------------------------
+# full-size workloads: routing on all tokens, outputs on sampled tokens
+# --------------------------------------------------------------------------
+
+def _sample_tokens(pos, indptr, rng, n_random):
+    """Every expert's first and last kept rows, rows at the capacity edge,
+    fully dropped tokens, and random tokens."""
+    T = pos.shape[0]
+    picks = set(rng.choice(T, size=min(n_random, T), replace=False).tolist())
+    R = int(indptr[-1])
+    row_of = {}
+    for t in range(T):
+        for j in range(pos.shape[1]):
+            if pos[t, j] >= 0:
+                row_of[int(pos[t, j])] = t
+    for e in range(len(indptr) - 1):
+        lo, hi = int(indptr[e]), int(indptr[e + 1])
+        if hi > lo:
+            picks.add(row_of[lo])
+            picks.add(row_of[hi - 1])
+    dropped = np.nonzero((pos < 0).all(axis=1))[0]
+    picks.update(dropped[:4].tolist())
+    return np.array(sorted(picks))
+
+
+@pytest.mark.parametrize("name,n_random", [("mixtral_prefill", 24), ("skewed_capacity", 16),
+                                           ("deepseek_v3", 6)])
+def test_forward_full_size(name, n_random):
+    cfg = inputs.workload(name)
+    L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=DEV)
+    Ld = to_device(L)
+    p, out, st, ws = gpu_forward(cfg, Ld)
+    pos = moe.workspace_view(ws, p, "pos").cpu().numpy()
+    indptr = moe.workspace_view(ws, p, "indptr").cpu().numpy()
+    rng = np.random.default_rng(0)
+    toks = _sample_tokens(pos, indptr, rng, n_random)
+    if name == "deepseek_v3":
+        toks = toks[:40]
+    _check_forward(cfg, L, tokens=toks)
+    s = moe.read_stats(st, cfg["E"])
+    if name == "skewed_capacity":
+        assert s.capacity == 5120 and s.dropped > 0
+
+
+@pytest.mark.parametrize("T", inputs.DECODE_TOKENS)
+def test_forward_decode(T):
+    cfg = inputs.workload(f"decode_t{T}")
+    L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=DEV)
+    _check_forward(cfg, L)

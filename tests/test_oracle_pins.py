@@ -306,6 +306,25 @@ def test_token_subset_matches_full():
     assert np.allclose(sub.y, full.y[[29, 0, 7]], rtol=1e-13, atol=1e-15)
 
 
+def test_unpermute_combine_reproduces_layer_output():
+    # expert outputs computed in permuted row order and mixed back give the
+    # per-pair layer output ([CMU 15-779 L21] §3.2 four steps)
+    rng = np.random.default_rng(13)
+    x, W_r, W1, W3, W2, sh = _rand_layer(rng, 40, 8, 6, 8, shared=True)
+    res = O.moe_forward(x, W_r, W1, W3, W2, k=3, capacity_factor=0.7, **sh)
+    perm = res.perm
+    R = perm.indptr[-1]
+    O_rows = np.zeros((R, 8))
+    for e in range(6):
+        lo, hi = perm.indptr[e], perm.indptr[e + 1]
+        if hi > lo:
+            O_rows[lo:hi] = O.swiglu_expert(x[perm.row_token[lo:hi]], W1[e], W3[e], W2[e])
+    S = O.swiglu_expert(x, sh["Ws1"], sh["Ws3"], sh["Ws2"])
+    y = O.unpermute_combine(O_rows, perm.pos, res.routing.gate, S)
+    assert np.allclose(y, res.y, rtol=1e-12, atol=1e-13)
+    assert res.stats.dropped > 0
+
+
 # --- closed forms ([CME295 W2D2] §2.3; [CMU 15-779 L21] §3.1 and exercise 4; §2.1 counts) ---
 
 def test_experts_touched_table():
