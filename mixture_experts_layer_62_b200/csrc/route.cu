@@ -10,8 +10,6 @@
 
 namespace moe {
 
-__device__ __forceinline__ float ld_f(const float* p) { return *p; }
-__device__ __forceinline__ float ld_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
 // ---- W_r [d, E] -> W_r^T [E, d] ------------------------------------------
 template <typename T>
@@ -39,9 +37,16 @@ cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, in
     return cudaGetLastError();
 }
 
-// ---- logits on CUDA cores: one thread per (token, expert) ----------------
-// Eight partial sums over i mod 8 (fixed assignment), combined by a fixed
-// tree: the same inputs always give the same bits.
+// ---- logits on CUDA cores -------------------------------------------------
+// One warp per group of kTokPerWarp tokens. Lane l owns the 8-element chunks
+// c = l, l + 32, ... of the row; per chunk it loads the tokens' x once and the
+// chunk of each of 8 experts' W_r^T rows, and accumulates acc[token][expert]
+// over its chunks in ascending order. The 32 lane partials of every logit are
+// then summed by an xor butterfly. The summation order is fixed, so the same
+// inputs always give the same bits. Experts are taken 8 at a time.
+constexpr int kTokPerWarp = 4;
+constexpr int kExpPerPass = 8;
+
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
     float4 a = *reinterpret_cast<const float4*>(p);
     float4 b = *reinterpret_cast<const float4*>(p + 4);
@@ -58,31 +63,64 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
 }
 
 template <typename T>
-__global__ void logits_kernel(const T* __restrict__ x, const T* __restrict__ wrt,
-                              float* __restrict__ logits, int Tn, int d, int E) {
-    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= (long long)Tn * E) return;
-    int t = (int)(gid / E), e = (int)(gid % E);
-    const T* xr = x + (size_t)t * d;
-    const T* wr = wrt + (size_t)e * d;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int i = 0; i < d; i += 8) {
-        float xv[8], wv[8];
-        load8(xr + i, xv);
-        load8(wr + i, wv);
+__global__ void __launch_bounds__(128)
+logits_kernel(const T* __restrict__ x, const T* __restrict__ wrt, float* __restrict__ logits, int Tn, int d,
+              int E) {
+    const int lane = threadIdx.x & 31;
+    const int t0 = ((blockIdx.x * blockDim.x + threadIdx.x) >> 5) * kTokPerWarp;
+    if (t0 >= Tn) return;
+    const int nchunk = d / 8;
+    int nt = Tn - t0;
+    if (nt > kTokPerWarp) nt = kTokPerWarp;
+    for (int e0 = 0; e0 < E; e0 += kExpPerPass) {
+        float acc[kTokPerWarp][kExpPerPass];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = fmaf(xv[j], wv[j], acc[j]);
+        for (int q = 0; q < kTokPerWarp; ++q)
+#pragma unroll
+            for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = 0.f;
+#pragma unroll 2
+        for (int c = lane; c < nchunk; c += 32) {
+            float xv[kTokPerWarp][8];
+#pragma unroll
+            for (int q = 0; q < kTokPerWarp; ++q) {
+                if (q < nt) {
+                    load8(x + (size_t)(t0 + q) * d + (size_t)c * 8, xv[q]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) xv[q][j] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < kExpPerPass; ++e) {
+                if (e0 + e < E) {
+                    float wv[8];
+                    load8(wrt + (size_t)(e0 + e) * d + (size_t)c * 8, wv);
+#pragma unroll
+                    for (int q = 0; q < kTokPerWarp; ++q)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[q][e] = fmaf(xv[q][j], wv[j], acc[q][e]);
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kTokPerWarp; ++q) {
+#pragma unroll
+            for (int e = 0; e < kExpPerPass; ++e) {
+                float v = acc[q][e];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0 && q < nt && e0 + e < E) logits[(size_t)(t0 + q) * E + e0 + e] = v;
+            }
+        }
     }
-    float z = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-    logits[gid] = z;
 }
 
 cudaError_t launch_logits_simt(int dtype, const void* x, const void* wrt, float* logits,
                                int T, int d, int E, cudaStream_t st) {
-    long long n = (long long)T * E;
-    if (n == 0) return cudaSuccess;
-    int block = 256;
-    unsigned grid = (unsigned)((n + block - 1) / block);
+    if (T == 0) return cudaSuccess;
+    const int warps = ceil_div(T, kTokPerWarp);
+    const int block = 128;
+    const int grid = ceil_div(warps * 32, block);
     if (dtype == MOE_DTYPE_BF16)
         logits_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
             (const __nv_bfloat16*)x, (const __nv_bfloat16*)wrt, logits, T, d, E);

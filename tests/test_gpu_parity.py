@@ -86,12 +86,18 @@ def test_route_from_logits_prob_bias(T, E, k):
     ok = m > 1e-6
     g_idx = idx.cpu().numpy()
     assert ok.mean() > 0.95
-    assert np.array_equal(g_idx[ok], r.idx[ok])
+    assert np.array_equal(np.sort(g_idx[ok], axis=1), np.sort(r.idx[ok], axis=1))
+    kg = np.take_along_axis(key, g_idx.astype(np.int64), axis=1)
+    assert (np.diff(kg, axis=1) <= 1e-6).all()          # descending up to rounding
     # near-tie rows: the GPU's set must still be a valid top-k within rounding
     kth = -np.sort(-key, axis=1)[:, k - 1]
     for t in np.nonzero(~ok)[0]:
         assert (key[t, g_idx[t]] >= kth[t] - 1e-6).all()
-    assert np.allclose(gate.cpu().numpy()[ok], r.gate[ok], rtol=2e-6, atol=1e-7)
+    # gates matched by expert (slot order of near-tied keys may differ)
+    for t in np.nonzero(ok)[0][:200]:
+        want = dict(zip(r.idx[t].tolist(), r.gate[t].tolist()))
+        for j in range(k):
+            assert gate[t, j].item() == pytest.approx(want[int(g_idx[t, j])], rel=2e-6, abs=1e-7)
 
 
 # --------------------------------------------------------------------------
@@ -146,7 +152,7 @@ def test_permute_bit_exact(T, E, k, cf, dtype):
 ])
 def test_experts_stage(dtype, d, d_ff, counts, shared, T):
     E = len(counts)
-    k = 2
+    k = min(2, E)
     Tt = max(T, (sum(counts) + k - 1) // k)
     rows = Tt * k
     assert sum(counts) <= rows
@@ -288,9 +294,15 @@ def _check_forward(cfg, L_cpu, tokens=None, check_own_routing=True):
         assert s.dropped == res.stats.dropped
         good = np.ones(T, dtype=bool)
     else:
+        # softmax keys are formed with each side's exp: compare the selected
+        # set away from k-th/(k+1)-th near-ties; inside the set, near-tied keys
+        # may be ordered either way, so check the order against rounding
         m = key_margin(res.routing.key, k)
         good = m > 1e-6
-        assert np.array_equal(g_idx[good], res.routing.idx[good])
+        assert good.mean() > 0.99
+        assert np.array_equal(np.sort(g_idx[good], axis=1), np.sort(res.routing.idx[good], axis=1))
+        kg = np.take_along_axis(res.routing.key, g_idx.astype(np.int64), axis=1)
+        assert (np.diff(kg, axis=1) <= 1e-6).all()
         assert cfg["cf"] <= 0, "PROB-key parity with capacity needs a drop-set argument"
     assert s.l_aux == pytest.approx(res.stats.l_aux, rel=TOL_LAUX)
     toks = res.tokens
@@ -322,11 +334,9 @@ def test_forward_zero_tokens():
     p = problem_of(cfg)
     ws = moe.alloc_workspace(p, DEV)
     st = moe.alloc_stats(8, DEV)
-    x = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
     W = torch.zeros((8, 128, 128), dtype=torch.bfloat16, device=DEV)
     W_r = torch.zeros((128, 8), dtype=torch.bfloat16, device=DEV)
-    out = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
-    # zero-size tensors may carry a null pointer: pass a 16-byte aligned stand-in
+    # zero-size tensors may carry a null pointer: pass 16-byte aligned stand-ins
     x = torch.empty((1, 128), dtype=torch.bfloat16, device=DEV)
     out = torch.empty((1, 128), dtype=torch.bfloat16, device=DEV)
     moe.forward(p, x, W_r, W, W, W, out, st, ws)
