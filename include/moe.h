@@ -210,6 +210,30 @@ int moe_expert_down(const moe_problem* p, const void* h, const int32_t* indptr, 
 int moe_combine(const moe_problem* p, const void* o, const int32_t* pos, const float* gate,
                 const void* s, void* out, void* stream);
 
+/* ---- allocation-free permutation ----------------------------------------
+ * Not a step of the notes (they have no counterpart): a variant of
+ * moe_permute for callers that cannot allocate device memory where they run
+ * the layer, e.g. a plugin of an inference runtime that owns all device
+ * memory and passes in only the input and output buffers, or a
+ * latency-critical loop in which cudaMalloc could block or synchronise the
+ * device. It takes no workspace: the scratch of the permutation (per-chunk
+ * expert counts and their scan) lives in a fixed 1 MiB array inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits. Arguments, outputs and results are those of moe_permute.
+ *  - Limit: E * ceil(T / 32) <= 131072 (e.g. T <= 16384 at E = 256);
+ *    larger problems return MOE_ERR_UNSUPPORTED before anything is launched.
+ *  - The first call on a device looks up the array's device address on that
+ *    device (the device must be current); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps the last call's contents
+ *    (every entry a call reads is written earlier in the same call). Calls
+ *    that overlap on the GPU (different streams, or different host threads,
+ *    on the same device) race on it: serialise them.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+int moe_permute_noalloc(const moe_problem* p, const void* x, const int32_t* idx,
+                        int32_t* pos, int32_t* indptr, int32_t* row_token, void* xp, void* stats,
+                        void* stream);
+
 /* Human-readable text of an MOE_* code (static storage). */
 const char* moe_error_string(int code);
 

@@ -240,6 +240,20 @@ def combine(p: Problem, o, pos, gate, out, s=None, stream=None):
     _check(rc, "moe_combine")
 
 
+def permute_noalloc(p: Problem, x, idx, pos, indptr, row_token, xp, stats, stream=None):
+    """moe_permute without a workspace: for callers that cannot allocate
+    device memory; the library's fixed 1 MiB scratch array is used instead
+    (see moe_permute_noalloc in include/moe.h for the limit and the rules)."""
+    lib = _lib()
+    fn = lib.moe_permute_noalloc
+    if fn.restype is not ctypes.c_int:
+        fn.argtypes = [ctypes.POINTER(Problem)] + [ctypes.c_void_p] * 8
+        fn.restype = ctypes.c_int
+    rc = fn(ctypes.byref(p), _ptr(x), _ptr(idx), _ptr(pos), _ptr(indptr), _ptr(row_token), _ptr(xp), _ptr(stats),
+            _stream(stream))
+    _check(rc, "moe_permute_noalloc")
+
+
 @dataclass
 class Stats:
     status: int
