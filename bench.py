@@ -166,19 +166,29 @@ def blas_threads():
     return os.cpu_count()
 
 
-def oracle_sample(cfg, L, n_tokens, seed=0):
+def oracle_sample(cfg, L, n_tokens, seed=0, needed_experts=None):
     """Time the CPU oracle: routing of all tokens plus the expert math of a
-    seeded sample of n_tokens tokens. Weights are copied to host numpy
-    before the clock starts."""
+    seeded sample of n_tokens tokens. The weights of the experts the sample
+    can touch are copied to host numpy before the clock starts."""
     from oracle import moe_oracle as O
     x = L["x"].float().cpu().numpy()
     W_r = L["W_r"].float().cpu().numpy()
     bias = None if L["bias"] is None else L["bias"].float().cpu().numpy()
     rng = np.random.default_rng(seed)
     tokens = np.sort(rng.choice(cfg["T"], size=min(n_tokens, cfg["T"]), replace=False))
-    W1 = {e: L["W1"][e].float().cpu().numpy() for e in range(cfg["E"])}
-    W3 = {e: L["W3"][e].float().cpu().numpy() for e in range(cfg["E"])}
-    W2 = {e: L["W2"][e].float().cpu().numpy() for e in range(cfg["E"])}
+    experts = range(cfg["E"]) if needed_experts is None else sorted(set(needed_experts(tokens)))
+    class _Host(dict):
+        # an expert the oracle's own routing picks beyond the prefetched set
+        # (a near-tie) is copied on demand
+        def __init__(self, W):
+            super().__init__({e: W[e].float().cpu().numpy() for e in experts})
+            self.W = W
+
+        def __missing__(self, e):
+            v = self[e] = self.W[e].float().cpu().numpy()
+            return v
+
+    W1, W3, W2 = _Host(L["W1"]), _Host(L["W3"]), _Host(L["W2"])
     sh = {}
     if cfg["d_ff_shared"]:
         sh = {n: L[n].float().cpu().numpy() for n in ("Ws1", "Ws3", "Ws2")}
@@ -187,6 +197,51 @@ def oracle_sample(cfg, L, n_tokens, seed=0):
                   sh.get("Ws1"), sh.get("Ws3"), sh.get("Ws2"), tokens=tokens)
     dt = time.perf_counter() - t0
     return len(tokens), dt
+
+
+def touched_experts(st):
+    return sum(1 for c in st.counts if c > 0)
+
+
+def decode_bytes(cfg, st):
+    """Bytes one forward must move: every touched expert's three matrices,
+    the router, x and y (the weight-read bound of small-batch decode)."""
+    d, dff, E, T = cfg["d"], cfg["d_ff"], cfg["E"], cfg["T"]
+    eb = 2 if cfg["dtype"] == "bf16" else 4
+    b = touched_experts(st) * 3 * d * dff * eb + d * E * eb + 2 * T * d * eb
+    if cfg["d_ff_shared"]:
+        b += 3 * d * cfg["d_ff_shared"] * eb
+    return b
+
+
+def workload_roofline(cfg, workload, stages, st, peaks, peak_src):
+    """Roofline of the dominant kernel, grouped GEMM 1/3 + SwiGLU."""
+    rows = st.rows
+    up_ms = stages["expert_up"]
+    down_ms = stages["expert_down"]
+    fl = up_flops(cfg, rows)
+    eb = 2 if cfg["dtype"] == "bf16" else 4
+    n_touch = touched_experts(st)
+    up_bytes = n_touch * 2 * cfg["d"] * cfg["d_ff"] * eb
+    up_bytes += rows * cfg["d"] * eb + rows * cfg["d_ff"] * eb
+    if cfg["d_ff_shared"]:
+        up_bytes += 2 * cfg["d"] * cfg["d_ff_shared"] * eb + cfg["T"] * cfg["d"] * eb + cfg["T"] * cfg["d_ff_shared"] * eb
+    t = up_ms / 1e3
+    tflops, gbs = fl / t / 1e12, up_bytes / t / 1e9
+    peak_tf, peak_bw = peaks["bf16_tflops"], peaks["hbm_gbs"]
+    t_compute, t_memory = fl / (peak_tf * 1e12), up_bytes / (peak_bw * 1e9)
+    common = {"kernel": "tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU)", "ms_per_launch": up_ms,
+              "flops_per_launch": fl, "bytes_per_launch": up_bytes,
+              "roofline_time_ms": 1e3 * max(t_compute, t_memory),
+              "frac_of_roofline_time": max(t_compute, t_memory) / t,
+              "traffic": traffic_for("tc_grouped_gemm_swiglu", workload),
+              "down_proj": {"ms_per_launch": down_ms, "tflops": down_flops(cfg, rows) / (down_ms / 1e3) / 1e12}}
+    if t_memory > t_compute:
+        return {"bound": "hbm", "achieved": gbs, "peak": peak_bw, "unit": "GB/s", "frac": gbs / peak_bw,
+                "peak_source": f"{peak_src} HBM copy", **common}
+    return {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s", "frac": tflops / peak_tf,
+            "peak_source": f"{peak_src} bf16 burst",
+            "frac_of_sustained": tflops / peaks.get("bf16_tflops_sustained", peak_tf), **common}
 
 
 def run_reference(args, cfg, rank):
@@ -239,7 +294,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral_prefill")
-    ap.add_argument("--cpu-sample", type=int, default=256, help="tokens of the timed CPU-oracle sample")
+    ap.add_argument("--cpu-sample", type=int, default=1024, help="tokens of the timed CPU-oracle sample")
     ap.add_argument("--ref-sample", type=int, default=16, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -365,34 +420,31 @@ def main():
     stages = breakdown(moe, p, cfg, L, dev, stream, flush, iters=max(3, min(10, args.steps)))
 
     peaks, peak_src = load_peaks()
-    up_ms = stages["expert_up"]
-    achieved = up_flops(cfg, rows) / (up_ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops"]
-    down_ms = stages["expert_down"]
-    roofline = {"bound": "tensor", "kernel": "tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU)",
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_source": f"{peak_src} bf16 burst",
-                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
-                "traffic": traffic_for("tc_grouped_gemm_swiglu", args.workload),
-                "flops_per_launch": up_flops(cfg, rows), "ms_per_launch": up_ms,
-                "down_proj": {"achieved": down_flops(cfg, rows) / (down_ms / 1e3) / 1e12, "ms_per_launch": down_ms}}
+    roofline = workload_roofline(cfg, args.workload, stages, st, peaks, peak_src)
+    if cfg["T"] <= 64:
+        # decode: weight-read bound; the headline figure is HBM bandwidth
+        roofline["forward_hbm_gbs"] = decode_bytes(cfg, st) / (ms_per_step / 1e3) / 1e9
+        roofline["forward_hbm_frac"] = roofline["forward_hbm_gbs"] / peaks["hbm_gbs"]
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if cfg["dtype"] == "bf16" else "f32", "data": "synthetic",
         "config": config_of(cfg, args), "tflops": tflops,
-        "tflops_frac_of_peak": tflops / peak,
+        "tflops_frac_of_peak": tflops / peaks["bf16_tflops"],
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
                 "d2h_bytes_per_step": nbytes},
         "gpu_launches": launches_per_forward(cfg) * args.steps,
         "clocks": clocks,
         "stages_ms": stages,
-        "routing": {"rows": rows, "dropped": st.dropped, "l_aux": st.l_aux, "max_over_mean": st.max_over_mean},
+        "routing": {"rows": rows, "dropped": st.dropped, "l_aux": st.l_aux, "max_over_mean": st.max_over_mean,
+                    "experts_touched": touched_experts(st), "counts": st.counts if E <= 16 else None,
+                    "kept": st.kept if E <= 16 else None},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, dt = oracle_sample(cfg, L, args.cpu_sample)
+        gidx = moe.workspace_view(layer.workspace, p, "idx").cpu().numpy()
+        n, dt = oracle_sample(cfg, L, args.cpu_sample, needed_experts=lambda toks: gidx[toks].reshape(-1).tolist())
         line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"routing of all {cfg['T']} tokens + expert math of {n} seeded random "
                                           f"tokens ({dt:.1f} s)"}

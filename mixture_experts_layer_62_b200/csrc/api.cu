@@ -30,15 +30,23 @@ Layout make_layout(const moe_problem& p) {
     L.blockcnt = take(E * NB * 4);
     L.blockoff = take(E * NB * 4);
     L.blockpsum = take(NB * E * 4);
-    L.tiles13 = take((E + 2) * 4);
-    L.tiles2 = take((E + 2) * 4);
+    L.tiles13 = take((E + 3) * 4);
+    L.tiles2 = take((E + 3) * 4);
     L.xp = take(T * k * d * eb);
     L.h = take(T * k * dff * eb);
     L.o = take(T * k * d * eb);
     L.hs = take(T * dfs * eb);
     L.s = take(dfs ? T * d * eb : 0);
+    const bool split = split_allowed(p);
+    L.part13 = take(split ? (size_t)kSplitMax * T * k * (size_t)ceil_div(p.d_ff, 128) * 256 * 4 : 0);
+    L.part2 = take(split ? (size_t)kSplitMax * T * k * d * 4 : 0);
     L.total = off;
     return L;
+}
+
+bool split_allowed(const moe_problem& p) {
+    return p.dtype == MOE_DTYPE_BF16 && p.d_ff_shared == 0 && p.T > 0 &&
+           (long long)p.T * p.k <= kSplitMaxRows;
 }
 
 int device_sm_count() {
@@ -126,7 +134,7 @@ int run_logits(const moe_problem* p, const void* x, const void* W_r, float* logi
 // Grouped GEMM 1/3 with the SwiGLU epilogue (and the shared expert's).
 int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13, const void* W1,
            const void* W3, const void* x, const void* Ws1, const void* Ws3, void* h, void* hs, int32_t* status,
-           cudaStream_t st) {
+           cudaStream_t st, float* part13 = nullptr) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
     if (p->dtype == MOE_DTYPE_BF16) {
@@ -141,7 +149,15 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
         a.K[0] = p->d; a.K[1] = p->d;
         a.out[0] = h; a.out[1] = hs;
         a.status = status;
+        if (part13 != nullptr) {
+            a.partial = part13;
+            a.partial_ld = ceil_div(p->d_ff, 128) * 256;
+            a.partial_stride = (long long)rows * a.partial_ld;
+        }
         CK(launch_tc_gemm(a, st));
+        if (part13 != nullptr)
+            CK(launch_swiglu_reduce(part13, a.partial_stride, a.partial_ld, tiles13 + p->E + has_shared + 1, indptr,
+                                    p->E, rows, p->d_ff, h, st));
     } else {
         GroupedArgs a = {};
         a.indptr = indptr; a.tiles = tiles13;
@@ -159,7 +175,8 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
 
 // Grouped GEMM 2 (down projection, and the shared expert's).
 int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const int32_t* tiles2, const void* W2,
-             const void* hs, const void* Ws2, void* o, void* s, int32_t* status, cudaStream_t st) {
+             const void* hs, const void* Ws2, void* o, void* s, int32_t* status, cudaStream_t st,
+             float* part2 = nullptr) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
     if (p->dtype == MOE_DTYPE_BF16) {
@@ -174,6 +191,11 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
         b.K[0] = p->d_ff; b.K[1] = p->d_ff_shared;
         b.out[0] = o; b.out[1] = s;
         b.status = status;
+        if (part2 != nullptr) {
+            b.partial = part2;
+            b.partial_ld = p->d;
+            b.partial_stride = (long long)rows * p->d;
+        }
         CK(launch_tc_gemm(b, st));
     } else {
         GroupedArgs b = {};
@@ -193,10 +215,10 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
 int run_experts(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13,
                 const int32_t* tiles2, const void* W1, const void* W3, const void* W2, const void* x,
                 const void* Ws1, const void* Ws3, const void* Ws2, void* h, void* hs, void* o, void* s,
-                int32_t* status, cudaStream_t st) {
-    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st);
+                int32_t* status, cudaStream_t st, float* part13 = nullptr, float* part2 = nullptr) {
+    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st, part13);
     if (rc != MOE_OK) return rc;
-    return run_down(p, h, indptr, tiles2, W2, hs, Ws2, o, s, status, st);
+    return run_down(p, h, indptr, tiles2, W2, hs, Ws2, o, s, status, st, part2);
 }
 
 void schedule_sizes(const moe_problem* p, int& tile_m, int& nt13, int& nt2, int& nt13s, int& nt2s) {
@@ -298,6 +320,11 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     sa.indptr = indptr; sa.stats = stats;
     sa.tiles13 = tiles13; sa.tiles2 = tiles2; sa.has_shared = shared ? 1 : 0;
     schedule_sizes(p, sa.tile_m, sa.ntiles13, sa.ntiles2, sa.ntiles13_shared, sa.ntiles2_shared);
+    const bool split = split_allowed(*p);
+    sa.split_max = split ? kSplitMax : 1;
+    sa.sm_count = device_sm_count();
+    sa.nkb13 = ceil_div(p->d, 64);
+    sa.nkb2 = ceil_div(p->d_ff, 64);
     CK(launch_scan(sa, st));
     void* xp = wsp(workspace, L.xp);
     CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, C, pos, row_token, xp,
@@ -306,9 +333,14 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     void* o = wsp(workspace, L.o);
     void* hs = shared ? wsp(workspace, L.hs) : nullptr;
     void* s = shared ? wsp(workspace, L.s) : nullptr;
-    rc = run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st);
+    float* part13 = split ? reinterpret_cast<float*>(wsp(workspace, L.part13)) : nullptr;
+    float* part2 = split ? reinterpret_cast<float*>(wsp(workspace, L.part2)) : nullptr;
+    rc = run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st, part13,
+                     part2);
     if (rc != MOE_OK) return rc;
-    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st));
+    const int G = p->E + (shared ? 1 : 0);
+    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st, part2,
+                      (long long)p->T * p->k * p->d, split ? tiles2 + G + 1 : nullptr));
     return MOE_OK;
 }
 

@@ -24,8 +24,17 @@ struct Layout {
     size_t idx, gate, pos, indptr, row_token, logits, wrt;
     size_t blockcnt, blockoff, blockpsum, tiles13, tiles2;
     size_t xp, h, o, hs, s;
+    size_t part13, part2;   // fp32 split-K partials (small-T forward only)
     size_t total;
 };
+
+// Split-K of the grouped GEMMs is used by moe_forward when the whole batch
+// fits one M-block per expert (T*k <= kSplitMaxRows) and there is no shared
+// expert; the split factor (<= kSplitMax) is chosen on the device from the
+// real tile counts.
+constexpr int kSplitMaxRows = 128;
+constexpr int kSplitMax = 8;
+bool split_allowed(const moe_problem& p);
 Layout make_layout(const moe_problem& p);
 
 // Kernel launchers (each returns cudaGetLastError() of its launches).
@@ -48,8 +57,9 @@ struct ScanArgs {
     int32_t* indptr;             // [E+1]
     void* stats;                 // moe_stats block
     // tile schedules (null pointers: skipped)
-    int32_t* tiles13; int32_t* tiles2;
+    int32_t* tiles13; int32_t* tiles2;   // [G+2]: cumulative tiles, then the split factor
     int tile_m, ntiles13, ntiles2, ntiles13_shared, ntiles2_shared, has_shared;
+    int split_max, sm_count, nkb13, nkb2;   // split_max <= 1: no split
 };
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st);
 cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
@@ -60,7 +70,13 @@ cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
                                   int T, int d, int E, int k, int capacity,
                                   int32_t* pos, int32_t* row_token, void* xp, cudaStream_t st);
 cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const float* gate,
-                           const void* s, void* out, int T, int d, int k, cudaStream_t st);
+                           const void* s, void* out, int T, int d, int k, cudaStream_t st,
+                           const float* opart = nullptr, long long opart_stride = 0,
+                           const int32_t* split2 = nullptr);
+// H = SiLU(sum_s gate partials) * (sum_s up partials) for the first indptr[E] rows.
+cudaError_t launch_swiglu_reduce(const float* part, long long split_stride, int ld, const int32_t* split13,
+                                 const int32_t* indptr, int E, int max_rows, int d_ff, void* h,
+                                 cudaStream_t st);
 cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st);
 
 // fp32 grouped GEMM on CUDA cores (the fp32 path). Tile 64 x 64.
@@ -96,6 +112,9 @@ struct TcArgs {
     void* out[2];
     int32_t* status;
     long long timeout_ns;
+    float* partial;            // split-K partials [split][rows][partial_ld] or null
+    long long partial_stride;  // elements between splits
+    int partial_ld;            // elements per row
 };
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
 

@@ -155,6 +155,9 @@ struct KParams {
     void* out[2];
     int32_t* status;
     long long timeout_ns;
+    float* partial;            // split-K partial rows, or null
+    long long partial_stride;  // elements between splits
+    int partial_ld;            // elements per partial row
 };
 
 struct Tile {
@@ -267,6 +270,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
     const int total = total_tiles(p, COLS_PER_TILE);
+    // split-K: the device-chosen factor is stored after the tile schedule;
+    // unit u covers tile u % total and the K-blocks of split u / total
+    const int nsplit = (p.partial != nullptr && p.tiles != nullptr) ? p.tiles[p.E + p.has_shared + 1] : 1;
+    const int units = total * nsplit;
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -275,8 +282,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             uint32_t ph = 0;
             uint32_t issued_mask = 0, issued_ph = 0;
             bool aborted = false;
-            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
-                const Tile t = decode_tile(p, tile);
+            for (int u = blockIdx.x; u < units && !aborted; u += gridDim.x) {
+                const int sp = u / total;
+                const Tile t = decode_tile(p, u - sp * total);
+                const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
                 const CUtensorMap* ma = t.kind ? &tmA1 : &tmA0;
                 const CUtensorMap* mb0 = t.kind ? &tmB10 : &tmB00;
                 const CUtensorMap* mb1 = t.kind ? &tmB11 : &tmB01;
@@ -289,7 +298,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                 } else {
                     brow0 = eoff + t.n_blk * 256; brow1 = brow0 + 128; mlo = mb0; mhi = mb0;
                 }
-                for (int kb = 0; kb < t.num_kb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bounded(&ctl->empty[s], ph ^ 1u, ctl, p)) { aborted = true; break; }
                     const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
                     mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
@@ -316,12 +325,14 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             int acc = 0;
             uint32_t aph = 0;
             bool aborted = false, issued_any = false;
-            for (int tile = blockIdx.x; tile < total && !aborted; tile += gridDim.x) {
-                const Tile t = decode_tile(p, tile);
+            for (int u = blockIdx.x; u < units && !aborted; u += gridDim.x) {
+                const int sp = u / total;
+                const Tile t = decode_tile(p, u - sp * total);
+                const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
                 if (!wait_bounded(&ctl->tempty[acc], aph ^ 1u, ctl, p)) { aborted = true; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
-                for (int kb = 0; kb < t.num_kb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bounded(&ctl->full[s], ph, ctl, p)) { aborted = true; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
@@ -329,7 +340,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                     const uint64_t bdesc = sw128_desc(sa + A_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        tc_mma(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
                     issued_any = true;
                     tc_commit(&ctl->empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -351,8 +362,9 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
         const int r = q * 32 + lane;            // accumulator row of this thread
         int acc = 0;
         uint32_t aph = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile(p, tile);
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            const int sp = u / total;
+            const Tile t = decode_tile(p, u - sp * total);
             if (!wait_bounded(&ctl->tfull[acc], aph, ctl, p)) break;
             tc_fence_after();
             const int grow = t.m_blk * BM + r;
@@ -361,7 +373,22 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             const int N = p.N[t.kind];
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                 static_cast<uint32_t>(acc * ACC_COLS);
-            if (MODE == TC_SWIGLU) {
+            if (nsplit > 1) {
+                // fp32 partial of this split: the raw 256 accumulator columns
+                float* out = p.partial + static_cast<size_t>(sp) * p.partial_stride + orow * p.partial_ld;
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tb + c, v);
+                    const int col = t.n_blk * 256 + c;
+                    if (valid && col < p.partial_ld) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    }
+                }
+            } else if (MODE == TC_SWIGLU) {
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
 #pragma unroll 1
                 for (int c = 0; c < 128; c += 32) {
@@ -516,6 +543,9 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     kp.out[0] = a.out[0]; kp.out[1] = a.out[1];
     kp.status = a.status;
     kp.timeout_ns = a.timeout_ns > 0 ? a.timeout_ns : 2000000000LL;
+    kp.partial = a.partial;
+    kp.partial_stride = a.partial_stride;
+    kp.partial_ld = a.partial_ld;
     switch (a.mode) {
         case TC_SWIGLU: return launch_mode<TC_SWIGLU>(a, kp, maps, st);
         case TC_PLAIN: return launch_mode<TC_PLAIN>(a, kp, maps, st);

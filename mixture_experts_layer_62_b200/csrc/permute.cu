@@ -46,6 +46,20 @@ __device__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
     return excl;
 }
 
+// Split factor of a GEMM with `tiles` output tiles of `nkb` K-blocks on `sm`
+// persistent CTAs: the s in [1, smax] that minimises rounds x K-blocks per
+// unit, ceil(tiles * s / sm) * ceil(nkb / s) (the smaller s on ties).
+__device__ int pick_split(int tiles, int nkb, int sm, int smax) {
+    if (smax <= 1 || tiles <= 0 || sm <= 0) return 1;
+    long long best = -1;
+    int bs = 1;
+    for (int s = 1; s <= smax && s <= nkb; ++s) {
+        long long c = ((long long)tiles * s + sm - 1) / sm * ((nkb + s - 1) / s);
+        if (best < 0 || c < best) { best = c; bs = s; }
+    }
+    return bs;
+}
+
 // Tile schedule of a grouped GEMM: tiles[g] = sum_{g' < g} mtiles(g') * ntiles(g').
 __device__ void build_schedule(const int* rows, int G, int E, int tile_m, int nt, int nt_shared,
                                int32_t* tiles, int* warp_tot) {
@@ -165,6 +179,10 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) 
         build_schedule(rows, G, E, a.tile_m, a.ntiles13, a.ntiles13_shared, a.tiles13, warp_tot);
         __syncthreads();
         build_schedule(rows, G, E, a.tile_m, a.ntiles2, a.ntiles2_shared, a.tiles2, warp_tot);
+        if (threadIdx.x == 0) {
+            a.tiles13[G + 1] = pick_split(a.tiles13[G], a.nkb13, a.sm_count, a.split_max);
+            a.tiles2[G + 1] = pick_split(a.tiles2[G], a.nkb2, a.sm_count, a.split_max);
+        }
     }
 }
 
@@ -187,6 +205,10 @@ schedule_kernel(const int32_t* __restrict__ indptr, int E, int T, int has_shared
     build_schedule(rows, G, E, tile_m, nt13, nt13s, tiles13, warp_tot);
     __syncthreads();
     build_schedule(rows, G, E, tile_m, nt2, nt2s, tiles2, warp_tot);
+    if (threadIdx.x == 0) {   // the stage entry points never split K
+        tiles13[G + 1] = 1;
+        tiles2[G + 1] = 1;
+    }
 }
 
 cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,

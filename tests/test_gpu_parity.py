@@ -244,6 +244,9 @@ SMALL = [
     dict(T=1, d=512, d_ff=256, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     dict(T=64, d=256, d_ff=128, E=256, k=8, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=256),
     dict(T=257, d=64, d_ff=128, E=6, k=3, cf=0.25, dtype="f32", bias_mode=1, d_ff_shared=64),
+    # T*k <= 128 rows: moe_forward may split K of both GEMMs (fp32 partials)
+    dict(T=16, d=1024, d_ff=512, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    dict(T=5, d=256, d_ff=1024, E=4, k=2, cf=0.0, dtype="bf16", bias_mode=1, d_ff_shared=0),
 ]
 
 
