@@ -315,6 +315,7 @@ def main():
 
     import mixture_experts_layer_62_b200 as moe
     import torch.distributed as dist
+    from mixture_experts_layer_62_b200 import parallel
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
@@ -335,16 +336,13 @@ def main():
     E = cfg["E"]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    gstats = torch.zeros(2 * E, dtype=torch.float64, device=dev)
 
     def step():
         layer(x)
         if world > 1:
-            # global load statistics: counts and sum of probabilities over ranks
-            cnt = layer.stats[32:32 + 4 * E].view(torch.int32).to(torch.float64)
-            psum = layer.stats[32 + 8 * E:32 + 12 * E].view(torch.float32).to(torch.float64) * cfg["T"]
-            torch.cat([cnt, psum], out=gstats)
-            dist.all_reduce(gstats)
+            # the one exchange of data-parallel replicas: global load statistics
+            v = parallel._local_vector(layer.stats, E, cfg["T"])
+            dist.all_reduce(v)
 
     def barrier():
         if world > 1:
@@ -378,6 +376,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     job_ms = float(t.item())
     st = layer.read_stats()
+    gst = parallel.global_stats(layer.stats, E, cfg["k"], cfg["T"]) if world > 1 else None
     if st.status != moe.MOE_OK:
         raise SystemExit(f"device status {st.status}: {moe.error_string(st.status)}")
     tokens_total = cfg["T"] * world * args.steps
@@ -442,6 +441,9 @@ def main():
                     "experts_touched": touched_experts(st), "counts": st.counts if E <= 16 else None,
                     "kept": st.kept if E <= 16 else None},
     }
+    if gst is not None:
+        line["global_stats"] = {"T": gst.T, "l_aux": gst.l_aux, "dropped": gst.dropped,
+                                "max_over_mean": gst.max_over_mean}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gidx = moe.workspace_view(layer.workspace, p, "idx").cpu().numpy()
         n, dt = oracle_sample(cfg, L, args.cpu_sample, needed_experts=lambda toks: gidx[toks].reshape(-1).tolist())

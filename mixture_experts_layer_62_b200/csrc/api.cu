@@ -311,6 +311,23 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     int32_t* tiles13 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles13));
     int32_t* tiles2 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles2));
 
+    const bool split = split_allowed(*p);
+    void* xp = wsp(workspace, L.xp);
+    if (small_route_ok(*p)) {
+        // decode-sized batch: routing, statistics, schedules and the gather in one block
+        SmallRouteArgs sr = {};
+        sr.x = x; sr.W_r = W_r; sr.bias = bias;
+        sr.bias_mode = p->bias_mode; sr.T = p->T; sr.d = p->d; sr.E = p->E; sr.k = p->k; sr.capacity = C;
+        sr.logits = logits; sr.idx = idx; sr.gate = gate; sr.pos = pos; sr.indptr = indptr; sr.row_token = row_token;
+        sr.xp = xp; sr.stats = stats; sr.tiles13 = tiles13; sr.tiles2 = tiles2;
+        int tile_m, nt13s, nt2s;
+        schedule_sizes(p, tile_m, sr.nt13, sr.nt2, nt13s, nt2s);
+        sr.split_max = split ? kSplitMax : 1;
+        sr.sm_count = device_sm_count();
+        sr.nkb13 = ceil_div(p->d, 64);
+        sr.nkb2 = ceil_div(p->d_ff, 64);
+        CK(launch_route_small(sr, st));
+    } else {
     rc = run_logits(p, x, W_r, logits, L, workspace, status, st);
     if (rc != MOE_OK) return rc;
     CK(launch_select(logits, bias, p->bias_mode, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum, st));
@@ -320,15 +337,14 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     sa.indptr = indptr; sa.stats = stats;
     sa.tiles13 = tiles13; sa.tiles2 = tiles2; sa.has_shared = shared ? 1 : 0;
     schedule_sizes(p, sa.tile_m, sa.ntiles13, sa.ntiles2, sa.ntiles13_shared, sa.ntiles2_shared);
-    const bool split = split_allowed(*p);
     sa.split_max = split ? kSplitMax : 1;
     sa.sm_count = device_sm_count();
     sa.nkb13 = ceil_div(p->d, 64);
     sa.nkb2 = ceil_div(p->d_ff, 64);
     CK(launch_scan(sa, st));
-    void* xp = wsp(workspace, L.xp);
     CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, C, pos, row_token, xp,
                              st));
+    }
     void* h = wsp(workspace, L.h);
     void* o = wsp(workspace, L.o);
     void* hs = shared ? wsp(workspace, L.hs) : nullptr;

@@ -42,17 +42,24 @@ template <> struct VecTraits<__nv_bfloat16> {
     }
 };
 
-// With split-K partials (opart != null and *split2 > 1) an expert output row
-// is the sum over the splits, s = 0, 1, ..., of the fp32 partial rows.
+// One warp per (token, slice of the row): a slice is 32 x kCbVecPerLane
+// 16-byte vectors, so small batches still spread over the whole GPU. With
+// split-K partials (opart != null and *split2 > 1) an expert output row is the
+// sum over the splits, s = 0, 1, ..., of the fp32 partial rows.
+constexpr int kCbVecPerLane = 2;
+constexpr int kCbWarps = 8;
+
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kCbWarps * 32, 4)
 combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const float* __restrict__ gate,
                const T* __restrict__ s, T* __restrict__ out, int Tn, int d, int k,
-               const float* __restrict__ opart, long long opart_stride, const int32_t* __restrict__ split2) {
+               const float* __restrict__ opart, long long opart_stride, const int32_t* __restrict__ split2,
+               int slices) {
     using V = VecTraits<T>;
     constexpr int VN = V::N;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+    const long long task = (long long)blockIdx.x * kCbWarps + warp;
+    const int t = (int)(task / slices), sl = (int)(task % slices);
     if (t >= Tn) return;
     const int S = (opart != nullptr && split2 != nullptr) ? *split2 : 1;
     int p[MOE_MAX_K];
@@ -65,37 +72,40 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const f
         }
     }
     const int nvec = d / VN;
-    for (int v = lane; v < nvec; v += 32) {
+#pragma unroll
+    for (int i = 0; i < kCbVecPerLane; ++i) {
+        const int v = (sl * kCbVecPerLane + i) * 32 + lane;
+        if (v >= nvec) break;
         float acc[VN];
 #pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-#pragma unroll
+        for (int e = 0; e < VN; ++e) acc[e] = 0.f;
+#pragma unroll 4
         for (int j = 0; j < MOE_MAX_K; ++j) {
             if (j < k && p[j] >= 0) {
                 float ov[VN];
                 if (S > 1) {
 #pragma unroll
-                    for (int i = 0; i < VN; ++i) ov[i] = 0.f;
+                    for (int e = 0; e < VN; ++e) ov[e] = 0.f;
                     for (int sp = 0; sp < S; ++sp) {
                         const float* src = opart + (size_t)sp * opart_stride + (size_t)p[j] * d + (size_t)v * VN;
 #pragma unroll
-                        for (int i = 0; i < VN; i += 4) {
-                            float4 q4 = *reinterpret_cast<const float4*>(src + i);
-                            ov[i] += q4.x; ov[i + 1] += q4.y; ov[i + 2] += q4.z; ov[i + 3] += q4.w;
+                        for (int e = 0; e < VN; e += 4) {
+                            float4 q4 = *reinterpret_cast<const float4*>(src + e);
+                            ov[e] += q4.x; ov[e + 1] += q4.y; ov[e + 2] += q4.z; ov[e + 3] += q4.w;
                         }
                     }
                 } else {
                     V::load(o + (size_t)p[j] * d + (size_t)v * VN, ov);
                 }
 #pragma unroll
-                for (int i = 0; i < VN; ++i) acc[i] = fmaf(g[j], ov[i], acc[i]);
+                for (int e = 0; e < VN; ++e) acc[e] = fmaf(g[j], ov[e], acc[e]);
             }
         }
         if (s != nullptr) {
             float sv[VN];
             V::load(s + (size_t)t * d + (size_t)v * VN, sv);
 #pragma unroll
-            for (int i = 0; i < VN; ++i) acc[i] += sv[i];
+            for (int e = 0; e < VN; ++e) acc[e] += sv[e];
         }
         V::store(out + (size_t)t * d + (size_t)v * VN, acc);
     }
@@ -105,15 +115,17 @@ cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const f
                            const void* s, void* out, int T, int d, int k, cudaStream_t st,
                            const float* opart, long long opart_stride, const int32_t* split2) {
     if (T == 0) return cudaSuccess;
-    const int per_block = 8;
-    dim3 grid(ceil_div(T, per_block)), block(per_block * 32);
+    const int vn = dtype == MOE_DTYPE_BF16 ? 8 : 4;
+    const int slices = ceil_div(d / vn, 32 * kCbVecPerLane);
+    const long long tasks = (long long)T * slices;
+    const unsigned grid = (unsigned)((tasks + kCbWarps - 1) / kCbWarps);
     if (dtype == MOE_DTYPE_BF16)
-        combine_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
+        combine_kernel<__nv_bfloat16><<<grid, kCbWarps * 32, 0, st>>>(
             (const __nv_bfloat16*)o, pos, gate, (const __nv_bfloat16*)s, (__nv_bfloat16*)out, T, d, k, opart,
-            opart_stride, split2);
+            opart_stride, split2, slices);
     else
-        combine_kernel<float><<<grid, block, 0, st>>>((const float*)o, pos, gate, (const float*)s,
-                                                      (float*)out, T, d, k, nullptr, 0, nullptr);
+        combine_kernel<float><<<grid, kCbWarps * 32, 0, st>>>((const float*)o, pos, gate, (const float*)s,
+                                                              (float*)out, T, d, k, nullptr, 0, nullptr, slices);
     return cudaGetLastError();
 }
 
@@ -130,24 +142,32 @@ swiglu_reduce_kernel(const float* __restrict__ part, long long split_stride, int
     if (S <= 1) return;
     const int r = blockIdx.x;
     if (r >= indptr[E]) return;
-    for (int c = threadIdx.x; c < d_ff; c += blockDim.x) {
-        const size_t col = (size_t)(c / 128) * 256 + (c % 128);
-        float g = 0.f, u = 0.f;
-        for (int sp = 0; sp < S; ++sp) {
-            const float* row = part + (size_t)sp * split_stride + (size_t)r * ld;
-            g += row[col];
-            u += row[col + 128];
-        }
-        h[(size_t)r * d_ff + c] = __float2bfloat16_rn(g / (1.f + __expf(-g)) * u);
+    const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;   // 4 columns inside one 128-column group
+    if (c >= d_ff) return;
+    const size_t col = (size_t)(c / 128) * 256 + (c % 128);
+    float4 g = make_float4(0.f, 0.f, 0.f, 0.f), u = g;
+    for (int sp = 0; sp < S; ++sp) {
+        const float* row = part + (size_t)sp * split_stride + (size_t)r * ld;
+        const float4 a = *reinterpret_cast<const float4*>(row + col);
+        const float4 b = *reinterpret_cast<const float4*>(row + col + 128);
+        g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
+        u.x += b.x; u.y += b.y; u.z += b.z; u.w += b.w;
     }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(g.x / (1.f + __expf(-g.x)) * u.x, g.y / (1.f + __expf(-g.y)) * u.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(g.z / (1.f + __expf(-g.z)) * u.z, g.w / (1.f + __expf(-g.w)) * u.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(h + (size_t)r * d_ff + c) = packed;
 }
 
 cudaError_t launch_swiglu_reduce(const float* part, long long split_stride, int ld, const int32_t* split13,
                                  const int32_t* indptr, int E, int max_rows, int d_ff, void* h,
                                  cudaStream_t st) {
     if (max_rows <= 0) return cudaSuccess;
-    swiglu_reduce_kernel<<<max_rows, 256, 0, st>>>(part, split_stride, ld, split13, indptr, E, d_ff,
-                                                   (__nv_bfloat16*)h);
+    dim3 grid(max_rows, ceil_div(d_ff, 256 * 4));
+    swiglu_reduce_kernel<<<grid, 256, 0, st>>>(part, split_stride, ld, split13, indptr, E, d_ff,
+                                               (__nv_bfloat16*)h);
     return cudaGetLastError();
 }
 

@@ -79,6 +79,23 @@ cudaError_t launch_swiglu_reduce(const float* part, long long split_stride, int 
                                  cudaStream_t st);
 cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st);
 
+// Small-batch router (T*k <= kSmallMaxPairs, E <= kSmallMaxE, E % 8 == 0,
+// bf16, no shared expert): logits, selection, statistics, capacity, indptr,
+// tile schedules with split factors, destinations and the row gather in one
+// single-block kernel.
+constexpr int kSmallMaxPairs = 64;
+constexpr int kSmallMaxE = 64;
+struct SmallRouteArgs {
+    const void* x; const void* W_r; const float* bias;
+    int bias_mode, T, d, E, k, capacity;
+    float* logits; int32_t* idx; float* gate; int32_t* pos; int32_t* indptr; int32_t* row_token;
+    void* xp; void* stats;
+    int32_t* tiles13; int32_t* tiles2;
+    int nt13, nt2, split_max, sm_count, nkb13, nkb2;
+};
+bool small_route_ok(const moe_problem& p);
+cudaError_t launch_route_small(const SmallRouteArgs& a, cudaStream_t st);
+
 // fp32 grouped GEMM on CUDA cores (the fp32 path). Tile 64 x 64.
 constexpr int kSimtTileM = 64;
 constexpr int kSimtTileN = 64;
@@ -117,6 +134,20 @@ struct TcArgs {
     int partial_ld;            // elements per row
 };
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
+
+// Split factor of a GEMM with `tiles` output tiles of `nkb` K-blocks on `sm`
+// persistent CTAs: the s in [1, smax] that minimises rounds x K-blocks per
+// unit, ceil(tiles * s / sm) * ceil(nkb / s) (the smaller s on ties).
+__device__ inline int pick_split(int tiles, int nkb, int sm, int smax) {
+    if (smax <= 1 || tiles <= 0 || sm <= 0) return 1;
+    long long best = -1;
+    int bs = 1;
+    for (int s = 1; s <= smax && s <= nkb; ++s) {
+        long long c = ((long long)tiles * s + sm - 1) / sm * ((nkb + s - 1) / s);
+        if (best < 0 || c < best) { best = c; bs = s; }
+    }
+    return bs;
+}
 
 int device_sm_count();
 

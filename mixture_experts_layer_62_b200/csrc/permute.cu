@@ -46,20 +46,6 @@ __device__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
     return excl;
 }
 
-// Split factor of a GEMM with `tiles` output tiles of `nkb` K-blocks on `sm`
-// persistent CTAs: the s in [1, smax] that minimises rounds x K-blocks per
-// unit, ceil(tiles * s / sm) * ceil(nkb / s) (the smaller s on ties).
-__device__ int pick_split(int tiles, int nkb, int sm, int smax) {
-    if (smax <= 1 || tiles <= 0 || sm <= 0) return 1;
-    long long best = -1;
-    int bs = 1;
-    for (int s = 1; s <= smax && s <= nkb; ++s) {
-        long long c = ((long long)tiles * s + sm - 1) / sm * ((nkb + s - 1) / s);
-        if (best < 0 || c < best) { best = c; bs = s; }
-    }
-    return bs;
-}
-
 // Tile schedule of a grouped GEMM: tiles[g] = sum_{g' < g} mtiles(g') * ntiles(g').
 __device__ void build_schedule(const int* rows, int G, int E, int tile_m, int nt, int nt_shared,
                                int32_t* tiles, int* warp_tot) {
@@ -82,27 +68,41 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) 
     __shared__ int kept_s[MOE_MAX_E + 1];
     __shared__ float fP[MOE_MAX_E];
     const int E = a.E;
-    const long long n = (long long)E * NB;
 
-    // 1. global exclusive scan of blockcnt (expert-major), written to blockoff
+    // 1. per expert row of chunk counts (expert-major order, chunk inner):
+    //    exclusive prefix inside the row -> blockoff, row total -> start[e].
+    //    One warp per row, 32 consecutive entries per step (coalesced).
     {
-        const long long per = (n + kScanThreads - 1) / kScanThreads;
-        const long long lo = min(n, per * threadIdx.x), hi = min(n, lo + per);
-        int local = 0;
-        for (long long i = lo; i < hi; ++i) local += a.blockcnt[i];
-        int tot;
-        int run = block_exclusive_scan(local, warp_tot, tot);
-        for (long long i = lo; i < hi; ++i) {
-            int c = a.blockcnt[i];
-            a.blockoff[i] = run;
-            if (i % NB == 0) start[i / NB] = run;
-            run += c;
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+        for (int e = warp; e < E; e += nw) {
+            const int32_t* row = a.blockcnt + (size_t)e * NB;
+            int32_t* orow = a.blockoff + (size_t)e * NB;
+            int carry = 0;
+            for (int b0 = 0; b0 < NB; b0 += 32) {
+                const int b = b0 + lane;
+                const int v = b < NB ? row[b] : 0;
+                int incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    int n_ = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += n_;
+                }
+                if (b < NB) orow[b] = carry + incl - v;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) start[e] = carry;   // c_e (converted to a prefix below)
         }
+    }
+    __syncthreads();
+    // 2. per-expert counts -> exclusive prefix over experts in start[]
+    {
+        int c_e = threadIdx.x < E ? start[threadIdx.x] : 0;
+        int tot;
+        int ex = block_exclusive_scan(c_e, warp_tot, tot);
+        if (threadIdx.x < E) start[threadIdx.x] = ex;
         if (threadIdx.x == 0) start[E] = tot;
     }
     __syncthreads();
-    // 2. make the chunk bases relative to their expert's first pair
-    for (long long i = threadIdx.x; i < n; i += kScanThreads) a.blockoff[i] -= start[i / NB];
 
     // 3. counts, capacity, kept and indptr over kept rows
     int c = 0, kp = 0;
@@ -219,7 +219,10 @@ cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared,
     return cudaGetLastError();
 }
 
-// Ranks, destinations and the row gather. One block per chunk.
+// Ranks, destinations and the row gather. Block (chunk, column group): every
+// block of a chunk derives the chunk's destinations (a few hundred integer
+// compares), the column-group-0 block writes pos and row_token, and each
+// block gathers its slice of the row vectors.
 // Gather: xp[pos[t, j]] = x[t] for every kept pair, 16-byte vectors; each
 // source vector is read once and written to all of the token's kept rows.
 __global__ void __launch_bounds__(256)
@@ -231,6 +234,9 @@ permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ i
     __shared__ int sidx[kChunk][MOE_MAX_K];
     __shared__ int spos[kChunk][MOE_MAX_K];
     const int chunk = blockIdx.x, NB = gridDim.x;
+    const bool writer = blockIdx.y == 0;
+    const int vper = (nvec + gridDim.y - 1) / gridDim.y;
+    const int v_lo = blockIdx.y * vper, v_hi = min(nvec, v_lo + vper);
     const int t0 = chunk * kChunk;
     const int ntok = min(kChunk, Tn - t0);
     for (int i = threadIdx.x; i < ntok * k; i += blockDim.x)
@@ -241,7 +247,7 @@ permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ i
         const int e = sidx[q][j];
         if (e < 0 || e >= E) {   // not an expert: the pair takes no row
             spos[q][j] = -1;
-            pos[(size_t)(t0 + q) * k + j] = -1;
+            if (writer) pos[(size_t)(t0 + q) * k + j] = -1;
             continue;
         }
         int before = 0;
@@ -251,8 +257,10 @@ permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ i
         int p = -1;
         if (capacity < 0 || rank < capacity) p = indptr[e] + rank;
         spos[q][j] = p;
-        pos[(size_t)(t0 + q) * k + j] = p;
-        if (p >= 0 && row_token != nullptr) row_token[p] = t0 + q;
+        if (writer) {
+            pos[(size_t)(t0 + q) * k + j] = p;
+            if (p >= 0 && row_token != nullptr) row_token[p] = t0 + q;
+        }
     }
     __syncthreads();
     if (xp == nullptr) return;
@@ -264,7 +272,7 @@ permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ i
         for (int j = 0; j < k; ++j)
             if (spos[q][j] >= 0) dst[nd++] = spos[q][j];
         if (nd == 0) continue;
-        for (int v = lane; v < nvec; v += 32) {
+        for (int v = v_lo + lane; v < v_hi; v += 32) {
             uint4 val = src[v];
             for (int j = 0; j < nd; ++j) xp[(size_t)dst[j] * nvec + v] = val;
         }
@@ -278,8 +286,14 @@ cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
     int NB = ceil_div(T, kChunk);
     if (NB == 0) return cudaSuccess;
     int nvec = (int)((size_t)d * elem_bytes(dtype) / 16);
-    permute_gather_kernel<<<NB, 256, 0, st>>>((const uint4*)x, idx, blockoff, indptr, T, nvec, E, k,
-                                              capacity, pos, row_token, (uint4*)xp);
+    // column groups so that small batches still cover the GPU (~4 blocks per SM)
+    int sms = device_sm_count();
+    if (sms <= 0) sms = 148;
+    int groups = xp == nullptr ? 1 : ceil_div(4 * sms, NB);
+    groups = max(1, min(groups, ceil_div(nvec, 32)));
+    dim3 grid(NB, groups);
+    permute_gather_kernel<<<grid, 256, 0, st>>>((const uint4*)x, idx, blockoff, indptr, T, nvec, E, k,
+                                                capacity, pos, row_token, (uint4*)xp);
     return cudaGetLastError();
 }
 

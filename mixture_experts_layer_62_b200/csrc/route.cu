@@ -38,13 +38,15 @@ cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, in
 }
 
 // ---- logits on CUDA cores -------------------------------------------------
-// One warp per group of kTokPerWarp tokens. Lane l owns the 8-element chunks
-// c = l, l + 32, ... of the row; per chunk it loads the tokens' x once and the
-// chunk of each of 8 experts' W_r^T rows, and accumulates acc[token][expert]
-// over its chunks in ascending order. The 32 lane partials of every logit are
-// then summed by an xor butterfly. The summation order is fixed, so the same
-// inputs always give the same bits. Experts are taken 8 at a time.
-constexpr int kTokPerWarp = 4;
+// One block per group of kLgTok tokens; its kLgWarps warps split the row into
+// contiguous slices of 8-element chunks (lane l takes chunks l, l + 32, ... of
+// its warp's slice). Per chunk a lane loads the tokens' x once and the chunk
+// of each of 8 experts' W_r^T rows, accumulating acc[token][expert] in
+// ascending chunk order. Lane partials are summed by an xor butterfly, warp
+// partials in warp order through shared memory: the summation order is fixed,
+// so the same inputs always give the same bits. Experts are taken 8 at a time.
+constexpr int kLgTok = 4;
+constexpr int kLgWarps = 8;
 constexpr int kExpPerPass = 8;
 
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
@@ -63,26 +65,26 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kLgWarps * 32)
 logits_kernel(const T* __restrict__ x, const T* __restrict__ wrt, float* __restrict__ logits, int Tn, int d,
               int E) {
-    const int lane = threadIdx.x & 31;
-    const int t0 = ((blockIdx.x * blockDim.x + threadIdx.x) >> 5) * kTokPerWarp;
-    if (t0 >= Tn) return;
+    __shared__ float part[kLgWarps][kLgTok][kExpPerPass];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kLgTok;
+    const int nt = min(kLgTok, Tn - t0);
     const int nchunk = d / 8;
-    int nt = Tn - t0;
-    if (nt > kTokPerWarp) nt = kTokPerWarp;
+    const int per = (nchunk + kLgWarps - 1) / kLgWarps;
+    const int c_lo = warp * per, c_hi = min(nchunk, c_lo + per);
     for (int e0 = 0; e0 < E; e0 += kExpPerPass) {
-        float acc[kTokPerWarp][kExpPerPass];
+        float acc[kLgTok][kExpPerPass];
 #pragma unroll
-        for (int q = 0; q < kTokPerWarp; ++q)
+        for (int q = 0; q < kLgTok; ++q)
 #pragma unroll
             for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = 0.f;
-#pragma unroll 2
-        for (int c = lane; c < nchunk; c += 32) {
-            float xv[kTokPerWarp][8];
+        for (int c = c_lo + lane; c < c_hi; c += 32) {
+            float xv[kLgTok][8];
 #pragma unroll
-            for (int q = 0; q < kTokPerWarp; ++q) {
+            for (int q = 0; q < kLgTok; ++q) {
                 if (q < nt) {
                     load8(x + (size_t)(t0 + q) * d + (size_t)c * 8, xv[q]);
                 } else {
@@ -96,36 +98,44 @@ logits_kernel(const T* __restrict__ x, const T* __restrict__ wrt, float* __restr
                     float wv[8];
                     load8(wrt + (size_t)(e0 + e) * d + (size_t)c * 8, wv);
 #pragma unroll
-                    for (int q = 0; q < kTokPerWarp; ++q)
+                    for (int q = 0; q < kLgTok; ++q)
 #pragma unroll
                         for (int j = 0; j < 8; ++j) acc[q][e] = fmaf(xv[q][j], wv[j], acc[q][e]);
                 }
             }
         }
 #pragma unroll
-        for (int q = 0; q < kTokPerWarp; ++q) {
+        for (int q = 0; q < kLgTok; ++q) {
 #pragma unroll
             for (int e = 0; e < kExpPerPass; ++e) {
                 float v = acc[q][e];
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0 && q < nt && e0 + e < E) logits[(size_t)(t0 + q) * E + e0 + e] = v;
+                if (lane == 0) part[warp][q][e] = v;
             }
         }
+        __syncthreads();
+        if (threadIdx.x < kLgTok * kExpPerPass) {
+            const int q = threadIdx.x / kExpPerPass, e = threadIdx.x % kExpPerPass;
+            if (q < nt && e0 + e < E) {
+                float v = 0.f;
+                for (int w = 0; w < kLgWarps; ++w) v += part[w][q][e];
+                logits[(size_t)(t0 + q) * E + e0 + e] = v;
+            }
+        }
+        __syncthreads();
     }
 }
 
 cudaError_t launch_logits_simt(int dtype, const void* x, const void* wrt, float* logits,
                                int T, int d, int E, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    const int warps = ceil_div(T, kTokPerWarp);
-    const int block = 128;
-    const int grid = ceil_div(warps * 32, block);
+    const int grid = ceil_div(T, kLgTok);
     if (dtype == MOE_DTYPE_BF16)
-        logits_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
+        logits_kernel<__nv_bfloat16><<<grid, kLgWarps * 32, 0, st>>>(
             (const __nv_bfloat16*)x, (const __nv_bfloat16*)wrt, logits, T, d, E);
     else
-        logits_kernel<float><<<grid, block, 0, st>>>((const float*)x, (const float*)wrt, logits, T, d, E);
+        logits_kernel<float><<<grid, kLgWarps * 32, 0, st>>>((const float*)x, (const float*)wrt, logits, T, d, E);
     return cudaGetLastError();
 }
 

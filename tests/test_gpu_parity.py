@@ -247,6 +247,10 @@ SMALL = [
     # T*k <= 128 rows: moe_forward may split K of both GEMMs (fp32 partials)
     dict(T=16, d=1024, d_ff=512, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     dict(T=5, d=256, d_ff=1024, E=4, k=2, cf=0.0, dtype="bf16", bias_mode=1, d_ff_shared=0),
+    # T*k <= 64, E % 8 == 0, E <= 64: the single-block small-batch router
+    dict(T=20, d=256, d_ff=256, E=64, k=2, cf=0.5, dtype="bf16", bias_mode=1, d_ff_shared=0),
+    dict(T=8, d=512, d_ff=256, E=16, k=4, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=0),
+    dict(T=3, d=128, d_ff=128, E=8, k=8, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
 ]
 
 
