@@ -29,7 +29,8 @@ Layout make_layout(const moe_problem& p) {
     L.wrt = take(E * d * eb);
     L.blockcnt = take(E * NB * 4);
     L.blockoff = take(E * NB * 4);
-    L.blockpsum = take(NB * E * 4);
+    // per-chunk probability sums; the small-batch router keeps [T][E] probabilities here
+    L.blockpsum = take((small_route_ok(p) ? T : NB) * E * 4);
     L.tiles13 = take((E + 3) * 4);
     L.tiles2 = take((E + 3) * 4);
     L.xp = take(T * k * d * eb);
@@ -48,6 +49,9 @@ bool split_allowed(const moe_problem& p) {
     return p.dtype == MOE_DTYPE_BF16 && p.d_ff_shared == 0 && p.T > 0 &&
            (long long)p.T * p.k <= kSplitMaxRows;
 }
+
+thread_local bool g_pdl = false;
+thread_local bool g_pdl_pass = false;
 
 int device_sm_count() {
     static int cache[64] = {};
@@ -106,9 +110,10 @@ char* wsp(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
 
 // Router: logits (fp32) for all tokens into `logits`.
 int run_logits(const moe_problem* p, const void* x, const void* W_r, float* logits, const Layout& L,
-               void* ws, int32_t* status, cudaStream_t st) {
+               void* ws, int32_t* status, cudaStream_t st, bool reset_status = false) {
     void* wrt = wsp(ws, L.wrt);
-    CK(launch_transpose_wr(p->dtype, W_r, wrt, p->d, p->E, st));
+    CK(launch_transpose_wr(p->dtype, W_r, wrt, p->d, p->E, st, reset_status ? status : nullptr));
+    g_pdl_after_first();
     if (p->dtype == MOE_DTYPE_BF16 && p->E >= 64 && p->E % 32 == 0) {
         // wide routers (e.g. 256 experts) are a real GEMM: tensor cores, fp32 out
         TcArgs a = {};
@@ -298,7 +303,12 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
         CK(launch_zero_stats(stats, p->E, C, st));
         return MOE_OK;
     }
-    CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
+    // launches after the first overlap their predecessor (programmatic
+    // dependent launch); the first kernel resets the status word
+    struct PdlPass {
+        PdlPass() { g_pdl_pass = true; g_pdl = false; }
+        ~PdlPass() { g_pdl_pass = false; g_pdl = false; }
+    } pdl_pass;
     float* logits = reinterpret_cast<float*>(wsp(workspace, L.logits));
     int32_t* idx = reinterpret_cast<int32_t*>(wsp(workspace, L.idx));
     float* gate = reinterpret_cast<float*>(wsp(workspace, L.gate));
@@ -318,8 +328,8 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
         SmallRouteArgs sr = {};
         sr.x = x; sr.W_r = W_r; sr.bias = bias;
         sr.bias_mode = p->bias_mode; sr.T = p->T; sr.d = p->d; sr.E = p->E; sr.k = p->k; sr.capacity = C;
-        sr.logits = logits; sr.idx = idx; sr.gate = gate; sr.pos = pos; sr.indptr = indptr; sr.row_token = row_token;
-        sr.xp = xp; sr.stats = stats; sr.tiles13 = tiles13; sr.tiles2 = tiles2;
+        sr.logits = logits; sr.probs = blockpsum; sr.idx = idx; sr.gate = gate; sr.pos = pos; sr.indptr = indptr; sr.row_token = row_token;
+        sr.xp = xp; sr.stats = stats; sr.tiles13 = tiles13; sr.tiles2 = tiles2; sr.status_reset = status;
         int tile_m, nt13s, nt2s;
         schedule_sizes(p, tile_m, sr.nt13, sr.nt2, nt13s, nt2s);
         sr.split_max = split ? kSplitMax : 1;
@@ -328,7 +338,7 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
         sr.nkb2 = ceil_div(p->d_ff, 64);
         CK(launch_route_small(sr, st));
     } else {
-    rc = run_logits(p, x, W_r, logits, L, workspace, status, st);
+    rc = run_logits(p, x, W_r, logits, L, workspace, status, st, /*reset_status=*/true);
     if (rc != MOE_OK) return rc;
     CK(launch_select(logits, bias, p->bias_mode, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum, st));
     ScanArgs sa = {};

@@ -57,6 +57,8 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const f
                int slices) {
     using V = VecTraits<T>;
     constexpr int VN = V::N;
+    pdl_wait();
+    pdl_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long task = (long long)blockIdx.x * kCbWarps + warp;
     const int t = (int)(task / slices), sl = (int)(task % slices);
@@ -120,13 +122,12 @@ cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const f
     const long long tasks = (long long)T * slices;
     const unsigned grid = (unsigned)((tasks + kCbWarps - 1) / kCbWarps);
     if (dtype == MOE_DTYPE_BF16)
-        combine_kernel<__nv_bfloat16><<<grid, kCbWarps * 32, 0, st>>>(
-            (const __nv_bfloat16*)o, pos, gate, (const __nv_bfloat16*)s, (__nv_bfloat16*)out, T, d, k, opart,
-            opart_stride, split2, slices);
-    else
-        combine_kernel<float><<<grid, kCbWarps * 32, 0, st>>>((const float*)o, pos, gate, (const float*)s,
-                                                              (float*)out, T, d, k, nullptr, 0, nullptr, slices);
-    return cudaGetLastError();
+        return launch_k(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(kCbWarps * 32), 0, st,
+                        (const __nv_bfloat16*)o, pos, gate, (const __nv_bfloat16*)s, (__nv_bfloat16*)out, T, d, k,
+                        opart, opart_stride, split2, slices);
+    return launch_k(combine_kernel<float>, dim3(grid), dim3(kCbWarps * 32), 0, st, (const float*)o, pos, gate,
+                    (const float*)s, (float*)out, T, d, k, (const float*)nullptr, 0LL, (const int32_t*)nullptr,
+                    slices);
 }
 
 // Split-K reduction of grouped GEMM 1/3: the partial rows hold, per 128
@@ -138,6 +139,8 @@ __global__ void __launch_bounds__(256)
 swiglu_reduce_kernel(const float* __restrict__ part, long long split_stride, int ld,
                      const int32_t* __restrict__ split13, const int32_t* __restrict__ indptr, int E, int d_ff,
                      __nv_bfloat16* __restrict__ h) {
+    pdl_wait();
+    pdl_launch();
     const int S = *split13;
     if (S <= 1) return;
     const int r = blockIdx.x;
@@ -166,9 +169,8 @@ cudaError_t launch_swiglu_reduce(const float* part, long long split_stride, int 
                                  cudaStream_t st) {
     if (max_rows <= 0) return cudaSuccess;
     dim3 grid(max_rows, ceil_div(d_ff, 256 * 4));
-    swiglu_reduce_kernel<<<grid, 256, 0, st>>>(part, split_stride, ld, split13, indptr, E, d_ff,
-                                               (__nv_bfloat16*)h);
-    return cudaGetLastError();
+    return launch_k(swiglu_reduce_kernel, grid, dim3(256), 0, st, part, split_stride, ld, split13, indptr, E, d_ff,
+                    (__nv_bfloat16*)h);
 }
 
 }  // namespace moe

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe.h"
 
 namespace moe {
@@ -15,6 +17,41 @@ namespace moe {
 constexpr int kChunk = 32;
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Programmatic dependent launch. moe_forward launches every kernel after its
+// first one with the programmatic-serialization attribute, so a kernel's
+// launch and prologue overlap the tail of the kernel before it. Every kernel
+// calls pdl_wait() before it touches anything an earlier kernel of the pass
+// wrote (the wait returns once the preceding grid has completed and its
+// writes are visible; without the attribute it returns at once), then
+// pdl_launch() to let the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Set by moe_forward (per host thread) while it enqueues the launches that
+// may overlap their predecessor: g_pdl_pass marks the pass, g_pdl turns the
+// attribute on once the pass's first kernel is enqueued.
+extern thread_local bool g_pdl;
+extern thread_local bool g_pdl_pass;
+inline void g_pdl_after_first() {
+    if (g_pdl_pass) g_pdl = true;
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = g_pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 inline size_t elem_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
@@ -33,12 +70,15 @@ struct Layout {
 // expert; the split factor (<= kSplitMax) is chosen on the device from the
 // real tile counts.
 constexpr int kSplitMaxRows = 128;
-constexpr int kSplitMax = 8;
+constexpr int kSplitMax = 16;
 bool split_allowed(const moe_problem& p);
 Layout make_layout(const moe_problem& p);
 
 // Kernel launchers (each returns cudaGetLastError() of its launches).
-cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, int E, cudaStream_t st);
+// status (may be null): the statistics' status word, reset to MOE_OK by the
+// first kernel of a pass.
+cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, int E, cudaStream_t st,
+                                int32_t* status = nullptr);
 cudaError_t launch_logits_simt(int dtype, const void* x, const void* wrt, float* logits,
                                int T, int d, int E, cudaStream_t st);
 cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
@@ -81,14 +121,15 @@ cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st)
 
 // Small-batch router (T*k <= kSmallMaxPairs, E <= kSmallMaxE, E % 8 == 0,
 // bf16, no shared expert): logits, selection, statistics, capacity, indptr,
-// tile schedules with split factors, destinations and the row gather in one
-// single-block kernel.
+// tile schedules with split factors, destinations and the row gather in two
+// launches (one block per token, then one finishing kernel).
 constexpr int kSmallMaxPairs = 64;
 constexpr int kSmallMaxE = 64;
 struct SmallRouteArgs {
     const void* x; const void* W_r; const float* bias;
     int bias_mode, T, d, E, k, capacity;
-    float* logits; int32_t* idx; float* gate; int32_t* pos; int32_t* indptr; int32_t* row_token;
+    float* logits; float* probs; int32_t* idx; float* gate; int32_t* pos; int32_t* indptr; int32_t* row_token;
+    int32_t* status_reset;
     void* xp; void* stats;
     int32_t* tiles13; int32_t* tiles2;
     int nt13, nt2, split_max, sm_count, nkb13, nkb2;
@@ -136,14 +177,15 @@ struct TcArgs {
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
 
 // Split factor of a GEMM with `tiles` output tiles of `nkb` K-blocks on `sm`
-// persistent CTAs: the s in [1, smax] that minimises rounds x K-blocks per
-// unit, ceil(tiles * s / sm) * ceil(nkb / s) (the smaller s on ties).
+// persistent CTAs: the s in [1, smax] that minimises rounds x (K-blocks per
+// unit + 1), ceil(tiles * s / sm) * (ceil(nkb / s) + 1); the + 1 charges each
+// unit one K-block of start/finish cost. The smaller s wins ties.
 __device__ inline int pick_split(int tiles, int nkb, int sm, int smax) {
     if (smax <= 1 || tiles <= 0 || sm <= 0) return 1;
     long long best = -1;
     int bs = 1;
     for (int s = 1; s <= smax && s <= nkb; ++s) {
-        long long c = ((long long)tiles * s + sm - 1) / sm * ((nkb + s - 1) / s);
+        long long c = ((long long)tiles * s + sm - 1) / sm * ((nkb + s - 1) / s + 1);
         if (best < 0 || c < best) { best = c; bs = s; }
     }
     return bs;

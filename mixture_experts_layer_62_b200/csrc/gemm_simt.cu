@@ -30,6 +30,8 @@ template <bool SWIGLU>
 __global__ void __launch_bounds__(256) simt_gemm_kernel(GroupedArgs a) {
     __shared__ float As[kBK][kSimtTileM + 4];
     __shared__ float Bs[SWIGLU ? 2 : 1][kBK][kSimtTileN + 4];
+    pdl_wait();
+    pdl_launch();
     const int G = a.E + a.has_shared;
     const int total = a.tiles[G];
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16 threads
@@ -108,9 +110,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(GroupedArgs a) {
 cudaError_t launch_simt_gemm(bool swiglu, const GroupedArgs& a, cudaStream_t st) {
     int grid = device_sm_count() * 4;
     if (grid <= 0) grid = 148 * 4;
-    if (swiglu) simt_gemm_kernel<true><<<grid, 256, 0, st>>>(a);
-    else simt_gemm_kernel<false><<<grid, 256, 0, st>>>(a);
-    return cudaGetLastError();
+    if (swiglu) return launch_k(simt_gemm_kernel<true>, dim3(grid), dim3(256), 0, st, a);
+    return launch_k(simt_gemm_kernel<false>, dim3(grid), dim3(256), 0, st, a);
 }
 
 }  // namespace moe

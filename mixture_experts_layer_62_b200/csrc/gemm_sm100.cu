@@ -269,9 +269,15 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
+    // everything above (barriers, TMEM, descriptor prefetch) overlapped the
+    // previous kernel; the schedule and the A rows are its outputs
+    pdl_wait();
+    pdl_launch();
     const int total = total_tiles(p, COLS_PER_TILE);
     // split-K: the device-chosen factor is stored after the tile schedule;
-    // unit u covers tile u % total and the K-blocks of split u / total
+    // unit u covers tile u / nsplit and the K-blocks of split u % nsplit, so
+    // CTAs running at the same time read different K ranges of the weights
+    // (spreading the traffic over all DRAM channels)
     const int nsplit = (p.partial != nullptr && p.tiles != nullptr) ? p.tiles[p.E + p.has_shared + 1] : 1;
     const int units = total * nsplit;
 
@@ -283,8 +289,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             uint32_t issued_mask = 0, issued_ph = 0;
             bool aborted = false;
             for (int u = blockIdx.x; u < units && !aborted; u += gridDim.x) {
-                const int sp = u / total;
-                const Tile t = decode_tile(p, u - sp * total);
+                const int sp = u % nsplit;
+                const Tile t = decode_tile(p, u / nsplit);
                 const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
                 const CUtensorMap* ma = t.kind ? &tmA1 : &tmA0;
                 const CUtensorMap* mb0 = t.kind ? &tmB10 : &tmB00;
@@ -326,8 +332,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             uint32_t aph = 0;
             bool aborted = false, issued_any = false;
             for (int u = blockIdx.x; u < units && !aborted; u += gridDim.x) {
-                const int sp = u / total;
-                const Tile t = decode_tile(p, u - sp * total);
+                const int sp = u % nsplit;
+                const Tile t = decode_tile(p, u / nsplit);
                 const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
                 if (!wait_bounded(&ctl->tempty[acc], aph ^ 1u, ctl, p)) { aborted = true; break; }
                 tc_fence_after();
@@ -363,8 +369,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
         int acc = 0;
         uint32_t aph = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const int sp = u / total;
-            const Tile t = decode_tile(p, u - sp * total);
+            const int sp = u % nsplit;
+            const Tile t = decode_tile(p, u / nsplit);
             if (!wait_bounded(&ctl->tfull[acc], aph, ctl, p)) break;
             tc_fence_after();
             const int grow = t.m_blk * BM + r;
@@ -502,9 +508,8 @@ cudaError_t launch_mode(const TcArgs& a, const KParams& kp, const CUtensorMap (&
     }
     int grid = device_sm_count();
     if (grid <= 0) return cudaErrorInvalidDevice;
-    tc_grouped_gemm<MODE><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                                maps[5], kp);
-    return cudaGetLastError();
+    return launch_k(tc_grouped_gemm<MODE>, dim3(grid), dim3(NUM_THREADS), (size_t)SMEM_BYTES, st, maps[0], maps[1],
+                    maps[2], maps[3], maps[4], maps[5], kp);
 }
 
 }  // namespace

@@ -67,6 +67,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) 
     __shared__ int start[MOE_MAX_E + 1];
     __shared__ int kept_s[MOE_MAX_E + 1];
     __shared__ float fP[MOE_MAX_E];
+    pdl_wait();
+    pdl_launch();
     const int E = a.E;
 
     // 1. per expert row of chunk counts (expert-major order, chunk inner):
@@ -188,8 +190,7 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) 
 
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st) {
     int NB = ceil_div(a.T, kChunk);
-    scan_kernel<<<1, kScanThreads, 0, st>>>(a, NB);
-    return cudaGetLastError();
+    return launch_k(scan_kernel, dim3(1), dim3(kScanThreads), 0, st, a, NB);
 }
 
 // Tile schedule from a given indptr (the standalone expert stage).
@@ -198,6 +199,8 @@ schedule_kernel(const int32_t* __restrict__ indptr, int E, int T, int has_shared
                 int nt13, int nt2, int nt13s, int nt2s, int32_t* tiles13, int32_t* tiles2) {
     __shared__ int warp_tot[33];
     __shared__ int rows[MOE_MAX_E + 1];
+    pdl_wait();
+    pdl_launch();
     for (int g = threadIdx.x; g < E; g += blockDim.x) rows[g] = indptr[g + 1] - indptr[g];
     if (threadIdx.x == 0) rows[E] = T;
     __syncthreads();
@@ -214,9 +217,8 @@ schedule_kernel(const int32_t* __restrict__ indptr, int E, int T, int has_shared
 cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
                             int ntiles13, int ntiles2, int ntiles13_shared, int ntiles2_shared,
                             int32_t* tiles13, int32_t* tiles2, cudaStream_t st) {
-    schedule_kernel<<<1, kScanThreads, 0, st>>>(indptr, E, T, has_shared, tile_m, ntiles13, ntiles2,
-                                                ntiles13_shared, ntiles2_shared, tiles13, tiles2);
-    return cudaGetLastError();
+    return launch_k(schedule_kernel, dim3(1), dim3(kScanThreads), 0, st, indptr, E, T, has_shared, tile_m, ntiles13,
+                    ntiles2, ntiles13_shared, ntiles2_shared, tiles13, tiles2);
 }
 
 // Ranks, destinations and the row gather. Block (chunk, column group): every
@@ -233,6 +235,8 @@ permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ i
                       uint4* __restrict__ xp) {
     __shared__ int sidx[kChunk][MOE_MAX_K];
     __shared__ int spos[kChunk][MOE_MAX_K];
+    pdl_wait();
+    pdl_launch();
     const int chunk = blockIdx.x, NB = gridDim.x;
     const bool writer = blockIdx.y == 0;
     const int vper = (nvec + gridDim.y - 1) / gridDim.y;
@@ -292,13 +296,14 @@ cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
     int groups = xp == nullptr ? 1 : ceil_div(4 * sms, NB);
     groups = max(1, min(groups, ceil_div(nvec, 32)));
     dim3 grid(NB, groups);
-    permute_gather_kernel<<<grid, 256, 0, st>>>((const uint4*)x, idx, blockoff, indptr, T, nvec, E, k,
-                                                capacity, pos, row_token, (uint4*)xp);
-    return cudaGetLastError();
+    return launch_k(permute_gather_kernel, grid, dim3(256), 0, st, (const uint4*)x, idx, blockoff, indptr, T, nvec,
+                    E, k, capacity, pos, row_token, (uint4*)xp);
 }
 
 // Statistics for T == 0 (nothing routed).
 __global__ void zero_stats_kernel(void* stats, int E, int capacity) {
+    pdl_wait();
+    pdl_launch();
     moe_stats* st = (moe_stats*)stats;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         MOE_STATS_COUNTS(stats, E)[e] = 0;
@@ -313,8 +318,7 @@ __global__ void zero_stats_kernel(void* stats, int E, int capacity) {
 }
 
 cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st) {
-    zero_stats_kernel<<<1, 256, 0, st>>>(stats, E, capacity);
-    return cudaGetLastError();
+    return launch_k(zero_stats_kernel, dim3(1), dim3(256), 0, st, stats, E, capacity);
 }
 
 }  // namespace moe

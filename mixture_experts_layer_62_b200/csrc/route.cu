@@ -13,8 +13,13 @@ namespace moe {
 
 // ---- W_r [d, E] -> W_r^T [E, d] ------------------------------------------
 template <typename T>
-__global__ void transpose_kernel(const T* __restrict__ in, T* __restrict__ out, int d, int E) {
+__global__ void transpose_kernel(const T* __restrict__ in, T* __restrict__ out, int d, int E,
+                                 int32_t* __restrict__ status) {
     __shared__ T tile[32][33];
+    pdl_wait();
+    pdl_launch();
+    if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0)
+        *status = MOE_OK;
     int i0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
     for (int r = threadIdx.y; r < 32; r += blockDim.y) {
         int i = i0 + r, e = e0 + threadIdx.x;
@@ -27,14 +32,13 @@ __global__ void transpose_kernel(const T* __restrict__ in, T* __restrict__ out, 
     }
 }
 
-cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, int E, cudaStream_t st) {
+cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, int E, cudaStream_t st,
+                                int32_t* status) {
     dim3 grid(ceil_div(d, 32), ceil_div(E, 32)), block(32, 8);
     if (dtype == MOE_DTYPE_BF16)
-        transpose_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(
-            (const __nv_bfloat16*)W_r, (__nv_bfloat16*)wrt, d, E);
-    else
-        transpose_kernel<float><<<grid, block, 0, st>>>((const float*)W_r, (float*)wrt, d, E);
-    return cudaGetLastError();
+        return launch_k(transpose_kernel<__nv_bfloat16>, grid, block, 0, st, (const __nv_bfloat16*)W_r,
+                        (__nv_bfloat16*)wrt, d, E, status);
+    return launch_k(transpose_kernel<float>, grid, block, 0, st, (const float*)W_r, (float*)wrt, d, E, status);
 }
 
 // ---- logits on CUDA cores -------------------------------------------------
@@ -69,6 +73,8 @@ __global__ void __launch_bounds__(kLgWarps * 32)
 logits_kernel(const T* __restrict__ x, const T* __restrict__ wrt, float* __restrict__ logits, int Tn, int d,
               int E) {
     __shared__ float part[kLgWarps][kLgTok][kExpPerPass];
+    pdl_wait();
+    pdl_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * kLgTok;
     const int nt = min(kLgTok, Tn - t0);
@@ -132,11 +138,10 @@ cudaError_t launch_logits_simt(int dtype, const void* x, const void* wrt, float*
     if (T == 0) return cudaSuccess;
     const int grid = ceil_div(T, kLgTok);
     if (dtype == MOE_DTYPE_BF16)
-        logits_kernel<__nv_bfloat16><<<grid, kLgWarps * 32, 0, st>>>(
-            (const __nv_bfloat16*)x, (const __nv_bfloat16*)wrt, logits, T, d, E);
-    else
-        logits_kernel<float><<<grid, kLgWarps * 32, 0, st>>>((const float*)x, (const float*)wrt, logits, T, d, E);
-    return cudaGetLastError();
+        return launch_k(logits_kernel<__nv_bfloat16>, dim3(grid), dim3(kLgWarps * 32), 0, st,
+                        (const __nv_bfloat16*)x, (const __nv_bfloat16*)wrt, logits, T, d, E);
+    return launch_k(logits_kernel<float>, dim3(grid), dim3(kLgWarps * 32), 0, st, (const float*)x,
+                    (const float*)wrt, logits, T, d, E);
 }
 
 // ---- selection: softmax, key, top-k, gates, chunk statistics -------------
@@ -163,6 +168,8 @@ select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, 
               int32_t* __restrict__ blockcnt, float* __restrict__ blockpsum) {
     __shared__ int cnt[MOE_MAX_E];
     __shared__ float ps[kSelWarps][MOE_MAX_E];
+    pdl_wait();
+    pdl_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunk = blockIdx.x, NB = gridDim.x;
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -289,15 +296,20 @@ cudaError_t launch_select(const float* logits, const float* bias, int bias_mode,
     dim3 grid(NB), block(kSelWarps * 32);
     int epl = ceil_div(E, 32);
     if (epl <= 1)
-        select_kernel<1><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+        return launch_k(select_kernel<1>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
+                        blockpsum);
     else if (epl <= 2)
-        select_kernel<2><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+        return launch_k(select_kernel<2>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
+                        blockpsum);
     else if (epl <= 4)
-        select_kernel<4><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+        return launch_k(select_kernel<4>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
+                        blockpsum);
     else if (epl <= 8)
-        select_kernel<8><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+        return launch_k(select_kernel<8>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
+                        blockpsum);
     else
-        select_kernel<16><<<grid, block, 0, st>>>(logits, bias, bias_mode, T, E, k, idx, gate, blockcnt, blockpsum);
+        return launch_k(select_kernel<16>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
+                        blockpsum);
     return cudaGetLastError();
 }
 
@@ -305,6 +317,8 @@ cudaError_t launch_select(const float* logits, const float* bias, int bias_mode,
 __global__ void hist_kernel(const int32_t* __restrict__ idx, int Tn, int k, int E,
                             int32_t* __restrict__ blockcnt) {
     __shared__ int cnt[MOE_MAX_E];
+    pdl_wait();
+    pdl_launch();
     const int chunk = blockIdx.x, NB = gridDim.x;
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
@@ -321,8 +335,7 @@ __global__ void hist_kernel(const int32_t* __restrict__ idx, int Tn, int k, int 
 cudaError_t launch_hist(const int32_t* idx, int T, int k, int E, int32_t* blockcnt, cudaStream_t st) {
     int NB = ceil_div(T, kChunk);
     if (NB == 0) return cudaSuccess;
-    hist_kernel<<<NB, 256, 0, st>>>(idx, T, k, E, blockcnt);
-    return cudaGetLastError();
+    return launch_k(hist_kernel, dim3(NB), dim3(256), 0, st, idx, T, k, E, blockcnt);
 }
 
 }  // namespace moe
