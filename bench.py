@@ -278,7 +278,8 @@ def config_of(cfg, args):
             "k": cfg["k"], "capacity_factor": cfg["cf"], "bias_mode": cfg["bias_mode"],
             "d_ff_shared": cfg["d_ff_shared"], "global_batch_tokens": cfg["T"] * args.gpus,
             "parallelism": f"dp{args.gpus} replicas" if args.gpus > 1 else "single GPU",
-            "l2": "512 MiB buffer written between timed steps (weights 2.8 GB also exceed L2)"}
+            "l2": "512 MiB buffer written between timed steps (weights 2.8 GB also exceed L2)",
+            "launch": "eager" if getattr(args, "no_graph", False) else "cuda_graph (captured moe_forward, replayed)"}
 
 
 def launches_per_forward(cfg):
@@ -297,6 +298,7 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=1024, help="tokens of the timed CPU-oracle sample")
     ap.add_argument("--ref-sample", type=int, default=16, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the forward eagerly in the timed loop")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -337,8 +339,21 @@ def main():
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    # the forward is captured once in a CUDA graph and replayed (the library's
+    # launches are asynchronous and allocation-free, so they capture as is)
+    for _ in range(args.warmup):
         layer(x)
+    torch.cuda.synchronize(dev)
+    fwd = (lambda: layer(x))
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer(x)
+        torch.cuda.synchronize(dev)
+        fwd = graph.replay
+
+    def step():
+        fwd()
         if world > 1:
             # the one exchange of data-parallel replicas: global load statistics
             v = parallel._local_vector(layer.stats, E, cfg["T"])
@@ -450,6 +465,8 @@ def main():
         line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"routing of all {cfg['T']} tokens + expert math of {n} seeded random "
                                           f"tokens ({dt:.1f} s)"}
+    if not args.no_graph:
+        del graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -29,8 +29,9 @@ Layout make_layout(const moe_problem& p) {
     L.wrt = take(E * d * eb);
     L.blockcnt = take(E * NB * 4);
     L.blockoff = take(E * NB * 4);
-    // per-chunk probability sums; the small-batch router keeps [T][E] probabilities here
-    L.blockpsum = take((small_route_ok(p) ? T : NB) * E * 4);
+    // per-chunk probability sums; the small-batch router keeps its partial
+    // logits [T][parts][E] here
+    L.blockpsum = take((small_route_ok(p) ? T * kSmallMaxParts : NB) * E * 4);
     L.tiles13 = take((E + 3) * 4);
     L.tiles2 = take((E + 3) * 4);
     L.xp = take(T * k * d * eb);

@@ -42,8 +42,9 @@ template <> struct VecTraits<__nv_bfloat16> {
     }
 };
 
-// One warp per (token, slice of the row): a slice is 32 x kCbVecPerLane
-// 16-byte vectors, so small batches still spread over the whole GPU. With
+// One warp per (token, slice of the row): a slice is 32 x vpl 16-byte
+// vectors (vpl = 1 for small batches), so few tokens still spread over many
+// warps. With
 // split-K partials (opart != null and *split2 > 1) an expert output row is the
 // sum over the splits, s = 0, 1, ..., of the fp32 partial rows.
 constexpr int kCbVecPerLane = 2;
@@ -54,29 +55,35 @@ __global__ void __launch_bounds__(kCbWarps * 32, 4)
 combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const float* __restrict__ gate,
                const T* __restrict__ s, T* __restrict__ out, int Tn, int d, int k,
                const float* __restrict__ opart, long long opart_stride, const int32_t* __restrict__ split2,
-               int slices) {
+               int slices, int vpl) {
     using V = VecTraits<T>;
     constexpr int VN = V::N;
-    pdl_wait();
-    pdl_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long task = (long long)blockIdx.x * kCbWarps + warp;
     const int t = (int)(task / slices), sl = (int)(task % slices);
-    if (t >= Tn) return;
-    const int S = (opart != nullptr && split2 != nullptr) ? *split2 : 1;
+    // pos, gate and the split factor come from kernels at least two launches
+    // back (routing and scan run before both GEMMs), so they are read before
+    // the dependency wait; the expert outputs are read after it
     int p[MOE_MAX_K];
     float g[MOE_MAX_K];
+    int S = 1;
+    if (t < Tn) {
+        S = (opart != nullptr && split2 != nullptr) ? *split2 : 1;
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j) {
-        if (j < k) {
-            p[j] = pos[(size_t)t * k + j];
-            g[j] = gate[(size_t)t * k + j];
+        for (int j = 0; j < MOE_MAX_K; ++j) {
+            if (j < k) {
+                p[j] = pos[(size_t)t * k + j];
+                g[j] = gate[(size_t)t * k + j];
+            }
         }
     }
+    pdl_wait();
+    pdl_launch();
+    if (t >= Tn) return;
     const int nvec = d / VN;
-#pragma unroll
-    for (int i = 0; i < kCbVecPerLane; ++i) {
-        const int v = (sl * kCbVecPerLane + i) * 32 + lane;
+#pragma unroll 2
+    for (int i = 0; i < vpl; ++i) {
+        const int v = (sl * vpl + i) * 32 + lane;
         if (v >= nvec) break;
         float acc[VN];
 #pragma unroll
@@ -118,16 +125,19 @@ cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const f
                            const float* opart, long long opart_stride, const int32_t* split2) {
     if (T == 0) return cudaSuccess;
     const int vn = dtype == MOE_DTYPE_BF16 ? 8 : 4;
-    const int slices = ceil_div(d / vn, 32 * kCbVecPerLane);
+    // small batches: one vector per lane per warp, so the few rows (and their
+    // split-K partials) are spread over more warps
+    const int vpl = T < 256 ? 1 : kCbVecPerLane;
+    const int slices = ceil_div(d / vn, 32 * vpl);
     const long long tasks = (long long)T * slices;
     const unsigned grid = (unsigned)((tasks + kCbWarps - 1) / kCbWarps);
     if (dtype == MOE_DTYPE_BF16)
         return launch_k(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(kCbWarps * 32), 0, st,
                         (const __nv_bfloat16*)o, pos, gate, (const __nv_bfloat16*)s, (__nv_bfloat16*)out, T, d, k,
-                        opart, opart_stride, split2, slices);
+                        opart, opart_stride, split2, slices, vpl);
     return launch_k(combine_kernel<float>, dim3(grid), dim3(kCbWarps * 32), 0, st, (const float*)o, pos, gate,
                     (const float*)s, (float*)out, T, d, k, (const float*)nullptr, 0LL, (const int32_t*)nullptr,
-                    slices);
+                    slices, vpl);
 }
 
 // Split-K reduction of grouped GEMM 1/3: the partial rows hold, per 128

@@ -125,10 +125,11 @@ cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st)
 // launches (one block per token, then one finishing kernel).
 constexpr int kSmallMaxPairs = 64;
 constexpr int kSmallMaxE = 64;
+constexpr int kSmallMaxParts = 16;   // partial-logit blocks per token
 struct SmallRouteArgs {
     const void* x; const void* W_r; const float* bias;
     int bias_mode, T, d, E, k, capacity;
-    float* logits; float* probs; int32_t* idx; float* gate; int32_t* pos; int32_t* indptr; int32_t* row_token;
+    float* logits; float* probs /* partial logits [T][parts][E] */; int32_t* idx; float* gate; int32_t* pos; int32_t* indptr; int32_t* row_token;
     int32_t* status_reset;
     void* xp; void* stats;
     int32_t* tiles13; int32_t* tiles2;

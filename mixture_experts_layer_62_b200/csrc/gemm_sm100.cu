@@ -484,7 +484,44 @@ bool get_encode() {
 
 // 2-D bf16 map over a [rows, cols] row-major matrix, box 64 columns x 128 rows,
 // 128-byte swizzle; reads outside the matrix return zeros.
+bool encode_map(CUtensorMap* m, const void* base, int rows, int cols);
+
+// Encoded maps keyed by (base, rows, cols): the same key always encodes to the
+// same map, so a hit is exactly a fresh encode, without the driver call.
+struct MapCacheEntry {
+    const void* base;
+    int rows, cols;
+    CUtensorMap map;
+};
+constexpr int kMapCacheSize = 64;
+MapCacheEntry g_map_cache[kMapCacheSize];
+int g_map_cache_n = 0, g_map_cache_next = 0;
+std::mutex g_map_cache_mu;
+
 bool make_map(CUtensorMap* m, const void* base, int rows, int cols) {
+    {
+        std::lock_guard<std::mutex> lk(g_map_cache_mu);
+        for (int i = 0; i < g_map_cache_n; ++i) {
+            const MapCacheEntry& c = g_map_cache[i];
+            if (c.base == base && c.rows == rows && c.cols == cols) {
+                *m = c.map;
+                return true;
+            }
+        }
+    }
+    if (!encode_map(m, base, rows, cols)) return false;
+    std::lock_guard<std::mutex> lk(g_map_cache_mu);
+    MapCacheEntry& c = g_map_cache[g_map_cache_next];
+    c.base = base;
+    c.rows = rows;
+    c.cols = cols;
+    c.map = *m;
+    g_map_cache_next = (g_map_cache_next + 1) % kMapCacheSize;
+    if (g_map_cache_n < kMapCacheSize) ++g_map_cache_n;
+    return true;
+}
+
+bool encode_map(CUtensorMap* m, const void* base, int rows, int cols) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
     cuuint32_t box[2] = {BK, 128};

@@ -1,7 +1,7 @@
 // Small-batch router: the whole routing and permutation of a decode-sized
-// batch (T*k <= 64 pairs) in two short launches instead of five: one block
-// per token for logits and selection, then one kernel for the statistics,
-// destinations, tile schedules and the row gather.
+// batch (T*k <= 64 pairs) in two short launches instead of five: partial
+// logits by (token, part of the row) blocks, then one kernel for the
+// selection, statistics, destinations, tile schedules and the row gather.
 //
 // It computes the same quantities, with the same definitions, as the general
 // path (route.cu, permute.cu): z = W_r^T x in fp32 ("Week 2 Day 2: Mixture of
@@ -40,26 +40,27 @@ __device__ __forceinline__ void bf16x8(const uint4& u, float (&v)[8]) {
     }
 }
 
-// ---- kernel 1: one block per token -----------------------------------------
-// Logits z_t (8 warps split the row; lane partials by xor butterfly, warp
-// partials in warp order), then warp 0 forms the softmax, the key, the top-k
-// and the gates, and writes idx, gate, logits and the softmax probabilities.
-constexpr int kTokWarps = 8;
+// ---- kernel 1: partial logits, one block per (token, part of the row) ---------
+// Block (t, part) sums x_t . W_r[:, e] over its slice of the row: 4 warps, lane
+// l takes chunks l, l + 32, ... of its warp's sub-slice, xor butterfly over
+// lanes, warp order over warps. Output: partial[(t * P + part) * E + e].
+constexpr int kPartWarps = 4;
 
-__global__ void __launch_bounds__(kTokWarps * 32) route_token_kernel(SmallRouteArgs a) {
-    __shared__ float part[kTokWarps][kSmallMaxE];
-    __shared__ float zs[kSmallMaxE];
+__global__ void __launch_bounds__(kPartWarps * 32) route_logits_kernel(SmallRouteArgs a, int P) {
+    __shared__ float wsum[kPartWarps][kSmallMaxE];
     pdl_wait();
     pdl_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x;
-    if (a.status_reset != nullptr && t == 0 && threadIdx.x == 0) *a.status_reset = MOE_OK;
-    const int d = a.d, E = a.E, k = a.k;
+    const int t = blockIdx.x, part = blockIdx.y;
+    if (a.status_reset != nullptr && t == 0 && part == 0 && threadIdx.x == 0) *a.status_reset = MOE_OK;
+    const int d = a.d, E = a.E;
     const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(a.x) + (size_t)t * d;
     const __nv_bfloat16* W_r = static_cast<const __nv_bfloat16*>(a.W_r);
     const int nchunk = d / 8;
-    const int per = (nchunk + kTokWarps - 1) / kTokWarps;
-    const int c_lo = warp * per, c_hi = min(nchunk, c_lo + per);
+    const int per_part = (nchunk + P - 1) / P;
+    const int p_lo = part * per_part, p_hi = min(nchunk, p_lo + per_part);
+    const int per_warp = (p_hi - p_lo + kPartWarps - 1) / kPartWarps;
+    const int c_lo = p_lo + warp * per_warp, c_hi = min(p_hi, c_lo + per_warp);
     for (int e0 = 0; e0 < E; e0 += 8) {
         float acc[8];
 #pragma unroll
@@ -78,104 +79,143 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_token_kernel(SmallRouteA
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const float v = warp_sum(acc[e]);
-            if (lane == 0) part[warp][e0 + e] = v;
+            if (lane == 0) wsum[warp][e0 + e] = v;
         }
     }
     __syncthreads();
     if (threadIdx.x < E) {
         float v = 0.f;
-        for (int w = 0; w < kTokWarps; ++w) v += part[w][threadIdx.x];
-        zs[threadIdx.x] = v;
-        a.logits[(size_t)t * E + threadIdx.x] = v;
-    }
-    __syncthreads();
-    if (warp != 0) return;
-    float zz[2], key[2], ex[2];
-    unsigned valid = 0;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int e = lane + 32 * i;
-        zz[i] = e < E ? zs[e] : -INFINITY;
-        if (e < E) valid |= 1u << i;
-    }
-    const float m = warp_max(fmaxf(zz[0], zz[1]));
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        ex[i] = ((valid >> i) & 1u) ? expf(zz[i] - m) : 0.f;
-        s += ex[i];
-    }
-    s = warp_sum(s);
-    const float inv_s = 1.f / s;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int e = lane + 32 * i;
-        const float p = ex[i] * inv_s;
-        const float b = (a.bias_mode != MOE_BIAS_NONE && e < E) ? a.bias[e] : 0.f;
-        if (e < E) a.probs[(size_t)t * E + e] = p;
-        key[i] = a.bias_mode == MOE_BIAS_NONE ? zz[i] : a.bias_mode == MOE_BIAS_LOGIT ? zz[i] + b : p + b;
-    }
-    unsigned taken = 0;
-    float zsel[MOE_MAX_K];
-    int esel[MOE_MAX_K];
-#pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j) {
-        if (j < k) {
-            float bk = -INFINITY, bz = 0.f;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
-                if (ok && (key[i] > bk || be == 0x7fffffff)) { bk = key[i]; be = lane + 32 * i; bz = zz[i]; }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-                const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
-                if (better) { bk = ok_; be = oe; bz = oz; }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            zsel[j] = bz;
-            esel[j] = be;
-        }
-    }
-    float zm = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) zm = fmaxf(zm, zsel[j]);
-    float gs = 0.f, ge[MOE_MAX_K];
-#pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
-    const float inv_g = 1.f / gs;
-#pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j) {
-        if (j < k && lane == j) {
-            a.idx[(size_t)t * k + j] = esel[j];
-            a.gate[(size_t)t * k + j] = ge[j] * inv_g;
-        }
+        for (int w = 0; w < kPartWarps; ++w) v += wsum[w][threadIdx.x];
+        a.probs[((size_t)t * P + part) * E + threadIdx.x] = v;   // partial logits
     }
 }
 
-// ---- kernel 2: statistics, destinations, schedules and the gather ------------
-// Every block derives the destinations of all (<= 64) pairs from idx (rank =
-// earlier pairs of the same expert, token order) and gathers its slice of the
-// row vectors; block 0 also writes pos, row_token, indptr, the statistics and
-// the tile schedules with their split factors.
-constexpr int kFinThreads = 256;
+// ---- kernel 2: logits, selection, statistics, destinations, gather -----------
+// Every block sums the partial logits (part order), selects (one warp per
+// token: softmax, key, top-k with the lowest index winning ties, gates over
+// the selected raw logits), counts, scans and places the <= 64 pairs (rank =
+// earlier pairs of the same expert, token order), then gathers its slice of
+// the row vectors. Block 0 alone writes logits, idx, gate, pos, row_token,
+// indptr, the statistics and the tile schedules with their split factors.
+constexpr int kFinWarps = 16;
 
-__global__ void __launch_bounds__(kFinThreads) route_finish_kernel(SmallRouteArgs a) {
+__global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRouteArgs a, int P) {
+    __shared__ float z[kSmallMaxPairs][kSmallMaxE];
+    __shared__ float psw[kFinWarps][kSmallMaxE];
     __shared__ int sidx[kSmallMaxPairs];
     __shared__ int spos[kSmallMaxPairs];
-    __shared__ int cnt[kSmallMaxE];
     __shared__ int indptr_s[kSmallMaxE + 1];
-    pdl_wait();
-    pdl_launch();
+    __shared__ float bias_s[kSmallMaxE];
     const int T = a.T, E = a.E, k = a.k;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool writer = blockIdx.x == 0;
-    for (int i = threadIdx.x; i < T * k; i += blockDim.x) sidx[i] = a.idx[i];
+    // Before the dependency wait: only inputs of the pass (bias, x), never an
+    // output of the preceding kernel. The x vectors this block gathers are
+    // loaded now and held in registers.
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        bias_s[e] = a.bias_mode != MOE_BIAS_NONE ? a.bias[e] : 0.f;
+    for (int i = threadIdx.x; i < kFinWarps * kSmallMaxE; i += blockDim.x) (&psw[0][0])[i] = 0.f;
+    const int nvec = a.d / 8;
+    const int vper = (nvec + gridDim.x - 1) / gridDim.x;
+    const int v_lo = blockIdx.x * vper, v_hi = min(nvec, v_lo + vper);
+    const int span = max(0, v_hi - v_lo);
+    const uint4* xv = static_cast<const uint4*>(a.x);
+    constexpr int kHeld = 4;
+    uint4 held[kHeld];
+#pragma unroll
+    for (int h = 0; h < kHeld; ++h) {
+        const int i = threadIdx.x + h * (int)blockDim.x;
+        if (i < T * span) held[h] = xv[(size_t)(i / span) * nvec + v_lo + i % span];
+    }
+    pdl_wait();
+    pdl_launch();
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
+        const int t = i / E, e = i % E;
+        float pv[kSmallMaxParts];
+#pragma unroll
+        for (int part = 0; part < kSmallMaxParts; ++part)
+            pv[part] = part < P ? a.probs[((size_t)t * P + part) * E + e] : 0.f;
+        float v = 0.f;
+#pragma unroll
+        for (int part = 0; part < kSmallMaxParts; ++part)
+            if (part < P) v += pv[part];
+        z[t][e] = v;
+        if (writer) a.logits[i] = v;
+    }
     __syncthreads();
+
+    for (int t = warp; t < T; t += kFinWarps) {
+        float zz[2], key[2], ex[2];
+        unsigned valid = 0;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int e = lane + 32 * i;
+            zz[i] = e < E ? z[t][e] : -INFINITY;
+            if (e < E) valid |= 1u << i;
+        }
+        const float m = warp_max(fmaxf(zz[0], zz[1]));
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            ex[i] = ((valid >> i) & 1u) ? expf(zz[i] - m) : 0.f;
+            s += ex[i];
+        }
+        s = warp_sum(s);
+        const float inv_s = 1.f / s;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int e = lane + 32 * i;
+            const float p = ex[i] * inv_s;
+            const float b = e < E ? bias_s[e] : 0.f;
+            if (e < E) psw[warp][e] += p;
+            key[i] = a.bias_mode == MOE_BIAS_NONE ? zz[i] : a.bias_mode == MOE_BIAS_LOGIT ? zz[i] + b : p + b;
+        }
+        unsigned taken = 0;
+        float zsel[MOE_MAX_K];
+        int esel[MOE_MAX_K];
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) {
+            if (j < k) {
+                float bk = -INFINITY, bz = 0.f;
+                int be = 0x7fffffff;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
+                    if (ok && (key[i] > bk || be == 0x7fffffff)) { bk = key[i]; be = lane + 32 * i; bz = zz[i]; }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                    const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+                    const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
+                    if (better) { bk = ok_; be = oe; bz = oz; }
+                }
+                if ((be & 31) == lane) taken |= 1u << (be >> 5);
+                zsel[j] = bz;
+                esel[j] = be;
+            }
+        }
+        float zm = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) zm = fmaxf(zm, zsel[j]);
+        float gs = 0.f, ge[MOE_MAX_K];
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
+        const float inv_g = 1.f / gs;
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) {
+            if (j < k && lane == j) {
+                sidx[t * k + j] = esel[j];
+                if (writer) {
+                    a.idx[(size_t)t * k + j] = esel[j];
+                    a.gate[(size_t)t * k + j] = ge[j] * inv_g;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
     if (warp == 0) {
         // counts, capacity, kept, indptr (experts lane, lane + 32)
         int c[2], kp[2];
@@ -187,7 +227,6 @@ __global__ void __launch_bounds__(kFinThreads) route_finish_kernel(SmallRouteArg
                 for (int q = 0; q < T * k; ++q) n_ += (sidx[q] == e);
             c[i] = n_;
             kp[i] = a.capacity < 0 ? n_ : min(n_, a.capacity);
-            if (e < E) cnt[e] = n_;
         }
         int run = 0;
 #pragma unroll
@@ -213,7 +252,7 @@ __global__ void __launch_bounds__(kFinThreads) route_finish_kernel(SmallRouteArg
                 t2[i] = (kp[i] > 0 ? 1 : 0) * a.nt2;
                 if (e < E) {
                     float acc = 0.f;
-                    for (int t = 0; t < T; ++t) acc += a.probs[(size_t)t * E + e];   // token order
+                    for (int w = 0; w < kFinWarps; ++w) acc += psw[w][e];   // fixed order over warps
                     const float Pe = acc / (float)T;
                     const float fe = (float)c[i] / ((float)T * (float)k);
                     MOE_STATS_P(a.stats, E)[e] = Pe;
@@ -280,17 +319,20 @@ __global__ void __launch_bounds__(kFinThreads) route_finish_kernel(SmallRouteArg
         }
     }
     __syncthreads();
-    // gather this block's slice of every token row
-    const int nvec = a.d / 8;
-    const int vper = (nvec + gridDim.x - 1) / gridDim.x;
-    const int v_lo = blockIdx.x * vper, v_hi = min(nvec, v_lo + vper);
-    const int span = v_hi - v_lo;
+    // gather this block's slice of every token row (the first kHeld vectors
+    // of each thread were loaded before the wait)
     if (span <= 0) return;
-    const uint4* xv = static_cast<const uint4*>(a.x);
     uint4* xp = static_cast<uint4*>(a.xp);
-    for (int i = threadIdx.x; i < T * span; i += blockDim.x) {
+    for (int i = threadIdx.x, h = 0; i < T * span; i += blockDim.x, ++h) {
         const int t = i / span, v = v_lo + i % span;
-        const uint4 val = xv[(size_t)t * nvec + v];
+        uint4 val;
+        if (h < kHeld) {
+#pragma unroll
+            for (int hh = 0; hh < kHeld; ++hh)
+                if (hh == h) val = held[hh];
+        } else {
+            val = xv[(size_t)t * nvec + v];
+        }
         for (int j = 0; j < k; ++j) {
             const int p = spos[t * k + j];
             if (p >= 0) xp[(size_t)p * nvec + v] = val;
@@ -306,13 +348,15 @@ bool small_route_ok(const moe_problem& p) {
 }
 
 cudaError_t launch_route_small(const SmallRouteArgs& a, cudaStream_t st) {
-    cudaError_t e = launch_k(route_token_kernel, dim3(a.T), dim3(kTokWarps * 32), 0, st, a);
+    const int nchunk = a.d / 8;
+    int P = (nchunk + 127) / 128;   // ~128 chunks (1 per lane of 4 warps) per block
+    P = P < 1 ? 1 : (P > kSmallMaxParts ? kSmallMaxParts : P);
+    cudaError_t e = launch_k(route_logits_kernel, dim3(a.T, P), dim3(kPartWarps * 32), 0, st, a, P);
     if (e != cudaSuccess) return e;
     g_pdl_after_first();
-    const int nvec = a.d / 8;
-    int blocks = (nvec + 63) / 64;              // >= 64 vectors per block
+    int blocks = (nchunk + 63) / 64;   // >= 64 vectors of the gather per block
     blocks = blocks < 1 ? 1 : (blocks > 32 ? 32 : blocks);
-    return launch_k(route_finish_kernel, dim3(blocks), dim3(kFinThreads), 0, st, a);
+    return launch_k(route_finish_kernel, dim3(blocks), dim3(kFinWarps * 32), 0, st, a, P);
 }
 
 }  // namespace moe

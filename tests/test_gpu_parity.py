@@ -400,6 +400,31 @@ def test_stages_compose_to_forward():
     assert torch.equal(out, out2)
 
 
+@pytest.mark.parametrize("cfg", [
+    dict(T=4, d=512, d_ff=512, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    dict(T=600, d=256, d_ff=384, E=16, k=4, cf=0.8, dtype="bf16", bias_mode=1, d_ff_shared=128),
+], ids=["decode_split_pdl", "general_pdl"])
+def test_forward_captures_in_a_cuda_graph(cfg):
+    # moe_forward is asynchronous and allocation-free: captured once and
+    # replayed, it gives the eager call's bits
+    L = to_device(_small_layer(cfg, 21))
+    p, out, st, ws = gpu_forward(cfg, L)
+    out_g = torch.empty_like(out)
+    st_g = moe.alloc_stats(cfg["E"], DEV)
+    ws_g = moe.alloc_workspace(p, DEV)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.forward(p, L["x"], L["W_r"], L["W1"], L["W3"], L["W2"], out_g, st_g, ws_g, bias=L["bias"],
+                    Ws1=L["Ws1"], Ws3=L["Ws3"], Ws2=L["Ws2"])
+    for _ in range(2):
+        out_g.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, out_g)
+    assert torch.equal(st, st_g)
+    del g
+
+
 # --------------------------------------------------------------------------
 # full-size workloads: routing on all tokens, outputs on sampled tokens
 # --------------------------------------------------------------------------
