@@ -55,6 +55,16 @@ BIAS_NONE = 0   # key = z
 BIAS_LOGIT = 1  # key = z + b      ([MoE tutorial] route(): bias on raw scores)
 BIAS_PROB = 2   # key = softmax(z) + b   ([CS336 L04] §2.3.3c: bias on s_{i,t})
 
+# Gate modes.
+GATE_SELECTED = 0  # softmax over the k selected raw logits ([CME295 W2D2] §1.3)
+GATE_FULL = 1      # full-softmax probability of each selected expert, not
+                   # renormalised (Switch top-1, [CMU 15-779 L21] §2.5)
+
+# Drop orders under capacity.
+DROP_TOKEN = 0     # rank inside an expert in token order ([CMU 15-779 L21] §3.3)
+DROP_SLOT = 1      # GShard Algorithm 1: every token's first choice before any
+                   # second choice ([CMU 15-779 L21] §3.5)
+
 
 # --------------------------------------------------------------------------
 # Router
@@ -133,6 +143,14 @@ def gates_from_selected(z, idx):
     return e / e.sum(axis=1, keepdims=True)
 
 
+def gates_full_softmax(z, idx):
+    """g_i = softmax(z)_i for each selected i, not renormalised over the
+    selected set: the Switch Transformer's top-1 gate y = p_i(x) E_i(x)
+    ([CMU 15-779 L21] §2.5; [CME295 W2D2] §1.3: Switch with k = 1 takes the
+    full softmax probability; [CS336 L04] §2.1.2, g_{i,t} = s_{i,t})."""
+    return np.take_along_axis(softmax_rows(z), idx, axis=1)
+
+
 @dataclass
 class Routing:
     idx: np.ndarray        # [T, k] int64, descending key order
@@ -141,7 +159,7 @@ class Routing:
     key: np.ndarray        # [T, E] the ranked key
 
 
-def route(z, k, bias=None, bias_mode=BIAS_NONE, key_dtype=np.float64):
+def route(z, k, bias=None, bias_mode=BIAS_NONE, key_dtype=np.float64, gate_mode=GATE_SELECTED):
     """Routing from logits: selection key, top-k, gates and full softmax.
 
     [CME295 W2D2] §1.3 and §4.2; [MoE tutorial] route().
@@ -149,7 +167,7 @@ def route(z, k, bias=None, bias_mode=BIAS_NONE, key_dtype=np.float64):
     z = np.asarray(z)
     key = selection_key(z, bias, bias_mode, dtype=key_dtype)
     idx = topk_lowest_index(key, k)
-    gate = gates_from_selected(z, idx)
+    gate = gates_from_selected(z, idx) if gate_mode == GATE_SELECTED else gates_full_softmax(z, idx)
     probs = softmax_rows(z)
     return Routing(idx=idx, gate=gate, probs=probs, key=key)
 
@@ -181,7 +199,7 @@ class Permutation:
     rank: np.ndarray       # [T, k] int64 rank of the pair inside its expert
 
 
-def permute(idx, E, C=None):
+def permute(idx, E, C=None, drop_order=DROP_TOKEN):
     """Permutation indices by prefix sum, with capacity truncation.
 
     [CMU 15-779 L21] §3.3: build the N x E 0/1 selection mask, flatten it
@@ -194,18 +212,41 @@ def permute(idx, E, C=None):
     Capacity ([CMU 15-779 L21] §3.5, [W11 routing] §3): a pair whose rank is
     >= C is dropped. The kept pairs are renumbered with the same expert-major
     order, so their rows are indptr_kept[e] + rank.
+
+    drop_order = DROP_SLOT (GShard's Algorithm 1, [CMU 15-779 L21] §3.5:
+    all first choices before the second choices, the rank again a prefix
+    sum): the mask gets a slot axis, [k, N, E] with mask[j, t, e] = 1 iff
+    idx[t, j] = e, and is flattened expert-major as (e, j, t), so inside an
+    expert the pairs are ordered by slot, then token.
     """
     idx = np.asarray(idx, dtype=np.int64)
     T, k = idx.shape
-    mask = np.zeros((T, E), dtype=np.int64)
-    for t in range(T):
-        for j in range(k):
-            mask[t, idx[t, j]] = 1
-    flat = mask.T.reshape(-1)                    # expert-major
-    cs = np.cumsum(flat).reshape(E, T).T         # [T, E] inclusive prefix sums
-    indptr_full = np.zeros(E + 1, dtype=np.int64)
-    indptr_full[1:] = cs[T - 1, :] if T > 0 else 0
-    counts = indptr_full[1:] - indptr_full[:-1]
+    if drop_order == DROP_SLOT:
+        mask3 = np.zeros((k, T, E), dtype=np.int64)
+        for t in range(T):
+            for j in range(k):
+                mask3[j, t, idx[t, j]] = 1
+        flat = mask3.transpose(2, 0, 1).reshape(-1)            # (e, j, t)
+        cs3 = np.cumsum(flat).reshape(E, k, T)                  # inclusive
+        indptr_full = np.zeros(E + 1, dtype=np.int64)
+        indptr_full[1:] = cs3[:, k - 1, T - 1] if T > 0 else 0
+        counts = indptr_full[1:] - indptr_full[:-1]
+
+        def rank_of(t, j, e):
+            return cs3[e, j, t] - 1 - indptr_full[e]
+    else:
+        mask = np.zeros((T, E), dtype=np.int64)
+        for t in range(T):
+            for j in range(k):
+                mask[t, idx[t, j]] = 1
+        flat = mask.T.reshape(-1)                    # expert-major
+        cs = np.cumsum(flat).reshape(E, T).T         # [T, E] inclusive prefix sums
+        indptr_full = np.zeros(E + 1, dtype=np.int64)
+        indptr_full[1:] = cs[T - 1, :] if T > 0 else 0
+        counts = indptr_full[1:] - indptr_full[:-1]
+
+        def rank_of(t, j, e):
+            return cs[t, e] - 1 - indptr_full[e]
 
     kept = counts.copy() if C is None else np.minimum(counts, C)
     indptr = np.zeros(E + 1, dtype=np.int64)
@@ -216,7 +257,7 @@ def permute(idx, E, C=None):
     for t in range(T):
         for j in range(k):
             e = idx[t, j]
-            r = cs[t, e] - 1 - indptr_full[e]
+            r = rank_of(t, j, e)
             rank[t, j] = r
             if C is None or r < C:
                 pos[t, j] = indptr[e] + r
@@ -271,6 +312,37 @@ def l_aux(f, P, alpha=1.0):
     return float(alpha * E * np.sum(f * P))
 
 
+def router_z_loss(z):
+    """L_z = (1/T) sum_t (log sum_i exp z_{t,i})^2 ([CME295 W2D2] §3.4;
+    [CS336 L04] §3.1: it penalises the overall size of the router logits)."""
+    z = np.asarray(z, dtype=np.float64)
+    m = z.max(axis=1, keepdims=True)
+    lse = m[:, 0] + np.log(np.exp(z - m).sum(axis=1))
+    return float(np.mean(lse ** 2)) if z.shape[0] else 0.0
+
+
+def router_entropy(probs):
+    """Mean over tokens of the router distribution's entropy, -sum_i p log p
+    ([W11 routing] §5, "router entropy"); 0 log 0 = 0."""
+    p = np.asarray(probs, dtype=np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        h = -np.where(p > 0, p * np.log(p), 0.0).sum(axis=1)
+    return float(h.mean()) if p.shape[0] else 0.0
+
+
+def router_top_gap(probs):
+    """Mean over tokens of the gap between the largest and second-largest
+    router probability ([W11 routing] §5, "top-1/top-2 gap"); with one expert
+    the second is taken as 0."""
+    p = np.asarray(probs, dtype=np.float64)
+    if p.shape[0] == 0:
+        return 0.0
+    if p.shape[1] == 1:
+        return float(p[:, 0].mean())
+    srt = -np.sort(-p, axis=1)
+    return float(np.mean(srt[:, 0] - srt[:, 1]))
+
+
 @dataclass
 class LoadStats:
     counts: np.ndarray     # [E] pairs routed before capacity
@@ -282,9 +354,12 @@ class LoadStats:
     max_count: int
     max_over_mean: float   # max_e c_e / (T k / E)
     capacity: Optional[int]
+    z_loss: float = 0.0    # router z-loss
+    entropy: float = 0.0   # mean router entropy
+    top_gap: float = 0.0   # mean top-1 minus top-2 probability
 
 
-def load_stats(perm: Permutation, probs, T, k, C):
+def load_stats(perm: Permutation, probs, T, k, C, z=None):
     """Per-expert load statistics of one batch.
 
     f and P per [CME295 W2D2] §3.2 (f counts all k choices, P is the mean
@@ -300,7 +375,10 @@ def load_stats(perm: Permutation, probs, T, k, C):
                      l_aux=l_aux(f, P), dropped=int(np.sum(counts - perm.kept)),
                      max_count=int(counts.max()) if E else 0,
                      max_over_mean=float(counts.max() / mean_load) if T > 0 else 0.0,
-                     capacity=C)
+                     capacity=C,
+                     z_loss=router_z_loss(z) if z is not None else 0.0,
+                     entropy=router_entropy(probs) if T > 0 else 0.0,
+                     top_gap=router_top_gap(probs) if T > 0 else 0.0)
 
 
 # --------------------------------------------------------------------------
@@ -319,7 +397,8 @@ class ForwardResult:
 
 def moe_forward(x, W_r, W1, W3, W2, k, capacity_factor=0.0, bias=None,
                 bias_mode=BIAS_NONE, Ws1=None, Ws3=None, Ws2=None,
-                logits=None, tokens=None, key_dtype=np.float64):
+                logits=None, tokens=None, key_dtype=np.float64,
+                gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN):
     """Forward pass of one MoE layer, the sparse per-pair definition.
 
     Steps in the order of [CMU 15-779 L21] §3.2 (route, permute, compute per
@@ -348,13 +427,13 @@ def moe_forward(x, W_r, W1, W3, W2, k, capacity_factor=0.0, bias=None,
         z_key = z
     key = selection_key(z_key, bias, bias_mode, dtype=key_dtype)
     idx = topk_lowest_index(key, k)
-    gate = gates_from_selected(z, idx)
+    gate = gates_from_selected(z, idx) if gate_mode == GATE_SELECTED else gates_full_softmax(z, idx)
     probs = softmax_rows(z)
     routing = Routing(idx=idx, gate=gate, probs=probs, key=key)
 
     C = capacity(capacity_factor, T, k, E)
-    perm = permute(idx, E, C)
-    stats = load_stats(perm, probs, T, k, C)
+    perm = permute(idx, E, C, drop_order)
+    stats = load_stats(perm, probs, T, k, C, z=z)
 
     if tokens is None:
         tokens = np.arange(T)

@@ -10,10 +10,12 @@ and dropped pairs (formulation 0, "every expert computes", of [CMU 15-779 L21]
 * gates as the full softmax renormalised over the selected pair set
   ([CMU 15-779 L21] §2.1, s_i = g_{e_i} / sum_j g_{e_j}) instead of a softmax
   over the selected logits;
-* capacity by a running per-expert counter over tokens in order instead of a
-  prefix sum;
-* destination rows by sorting the kept pairs on (expert, token);
-* experts by explicit per-token loops over the hidden units.
+* capacity by a running per-expert counter over the pairs in visiting order
+  (token by token, or, for GShard's slot priority, all first choices before
+  any second choice) instead of a prefix sum;
+* destination rows by sorting the kept pairs on (expert, visiting order);
+* experts by explicit per-token loops over the hidden units;
+* z-loss, entropy and top-1/top-2 gap by explicit per-token loops.
 """
 
 from __future__ import annotations
@@ -31,7 +33,7 @@ def _softmax(v):
 
 
 def brute_forward(x, W_r, W1, W3, W2, k, cf=0.0, bias=None, bias_mode=0,
-                  Ws1=None, Ws3=None, Ws2=None):
+                  Ws1=None, Ws3=None, Ws2=None, gate_mode=0, drop_order=0):
     x = np.asarray(x, dtype=np.float64)
     W_r = np.asarray(W_r, dtype=np.float64)
     T, d = x.shape
@@ -52,11 +54,12 @@ def brute_forward(x, W_r, W1, W3, W2, k, cf=0.0, bias=None, bias_mode=0,
             idx[t, j] = e
             key[e] = -np.inf
 
-    # gates: full softmax renormalised over the selected set
+    # gates: full softmax renormalised over the selected set (gate_mode 0),
+    # or the full-softmax probability itself (gate_mode 1)
     gate = np.zeros((T, k))
     for t in range(T):
         p = _softmax(list(z[t]))
-        den = sum(p[idx[t, j]] for j in range(k))
+        den = sum(p[idx[t, j]] for j in range(k)) if gate_mode == 0 else 1.0
         for j in range(k):
             gate[t, j] = p[idx[t, j]] / den
 
@@ -68,16 +71,21 @@ def brute_forward(x, W_r, W1, W3, W2, k, cf=0.0, bias=None, bias_mode=0,
     used = [0] * E
     keep = np.zeros((T, k), dtype=bool)
     counts = np.zeros(E, dtype=np.int64)
-    for t in range(T):
-        for j in range(k):
-            e = idx[t, j]
-            counts[e] += 1
-            if C is None or used[e] < C:
-                keep[t, j] = True
-                used[e] += 1
+    # visiting order: token by token (drop_order 0), or all first choices,
+    # then all second choices, ... (drop_order 1)
+    order = ([(t, j) for t in range(T) for j in range(k)] if drop_order == 0
+             else [(t, j) for j in range(k) for t in range(T)])
+    for t, j in order:
+        e = idx[t, j]
+        counts[e] += 1
+        if C is None or used[e] < C:
+            keep[t, j] = True
+            used[e] += 1
 
-    # destination rows: kept pairs sorted by (expert, token)
-    pairs = sorted((idx[t, j], t, j) for t in range(T) for j in range(k) if keep[t, j])
+    # destination rows: kept pairs sorted by expert, then in visiting order
+    rank_in_order = {tj: r for r, tj in enumerate(order)}
+    pairs = sorted((idx[t, j], rank_in_order[(t, j)], t, j) for t in range(T) for j in range(k) if keep[t, j])
+    pairs = [(e, t, j) for e, _, t, j in pairs]
     pos = np.full((T, k), -1, dtype=np.int64)
     for r, (_, t, j) in enumerate(pairs):
         pos[t, j] = r
@@ -113,6 +121,14 @@ def brute_forward(x, W_r, W1, W3, W2, k, cf=0.0, bias=None, bias_mode=0,
     p_all = np.array([_softmax(list(z[t])) for t in range(T)])
     f = counts / (T * k)
     P = p_all.mean(axis=0)
+    # router statistics by explicit loops
+    zl = ent = gap = 0.0
+    for t in range(T):
+        lse = math.log(sum(math.exp(v) for v in z[t]))
+        zl += lse * lse
+        ent += -sum(pv * math.log(pv) for pv in p_all[t] if pv > 0)
+        srt = sorted(p_all[t], reverse=True)
+        gap += srt[0] - (srt[1] if E > 1 else 0.0)
     return dict(z=z, idx=idx, gate=gate, pos=pos, keep=keep, counts=counts,
                 kept=np.array(used), y=y, f=f, P=P, l_aux=E * float(np.sum(f * P)),
-                capacity=C)
+                capacity=C, z_loss=zl / T, entropy=ent / T, top_gap=gap / T)

@@ -256,6 +256,9 @@ def test_k_equal_E_is_dense_mixture():
     dict(T=33, d=8, E=16, d_ff=16, k=4, cf=1.0, mode=2, shared=True),
     dict(T=50, d=8, E=8, d_ff=8, k=2, cf=1.25, mode=1, shared=False),
     dict(T=17, d=8, E=4, d_ff=8, k=1, cf=0.5, mode=1, shared=True),
+    dict(T=48, d=8, E=6, d_ff=8, k=3, cf=0.6, mode=0, shared=False, gate=1, drop=1),
+    dict(T=30, d=8, E=8, d_ff=8, k=1, cf=0.5, mode=1, shared=False, gate=1, drop=0),
+    dict(T=41, d=8, E=4, d_ff=8, k=2, cf=0.7, mode=2, shared=True, gate=0, drop=1),
 ])
 def test_oracle_matches_dense_masked_brute_force(case):
     rng = np.random.default_rng(case["T"] * 7 + case["E"])
@@ -264,10 +267,11 @@ def test_oracle_matches_dense_masked_brute_force(case):
     bias = rng.uniform(-0.5, 0.5, case["E"]) if case["mode"] else None
     if case["mode"] == 1:
         bias = bias * 4
+    gm, do = case.get("gate", 0), case.get("drop", 0)
     res = O.moe_forward(x, W_r, W1, W3, W2, k=case["k"], capacity_factor=case["cf"],
-                        bias=bias, bias_mode=case["mode"], **sh)
+                        bias=bias, bias_mode=case["mode"], gate_mode=gm, drop_order=do, **sh)
     b = brute_forward(x, W_r, W1, W3, W2, k=case["k"], cf=case["cf"], bias=bias,
-                      bias_mode=case["mode"], **sh)
+                      bias_mode=case["mode"], gate_mode=gm, drop_order=do, **sh)
     assert np.array_equal(res.routing.idx, b["idx"])
     assert np.array_equal(res.perm.pos, b["pos"])
     assert np.array_equal(res.perm.counts, b["counts"])
@@ -279,6 +283,9 @@ def test_oracle_matches_dense_masked_brute_force(case):
     assert res.stats.l_aux == pytest.approx(b["l_aux"], rel=1e-12)
     if case["cf"] > 0:
         assert res.stats.dropped == int((b["counts"] - b["kept"]).sum())
+    assert res.stats.z_loss == pytest.approx(b["z_loss"], rel=1e-12)
+    assert res.stats.entropy == pytest.approx(b["entropy"], rel=1e-12)
+    assert res.stats.top_gap == pytest.approx(b["top_gap"], rel=1e-12)
 
 
 def test_fully_dropped_token_gets_zero_row():
@@ -323,6 +330,85 @@ def test_unpermute_combine_reproduces_layer_output():
     y = O.unpermute_combine(O_rows, perm.pos, res.routing.gate, S)
     assert np.allclose(y, res.y, rtol=1e-12, atol=1e-13)
     assert res.stats.dropped > 0
+
+
+# --- routing variants ([CMU 15-779 L21] §2.5 and §3.5; [CME295 W2D2] §3.4; [W11 routing] §5) ---
+
+def test_z_loss_and_max_probability_match_printed_values():
+    # 8 experts, logits N(0, std^2): the page's z-loss 6.2 / 59.6 / 988.9 and mean
+    # largest probability 0.355 -> 0.949 come from a finite sample; the expected
+    # values over a large sample sit within 6 % of them
+    g = load("z_loss_table.txt")
+    rng = np.random.default_rng(7)
+    for std, want in zip(g["std"], g["z_loss"]):
+        z = rng.standard_normal((50000, g["E"])) * std
+        assert O.router_z_loss(z) == pytest.approx(want, rel=0.06)
+    z = rng.standard_normal((50000, g["E"]))
+    assert O.softmax_rows(z).max(axis=1).mean() == pytest.approx(g["max_prob_std1"], rel=0.03)
+    z = rng.standard_normal((50000, g["E"])) * 20
+    assert O.softmax_rows(z).max(axis=1).mean() == pytest.approx(g["max_prob_std20"], rel=0.03)
+
+
+def test_router_statistics_closed_forms():
+    for E in (2, 8, 64):
+        z = np.zeros((5, E))
+        assert O.router_z_loss(z) == pytest.approx(math.log(E) ** 2, rel=1e-14)
+        p = O.softmax_rows(z)
+        assert O.router_entropy(p) == pytest.approx(math.log(E), rel=1e-14)
+        assert O.router_top_gap(p) == 0.0
+        # a shift c of every logit moves log-sum-exp by c
+        assert O.router_z_loss(z + 3.0) == pytest.approx((math.log(E) + 3.0) ** 2, rel=1e-14)
+        zd = np.zeros((3, E))
+        zd[:, 0] = 80.0                       # one dominant expert
+        pd = O.softmax_rows(zd)
+        assert O.router_entropy(pd) < 1e-30 + 1e-20 * E
+        assert O.router_top_gap(pd) == pytest.approx(1.0, abs=1e-30)
+
+
+def test_full_softmax_gates_are_switch_top1():
+    # k = 1 with gates renormalised over the selected set is always 1 (the
+    # router gets no gradient); the Switch gate is the full-softmax probability
+    rng = np.random.default_rng(14)
+    z = rng.standard_normal((20, 8)) * 2
+    idx = O.topk_lowest_index(z, 1)
+    assert np.array_equal(O.gates_from_selected(z, idx), np.ones((20, 1)))
+    full = O.gates_full_softmax(z, idx)
+    assert np.allclose(full[:, 0], O.softmax_rows(z).max(axis=1), rtol=1e-15)
+    assert (full < 1).all()
+    # top-2 full gates sum to the two largest probabilities
+    idx2 = O.topk_lowest_index(z, 2)
+    srt = -np.sort(-O.softmax_rows(z), axis=1)
+    assert np.allclose(O.gates_full_softmax(z, idx2).sum(axis=1), srt[:, 0] + srt[:, 1], rtol=1e-14)
+
+
+def test_slot_priority_drop_order_worked_example():
+    # GShard's Algorithm 1: all first choices are placed before any second
+    # choice. Three tokens, two experts, top-2, capacity 2:
+    # x0 -> (0, 1), x1 -> (1, 0), x2 -> (0, 1)
+    idx = np.array([[0, 1], [1, 0], [0, 1]])
+    tok = O.permute(idx, 2, 2, O.DROP_TOKEN)
+    slot = O.permute(idx, 2, 2, O.DROP_SLOT)
+    # token order keeps x0 and x1 in both experts; x2 loses both pairs
+    assert tok.pos.tolist() == [[0, 2], [3, 1], [-1, -1]]
+    # slot priority: expert 0 keeps x0 (1st) and x2 (1st) and drops x1's 2nd
+    # choice; expert 1 keeps x1 (1st) and x0 (2nd) and drops x2's 2nd choice
+    assert slot.pos.tolist() == [[0, 3], [2, -1], [1, -1]]
+    assert slot.counts.tolist() == [3, 3] and slot.kept.tolist() == [2, 2]
+
+
+def test_drop_orders_agree_without_capacity_and_for_top1():
+    rng = np.random.default_rng(15)
+    z = rng.standard_normal((200, 8))
+    idx = O.topk_lowest_index(z, 3)
+    a = O.permute(idx, 8, None, O.DROP_TOKEN)
+    b = O.permute(idx, 8, None, O.DROP_SLOT)
+    assert np.array_equal(a.indptr, b.indptr)
+    for e in range(8):   # same pairs per expert, possibly in another order
+        sa = {tuple(x) for x in np.argwhere(idx == e).tolist()}
+        rows_b = set(range(b.indptr[e], b.indptr[e + 1]))
+        assert {tuple(x) for x in np.argwhere((idx == e) & np.isin(b.pos, list(rows_b))).tolist()} == sa
+    idx1 = O.topk_lowest_index(z, 1)
+    assert np.array_equal(O.permute(idx1, 8, 20, O.DROP_TOKEN).pos, O.permute(idx1, 8, 20, O.DROP_SLOT).pos)
 
 
 # --- closed forms ([CME295 W2D2] §2.3; [CMU 15-779 L21] §3.1 and exercise 4; §2.1 counts) ---
