@@ -61,6 +61,20 @@ extern "C" {
 #define MOE_BIAS_LOGIT 1
 #define MOE_BIAS_PROB  2
 
+/* Gate of a selected expert:
+ * SELECTED: softmax over the k selected raw logits (Week 2 Day 2, §1.3)
+ * FULL    : full-softmax probability of the expert, not renormalised
+ *           (the Switch top-1 gate; Lecture 21, §2.5)                     */
+#define MOE_GATE_SELECTED 0
+#define MOE_GATE_FULL     1
+
+/* Order in which pairs claim an expert's capacity (and rows):
+ * TOKEN: token order inside each expert (Lecture 21, §3.3 prefix sum)
+ * SLOT : every token's first choice before any second choice, then token
+ *        order (GShard's Algorithm 1; Lecture 21, §3.5). Requires E*k <= 4096. */
+#define MOE_DROP_TOKEN 0
+#define MOE_DROP_SLOT  1
+
 /* Limits of this build. */
 #define MOE_MAX_E 512
 #define MOE_MAX_K 16
@@ -76,6 +90,8 @@ typedef struct moe_problem {
     int32_t dtype;            /* MOE_DTYPE_*                                              */
     int32_t bias_mode;        /* MOE_BIAS_*                                               */
     int32_t d_ff_shared;      /* hidden width of the always-on shared expert, 0 = none    */
+    int32_t gate_mode;        /* MOE_GATE_*  (0 = selected softmax)                       */
+    int32_t drop_order;       /* MOE_DROP_*  (0 = token order)                            */
 } moe_problem;
 
 /* ---- statistics block (device memory, moe_stats_size(E) bytes) ----------
@@ -95,7 +111,10 @@ typedef struct moe_stats {
     int32_t max_count;     /* max_e c_e                                                   */
     float   l_aux;         /* E * sum_e f_e P_e                                           */
     float   max_over_mean; /* max_e c_e / (T k / E)                                       */
-    int32_t reserved;
+    float   z_loss;        /* (1/T) sum_t (log sum_e exp z_{t,e})^2 (Week 2 Day 2, §3.4)  */
+    float   entropy;       /* mean over tokens of -sum_e p log p    (W11 routing, §5)     */
+    float   top_gap;       /* mean over tokens of p_(1) - p_(2)     (W11 routing, §5)     */
+    int32_t reserved[2];
 } moe_stats;
 
 #define MOE_STATS_COUNTS(base, E) ((int32_t*)((char*)(base) + sizeof(moe_stats)))
@@ -103,7 +122,7 @@ typedef struct moe_stats {
 #define MOE_STATS_P(base, E)      ((float*)((int32_t*)((char*)(base) + sizeof(moe_stats)) + 2 * (E)))
 #define MOE_STATS_F(base, E)      ((float*)((int32_t*)((char*)(base) + sizeof(moe_stats)) + 3 * (E)))
 
-/* Bytes of the statistics block for E experts. */
+/* Bytes of the statistics block for E experts (48-byte header + 16 E). */
 size_t moe_stats_size(int32_t E);
 
 /* ---- workspace ---------------------------------------------------------

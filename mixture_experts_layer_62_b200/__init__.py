@@ -32,17 +32,22 @@ DTYPE_BF16 = 1
 BIAS_NONE = 0
 BIAS_LOGIT = 1
 BIAS_PROB = 2
+GATE_SELECTED = 0
+GATE_FULL = 1
+DROP_TOKEN = 0
+DROP_SLOT = 1
 MAX_E = 512
 MAX_K = 16
 
-STATS_HEADER_BYTES = 32
+STATS_HEADER_BYTES = 48
 
 
 class Problem(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("d_ff", ctypes.c_int32),
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
                 ("dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
-                ("d_ff_shared", ctypes.c_int32)]
+                ("d_ff_shared", ctypes.c_int32), ("gate_mode", ctypes.c_int32),
+                ("drop_order", ctypes.c_int32)]
 
 
 class WorkspaceLayout(ctypes.Structure):
@@ -131,9 +136,10 @@ def torch_dtype(code: int):
     return torch.bfloat16 if code == DTYPE_BF16 else torch.float32
 
 
-def problem(T, d, d_ff, E, k, capacity_factor=0.0, dtype="bf16", bias_mode=BIAS_NONE, d_ff_shared=0) -> Problem:
+def problem(T, d, d_ff, E, k, capacity_factor=0.0, dtype="bf16", bias_mode=BIAS_NONE, d_ff_shared=0,
+            gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN) -> Problem:
     return Problem(int(T), int(d), int(d_ff), int(E), int(k), float(capacity_factor),
-                   _dtype_code(dtype), int(bias_mode), int(d_ff_shared))
+                   _dtype_code(dtype), int(bias_mode), int(d_ff_shared), int(gate_mode), int(drop_order))
 
 
 def stats_size(E: int) -> int:
@@ -263,6 +269,9 @@ class Stats:
     max_count: int
     l_aux: float
     max_over_mean: float
+    z_loss: float
+    entropy: float
+    top_gap: float
     counts: list
     kept: list
     P: list
@@ -279,6 +288,7 @@ def read_stats(stats: torch.Tensor, E: int) -> Stats:
     flts = body[8 * E:].view(torch.float32)
     return Stats(status=int(hdr_i[0]), capacity=int(hdr_i[1]), rows=int(hdr_i[2]), dropped=int(hdr_i[3]),
                  max_count=int(hdr_i[4]), l_aux=float(hdr_f[5]), max_over_mean=float(hdr_f[6]),
+                 z_loss=float(hdr_f[7]), entropy=float(hdr_f[8]), top_gap=float(hdr_f[9]),
                  counts=ints[:E].tolist(), kept=ints[E:].tolist(), P=flts[:E].tolist(), f=flts[E:].tolist())
 
 

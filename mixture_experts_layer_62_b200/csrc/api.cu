@@ -27,11 +27,13 @@ Layout make_layout(const moe_problem& p) {
     L.row_token = take(T * k * 4);
     L.logits = take(T * E * 4);
     L.wrt = take(E * d * eb);
-    L.blockcnt = take(E * NB * 4);
-    L.blockoff = take(E * NB * 4);
+    const size_t kk = (size_t)count_slots(p);
+    L.blockcnt = take(E * kk * NB * 4);
+    L.blockoff = take(E * kk * NB * 4);
     // per-chunk probability sums; the small-batch router keeps its partial
     // logits [T][parts][E] here
     L.blockpsum = take((small_route_ok(p) ? T * kSmallMaxParts : NB) * E * 4);
+    L.blockextra = take(NB * 3 * 4);
     L.tiles13 = take((E + 3) * 4);
     L.tiles2 = take((E + 3) * 4);
     L.xp = take(T * k * d * eb);
@@ -81,6 +83,9 @@ int check_problem(const moe_problem* p) {
         return MOE_ERR_INVALID_ARG;
     if (p->dtype != MOE_DTYPE_F32 && p->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
     if (p->bias_mode < MOE_BIAS_NONE || p->bias_mode > MOE_BIAS_PROB) return MOE_ERR_INVALID_ARG;
+    if (p->gate_mode != MOE_GATE_SELECTED && p->gate_mode != MOE_GATE_FULL) return MOE_ERR_INVALID_ARG;
+    if (p->drop_order != MOE_DROP_TOKEN && p->drop_order != MOE_DROP_SLOT) return MOE_ERR_INVALID_ARG;
+    if (p->drop_order == MOE_DROP_SLOT && p->E * p->k > kMaxSlotCounts) return MOE_ERR_UNSUPPORTED;
     if (!std::isfinite(p->capacity_factor)) return MOE_ERR_INVALID_ARG;
     const long long rows = (long long)p->T * p->k;
     if (rows * (long long)(p->d > p->d_ff ? p->d : p->d_ff) >= (1LL << 40) || rows >= (1LL << 30))
@@ -328,7 +333,8 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
         // decode-sized batch: routing, statistics, schedules and the gather in one block
         SmallRouteArgs sr = {};
         sr.x = x; sr.W_r = W_r; sr.bias = bias;
-        sr.bias_mode = p->bias_mode; sr.T = p->T; sr.d = p->d; sr.E = p->E; sr.k = p->k; sr.capacity = C;
+        sr.bias_mode = p->bias_mode; sr.gate_mode = p->gate_mode; sr.drop_slot = p->drop_order == MOE_DROP_SLOT;
+        sr.T = p->T; sr.d = p->d; sr.E = p->E; sr.k = p->k; sr.capacity = C;
         sr.logits = logits; sr.probs = blockpsum; sr.idx = idx; sr.gate = gate; sr.pos = pos; sr.indptr = indptr; sr.row_token = row_token;
         sr.xp = xp; sr.stats = stats; sr.tiles13 = tiles13; sr.tiles2 = tiles2; sr.status_reset = status;
         int tile_m, nt13s, nt2s;
@@ -341,10 +347,13 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     } else {
     rc = run_logits(p, x, W_r, logits, L, workspace, status, st, /*reset_status=*/true);
     if (rc != MOE_OK) return rc;
-    CK(launch_select(logits, bias, p->bias_mode, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum, st));
+    float* blockextra = reinterpret_cast<float*>(wsp(workspace, L.blockextra));
+    const int kk = count_slots(*p);
+    CK(launch_select(logits, bias, p->bias_mode, p->gate_mode, kk, p->T, p->E, p->k, idx, gate, blockcnt,
+                     blockpsum, blockextra, st));
     ScanArgs sa = {};
-    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
-    sa.blockcnt = blockcnt; sa.blockoff = blockoff; sa.blockpsum = blockpsum;
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C; sa.kk = kk;
+    sa.blockcnt = blockcnt; sa.blockoff = blockoff; sa.blockpsum = blockpsum; sa.blockextra = blockextra;
     sa.indptr = indptr; sa.stats = stats;
     sa.tiles13 = tiles13; sa.tiles2 = tiles2; sa.has_shared = shared ? 1 : 0;
     schedule_sizes(p, sa.tile_m, sa.ntiles13, sa.ntiles2, sa.ntiles13_shared, sa.ntiles2_shared);
@@ -353,7 +362,7 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     sa.nkb13 = ceil_div(p->d, 64);
     sa.nkb2 = ceil_div(p->d_ff, 64);
     CK(launch_scan(sa, st));
-    CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, C, pos, row_token, xp,
+    CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, kk, C, pos, row_token, xp,
                              st));
     }
     void* h = wsp(workspace, L.h);
@@ -396,11 +405,14 @@ int moe_route(const moe_problem* p, const void* x, const void* W_r, const float*
     if (rc != MOE_OK) return rc;
     int32_t* blockcnt = reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
     float* blockpsum = reinterpret_cast<float*>(wsp(workspace, L.blockpsum));
-    CK(launch_select(lg, bias, p->bias_mode, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum, st));
+    float* blockextra = reinterpret_cast<float*>(wsp(workspace, L.blockextra));
+    const int kk = count_slots(*p);
+    CK(launch_select(lg, bias, p->bias_mode, p->gate_mode, kk, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum,
+                     blockextra, st));
     ScanArgs sa = {};
-    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C; sa.kk = kk;
     sa.blockcnt = blockcnt; sa.blockoff = reinterpret_cast<int32_t*>(wsp(workspace, L.blockoff));
-    sa.blockpsum = blockpsum;
+    sa.blockpsum = blockpsum; sa.blockextra = blockextra;
     sa.indptr = reinterpret_cast<int32_t*>(wsp(workspace, L.indptr));
     sa.stats = stats;
     CK(launch_scan(sa, st));
@@ -426,11 +438,14 @@ int moe_route_from_logits(const moe_problem* p, const float* logits, const float
     CK(cudaMemsetAsync(stats, 0, sizeof(int32_t), st));
     int32_t* blockcnt = reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
     float* blockpsum = reinterpret_cast<float*>(wsp(workspace, L.blockpsum));
-    CK(launch_select(logits, bias, p->bias_mode, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum, st));
+    float* blockextra = reinterpret_cast<float*>(wsp(workspace, L.blockextra));
+    const int kk = count_slots(*p);
+    CK(launch_select(logits, bias, p->bias_mode, p->gate_mode, kk, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum,
+                     blockextra, st));
     ScanArgs sa = {};
-    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C; sa.kk = kk;
     sa.blockcnt = blockcnt; sa.blockoff = reinterpret_cast<int32_t*>(wsp(workspace, L.blockoff));
-    sa.blockpsum = blockpsum;
+    sa.blockpsum = blockpsum; sa.blockextra = blockextra;
     sa.indptr = reinterpret_cast<int32_t*>(wsp(workspace, L.indptr));
     sa.stats = stats;
     CK(launch_scan(sa, st));
@@ -457,13 +472,14 @@ int moe_permute(const moe_problem* p, const void* x, const int32_t* idx, int32_t
     CK(cudaMemsetAsync(stats, 0, sizeof(int32_t), st));
     int32_t* blockcnt = reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
     int32_t* blockoff = reinterpret_cast<int32_t*>(wsp(workspace, L.blockoff));
-    CK(launch_hist(idx, p->T, p->k, p->E, blockcnt, st));
+    const int kk = count_slots(*p);
+    CK(launch_hist(idx, p->T, p->k, kk, p->E, blockcnt, st));
     ScanArgs sa = {};
-    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C; sa.kk = kk;
     sa.blockcnt = blockcnt; sa.blockoff = blockoff; sa.blockpsum = nullptr;
     sa.indptr = indptr; sa.stats = stats;
     CK(launch_scan(sa, st));
-    CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, C, pos, row_token, xp,
+    CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, kk, C, pos, row_token, xp,
                              st));
     return MOE_OK;
 }

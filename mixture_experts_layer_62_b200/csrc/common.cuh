@@ -59,7 +59,7 @@ inline size_t elem_bytes(int dtype) { return dtype == MOE_DTYPE_BF16 ? 2 : 4; }
 // Byte offsets of everything the library keeps in the caller's workspace.
 struct Layout {
     size_t idx, gate, pos, indptr, row_token, logits, wrt;
-    size_t blockcnt, blockoff, blockpsum, tiles13, tiles2;
+    size_t blockcnt, blockoff, blockpsum, blockextra, tiles13, tiles2;
     size_t xp, h, o, hs, s;
     size_t part13, part2;   // fp32 split-K partials (small-T forward only)
     size_t total;
@@ -81,19 +81,25 @@ cudaError_t launch_transpose_wr(int dtype, const void* W_r, void* wrt, int d, in
                                 int32_t* status = nullptr);
 cudaError_t launch_logits_simt(int dtype, const void* x, const void* wrt, float* logits,
                                int T, int d, int E, cudaStream_t st);
-cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
-                          int32_t* idx, float* gate, int32_t* blockcnt, float* blockpsum,
-                          cudaStream_t st);
-cudaError_t launch_hist(const int32_t* idx, int T, int k, int E, int32_t* blockcnt, cudaStream_t st);
+// Per-chunk expert counts are laid out [E][kk][NB] (expert, slot, chunk) with
+// kk = k under the slot-priority drop order and kk = 1 otherwise.
+constexpr int kMaxSlotCounts = 4096;   // E * k limit of the slot-priority order
+inline int count_slots(const moe_problem& p) { return p.drop_order == MOE_DROP_SLOT ? p.k : 1; }
+cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int gate_mode, int kk, int T,
+                          int E, int k, int32_t* idx, float* gate, int32_t* blockcnt, float* blockpsum,
+                          float* blockextra, cudaStream_t st);
+cudaError_t launch_hist(const int32_t* idx, int T, int k, int kk, int E, int32_t* blockcnt, cudaStream_t st);
 
 // Scan over per-chunk expert counts: per-expert totals, capacity, indptr,
 // chunk rank bases, statistics and (optionally) the tile schedules of the
 // two grouped GEMMs.
 struct ScanArgs {
     int T, k, E, capacity;       // capacity < 0: unlimited
-    const int32_t* blockcnt;     // [E][NB]
-    int32_t* blockoff;           // [E][NB]
+    int kk;                      // count slots per expert (k for slot priority, else 1)
+    const int32_t* blockcnt;     // [E][kk][NB]
+    int32_t* blockoff;           // [E][kk][NB]
     const float* blockpsum;      // [NB][E] or null (then P, f, l_aux untouched)
+    const float* blockextra;     // [NB][3] z-loss, entropy, gap sums, or null
     int32_t* indptr;             // [E+1]
     void* stats;                 // moe_stats block
     // tile schedules (null pointers: skipped)
@@ -107,7 +113,7 @@ cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared,
                             int32_t* tiles13, int32_t* tiles2, cudaStream_t st);
 cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
                                   const int32_t* blockoff, const int32_t* indptr,
-                                  int T, int d, int E, int k, int capacity,
+                                  int T, int d, int E, int k, int kk, int capacity,
                                   int32_t* pos, int32_t* row_token, void* xp, cudaStream_t st);
 cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const float* gate,
                            const void* s, void* out, int T, int d, int k, cudaStream_t st,
@@ -128,7 +134,7 @@ constexpr int kSmallMaxE = 64;
 constexpr int kSmallMaxParts = 16;   // partial-logit blocks per token
 struct SmallRouteArgs {
     const void* x; const void* W_r; const float* bias;
-    int bias_mode, T, d, E, k, capacity;
+    int bias_mode, gate_mode, drop_slot, T, d, E, k, capacity;
     float* logits; float* probs /* partial logits [T][parts][E] */; int32_t* idx; float* gate; int32_t* pos; int32_t* indptr; int32_t* row_token;
     int32_t* status_reset;
     void* xp; void* stats;

@@ -76,20 +76,21 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) 
     //    One warp per row, 32 consecutive entries per step (coalesced).
     {
         const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+        const int len = a.kk * NB;   // (slot, chunk) entries of one expert
         for (int e = warp; e < E; e += nw) {
-            const int32_t* row = a.blockcnt + (size_t)e * NB;
-            int32_t* orow = a.blockoff + (size_t)e * NB;
+            const int32_t* row = a.blockcnt + (size_t)e * len;
+            int32_t* orow = a.blockoff + (size_t)e * len;
             int carry = 0;
-            for (int b0 = 0; b0 < NB; b0 += 32) {
+            for (int b0 = 0; b0 < len; b0 += 32) {
                 const int b = b0 + lane;
-                const int v = b < NB ? row[b] : 0;
+                const int v = b < len ? row[b] : 0;
                 int incl = v;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     int n_ = __shfl_up_sync(0xffffffffu, incl, o);
                     if (lane >= o) incl += n_;
                 }
-                if (b < NB) orow[b] = carry + incl - v;
+                if (b < len) orow[b] = carry + incl - v;
                 carry += __shfl_sync(0xffffffffu, incl, 31);
             }
             if (lane == 0) start[e] = carry;   // c_e (converted to a prefix below)
@@ -148,6 +149,16 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) 
             }
         }
     }
+    // router statistics: per-chunk sums of (z-loss, entropy, gap), one warp
+    // each, lane-strided then butterfly (fixed order)
+    __shared__ float extra_s[3];
+    if (a.blockextra != nullptr && warp < 3) {
+        float acc = 0.f;
+        for (int b = lane; b < NB; b += 32) acc += a.blockextra[(size_t)b * 3 + warp];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) extra_s[warp] = a.T > 0 ? acc / (float)a.T : 0.f;
+    }
     __syncthreads();
     // 5. header: fixed-order sums in one thread
     if (threadIdx.x == 0) {
@@ -169,7 +180,13 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) 
             for (int ee = 0; ee < E; ++ee) s += fP[ee];
             st->l_aux = (float)E * s;
         }
-        st->reserved = 0;
+        if (a.blockextra != nullptr) {
+            st->z_loss = extra_s[0];
+            st->entropy = extra_s[1];
+            st->top_gap = extra_s[2];
+        }
+        st->reserved[0] = 0;
+        st->reserved[1] = 0;
     }
     // 6. tile schedules of the grouped GEMMs
     if (a.tiles13 != nullptr) {
@@ -230,7 +247,7 @@ cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared,
 __global__ void __launch_bounds__(256)
 permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
                       const int32_t* __restrict__ blockoff, const int32_t* __restrict__ indptr,
-                      int Tn, int nvec, int E, int k, int capacity,
+                      int Tn, int nvec, int E, int k, int kk, int capacity,
                       int32_t* __restrict__ pos, int32_t* __restrict__ row_token,
                       uint4* __restrict__ xp) {
     __shared__ int sidx[kChunk][MOE_MAX_K];
@@ -254,10 +271,17 @@ permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ i
             if (writer) pos[(size_t)(t0 + q) * k + j] = -1;
             continue;
         }
+        // pairs of this expert earlier in the chunk: any slot of an earlier
+        // token (token order), or the same slot of an earlier token (slot
+        // priority, where the chunk's base already counts earlier slots)
         int before = 0;
-        for (int q2 = 0; q2 < q; ++q2)
-            for (int j2 = 0; j2 < k; ++j2) before += (sidx[q2][j2] == e);
-        const int rank = blockoff[(size_t)e * NB + chunk] + before;
+        if (kk > 1) {
+            for (int q2 = 0; q2 < q; ++q2) before += (sidx[q2][j] == e);
+        } else {
+            for (int q2 = 0; q2 < q; ++q2)
+                for (int j2 = 0; j2 < k; ++j2) before += (sidx[q2][j2] == e);
+        }
+        const int rank = blockoff[((size_t)e * kk + (kk > 1 ? j : 0)) * NB + chunk] + before;
         int p = -1;
         if (capacity < 0 || rank < capacity) p = indptr[e] + rank;
         spos[q][j] = p;
@@ -285,7 +309,7 @@ permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ i
 
 cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
                                   const int32_t* blockoff, const int32_t* indptr,
-                                  int T, int d, int E, int k, int capacity,
+                                  int T, int d, int E, int k, int kk, int capacity,
                                   int32_t* pos, int32_t* row_token, void* xp, cudaStream_t st) {
     int NB = ceil_div(T, kChunk);
     if (NB == 0) return cudaSuccess;
@@ -297,7 +321,7 @@ cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
     groups = max(1, min(groups, ceil_div(nvec, 32)));
     dim3 grid(NB, groups);
     return launch_k(permute_gather_kernel, grid, dim3(256), 0, st, (const uint4*)x, idx, blockoff, indptr, T, nvec,
-                    E, k, capacity, pos, row_token, (uint4*)xp);
+                    E, k, kk, capacity, pos, row_token, (uint4*)xp);
 }
 
 // Statistics for T == 0 (nothing routed).
@@ -313,7 +337,9 @@ __global__ void zero_stats_kernel(void* stats, int E, int capacity) {
     }
     if (threadIdx.x == 0) {
         st->status = MOE_OK; st->capacity = capacity; st->rows = 0; st->dropped = 0;
-        st->max_count = 0; st->l_aux = 0.f; st->max_over_mean = 0.f; st->reserved = 0;
+        st->max_count = 0; st->l_aux = 0.f; st->max_over_mean = 0.f;
+        st->z_loss = 0.f; st->entropy = 0.f; st->top_gap = 0.f;
+        st->reserved[0] = 0; st->reserved[1] = 0;
     }
 }
 

@@ -21,7 +21,8 @@
 
 namespace {
 
-// Scratch capacity: E * ceil(T / 32) entries for each of the two arrays.
+// Scratch capacity: E * kk * ceil(T / 32) entries for each of the two arrays
+// (kk = k under the slot-priority drop order, else 1).
 constexpr long long kMaxEntries = 1LL << 17;
 constexpr int kMaxDevices = 64;
 
@@ -74,7 +75,11 @@ extern "C" int moe_permute_noalloc(const moe_problem* p, const void* x, const in
     if (xp && (!x || !aligned16(x) || !aligned16(xp))) return MOE_ERR_INVALID_ARG;
     if (!aligned16(stats)) return MOE_ERR_INVALID_ARG;
     const long long nb = (p->T + moe::kChunk - 1) / moe::kChunk;
-    if ((long long)p->E * nb > kMaxEntries) return MOE_ERR_UNSUPPORTED;   // beyond the static scratch
+    if (p->gate_mode != MOE_GATE_SELECTED && p->gate_mode != MOE_GATE_FULL) return MOE_ERR_INVALID_ARG;
+    if (p->drop_order != MOE_DROP_TOKEN && p->drop_order != MOE_DROP_SLOT) return MOE_ERR_INVALID_ARG;
+    const int kk = moe::count_slots(*p);
+    if (kk > 1 && p->E * p->k > moe::kMaxSlotCounts) return MOE_ERR_UNSUPPORTED;
+    if ((long long)p->E * kk * nb > kMaxEntries) return MOE_ERR_UNSUPPORTED;   // beyond the static scratch
 
     int32_t* scratch = scratch_on_current_device();
     if (scratch == nullptr) return MOE_ERR_CUDA;
@@ -93,14 +98,14 @@ extern "C" int moe_permute_noalloc(const moe_problem* p, const void* x, const in
         return MOE_OK;
     }
     if (cudaMemsetAsync(stats, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (moe::launch_hist(idx, p->T, p->k, p->E, blockcnt, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe::launch_hist(idx, p->T, p->k, kk, p->E, blockcnt, st) != cudaSuccess) return MOE_ERR_CUDA;
     moe::ScanArgs sa = {};
-    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C;
+    sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C; sa.kk = kk;
     sa.blockcnt = blockcnt; sa.blockoff = blockoff; sa.blockpsum = nullptr;
     sa.indptr = indptr; sa.stats = stats;
     if (moe::launch_scan(sa, st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (moe::launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, C, pos, row_token,
-                                   xp, st) != cudaSuccess)
+    if (moe::launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, kk, C, pos,
+                                   row_token, xp, st) != cudaSuccess)
         return MOE_ERR_CUDA;
     return MOE_OK;
 }

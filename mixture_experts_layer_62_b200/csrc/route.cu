@@ -161,18 +161,24 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Per token it also accumulates the router statistics of the warp's tokens:
+// (log sum_e exp z)^2 for the z-loss, the entropy log-sum-exp - sum_e p z, and
+// the gap between the two largest probabilities, p_(1) - p_(2) =
+// (1 - exp(z_(2) - z_(1))) / sum_e exp(z_e - z_(1)).
 template <int EPL>
 __global__ void __launch_bounds__(kSelWarps * 32)
-select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int bias_mode,
-              int Tn, int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
-              int32_t* __restrict__ blockcnt, float* __restrict__ blockpsum) {
-    __shared__ int cnt[MOE_MAX_E];
+select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int bias_mode, int gate_mode,
+              int kk, int Tn, int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+              int32_t* __restrict__ blockcnt, float* __restrict__ blockpsum, float* __restrict__ blockextra) {
+    __shared__ int cnt[kMaxSlotCounts];
     __shared__ float ps[kSelWarps][MOE_MAX_E];
+    __shared__ float ext[kSelWarps][3];
     pdl_wait();
     pdl_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunk = blockIdx.x, NB = gridDim.x;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    for (int e = threadIdx.x; e < E * kk; e += blockDim.x) cnt[e] = 0;
+    float ex_z = 0.f, ex_h = 0.f, ex_g = 0.f;
     __syncthreads();
 
     float b[EPL];
@@ -210,6 +216,30 @@ select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, 
         }
         s = warp_sum(s);
         const float inv_s = 1.f / s;
+        // router statistics of this token
+        {
+            float pz = 0.f, z1 = -INFINITY, z2 = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                if (lane + 32 * i < E) {
+                    pz += ex[i] * z[i];
+                    if (z[i] > z1) { z2 = z1; z1 = z[i]; } else if (z[i] > z2) { z2 = z[i]; }
+                }
+            }
+            pz = warp_sum(pz) * inv_s;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float o1 = __shfl_xor_sync(0xffffffffu, z1, o);
+                const float o2 = __shfl_xor_sync(0xffffffffu, z2, o);
+                const float hi = fmaxf(z1, o1);
+                z2 = fmaxf(fminf(z1, o1), fmaxf(z2, o2));
+                z1 = hi;
+            }
+            const float lse = m + logf(s);
+            ex_z += lse * lse;
+            ex_h += lse - pz;
+            ex_g += (1.f - expf(z2 - m)) * inv_s;
+        }
         unsigned valid = 0;
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
@@ -268,11 +298,18 @@ select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, 
             for (int j = 0; j < MOE_MAX_K; ++j) {
                 if (j < k) {
                     idx_out[(size_t)t * k + j] = esel[j];
-                    gate_out[(size_t)t * k + j] = ge[j] * inv_g;
-                    atomicAdd(&cnt[esel[j]], 1);   // integer: order does not matter
+                    // selected softmax, or the full-softmax probability (Switch gate)
+                    gate_out[(size_t)t * k + j] =
+                        gate_mode == MOE_GATE_FULL ? expf(zsel[j] - m) * inv_s : ge[j] * inv_g;
+                    atomicAdd(&cnt[esel[j] * kk + (kk > 1 ? j : 0)], 1);   // integer: order does not matter
                 }
             }
         }
+    }
+    if (lane == 0) {
+        ext[warp][0] = ex_z;
+        ext[warp][1] = ex_h;
+        ext[warp][2] = ex_g;
     }
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
@@ -284,58 +321,56 @@ select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, 
         float acc = 0.f;
         for (int w = 0; w < kSelWarps; ++w) acc += ps[w][e];   // fixed order over warps
         blockpsum[(size_t)chunk * E + e] = acc;
-        blockcnt[(size_t)e * NB + chunk] = cnt[e];
+    }
+    for (int i = threadIdx.x; i < E * kk; i += blockDim.x) blockcnt[(size_t)i * NB + chunk] = cnt[i];
+    if (threadIdx.x < 3 && blockextra != nullptr) {
+        float acc = 0.f;
+        for (int w = 0; w < kSelWarps; ++w) acc += ext[w][threadIdx.x];
+        blockextra[(size_t)chunk * 3 + threadIdx.x] = acc;
     }
 }
 
-cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int T, int E, int k,
-                          int32_t* idx, float* gate, int32_t* blockcnt, float* blockpsum,
-                          cudaStream_t st) {
+cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int gate_mode, int kk, int T,
+                          int E, int k, int32_t* idx, float* gate, int32_t* blockcnt, float* blockpsum,
+                          float* blockextra, cudaStream_t st) {
     int NB = ceil_div(T, kChunk);
     if (NB == 0) return cudaSuccess;
     dim3 grid(NB), block(kSelWarps * 32);
     int epl = ceil_div(E, 32);
-    if (epl <= 1)
-        return launch_k(select_kernel<1>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
-                        blockpsum);
-    else if (epl <= 2)
-        return launch_k(select_kernel<2>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
-                        blockpsum);
-    else if (epl <= 4)
-        return launch_k(select_kernel<4>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
-                        blockpsum);
-    else if (epl <= 8)
-        return launch_k(select_kernel<8>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
-                        blockpsum);
-    else
-        return launch_k(select_kernel<16>, grid, block, 0, st, logits, bias, bias_mode, T, E, k, idx, gate, blockcnt,
-                        blockpsum);
-    return cudaGetLastError();
+#define MOE_SELECT(EPLV)                                                                                        \
+    return launch_k(select_kernel<EPLV>, grid, block, 0, st, logits, bias, bias_mode, gate_mode, kk, T, E, k, idx, \
+                    gate, blockcnt, blockpsum, blockextra)
+    if (epl <= 1) MOE_SELECT(1);
+    if (epl <= 2) MOE_SELECT(2);
+    if (epl <= 4) MOE_SELECT(4);
+    if (epl <= 8) MOE_SELECT(8);
+    MOE_SELECT(16);
+#undef MOE_SELECT
 }
 
 // ---- per-chunk histogram of given selections (standalone permutation) ----
-__global__ void hist_kernel(const int32_t* __restrict__ idx, int Tn, int k, int E,
+__global__ void hist_kernel(const int32_t* __restrict__ idx, int Tn, int k, int kk, int E,
                             int32_t* __restrict__ blockcnt) {
-    __shared__ int cnt[MOE_MAX_E];
+    __shared__ int cnt[kMaxSlotCounts];
     pdl_wait();
     pdl_launch();
     const int chunk = blockIdx.x, NB = gridDim.x;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    for (int e = threadIdx.x; e < E * kk; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     const int t0 = chunk * kChunk;
     const int n = min(kChunk, Tn - t0) * k;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         int e = idx[(size_t)t0 * k + i];
-        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+        if (e >= 0 && e < E) atomicAdd(&cnt[e * kk + (kk > 1 ? i % k : 0)], 1);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) blockcnt[(size_t)e * NB + chunk] = cnt[e];
+    for (int i = threadIdx.x; i < E * kk; i += blockDim.x) blockcnt[(size_t)i * NB + chunk] = cnt[i];
 }
 
-cudaError_t launch_hist(const int32_t* idx, int T, int k, int E, int32_t* blockcnt, cudaStream_t st) {
+cudaError_t launch_hist(const int32_t* idx, int T, int k, int kk, int E, int32_t* blockcnt, cudaStream_t st) {
     int NB = ceil_div(T, kChunk);
     if (NB == 0) return cudaSuccess;
-    return launch_k(hist_kernel, dim3(NB), dim3(256), 0, st, idx, T, k, E, blockcnt);
+    return launch_k(hist_kernel, dim3(NB), dim3(256), 0, st, idx, T, k, kk, E, blockcnt);
 }
 
 }  // namespace moe

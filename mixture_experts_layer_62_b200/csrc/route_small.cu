@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
     __shared__ int spos[kSmallMaxPairs];
     __shared__ int indptr_s[kSmallMaxE + 1];
     __shared__ float bias_s[kSmallMaxE];
+    __shared__ float extw[kFinWarps][3];
     const int T = a.T, E = a.E, k = a.k;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool writer = blockIdx.x == 0;
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
     }
     __syncthreads();
 
+    float ex_z = 0.f, ex_h = 0.f, ex_g = 0.f;
     for (int t = warp; t < T; t += kFinWarps) {
         float zz[2], key[2], ex[2];
         unsigned valid = 0;
@@ -162,6 +164,29 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
         }
         s = warp_sum(s);
         const float inv_s = 1.f / s;
+        {   // router statistics of this token (z-loss, entropy, top-1/top-2 gap)
+            float pz = 0.f, z1 = -INFINITY, z2 = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if ((valid >> i) & 1u) {
+                    pz += ex[i] * zz[i];
+                    if (zz[i] > z1) { z2 = z1; z1 = zz[i]; } else if (zz[i] > z2) { z2 = zz[i]; }
+                }
+            }
+            pz = warp_sum(pz) * inv_s;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float o1 = __shfl_xor_sync(0xffffffffu, z1, o);
+                const float o2 = __shfl_xor_sync(0xffffffffu, z2, o);
+                const float hi = fmaxf(z1, o1);
+                z2 = fmaxf(fminf(z1, o1), fmaxf(z2, o2));
+                z1 = hi;
+            }
+            const float lse = m + logf(s);
+            ex_z += lse * lse;
+            ex_h += lse - pz;
+            ex_g += (1.f - expf(z2 - m)) * inv_s;
+        }
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int e = lane + 32 * i;
@@ -209,10 +234,16 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
                 sidx[t * k + j] = esel[j];
                 if (writer) {
                     a.idx[(size_t)t * k + j] = esel[j];
-                    a.gate[(size_t)t * k + j] = ge[j] * inv_g;
+                    a.gate[(size_t)t * k + j] =
+                        a.gate_mode == MOE_GATE_FULL ? expf(zsel[j] - m) * inv_s : ge[j] * inv_g;
                 }
             }
         }
+    }
+    if (lane == 0) {
+        extw[warp][0] = ex_z;
+        extw[warp][1] = ex_h;
+        extw[warp][2] = ex_g;
     }
     __syncthreads();
 
@@ -302,15 +333,32 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
                 st->max_count = maxc;
                 st->l_aux = laux;
                 st->max_over_mean = (float)maxc / ((float)T * (float)k / (float)E);
-                st->reserved = 0;
+                float ez = 0.f, eh = 0.f, eg = 0.f;
+                for (int w = 0; w < kFinWarps; ++w) {   // fixed order over warps
+                    ez += extw[w][0];
+                    eh += extw[w][1];
+                    eg += extw[w][2];
+                }
+                st->z_loss = ez / (float)T;
+                st->entropy = eh / (float)T;
+                st->top_gap = eg / (float)T;
+                st->reserved[0] = 0;
+                st->reserved[1] = 0;
             }
         }
     }
     __syncthreads();
     for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-        const int t = i / k, e = sidx[i];
+        const int t = i / k, j = i % k, e = sidx[i];
         int rank = 0;
-        for (int q = 0; q < t * k; ++q) rank += (sidx[q] == e);
+        if (a.drop_slot) {   // earlier slots of every token, then this slot of earlier tokens
+            for (int q = 0; q < T * k; ++q) {
+                const int tq = q / k, jq = q % k;
+                rank += (sidx[q] == e) && (jq < j || (jq == j && tq < t));
+            }
+        } else {
+            for (int q = 0; q < t * k; ++q) rank += (sidx[q] == e);
+        }
         const int p = (a.capacity < 0 || rank < a.capacity) ? indptr_s[e] + rank : -1;
         spos[i] = p;
         if (writer) {

@@ -23,7 +23,7 @@ from dataclasses import dataclass
 import torch
 import torch.distributed as dist
 
-STATS_HEADER_BYTES = 32
+STATS_HEADER_BYTES = 48
 
 
 def shard_range(T_global: int, world: int, rank: int):

@@ -42,8 +42,8 @@ def test_error_strings():
 
 
 def test_stats_size_matches_header_layout():
-    assert moe.stats_size(8) == 32 + 16 * 8
-    assert moe.stats_size(256) == 32 + 16 * 256
+    assert moe.stats_size(8) == 48 + 16 * 8
+    assert moe.stats_size(256) == 48 + 16 * 256
 
 
 def test_workspace_layout_is_aligned_and_ordered():
@@ -88,6 +88,17 @@ def test_bad_bias_mode_and_dtype_rejected():
     p = moe.problem(16, 64, 64, 4, 2)
     p.dtype = 5
     assert moe.lib.moe_forward(ctypes.byref(p), *([fake] * 11), fake, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_bad_gate_and_drop_modes_rejected():
+    fake = ctypes.c_void_p(1 << 20)
+    for kw, code in ((dict(gate_mode=2), moe.MOE_ERR_INVALID_ARG), (dict(drop_order=5), moe.MOE_ERR_INVALID_ARG),
+                     (dict(drop_order=moe.DROP_SLOT), moe.MOE_ERR_UNSUPPORTED)):
+        E, k = (512, 16) if kw.get("drop_order") == moe.DROP_SLOT else (4, 2)   # slot order: E*k <= 4096
+        p = moe.problem(16, 64, 64, E, k, **kw)
+        assert moe.lib.moe_forward(ctypes.byref(p), *([fake] * 11), fake, 1 << 30, None) == code
+    p = moe.problem(16, 64, 64, 256, 16, drop_order=moe.DROP_SLOT)   # 4096: allowed
+    assert moe.lib.moe_workspace_size(ctypes.byref(p)) > 0
 
 
 def test_null_and_misaligned_pointers_rejected():

@@ -35,17 +35,18 @@ def _dt(name):
 # routing from given logits
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("T,E,k,mode", [
-    (1000, 8, 2, 0), (777, 8, 2, 1), (300, 64, 8, 0), (513, 256, 8, 1), (64, 256, 8, 0),
-    (40, 5, 5, 0), (33, 1, 1, 0), (1, 8, 2, 1), (95, 512, 16, 0), (200, 32, 1, 1),
+@pytest.mark.parametrize("T,E,k,mode,gm", [
+    (1000, 8, 2, 0, 0), (777, 8, 2, 1, 0), (300, 64, 8, 0, 0), (513, 256, 8, 1, 0), (64, 256, 8, 0, 0),
+    (40, 5, 5, 0, 0), (33, 1, 1, 0, 0), (1, 8, 2, 1, 0), (95, 512, 16, 0, 0), (200, 32, 1, 1, 0),
+    (500, 8, 1, 0, 1), (300, 64, 2, 1, 1), (129, 256, 8, 0, 1),
 ])
-def test_route_from_logits_bit_exact(T, E, k, mode):
+def test_route_from_logits_bit_exact(T, E, k, mode, gm):
     rng = np.random.default_rng(T * 31 + E)
     z = rng.standard_normal((T, E)).astype(np.float32) * 2
     if E >= 3:
         z[::7, 1:3] = z[::7, 0:1]           # exact ties: the lower index must win
     bias = rng.uniform(-0.5, 0.5, E).astype(np.float32) if mode else None
-    p = moe.problem(T, 64, 64, E, k, 0.0, "bf16", mode)
+    p = moe.problem(T, 64, 64, E, k, 0.0, "bf16", mode, gate_mode=gm)
     ws = moe.alloc_workspace(p, DEV)
     st = moe.alloc_stats(E, DEV)
     idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
@@ -53,16 +54,19 @@ def test_route_from_logits_bit_exact(T, E, k, mode):
     moe.route_from_logits(p, torch.from_numpy(z).to(DEV), idx, gate, st, ws,
                           bias=None if bias is None else torch.from_numpy(bias).to(DEV))
     torch.cuda.synchronize()
-    r = O.route(z, k, bias, mode, key_dtype=np.float32)
+    r = O.route(z, k, bias, mode, key_dtype=np.float32, gate_mode=gm)
     assert np.array_equal(idx.cpu().numpy(), r.idx)
     assert np.allclose(gate.cpu().numpy(), r.gate, rtol=2e-6, atol=1e-7)
     s = moe.read_stats(st, E)
     perm = O.permute(r.idx, E)
-    ls = O.load_stats(perm, r.probs, T, k, None)
+    ls = O.load_stats(perm, r.probs, T, k, None, z=z)
     assert s.status == moe.MOE_OK
     assert s.counts == ls.counts.tolist()
     assert np.allclose(s.P, ls.P, rtol=1e-5, atol=1e-7)
     assert s.l_aux == pytest.approx(ls.l_aux, rel=TOL_LAUX)
+    assert s.z_loss == pytest.approx(ls.z_loss, rel=1e-5)
+    assert s.entropy == pytest.approx(ls.entropy, rel=1e-5, abs=1e-6)
+    assert s.top_gap == pytest.approx(ls.top_gap, rel=1e-5, abs=1e-6)
     assert s.rows == T * k and s.dropped == 0 and s.capacity == -1
 
 
@@ -104,18 +108,20 @@ def test_route_from_logits_prob_bias(T, E, k):
 # permutation
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("T,E,k,cf,dtype", [
-    (1000, 8, 2, 0.0, "bf16"), (1000, 8, 2, 0.6, "bf16"), (31, 4, 2, 0.5, "f32"), (1, 8, 2, 0.0, "bf16"),
-    (2049, 256, 8, 1.0, "bf16"), (300, 64, 8, 0.3, "f32"), (64, 3, 3, 0.9, "bf16"), (4096, 8, 2, 1.25, "bf16"),
+@pytest.mark.parametrize("T,E,k,cf,dtype,drop", [
+    (1000, 8, 2, 0.0, "bf16", 0), (1000, 8, 2, 0.6, "bf16", 0), (31, 4, 2, 0.5, "f32", 0), (1, 8, 2, 0.0, "bf16", 0),
+    (2049, 256, 8, 1.0, "bf16", 0), (300, 64, 8, 0.3, "f32", 0), (64, 3, 3, 0.9, "bf16", 0),
+    (4096, 8, 2, 1.25, "bf16", 0),
+    (1000, 8, 2, 0.6, "bf16", 1), (2049, 256, 8, 1.0, "bf16", 1), (77, 6, 3, 0.4, "f32", 1), (1, 8, 2, 0.3, "bf16", 1),
 ])
-def test_permute_bit_exact(T, E, k, cf, dtype):
+def test_permute_bit_exact(T, E, k, cf, dtype, drop):
     rng = np.random.default_rng(T + E * 7)
     z = rng.standard_normal((T, E))
     z[:, 0] += 1.0                                    # skew toward expert 0 so capacity bites
     idx_np = O.topk_lowest_index(z, k)
     d = 128 if dtype == "bf16" else 64
     x = torch.randn((T, d), dtype=torch.float32).to(_dt(dtype)).to(DEV)
-    p = moe.problem(T, d, 64, E, k, cf, dtype)
+    p = moe.problem(T, d, 64, E, k, cf, dtype, drop_order=drop)
     ws = moe.alloc_workspace(p, DEV)
     st = moe.alloc_stats(E, DEV)
     idx = torch.from_numpy(idx_np.astype(np.int32)).to(DEV)
@@ -126,7 +132,7 @@ def test_permute_bit_exact(T, E, k, cf, dtype):
     moe.permute(p, x, idx, pos, indptr, row_token, xp, st, ws)
     torch.cuda.synchronize()
     C = O.capacity(cf, T, k, E)
-    perm = O.permute(idx_np, E, C)
+    perm = O.permute(idx_np, E, C, drop)
     assert np.array_equal(pos.cpu().numpy(), perm.pos)
     assert np.array_equal(indptr.cpu().numpy(), perm.indptr)
     R = int(perm.indptr[-1])
@@ -247,10 +253,15 @@ SMALL = [
     # T*k <= 128 rows: moe_forward may split K of both GEMMs (fp32 partials)
     dict(T=16, d=1024, d_ff=512, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     dict(T=5, d=256, d_ff=1024, E=4, k=2, cf=0.0, dtype="bf16", bias_mode=1, d_ff_shared=0),
-    # T*k <= 64, E % 8 == 0, E <= 64: the single-block small-batch router
+    # T*k <= 64, E % 8 == 0, E <= 64: the small-batch router
     dict(T=20, d=256, d_ff=256, E=64, k=2, cf=0.5, dtype="bf16", bias_mode=1, d_ff_shared=0),
     dict(T=8, d=512, d_ff=256, E=16, k=4, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=0),
     dict(T=3, d=128, d_ff=128, E=8, k=8, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    # routing variants: Switch full-softmax gates, GShard slot-priority drops
+    dict(T=500, d=256, d_ff=256, E=8, k=1, cf=1.0, dtype="bf16", bias_mode=0, d_ff_shared=0, gate=1, drop=0),
+    dict(T=700, d=128, d_ff=256, E=16, k=2, cf=0.7, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=0, drop=1),
+    dict(T=24, d=256, d_ff=128, E=8, k=2, cf=0.6, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=1, drop=1),
+    dict(T=200, d=64, d_ff=64, E=6, k=3, cf=0.5, dtype="f32", bias_mode=0, d_ff_shared=0, gate=1, drop=1),
 ]
 
 
@@ -292,7 +303,8 @@ def _check_forward(cfg, L_cpu, tokens=None, check_own_routing=True):
     exact_key = cfg["bias_mode"] != O.BIAS_PROB
     res = O.moe_forward(x_np, None, W["W1"], W["W3"], W["W2"], k, cfg["cf"], bias, cfg["bias_mode"],
                         W["Ws1"], W["Ws3"], W["Ws2"], logits=logits, tokens=tokens,
-                        key_dtype=np.float32 if exact_key else np.float64)
+                        key_dtype=np.float32 if exact_key else np.float64,
+                        gate_mode=cfg.get("gate", 0), drop_order=cfg.get("drop", 0))
     if exact_key:
         assert np.array_equal(g_idx, res.routing.idx)
         assert np.array_equal(g_pos, res.perm.pos)
@@ -312,6 +324,9 @@ def _check_forward(cfg, L_cpu, tokens=None, check_own_routing=True):
         assert (np.diff(kg, axis=1) <= 1e-6).all()
         assert cfg["cf"] <= 0, "PROB-key parity with capacity needs a drop-set argument"
     assert s.l_aux == pytest.approx(res.stats.l_aux, rel=TOL_LAUX)
+    assert s.z_loss == pytest.approx(res.stats.z_loss, rel=1e-4)
+    assert s.entropy == pytest.approx(res.stats.entropy, rel=1e-4, abs=1e-6)
+    assert s.top_gap == pytest.approx(res.stats.top_gap, rel=1e-4, abs=1e-6)
     toks = res.tokens
     sel = good[toks]
     got = out.float().cpu().numpy()[toks]
@@ -331,7 +346,8 @@ def _check_forward(cfg, L_cpu, tokens=None, check_own_routing=True):
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=[f"T{c['T']}_E{c['E']}_k{c['k']}_{c['dtype']}_b{c['bias_mode']}"
-                                            f"_cf{c['cf']}_s{c['d_ff_shared']}" for c in SMALL])
+                                            f"_cf{c['cf']}_s{c['d_ff_shared']}_g{c.get('gate', 0)}"
+                                            f"_d{c.get('drop', 0)}" for c in SMALL])
 def test_forward_small(cfg):
     _check_forward(cfg, _small_layer(cfg, cfg["T"] + cfg["E"]))
 
