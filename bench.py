@@ -283,9 +283,17 @@ def config_of(cfg, args):
 
 
 def launches_per_forward(cfg):
+    """Kernels one moe_forward launches (the library's own choice of path)."""
+    if cfg["T"] == 0:
+        return 1
+    small = (cfg["dtype"] == "bf16" and cfg["d_ff_shared"] == 0 and cfg["T"] * cfg["k"] <= 64
+             and cfg["E"] <= 64 and cfg["E"] % 8 == 0 and cfg["d"] % 8 == 0)
+    if small:
+        # partial router logits, routing finisher, grouped GEMM 1/3, grouped GEMM 2, combine
+        return 5
     # transpose W_r, logits (SIMT or tensor-core), select, scan, permute+gather,
     # grouped GEMM 1/3, grouped GEMM 2, combine
-    return 8 if cfg["T"] > 0 else 1
+    return 8
 
 
 def main():

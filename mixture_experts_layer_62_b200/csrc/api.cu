@@ -44,8 +44,44 @@ Layout make_layout(const moe_problem& p) {
     const bool split = split_allowed(p);
     L.part13 = take(split ? (size_t)kSplitMax * T * k * (size_t)ceil_div(p.d_ff, 128) * 256 * 4 : 0);
     L.part2 = take(split ? (size_t)kSplitMax * T * k * d * 4 : 0);
+    // at most min(E, T*k) experts are active, each with one M-block of tiles
+    const size_t active = split ? (T * k < E ? T * k : E) : 0;
+    L.sem13_n = (int)(active * (size_t)ceil_div(p.d_ff, 128) * kSemPerTile);
+    L.sem2_n = (int)(active * (size_t)ceil_div(p.d, 256) * kSemPerTile);
+    L.sem = take(((size_t)L.sem13_n + (size_t)L.sem2_n) * 4);
     L.total = off;
     return L;
+}
+
+int pick_split(int tiles, int nkb, int sm, int smax) {
+    if (smax <= 1 || tiles <= 0 || sm <= 0) return 1;
+    long long best = -1;
+    int bs = 1;
+    for (int s = 1; s <= smax && s <= nkb; ++s) {
+        const long long c = ((long long)tiles * s + sm - 1) / sm * ((nkb + s - 1) / s + 1);
+        if (best < 0 || c < best) {
+            best = c;
+            bs = s;
+        }
+    }
+    return bs;
+}
+
+void fill_split_table(SplitTable& t, int nt13, int nt2, int nkb13, int nkb2, int sm, int smax) {
+    // the table depends on six integers; reuse the last one this thread built
+    static thread_local int key[6] = {-1, -1, -1, -1, -1, -1};
+    static thread_local SplitTable last;
+    const int k6[6] = {nt13, nt2, nkb13, nkb2, sm, smax};
+    bool hit = true;
+    for (int i = 0; i < 6; ++i) hit = hit && key[i] == k6[i];
+    if (!hit) {
+        for (int n = 0; n <= kSplitMaxRows; ++n) {
+            last.s13[n] = (uint8_t)pick_split(n * nt13, nkb13, sm, smax);
+            last.s2[n] = (uint8_t)pick_split(n * nt2, nkb2, sm, smax);
+        }
+        for (int i = 0; i < 6; ++i) key[i] = k6[i];
+    }
+    t = last;
 }
 
 bool split_allowed(const moe_problem& p) {
@@ -145,12 +181,13 @@ int run_logits(const moe_problem* p, const void* x, const void* W_r, float* logi
 // Grouped GEMM 1/3 with the SwiGLU epilogue (and the shared expert's).
 int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13, const void* W1,
            const void* W3, const void* x, const void* Ws1, const void* Ws3, void* h, void* hs, int32_t* status,
-           cudaStream_t st, float* part13 = nullptr) {
+           cudaStream_t st, float* part13 = nullptr, int32_t* sem13 = nullptr, bool sched_early = true) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
     if (p->dtype == MOE_DTYPE_BF16) {
         TcArgs a = {};
         a.mode = TC_SWIGLU;
+        a.b_before_wait = sched_early ? 1 : 0;
         a.indptr = indptr; a.tiles = tiles13;
         a.E = p->E; a.has_shared = has_shared; a.T = p->T;
         a.A[0] = xp; a.a_rows[0] = rows; a.A[1] = has_shared ? x : nullptr; a.a_rows[1] = p->T;
@@ -164,11 +201,9 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
             a.partial = part13;
             a.partial_ld = ceil_div(p->d_ff, 128) * 256;
             a.partial_stride = (long long)rows * a.partial_ld;
+            a.sem = sem13;
         }
         CK(launch_tc_gemm(a, st));
-        if (part13 != nullptr)
-            CK(launch_swiglu_reduce(part13, a.partial_stride, a.partial_ld, tiles13 + p->E + has_shared + 1, indptr,
-                                    p->E, rows, p->d_ff, h, st));
     } else {
         GroupedArgs a = {};
         a.indptr = indptr; a.tiles = tiles13;
@@ -187,12 +222,13 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
 // Grouped GEMM 2 (down projection, and the shared expert's).
 int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const int32_t* tiles2, const void* W2,
              const void* hs, const void* Ws2, void* o, void* s, int32_t* status, cudaStream_t st,
-             float* part2 = nullptr) {
+             float* part2 = nullptr, int32_t* sem2 = nullptr) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
     if (p->dtype == MOE_DTYPE_BF16) {
         TcArgs b = {};
         b.mode = TC_PLAIN;
+        b.b_before_wait = 1;   // the schedule comes from the router, two or more launches back
         b.indptr = indptr; b.tiles = tiles2;
         b.E = p->E; b.has_shared = has_shared; b.T = p->T;
         b.A[0] = h; b.a_rows[0] = rows; b.A[1] = has_shared ? hs : nullptr; b.a_rows[1] = p->T;
@@ -206,6 +242,7 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
             b.partial = part2;
             b.partial_ld = p->d;
             b.partial_stride = (long long)rows * p->d;
+            b.sem = sem2;
         }
         CK(launch_tc_gemm(b, st));
     } else {
@@ -226,10 +263,11 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
 int run_experts(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13,
                 const int32_t* tiles2, const void* W1, const void* W3, const void* W2, const void* x,
                 const void* Ws1, const void* Ws3, const void* Ws2, void* h, void* hs, void* o, void* s,
-                int32_t* status, cudaStream_t st, float* part13 = nullptr, float* part2 = nullptr) {
-    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st, part13);
+                int32_t* status, cudaStream_t st, float* part13 = nullptr, float* part2 = nullptr,
+                int32_t* sem13 = nullptr, int32_t* sem2 = nullptr, bool sched_early = true) {
+    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st, part13, sem13, sched_early);
     if (rc != MOE_OK) return rc;
-    return run_down(p, h, indptr, tiles2, W2, hs, Ws2, o, s, status, st, part2);
+    return run_down(p, h, indptr, tiles2, W2, hs, Ws2, o, s, status, st, part2, sem2);
 }
 
 void schedule_sizes(const moe_problem* p, int& tile_m, int& nt13, int& nt2, int& nt13s, int& nt2s) {
@@ -328,8 +366,10 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     int32_t* tiles2 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles2));
 
     const bool split = split_allowed(*p);
+    int32_t* sem = split ? reinterpret_cast<int32_t*>(wsp(workspace, L.sem)) : nullptr;
     void* xp = wsp(workspace, L.xp);
-    if (small_route_ok(*p)) {
+    const bool small = small_route_ok(*p);
+    if (small) {
         // decode-sized batch: routing, statistics, schedules and the gather in one block
         SmallRouteArgs sr = {};
         sr.x = x; sr.W_r = W_r; sr.bias = bias;
@@ -339,10 +379,13 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
         sr.xp = xp; sr.stats = stats; sr.tiles13 = tiles13; sr.tiles2 = tiles2; sr.status_reset = status;
         int tile_m, nt13s, nt2s;
         schedule_sizes(p, tile_m, sr.nt13, sr.nt2, nt13s, nt2s);
-        sr.split_max = split ? kSplitMax : 1;
-        sr.sm_count = device_sm_count();
-        sr.nkb13 = ceil_div(p->d, 64);
-        sr.nkb2 = ceil_div(p->d_ff, 64);
+        sr.split_on = split ? 1 : 0;
+        if (split) {
+            sr.sem = sem;
+            sr.sem_n = L.sem13_n + L.sem2_n;
+            fill_split_table(sr.split, sr.nt13, sr.nt2, ceil_div(p->d, 64), ceil_div(p->d_ff, 64),
+                             device_sm_count(), kSplitMax);
+        }
         CK(launch_route_small(sr, st));
     } else {
     rc = run_logits(p, x, W_r, logits, L, workspace, status, st, /*reset_status=*/true);
@@ -357,10 +400,13 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     sa.indptr = indptr; sa.stats = stats;
     sa.tiles13 = tiles13; sa.tiles2 = tiles2; sa.has_shared = shared ? 1 : 0;
     schedule_sizes(p, sa.tile_m, sa.ntiles13, sa.ntiles2, sa.ntiles13_shared, sa.ntiles2_shared);
-    sa.split_max = split ? kSplitMax : 1;
-    sa.sm_count = device_sm_count();
-    sa.nkb13 = ceil_div(p->d, 64);
-    sa.nkb2 = ceil_div(p->d_ff, 64);
+    sa.split_on = split ? 1 : 0;
+    if (split) {
+        sa.sem = sem;
+        sa.sem_n = L.sem13_n + L.sem2_n;
+        fill_split_table(sa.split, sa.ntiles13, sa.ntiles2, ceil_div(p->d, 64), ceil_div(p->d_ff, 64),
+                         device_sm_count(), kSplitMax);
+    }
     CK(launch_scan(sa, st));
     CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, kk, C, pos, row_token, xp,
                              st));
@@ -371,12 +417,12 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     void* s = shared ? wsp(workspace, L.s) : nullptr;
     float* part13 = split ? reinterpret_cast<float*>(wsp(workspace, L.part13)) : nullptr;
     float* part2 = split ? reinterpret_cast<float*>(wsp(workspace, L.part2)) : nullptr;
+    // the small router writes the schedule right before GEMM 1/3; the general
+    // path writes it in the scan, two launches before
     rc = run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st, part13,
-                     part2);
+                     part2, sem, sem ? sem + L.sem13_n : nullptr, /*sched_early=*/!small);
     if (rc != MOE_OK) return rc;
-    const int G = p->E + (shared ? 1 : 0);
-    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st, part2,
-                      (long long)p->T * p->k * p->d, split ? tiles2 + G + 1 : nullptr));
+    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st));
     return MOE_OK;
 }
 

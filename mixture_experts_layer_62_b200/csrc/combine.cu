@@ -44,31 +44,25 @@ template <> struct VecTraits<__nv_bfloat16> {
 
 // One warp per (token, slice of the row): a slice is 32 x vpl 16-byte
 // vectors (vpl = 1 for small batches), so few tokens still spread over many
-// warps. With
-// split-K partials (opart != null and *split2 > 1) an expert output row is the
-// sum over the splits, s = 0, 1, ..., of the fp32 partial rows.
+// warps.
 constexpr int kCbVecPerLane = 2;
 constexpr int kCbWarps = 8;
 
 template <typename T>
 __global__ void __launch_bounds__(kCbWarps * 32, 4)
 combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const float* __restrict__ gate,
-               const T* __restrict__ s, T* __restrict__ out, int Tn, int d, int k,
-               const float* __restrict__ opart, long long opart_stride, const int32_t* __restrict__ split2,
-               int slices, int vpl) {
+               const T* __restrict__ s, T* __restrict__ out, int Tn, int d, int k, int slices, int vpl) {
     using V = VecTraits<T>;
     constexpr int VN = V::N;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long task = (long long)blockIdx.x * kCbWarps + warp;
     const int t = (int)(task / slices), sl = (int)(task % slices);
-    // pos, gate and the split factor come from kernels at least two launches
-    // back (routing and scan run before both GEMMs), so they are read before
-    // the dependency wait; the expert outputs are read after it
+    // pos and gate come from the routing, at least two launches back (both
+    // GEMMs run after it), so they are read before the dependency wait; the
+    // expert outputs are read after it
     int p[MOE_MAX_K];
     float g[MOE_MAX_K];
-    int S = 1;
     if (t < Tn) {
-        S = (opart != nullptr && split2 != nullptr) ? *split2 : 1;
 #pragma unroll
         for (int j = 0; j < MOE_MAX_K; ++j) {
             if (j < k) {
@@ -92,20 +86,7 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const f
         for (int j = 0; j < MOE_MAX_K; ++j) {
             if (j < k && p[j] >= 0) {
                 float ov[VN];
-                if (S > 1) {
-#pragma unroll
-                    for (int e = 0; e < VN; ++e) ov[e] = 0.f;
-                    for (int sp = 0; sp < S; ++sp) {
-                        const float* src = opart + (size_t)sp * opart_stride + (size_t)p[j] * d + (size_t)v * VN;
-#pragma unroll
-                        for (int e = 0; e < VN; e += 4) {
-                            float4 q4 = *reinterpret_cast<const float4*>(src + e);
-                            ov[e] += q4.x; ov[e + 1] += q4.y; ov[e + 2] += q4.z; ov[e + 3] += q4.w;
-                        }
-                    }
-                } else {
-                    V::load(o + (size_t)p[j] * d + (size_t)v * VN, ov);
-                }
+                V::load(o + (size_t)p[j] * d + (size_t)v * VN, ov);
 #pragma unroll
                 for (int e = 0; e < VN; ++e) acc[e] = fmaf(g[j], ov[e], acc[e]);
             }
@@ -121,12 +102,11 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const f
 }
 
 cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const float* gate,
-                           const void* s, void* out, int T, int d, int k, cudaStream_t st,
-                           const float* opart, long long opart_stride, const int32_t* split2) {
+                           const void* s, void* out, int T, int d, int k, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int vn = dtype == MOE_DTYPE_BF16 ? 8 : 4;
-    // small batches: one vector per lane per warp, so the few rows (and their
-    // split-K partials) are spread over more warps
+    // small batches: one vector per lane per warp, so the few rows are spread
+    // over more warps
     const int vpl = T < 256 ? 1 : kCbVecPerLane;
     const int slices = ceil_div(d / vn, 32 * vpl);
     const long long tasks = (long long)T * slices;
@@ -134,53 +114,9 @@ cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const f
     if (dtype == MOE_DTYPE_BF16)
         return launch_k(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(kCbWarps * 32), 0, st,
                         (const __nv_bfloat16*)o, pos, gate, (const __nv_bfloat16*)s, (__nv_bfloat16*)out, T, d, k,
-                        opart, opart_stride, split2, slices, vpl);
+                        slices, vpl);
     return launch_k(combine_kernel<float>, dim3(grid), dim3(kCbWarps * 32), 0, st, (const float*)o, pos, gate,
-                    (const float*)s, (float*)out, T, d, k, (const float*)nullptr, 0LL, (const int32_t*)nullptr,
-                    slices, vpl);
-}
-
-// Split-K reduction of grouped GEMM 1/3: the partial rows hold, per 128
-// output columns, 128 gate sums followed by 128 up sums (the accumulator
-// layout of a SwiGLU tile). h[r][c] = SiLU(sum_s gate) * (sum_s up), summed
-// s = 0, 1, ... in order. One block per row; nothing to do when the split
-// factor chosen on the device is 1 (the GEMM then wrote h itself).
-__global__ void __launch_bounds__(256)
-swiglu_reduce_kernel(const float* __restrict__ part, long long split_stride, int ld,
-                     const int32_t* __restrict__ split13, const int32_t* __restrict__ indptr, int E, int d_ff,
-                     __nv_bfloat16* __restrict__ h) {
-    pdl_wait();
-    pdl_launch();
-    const int S = *split13;
-    if (S <= 1) return;
-    const int r = blockIdx.x;
-    if (r >= indptr[E]) return;
-    const int c = (blockIdx.y * blockDim.x + threadIdx.x) * 4;   // 4 columns inside one 128-column group
-    if (c >= d_ff) return;
-    const size_t col = (size_t)(c / 128) * 256 + (c % 128);
-    float4 g = make_float4(0.f, 0.f, 0.f, 0.f), u = g;
-    for (int sp = 0; sp < S; ++sp) {
-        const float* row = part + (size_t)sp * split_stride + (size_t)r * ld;
-        const float4 a = *reinterpret_cast<const float4*>(row + col);
-        const float4 b = *reinterpret_cast<const float4*>(row + col + 128);
-        g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
-        u.x += b.x; u.y += b.y; u.z += b.z; u.w += b.w;
-    }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(g.x / (1.f + __expf(-g.x)) * u.x, g.y / (1.f + __expf(-g.y)) * u.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(g.z / (1.f + __expf(-g.z)) * u.z, g.w / (1.f + __expf(-g.w)) * u.w);
-    uint2 packed;
-    packed.x = *reinterpret_cast<uint32_t*>(&lo);
-    packed.y = *reinterpret_cast<uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(h + (size_t)r * d_ff + c) = packed;
-}
-
-cudaError_t launch_swiglu_reduce(const float* part, long long split_stride, int ld, const int32_t* split13,
-                                 const int32_t* indptr, int E, int max_rows, int d_ff, void* h,
-                                 cudaStream_t st) {
-    if (max_rows <= 0) return cudaSuccess;
-    dim3 grid(max_rows, ceil_div(d_ff, 256 * 4));
-    return launch_k(swiglu_reduce_kernel, grid, dim3(256), 0, st, part, split_stride, ld, split13, indptr, E, d_ff,
-                    (__nv_bfloat16*)h);
+                    (const float*)s, (float*)out, T, d, k, slices, vpl);
 }
 
 }  // namespace moe

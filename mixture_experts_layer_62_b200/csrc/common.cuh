@@ -62,6 +62,8 @@ struct Layout {
     size_t blockcnt, blockoff, blockpsum, blockextra, tiles13, tiles2;
     size_t xp, h, o, hs, s;
     size_t part13, part2;   // fp32 split-K partials (small-T forward only)
+    size_t sem;             // split-K arrival counters: [sem13_n] then [sem2_n]
+    int sem13_n, sem2_n;
     size_t total;
 };
 
@@ -73,6 +75,25 @@ constexpr int kSplitMaxRows = 128;
 constexpr int kSplitMax = 16;
 bool split_allowed(const moe_problem& p);
 Layout make_layout(const moe_problem& p);
+
+// Split factors by the number of active experts (0 .. kSplitMaxRows): with at
+// most kSplitMaxRows rows every active expert is one M-block, so a GEMM has
+// n_active x (N-blocks) tiles and its factor is a function of n_active alone.
+// Filled on the host (pick_split), read by the kernel that writes the tile
+// schedule.
+struct SplitTable {
+    uint8_t s13[kSplitMaxRows + 1];
+    uint8_t s2[kSplitMaxRows + 1];
+};
+// Split factor of a GEMM with `tiles` output tiles of `nkb` K-blocks on `sm`
+// persistent CTAs: the s in [1, smax] that minimises rounds x (K-blocks per
+// unit + 1), ceil(tiles * s / sm) * (ceil(nkb / s) + 1); the + 1 charges each
+// unit one K-block of start/finish cost. The smaller s wins ties.
+int pick_split(int tiles, int nkb, int sm, int smax);
+void fill_split_table(SplitTable& t, int nt13, int nt2, int nkb13, int nkb2, int sm, int smax);
+// Arrival counters of the split-K GEMMs: one per (tile, quarter of the
+// 128-row M-block), zeroed by the kernel that writes the tile schedule.
+constexpr int kSemPerTile = 4;
 
 // Kernel launchers (each returns cudaGetLastError() of its launches).
 // status (may be null): the statistics' status word, reset to MOE_OK by the
@@ -105,7 +126,9 @@ struct ScanArgs {
     // tile schedules (null pointers: skipped)
     int32_t* tiles13; int32_t* tiles2;   // [G+2]: cumulative tiles, then the split factor
     int tile_m, ntiles13, ntiles2, ntiles13_shared, ntiles2_shared, has_shared;
-    int split_max, sm_count, nkb13, nkb2;   // split_max <= 1: no split
+    int split_on;                // 0: no split (factors 1)
+    int32_t* sem; int sem_n;     // split-K counters to zero (sem_n ints), or null
+    SplitTable split;
 };
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st);
 cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
@@ -116,13 +139,7 @@ cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
                                   int T, int d, int E, int k, int kk, int capacity,
                                   int32_t* pos, int32_t* row_token, void* xp, cudaStream_t st);
 cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const float* gate,
-                           const void* s, void* out, int T, int d, int k, cudaStream_t st,
-                           const float* opart = nullptr, long long opart_stride = 0,
-                           const int32_t* split2 = nullptr);
-// H = SiLU(sum_s gate partials) * (sum_s up partials) for the first indptr[E] rows.
-cudaError_t launch_swiglu_reduce(const float* part, long long split_stride, int ld, const int32_t* split13,
-                                 const int32_t* indptr, int E, int max_rows, int d_ff, void* h,
-                                 cudaStream_t st);
+                           const void* s, void* out, int T, int d, int k, cudaStream_t st);
 cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st);
 
 // Small-batch router (T*k <= kSmallMaxPairs, E <= kSmallMaxE, E % 8 == 0,
@@ -139,7 +156,9 @@ struct SmallRouteArgs {
     int32_t* status_reset;
     void* xp; void* stats;
     int32_t* tiles13; int32_t* tiles2;
-    int nt13, nt2, split_max, sm_count, nkb13, nkb2;
+    int nt13, nt2, split_on;
+    int32_t* sem; int sem_n;     // split-K counters to zero, or null
+    SplitTable split;
 };
 bool small_route_ok(const moe_problem& p);
 cudaError_t launch_route_small(const SmallRouteArgs& a, cudaStream_t st);
@@ -180,23 +199,13 @@ struct TcArgs {
     float* partial;            // split-K partials [split][rows][partial_ld] or null
     long long partial_stride;  // elements between splits
     int partial_ld;            // elements per row
+    int32_t* sem;              // split-K arrival counters [tiles][kSemPerTile] (with partial)
+    // the tile schedule (indptr, tiles) was written two or more launches
+    // back, so the weight loads of the first stages may start before the
+    // dependency wait
+    int b_before_wait;
 };
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
-
-// Split factor of a GEMM with `tiles` output tiles of `nkb` K-blocks on `sm`
-// persistent CTAs: the s in [1, smax] that minimises rounds x (K-blocks per
-// unit + 1), ceil(tiles * s / sm) * (ceil(nkb / s) + 1); the + 1 charges each
-// unit one K-block of start/finish cost. The smaller s wins ties.
-__device__ inline int pick_split(int tiles, int nkb, int sm, int smax) {
-    if (smax <= 1 || tiles <= 0 || sm <= 0) return 1;
-    long long best = -1;
-    int bs = 1;
-    for (int s = 1; s <= smax && s <= nkb; ++s) {
-        long long c = ((long long)tiles * s + sm - 1) / sm * ((nkb + s - 1) / s + 1);
-        if (best < 0 || c < best) { best = c; bs = s; }
-    }
-    return bs;
-}
 
 int device_sm_count();
 

@@ -158,6 +158,8 @@ struct KParams {
     float* partial;            // split-K partial rows, or null
     long long partial_stride;  // elements between splits
     int partial_ld;            // elements per partial row
+    int32_t* sem;              // split-K arrival counters [tile][kSemPerTile]
+    int b_before_wait;         // weight tiles of the first stages may load before the dependency wait
 };
 
 struct Tile {
@@ -232,6 +234,108 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// TMA coordinates of one unit's tiles: A rows of the group, and the two
+// 128-row halves of the B tile (W1 and W3 rows of the same output columns in
+// SWIGLU mode, 256 consecutive rows of one matrix otherwise).
+struct TileLoads {
+    const CUtensorMap *ma, *mlo, *mhi;
+    int arow, brow0, brow1;
+};
+template <int MODE>
+__device__ __forceinline__ TileLoads tile_loads(const KParams& p, const Tile& t, const CUtensorMap* tmA0,
+                                                const CUtensorMap* tmA1, const CUtensorMap* tmB00,
+                                                const CUtensorMap* tmB01, const CUtensorMap* tmB10,
+                                                const CUtensorMap* tmB11) {
+    TileLoads l;
+    l.ma = t.kind ? tmA1 : tmA0;
+    const CUtensorMap* mb0 = t.kind ? tmB10 : tmB00;
+    const CUtensorMap* mb1 = t.kind ? tmB11 : tmB01;
+    l.arow = t.row0 + t.m_blk * BM;
+    const int eoff = t.kind ? 0 : t.g * p.b_rows[0];
+    if (MODE == TC_SWIGLU) {
+        l.brow0 = eoff + t.n_blk * 128; l.brow1 = l.brow0; l.mlo = mb0; l.mhi = mb1;
+    } else {
+        l.brow0 = eoff + t.n_blk * 256; l.brow1 = l.brow0 + 128; l.mlo = mb0; l.mhi = mb0;
+    }
+    return l;
+}
+
+// Split-K finish of the 32 rows of quarter q of a tile. Every split's warp
+// writes its fp32 partial rows, then arrives on the (tile, quarter) counter;
+// the warp that arrives last sums the splits in the fixed order 0, 1, ...,
+// S-1 (so the result does not depend on which CTA came last) and writes the
+// output rows: SiLU(gate) * up in SWIGLU mode, the plain sum otherwise.
+// Lane l owns 4 (SWIGLU) or 8 (PLAIN) output columns of every row; two rows
+// and four splits are loaded per step so the L2 round trips overlap.
+template <int MODE>
+__device__ __forceinline__ void splitk_sum_rows(const KParams& p, const Tile& t, int lane, int nsplit, int r0,
+                                                int nrows) {
+    const int N = p.N[t.kind];
+    constexpr int CPL = MODE == TC_SWIGLU ? 4 : 8;   // output columns per lane
+    const int c = lane * CPL;
+    const int col = (MODE == TC_SWIGLU ? t.n_blk * 128 : t.n_blk * 256) + c;
+    if (col >= N) return;
+    // SWIGLU: gate sums at partial column c, up sums at c + 128;
+    // PLAIN: the 8 sums at c .. c + 7
+    const int off0 = c, off1 = MODE == TC_SWIGLU ? 128 + c : c + 4;
+    __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(p.out[t.kind]);
+#pragma unroll 1
+    for (int i = 0; i < nrows; i += 2) {
+        const int ib = i + 1 < nrows ? i + 1 : i;   // second row (a repeat of the first on an odd tail)
+        const size_t oa = static_cast<size_t>(t.row0) + static_cast<size_t>(r0 + i);
+        const size_t ob = static_cast<size_t>(t.row0) + static_cast<size_t>(r0 + ib);
+        const float* pa = p.partial + oa * p.partial_ld + static_cast<size_t>(t.n_blk) * 256;
+        const float* pb = p.partial + ob * p.partial_ld + static_cast<size_t>(t.n_blk) * 256;
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
+#pragma unroll 4
+        for (int sp = 0; sp < nsplit; ++sp) {
+            const size_t so = static_cast<size_t>(sp) * p.partial_stride;
+            const float4 x0 = __ldcg(reinterpret_cast<const float4*>(pa + so + off0));
+            const float4 x1 = __ldcg(reinterpret_cast<const float4*>(pa + so + off1));
+            const float4 y0 = __ldcg(reinterpret_cast<const float4*>(pb + so + off0));
+            const float4 y1 = __ldcg(reinterpret_cast<const float4*>(pb + so + off1));
+            a0.x += x0.x; a0.y += x0.y; a0.z += x0.z; a0.w += x0.w;
+            a1.x += x1.x; a1.y += x1.y; a1.z += x1.z; a1.w += x1.w;
+            b0.x += y0.x; b0.y += y0.y; b0.z += y0.z; b0.w += y0.w;
+            b1.x += y1.x; b1.y += y1.y; b1.z += y1.z; b1.w += y1.w;
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            if (r == 1 && ib == i) break;
+            const float4 g = r ? b0 : a0, v = r ? b1 : a1;
+            const size_t orow = r ? ob : oa;
+            if (MODE == TC_SWIGLU) {
+                uint2 packed;
+                packed.x = pack_bf16(silu(g.x) * v.x, silu(g.y) * v.y);
+                packed.y = pack_bf16(silu(g.z) * v.z, silu(g.w) * v.w);
+                *reinterpret_cast<uint2*>(outp + orow * N + col) = packed;
+            } else {
+                *reinterpret_cast<uint4*>(outp + orow * N + col) =
+                    make_uint4(pack_bf16(g.x, g.y), pack_bf16(g.z, g.w), pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+            }
+        }
+    }
+}
+
+template <int MODE>
+__device__ __noinline__ void splitk_finish(const KParams& p, const Tile& t, int q, int lane, int nsplit, int tile) {
+    int32_t* cnt = p.sem + static_cast<size_t>(tile) * kSemPerTile + q;
+    __syncwarp();   // every lane's partial stores precede lane 0's release below
+    int old = 0;
+    if (lane == 0) {
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");   // release the warp's partial rows
+        old = atomicAdd(cnt, 1);
+        if (old == nsplit - 1) {
+            *cnt = 0;   // ready for the next pass (the schedule writer zeroes it too)
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");   // acquire the other splits' rows
+        }
+    }
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != nsplit - 1) return;
+    const int r0 = t.m_blk * BM + q * 32;
+    splitk_sum_rows<MODE>(p, t, lane, nsplit, r0, min(32, t.rows - r0));
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -269,10 +373,16 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
-    // everything above (barriers, TMEM, descriptor prefetch) overlapped the
-    // previous kernel; the schedule and the A rows are its outputs
-    pdl_wait();
-    pdl_launch();
+    // Everything above (barriers, TMEM, descriptor prefetch) overlapped the
+    // previous kernel. The A rows are always an output of the previous
+    // kernel; the schedule is one too unless b_before_wait says it was
+    // written earlier, in which case the schedule is read and the first
+    // stages' weight tiles are requested before the wait.
+    const bool early = p.b_before_wait != 0;
+    if (!early) {
+        pdl_wait();
+        pdl_launch();
+    }
     const int total = total_tiles(p, COLS_PER_TILE);
     // split-K: the device-chosen factor is stored after the tile schedule;
     // unit u covers tile u / nsplit and the K-blocks of split u % nsplit, so
@@ -288,29 +398,42 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             uint32_t ph = 0;
             uint32_t issued_mask = 0, issued_ph = 0;
             bool aborted = false;
+            int pre = 0;   // stages of the first unit whose weight tiles were requested before the wait
+            if (early) {
+                if (static_cast<int>(blockIdx.x) < units) {
+                    const int sp = blockIdx.x % nsplit;
+                    const Tile t = decode_tile(p, blockIdx.x / nsplit);
+                    const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
+                    const TileLoads l = tile_loads<MODE>(p, t, &tmA0, &tmA1, &tmB00, &tmB01, &tmB10, &tmB11);
+                    for (int kb = kb0; kb < kb1 && pre < STAGES; ++kb, ++pre) {
+                        // every stage is free at the start: no empty-barrier wait
+                        const uint32_t sa = smem_u32(smem + pre * STAGE_BYTES);
+                        mbar_arrive_expect_tx(&ctl->full[pre], STAGE_BYTES);
+                        tma_load_2d(sa + A_BYTES, l.mlo, &ctl->full[pre], kb * BK, l.brow0);
+                        tma_load_2d(sa + A_BYTES + B_HALF_BYTES, l.mhi, &ctl->full[pre], kb * BK, l.brow1);
+                        issued_mask |= 1u << pre;
+                    }
+                }
+                pdl_wait();
+                pdl_launch();
+            }
             for (int u = blockIdx.x; u < units && !aborted; u += gridDim.x) {
                 const int sp = u % nsplit;
                 const Tile t = decode_tile(p, u / nsplit);
                 const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
-                const CUtensorMap* ma = t.kind ? &tmA1 : &tmA0;
-                const CUtensorMap* mb0 = t.kind ? &tmB10 : &tmB00;
-                const CUtensorMap* mb1 = t.kind ? &tmB11 : &tmB01;
-                const int arow = t.row0 + t.m_blk * BM;
-                const int eoff = t.kind ? 0 : t.g * p.b_rows[0];
-                int brow0, brow1;
-                const CUtensorMap *mlo, *mhi;
-                if (MODE == TC_SWIGLU) {
-                    brow0 = eoff + t.n_blk * 128; brow1 = brow0; mlo = mb0; mhi = mb1;
-                } else {
-                    brow0 = eoff + t.n_blk * 256; brow1 = brow0 + 128; mlo = mb0; mhi = mb0;
-                }
+                const TileLoads l = tile_loads<MODE>(p, t, &tmA0, &tmA1, &tmB00, &tmB01, &tmB10, &tmB11);
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!wait_bounded(&ctl->empty[s], ph ^ 1u, ctl, p)) { aborted = true; break; }
                     const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-                    mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
-                    tma_load_2d(sa, ma, &ctl->full[s], kb * BK, arow);
-                    tma_load_2d(sa + A_BYTES, mlo, &ctl->full[s], kb * BK, brow0);
-                    tma_load_2d(sa + A_BYTES + B_HALF_BYTES, mhi, &ctl->full[s], kb * BK, brow1);
+                    if (u == static_cast<int>(blockIdx.x) && kb - kb0 < pre) {
+                        // weights already requested: the A rows complete the stage
+                        tma_load_2d(sa, l.ma, &ctl->full[s], kb * BK, l.arow);
+                    } else {
+                        if (!wait_bounded(&ctl->empty[s], ph ^ 1u, ctl, p)) { aborted = true; break; }
+                        mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
+                        tma_load_2d(sa, l.ma, &ctl->full[s], kb * BK, l.arow);
+                        tma_load_2d(sa + A_BYTES, l.mlo, &ctl->full[s], kb * BK, l.brow0);
+                        tma_load_2d(sa + A_BYTES + B_HALF_BYTES, l.mhi, &ctl->full[s], kb * BK, l.brow1);
+                    }
                     issued_mask |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -318,12 +441,21 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             }
             if (aborted) {
                 // let every load this thread started land before the CTA exits
+                // (the stages requested before the wait got their A rows before
+                // any wait could give up, so their barriers complete too)
                 for (int st = 0; st < STAGES; ++st)
                     if ((issued_mask >> st) & 1u) wait_drain(&ctl->full[st], (issued_ph >> st) & 1u, p);
             }
+        } else if (early) {
+            pdl_wait();
+            pdl_launch();
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
+        if (early) {
+            pdl_wait();
+            pdl_launch();
+        }
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc(BM, 256);
             int s = 0;
@@ -364,6 +496,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
         }
     } else {
         // ---------------- epilogue (warps 2..5) ----------------
+        if (early) {
+            pdl_wait();
+            pdl_launch();
+        }
         const int q = warp & 3;                 // TMEM lane quarter of this warp
         const int r = q * 32 + lane;            // accumulator row of this thread
         int acc = 0;
@@ -379,7 +515,8 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             const int N = p.N[t.kind];
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                 static_cast<uint32_t>(acc * ACC_COLS);
-            if (nsplit > 1) {
+            bool released = false;
+            if (MODE != TC_F32OUT && nsplit > 1) {
                 // fp32 partial of this split: the raw 256 accumulator columns
                 float* out = p.partial + static_cast<size_t>(sp) * p.partial_stride + orow * p.partial_ld;
 #pragma unroll 1
@@ -394,6 +531,12 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                             dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                     }
                 }
+                // the accumulator is free as soon as it is read
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+                released = true;
+                if (t.m_blk * BM + q * 32 < t.rows) splitk_finish<MODE>(p, t, q, lane, nsplit, u / nsplit);
             } else if (MODE == TC_SWIGLU) {
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
 #pragma unroll 1
@@ -449,9 +592,11 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+            if (!released) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->tempty[acc]);
+            }
             acc ^= 1;
             if (acc == 0) aph ^= 1u;
         }
@@ -588,6 +733,9 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     kp.partial = a.partial;
     kp.partial_stride = a.partial_stride;
     kp.partial_ld = a.partial_ld;
+    kp.sem = a.sem;
+    kp.b_before_wait = a.b_before_wait;
+    if (kp.partial != nullptr && kp.sem == nullptr) return cudaErrorInvalidValue;
     switch (a.mode) {
         case TC_SWIGLU: return launch_mode<TC_SWIGLU>(a, kp, maps, st);
         case TC_PLAIN: return launch_mode<TC_PLAIN>(a, kp, maps, st);

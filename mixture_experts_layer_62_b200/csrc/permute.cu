@@ -62,7 +62,7 @@ __device__ void build_schedule(const int* rows, int G, int E, int tile_m, int nt
     if (threadIdx.x == 0) tiles[G] = carry;
 }
 
-__global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) {
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(const __grid_constant__ ScanArgs a, int NB) {
     __shared__ int warp_tot[33];
     __shared__ int start[MOE_MAX_E + 1];
     __shared__ int kept_s[MOE_MAX_E + 1];
@@ -198,10 +198,17 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(ScanArgs a, int NB) 
         build_schedule(rows, G, E, a.tile_m, a.ntiles13, a.ntiles13_shared, a.tiles13, warp_tot);
         __syncthreads();
         build_schedule(rows, G, E, a.tile_m, a.ntiles2, a.ntiles2_shared, a.tiles2, warp_tot);
+        // split factors: with split-K on, every active expert is one M-block,
+        // so the host-built table indexed by the active-expert count applies
+        int n_active;
+        block_exclusive_scan(threadIdx.x < E && kept_s[threadIdx.x] > 0 ? 1 : 0, warp_tot, n_active);
         if (threadIdx.x == 0) {
-            a.tiles13[G + 1] = pick_split(a.tiles13[G], a.nkb13, a.sm_count, a.split_max);
-            a.tiles2[G + 1] = pick_split(a.tiles2[G], a.nkb2, a.sm_count, a.split_max);
+            const int n = n_active < kSplitMaxRows ? n_active : kSplitMaxRows;
+            a.tiles13[G + 1] = a.split_on ? a.split.s13[n] : 1;
+            a.tiles2[G + 1] = a.split_on ? a.split.s2[n] : 1;
         }
+        // split-K arrival counters start at zero on every pass
+        for (int i = threadIdx.x; i < a.sem_n; i += blockDim.x) a.sem[i] = 0;
     }
 }
 

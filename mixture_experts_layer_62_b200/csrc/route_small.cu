@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kPartWarps * 32) route_logits_kernel(SmallRout
 // indptr, the statistics and the tile schedules with their split factors.
 constexpr int kFinWarps = 16;
 
-__global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRouteArgs a, int P) {
+__global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(const __grid_constant__ SmallRouteArgs a, int P) {
     __shared__ float z[kSmallMaxPairs][kSmallMaxE];
     __shared__ float psw[kFinWarps][kSmallMaxE];
     __shared__ int sidx[kSmallMaxPairs];
@@ -107,6 +107,8 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
     __shared__ int indptr_s[kSmallMaxE + 1];
     __shared__ float bias_s[kSmallMaxE];
     __shared__ float extw[kFinWarps][3];
+    __shared__ float zsel_s[kFinWarps][MOE_MAX_K];
+    __shared__ int esel_s[kFinWarps][MOE_MAX_K];
     const int T = a.T, E = a.E, k = a.k;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool writer = blockIdx.x == 0;
@@ -130,6 +132,8 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
     }
     pdl_wait();
     pdl_launch();
+    if (writer)   // split-K arrival counters start at zero on every pass
+        for (int i = threadIdx.x; i < a.sem_n; i += blockDim.x) a.sem[i] = 0;
     for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
         const int t = i / E, e = i % E;
         float pv[kSmallMaxParts];
@@ -195,50 +199,50 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
             if (e < E) psw[warp][e] += p;
             key[i] = a.bias_mode == MOE_BIAS_NONE ? zz[i] : a.bias_mode == MOE_BIAS_LOGIT ? zz[i] + b : p + b;
         }
+        // k rounds of a warp arg-max (the lowest index wins ties); the selected
+        // logits and experts go to shared memory, lane j then finishes slot j
         unsigned taken = 0;
-        float zsel[MOE_MAX_K];
-        int esel[MOE_MAX_K];
+#pragma unroll 1
+        for (int j = 0; j < k; ++j) {
+            float bk = -INFINITY, bz = 0.f;
+            int be = 0x7fffffff;
 #pragma unroll
-        for (int j = 0; j < MOE_MAX_K; ++j) {
-            if (j < k) {
-                float bk = -INFINITY, bz = 0.f;
-                int be = 0x7fffffff;
+            for (int i = 0; i < 2; ++i) {
+                const bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
+                if (ok && (key[i] > bk || be == 0x7fffffff)) { bk = key[i]; be = lane + 32 * i; bz = zz[i]; }
+            }
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
-                    if (ok && (key[i] > bk || be == 0x7fffffff)) { bk = key[i]; be = lane + 32 * i; bz = zz[i]; }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-                    const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
-                    if (better) { bk = ok_; be = oe; bz = oz; }
-                }
-                if ((be & 31) == lane) taken |= 1u << (be >> 5);
-                zsel[j] = bz;
-                esel[j] = be;
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+                const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
+                if (better) { bk = ok_; be = oe; bz = oz; }
+            }
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            if (lane == 0) {
+                zsel_s[warp][j] = bz;
+                esel_s[warp][j] = be;
             }
         }
-        float zm = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) zm = fmaxf(zm, zsel[j]);
-        float gs = 0.f, ge[MOE_MAX_K];
-#pragma unroll
-        for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
-        const float inv_g = 1.f / gs;
-#pragma unroll
-        for (int j = 0; j < MOE_MAX_K; ++j) {
-            if (j < k && lane == j) {
-                sidx[t * k + j] = esel[j];
-                if (writer) {
-                    a.idx[(size_t)t * k + j] = esel[j];
-                    a.gate[(size_t)t * k + j] =
-                        a.gate_mode == MOE_GATE_FULL ? expf(zsel[j] - m) * inv_s : ge[j] * inv_g;
-                }
+        __syncwarp();
+        if (lane < k) {
+            // gates: softmax over the k selected raw logits, summed in slot order
+            float zm = -INFINITY;
+            for (int j = 0; j < k; ++j) zm = fmaxf(zm, zsel_s[warp][j]);
+            float gs = 0.f;
+            for (int j = 0; j < k; ++j) gs += expf(zsel_s[warp][j] - zm);
+            const float inv_g = 1.f / gs;
+            const float zj = zsel_s[warp][lane];
+            const int ej = esel_s[warp][lane];
+            sidx[t * k + lane] = ej;
+            if (writer) {
+                a.idx[(size_t)t * k + lane] = ej;
+                a.gate[(size_t)t * k + lane] =
+                    a.gate_mode == MOE_GATE_FULL ? expf(zj - m) * inv_s : expf(zj - zm) * inv_g;
             }
         }
+        __syncwarp();
     }
     if (lane == 0) {
         extw[warp][0] = ex_z;
@@ -313,6 +317,9 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
                 run13 += __shfl_sync(0xffffffffu, i13, 31);
                 run2 += __shfl_sync(0xffffffffu, i2, 31);
             }
+            // active experts (<= 64 here) index the host-built split table
+            const int n_active = __popc(__ballot_sync(0xffffffffu, kp[0] > 0)) +
+                                 __popc(__ballot_sync(0xffffffffu, kp[1] > 0));
             int maxc = max(c[0], c[1]);
             int drop = (c[0] - kp[0]) + (c[1] - kp[1]);
 #pragma unroll
@@ -324,8 +331,8 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(SmallRoute
                 a.indptr[E] = run;
                 a.tiles13[E] = run13;
                 a.tiles2[E] = run2;
-                a.tiles13[E + 1] = pick_split(run13, a.nkb13, a.sm_count, a.split_max);
-                a.tiles2[E + 1] = pick_split(run2, a.nkb2, a.sm_count, a.split_max);
+                a.tiles13[E + 1] = a.split_on ? a.split.s13[n_active] : 1;
+                a.tiles2[E + 1] = a.split_on ? a.split.s2[n_active] : 1;
                 moe_stats* st = static_cast<moe_stats*>(a.stats);
                 st->capacity = a.capacity;
                 st->rows = run;
