@@ -53,12 +53,18 @@ Layout make_layout(const moe_problem& p) {
     return L;
 }
 
-int pick_split(int tiles, int nkb, int sm, int smax) {
+int pick_split(int tiles, int nkb, int sm, int smax, int rows_q) {
     if (smax <= 1 || tiles <= 0 || sm <= 0) return 1;
+    // a split unit costs at least the split epilogue (partial rows out, the
+    // arrival, and for the last split the sum over all splits), charged in
+    // K-blocks: 12 plus 2.5 per row of the busiest 32-row quarter
+    const int epi = 12 + (5 * (rows_q < 32 ? rows_q : 32) + 1) / 2;
     long long best = -1;
     int bs = 1;
     for (int s = 1; s <= smax && s <= nkb; ++s) {
-        const long long c = ((long long)tiles * s + sm - 1) / sm * ((nkb + s - 1) / s + 1);
+        int unit = (nkb + s - 1) / s + 1;
+        if (s > 1 && unit < epi) unit = epi;
+        const long long c = ((long long)tiles * s + sm - 1) / sm * unit;
         if (best < 0 || c < best) {
             best = c;
             bs = s;
@@ -67,19 +73,21 @@ int pick_split(int tiles, int nkb, int sm, int smax) {
     return bs;
 }
 
-void fill_split_table(SplitTable& t, int nt13, int nt2, int nkb13, int nkb2, int sm, int smax) {
-    // the table depends on six integers; reuse the last one this thread built
-    static thread_local int key[6] = {-1, -1, -1, -1, -1, -1};
+void fill_split_table(SplitTable& t, int nt13, int nt2, int nkb13, int nkb2, int sm, int smax, int rows) {
+    // the table depends on seven integers; reuse the last one this thread built
+    static thread_local int key[7] = {-1, -1, -1, -1, -1, -1, -1};
     static thread_local SplitTable last;
-    const int k6[6] = {nt13, nt2, nkb13, nkb2, sm, smax};
+    const int k7[7] = {nt13, nt2, nkb13, nkb2, sm, smax, rows};
     bool hit = true;
-    for (int i = 0; i < 6; ++i) hit = hit && key[i] == k6[i];
+    for (int i = 0; i < 7; ++i) hit = hit && key[i] == k7[i];
     if (!hit) {
         for (int n = 0; n <= kSplitMaxRows; ++n) {
-            last.s13[n] = (uint8_t)pick_split(n * nt13, nkb13, sm, smax);
-            last.s2[n] = (uint8_t)pick_split(n * nt2, nkb2, sm, smax);
+            // rows of the busiest expert, estimated as 1.5 x the mean
+            const int rq = n > 0 ? (3 * rows + 2 * n - 1) / (2 * n) : 0;
+            last.s13[n] = (uint8_t)pick_split(n * nt13, nkb13, sm, smax, rq);
+            last.s2[n] = (uint8_t)pick_split(n * nt2, nkb2, sm, smax, rq);
         }
-        for (int i = 0; i < 6; ++i) key[i] = k6[i];
+        for (int i = 0; i < 7; ++i) key[i] = k7[i];
     }
     t = last;
 }
@@ -287,6 +295,31 @@ void schedule_sizes(const moe_problem* p, int& tile_m, int& nt13, int& nt2, int&
     }
 }
 
+// Split-K state of the expert stages: factors, partial buffers, counters.
+struct StageSplit {
+    ScheduleSplit sched = {};
+    float* part13 = nullptr;
+    float* part2 = nullptr;
+    int32_t* sem13 = nullptr;
+    int32_t* sem2 = nullptr;
+};
+StageSplit stage_split(const moe_problem* p, const Layout& L, void* ws) {
+    StageSplit s;
+    if (!split_allowed(*p)) return s;
+    int tile_m, nt13, nt2, nt13s, nt2s;
+    schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
+    s.sched.split_on = 1;
+    s.sem13 = reinterpret_cast<int32_t*>(wsp(ws, L.sem));
+    s.sem2 = s.sem13 + L.sem13_n;
+    s.sched.sem = s.sem13;
+    s.sched.sem_n = L.sem13_n + L.sem2_n;
+    fill_split_table(s.sched.split, nt13, nt2, ceil_div(p->d, 64), ceil_div(p->d_ff, 64), device_sm_count(),
+                     kSplitMax, p->T * p->k);
+    s.part13 = reinterpret_cast<float*>(wsp(ws, L.part13));
+    s.part2 = reinterpret_cast<float*>(wsp(ws, L.part2));
+    return s;
+}
+
 }  // namespace
 
 extern "C" {
@@ -384,7 +417,7 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
             sr.sem = sem;
             sr.sem_n = L.sem13_n + L.sem2_n;
             fill_split_table(sr.split, sr.nt13, sr.nt2, ceil_div(p->d, 64), ceil_div(p->d_ff, 64),
-                             device_sm_count(), kSplitMax);
+                             device_sm_count(), kSplitMax, p->T * p->k);
         }
         CK(launch_route_small(sr, st));
     } else {
@@ -405,7 +438,7 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
         sa.sem = sem;
         sa.sem_n = L.sem13_n + L.sem2_n;
         fill_split_table(sa.split, sa.ntiles13, sa.ntiles2, ceil_div(p->d, 64), ceil_div(p->d_ff, 64),
-                         device_sm_count(), kSplitMax);
+                         device_sm_count(), kSplitMax, p->T * p->k);
     }
     CK(launch_scan(sa, st));
     CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, kk, C, pos, row_token, xp,
@@ -555,10 +588,13 @@ int moe_experts(const moe_problem* p, const void* xp, const int32_t* indptr, con
     int32_t* tiles2 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles2));
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
-    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2, st));
+    const StageSplit sp = stage_split(p, L, workspace);
+    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2,
+                       sp.sched, st));
     void* h = wsp(workspace, L.h);
     void* hs = shared ? wsp(workspace, L.hs) : nullptr;
-    return run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st);
+    return run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st,
+                       sp.part13, sp.part2, sp.sem13, sp.sem2);
 }
 
 // Shared prologue of the expert-stage entry points: checks, status reset and
@@ -595,8 +631,11 @@ int moe_expert_up(const moe_problem* p, const void* xp, const int32_t* indptr, c
     CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
-    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2, st));
-    return run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, shared ? hs : nullptr, status, st);
+    const StageSplit sp = stage_split(p, make_layout(*p), workspace);
+    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2,
+                       sp.sched, st));
+    return run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, shared ? hs : nullptr, status, st, sp.part13,
+                  sp.sem13);
 }
 
 int moe_expert_down(const moe_problem* p, const void* h, const int32_t* indptr, const void* W2, const void* hs,
@@ -620,8 +659,11 @@ int moe_expert_down(const moe_problem* p, const void* h, const int32_t* indptr, 
     CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
-    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2, st));
-    return run_down(p, h, indptr, tiles2, W2, shared ? hs : nullptr, Ws2, o, shared ? s : nullptr, status, st);
+    const StageSplit sp = stage_split(p, make_layout(*p), workspace);
+    CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2,
+                       sp.sched, st));
+    return run_down(p, h, indptr, tiles2, W2, shared ? hs : nullptr, Ws2, o, shared ? s : nullptr, status, st,
+                    sp.part2, sp.sem2);
 }
 
 int moe_combine(const moe_problem* p, const void* o, const int32_t* pos, const float* gate, const void* s, void* out,

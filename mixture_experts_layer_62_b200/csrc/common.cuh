@@ -86,11 +86,14 @@ struct SplitTable {
     uint8_t s2[kSplitMaxRows + 1];
 };
 // Split factor of a GEMM with `tiles` output tiles of `nkb` K-blocks on `sm`
-// persistent CTAs: the s in [1, smax] that minimises rounds x (K-blocks per
-// unit + 1), ceil(tiles * s / sm) * (ceil(nkb / s) + 1); the + 1 charges each
-// unit one K-block of start/finish cost. The smaller s wins ties.
-int pick_split(int tiles, int nkb, int sm, int smax);
-void fill_split_table(SplitTable& t, int nt13, int nt2, int nkb13, int nkb2, int sm, int smax);
+// persistent CTAs: the s in [1, smax] that minimises rounds x unit cost,
+// ceil(tiles * s / sm) * u(s), u(s) = ceil(nkb / s) + 1 K-blocks (the + 1 is
+// each unit's pipeline start/finish), and for s > 1 at least the split
+// epilogue's cost, which grows with the rows of the busiest expert (rows_q).
+// The smaller s wins ties.
+int pick_split(int tiles, int nkb, int sm, int smax, int rows_q);
+// rows: T*k, the permuted rows of the pass
+void fill_split_table(SplitTable& t, int nt13, int nt2, int nkb13, int nkb2, int sm, int smax, int rows);
 // Arrival counters of the split-K GEMMs: one per (tile, quarter of the
 // 128-row M-block), zeroed by the kernel that writes the tile schedule.
 constexpr int kSemPerTile = 4;
@@ -131,9 +134,16 @@ struct ScanArgs {
     SplitTable split;
 };
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st);
+// Split-K setup of a tile schedule: factors by active-expert count and the
+// counters to zero.
+struct ScheduleSplit {
+    int split_on;
+    int32_t* sem; int sem_n;
+    SplitTable split;
+};
 cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
                             int ntiles13, int ntiles2, int ntiles13_shared, int ntiles2_shared,
-                            int32_t* tiles13, int32_t* tiles2, cudaStream_t st);
+                            int32_t* tiles13, int32_t* tiles2, const ScheduleSplit& sp, cudaStream_t st);
 cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
                                   const int32_t* blockoff, const int32_t* indptr,
                                   int T, int d, int E, int k, int kk, int capacity,

@@ -217,10 +217,12 @@ cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st) {
     return launch_k(scan_kernel, dim3(1), dim3(kScanThreads), 0, st, a, NB);
 }
 
-// Tile schedule from a given indptr (the standalone expert stage).
+// Tile schedule from a given indptr (the standalone expert stages), with the
+// same split factors and counter reset as the scan of the forward pass.
 __global__ void __launch_bounds__(kScanThreads)
 schedule_kernel(const int32_t* __restrict__ indptr, int E, int T, int has_shared, int tile_m,
-                int nt13, int nt2, int nt13s, int nt2s, int32_t* tiles13, int32_t* tiles2) {
+                int nt13, int nt2, int nt13s, int nt2s, int32_t* tiles13, int32_t* tiles2,
+                const __grid_constant__ ScheduleSplit sp) {
     __shared__ int warp_tot[33];
     __shared__ int rows[MOE_MAX_E + 1];
     pdl_wait();
@@ -232,17 +234,21 @@ schedule_kernel(const int32_t* __restrict__ indptr, int E, int T, int has_shared
     build_schedule(rows, G, E, tile_m, nt13, nt13s, tiles13, warp_tot);
     __syncthreads();
     build_schedule(rows, G, E, tile_m, nt2, nt2s, tiles2, warp_tot);
-    if (threadIdx.x == 0) {   // the stage entry points never split K
-        tiles13[G + 1] = 1;
-        tiles2[G + 1] = 1;
+    int n_active;
+    block_exclusive_scan(threadIdx.x < E && rows[threadIdx.x] > 0 ? 1 : 0, warp_tot, n_active);
+    if (threadIdx.x == 0) {
+        const int n = n_active < kSplitMaxRows ? n_active : kSplitMaxRows;
+        tiles13[G + 1] = sp.split_on ? sp.split.s13[n] : 1;
+        tiles2[G + 1] = sp.split_on ? sp.split.s2[n] : 1;
     }
+    for (int i = threadIdx.x; i < sp.sem_n; i += blockDim.x) sp.sem[i] = 0;
 }
 
 cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
                             int ntiles13, int ntiles2, int ntiles13_shared, int ntiles2_shared,
-                            int32_t* tiles13, int32_t* tiles2, cudaStream_t st) {
+                            int32_t* tiles13, int32_t* tiles2, const ScheduleSplit& sp, cudaStream_t st) {
     return launch_k(schedule_kernel, dim3(1), dim3(kScanThreads), 0, st, indptr, E, T, has_shared, tile_m, ntiles13,
-                    ntiles2, ntiles13_shared, ntiles2_shared, tiles13, tiles2);
+                    ntiles2, ntiles13_shared, ntiles2_shared, tiles13, tiles2, sp);
 }
 
 // Ranks, destinations and the row gather. Block (chunk, column group): every

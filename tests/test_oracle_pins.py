@@ -496,3 +496,19 @@ def test_planted_missing_shared_expert_is_caught():
     b = brute_forward(x, W_r, W1, W3, W2, k=2, **sh)
     res = O.moe_forward(x, W_r, W1, W3, W2, k=2)   # shared expert left out
     assert not np.allclose(res.y, b["y"], rtol=1e-6)
+
+
+def test_planted_slot_order_ignored_is_caught(monkeypatch):
+    idx = np.array([[0, 1], [1, 0], [0, 1]])
+    orig = O.permute
+    monkeypatch.setattr(O, "permute", lambda idx_, E, C, drop_order=O.DROP_TOKEN: orig(idx_, E, C, O.DROP_TOKEN))
+    assert O.permute(idx, 2, 2, O.DROP_SLOT).pos.tolist() != [[0, 3], [2, -1], [1, -1]]
+
+
+def test_planted_unsquared_z_loss_is_caught(monkeypatch):
+    def wrong(z):
+        z = np.asarray(z, dtype=np.float64)
+        m = z.max(axis=1, keepdims=True)
+        return float(np.mean(m[:, 0] + np.log(np.exp(z - m).sum(axis=1))))
+    monkeypatch.setattr(O, "router_z_loss", wrong)
+    assert O.router_z_loss(np.zeros((5, 8))) != pytest.approx(math.log(8) ** 2, rel=1e-14)
