@@ -199,7 +199,7 @@ class Permutation:
     rank: np.ndarray       # [T, k] int64 rank of the pair inside its expert
 
 
-def permute(idx, E, C=None, drop_order=DROP_TOKEN):
+def permute(idx, E, C=None, drop_order=DROP_TOKEN, pad=None):
     """Permutation indices by prefix sum, with capacity truncation.
 
     [CMU 15-779 L21] §3.3: build the N x E 0/1 selection mask, flatten it
@@ -218,6 +218,11 @@ def permute(idx, E, C=None, drop_order=DROP_TOKEN):
     sum): the mask gets a slot axis, [k, N, E] with mask[j, t, e] = 1 iff
     idx[t, j] = e, and is flattened expert-major as (e, j, t), so inside an
     expert the pairs are ordered by slot, then token.
+
+    pad = P (MegaBlocks, [CMU 15-779 L21] §3.6: every expert's row count is
+    padded to a multiple of the block size inside the permutation): the
+    indptr is the prefix sum of ceil(kept_e / P) * P; the padding rows follow
+    each expert's kept rows and belong to no token (row_token -1).
     """
     idx = np.asarray(idx, dtype=np.int64)
     T, k = idx.shape
@@ -250,7 +255,8 @@ def permute(idx, E, C=None, drop_order=DROP_TOKEN):
 
     kept = counts.copy() if C is None else np.minimum(counts, C)
     indptr = np.zeros(E + 1, dtype=np.int64)
-    indptr[1:] = np.cumsum(kept)
+    rows_e = kept if not pad else -(-kept // pad) * pad
+    indptr[1:] = np.cumsum(rows_e)
 
     pos = np.full((T, k), -1, dtype=np.int64)
     rank = np.zeros((T, k), dtype=np.int64)
@@ -276,6 +282,28 @@ def permute(idx, E, C=None, drop_order=DROP_TOKEN):
 # --------------------------------------------------------------------------
 # Experts
 # --------------------------------------------------------------------------
+
+def block_sparse_topology(rows_per_expert, block, blocks_per_expert):
+    """Block-sparse metadata of the padded expert matrix (MegaBlocks,
+    [CMU 15-779 L21] §3.6, Figure 5): the rows of expert e, padded to a
+    multiple of ``block``, form block rows that are nonzero exactly in the
+    expert's own ``blocks_per_expert`` block columns. Nonzero blocks are
+    numbered row-major. Returns (BCSR row offsets, column index of every
+    block, row index of every block (the COO part), transpose index: the
+    block numbers listed column by column, rows ascending).
+    """
+    rows = np.asarray(rows_per_expert, dtype=np.int64)
+    brows_e = -(-rows // block)                     # block rows per expert
+    row_expert = np.repeat(np.arange(len(rows)), brows_e)
+    nbr = int(brows_e.sum())
+    offsets = np.arange(nbr + 1, dtype=np.int64) * blocks_per_expert
+    col = np.concatenate([row_expert[r] * blocks_per_expert + np.arange(blocks_per_expert)
+                          for r in range(nbr)]) if nbr else np.zeros(0, dtype=np.int64)
+    row = np.repeat(np.arange(nbr), blocks_per_expert)
+    # column-major listing: stable sort of the blocks by column
+    transpose = np.argsort(col, kind="stable")
+    return offsets, col.astype(np.int64), row.astype(np.int64), transpose.astype(np.int64)
+
 
 def silu(a):
     """SiLU(a) = a * sigmoid(a) (the gate of SwiGLU)."""
@@ -398,7 +426,7 @@ class ForwardResult:
 def moe_forward(x, W_r, W1, W3, W2, k, capacity_factor=0.0, bias=None,
                 bias_mode=BIAS_NONE, Ws1=None, Ws3=None, Ws2=None,
                 logits=None, tokens=None, key_dtype=np.float64,
-                gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN):
+                gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN, pad=None):
     """Forward pass of one MoE layer, the sparse per-pair definition.
 
     Steps in the order of [CMU 15-779 L21] §3.2 (route, permute, compute per
@@ -432,7 +460,7 @@ def moe_forward(x, W_r, W1, W3, W2, k, capacity_factor=0.0, bias=None,
     routing = Routing(idx=idx, gate=gate, probs=probs, key=key)
 
     C = capacity(capacity_factor, T, k, E)
-    perm = permute(idx, E, C, drop_order)
+    perm = permute(idx, E, C, drop_order, pad)
     stats = load_stats(perm, probs, T, k, C, z=z)
 
     if tokens is None:

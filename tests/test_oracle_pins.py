@@ -411,6 +411,40 @@ def test_drop_orders_agree_without_capacity_and_for_top1():
     assert np.array_equal(O.permute(idx1, 8, 20, O.DROP_TOKEN).pos, O.permute(idx1, 8, 20, O.DROP_SLOT).pos)
 
 
+def test_megablocks_figure5_topology():
+    g = load("megablocks_figure5.txt")
+    off, col, row, tr = O.block_sparse_topology(g["rows"], g["block"], g["blocks_per_expert"])
+    assert off.tolist() == g["offsets"].tolist()
+    assert col.tolist() == g["col"].tolist()
+    assert row.tolist() == g["row"].tolist()
+    assert tr.tolist() == g["transpose"].tolist()
+
+
+def test_padded_permutation_follows_figure5_rows():
+    # one pick per token so that the experts get the figure's 3 / 1 / 6 rows;
+    # padded to blocks of 2 they hold 4 / 2 / 6 rows, the figure's 6 block rows
+    g = load("megablocks_figure5.txt")
+    idx = np.array([[0], [2], [0], [2], [1], [2], [0], [2], [2], [2]])
+    perm = O.permute(idx, 3, None, O.DROP_TOKEN, pad=g["block"])
+    assert perm.kept.tolist() == g["rows"].tolist()
+    assert perm.indptr.tolist() == [0, 4, 6, 12]
+    assert (perm.indptr[1:] - perm.indptr[:-1]).sum() // g["block"] == len(g["offsets"]) - 1
+    assert perm.pos[:, 0].tolist() == [0, 6, 1, 7, 4, 8, 2, 9, 10, 11]
+    assert perm.row_token.tolist() == [0, 2, 6, -1, 4, -1, 1, 3, 5, 7, 8, 9]
+    # without padding the same pairs are numbered densely
+    assert O.permute(idx, 3).indptr.tolist() == [0, 3, 4, 10]
+
+
+def test_padding_does_not_change_the_layer_output():
+    rng = np.random.default_rng(16)
+    x, W_r, W1, W3, W2, _ = _rand_layer(rng, 40, 16, 8, 8)
+    a = O.moe_forward(x, W_r, W1, W3, W2, k=2, capacity_factor=1.0)
+    b = O.moe_forward(x, W_r, W1, W3, W2, k=2, capacity_factor=1.0, pad=4)
+    assert np.array_equal(a.y, b.y)
+    assert np.array_equal(a.perm.kept, b.perm.kept)
+    assert (b.perm.indptr % 4 == 0).all() and b.perm.indptr[-1] >= a.perm.indptr[-1]
+
+
 # --- closed forms ([CME295 W2D2] §2.3; [CMU 15-779 L21] §3.1 and exercise 4; §2.1 counts) ---
 
 def test_experts_touched_table():
