@@ -279,21 +279,22 @@ def config_of(cfg, args):
             "d_ff_shared": cfg["d_ff_shared"], "global_batch_tokens": cfg["T"] * args.gpus,
             "parallelism": f"dp{args.gpus} replicas" if args.gpus > 1 else "single GPU",
             "l2": "512 MiB buffer written between timed steps (weights 2.8 GB also exceed L2)",
-            "launch": "eager" if getattr(args, "no_graph", False) else "cuda_graph (captured moe_forward, replayed)"}
+            "launch": "eager" if getattr(args, "no_graph", False) else "cuda_graph (captured moe_forward, replayed)",
+            "pad_rows": getattr(args, "pad_rows", 0)}
 
 
-def launches_per_forward(cfg):
+def launches_per_forward(cfg, pad_rows=0):
     """Kernels one moe_forward launches (the library's own choice of path)."""
     if cfg["T"] == 0:
         return 1
     small = (cfg["dtype"] == "bf16" and cfg["d_ff_shared"] == 0 and cfg["T"] * cfg["k"] <= 64
              and cfg["E"] <= 64 and cfg["E"] % 8 == 0 and cfg["d"] % 8 == 0)
-    if small:
+    if small and not pad_rows:
         # partial router logits, routing finisher, grouped GEMM 1/3, grouped GEMM 2, combine
         return 5
     # transpose W_r, logits (SIMT or tensor-core), select, scan, permute+gather,
-    # grouped GEMM 1/3, grouped GEMM 2, combine
-    return 8
+    # (padding fill,) grouped GEMM 1/3, grouped GEMM 2, combine
+    return 8 + (1 if pad_rows else 0)
 
 
 def main():
@@ -307,6 +308,8 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=16, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the forward eagerly in the timed loop")
+    ap.add_argument("--pad-rows", type=int, default=0, choices=[0, 64, 128],
+                    help="pad every expert's rows to a multiple of this (the MegaBlocks layout), for comparison")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -339,7 +342,7 @@ def main():
         L["x"] = x_r
     L = {k_: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k_, v in L.items()}
     p = moe.problem(cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg["cf"], cfg["dtype"], cfg["bias_mode"],
-                    cfg["d_ff_shared"])
+                    cfg["d_ff_shared"], pad_rows=args.pad_rows)
     layer = moe.MoELayer(p, L["W_r"], L["W1"], L["W3"], L["W2"], bias=L["bias"], Ws1=L["Ws1"], Ws3=L["Ws3"],
                          Ws2=L["Ws2"])
     x = L["x"]
@@ -457,7 +460,7 @@ def main():
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
                 "d2h_bytes_per_step": nbytes},
-        "gpu_launches": launches_per_forward(cfg) * args.steps,
+        "gpu_launches": launches_per_forward(cfg, args.pad_rows) * args.steps,
         "clocks": clocks,
         "stages_ms": stages,
         "routing": {"rows": rows, "dropped": st.dropped, "l_aux": st.l_aux, "max_over_mean": st.max_over_mean,
@@ -492,10 +495,11 @@ def breakdown(moe, p, cfg, L, dev, stream, flush, iters):
     gate = torch.empty((T, k), dtype=torch.float32, device=dev)
     pos = torch.empty((T, k), dtype=torch.int32, device=dev)
     indptr = torch.empty((E + 1,), dtype=torch.int32, device=dev)
-    row_token = torch.empty((T * k,), dtype=torch.int32, device=dev)
-    xp = torch.empty((T * k, d), dtype=dt, device=dev)
-    h = torch.empty((T * k, dff), dtype=dt, device=dev)
-    o = torch.empty((T * k, d), dtype=dt, device=dev)
+    R = moe.permuted_rows(p)
+    row_token = torch.empty((R,), dtype=torch.int32, device=dev)
+    xp = torch.empty((R, d), dtype=dt, device=dev)
+    h = torch.empty((R, dff), dtype=dt, device=dev)
+    o = torch.empty((R, d), dtype=dt, device=dev)
     hs = torch.empty((T, dfs), dtype=dt, device=dev) if dfs else None
     s = torch.empty((T, d), dtype=dt, device=dev) if dfs else None
     out = torch.empty((T, d), dtype=dt, device=dev)

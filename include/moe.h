@@ -92,6 +92,10 @@ typedef struct moe_problem {
     int32_t d_ff_shared;      /* hidden width of the always-on shared expert, 0 = none    */
     int32_t gate_mode;        /* MOE_GATE_*  (0 = selected softmax)                       */
     int32_t drop_order;       /* MOE_DROP_*  (0 = token order)                            */
+    int32_t pad_rows;         /* 0, 64 or 128: pad every expert's kept rows to a multiple
+                                 of this inside the permutation (the MegaBlocks layout,
+                                 "Lecture 21 · LLM: Mixture-of-Experts" §3.6); padding rows
+                                 are zero in Xp and belong to no token. 0 = dense rows.  */
 } moe_problem;
 
 /* ---- statistics block (device memory, moe_stats_size(E) bytes) ----------
@@ -106,7 +110,8 @@ typedef struct moe_problem {
 typedef struct moe_stats {
     int32_t status;        /* MOE_OK, or MOE_ERR_TIMEOUT from a device-side bounded wait */
     int32_t capacity;      /* C, or -1 when unlimited                                     */
-    int32_t rows;          /* R = sum_e kept_e (rows of the permuted buffer)             */
+    int32_t rows;          /* R = sum_e kept_e (kept pairs; with pad_rows the permuted
+                              buffer holds indptr[E] >= R rows, the rest zero padding)   */
     int32_t dropped;       /* sum_e (c_e - kept_e)                                        */
     int32_t max_count;     /* max_e c_e                                                   */
     float   l_aux;         /* E * sum_e f_e P_e                                           */
@@ -136,11 +141,11 @@ typedef struct moe_workspace_layout_t {
     size_t gate;       /* fp32  [T, k]  gates                                         */
     size_t pos;        /* int32 [T, k]  permuted row of (t, j), -1 = dropped          */
     size_t indptr;     /* int32 [E+1]   CSR row offsets over kept rows                */
-    size_t row_token;  /* int32 [T*k]   token of each permuted row (first R valid)    */
+    size_t row_token;  /* int32 [Rmax]  token of each permuted row, -1 on padding     */
     size_t logits;     /* fp32  [T, E]  router logits                                 */
-    size_t xp;         /* dtype [T*k, d]      permuted activations (first R rows)     */
-    size_t h;          /* dtype [T*k, d_ff]   SwiGLU hidden rows                      */
-    size_t o;          /* dtype [T*k, d]      expert outputs, permuted order          */
+    size_t xp;         /* dtype [Rmax, d]     permuted activations (first indptr[E])  */
+    size_t h;          /* dtype [Rmax, d_ff]  SwiGLU hidden rows                      */
+    size_t o;          /* dtype [Rmax, d]     expert outputs, permuted order          */
     size_t hs;         /* dtype [T, d_ff_shared]  shared-expert hidden rows           */
     size_t s;          /* dtype [T, d]        shared-expert output                    */
     size_t total;      /* = moe_workspace_size(p)                                    */
@@ -148,6 +153,10 @@ typedef struct moe_workspace_layout_t {
 
 size_t moe_workspace_size(const moe_problem* p);
 int    moe_workspace_layout(const moe_problem* p, moe_workspace_layout_t* out);
+
+/* Rmax: rows a permuted buffer (xp, h, o, row_token) must hold for p:
+ * T*k, plus E*(pad_rows-1) when pad_rows > 0; 0 when p is invalid. */
+int32_t moe_permuted_rows(const moe_problem* p);
 
 /* ---- the whole layer ----------------------------------------------------
  * moe_forward: out[t] = sum_{j<k, kept} gate[t,j] * FFN_{idx[t,j]}(x[t]) + FFN_shared(x[t]).
@@ -186,8 +195,11 @@ int moe_route_from_logits(const moe_problem* p, const float* logits, const float
 /* Permutation (Lecture 21 §3.3 and §3.5): per-expert histogram, expert-major
  * exclusive scan, rank of each pair in token order, capacity truncation,
  * and gather of token rows: xp[pos[t,j]] = x[t] for kept pairs.
- *   idx [T, k] int32 in; pos [T, k], indptr [E+1], row_token [T*k] int32 out;
- *   xp [T*k, d] dtype out (rows >= R untouched).
+ *   idx [T, k] int32 in; pos [T, k], indptr [E+1], row_token [Rmax] int32 out;
+ *   xp [Rmax, d] dtype out (rows >= indptr[E] untouched).
+ * With pad_rows > 0 (§3.6) indptr counts every expert's kept rows rounded up
+ * to a multiple of pad_rows; the padding rows after an expert's kept rows
+ * are written as zeros in xp and -1 in row_token.
  * stats receives counts/kept/capacity/rows/dropped/max_count; P, f and
  * l_aux are left as they are. */
 int moe_permute(const moe_problem* p, const void* x, const int32_t* idx,
@@ -198,9 +210,9 @@ int moe_permute(const moe_problem* p, const void* x, const int32_t* idx,
  * indptr, weights)): for every expert e and row r in [indptr[e], indptr[e+1]):
  *   o[r] = W2_e (SiLU(W1_e xp[r]) * (W3_e xp[r]))
  * and, when d_ff_shared > 0, s[t] = Ws2 (SiLU(Ws1 x[t]) * (Ws3 x[t])).
- *   xp [T*k, d], o [T*k, d] (rows >= indptr[E] untouched), x [T, d], s [T, d].
+ *   xp [Rmax, d], o [Rmax, d] (rows >= indptr[E] untouched), x [T, d], s [T, d].
  * indptr is read on the device; the host never waits for it; its entries must
- * be non-decreasing with indptr[0] = 0 and indptr[E] <= T*k.
+ * be non-decreasing with indptr[0] = 0 and indptr[E] <= Rmax.
  * stats (may be NULL): only the status word is written (MOE_OK, or
  * MOE_ERR_TIMEOUT if a bounded wait of the tensor-core kernel gave up). */
 int moe_experts(const moe_problem* p, const void* xp, const int32_t* indptr,
@@ -210,9 +222,9 @@ int moe_experts(const moe_problem* p, const void* xp, const int32_t* indptr,
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* The two halves of moe_experts, for per-stage timing and inspection:
- *   moe_expert_up:   h[r] = SiLU(W1_e xp[r]) * (W3_e xp[r])      h  [T*k, d_ff]
+ *   moe_expert_up:   h[r] = SiLU(W1_e xp[r]) * (W3_e xp[r])      h  [Rmax, d_ff]
  *                    hs[t] = SiLU(Ws1 x[t]) * (Ws3 x[t])          hs [T, d_ff_shared]
- *   moe_expert_down: o[r] = W2_e h[r];  s[t] = Ws2 hs[t]          o [T*k, d], s [T, d]
+ *   moe_expert_down: o[r] = W2_e h[r];  s[t] = Ws2 hs[t]          o [Rmax, d], s [T, d]
  * Same indptr rules and workspace as moe_experts (the tile schedule is
  * rebuilt from indptr by each call). */
 int moe_expert_up(const moe_problem* p, const void* xp, const int32_t* indptr,
@@ -249,6 +261,7 @@ int moe_combine(const moe_problem* p, const void* o, const int32_t* pos, const f
  *    that overlap on the GPU (different streams, or different host threads,
  *    on the same device) race on it: serialise them.
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+/* (pad_rows must be 0 here: MOE_ERR_UNSUPPORTED otherwise.) */
 int moe_permute_noalloc(const moe_problem* p, const void* x, const int32_t* idx,
                         int32_t* pos, int32_t* indptr, int32_t* row_token, void* xp, void* stats,
                         void* stream);

@@ -47,7 +47,7 @@ class Problem(ctypes.Structure):
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
                 ("dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
                 ("d_ff_shared", ctypes.c_int32), ("gate_mode", ctypes.c_int32),
-                ("drop_order", ctypes.c_int32)]
+                ("drop_order", ctypes.c_int32), ("pad_rows", ctypes.c_int32)]
 
 
 class WorkspaceLayout(ctypes.Structure):
@@ -79,6 +79,8 @@ def _load():
     lib.moe_error_string.restype = ctypes.c_char_p
     lib.moe_device_sm_count.argtypes = []
     lib.moe_device_sm_count.restype = ctypes.c_int
+    lib.moe_permuted_rows.argtypes = [P]
+    lib.moe_permuted_rows.restype = ctypes.c_int32
     lib.moe_forward.argtypes = [P] + [vp] * 11 + [vp, sz, vp]
     lib.moe_forward.restype = ctypes.c_int
     lib.moe_route.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -137,9 +139,18 @@ def torch_dtype(code: int):
 
 
 def problem(T, d, d_ff, E, k, capacity_factor=0.0, dtype="bf16", bias_mode=BIAS_NONE, d_ff_shared=0,
-            gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN) -> Problem:
+            gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN, pad_rows=0) -> Problem:
     return Problem(int(T), int(d), int(d_ff), int(E), int(k), float(capacity_factor),
-                   _dtype_code(dtype), int(bias_mode), int(d_ff_shared), int(gate_mode), int(drop_order))
+                   _dtype_code(dtype), int(bias_mode), int(d_ff_shared), int(gate_mode), int(drop_order),
+                   int(pad_rows))
+
+
+def permuted_rows(p: Problem) -> int:
+    """Rows the permuted buffers (xp, h, o, row_token) must hold for p."""
+    n = int(_lib().moe_permuted_rows(ctypes.byref(p)))
+    if n == 0 and p.T * p.k > 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_permuted_rows")
+    return n
 
 
 def stats_size(E: int) -> int:

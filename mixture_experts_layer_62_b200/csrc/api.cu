@@ -8,8 +8,14 @@
 
 namespace moe {
 
+long long permuted_rows(const moe_problem& p) {
+    const long long T = p.T > 0 ? p.T : 0;
+    return T * p.k + (p.pad_rows > 0 ? (long long)p.E * (p.pad_rows - 1) : 0);
+}
+
 Layout make_layout(const moe_problem& p) {
     const size_t T = p.T > 0 ? (size_t)p.T : 0, k = (size_t)p.k, E = (size_t)p.E;
+    const size_t Rmax = (size_t)permuted_rows(p);
     const size_t d = (size_t)p.d, dff = (size_t)p.d_ff, dfs = (size_t)(p.d_ff_shared > 0 ? p.d_ff_shared : 0);
     const size_t eb = elem_bytes(p.dtype);
     const size_t NB = (T + kChunk - 1) / kChunk;
@@ -24,7 +30,7 @@ Layout make_layout(const moe_problem& p) {
     L.gate = take(T * k * 4);
     L.pos = take(T * k * 4);
     L.indptr = take((E + 1) * 4);
-    L.row_token = take(T * k * 4);
+    L.row_token = take(Rmax * 4);
     L.logits = take(T * E * 4);
     L.wrt = take(E * d * eb);
     const size_t kk = (size_t)count_slots(p);
@@ -36,9 +42,9 @@ Layout make_layout(const moe_problem& p) {
     L.blockextra = take(NB * 3 * 4);
     L.tiles13 = take((E + 3) * 4);
     L.tiles2 = take((E + 3) * 4);
-    L.xp = take(T * k * d * eb);
-    L.h = take(T * k * dff * eb);
-    L.o = take(T * k * d * eb);
+    L.xp = take(Rmax * d * eb);
+    L.h = take(Rmax * dff * eb);
+    L.o = take(Rmax * d * eb);
     L.hs = take(T * dfs * eb);
     L.s = take(dfs ? T * d * eb : 0);
     const bool split = split_allowed(p);
@@ -93,7 +99,7 @@ void fill_split_table(SplitTable& t, int nt13, int nt2, int nkb13, int nkb2, int
 }
 
 bool split_allowed(const moe_problem& p) {
-    return p.dtype == MOE_DTYPE_BF16 && p.d_ff_shared == 0 && p.T > 0 &&
+    return p.dtype == MOE_DTYPE_BF16 && p.d_ff_shared == 0 && p.T > 0 && p.pad_rows == 0 &&
            (long long)p.T * p.k <= kSplitMaxRows;
 }
 
@@ -131,7 +137,8 @@ int check_problem(const moe_problem* p) {
     if (p->drop_order != MOE_DROP_TOKEN && p->drop_order != MOE_DROP_SLOT) return MOE_ERR_INVALID_ARG;
     if (p->drop_order == MOE_DROP_SLOT && p->E * p->k > kMaxSlotCounts) return MOE_ERR_UNSUPPORTED;
     if (!std::isfinite(p->capacity_factor)) return MOE_ERR_INVALID_ARG;
-    const long long rows = (long long)p->T * p->k;
+    if (p->pad_rows != 0 && p->pad_rows != 64 && p->pad_rows != 128) return MOE_ERR_INVALID_ARG;
+    const long long rows = permuted_rows(*p);
     if (rows * (long long)(p->d > p->d_ff ? p->d : p->d_ff) >= (1LL << 40) || rows >= (1LL << 30))
         return MOE_ERR_UNSUPPORTED;
     if (p->dtype == MOE_DTYPE_BF16) {
@@ -192,13 +199,14 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
            cudaStream_t st, float* part13 = nullptr, int32_t* sem13 = nullptr, bool sched_early = true) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
+    const int arows = (int)permuted_rows(*p);   // rows of the permuted buffers
     if (p->dtype == MOE_DTYPE_BF16) {
         TcArgs a = {};
         a.mode = TC_SWIGLU;
         a.b_before_wait = sched_early ? 1 : 0;
         a.indptr = indptr; a.tiles = tiles13;
         a.E = p->E; a.has_shared = has_shared; a.T = p->T;
-        a.A[0] = xp; a.a_rows[0] = rows; a.A[1] = has_shared ? x : nullptr; a.a_rows[1] = p->T;
+        a.A[0] = xp; a.a_rows[0] = arows; a.A[1] = has_shared ? x : nullptr; a.a_rows[1] = p->T;
         a.B[0][0] = W1; a.B[0][1] = W3; a.b_rows[0] = p->d_ff; a.b_total_rows[0] = p->E * p->d_ff;
         a.B[1][0] = Ws1; a.B[1][1] = Ws3; a.b_rows[1] = p->d_ff_shared; a.b_total_rows[1] = p->d_ff_shared;
         a.N[0] = p->d_ff; a.N[1] = p->d_ff_shared;
@@ -216,7 +224,7 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
         GroupedArgs a = {};
         a.indptr = indptr; a.tiles = tiles13;
         a.E = p->E; a.has_shared = has_shared; a.T = p->T;
-        a.A[0] = xp; a.a_rows[0] = rows; a.A[1] = x; a.a_rows[1] = p->T;
+        a.A[0] = xp; a.a_rows[0] = arows; a.A[1] = x; a.a_rows[1] = p->T;
         a.B[0][0] = W1; a.B[0][1] = W3; a.B[1][0] = Ws1; a.B[1][1] = Ws3;
         a.N[0] = p->d_ff; a.N[1] = p->d_ff_shared;
         a.K[0] = p->d; a.K[1] = p->d;
@@ -233,13 +241,14 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
              float* part2 = nullptr, int32_t* sem2 = nullptr) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
+    const int arows = (int)permuted_rows(*p);   // rows of the permuted buffers
     if (p->dtype == MOE_DTYPE_BF16) {
         TcArgs b = {};
         b.mode = TC_PLAIN;
         b.b_before_wait = 1;   // the schedule comes from the router, two or more launches back
         b.indptr = indptr; b.tiles = tiles2;
         b.E = p->E; b.has_shared = has_shared; b.T = p->T;
-        b.A[0] = h; b.a_rows[0] = rows; b.A[1] = has_shared ? hs : nullptr; b.a_rows[1] = p->T;
+        b.A[0] = h; b.a_rows[0] = arows; b.A[1] = has_shared ? hs : nullptr; b.a_rows[1] = p->T;
         b.B[0][0] = W2; b.B[0][1] = W2; b.b_rows[0] = p->d; b.b_total_rows[0] = p->E * p->d;
         b.B[1][0] = Ws2; b.B[1][1] = Ws2; b.b_rows[1] = p->d; b.b_total_rows[1] = p->d;
         b.N[0] = p->d; b.N[1] = p->d;
@@ -257,7 +266,7 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
         GroupedArgs b = {};
         b.indptr = indptr; b.tiles = tiles2;
         b.E = p->E; b.has_shared = has_shared; b.T = p->T;
-        b.A[0] = h; b.a_rows[0] = rows; b.A[1] = hs; b.a_rows[1] = p->T;
+        b.A[0] = h; b.a_rows[0] = arows; b.A[1] = hs; b.a_rows[1] = p->T;
         b.B[0][0] = W2; b.B[0][1] = nullptr; b.B[1][0] = Ws2; b.B[1][1] = nullptr;
         b.N[0] = p->d; b.N[1] = p->d;
         b.K[0] = p->d_ff; b.K[1] = p->d_ff_shared;
@@ -343,6 +352,11 @@ int moe_workspace_layout(const moe_problem* p, moe_workspace_layout_t* out) {
 }
 
 int moe_device_sm_count(void) { return device_sm_count(); }
+
+int32_t moe_permuted_rows(const moe_problem* p) {
+    if (check_problem(p) != MOE_OK) return 0;
+    return (int32_t)permuted_rows(*p);
+}
 
 const char* moe_error_string(int code) {
     switch (code) {
@@ -440,9 +454,12 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
         fill_split_table(sa.split, sa.ntiles13, sa.ntiles2, ceil_div(p->d, 64), ceil_div(p->d_ff, 64),
                          device_sm_count(), kSplitMax, p->T * p->k);
     }
+    sa.pad = p->pad_rows;
     CK(launch_scan(sa, st));
     CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, kk, C, pos, row_token, xp,
                              st));
+    if (p->pad_rows > 0)
+        CK(launch_pad_fill(p->dtype, indptr, stats, p->E, p->d, xp, row_token, p->pad_rows, st));
     }
     void* h = wsp(workspace, L.h);
     void* o = wsp(workspace, L.o);
@@ -494,6 +511,7 @@ int moe_route(const moe_problem* p, const void* x, const void* W_r, const float*
     sa.blockpsum = blockpsum; sa.blockextra = blockextra;
     sa.indptr = reinterpret_cast<int32_t*>(wsp(workspace, L.indptr));
     sa.stats = stats;
+    sa.pad = p->pad_rows;
     CK(launch_scan(sa, st));
     return MOE_OK;
 }
@@ -527,6 +545,7 @@ int moe_route_from_logits(const moe_problem* p, const float* logits, const float
     sa.blockpsum = blockpsum; sa.blockextra = blockextra;
     sa.indptr = reinterpret_cast<int32_t*>(wsp(workspace, L.indptr));
     sa.stats = stats;
+    sa.pad = p->pad_rows;
     CK(launch_scan(sa, st));
     return MOE_OK;
 }
@@ -557,9 +576,12 @@ int moe_permute(const moe_problem* p, const void* x, const int32_t* idx, int32_t
     sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C; sa.kk = kk;
     sa.blockcnt = blockcnt; sa.blockoff = blockoff; sa.blockpsum = nullptr;
     sa.indptr = indptr; sa.stats = stats;
+    sa.pad = p->pad_rows;
     CK(launch_scan(sa, st));
     CK(launch_permute_gather(p->dtype, x, idx, blockoff, indptr, p->T, p->d, p->E, p->k, kk, C, pos, row_token, xp,
                              st));
+    if (p->pad_rows > 0)
+        CK(launch_pad_fill(p->dtype, indptr, stats, p->E, p->d, xp, row_token, p->pad_rows, st));
     return MOE_OK;
 }
 

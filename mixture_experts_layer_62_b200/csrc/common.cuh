@@ -75,6 +75,8 @@ constexpr int kSplitMaxRows = 128;
 constexpr int kSplitMax = 16;
 bool split_allowed(const moe_problem& p);
 Layout make_layout(const moe_problem& p);
+// Rows a permuted buffer holds: T*k, plus E*(pad_rows-1) when rows are padded.
+long long permuted_rows(const moe_problem& p);
 
 // Split factors by the number of active experts (0 .. kSplitMaxRows): with at
 // most kSplitMaxRows rows every active expert is one M-block, so a GEMM has
@@ -132,8 +134,13 @@ struct ScanArgs {
     int split_on;                // 0: no split (factors 1)
     int32_t* sem; int sem_n;     // split-K counters to zero (sem_n ints), or null
     SplitTable split;
+    int pad;                     // > 0: indptr over kept rows rounded up to a multiple of pad
 };
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st);
+// Padding rows of a padded permutation: rows [indptr[e] + kept[e], indptr[e+1])
+// of xp become zeros and their row_token -1 (kept[] from the stats block).
+cudaError_t launch_pad_fill(int dtype, const int32_t* indptr, const void* stats, int E, int d, void* xp,
+                            int32_t* row_token, int pad, cudaStream_t st);
 // Split-K setup of a tile schedule: factors by active-expert count and the
 // counters to zero.
 struct ScheduleSplit {

@@ -114,13 +114,17 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const __grid_constan
         c = start[e + 1] - start[e];
         kp = a.capacity < 0 ? c : min(c, a.capacity);
     }
-    int tot_kept;
-    int ex = block_exclusive_scan(e < E ? kp : 0, warp_tot, tot_kept);
+    // rows an expert occupies: its kept pairs, rounded up to a multiple of
+    // the block size in the padded (MegaBlocks) layout
+    const int kr = a.pad > 0 ? (kp + a.pad - 1) / a.pad * a.pad : kp;
+    int tot_rows, tot_kept;
+    int ex = block_exclusive_scan(e < E ? kr : 0, warp_tot, tot_rows);
+    block_exclusive_scan(e < E ? kp : 0, warp_tot, tot_kept);
     if (e < E) {
         a.indptr[e] = ex;
         kept_s[e] = kp;
     }
-    if (threadIdx.x == 0) a.indptr[E] = tot_kept;
+    if (threadIdx.x == 0) a.indptr[E] = tot_rows;
 
     moe_stats* st = (moe_stats*)a.stats;
     int32_t* counts = MOE_STATS_COUNTS(a.stats, E);
@@ -191,7 +195,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const __grid_constan
     // 6. tile schedules of the grouped GEMMs
     if (a.tiles13 != nullptr) {
         __shared__ int rows[MOE_MAX_E + 1];
-        if (threadIdx.x < E) rows[threadIdx.x] = kept_s[threadIdx.x];
+        if (threadIdx.x < E) rows[threadIdx.x] = a.pad > 0 ? (kept_s[threadIdx.x] + a.pad - 1) / a.pad * a.pad
+                                                           : kept_s[threadIdx.x];
         if (threadIdx.x == 0) rows[E] = a.T;
         __syncthreads();
         const int G = E + a.has_shared;
@@ -338,6 +343,33 @@ cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
 }
 
 // Statistics for T == 0 (nothing routed).
+// Padding rows of the padded layout: one block per (expert, slice of the
+// row's 16-byte vectors); the expert's last pad-1 rows at most.
+__global__ void __launch_bounds__(256)
+pad_fill_kernel(const int32_t* __restrict__ indptr, const void* __restrict__ stats, int E, int nvec,
+                uint4* __restrict__ xp, int32_t* __restrict__ row_token) {
+    pdl_wait();
+    pdl_launch();
+    const int e = blockIdx.x;
+    const int r0 = indptr[e] + MOE_STATS_KEPT(stats, E)[e], r1 = indptr[e + 1];
+    const int n = xp != nullptr ? (r1 - r0) * nvec : 0;
+    for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < n; i += gridDim.y * blockDim.x)
+        xp[(size_t)(r0 + i / nvec) * nvec + i % nvec] = make_uint4(0u, 0u, 0u, 0u);
+    if (blockIdx.y == 0 && row_token != nullptr)
+        for (int r = r0 + (int)threadIdx.x; r < r1; r += blockDim.x) row_token[r] = -1;
+}
+
+cudaError_t launch_pad_fill(int dtype, const int32_t* indptr, const void* stats, int E, int d, void* xp,
+                            int32_t* row_token, int pad, cudaStream_t st) {
+    const int nvec = (int)((size_t)d * elem_bytes(dtype) / 16);
+    // at most pad - 1 rows per expert
+    const int per_expert = (pad - 1) * nvec;
+    int gy = (per_expert + 256 * 4 - 1) / (256 * 4);
+    gy = gy < 1 ? 1 : gy;
+    return launch_k(pad_fill_kernel, dim3(E, gy), dim3(256), 0, st, indptr, stats, E, nvec,
+                    static_cast<uint4*>(xp), row_token);
+}
+
 __global__ void zero_stats_kernel(void* stats, int E, int capacity) {
     pdl_wait();
     pdl_launch();

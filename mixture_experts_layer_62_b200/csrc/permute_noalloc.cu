@@ -80,6 +80,7 @@ extern "C" int moe_permute_noalloc(const moe_problem* p, const void* x, const in
     const int kk = moe::count_slots(*p);
     if (kk > 1 && p->E * p->k > moe::kMaxSlotCounts) return MOE_ERR_UNSUPPORTED;
     if ((long long)p->E * kk * nb > kMaxEntries) return MOE_ERR_UNSUPPORTED;   // beyond the static scratch
+    if (p->pad_rows != 0) return MOE_ERR_UNSUPPORTED;                         // dense rows only
 
     int32_t* scratch = scratch_on_current_device();
     if (scratch == nullptr) return MOE_ERR_CUDA;

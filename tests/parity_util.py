@@ -43,7 +43,8 @@ class LazyExperts:
 
 def problem_of(cfg):
     return moe.problem(cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg["cf"], cfg["dtype"],
-                       cfg["bias_mode"], cfg["d_ff_shared"], cfg.get("gate", 0), cfg.get("drop", 0))
+                       cfg["bias_mode"], cfg["d_ff_shared"], cfg.get("gate", 0), cfg.get("drop", 0),
+                       cfg.get("pad", 0))
 
 
 def gpu_forward(cfg, L, device="cuda"):

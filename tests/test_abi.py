@@ -17,7 +17,7 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"^\s*(?:int|size_t|const\s+char\s*\*)\s+(moe_\w+)\s*\(", src, flags=re.M)
+    names = re.findall(r"^\s*(?:int|int32_t|size_t|const\s+char\s*\*)\s+(moe_\w+)\s*\(", src, flags=re.M)
     assert names, "no declarations parsed"
     return sorted(set(names))
 
@@ -39,6 +39,22 @@ def test_error_strings():
     for code in range(1, 6):
         assert moe.error_string(code) not in ("ok", "unknown error")
     assert moe.error_string(99) == "unknown error"
+
+
+def test_permuted_rows_and_padding_validation():
+    p = moe.problem(100, 64, 64, 8, 2)
+    assert moe.permuted_rows(p) == 200
+    p = moe.problem(100, 64, 64, 8, 2, pad_rows=128)
+    assert moe.permuted_rows(p) == 200 + 8 * 127
+    lay = moe.workspace_layout(p)
+    assert lay["h"] - lay["xp"] >= (200 + 8 * 127) * 64 * 2
+    fake = ctypes.c_void_p(1 << 20)
+    for bad in (32, 100, 256, -1):
+        q = moe.problem(16, 64, 64, 4, 2, pad_rows=bad)
+        assert moe.lib.moe_forward(ctypes.byref(q), *([fake] * 11), fake, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+        assert moe.lib.moe_permuted_rows(ctypes.byref(q)) == 0
+    q = moe.problem(16, 64, 64, 4, 2, pad_rows=64)
+    assert moe.lib.moe_permute_noalloc(ctypes.byref(q), *([fake] * 7), None) == moe.MOE_ERR_UNSUPPORTED
 
 
 def test_stats_size_matches_header_layout():

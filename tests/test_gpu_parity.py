@@ -145,6 +145,60 @@ def test_permute_bit_exact(T, E, k, cf, dtype, drop):
     assert torch.equal(xp[:R].cpu(), x.cpu()[torch.from_numpy(perm.row_token)])
 
 
+@pytest.mark.parametrize("T,E,k,cf,dtype,pad", [
+    (1000, 8, 2, 0.6, "bf16", 128), (300, 64, 8, 0.0, "bf16", 64), (77, 6, 3, 0.4, "f32", 128),
+    (2049, 256, 8, 1.0, "bf16", 128), (1, 8, 2, 0.0, "bf16", 64),
+])
+def test_permute_padded_bit_exact(T, E, k, cf, dtype, pad):
+    rng = np.random.default_rng(T + E * 11)
+    z = rng.standard_normal((T, E))
+    z[:, 0] += 1.0
+    idx_np = O.topk_lowest_index(z, k)
+    d = 128 if dtype == "bf16" else 64
+    x = torch.randn((T, d), dtype=torch.float32).to(_dt(dtype)).to(DEV)
+    p = moe.problem(T, d, 64, E, k, cf, dtype, pad_rows=pad)
+    Rmax = moe.permuted_rows(p)
+    assert Rmax == T * k + E * (pad - 1)
+    ws = moe.alloc_workspace(p, DEV)
+    st = moe.alloc_stats(E, DEV)
+    idx = torch.from_numpy(idx_np.astype(np.int32)).to(DEV)
+    pos = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    indptr = torch.empty((E + 1,), dtype=torch.int32, device=DEV)
+    row_token = torch.full((Rmax,), -7, dtype=torch.int32, device=DEV)
+    xp = torch.full((Rmax, d), 3.0, dtype=_dt(dtype), device=DEV)     # padding must be overwritten
+    moe.permute(p, x, idx, pos, indptr, row_token, xp, st, ws)
+    torch.cuda.synchronize()
+    C = O.capacity(cf, T, k, E)
+    perm = O.permute(idx_np, E, C, O.DROP_TOKEN, pad=pad)
+    assert np.array_equal(pos.cpu().numpy(), perm.pos)
+    assert np.array_equal(indptr.cpu().numpy(), perm.indptr)
+    R = int(perm.indptr[-1])
+    assert R % pad == 0 or R == 0
+    rt = row_token.cpu().numpy()
+    assert np.array_equal(rt[:R], perm.row_token)
+    s = moe.read_stats(st, E)
+    assert s.kept == perm.kept.tolist() and s.rows == int(perm.kept.sum())
+    xh = xp[:R].cpu()
+    real = torch.from_numpy(perm.row_token >= 0)
+    assert torch.equal(xh[real], x.cpu()[torch.from_numpy(perm.row_token[perm.row_token >= 0])])
+    assert (xh[~real] == 0).all()
+
+
+def test_padded_forward_equals_dense():
+    # same kernels per row: padding moves rows to other tiles but computes
+    # every kept row the same way (no split-K at these sizes)
+    for cfg in (dict(T=600, d=256, d_ff=384, E=8, k=2, cf=0.7, dtype="bf16", bias_mode=1, d_ff_shared=0),
+                dict(T=200, d=128, d_ff=128, E=32, k=4, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=128),
+                dict(T=300, d=64, d_ff=128, E=6, k=2, cf=0.0, dtype="f32", bias_mode=0, d_ff_shared=0)):
+        L = to_device(_small_layer(cfg, seed=21))
+        outs = []
+        for pad in (0, 64, 128):
+            p, out, st, ws = gpu_forward(dict(cfg, pad=pad), L)
+            assert moe.read_stats(st, cfg["E"]).status == moe.MOE_OK
+            outs.append(out.cpu())
+        assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
 # --------------------------------------------------------------------------
 # expert GEMMs (tcgen05 for bf16, CUDA cores for fp32)
 # --------------------------------------------------------------------------
@@ -262,6 +316,12 @@ SMALL = [
     dict(T=700, d=128, d_ff=256, E=16, k=2, cf=0.7, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=0, drop=1),
     dict(T=24, d=256, d_ff=128, E=8, k=2, cf=0.6, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=1, drop=1),
     dict(T=200, d=64, d_ff=64, E=6, k=3, cf=0.5, dtype="f32", bias_mode=0, d_ff_shared=0, gate=1, drop=1),
+    # padded (MegaBlocks) layout: every expert's rows rounded up to 128 or 64
+    dict(T=300, d=256, d_ff=384, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0, pad=128),
+    dict(T=1000, d=256, d_ff=256, E=8, k=2, cf=0.6, dtype="bf16", bias_mode=1, d_ff_shared=0, pad=64),
+    dict(T=130, d=128, d_ff=128, E=64, k=8, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=128, pad=128),
+    dict(T=20, d=256, d_ff=256, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0, pad=128),
+    dict(T=257, d=64, d_ff=128, E=6, k=3, cf=0.25, dtype="f32", bias_mode=1, d_ff_shared=64, pad=128),
 ]
 
 
@@ -304,7 +364,8 @@ def _check_forward(cfg, L_cpu, tokens=None, check_own_routing=True):
     res = O.moe_forward(x_np, None, W["W1"], W["W3"], W["W2"], k, cfg["cf"], bias, cfg["bias_mode"],
                         W["Ws1"], W["Ws3"], W["Ws2"], logits=logits, tokens=tokens,
                         key_dtype=np.float32 if exact_key else np.float64,
-                        gate_mode=cfg.get("gate", 0), drop_order=cfg.get("drop", 0))
+                        gate_mode=cfg.get("gate", 0), drop_order=cfg.get("drop", 0),
+                        pad=cfg.get("pad") or None)
     if exact_key:
         assert np.array_equal(g_idx, res.routing.idx)
         assert np.array_equal(g_pos, res.perm.pos)
@@ -347,7 +408,7 @@ def _check_forward(cfg, L_cpu, tokens=None, check_own_routing=True):
 
 @pytest.mark.parametrize("cfg", SMALL, ids=[f"T{c['T']}_E{c['E']}_k{c['k']}_{c['dtype']}_b{c['bias_mode']}"
                                             f"_cf{c['cf']}_s{c['d_ff_shared']}_g{c.get('gate', 0)}"
-                                            f"_d{c.get('drop', 0)}" for c in SMALL])
+                                            f"_d{c.get('drop', 0)}_p{c.get('pad', 0)}" for c in SMALL])
 def test_forward_small(cfg):
     _check_forward(cfg, _small_layer(cfg, cfg["T"] + cfg["E"]))
 
@@ -458,18 +519,21 @@ def _sample_tokens(pos, indptr, rng, n_random):
                 row_of[int(pos[t, j])] = t
     for e in range(len(indptr) - 1):
         lo, hi = int(indptr[e]), int(indptr[e + 1])
-        if hi > lo:
-            picks.add(row_of[lo])
-            picks.add(row_of[hi - 1])
+        rows = [r for r in (lo, hi - 1) if r in row_of]
+        while hi - 1 > lo and hi - 1 not in row_of:   # padded layout: last kept row
+            hi -= 1
+        if hi - 1 in row_of:
+            rows.append(hi - 1)
+        picks.update(row_of[r] for r in rows)
     dropped = np.nonzero((pos < 0).all(axis=1))[0]
     picks.update(dropped[:4].tolist())
     return np.array(sorted(picks))
 
 
-@pytest.mark.parametrize("name,n_random", [("mixtral_prefill", 24), ("skewed_capacity", 16),
-                                           ("deepseek_v3", 6)])
-def test_forward_full_size(name, n_random):
-    cfg = inputs.workload(name)
+@pytest.mark.parametrize("name,n_random,pad", [("mixtral_prefill", 24, 0), ("skewed_capacity", 16, 0),
+                                               ("deepseek_v3", 6, 0), ("mixtral_prefill", 8, 128)])
+def test_forward_full_size(name, n_random, pad):
+    cfg = dict(inputs.workload(name), pad=pad)
     L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=DEV)
     Ld = to_device(L)
     p, out, st, ws = gpu_forward(cfg, Ld)
