@@ -96,6 +96,9 @@ typedef struct moe_problem {
                                  of this inside the permutation (the MegaBlocks layout,
                                  "Lecture 21 · LLM: Mixture-of-Experts" §3.6); padding rows
                                  are zero in Xp and belong to no token. 0 = dense rows.  */
+    int32_t train;            /* 1: moe_forward also keeps the experts' gate and up
+                                 pre-activations (W1 x, W3 x) in the workspace for
+                                 moe_backward (bf16 only); 0: inference               */
 } moe_problem;
 
 /* ---- statistics block (device memory, moe_stats_size(E) bytes) ----------
@@ -148,6 +151,8 @@ typedef struct moe_workspace_layout_t {
     size_t o;          /* dtype [Rmax, d]     expert outputs, permuted order          */
     size_t hs;         /* dtype [T, d_ff_shared]  shared-expert hidden rows           */
     size_t s;          /* dtype [T, d]        shared-expert output                    */
+    size_t ab;         /* dtype [Rmax, 2*d_ff] with train: per 128 hidden units, 128
+                          gate pre-activations then the 128 up pre-activations   */
     size_t total;      /* = moe_workspace_size(p)                                    */
 } moe_workspace_layout_t;
 
@@ -265,6 +270,40 @@ int moe_combine(const moe_problem* p, const void* o, const int32_t* pos, const f
 int moe_permute_noalloc(const moe_problem* p, const void* x, const int32_t* idx,
                         int32_t* pos, int32_t* indptr, int32_t* row_token, void* xp, void* stats,
                         void* stream);
+
+/* ---- backward pass ------------------------------------------------------
+ * Gradients of L = sum_t <dy_t, y_t> + alpha * L_aux + beta * L_z, where y is
+ * the output of the moe_forward call that filled `workspace` and `stats`
+ * (same p, same inputs, nothing run on the workspace since), L_aux =
+ * E sum_e f_e P_e with the counts f frozen (Week 2 Day 2 §3.2: its gradient
+ * reaches the router through P only) and L_z the router z-loss (§3.4). The
+ * expert selection and the capacity drops carry no gradient; the selection
+ * bias gets none.
+ * Requires p->train = 1 (the forward kept the gate/up pre-activations),
+ * p->pad_rows = 64 or 128 (the weight-gradient GEMMs contract over each
+ * expert's rows, which padding keeps in whole 64-row blocks), bf16 and no
+ * shared expert; otherwise MOE_ERR_UNSUPPORTED.
+ *   dy [T, d] bf16 in; dx [T, d] bf16 out;
+ *   dW_r [d, E] fp32, dW1 and dW3 [E, d_ff, d] fp32, dW2 [E, d, d_ff] fp32
+ *   out, each written fully (an expert without rows gets zeros);
+ *   stats: the forward's block (f is read; the status word gets
+ *   MOE_ERR_TIMEOUT if a bounded wait of a tensor-core kernel gave up);
+ *   bwd_workspace: moe_backward_workspace_size(p) bytes, 256-byte aligned,
+ *   no initialisation needed.
+ * Reductions run in a fixed order: repeated calls give identical results. */
+size_t moe_backward_workspace_size(const moe_problem* p);
+int moe_backward(const moe_problem* p, const void* x, const void* W_r, const void* W1, const void* W3,
+                 const void* W2, const void* dy, float alpha, float beta,
+                 void* dx, float* dW_r, float* dW1, float* dW3, float* dW2, void* stats,
+                 const void* workspace, size_t workspace_bytes,
+                 void* bwd_workspace, size_t bwd_workspace_bytes, void* stream);
+
+/* Auxiliary-loss-free balancing step (Lecture 21 §2.4, DeepSeek-V3): for
+ * every expert, bias[e] -= gamma if its count c_e in `stats` is above the
+ * mean load T*k/E, bias[e] += gamma if below, unchanged if equal (decided
+ * exactly, as the sign of c_e*E - T*k). bias [E] fp32 device memory, updated
+ * in place on the stream. */
+int moe_bias_update(const moe_problem* p, const void* stats, float gamma, float* bias, void* stream);
 
 /* Human-readable text of an MOE_* code (static storage). */
 const char* moe_error_string(int code);

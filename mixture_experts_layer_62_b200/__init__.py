@@ -47,12 +47,12 @@ class Problem(ctypes.Structure):
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
                 ("dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
                 ("d_ff_shared", ctypes.c_int32), ("gate_mode", ctypes.c_int32),
-                ("drop_order", ctypes.c_int32), ("pad_rows", ctypes.c_int32)]
+                ("drop_order", ctypes.c_int32), ("pad_rows", ctypes.c_int32), ("train", ctypes.c_int32)]
 
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ("idx", "gate", "pos", "indptr", "row_token", "logits", "xp", "h", "o", "hs", "s", "total")]
+                ("idx", "gate", "pos", "indptr", "row_token", "logits", "xp", "h", "o", "hs", "s", "ab", "total")]
 
 
 class MoEError(RuntimeError):
@@ -81,6 +81,13 @@ def _load():
     lib.moe_device_sm_count.restype = ctypes.c_int
     lib.moe_permuted_rows.argtypes = [P]
     lib.moe_permuted_rows.restype = ctypes.c_int32
+    lib.moe_backward_workspace_size.argtypes = [P]
+    lib.moe_backward_workspace_size.restype = sz
+    f32 = ctypes.c_float
+    lib.moe_backward.argtypes = [P] + [vp] * 6 + [f32, f32] + [vp] * 6 + [vp, sz, vp, sz, vp]
+    lib.moe_backward.restype = ctypes.c_int
+    lib.moe_bias_update.argtypes = [P, vp, f32, vp, vp]
+    lib.moe_bias_update.restype = ctypes.c_int
     lib.moe_forward.argtypes = [P] + [vp] * 11 + [vp, sz, vp]
     lib.moe_forward.restype = ctypes.c_int
     lib.moe_route.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -139,10 +146,10 @@ def torch_dtype(code: int):
 
 
 def problem(T, d, d_ff, E, k, capacity_factor=0.0, dtype="bf16", bias_mode=BIAS_NONE, d_ff_shared=0,
-            gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN, pad_rows=0) -> Problem:
+            gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN, pad_rows=0, train=0) -> Problem:
     return Problem(int(T), int(d), int(d_ff), int(E), int(k), float(capacity_factor),
                    _dtype_code(dtype), int(bias_mode), int(d_ff_shared), int(gate_mode), int(drop_order),
-                   int(pad_rows))
+                   int(pad_rows), int(train))
 
 
 def permuted_rows(p: Problem) -> int:
@@ -206,6 +213,35 @@ def forward(p: Problem, x, W_r, W1, W3, W2, out, stats, workspace, bias=None,
                          workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "moe_forward")
     return out
+
+
+def backward_workspace_size(p: Problem) -> int:
+    n = int(_lib().moe_backward_workspace_size(ctypes.byref(p)))
+    if n == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_backward_workspace_size")
+    return n
+
+
+def alloc_backward_workspace(p: Problem, device=None) -> torch.Tensor:
+    return torch.empty(backward_workspace_size(p), dtype=torch.uint8, device=device or "cuda")
+
+
+def backward(p: Problem, x, W_r, W1, W3, W2, dy, dx, dW_r, dW1, dW3, dW2, stats, workspace, bwd_workspace,
+             alpha=0.0, beta=0.0, stream=None):
+    """Gradients of <dy, y> + alpha L_aux + beta L_z after a moe_forward with
+    p.train = 1 on the same workspace; see moe_backward."""
+    rc = _lib().moe_backward(ctypes.byref(p), _ptr(x), _ptr(W_r), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy),
+                             float(alpha), float(beta), _ptr(dx), _ptr(dW_r), _ptr(dW1), _ptr(dW3), _ptr(dW2),
+                             _ptr(stats), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _ptr(bwd_workspace), bwd_workspace.numel() * bwd_workspace.element_size(),
+                             _stream(stream))
+    _check(rc, "moe_backward")
+
+
+def bias_update(p: Problem, stats, bias, gamma, stream=None):
+    """bias[e] -= gamma above the mean load, += gamma below (in place)."""
+    _check(_lib().moe_bias_update(ctypes.byref(p), _ptr(stats), float(gamma), _ptr(bias), _stream(stream)),
+           "moe_bias_update")
 
 
 def route(p: Problem, x, W_r, idx, gate, stats, workspace, bias=None, logits=None, stream=None):

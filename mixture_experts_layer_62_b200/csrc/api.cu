@@ -47,6 +47,7 @@ Layout make_layout(const moe_problem& p) {
     L.o = take(Rmax * d * eb);
     L.hs = take(T * dfs * eb);
     L.s = take(dfs ? T * d * eb : 0);
+    L.ab = take(p.train ? Rmax * 2 * dff * eb : 0);
     const bool split = split_allowed(p);
     L.part13 = take(split ? (size_t)kSplitMax * T * k * (size_t)ceil_div(p.d_ff, 128) * 256 * 4 : 0);
     L.part2 = take(split ? (size_t)kSplitMax * T * k * d * 4 : 0);
@@ -57,6 +58,28 @@ Layout make_layout(const moe_problem& p) {
     L.sem = take(((size_t)L.sem13_n + (size_t)L.sem2_n) * 4);
     L.total = off;
     return L;
+}
+
+BwdLayout make_bwd_layout(const moe_problem& p) {
+    const size_t T = p.T > 0 ? (size_t)p.T : 0, k = (size_t)p.k, E = (size_t)p.E;
+    const size_t d = (size_t)p.d, dff = (size_t)p.d_ff, eb = elem_bytes(p.dtype);
+    const size_t Rmax = (size_t)permuted_rows(p);
+    BwdLayout B;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + (bytes > 0 ? bytes : 1), 256);
+        return o;
+    };
+    B.dO = take(Rmax * d * eb);
+    B.dAB = take(Rmax * 2 * dff * eb);
+    B.dXp = take(Rmax * d * eb);
+    B.dz = take(T * E * 4);
+    B.dgate = take(T * k * 4);
+    B.tiles_dh = take((E + 3) * 4);
+    B.tiles_dx = take((E + 3) * 4);
+    B.total = off;
+    return B;
 }
 
 int pick_split(int tiles, int nkb, int sm, int smax, int rows_q) {
@@ -99,7 +122,7 @@ void fill_split_table(SplitTable& t, int nt13, int nt2, int nkb13, int nkb2, int
 }
 
 bool split_allowed(const moe_problem& p) {
-    return p.dtype == MOE_DTYPE_BF16 && p.d_ff_shared == 0 && p.T > 0 && p.pad_rows == 0 &&
+    return p.dtype == MOE_DTYPE_BF16 && p.d_ff_shared == 0 && p.T > 0 && p.pad_rows == 0 && !p.train &&
            (long long)p.T * p.k <= kSplitMaxRows;
 }
 
@@ -138,6 +161,8 @@ int check_problem(const moe_problem* p) {
     if (p->drop_order == MOE_DROP_SLOT && p->E * p->k > kMaxSlotCounts) return MOE_ERR_UNSUPPORTED;
     if (!std::isfinite(p->capacity_factor)) return MOE_ERR_INVALID_ARG;
     if (p->pad_rows != 0 && p->pad_rows != 64 && p->pad_rows != 128) return MOE_ERR_INVALID_ARG;
+    if (p->train != 0 && p->train != 1) return MOE_ERR_INVALID_ARG;
+    if (p->train && (p->dtype != MOE_DTYPE_BF16 || p->d_ff % 128)) return MOE_ERR_UNSUPPORTED;
     const long long rows = permuted_rows(*p);
     if (rows * (long long)(p->d > p->d_ff ? p->d : p->d_ff) >= (1LL << 40) || rows >= (1LL << 30))
         return MOE_ERR_UNSUPPORTED;
@@ -196,7 +221,8 @@ int run_logits(const moe_problem* p, const void* x, const void* W_r, float* logi
 // Grouped GEMM 1/3 with the SwiGLU epilogue (and the shared expert's).
 int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13, const void* W1,
            const void* W3, const void* x, const void* Ws1, const void* Ws3, void* h, void* hs, int32_t* status,
-           cudaStream_t st, float* part13 = nullptr, int32_t* sem13 = nullptr, bool sched_early = true) {
+           cudaStream_t st, float* part13 = nullptr, int32_t* sem13 = nullptr, bool sched_early = true,
+           void* ab = nullptr) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
     const int arows = (int)permuted_rows(*p);   // rows of the permuted buffers
@@ -212,6 +238,7 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
         a.N[0] = p->d_ff; a.N[1] = p->d_ff_shared;
         a.K[0] = p->d; a.K[1] = p->d;
         a.out[0] = h; a.out[1] = hs;
+        a.ab_out = ab;
         a.status = status;
         if (part13 != nullptr) {
             a.partial = part13;
@@ -281,8 +308,8 @@ int run_experts(const moe_problem* p, const void* xp, const int32_t* indptr, con
                 const int32_t* tiles2, const void* W1, const void* W3, const void* W2, const void* x,
                 const void* Ws1, const void* Ws3, const void* Ws2, void* h, void* hs, void* o, void* s,
                 int32_t* status, cudaStream_t st, float* part13 = nullptr, float* part2 = nullptr,
-                int32_t* sem13 = nullptr, int32_t* sem2 = nullptr, bool sched_early = true) {
-    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st, part13, sem13, sched_early);
+                int32_t* sem13 = nullptr, int32_t* sem2 = nullptr, bool sched_early = true, void* ab = nullptr) {
+    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st, part13, sem13, sched_early, ab);
     if (rc != MOE_OK) return rc;
     return run_down(p, h, indptr, tiles2, W2, hs, Ws2, o, s, status, st, part2, sem2);
 }
@@ -347,11 +374,117 @@ int moe_workspace_layout(const moe_problem* p, moe_workspace_layout_t* out) {
     Layout L = make_layout(*p);
     out->idx = L.idx; out->gate = L.gate; out->pos = L.pos; out->indptr = L.indptr;
     out->row_token = L.row_token; out->logits = L.logits; out->xp = L.xp; out->h = L.h;
-    out->o = L.o; out->hs = L.hs; out->s = L.s; out->total = L.total;
+    out->o = L.o; out->hs = L.hs; out->s = L.s; out->ab = L.ab; out->total = L.total;
     return MOE_OK;
 }
 
 int moe_device_sm_count(void) { return device_sm_count(); }
+
+// ---- backward ----------------------------------------------------------------
+
+size_t moe_backward_workspace_size(const moe_problem* p) {
+    if (check_problem(p) != MOE_OK) return 0;
+    return make_bwd_layout(*p).total;
+}
+
+int moe_backward(const moe_problem* p, const void* x, const void* W_r, const void* W1, const void* W3,
+                 const void* W2, const void* dy, float alpha, float beta, void* dx, float* dW_r, float* dW1,
+                 float* dW3, float* dW2, void* stats, const void* workspace, size_t workspace_bytes,
+                 void* bwd_workspace, size_t bwd_workspace_bytes, void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    if (!p->train || (p->pad_rows != 64 && p->pad_rows != 128) || p->d_ff_shared > 0) return MOE_ERR_UNSUPPORTED;
+    if (!x || !W_r || !W1 || !W3 || !W2 || !dy || !dx || !dW_r || !dW1 || !dW3 || !dW2 || !stats)
+        return MOE_ERR_INVALID_ARG;
+    for (const void* q : {x, W_r, W1, W3, W2, dy, (const void*)dx, (const void*)dW_r, (const void*)dW1,
+                          (const void*)dW3, (const void*)dW2, (const void*)stats})
+        if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(alpha) || !std::isfinite(beta)) return MOE_ERR_INVALID_ARG;
+    const Layout L = make_layout(*p);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    const BwdLayout B = make_bwd_layout(*p);
+    if (!bwd_workspace || bwd_workspace_bytes < B.total || (reinterpret_cast<uintptr_t>(bwd_workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (p->T == 0) {
+        CK(cudaMemsetAsync(dW_r, 0, sizeof(float) * (size_t)p->d * p->E, st));
+        const size_t nw = (size_t)p->E * p->d_ff * p->d * sizeof(float);
+        CK(cudaMemsetAsync(dW1, 0, nw, st));
+        CK(cudaMemsetAsync(dW3, 0, nw, st));
+        CK(cudaMemsetAsync(dW2, 0, nw, st));
+        return MOE_OK;
+    }
+    struct PdlPass {
+        PdlPass() { g_pdl_pass = true; g_pdl = false; }
+        ~PdlPass() { g_pdl_pass = false; g_pdl = false; }
+    } pdl_pass;
+    char* ws = static_cast<char*>(const_cast<void*>(workspace));
+    char* bw = static_cast<char*>(bwd_workspace);
+    const int32_t* pos = reinterpret_cast<const int32_t*>(ws + L.pos);
+    const int32_t* idx = reinterpret_cast<const int32_t*>(ws + L.idx);
+    const float* gate = reinterpret_cast<const float*>(ws + L.gate);
+    const int32_t* indptr = reinterpret_cast<const int32_t*>(ws + L.indptr);
+    const float* logits = reinterpret_cast<const float*>(ws + L.logits);
+    void* dO = bw + B.dO;
+    void* dAB = bw + B.dAB;
+    void* dXp = bw + B.dXp;
+    float* dz = reinterpret_cast<float*>(bw + B.dz);
+    float* dgate = reinterpret_cast<float*>(bw + B.dgate);
+    int32_t* tiles_dh = reinterpret_cast<int32_t*>(bw + B.tiles_dh);
+    int32_t* tiles_dx = reinterpret_cast<int32_t*>(bw + B.tiles_dx);
+    int32_t* status = static_cast<int32_t*>(stats);
+    const int Rmax = (int)permuted_rows(*p);
+
+    CK(launch_bwd_gather(dy, ws + L.o, pos, gate, p->T, p->d, p->k, dO, dgate, st));
+    g_pdl_after_first();
+    CK(launch_pad_fill(p->dtype, indptr, stats, p->E, p->d, dO, nullptr, p->pad_rows, st));
+    CK(launch_router_bwd(logits, idx, gate, dgate, stats, p->T, p->E, p->k, p->gate_mode, alpha, beta, dz, st));
+    CK(launch_dwr(x, dz, p->T, p->d, p->E, dW_r, st));
+    ScheduleSplit nosplit = {};
+    CK(launch_schedule(indptr, p->E, p->T, 0, kTcTileM, ceil_div(p->d_ff, 256), ceil_div(p->d, 256), 0, 0,
+                       tiles_dh, tiles_dx, nosplit, st));
+    BwdGemmArgs g = {};
+    g.indptr = indptr;
+    g.E = p->E;
+    g.d = p->d;
+    g.d_ff = p->d_ff;
+    g.status = status;
+    // dH = dO W2_e, with the SwiGLU derivative in the epilogue -> dAB
+    g.mode = BW_DH; g.tiles = tiles_dh; g.N = p->d_ff; g.K = p->d;
+    g.A = dO; g.a_rows = Rmax; g.a_cols = p->d;
+    g.B0 = W2; g.B1 = nullptr; g.b_rows = p->E * p->d; g.b_cols = p->d_ff;
+    g.ab = ws + L.ab; g.out_bf16 = dAB;
+    CK(launch_bwd_gemm(g, st));
+    // dXp = dA W1_e + dB W3_e
+    g.mode = BW_DX; g.tiles = tiles_dx; g.N = p->d; g.K = 2 * p->d_ff;
+    g.A = dAB; g.a_rows = Rmax; g.a_cols = 2 * p->d_ff;
+    g.B0 = W1; g.B1 = W3; g.b_rows = p->E * p->d_ff; g.b_cols = p->d;
+    g.ab = nullptr; g.out_bf16 = dXp;
+    CK(launch_bwd_gemm(g, st));
+    // dW2_e = dO_e^T H_e
+    g.mode = BW_DW2; g.tiles = nullptr; g.M = p->d; g.N = p->d_ff; g.K = 0;
+    g.A = dO; g.a_rows = Rmax; g.a_cols = p->d;
+    g.B0 = ws + L.h; g.B1 = nullptr; g.b_rows = Rmax; g.b_cols = p->d_ff;
+    g.out_bf16 = nullptr; g.out0 = dW2; g.out1 = nullptr;
+    CK(launch_bwd_gemm(g, st));
+    // [dW1_e; dW3_e] = dAB_e^T Xp_e
+    g.mode = BW_DW13; g.M = 2 * p->d_ff; g.N = p->d;
+    g.A = dAB; g.a_rows = Rmax; g.a_cols = 2 * p->d_ff;
+    g.B0 = ws + L.xp; g.b_rows = Rmax; g.b_cols = p->d;
+    g.out0 = dW1; g.out1 = dW3;
+    CK(launch_bwd_gemm(g, st));
+    CK(launch_bwd_dx(dXp, pos, W_r, dz, p->T, p->d, p->E, p->k, dx, st));
+    return MOE_OK;
+}
+
+int moe_bias_update(const moe_problem* p, const void* stats, float gamma, float* bias, void* stream) {
+    int rc = check_problem(p);
+    if (rc != MOE_OK) return rc;
+    if (!stats || !bias || !aligned16(stats) || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+    CK(launch_bias_update(stats, p->T, p->E, p->k, gamma, bias, static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
+}
 
 int32_t moe_permuted_rows(const moe_problem* p) {
     if (check_problem(p) != MOE_OK) return 0;
@@ -470,7 +603,8 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     // the small router writes the schedule right before GEMM 1/3; the general
     // path writes it in the scan, two launches before
     rc = run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st, part13,
-                     part2, sem, sem ? sem + L.sem13_n : nullptr, /*sched_early=*/!small);
+                     part2, sem, sem ? sem + L.sem13_n : nullptr, /*sched_early=*/!small,
+                     p->train ? wsp(workspace, L.ab) : nullptr);
     if (rc != MOE_OK) return rc;
     CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st));
     return MOE_OK;

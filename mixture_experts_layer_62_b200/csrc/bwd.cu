@@ -1,0 +1,300 @@
+// Backward pass of the MoE layer outside the grouped GEMMs: the gate-scaled
+// gather of the output gradient, the router-logit gradient, the router
+// weight gradient, the input gradient and the auxiliary-loss-free bias
+// update. The loss is L = <dy, y> + alpha L_aux + beta L_z.
+//
+//  * combine y_t = sum_j g_{t,j} o_{t,j} ("Lecture 21 · LLM: Mixture-of-
+//    Experts" §3.2 step 4): dO[pos] = g dy_t, dgate_{t,j} = <dy_t, o_{t,j}>;
+//  * gates, softmax of the selected raw logits ("Week 2 Day 2: Mixture of
+//    Experts" §1.3): dz_{e_j} += g_j (dg_j - sum_l g_l dg_l); full-softmax
+//    gates: dz += p (v - <p, v>), v_{e_j} = dg_j;
+//  * balance loss with f frozen (same page §3.2): dz_{t,i} += alpha E/T
+//    p_{t,i} (f_i - sum_j p_{t,j} f_j); z-loss (§3.4): dz += beta 2/T lse p;
+//  * router z = W_r^T x: dW_r = x^T dz, dx += W_r dz;
+//  * bias update ("Lecture 21" §2.4): above-mean experts b -= gamma, below
+//    b += gamma, decided exactly by the sign of c_e E - T k.
+// Every reduction runs in a fixed order; no atomics.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ float wsum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float wmax(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+constexpr int kWarps = 8;
+
+// One warp per (token, slot): the gate-scaled gradient row and the gate's
+// gradient (lane-strided partial dot products, then a butterfly).
+__global__ void __launch_bounds__(kWarps * 32)
+bwd_gather_kernel(const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ o,
+                  const int32_t* __restrict__ pos, const float* __restrict__ gate, int npairs, int d, int k,
+                  __nv_bfloat16* __restrict__ dO, float* __restrict__ dgate) {
+    pdl_wait();
+    pdl_launch();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int pr = blockIdx.x * kWarps + warp;
+    if (pr >= npairs) return;
+    const int t = pr / k;
+    const int r = pos[pr];
+    if (r < 0) {
+        if (lane == 0) dgate[pr] = 0.f;
+        return;
+    }
+    const float g = gate[pr];
+    const int nvec = d / 8;
+    const uint4* dyv = reinterpret_cast<const uint4*>(dy + static_cast<size_t>(t) * d);
+    const uint4* ov = reinterpret_cast<const uint4*>(o + static_cast<size_t>(r) * d);
+    uint4* dov = reinterpret_cast<uint4*>(dO + static_cast<size_t>(r) * d);
+    float acc = 0.f;
+    for (int v = lane; v < nvec; v += 32) {
+        float a[8], b[8];
+        unpack8(dyv[v], a);
+        unpack8(ov[v], b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc = fmaf(a[i], b[i], acc);
+        dov[v] = make_uint4(pack2(g * a[0], g * a[1]), pack2(g * a[2], g * a[3]), pack2(g * a[4], g * a[5]),
+                            pack2(g * a[6], g * a[7]));
+    }
+    acc = wsum(acc);
+    if (lane == 0) dgate[pr] = acc;
+}
+
+constexpr int kMaxEPL = MOE_MAX_E / 32;   // experts per lane
+
+// One warp per token: softmax of its logits, then the three terms of dz.
+__global__ void __launch_bounds__(kWarps * 32)
+router_bwd_kernel(const float* __restrict__ logits, const int32_t* __restrict__ idx, const float* __restrict__ gate,
+                  const float* __restrict__ dgate, const void* __restrict__ stats, int T, int E, int k,
+                  int gate_mode, float alpha, float beta, float* __restrict__ dz) {
+    pdl_wait();
+    pdl_launch();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kWarps + warp;
+    if (t >= T) return;
+    const float* f = MOE_STATS_F(stats, E);
+    const int epl = (E + 31) / 32;
+    float z[kMaxEPL], p[kMaxEPL], g[kMaxEPL];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMaxEPL; ++i) {
+        const int e = lane + 32 * i;
+        z[i] = (i < epl && e < E) ? logits[static_cast<size_t>(t) * E + e] : -INFINITY;
+        m = fmaxf(m, z[i]);
+    }
+    m = wmax(m);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxEPL; ++i) {
+        const int e = lane + 32 * i;
+        p[i] = (i < epl && e < E) ? expf(z[i] - m) : 0.f;
+        s += p[i];
+    }
+    s = wsum(s);
+    const float inv = 1.f / s;
+#pragma unroll
+    for (int i = 0; i < kMaxEPL; ++i) {
+        p[i] *= inv;
+        g[i] = 0.f;
+    }
+    const int32_t* it = idx + static_cast<size_t>(t) * k;
+    const float* gt = gate + static_cast<size_t>(t) * k;
+    const float* dgt = dgate + static_cast<size_t>(t) * k;
+    if (gate_mode == MOE_GATE_SELECTED) {
+        float sg = 0.f;   // sum_l g_l dg_l, slot order
+        for (int j = 0; j < k; ++j) sg += gt[j] * dgt[j];
+        for (int j = 0; j < k; ++j) {
+            const int e = it[j];
+            if ((e & 31) == lane) {
+                const float add = gt[j] * (dgt[j] - sg);
+#pragma unroll
+                for (int i = 0; i < kMaxEPL; ++i)
+                    if ((e >> 5) == i) g[i] += add;
+            }
+        }
+    } else {
+        float v[kMaxEPL];
+#pragma unroll
+        for (int i = 0; i < kMaxEPL; ++i) v[i] = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const int e = it[j];
+            if ((e & 31) == lane) {
+#pragma unroll
+                for (int i = 0; i < kMaxEPL; ++i)
+                    if ((e >> 5) == i) v[i] += dgt[j];
+            }
+        }
+        float pv = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxEPL; ++i) pv += p[i] * v[i];
+        pv = wsum(pv);
+#pragma unroll
+        for (int i = 0; i < kMaxEPL; ++i) g[i] += p[i] * (v[i] - pv);
+    }
+    if (alpha != 0.f) {
+        float pf = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxEPL; ++i) {
+            const int e = lane + 32 * i;
+            if (i < epl && e < E) pf += p[i] * f[e];
+        }
+        pf = wsum(pf);
+        const float c = alpha * static_cast<float>(E) / static_cast<float>(T);
+#pragma unroll
+        for (int i = 0; i < kMaxEPL; ++i) {
+            const int e = lane + 32 * i;
+            if (i < epl && e < E) g[i] += c * p[i] * (f[e] - pf);
+        }
+    }
+    if (beta != 0.f) {
+        const float lse = m + logf(s);
+        const float c = beta * 2.f / static_cast<float>(T) * lse;
+#pragma unroll
+        for (int i = 0; i < kMaxEPL; ++i) g[i] += c * p[i];
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxEPL; ++i) {
+        const int e = lane + 32 * i;
+        if (i < epl && e < E) dz[static_cast<size_t>(t) * E + e] = g[i];
+    }
+}
+
+// dW_r[i][e] = sum_t x[t][i] dz[t][e]: one thread per (i, e), tokens in order.
+__global__ void __launch_bounds__(256)
+dwr_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dz, int T, int d, int E,
+           float* __restrict__ dW_r) {
+    pdl_wait();
+    pdl_launch();
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const int e = blockIdx.y;
+    if (i >= d) return;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < T; ++t)
+        acc = fmaf(__bfloat162float(x[static_cast<size_t>(t) * d + i]), dz[static_cast<size_t>(t) * E + e], acc);
+    dW_r[static_cast<size_t>(i) * E + e] = acc;
+}
+
+// dx_t = sum_j dXp[pos_{t,j}] + W_r dz_t: one warp per (token, 256-wide
+// slice); the token's dz row is staged in shared memory.
+__global__ void __launch_bounds__(kWarps * 32)
+bwd_dx_kernel(const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__ pos,
+              const __nv_bfloat16* __restrict__ W_r, const float* __restrict__ dz, int T, int d, int E, int k,
+              int slices, __nv_bfloat16* __restrict__ dx) {
+    __shared__ float dzs[kWarps][MOE_MAX_E];
+    pdl_wait();
+    pdl_launch();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long task = static_cast<long long>(blockIdx.x) * kWarps + warp;
+    const int t = static_cast<int>(task / slices), sl = static_cast<int>(task % slices);
+    if (t >= T) return;
+    for (int e = lane; e < E; e += 32) dzs[warp][e] = dz[static_cast<size_t>(t) * E + e];
+    __syncwarp();
+    const int v = sl * 32 + lane;   // 8 consecutive columns
+    if (v >= d / 8) return;
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    for (int j = 0; j < k; ++j) {
+        const int r = pos[static_cast<size_t>(t) * k + j];
+        if (r < 0) continue;
+        float a[8];
+        unpack8(reinterpret_cast<const uint4*>(dXp + static_cast<size_t>(r) * d)[v], a);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] += a[c];
+    }
+    // router term, rows 8v .. 8v+7 of W_r [d][E], experts in order
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const __nv_bfloat16* wrow = W_r + static_cast<size_t>(8 * v + c) * E;
+        float s = 0.f;
+        if ((E & 7) == 0) {
+            for (int e = 0; e < E; e += 8) {
+                float w[8];
+                unpack8(*reinterpret_cast<const uint4*>(wrow + e), w);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) s = fmaf(w[q], dzs[warp][e + q], s);
+            }
+        } else {
+            for (int e = 0; e < E; ++e) s = fmaf(__bfloat162float(wrow[e]), dzs[warp][e], s);
+        }
+        acc[c] += s;
+    }
+    reinterpret_cast<uint4*>(dx + static_cast<size_t>(t) * d)[v] =
+        make_uint4(pack2(acc[0], acc[1]), pack2(acc[2], acc[3]), pack2(acc[4], acc[5]), pack2(acc[6], acc[7]));
+}
+
+__global__ void bias_update_kernel(const void* __restrict__ stats, int T, int E, int k, float gamma,
+                                   float* __restrict__ bias) {
+    pdl_wait();
+    pdl_launch();
+    const int32_t* c = MOE_STATS_COUNTS(stats, E);
+    const long long tk = static_cast<long long>(T) * k;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const long long s = static_cast<long long>(c[e]) * E - tk;   // sign of c_e - T k / E, exactly
+        if (s > 0) bias[e] -= gamma;
+        else if (s < 0) bias[e] += gamma;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_gather(const void* dy, const void* o, const int32_t* pos, const float* gate, int T, int d,
+                              int k, void* dO, float* dgate, cudaStream_t st) {
+    const int np = T * k;
+    if (np == 0) return cudaSuccess;
+    return launch_k(bwd_gather_kernel, dim3(ceil_div(np, kWarps)), dim3(kWarps * 32), 0, st,
+                    static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(o), pos, gate, np, d, k,
+                    static_cast<__nv_bfloat16*>(dO), dgate);
+}
+
+cudaError_t launch_router_bwd(const float* logits, const int32_t* idx, const float* gate, const float* dgate,
+                              const void* stats, int T, int E, int k, int gate_mode, float alpha, float beta,
+                              float* dz, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    return launch_k(router_bwd_kernel, dim3(ceil_div(T, kWarps)), dim3(kWarps * 32), 0, st, logits, idx, gate, dgate,
+                    stats, T, E, k, gate_mode, alpha, beta, dz);
+}
+
+cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* dW_r, cudaStream_t st) {
+    return launch_k(dwr_kernel, dim3(ceil_div(d, 256), E), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x),
+                    dz, T, d, E, dW_r);
+}
+
+cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, int T, int d,
+                          int E, int k, void* dx, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int slices = ceil_div(d / 8, 32);
+    const long long tasks = static_cast<long long>(T) * slices;
+    return launch_k(bwd_dx_kernel, dim3(static_cast<unsigned>((tasks + kWarps - 1) / kWarps)), dim3(kWarps * 32), 0,
+                    st, static_cast<const __nv_bfloat16*>(dXp), pos, static_cast<const __nv_bfloat16*>(W_r), dz, T,
+                    d, E, k, slices, static_cast<__nv_bfloat16*>(dx));
+}
+
+cudaError_t launch_bias_update(const void* stats, int T, int E, int k, float gamma, float* bias, cudaStream_t st) {
+    return launch_k(bias_update_kernel, dim3(1), dim3(512), 0, st, stats, T, E, k, gamma, bias);
+}
+
+}  // namespace moe

@@ -61,6 +61,7 @@ struct Layout {
     size_t idx, gate, pos, indptr, row_token, logits, wrt;
     size_t blockcnt, blockoff, blockpsum, blockextra, tiles13, tiles2;
     size_t xp, h, o, hs, s;
+    size_t ab;              // gate/up pre-activations kept for the backward (train)
     size_t part13, part2;   // fp32 split-K partials (small-T forward only)
     size_t sem;             // split-K arrival counters: [sem13_n] then [sem2_n]
     int sem13_n, sem2_n;
@@ -77,6 +78,11 @@ bool split_allowed(const moe_problem& p);
 Layout make_layout(const moe_problem& p);
 // Rows a permuted buffer holds: T*k, plus E*(pad_rows-1) when rows are padded.
 long long permuted_rows(const moe_problem& p);
+// Byte offsets of the backward pass's own workspace.
+struct BwdLayout {
+    size_t dO, dAB, dXp, dz, dgate, tiles_dh, tiles_dx, total;
+};
+BwdLayout make_bwd_layout(const moe_problem& p);
 
 // Split factors by the number of active experts (0 .. kSplitMaxRows): with at
 // most kSplitMaxRows rows every active expert is one M-block, so a GEMM has
@@ -217,12 +223,45 @@ struct TcArgs {
     long long partial_stride;  // elements between splits
     int partial_ld;            // elements per row
     int32_t* sem;              // split-K arrival counters [tiles][kSemPerTile] (with partial)
+    void* ab_out;              // SWIGLU, routed groups: also store the raw gate/up
+                               // accumulators as bf16 [rows][2 N] (null: not kept)
     // the tile schedule (indptr, tiles) was written two or more launches
     // back, so the weight loads of the first stages may start before the
     // dependency wait
     int b_before_wait;
 };
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
+// Backward grouped GEMMs (tcgen05): see gemm_bwd_sm100.cu.
+enum BwMode { BW_DH = 0, BW_DX = 1, BW_DW2 = 2, BW_DW13 = 3 };
+struct BwdGemmArgs {
+    int mode;
+    const int32_t* indptr;   // padded group row offsets [E+1]
+    const int32_t* tiles;    // BW_DH / BW_DX tile schedule [E+1] (null for the weight gradients)
+    int E, M, N, K, d, d_ff;
+    const void* A; int a_rows, a_cols;         // A operand matrix (row-major)
+    const void* B0; const void* B1; int b_rows, b_cols;   // B operand matrices (B1: W3 for BW_DX)
+    const void* ab;          // BW_DH: forward gate/up pre-activations
+    void* out_bf16;          // BW_DH: dAB; BW_DX: dXp
+    float* out0; float* out1;   // weight gradients
+    int32_t* status;
+};
+cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, cudaStream_t st);
+
+// Backward elementwise and reduction kernels: see bwd.cu.
+cudaError_t launch_bwd_gather(const void* dy, const void* o, const int32_t* pos, const float* gate, int T, int d,
+                              int k, void* dO, float* dgate, cudaStream_t st);
+cudaError_t launch_router_bwd(const float* logits, const int32_t* idx, const float* gate, const float* dgate,
+                              const void* stats, int T, int E, int k, int gate_mode, float alpha, float beta,
+                              float* dz, cudaStream_t st);
+cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* dW_r, cudaStream_t st);
+cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, int T, int d,
+                          int E, int k, void* dx, cudaStream_t st);
+cudaError_t launch_bias_update(const void* stats, int T, int E, int k, float gamma, float* bias, cudaStream_t st);
+
+// A cached 2-D bf16 tensor map over a row-major [rows, cols] matrix: box 64
+// columns x box_rows rows, 128-byte swizzle, zeros outside (CUtensorMap is
+// the driver type; passed as void* so this header needs no driver header).
+bool make_tmap(void* map, const void* base, int rows, int cols, int box_rows);
 
 int device_sm_count();
 

@@ -34,10 +34,13 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace moe {
 
 namespace {
+
+using namespace tc;
 
 constexpr int BM = 128;
 constexpr int BK = 64;                       // 64 bf16 = 128 bytes = one swizzle row
@@ -50,100 +53,6 @@ constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int NUM_THREADS = 192;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-
-// ---- PTX wrappers -----------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_timer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-        : "memory");
-}
-__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// 32 consecutive fp32 columns of this thread's TMEM lane; the wait is in the
-// same statement so no register is read before the load has landed.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
-// 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), descriptor
-// version 1, tile base 1024-byte aligned (base offset 0).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-    d |= static_cast<uint64_t>(1) << 16;              // leading byte offset (ignored for SW128 K-major)
-    d |= static_cast<uint64_t>(1024 >> 4) << 32;      // stride byte offset
-    d |= static_cast<uint64_t>(1) << 46;              // version
-    d |= static_cast<uint64_t>(2) << 61;              // SWIZZLE_128B
-    return d;
-}
-// Instruction descriptor of kind::f16: bf16 A and B, fp32 D, both K-major.
-constexpr uint32_t make_idesc(int M, int N) {
-    return (1u << 4)      // D format fp32
-         | (1u << 7)      // A format bf16
-         | (1u << 10)     // B format bf16
-         | (static_cast<uint32_t>(N >> 3) << 17)
-         | (static_cast<uint32_t>(M >> 4) << 24);
-}
 
 struct KParams {
     const int32_t* indptr;
@@ -159,6 +68,7 @@ struct KParams {
     long long partial_stride;  // elements between splits
     int partial_ld;            // elements per partial row
     int32_t* sem;              // split-K arrival counters [tile][kSemPerTile]
+    __nv_bfloat16* ab_out;     // SWIGLU: raw gate/up accumulators of routed rows, or null
     int b_before_wait;         // weight tiles of the first stages may load before the dependency wait
 };
 
@@ -539,12 +449,32 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                 if (t.m_blk * BM + q * 32 < t.rows) splitk_finish<MODE>(p, t, q, lane, nsplit, u / nsplit);
             } else if (MODE == TC_SWIGLU) {
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
+                // training: the gate and up pre-activations of the tile, in the
+                // accumulator's own column order ([128 gate | 128 up] per tile)
+                __nv_bfloat16* abrow = (p.ab_out != nullptr && t.kind == 0)
+                                           ? p.ab_out + orow * (2 * static_cast<size_t>(N)) + t.n_blk * 256
+                                           : nullptr;
 #pragma unroll 1
                 for (int c = 0; c < 128; c += 32) {
                     uint32_t gv[32], uv[32];
                     tmem_ld32(tb + c, gv);
                     tmem_ld32(tb + 128 + c, uv);
                     const int col = t.n_blk * 128 + c;
+                    if (valid && col < N && abrow != nullptr) {
+                        uint32_t pg[16], pu[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            pg[i] = pack_bf16(__uint_as_float(gv[2 * i]), __uint_as_float(gv[2 * i + 1]));
+                            pu[i] = pack_bf16(__uint_as_float(uv[2 * i]), __uint_as_float(uv[2 * i + 1]));
+                        }
+                        uint4* dg = reinterpret_cast<uint4*>(abrow + c);
+                        uint4* du = reinterpret_cast<uint4*>(abrow + 128 + c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            dg[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+                            du[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+                        }
+                    }
                     if (valid && col < N) {
                         uint32_t packed[16];
 #pragma unroll
@@ -627,15 +557,15 @@ bool get_encode() {
     return g_encode != nullptr;
 }
 
-// 2-D bf16 map over a [rows, cols] row-major matrix, box 64 columns x 128 rows,
-// 128-byte swizzle; reads outside the matrix return zeros.
-bool encode_map(CUtensorMap* m, const void* base, int rows, int cols);
+// 2-D bf16 map over a [rows, cols] row-major matrix, box 64 columns x
+// box_rows rows, 128-byte swizzle; reads outside the matrix return zeros.
+bool encode_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows);
 
 // Encoded maps keyed by (base, rows, cols): the same key always encodes to the
 // same map, so a hit is exactly a fresh encode, without the driver call.
 struct MapCacheEntry {
     const void* base;
-    int rows, cols;
+    int rows, cols, box_rows;
     CUtensorMap map;
 };
 constexpr int kMapCacheSize = 64;
@@ -643,33 +573,34 @@ MapCacheEntry g_map_cache[kMapCacheSize];
 int g_map_cache_n = 0, g_map_cache_next = 0;
 std::mutex g_map_cache_mu;
 
-bool make_map(CUtensorMap* m, const void* base, int rows, int cols) {
+bool make_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows = 128) {
     {
         std::lock_guard<std::mutex> lk(g_map_cache_mu);
         for (int i = 0; i < g_map_cache_n; ++i) {
             const MapCacheEntry& c = g_map_cache[i];
-            if (c.base == base && c.rows == rows && c.cols == cols) {
+            if (c.base == base && c.rows == rows && c.cols == cols && c.box_rows == box_rows) {
                 *m = c.map;
                 return true;
             }
         }
     }
-    if (!encode_map(m, base, rows, cols)) return false;
+    if (!encode_map(m, base, rows, cols, box_rows)) return false;
     std::lock_guard<std::mutex> lk(g_map_cache_mu);
     MapCacheEntry& c = g_map_cache[g_map_cache_next];
     c.base = base;
     c.rows = rows;
     c.cols = cols;
+    c.box_rows = box_rows;
     c.map = *m;
     g_map_cache_next = (g_map_cache_next + 1) % kMapCacheSize;
     if (g_map_cache_n < kMapCacheSize) ++g_map_cache_n;
     return true;
 }
 
-bool encode_map(CUtensorMap* m, const void* base, int rows, int cols) {
+bool encode_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    cuuint32_t box[2] = {BK, 128};
+    cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -697,6 +628,10 @@ cudaError_t launch_mode(const TcArgs& a, const KParams& kp, const CUtensorMap (&
 }  // namespace
 
 int tc_out_cols_per_tile(int mode) { return mode == TC_SWIGLU ? 128 : 256; }
+
+bool make_tmap(void* m, const void* base, int rows, int cols, int box_rows) {
+    return get_encode() && make_map(static_cast<CUtensorMap*>(m), base, rows, cols, box_rows);
+}
 
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     if (!get_encode()) return cudaErrorNotSupported;
@@ -734,6 +669,7 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     kp.partial_stride = a.partial_stride;
     kp.partial_ld = a.partial_ld;
     kp.sem = a.sem;
+    kp.ab_out = static_cast<__nv_bfloat16*>(a.ab_out);
     kp.b_before_wait = a.b_before_wait;
     if (kp.partial != nullptr && kp.sem == nullptr) return cudaErrorInvalidValue;
     switch (a.mode) {

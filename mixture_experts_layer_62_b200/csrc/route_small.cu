@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(const __gr
 }  // namespace
 
 bool small_route_ok(const moe_problem& p) {
-    return p.dtype == MOE_DTYPE_BF16 && p.d_ff_shared == 0 && p.pad_rows == 0 && p.T > 0 &&
+    return p.dtype == MOE_DTYPE_BF16 && p.d_ff_shared == 0 && p.pad_rows == 0 && !p.train && p.T > 0 &&
            (long long)p.T * p.k <= kSmallMaxPairs &&
            p.E <= kSmallMaxE && p.E % 8 == 0 && p.d % 8 == 0;
 }

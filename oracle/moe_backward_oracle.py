@@ -127,7 +127,7 @@ class BackwardResult:
 
 def moe_backward(x, W_r, W1, W3, W2, k, dy, capacity_factor=0.0, bias=None, bias_mode=O.BIAS_NONE,
                  Ws1=None, Ws3=None, Ws2=None, alpha=0.0, beta=0.0, gate_mode=O.GATE_SELECTED,
-                 drop_order=O.DROP_TOKEN, logits=None, key_dtype=np.float64):
+                 drop_order=O.DROP_TOKEN, logits=None, key_dtype=np.float64, idx=None):
     """Gradients of L = <dy, y> + alpha L_aux + beta L_z w.r.t. x, W_r and the
     expert weights. ``W1``, ``W3``, ``W2`` are indexable by expert."""
     x = np.asarray(x, dtype=np.float64)
@@ -135,7 +135,7 @@ def moe_backward(x, W_r, W1, W3, W2, k, dy, capacity_factor=0.0, bias=None, bias
     T, d = x.shape
     W_r64 = None if W_r is None else np.asarray(W_r, dtype=np.float64)
     fwd = O.moe_forward(x, W_r, W1, W3, W2, k, capacity_factor, bias, bias_mode, logits=logits,
-                        key_dtype=key_dtype, gate_mode=gate_mode, drop_order=drop_order)
+                        key_dtype=key_dtype, gate_mode=gate_mode, drop_order=drop_order, idx=idx)
     idx, gate = fwd.routing.idx, fwd.routing.gate
     pos = fwd.perm.pos
     keep = pos >= 0

@@ -426,7 +426,7 @@ class ForwardResult:
 def moe_forward(x, W_r, W1, W3, W2, k, capacity_factor=0.0, bias=None,
                 bias_mode=BIAS_NONE, Ws1=None, Ws3=None, Ws2=None,
                 logits=None, tokens=None, key_dtype=np.float64,
-                gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN, pad=None):
+                gate_mode=GATE_SELECTED, drop_order=DROP_TOKEN, pad=None, idx=None):
     """Forward pass of one MoE layer, the sparse per-pair definition.
 
     Steps in the order of [CMU 15-779 L21] §3.2 (route, permute, compute per
@@ -441,6 +441,8 @@ def moe_forward(x, W_r, W1, W3, W2, k, capacity_factor=0.0, bias=None,
        §2.1.3b).
 
     ``W1``, ``W3``, ``W2`` are indexable by expert (``W1[e]`` -> [d_ff, d]);
+    ``idx`` [T, k], when given, replaces the top-k selection (for checking a
+    selection made by another implementation from the same logits);
     ``tokens`` restricts step 4-5 to a subset of tokens (routing, permutation
     and statistics always cover all tokens). Returns a ForwardResult whose
     ``y`` rows follow ``tokens``.
@@ -454,7 +456,10 @@ def moe_forward(x, W_r, W1, W3, W2, k, capacity_factor=0.0, bias=None,
     else:
         z_key = z
     key = selection_key(z_key, bias, bias_mode, dtype=key_dtype)
-    idx = topk_lowest_index(key, k)
+    if idx is None:
+        idx = topk_lowest_index(key, k)
+    else:   # a selection decided elsewhere (the gates still follow from z)
+        idx = np.asarray(idx, dtype=np.int64)
     gate = gates_from_selected(z, idx) if gate_mode == GATE_SELECTED else gates_full_softmax(z, idx)
     probs = softmax_rows(z)
     routing = Routing(idx=idx, gate=gate, probs=probs, key=key)

@@ -1,0 +1,184 @@
+"""GPU parity of the backward pass (moe_backward, moe_bias_update) against
+the backward oracle, on the GPU forward's own routing (the oracle consumes
+the GPU's fp32 logits, so both sides differentiate the same selection)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_62_b200 as moe
+from oracle import moe_oracle as O
+from oracle import moe_backward_oracle as B
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+# Acceptance bars for bf16 gradients. The GPU path rounds five intermediates
+# to bf16 (dO = g dy, the gate/up pre-activations a and b, dA and dB, dXp),
+# each a relative error <= 2^-9 per element, and accumulates every GEMM in
+# fp32; two chained rounding steps on the dx path and one on the weight
+# gradients give a few 1e-3 relative on a token's dx row and on an expert's
+# weight-gradient matrix. A single hidden unit's row of dW1 / dW3 of an
+# expert with a handful of rows can be a near-cancelled sum (dH = dO W2 with
+# dO rounded), so its own relative error is not bounded by the rounding and
+# is not a bar. Bars: every token's dx row within 3e-2 (L2, rows with a
+# nonzero reference), every expert's dW1, dW3, dW2 and dW_r as a whole within
+# 2e-2 (Frobenius), every whole tensor within 1e-2.
+TOL_ROW = 3e-2
+TOL_MAT = 2e-2
+TOL_ALL = 1e-2
+
+
+def _layer(cfg, seed):
+    g = torch.Generator().manual_seed(seed)
+    T, d, dff, E = cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"]
+    bf = torch.bfloat16
+    L = dict(x=torch.randn((T, d), generator=g).to(bf),
+             W_r=(torch.randn((d, E), generator=g) / math.sqrt(d)).to(bf),
+             W1=(torch.randn((E, dff, d), generator=g) / math.sqrt(d)).to(bf),
+             W3=(torch.randn((E, dff, d), generator=g) / math.sqrt(d)).to(bf),
+             W2=(torch.randn((E, d, dff), generator=g) / math.sqrt(dff)).to(bf),
+             dy=torch.randn((T, d), generator=g).to(bf), bias=None)
+    if cfg.get("bias_mode", 0) == O.BIAS_LOGIT:
+        L["bias"] = torch.linspace(0.5, -0.5, E)
+    elif cfg.get("bias_mode", 0) == O.BIAS_PROB:
+        L["bias"] = torch.rand((E,), generator=g) * 0.2 - 0.1
+    return L
+
+
+def _problem(cfg):
+    return moe.problem(cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg.get("cf", 0.0), "bf16",
+                       cfg.get("bias_mode", 0), 0, cfg.get("gate", 0), cfg.get("drop", 0),
+                       pad_rows=cfg["pad"], train=1)
+
+
+def _gpu(cfg, L):
+    p = _problem(cfg)
+    D = {k_: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k_, v in L.items()}
+    T, d, dff, E = cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"]
+    ws = moe.alloc_workspace(p, DEV)
+    st = moe.alloc_stats(E, DEV)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
+    moe.forward(p, D["x"], D["W_r"], D["W1"], D["W3"], D["W2"], out, st, ws, bias=D["bias"])
+    bws = moe.alloc_backward_workspace(p, DEV)
+    G = dict(dx=torch.full((T, d), float("nan"), dtype=torch.bfloat16, device=DEV),
+             dW_r=torch.full((d, E), float("nan"), device=DEV),
+             dW1=torch.full((E, dff, d), float("nan"), device=DEV),
+             dW3=torch.full((E, dff, d), float("nan"), device=DEV),
+             dW2=torch.full((E, d, dff), float("nan"), device=DEV))
+    moe.backward(p, D["x"], D["W_r"], D["W1"], D["W3"], D["W2"], D["dy"], G["dx"], G["dW_r"], G["dW1"],
+                 G["dW3"], G["dW2"], st, ws, bws, alpha=cfg.get("alpha", 0.0), beta=cfg.get("beta", 0.0))
+    torch.cuda.synchronize()
+    assert moe.read_stats(st, E).status == moe.MOE_OK
+    logits = moe.workspace_view(ws, p, "logits").cpu().numpy()
+    G["idx"] = moe.workspace_view(ws, p, "idx").cpu().numpy()
+    return p, ws, st, {k_: (v.float().cpu().numpy() if isinstance(v, torch.Tensor) else v) for k_, v in G.items()}, logits
+
+
+def _oracle(cfg, L, logits, idx):
+    """The oracle's gradients for the GPU's logits and selection (softmax-plus-
+    bias keys are formed with each side's exp, so near-ties could pick other
+    experts; the selection is a discrete input of the backward, not part of
+    what it differentiates). Where the oracle's own selection is exact (no
+    softmax key), it must equal the GPU's."""
+    f = lambda t: t.float().numpy()
+    exact = cfg.get("bias_mode", 0) != O.BIAS_PROB
+    bias = None if L["bias"] is None else L["bias"].numpy()
+    if exact:
+        own = O.route(logits, cfg["k"], bias, cfg.get("bias_mode", 0), key_dtype=np.float32)
+        assert np.array_equal(own.idx, idx)
+    return B.moe_backward(f(L["x"]), f(L["W_r"]), f(L["W1"]), f(L["W3"]), f(L["W2"]), cfg["k"], f(L["dy"]),
+                          cfg.get("cf", 0.0), bias, cfg.get("bias_mode", 0), alpha=cfg.get("alpha", 0.0),
+                          beta=cfg.get("beta", 0.0), gate_mode=cfg.get("gate", 0), drop_order=cfg.get("drop", 0),
+                          logits=logits, key_dtype=np.float32 if exact else np.float64, idx=idx)
+
+
+def _compare(name, got, ref, per_matrix=False):
+    """Rows (dx: tokens) or whole matrices (per expert) against the bars; a
+    zero reference must be matched exactly."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.isfinite(got).all(), name
+    if per_matrix:
+        got = got.reshape(got.shape[0], -1)
+        ref = ref.reshape(ref.shape[0], -1)
+    nr = np.linalg.norm(ref, axis=1)
+    nz = nr > 0
+    zero_rows = np.abs(got[~nz]).max() if (~nz).any() else 0.0
+    assert zero_rows == 0.0, (name, "a zero reference must be matched exactly", zero_rows)
+    worst = float(np.max(np.linalg.norm(got[nz] - ref[nz], axis=1) / nr[nz])) if nz.any() else 0.0
+    tot = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    assert worst < (TOL_MAT if per_matrix else TOL_ROW) and tot < TOL_ALL, (name, worst, tot)
+    return worst, tot
+
+
+CASES = [
+    dict(T=300, d=256, d_ff=256, E=8, k=2, pad=128, alpha=0.01, beta=0.001),
+    dict(T=1000, d=512, d_ff=1024, E=8, k=2, cf=0.8, pad=64, bias_mode=O.BIAS_LOGIT, alpha=0.1),
+    dict(T=200, d=256, d_ff=384, E=16, k=4, cf=0.9, pad=128, gate=O.GATE_FULL, drop=O.DROP_SLOT,
+         alpha=0.05, beta=0.01),
+    dict(T=64, d=128, d_ff=128, E=32, k=2, pad=64, bias_mode=O.BIAS_PROB),
+]
+
+
+@pytest.mark.parametrize("cfg", CASES, ids=[f"T{c['T']}_d{c['d']}_f{c['d_ff']}_E{c['E']}_k{c['k']}_p{c['pad']}"
+                                            for c in CASES])
+def test_backward_matches_oracle(cfg):
+    L = _layer(cfg, seed=cfg["T"] + cfg["E"])
+    p, ws, st, G, logits = _gpu(cfg, L)
+    ref = _oracle(cfg, L, logits, G["idx"])
+    _compare("dx", G["dx"], ref.dx)
+    _compare("dW_r", G["dW_r"][None], ref.dW_r[None], per_matrix=True)
+    for n in ("dW1", "dW3", "dW2"):
+        _compare(n, G[n], getattr(ref, n), per_matrix=True)
+    # experts that received no rows get exactly zero weight gradients
+    s = moe.read_stats(st, cfg["E"])
+    for e, kept in enumerate(s.kept):
+        if kept == 0:
+            assert not G["dW1"][e].any() and not G["dW2"][e].any()
+
+
+def test_backward_is_deterministic():
+    cfg = CASES[1]
+    L = _layer(cfg, seed=3)
+    a = _gpu(cfg, L)[3]
+    b = _gpu(cfg, L)[3]
+    for n in a:
+        assert np.array_equal(a[n], b[n]), n
+
+
+def test_backward_rejects_unsupported_problems():
+    cfg = dict(CASES[0])
+    L = _layer(cfg, seed=1)
+    for bad in (dict(pad=0), dict(train=0)):
+        c = dict(cfg, **bad)
+        p = moe.problem(c["T"], c["d"], c["d_ff"], c["E"], c["k"], 0.0, "bf16", pad_rows=c["pad"],
+                        train=c.get("train", 1))
+        ws = moe.alloc_workspace(p, DEV)
+        st = moe.alloc_stats(c["E"], DEV)
+        bws = torch.empty(1 << 20, dtype=torch.uint8, device=DEV)
+        z = torch.zeros(1, device=DEV)
+        with pytest.raises(moe.MoEError) as ei:
+            moe.backward(p, *(t.to(DEV) for t in (L["x"], L["W_r"], L["W1"], L["W3"], L["W2"], L["dy"], L["x"])),
+                         z, z, z, z, st, ws, bws)
+        assert ei.value.code == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_bias_update_matches_the_rule_exactly():
+    cfg = dict(T=333, d=128, d_ff=128, E=16, k=2, pad=64)
+    L = _layer(cfg, seed=9)
+    p, ws, st, _, _ = _gpu(cfg, L)
+    counts = np.array(moe.read_stats(st, cfg["E"]).counts)
+    b0 = torch.randn(cfg["E"]) * 0.01
+    bias = b0.clone().to(DEV)
+    moe.bias_update(p, st, bias, 0.001)
+    torch.cuda.synchronize()
+    # fp32 on both sides: b - gamma, b + gamma or b, by the sign of c E - T k
+    s = np.sign(counts * cfg["E"] - cfg["T"] * cfg["k"])
+    want = np.where(s > 0, b0.numpy() - np.float32(0.001),
+                    np.where(s < 0, b0.numpy() + np.float32(0.001), b0.numpy())).astype(np.float32)
+    assert np.array_equal(bias.cpu().numpy(), want)
+    ref = B.bias_update(b0.numpy().astype(np.float64), counts, 0.001, cfg["T"], cfg["k"])
+    assert np.allclose(bias.cpu().numpy(), ref, atol=1e-7)
