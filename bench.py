@@ -308,6 +308,8 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=16, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the forward eagerly in the timed loop")
+    ap.add_argument("--train", action="store_true",
+                    help="time a training step (forward + backward) instead of the forward")
     ap.add_argument("--pad-rows", type=int, default=0, choices=[0, 64, 128],
                     help="pad every expert's rows to a multiple of this (the MegaBlocks layout), for comparison")
     args = ap.parse_args()
@@ -349,6 +351,11 @@ def main():
     E = cfg["E"]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if args.train:
+        if world > 1:
+            raise SystemExit("--train runs on one GPU")
+        run_train(args, cfg, moe, L, dev, stream, flush)
+        return
 
     # the forward is captured once in a CUDA graph and replayed (the library's
     # launches are asynchronous and allocation-free, so they capture as is)
@@ -483,6 +490,91 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def run_train(args, cfg, moe, L, dev, stream, flush):
+    """Training step: forward with the pre-activations kept, then the backward
+    of <dy, y> + alpha L_aux + beta L_z (both captured in one CUDA graph),
+    on the padded-row layout the backward needs; rank 0 prints one JSON line."""
+    T, d, dff, E, k = cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"]
+    pad = args.pad_rows or 128
+    p = moe.problem(T, d, dff, E, k, cfg["cf"], cfg["dtype"], cfg["bias_mode"], cfg["d_ff_shared"],
+                    pad_rows=pad, train=1)
+    ws = moe.alloc_workspace(p, dev)
+    st = moe.alloc_stats(E, dev)
+    bws = moe.alloc_backward_workspace(p, dev)
+    out = torch.empty((T, d), dtype=L["x"].dtype, device=dev)
+    g = torch.Generator().manual_seed(1)
+    dy = torch.randn((T, d), generator=g).to(L["x"].dtype).to(dev)
+    dx = torch.empty_like(L["x"])
+    dW_r = torch.empty((d, E), device=dev)
+    dW1 = torch.empty((E, dff, d), device=dev)
+    dW3 = torch.empty((E, dff, d), device=dev)
+    dW2 = torch.empty((E, d, dff), device=dev)
+
+    def fwd():
+        moe.forward(p, L["x"], L["W_r"], L["W1"], L["W3"], L["W2"], out, st, ws, bias=L["bias"])
+
+    def bwd():
+        moe.backward(p, L["x"], L["W_r"], L["W1"], L["W3"], L["W2"], dy, dx, dW_r, dW1, dW3, dW2, st, ws, bws,
+                     alpha=0.01, beta=0.001)
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    graphs = {}
+    for name, fn in (("step", lambda: (fwd(), bwd())), ("fwd", fwd), ("bwd", bwd)):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        graphs[name] = gr
+    torch.cuda.synchronize(dev)
+
+    def timed(gr, n):
+        evs = []
+        for _ in range(n):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            gr.replay()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in evs) / n
+
+    for _ in range(3):
+        graphs["step"].replay()
+    sampler = ClockSampler(gpu_index_for(0))
+    sampler.start()
+    step_ms = timed(graphs["step"], args.steps)
+    clocks = sampler.stop()
+    fwd_ms = timed(graphs["fwd"], max(3, args.steps // 3))
+    bwd_ms = timed(graphs["bwd"], max(3, args.steps // 3))
+    s = moe.read_stats(st, E)
+    if s.status != moe.MOE_OK:
+        raise SystemExit(f"device status {s.status}: {moe.error_string(s.status)}")
+    R = s.rows
+    fl_fwd = flops_per_step(cfg, R)
+    # backward: dH and dXp (2 R d d_ff + 4 R d d_ff), dW2 and [dW1; dW3] (the same), router 2 x 2 T d E
+    fl_bwd = 2.0 * (2.0 * R * d * dff + 4.0 * R * d * dff) + 4.0 * T * d * E
+    peaks, peak_src = load_peaks()
+    tf_step = (fl_fwd + fl_bwd) / (step_ms / 1e3) / 1e12
+    line = {
+        "metric": "MoE-layer training step (fwd+bwd) tokens/s & TFLOP/s vs bf16 peak", "impl": "ours",
+        "value": T / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": dict(config_of(cfg, args), pad_rows=pad, train=1, alpha=0.01, beta=0.001),
+        "tflops": tf_step, "tflops_frac_of_peak": tf_step / peaks["bf16_tflops"],
+        "tflops_frac_of_sustained": tf_step / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+        "peak_source": peak_src,
+        "forward": {"ms": fwd_ms, "tflops": fl_fwd / (fwd_ms / 1e3) / 1e12},
+        "backward": {"ms": bwd_ms, "tflops": fl_bwd / (bwd_ms / 1e3) / 1e12},
+        "gpu_launches": (launches_per_forward(cfg, pad) + 10) * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
 
 
 def breakdown(moe, p, cfg, L, dev, stream, flush, iters):

@@ -78,6 +78,7 @@ BwdLayout make_bwd_layout(const moe_problem& p) {
     B.dgate = take(T * k * 4);
     B.tiles_dh = take((E + 3) * 4);
     B.tiles_dx = take((E + 3) * 4);
+    B.dwr_part = take((size_t)ceil_div((int)T, 128) * d * E * 4);
     B.total = off;
     return B;
 }
@@ -440,7 +441,7 @@ int moe_backward(const moe_problem* p, const void* x, const void* W_r, const voi
     g_pdl_after_first();
     CK(launch_pad_fill(p->dtype, indptr, stats, p->E, p->d, dO, nullptr, p->pad_rows, st));
     CK(launch_router_bwd(logits, idx, gate, dgate, stats, p->T, p->E, p->k, p->gate_mode, alpha, beta, dz, st));
-    CK(launch_dwr(x, dz, p->T, p->d, p->E, dW_r, st));
+    CK(launch_dwr(x, dz, p->T, p->d, p->E, reinterpret_cast<float*>(bw + B.dwr_part), dW_r, st));
     ScheduleSplit nosplit = {};
     CK(launch_schedule(indptr, p->E, p->T, 0, kTcTileM, ceil_div(p->d_ff, 256), ceil_div(p->d, 256), 0, 0,
                        tiles_dh, tiles_dx, nosplit, st));

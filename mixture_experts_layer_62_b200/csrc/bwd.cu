@@ -14,6 +14,8 @@
 //  * bias update ("Lecture 21" §2.4): above-mean experts b -= gamma, below
 //    b += gamma, decided exactly by the sign of c_e E - T k.
 // Every reduction runs in a fixed order; no atomics.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -181,69 +183,107 @@ router_bwd_kernel(const float* __restrict__ logits, const int32_t* __restrict__ 
     }
 }
 
-// dW_r[i][e] = sum_t x[t][i] dz[t][e]: one thread per (i, e), tokens in order.
+// dW_r[i][e] = sum_t x[t][i] dz[t][e] in two fixed-order passes: block
+// (i-block, token chunk, expert group) sums its kDwrTok tokens into a
+// partial, then the partials are summed over chunks in order. A thread owns
+// one column i and kDwrE experts; the chunk's dz rows are staged in shared
+// memory.
+constexpr int kDwrTok = 128;   // tokens per chunk
+constexpr int kDwrE = 32;      // experts per block (grid z)
+
 __global__ void __launch_bounds__(256)
-dwr_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dz, int T, int d, int E,
-           float* __restrict__ dW_r) {
+dwr_partial_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dz, int T, int d, int E,
+                   float* __restrict__ part) {
+    __shared__ float dzs[kDwrTok][kDwrE];
     pdl_wait();
     pdl_launch();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    const int e = blockIdx.y;
+    const int t0 = blockIdx.y * kDwrTok;
+    const int e0 = blockIdx.z * kDwrE;
+    const int ne = min(kDwrE, E - e0);
+    const int nt = min(kDwrTok, T - t0);
+    for (int q = threadIdx.x; q < kDwrTok * kDwrE; q += blockDim.x) {
+        const int tt = q / kDwrE, ee = q % kDwrE;
+        dzs[tt][ee] = (tt < nt && ee < ne) ? dz[static_cast<size_t>(t0 + tt) * E + e0 + ee] : 0.f;
+    }
+    __syncthreads();
     if (i >= d) return;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < T; ++t)
-        acc = fmaf(__bfloat162float(x[static_cast<size_t>(t) * d + i]), dz[static_cast<size_t>(t) * E + e], acc);
-    dW_r[static_cast<size_t>(i) * E + e] = acc;
+    float acc[kDwrE];
+#pragma unroll
+    for (int e = 0; e < kDwrE; ++e) acc[e] = 0.f;
+    const __nv_bfloat16* xc = x + static_cast<size_t>(t0) * d + i;
+#pragma unroll 4
+    for (int tt = 0; tt < nt; ++tt) {
+        const float xv = __bfloat162float(xc[static_cast<size_t>(tt) * d]);
+#pragma unroll
+        for (int e = 0; e < kDwrE; ++e) acc[e] = fmaf(xv, dzs[tt][e], acc[e]);
+    }
+    float* out = part + (static_cast<size_t>(blockIdx.y) * d + i) * E + e0;
+#pragma unroll
+    for (int e = 0; e < kDwrE; ++e)
+        if (e < ne) out[e] = acc[e];
 }
 
-// dx_t = sum_j dXp[pos_{t,j}] + W_r dz_t: one warp per (token, 256-wide
-// slice); the token's dz row is staged in shared memory.
-__global__ void __launch_bounds__(kWarps * 32)
-bwd_dx_kernel(const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__ pos,
-              const __nv_bfloat16* __restrict__ W_r, const float* __restrict__ dz, int T, int d, int E, int k,
-              int slices, __nv_bfloat16* __restrict__ dx) {
-    __shared__ float dzs[kWarps][MOE_MAX_E];
+__global__ void __launch_bounds__(256)
+dwr_reduce_kernel(const float* __restrict__ part, int nchunks, int d, int E, float* __restrict__ dW_r) {
     pdl_wait();
     pdl_launch();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long task = static_cast<long long>(blockIdx.x) * kWarps + warp;
-    const int t = static_cast<int>(task / slices), sl = static_cast<int>(task % slices);
-    if (t >= T) return;
-    for (int e = lane; e < E; e += 32) dzs[warp][e] = dz[static_cast<size_t>(t) * E + e];
-    __syncwarp();
-    const int v = sl * 32 + lane;   // 8 consecutive columns
-    if (v >= d / 8) return;
-    float acc[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-    for (int j = 0; j < k; ++j) {
-        const int r = pos[static_cast<size_t>(t) * k + j];
-        if (r < 0) continue;
-        float a[8];
-        unpack8(reinterpret_cast<const uint4*>(dXp + static_cast<size_t>(r) * d)[v], a);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] += a[c];
-    }
-    // router term, rows 8v .. 8v+7 of W_r [d][E], experts in order
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const __nv_bfloat16* wrow = W_r + static_cast<size_t>(8 * v + c) * E;
+    const size_t n = static_cast<size_t>(d) * E;
+    for (size_t q = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < n;
+         q += static_cast<size_t>(gridDim.x) * blockDim.x) {
         float s = 0.f;
-        if ((E & 7) == 0) {
-            for (int e = 0; e < E; e += 8) {
-                float w[8];
-                unpack8(*reinterpret_cast<const uint4*>(wrow + e), w);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) s = fmaf(w[q], dzs[warp][e + q], s);
-            }
-        } else {
-            for (int e = 0; e < E; ++e) s = fmaf(__bfloat162float(wrow[e]), dzs[warp][e], s);
-        }
-        acc[c] += s;
+        for (int c = 0; c < nchunks; ++c) s += part[static_cast<size_t>(c) * n + q];
+        dW_r[q] = s;
     }
-    reinterpret_cast<uint4*>(dx + static_cast<size_t>(t) * d)[v] =
-        make_uint4(pack2(acc[0], acc[1]), pack2(acc[2], acc[3]), pack2(acc[4], acc[5]), pack2(acc[6], acc[7]));
+}
+
+// dx_t = sum_j dXp[pos_{t,j}] + W_r dz_t: one block per token, a thread per
+// 8 consecutive columns; the token's dz row is staged in shared memory.
+__global__ void __launch_bounds__(256)
+bwd_dx_kernel(const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__ pos,
+              const __nv_bfloat16* __restrict__ W_r, const float* __restrict__ dz, int T, int d, int E, int k,
+              __nv_bfloat16* __restrict__ dx) {
+    __shared__ float dzs[MOE_MAX_E];
+    __shared__ int rows[MOE_MAX_K];
+    pdl_wait();
+    pdl_launch();
+    const int t = blockIdx.x;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) dzs[e] = dz[static_cast<size_t>(t) * E + e];
+    if (threadIdx.x < k) rows[threadIdx.x] = pos[static_cast<size_t>(t) * k + threadIdx.x];
+    __syncthreads();
+    const int nvec = d / 8;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const int r = rows[j];
+            if (r < 0) continue;
+            float a[8];
+            unpack8(reinterpret_cast<const uint4*>(dXp + static_cast<size_t>(r) * d)[v], a);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[c] += a[c];
+        }
+        // router term, rows 8v .. 8v+7 of W_r [d][E], experts in order
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const __nv_bfloat16* wrow = W_r + static_cast<size_t>(8 * v + c) * E;
+            float s = 0.f;
+            if ((E & 7) == 0) {
+                for (int e = 0; e < E; e += 8) {
+                    float w[8];
+                    unpack8(*reinterpret_cast<const uint4*>(wrow + e), w);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) s = fmaf(w[q], dzs[e + q], s);
+                }
+            } else {
+                for (int e = 0; e < E; ++e) s = fmaf(__bfloat162float(wrow[e]), dzs[e], s);
+            }
+            acc[c] += s;
+        }
+        reinterpret_cast<uint4*>(dx + static_cast<size_t>(t) * d)[v] =
+            make_uint4(pack2(acc[0], acc[1]), pack2(acc[2], acc[3]), pack2(acc[4], acc[5]), pack2(acc[6], acc[7]));
+    }
 }
 
 __global__ void bias_update_kernel(const void* __restrict__ stats, int T, int E, int k, float gamma,
@@ -278,19 +318,22 @@ cudaError_t launch_router_bwd(const float* logits, const int32_t* idx, const flo
                     stats, T, E, k, gate_mode, alpha, beta, dz);
 }
 
-cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* dW_r, cudaStream_t st) {
-    return launch_k(dwr_kernel, dim3(ceil_div(d, 256), E), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(x),
-                    dz, T, d, E, dW_r);
+cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* part, float* dW_r,
+                       cudaStream_t st) {
+    const int nchunks = ceil_div(T, kDwrTok);
+    cudaError_t e = launch_k(dwr_partial_kernel, dim3(ceil_div(d, 256), nchunks, ceil_div(E, kDwrE)), dim3(256), 0,
+                             st, static_cast<const __nv_bfloat16*>(x), dz, T, d, E, part);
+    if (e != cudaSuccess) return e;
+    const long long n = static_cast<long long>(d) * E;
+    return launch_k(dwr_reduce_kernel, dim3(static_cast<unsigned>(std::min<long long>(ceil_div((int)n, 256), 1184))),
+                    dim3(256), 0, st, static_cast<const float*>(part), nchunks, d, E, dW_r);
 }
 
 cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, int T, int d,
                           int E, int k, void* dx, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    const int slices = ceil_div(d / 8, 32);
-    const long long tasks = static_cast<long long>(T) * slices;
-    return launch_k(bwd_dx_kernel, dim3(static_cast<unsigned>((tasks + kWarps - 1) / kWarps)), dim3(kWarps * 32), 0,
-                    st, static_cast<const __nv_bfloat16*>(dXp), pos, static_cast<const __nv_bfloat16*>(W_r), dz, T,
-                    d, E, k, slices, static_cast<__nv_bfloat16*>(dx));
+    return launch_k(bwd_dx_kernel, dim3(T), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(dXp), pos,
+                    static_cast<const __nv_bfloat16*>(W_r), dz, T, d, E, k, static_cast<__nv_bfloat16*>(dx));
 }
 
 cudaError_t launch_bias_update(const void* stats, int T, int E, int k, float gamma, float* bias, cudaStream_t st) {

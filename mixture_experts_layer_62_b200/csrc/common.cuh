@@ -80,7 +80,7 @@ Layout make_layout(const moe_problem& p);
 long long permuted_rows(const moe_problem& p);
 // Byte offsets of the backward pass's own workspace.
 struct BwdLayout {
-    size_t dO, dAB, dXp, dz, dgate, tiles_dh, tiles_dx, total;
+    size_t dO, dAB, dXp, dz, dgate, tiles_dh, tiles_dx, dwr_part, total;
 };
 BwdLayout make_bwd_layout(const moe_problem& p);
 
@@ -253,7 +253,9 @@ cudaError_t launch_bwd_gather(const void* dy, const void* o, const int32_t* pos,
 cudaError_t launch_router_bwd(const float* logits, const int32_t* idx, const float* gate, const float* dgate,
                               const void* stats, int T, int E, int k, int gate_mode, float alpha, float beta,
                               float* dz, cudaStream_t st);
-cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* dW_r, cudaStream_t st);
+// dW_r = x^T dz via fp32 partials over 128-token chunks (part: ceil(T/128) * d * E floats)
+cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* part, float* dW_r,
+                       cudaStream_t st);
 cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, int T, int d,
                           int E, int k, void* dx, cudaStream_t st);
 cudaError_t launch_bias_update(const void* stats, int T, int E, int k, float gamma, float* bias, cudaStream_t st);

@@ -46,7 +46,9 @@ constexpr int MN_CHUNK = 64 * BK * 2;         // one 64-wide chunk of an MN-majo
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int NUM_THREADS = 192;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int STAGE_PITCH = 33;               // floats per staged row (conflict-free banks)
+constexpr int STAGE_WARP_BYTES = 32 * STAGE_PITCH * 4;   // one epilogue warp's 32 x 32 fp32 block
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + 4 * STAGE_WARP_BYTES;
 
 struct BParams {
     const int32_t* indptr;    // padded row offsets of the groups [E+1]
@@ -285,33 +287,51 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUte
         const int r = q * 32 + lane;
         int acc = 0;
         uint32_t aph = 0;
+        float* stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256) + q * (32 * STAGE_PITCH);
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
             const BTile t = decode<MODE>(p, u);
-            if (!wait_b(&ctl->tfull[acc], aph, ctl, p)) break;
-            tc_fence_after();
-            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_COLS);
-            const bool empty_k = t.num_kb == 0;   // an expert without rows: its weight gradient is 0
             if (MODE == BW_DH) {
+                // the forward's pre-activations of this thread's row, 32 hidden
+                // units per chunk; chunk c + 1 is requested before chunk c is
+                // used, and chunk 0 before the accumulator is ready
                 const int grow = t.m_blk * BM + r;
                 const bool valid = grow < t.rows;
                 const size_t orow = static_cast<size_t>(t.row0) + static_cast<size_t>(grow);
                 const size_t ld = 2 * static_cast<size_t>(p.d_ff);
+                auto chunk_off = [&](int c) {
+                    const int j0 = t.n_blk * BN + c;
+                    return orow * ld + static_cast<size_t>(j0 >> 7) * 256 + (j0 & 127);
+                };
+                auto chunk_ok = [&](int c) { return valid && t.n_blk * BN + c < p.d_ff; };
+                uint4 na[4], nb[4];
+                if (chunk_ok(0)) {
+                    const uint4* pa = reinterpret_cast<const uint4*>(p.ab + chunk_off(0));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) { na[i] = pa[i]; nb[i] = pa[16 + i]; }
+                }
+                if (!wait_b(&ctl->tfull[acc], aph, ctl, p)) break;
+                tc_fence_after();
+                const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                    static_cast<uint32_t>(acc * ACC_COLS);
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 32) {
+                    uint4 ca[4], cb[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) { ca[i] = na[i]; cb[i] = nb[i]; }
+                    if (c + 32 < BN && chunk_ok(c + 32)) {
+                        const uint4* pa = reinterpret_cast<const uint4*>(p.ab + chunk_off(c + 32));
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) { na[i] = pa[i]; nb[i] = pa[16 + i]; }
+                    }
                     uint32_t v[32];
                     tmem_ld32(tb + c, v);
-                    const int j0 = t.n_blk * BN + c;               // hidden unit of column c
-                    if (valid && j0 < p.d_ff) {
-                        const size_t off = orow * ld + static_cast<size_t>(j0 >> 7) * 256 + (j0 & 127);
-                        const uint4* pa = reinterpret_cast<const uint4*>(p.ab + off);
-                        const uint4* pb = reinterpret_cast<const uint4*>(p.ab + off + 128);
-                        uint4* qa = reinterpret_cast<uint4*>(p.out_bf16 + off);
-                        uint4* qb = reinterpret_cast<uint4*>(p.out_bf16 + off + 128);
+                    if (chunk_ok(c)) {
+                        uint4* qa = reinterpret_cast<uint4*>(p.out_bf16 + chunk_off(c));
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             float a[8], b[8];
-                            unpack8(pa[i], a);
-                            unpack8(pb[i], b);
+                            unpack8(ca[i], a);
+                            unpack8(cb[i], b);
                             uint32_t da[4], db[4];
 #pragma unroll
                             for (int e2 = 0; e2 < 4; ++e2) {
@@ -328,11 +348,15 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUte
                                 db[e2] = pack2(rdb[0], rdb[1]);
                             }
                             qa[i] = make_uint4(da[0], da[1], da[2], da[3]);
-                            qb[i] = make_uint4(db[0], db[1], db[2], db[3]);
+                            qa[16 + i] = make_uint4(db[0], db[1], db[2], db[3]);
                         }
                     }
                 }
             } else if (MODE == BW_DX) {
+                if (!wait_b(&ctl->tfull[acc], aph, ctl, p)) break;
+                tc_fence_after();
+                const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                    static_cast<uint32_t>(acc * ACC_COLS);
                 const int grow = t.m_blk * BM + r;
                 const bool valid = grow < t.rows;
                 const size_t orow = static_cast<size_t>(t.row0) + static_cast<size_t>(grow);
@@ -353,31 +377,47 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUte
                     }
                 }
             } else {
-                // weight gradients, fp32: BW_DW2 row m of dW2_e; BW_DW13 row of dW1_e
-                // (gate half of a 256-row AB group) or dW3_e (up half)
-                const int m = t.m_blk * BM + r;
-                float* orow_ptr;
-                bool valid;
+                // weight gradients, fp32: BW_DW2 row m of dW2_e; BW_DW13 row of
+                // dW1_e (gate half of a 256-row AB group) or dW3_e (up half).
+                // Each 32 x 32 block of the warp goes through shared memory so
+                // that global stores cover whole 128-byte row segments.
+                if (!wait_b(&ctl->tfull[acc], aph, ctl, p)) break;
+                tc_fence_after();
+                const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                    static_cast<uint32_t>(acc * ACC_COLS);
+                const bool empty_k = t.num_kb == 0;   // an expert without rows: its gradient is 0
+                const int m0 = t.m_blk * BM + q * 32;  // first row of this warp's block
+                float* base;
+                int rows_ok;                           // valid rows of the block
                 if (MODE == BW_DW2) {
-                    valid = m < p.M;
-                    orow_ptr = p.out0 + (static_cast<size_t>(t.g) * p.M + m) * static_cast<size_t>(p.N);
+                    base = p.out0 + (static_cast<size_t>(t.g) * p.M + m0) * static_cast<size_t>(p.N);
+                    rows_ok = min(32, p.M - m0);
                 } else {
-                    const int wrow = (t.m_blk >> 1) * 128 + r;
-                    valid = wrow < p.d_ff;
-                    float* base = (t.m_blk & 1) ? p.out1 : p.out0;
-                    orow_ptr = base + (static_cast<size_t>(t.g) * p.d_ff + wrow) * static_cast<size_t>(p.N);
+                    const int w0 = (t.m_blk >> 1) * 128 + q * 32;
+                    base = ((t.m_blk & 1) ? p.out1 : p.out0) +
+                           (static_cast<size_t>(t.g) * p.d_ff + w0) * static_cast<size_t>(p.N);
+                    rows_ok = min(32, p.d_ff - w0);
                 }
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 32) {
                     uint32_t v[32];
                     if (!empty_k) tmem_ld32(tb + c, v);
                     const int col = t.n_blk * BN + c;
-                    if (valid && col < p.N) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow_ptr + col);
+                    if (col >= p.N) continue;         // the same for the whole warp
+                    __syncwarp();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = empty_k ? make_uint4(0u, 0u, 0u, 0u)
-                                             : make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    for (int i = 0; i < 32; ++i) stage[lane * STAGE_PITCH + i] = empty_k ? 0.f : __uint_as_float(v[i]);
+                    __syncwarp();
+                    // lanes 8q..8q+7 write row 4 i + q's 32 columns (128 bytes)
+                    const int rl = lane >> 3, cl = (lane & 7) * 4;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = 4 * i + rl;
+                        if (rr < rows_ok) {
+                            const float* sp = stage + rr * STAGE_PITCH + cl;
+                            *reinterpret_cast<float4*>(base + static_cast<size_t>(rr) * p.N + col + cl) =
+                                make_float4(sp[0], sp[1], sp[2], sp[3]);
+                        }
                     }
                 }
             }

@@ -120,6 +120,8 @@ CASES = [
     dict(T=200, d=256, d_ff=384, E=16, k=4, cf=0.9, pad=128, gate=O.GATE_FULL, drop=O.DROP_SLOT,
          alpha=0.05, beta=0.01),
     dict(T=64, d=128, d_ff=128, E=32, k=2, pad=64, bias_mode=O.BIAS_PROB),
+    # many tiles in every GEMM: 8 experts x ~512 rows, d = 1024, d_ff = 2048
+    dict(T=2048, d=1024, d_ff=2048, E=8, k=2, cf=1.0, pad=128, alpha=0.01, beta=0.001),
 ]
 
 
