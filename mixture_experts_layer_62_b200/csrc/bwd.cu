@@ -186,42 +186,48 @@ router_bwd_kernel(const float* __restrict__ logits, const int32_t* __restrict__ 
 // dW_r[i][e] = sum_t x[t][i] dz[t][e] in two fixed-order passes: block
 // (i-block, token chunk, expert group) sums its kDwrTok tokens into a
 // partial, then the partials are summed over chunks in order. A thread owns
-// one column i and kDwrE experts; the chunk's dz rows are staged in shared
-// memory.
+// two columns and a group of experts; the chunk's dz rows are staged in
+// shared memory.
 constexpr int kDwrTok = 128;   // tokens per chunk
-constexpr int kDwrE = 32;      // experts per block (grid z)
 
+template <int EB>   // experts per block (grid z): 8 for routers of 8, 32 otherwise
 __global__ void __launch_bounds__(256)
 dwr_partial_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dz, int T, int d, int E,
                    float* __restrict__ part) {
-    __shared__ float dzs[kDwrTok][kDwrE];
+    __shared__ float dzs[kDwrTok][EB];
     pdl_wait();
     pdl_launch();
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);   // two consecutive columns
     const int t0 = blockIdx.y * kDwrTok;
-    const int e0 = blockIdx.z * kDwrE;
-    const int ne = min(kDwrE, E - e0);
+    const int e0 = blockIdx.z * EB;
+    const int ne = min(EB, E - e0);
     const int nt = min(kDwrTok, T - t0);
-    for (int q = threadIdx.x; q < kDwrTok * kDwrE; q += blockDim.x) {
-        const int tt = q / kDwrE, ee = q % kDwrE;
+    for (int q = threadIdx.x; q < kDwrTok * EB; q += blockDim.x) {
+        const int tt = q / EB, ee = q % EB;
         dzs[tt][ee] = (tt < nt && ee < ne) ? dz[static_cast<size_t>(t0 + tt) * E + e0 + ee] : 0.f;
     }
     __syncthreads();
     if (i >= d) return;
-    float acc[kDwrE];
+    float a0[EB], a1[EB];
 #pragma unroll
-    for (int e = 0; e < kDwrE; ++e) acc[e] = 0.f;
-    const __nv_bfloat16* xc = x + static_cast<size_t>(t0) * d + i;
+    for (int e = 0; e < EB; ++e) a0[e] = a1[e] = 0.f;
+    const __nv_bfloat162* xc = reinterpret_cast<const __nv_bfloat162*>(x + static_cast<size_t>(t0) * d + i);
 #pragma unroll 4
     for (int tt = 0; tt < nt; ++tt) {
-        const float xv = __bfloat162float(xc[static_cast<size_t>(tt) * d]);
+        const float2 xv = __bfloat1622float2(xc[static_cast<size_t>(tt) * (d / 2)]);
 #pragma unroll
-        for (int e = 0; e < kDwrE; ++e) acc[e] = fmaf(xv, dzs[tt][e], acc[e]);
+        for (int e = 0; e < EB; ++e) {
+            a0[e] = fmaf(xv.x, dzs[tt][e], a0[e]);
+            a1[e] = fmaf(xv.y, dzs[tt][e], a1[e]);
+        }
     }
     float* out = part + (static_cast<size_t>(blockIdx.y) * d + i) * E + e0;
 #pragma unroll
-    for (int e = 0; e < kDwrE; ++e)
-        if (e < ne) out[e] = acc[e];
+    for (int e = 0; e < EB; ++e)
+        if (e < ne) {
+            out[e] = a0[e];
+            out[E + e] = a1[e];
+        }
 }
 
 __global__ void __launch_bounds__(256)
@@ -237,27 +243,44 @@ dwr_reduce_kernel(const float* __restrict__ part, int nchunks, int d, int E, flo
     }
 }
 
-// dx_t = sum_j dXp[pos_{t,j}] + W_r dz_t: one block per token, a thread per
-// 8 consecutive columns; the token's dz row is staged in shared memory.
+// dx_t = sum_j dXp[pos_{t,j}] + W_r dz_t. A thread owns 8 consecutive
+// columns of dx for a tile of kDxTok tokens; with E <= 16 its 8 rows of W_r
+// are loaded once into registers and reused across the tile (the rows of a
+// thread are contiguous but 128+ bytes apart from its neighbours', so
+// re-reading them per token was bound by L1 wavefronts); wider routers read
+// W_r per token. The tile's dz rows are staged in shared memory.
+constexpr int kDxTok = 16;
+
+template <int EG>   // EG = E / 8 uint4 per W_r row when staged in registers (1 or 2), 0: streamed
 __global__ void __launch_bounds__(256)
 bwd_dx_kernel(const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__ pos,
               const __nv_bfloat16* __restrict__ W_r, const float* __restrict__ dz, int T, int d, int E, int k,
               __nv_bfloat16* __restrict__ dx) {
-    __shared__ float dzs[MOE_MAX_E];
-    __shared__ int rows[MOE_MAX_K];
+    extern __shared__ float dzs[];   // [kDxTok][E]
     pdl_wait();
     pdl_launch();
-    const int t = blockIdx.x;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) dzs[e] = dz[static_cast<size_t>(t) * E + e];
-    if (threadIdx.x < k) rows[threadIdx.x] = pos[static_cast<size_t>(t) * k + threadIdx.x];
+    const int t0 = blockIdx.x * kDxTok;
+    const int nt = min(kDxTok, T - t0);
+    for (int q = threadIdx.x; q < nt * E; q += blockDim.x) dzs[q] = dz[static_cast<size_t>(t0) * E + q];
     __syncthreads();
-    const int nvec = d / 8;
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    const int v = blockIdx.y * blockDim.x + threadIdx.x;   // 8 consecutive columns
+    if (v >= d / 8) return;
+    uint4 w[8][EG > 0 ? EG : 1];
+    if (EG > 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+            for (int g = 0; g < EG; ++g)
+                w[c][g] = reinterpret_cast<const uint4*>(W_r + static_cast<size_t>(8 * v + c) * E)[g];
+    }
+    for (int tt = 0; tt < nt; ++tt) {
+        const int t = t0 + tt;
+        const float* dzt = dzs + tt * E;
         float acc[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[c] = 0.f;
         for (int j = 0; j < k; ++j) {
-            const int r = rows[j];
+            const int r = pos[static_cast<size_t>(t) * k + j];
             if (r < 0) continue;
             float a[8];
             unpack8(reinterpret_cast<const uint4*>(dXp + static_cast<size_t>(r) * d)[v], a);
@@ -267,17 +290,18 @@ bwd_dx_kernel(const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__
         // router term, rows 8v .. 8v+7 of W_r [d][E], experts in order
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            const __nv_bfloat16* wrow = W_r + static_cast<size_t>(8 * v + c) * E;
             float s = 0.f;
-            if ((E & 7) == 0) {
-                for (int e = 0; e < E; e += 8) {
-                    float w[8];
-                    unpack8(*reinterpret_cast<const uint4*>(wrow + e), w);
+            if (EG > 0) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) s = fmaf(w[q], dzs[e + q], s);
+                for (int g = 0; g < (EG > 0 ? EG : 1); ++g) {
+                    float wf[8];
+                    unpack8(w[c][g], wf);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) s = fmaf(wf[q], dzt[8 * g + q], s);
                 }
             } else {
-                for (int e = 0; e < E; ++e) s = fmaf(__bfloat162float(wrow[e]), dzs[e], s);
+                const __nv_bfloat16* wrow = W_r + static_cast<size_t>(8 * v + c) * E;
+                for (int e = 0; e < E; ++e) s = fmaf(__bfloat162float(wrow[e]), dzt[e], s);
             }
             acc[c] += s;
         }
@@ -321,8 +345,13 @@ cudaError_t launch_router_bwd(const float* logits, const int32_t* idx, const flo
 cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* part, float* dW_r,
                        cudaStream_t st) {
     const int nchunks = ceil_div(T, kDwrTok);
-    cudaError_t e = launch_k(dwr_partial_kernel, dim3(ceil_div(d, 256), nchunks, ceil_div(E, kDwrE)), dim3(256), 0,
-                             st, static_cast<const __nv_bfloat16*>(x), dz, T, d, E, part);
+    cudaError_t e;
+    if (E <= 8)
+        e = launch_k(dwr_partial_kernel<8>, dim3(ceil_div(d, 512), nchunks, 1), dim3(256), 0, st,
+                     static_cast<const __nv_bfloat16*>(x), dz, T, d, E, part);
+    else
+        e = launch_k(dwr_partial_kernel<32>, dim3(ceil_div(d, 512), nchunks, ceil_div(E, 32)), dim3(256), 0, st,
+                     static_cast<const __nv_bfloat16*>(x), dz, T, d, E, part);
     if (e != cudaSuccess) return e;
     const long long n = static_cast<long long>(d) * E;
     return launch_k(dwr_reduce_kernel, dim3(static_cast<unsigned>(std::min<long long>(ceil_div((int)n, 256), 1184))),
@@ -332,8 +361,15 @@ cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, floa
 cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, int T, int d,
                           int E, int k, void* dx, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    return launch_k(bwd_dx_kernel, dim3(T), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(dXp), pos,
-                    static_cast<const __nv_bfloat16*>(W_r), dz, T, d, E, k, static_cast<__nv_bfloat16*>(dx));
+    const dim3 grid(ceil_div(T, kDxTok), ceil_div(d / 8, 256));
+    const size_t smem = sizeof(float) * kDxTok * E;
+    auto args = [&](auto kern) {
+        return launch_k(kern, grid, dim3(256), smem, st, static_cast<const __nv_bfloat16*>(dXp), pos,
+                        static_cast<const __nv_bfloat16*>(W_r), dz, T, d, E, k, static_cast<__nv_bfloat16*>(dx));
+    };
+    if (E == 8) return args(bwd_dx_kernel<1>);
+    if (E == 16) return args(bwd_dx_kernel<2>);
+    return args(bwd_dx_kernel<0>);
 }
 
 cudaError_t launch_bias_update(const void* stats, int T, int E, int k, float gamma, float* bias, cudaStream_t st) {
