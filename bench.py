@@ -561,6 +561,10 @@ def run_train(args, cfg, moe, L, dev, stream, flush):
     fl_bwd = 2.0 * (2.0 * R * d * dff + 4.0 * R * d * dff) + 4.0 * T * d * E
     peaks, peak_src = load_peaks()
     tf_step = (fl_fwd + fl_bwd) / (step_ms / 1e3) / 1e12
+    tf_bwd = fl_bwd / (bwd_ms / 1e3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu = train_cpu_baseline(cfg, L, min(args.cpu_sample, 64))
     line = {
         "metric": "MoE-layer training step (fwd+bwd) tokens/s & TFLOP/s vs bf16 peak", "impl": "ours",
         "value": T / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -570,11 +574,52 @@ def run_train(args, cfg, moe, L, dev, stream, flush):
         "tflops_frac_of_sustained": tf_step / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
         "peak_source": peak_src,
         "forward": {"ms": fwd_ms, "tflops": fl_fwd / (fwd_ms / 1e3) / 1e12},
-        "backward": {"ms": bwd_ms, "tflops": fl_bwd / (bwd_ms / 1e3) / 1e12},
+        "backward": {"ms": bwd_ms, "tflops": tf_bwd},
+        # the backward pass as the unit: its four grouped GEMMs are 99 % of its FLOPs
+        "roofline": {"bound": "tensor", "kernel": "backward pass (tc_bwd_gemm x 4 + router/gather kernels)",
+                     "achieved": tf_bwd, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tf_bwd / peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16 burst",
+                     "frac_of_sustained": tf_bwd / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                     "flops_per_launch": fl_bwd, "traffic": None},
+        "cpu_baseline": cpu,
         "gpu_launches": (launches_per_forward(cfg, pad) + 10) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
+
+
+def train_cpu_baseline(cfg, L, n_tokens, seed=0):
+    """The backward oracle on a seeded token sample: routing of all tokens,
+    expert forward and backward of the sampled tokens only (dy is zero on the
+    others), timed on the host cores."""
+    from oracle import moe_oracle as O
+    from oracle import moe_backward_oracle as BO
+    rng = np.random.default_rng(seed)
+    tokens = np.sort(rng.choice(cfg["T"], size=min(n_tokens, cfg["T"]), replace=False))
+    x = L["x"].float().cpu().numpy()[tokens]
+    W_r = L["W_r"].float().cpu().numpy()
+    bias = None if L["bias"] is None else L["bias"].float().cpu().numpy()
+    z = O.router_logits(x, W_r)
+    key = O.selection_key(z, bias, cfg["bias_mode"])
+    used = sorted(set(O.topk_lowest_index(key, cfg["k"]).reshape(-1).tolist()))
+
+    class _Host(dict):
+        def __init__(self, W):
+            super().__init__({e: W[e].float().cpu().numpy() for e in used})
+            self.W = W
+
+        def __missing__(self, e):
+            v = self[e] = self.W[e].float().cpu().numpy()
+            return v
+
+    W1, W3, W2 = _Host(L["W1"]), _Host(L["W3"]), _Host(L["W2"])
+    dy = rng.standard_normal(x.shape)
+    t0 = time.perf_counter()
+    BO.moe_backward(x, W_r, W1, W3, W2, cfg["k"], dy, 0.0, bias, cfg["bias_mode"], alpha=0.01, beta=0.001)
+    dt = time.perf_counter() - t0
+    return {"value": len(tokens) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"forward + backward of {len(tokens)} seeded random tokens as their own batch "
+                      f"(no capacity), {dt:.1f} s"}
 
 
 def breakdown(moe, p, cfg, L, dev, stream, flush, iters):

@@ -42,6 +42,9 @@ WORKLOADS = {
     # logits, capacity factor 1.25
     "skewed_capacity": dict(T=16384, d=4096, d_ff=14336, E=8, k=2, cf=1.25, dtype="bf16", bias_mode=1,
                             d_ff_shared=0),
+    # half the Mixtral width, half the tokens: a training step that holds
+    # about 2.5 GB on the device (the size for full profiler captures)
+    "train_small": dict(T=2048, d=2048, d_ff=7168, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
 }
 DECODE_TOKENS = (1, 2, 4, 8, 16, 32)
 
