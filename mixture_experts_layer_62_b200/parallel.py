@@ -76,6 +76,35 @@ def global_stats(stats_block: torch.Tensor, E: int, k: int, T_local: int, group=
     return GlobalStats(T=T, counts=counts, kept=kept, f=f, P=P, l_aux=l_aux, dropped=dropped, max_over_mean=mom)
 
 
+# ---- data-parallel training --------------------------------------------------
+#
+# A replica's backward differentiates its own tokens' share of the global
+# loss L = sum_t <dy_t, y_t> + alpha L_aux + beta L_z. L_aux uses the global
+# f and the global token count ("Week 2 Day 2" §3.2: f and P over the whole
+# batch), so before moe_backward a replica writes the global f into its
+# statistics block and scales alpha and beta by T_local / T_global (the
+# backward divides by its own T); afterwards one all-reduce (sum) of each
+# weight gradient gives every replica the gradient of the global loss. dx
+# stays local.
+
+def set_global_f(stats_block: torch.Tensor, E: int, g: GlobalStats) -> None:
+    """Overwrite the f array of a statistics block with the global f."""
+    body = stats_block[STATS_HEADER_BYTES:STATS_HEADER_BYTES + 16 * E]
+    body[12 * E:16 * E].view(torch.float32).copy_(g.f.to(torch.float32).to(stats_block.device))
+
+
+def loss_scale(T_local: int, T_global: int) -> float:
+    """Factor for alpha and beta on a replica holding T_local of T_global tokens."""
+    return float(T_local) / float(T_global) if T_global > 0 else 0.0
+
+
+def allreduce_gradients(grads, group=None) -> None:
+    """Sum each gradient tensor over the replicas, in place."""
+    if dist.is_available() and dist.is_initialized():
+        for t in grads:
+            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+
+
 def stats_block_from_parts(counts, kept, P, dropped=0, capacity=-1, device="cpu") -> torch.Tensor:
     """Build a statistics block (the library's layout) from host values; used
     to feed global_stats from statistics computed elsewhere."""

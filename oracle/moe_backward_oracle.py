@@ -127,9 +127,11 @@ class BackwardResult:
 
 def moe_backward(x, W_r, W1, W3, W2, k, dy, capacity_factor=0.0, bias=None, bias_mode=O.BIAS_NONE,
                  Ws1=None, Ws3=None, Ws2=None, alpha=0.0, beta=0.0, gate_mode=O.GATE_SELECTED,
-                 drop_order=O.DROP_TOKEN, logits=None, key_dtype=np.float64, idx=None):
+                 drop_order=O.DROP_TOKEN, logits=None, key_dtype=np.float64, idx=None, f=None):
     """Gradients of L = <dy, y> + alpha L_aux + beta L_z w.r.t. x, W_r and the
-    expert weights. ``W1``, ``W3``, ``W2`` are indexable by expert."""
+    expert weights. ``W1``, ``W3``, ``W2`` are indexable by expert; ``f``
+    replaces the batch's own f in L_aux (a data-parallel replica uses the
+    global one)."""
     x = np.asarray(x, dtype=np.float64)
     dy = np.asarray(dy, dtype=np.float64)
     T, d = x.shape
@@ -165,7 +167,8 @@ def moe_backward(x, W_r, W1, W3, W2, k, dy, capacity_factor=0.0, bias=None, bias
         dXs, dWs1, dWs3, dWs2, _ = expert_backward(x, dy, Ws1, Ws3, Ws2)
         dx += dXs
 
-    dz = router_dz(z, idx, keep, dgate, gate_mode, fwd.stats.f, alpha, beta)
+    dz = router_dz(z, idx, keep, dgate, gate_mode, fwd.stats.f if f is None else np.asarray(f, dtype=np.float64),
+                   alpha, beta)
     dW_r = x.T @ dz
     if W_r64 is not None:
         dx += dz @ W_r64.T

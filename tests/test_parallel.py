@@ -97,3 +97,68 @@ def test_global_stats_single_process_is_identity():
     assert g.counts.tolist() == [3, 1, 0, 2] and g.kept.tolist() == [3, 1, 0, 1] and g.dropped == 1
     assert g.f.tolist() == [0.5, 1 / 6, 0.0, 1 / 3]
     assert g.l_aux == pytest.approx(4 * (0.5 * 0.5 + 0.2 / 6 + 0.2 / 3), rel=1e-6)
+
+
+# --- data-parallel training: global f, scaled alpha/beta, summed gradients ---
+
+d_ff = 6
+ALPHA, BETA = 0.3, 0.05
+
+
+def _train_data():
+    rng = np.random.default_rng(1)
+    x, W_r = _data()
+    W1 = rng.standard_normal((E, d_ff, d)) / math.sqrt(d)
+    W3 = rng.standard_normal((E, d_ff, d)) / math.sqrt(d)
+    W2 = rng.standard_normal((E, d, d_ff)) / math.sqrt(d_ff)
+    dy = rng.standard_normal((T, d))
+    return x, W_r, W1, W3, W2, dy
+
+
+def _train_worker(rank, world, port, q):
+    from oracle import moe_backward_oracle as BO
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        x, W_r, W1, W3, W2, dy = _train_data()
+        lo, hi = parallel.shard_range(T, world, rank)
+        # the replica's forward statistics, exchanged
+        z = O.router_logits(x[lo:hi], W_r)
+        r = O.route(z, k)
+        perm = O.permute(r.idx, E)
+        st = O.load_stats(perm, r.probs, hi - lo, k, None)
+        blk = parallel.stats_block_from_parts(st.counts.tolist(), st.kept.tolist(), st.P.tolist())
+        g = parallel.global_stats(blk, E, k, hi - lo)
+        parallel.set_global_f(blk, E, g)
+        f_blk = blk[48 + 12 * E:48 + 16 * E].view(torch.float32).double().numpy()
+        s = parallel.loss_scale(hi - lo, g.T)
+        res = BO.moe_backward(x[lo:hi], W_r, W1, W3, W2, k, dy[lo:hi], alpha=ALPHA * s, beta=BETA * s, f=f_blk)
+        grads = [torch.from_numpy(a.copy()) for a in (res.dW_r, res.dW1, res.dW3, res.dW2)]
+        parallel.allreduce_gradients(grads)
+        q.put((rank, lo, hi, res.dx, [t.numpy() for t in grads], f_blk))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_gradients_equal_full_batch_backward():
+    from oracle import moe_backward_oracle as BO
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_train_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    x, W_r, W1, W3, W2, dy = _train_data()
+    ref = BO.moe_backward(x, W_r, W1, W3, W2, k, dy, alpha=ALPHA, beta=BETA)
+    for rank, lo, hi, dx, grads, f_blk in results:
+        # the global f went through the block in fp32
+        assert np.allclose(f_blk, ref.forward.stats.f, rtol=1e-7, atol=0)
+        assert np.allclose(dx, ref.dx[lo:hi], rtol=1e-6, atol=1e-9)
+        for got, want in zip(grads, (ref.dW_r, ref.dW1, ref.dW3, ref.dW2)):
+            assert np.allclose(got, want, rtol=1e-6, atol=1e-9)
