@@ -511,13 +511,18 @@ def run_train(args, cfg, moe, L, dev, stream, flush):
     dW1 = torch.empty((E, dff, d), device=dev)
     dW3 = torch.empty((E, dff, d), device=dev)
     dW2 = torch.empty((E, d, dff), device=dev)
+    dfs = cfg["d_ff_shared"]
+    dWs = [torch.empty((dfs, d), device=dev), torch.empty((dfs, d), device=dev),
+           torch.empty((d, dfs), device=dev)] if dfs else [None, None, None]
 
     def fwd():
-        moe.forward(p, L["x"], L["W_r"], L["W1"], L["W3"], L["W2"], out, st, ws, bias=L["bias"])
+        moe.forward(p, L["x"], L["W_r"], L["W1"], L["W3"], L["W2"], out, st, ws, bias=L["bias"], Ws1=L["Ws1"],
+                    Ws3=L["Ws3"], Ws2=L["Ws2"])
 
     def bwd():
         moe.backward(p, L["x"], L["W_r"], L["W1"], L["W3"], L["W2"], dy, dx, dW_r, dW1, dW3, dW2, st, ws, bws,
-                     alpha=0.01, beta=0.001)
+                     alpha=0.01, beta=0.001, Ws1=L["Ws1"], Ws3=L["Ws3"], Ws2=L["Ws2"], dWs1=dWs[0], dWs3=dWs[1],
+                     dWs2=dWs[2])
 
     for _ in range(args.warmup):
         fwd()
@@ -557,8 +562,9 @@ def run_train(args, cfg, moe, L, dev, stream, flush):
         raise SystemExit(f"device status {s.status}: {moe.error_string(s.status)}")
     R = s.rows
     fl_fwd = flops_per_step(cfg, R)
-    # backward: dH and dXp (2 R d d_ff + 4 R d d_ff), dW2 and [dW1; dW3] (the same), router 2 x 2 T d E
-    fl_bwd = 2.0 * (2.0 * R * d * dff + 4.0 * R * d * dff) + 4.0 * T * d * E
+    # backward: dH and dXp (2 R d d_ff + 4 R d d_ff), dW2 and [dW1; dW3] (the same), router 2 x 2 T d E,
+    # and the shared expert's four GEMMs over all T rows
+    fl_bwd = 2.0 * (2.0 * R * d * dff + 4.0 * R * d * dff) + 4.0 * T * d * E + 2.0 * 6.0 * T * d * dfs
     peaks, peak_src = load_peaks()
     tf_step = (fl_fwd + fl_bwd) / (step_ms / 1e3) / 1e12
     tf_bwd = fl_bwd / (bwd_ms / 1e3) / 1e12
@@ -582,7 +588,7 @@ def run_train(args, cfg, moe, L, dev, stream, flush):
                      "frac_of_sustained": tf_bwd / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                      "flops_per_launch": fl_bwd, "traffic": None},
         "cpu_baseline": cpu,
-        "gpu_launches": (launches_per_forward(cfg, pad) + 10) * args.steps,
+        "gpu_launches": (launches_per_forward(cfg, pad) + 10 + (6 if dfs else 0)) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
@@ -613,9 +619,10 @@ def train_cpu_baseline(cfg, L, n_tokens, seed=0):
             return v
 
     W1, W3, W2 = _Host(L["W1"]), _Host(L["W3"]), _Host(L["W2"])
+    sh = {n: (None if L[n] is None else L[n].float().cpu().numpy()) for n in ("Ws1", "Ws3", "Ws2")}
     dy = rng.standard_normal(x.shape)
     t0 = time.perf_counter()
-    BO.moe_backward(x, W_r, W1, W3, W2, cfg["k"], dy, 0.0, bias, cfg["bias_mode"], alpha=0.01, beta=0.001)
+    BO.moe_backward(x, W_r, W1, W3, W2, cfg["k"], dy, 0.0, bias, cfg["bias_mode"], **sh, alpha=0.01, beta=0.001)
     dt = time.perf_counter() - t0
     return {"value": len(tokens) / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"forward + backward of {len(tokens)} seeded random tokens as their own batch "

@@ -279,13 +279,15 @@ int moe_permute_noalloc(const moe_problem* p, const void* x, const int32_t* idx,
  * reaches the router through P only) and L_z the router z-loss (§3.4). The
  * expert selection and the capacity drops carry no gradient; the selection
  * bias gets none.
- * Requires p->train = 1 (the forward kept the gate/up pre-activations),
+ * Requires p->train = 1 (the forward kept the gate/up pre-activations) and
  * p->pad_rows = 64 or 128 (the weight-gradient GEMMs contract over each
- * expert's rows, which padding keeps in whole 64-row blocks), bf16 and no
- * shared expert; otherwise MOE_ERR_UNSUPPORTED.
+ * expert's rows, which padding keeps in whole 64-row blocks), bf16 and
+ * E % 8 == 0; otherwise MOE_ERR_UNSUPPORTED.
  *   dy [T, d] bf16 in; dx [T, d] bf16 out;
  *   dW_r [d, E] fp32, dW1 and dW3 [E, d_ff, d] fp32, dW2 [E, d, d_ff] fp32
  *   out, each written fully (an expert without rows gets zeros);
+ *   with d_ff_shared > 0: Ws1, Ws3, Ws2 as in moe_forward, and dWs1, dWs3
+ *   [d_ff_shared, d], dWs2 [d, d_ff_shared] fp32 out (NULL otherwise);
  *   stats: the forward's block (f is read; the status word gets
  *   MOE_ERR_TIMEOUT if a bounded wait of a tensor-core kernel gave up);
  *   bwd_workspace: moe_backward_workspace_size(p) bytes, 256-byte aligned,
@@ -293,8 +295,10 @@ int moe_permute_noalloc(const moe_problem* p, const void* x, const int32_t* idx,
  * Reductions run in a fixed order: repeated calls give identical results. */
 size_t moe_backward_workspace_size(const moe_problem* p);
 int moe_backward(const moe_problem* p, const void* x, const void* W_r, const void* W1, const void* W3,
-                 const void* W2, const void* dy, float alpha, float beta,
-                 void* dx, float* dW_r, float* dW1, float* dW3, float* dW2, void* stats,
+                 const void* W2, const void* Ws1, const void* Ws3, const void* Ws2,
+                 const void* dy, float alpha, float beta,
+                 void* dx, float* dW_r, float* dW1, float* dW3, float* dW2,
+                 float* dWs1, float* dWs3, float* dWs2, void* stats,
                  const void* workspace, size_t workspace_bytes,
                  void* bwd_workspace, size_t bwd_workspace_bytes, void* stream);
 

@@ -84,7 +84,7 @@ def _load():
     lib.moe_backward_workspace_size.argtypes = [P]
     lib.moe_backward_workspace_size.restype = sz
     f32 = ctypes.c_float
-    lib.moe_backward.argtypes = [P] + [vp] * 6 + [f32, f32] + [vp] * 6 + [vp, sz, vp, sz, vp]
+    lib.moe_backward.argtypes = [P] + [vp] * 9 + [f32, f32] + [vp] * 9 + [vp, sz, vp, sz, vp]
     lib.moe_backward.restype = ctypes.c_int
     lib.moe_bias_update.argtypes = [P, vp, f32, vp, vp]
     lib.moe_bias_update.restype = ctypes.c_int
@@ -227,12 +227,13 @@ def alloc_backward_workspace(p: Problem, device=None) -> torch.Tensor:
 
 
 def backward(p: Problem, x, W_r, W1, W3, W2, dy, dx, dW_r, dW1, dW3, dW2, stats, workspace, bwd_workspace,
-             alpha=0.0, beta=0.0, stream=None):
+             alpha=0.0, beta=0.0, Ws1=None, Ws3=None, Ws2=None, dWs1=None, dWs3=None, dWs2=None, stream=None):
     """Gradients of <dy, y> + alpha L_aux + beta L_z after a moe_forward with
     p.train = 1 on the same workspace; see moe_backward."""
-    rc = _lib().moe_backward(ctypes.byref(p), _ptr(x), _ptr(W_r), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(dy),
-                             float(alpha), float(beta), _ptr(dx), _ptr(dW_r), _ptr(dW1), _ptr(dW3), _ptr(dW2),
-                             _ptr(stats), _ptr(workspace), workspace.numel() * workspace.element_size(),
+    rc = _lib().moe_backward(ctypes.byref(p), _ptr(x), _ptr(W_r), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(Ws1),
+                             _ptr(Ws3), _ptr(Ws2), _ptr(dy), float(alpha), float(beta), _ptr(dx), _ptr(dW_r),
+                             _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(dWs1), _ptr(dWs3), _ptr(dWs2), _ptr(stats),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(),
                              _ptr(bwd_workspace), bwd_workspace.numel() * bwd_workspace.element_size(),
                              _stream(stream))
     _check(rc, "moe_backward")

@@ -48,6 +48,7 @@ Layout make_layout(const moe_problem& p) {
     L.hs = take(T * dfs * eb);
     L.s = take(dfs ? T * d * eb : 0);
     L.ab = take(p.train ? Rmax * 2 * dff * eb : 0);
+    L.abs = take(p.train ? T * 2 * dfs * eb : 0);
     const bool split = split_allowed(p);
     L.part13 = take(split ? (size_t)kSplitMax * T * k * (size_t)ceil_div(p.d_ff, 128) * 256 * 4 : 0);
     L.part2 = take(split ? (size_t)kSplitMax * T * k * d * 4 : 0);
@@ -78,7 +79,16 @@ BwdLayout make_bwd_layout(const moe_problem& p) {
     B.dgate = take(T * k * 4);
     B.tiles_dh = take((E + 3) * 4);
     B.tiles_dx = take((E + 3) * 4);
-    B.dwr_part = take((size_t)ceil_div((int)T, 128) * d * E * 4);
+    const bool tc_router = E % 64 == 0;
+    B.dwr_part = take(tc_router ? 0 : (size_t)ceil_div((int)T, 128) * d * E * 4);
+    B.dz16 = take(tc_router ? T * E * 2 : 0);
+    B.dxr = take(tc_router ? T * d * 4 : 0);
+    const size_t dfs = (size_t)(p.d_ff_shared > 0 ? p.d_ff_shared : 0);
+    B.dABs = take(T * 2 * dfs * eb);
+    B.dXs = take(dfs ? T * d * eb : 0);
+    B.indptr_s = take(2 * 4);
+    B.tiles_s_dh = take(4 * 4);
+    B.tiles_s_dx = take(4 * 4);
     B.total = off;
     return B;
 }
@@ -163,7 +173,7 @@ int check_problem(const moe_problem* p) {
     if (!std::isfinite(p->capacity_factor)) return MOE_ERR_INVALID_ARG;
     if (p->pad_rows != 0 && p->pad_rows != 64 && p->pad_rows != 128) return MOE_ERR_INVALID_ARG;
     if (p->train != 0 && p->train != 1) return MOE_ERR_INVALID_ARG;
-    if (p->train && (p->dtype != MOE_DTYPE_BF16 || p->d_ff % 128)) return MOE_ERR_UNSUPPORTED;
+    if (p->train && (p->dtype != MOE_DTYPE_BF16 || p->d_ff % 128 || p->d_ff_shared % 128)) return MOE_ERR_UNSUPPORTED;
     const long long rows = permuted_rows(*p);
     if (rows * (long long)(p->d > p->d_ff ? p->d : p->d_ff) >= (1LL << 40) || rows >= (1LL << 30))
         return MOE_ERR_UNSUPPORTED;
@@ -223,7 +233,7 @@ int run_logits(const moe_problem* p, const void* x, const void* W_r, float* logi
 int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13, const void* W1,
            const void* W3, const void* x, const void* Ws1, const void* Ws3, void* h, void* hs, int32_t* status,
            cudaStream_t st, float* part13 = nullptr, int32_t* sem13 = nullptr, bool sched_early = true,
-           void* ab = nullptr) {
+           void* ab = nullptr, void* ab_s = nullptr) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
     const int arows = (int)permuted_rows(*p);   // rows of the permuted buffers
@@ -240,6 +250,7 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
         a.K[0] = p->d; a.K[1] = p->d;
         a.out[0] = h; a.out[1] = hs;
         a.ab_out = ab;
+        a.ab_out_s = ab_s;
         a.status = status;
         if (part13 != nullptr) {
             a.partial = part13;
@@ -309,8 +320,10 @@ int run_experts(const moe_problem* p, const void* xp, const int32_t* indptr, con
                 const int32_t* tiles2, const void* W1, const void* W3, const void* W2, const void* x,
                 const void* Ws1, const void* Ws3, const void* Ws2, void* h, void* hs, void* o, void* s,
                 int32_t* status, cudaStream_t st, float* part13 = nullptr, float* part2 = nullptr,
-                int32_t* sem13 = nullptr, int32_t* sem2 = nullptr, bool sched_early = true, void* ab = nullptr) {
-    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st, part13, sem13, sched_early, ab);
+                int32_t* sem13 = nullptr, int32_t* sem2 = nullptr, bool sched_early = true, void* ab = nullptr,
+                void* ab_s = nullptr) {
+    int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st, part13, sem13, sched_early, ab,
+                    ab_s);
     if (rc != MOE_OK) return rc;
     return run_down(p, h, indptr, tiles2, W2, hs, Ws2, o, s, status, st, part2, sem2);
 }
@@ -389,17 +402,23 @@ size_t moe_backward_workspace_size(const moe_problem* p) {
 }
 
 int moe_backward(const moe_problem* p, const void* x, const void* W_r, const void* W1, const void* W3,
-                 const void* W2, const void* dy, float alpha, float beta, void* dx, float* dW_r, float* dW1,
-                 float* dW3, float* dW2, void* stats, const void* workspace, size_t workspace_bytes,
-                 void* bwd_workspace, size_t bwd_workspace_bytes, void* stream) {
+                 const void* W2, const void* Ws1, const void* Ws3, const void* Ws2, const void* dy, float alpha,
+                 float beta, void* dx, float* dW_r, float* dW1, float* dW3, float* dW2, float* dWs1, float* dWs3,
+                 float* dWs2, void* stats, const void* workspace, size_t workspace_bytes, void* bwd_workspace,
+                 size_t bwd_workspace_bytes, void* stream) {
     int rc = check_problem(p);
     if (rc != MOE_OK) return rc;
-    if (!p->train || (p->pad_rows != 64 && p->pad_rows != 128) || p->d_ff_shared > 0) return MOE_ERR_UNSUPPORTED;
+    if (!p->train || (p->pad_rows != 64 && p->pad_rows != 128) || p->E % 8) return MOE_ERR_UNSUPPORTED;
+    const bool shared = p->d_ff_shared > 0;
     if (!x || !W_r || !W1 || !W3 || !W2 || !dy || !dx || !dW_r || !dW1 || !dW3 || !dW2 || !stats)
         return MOE_ERR_INVALID_ARG;
+    if (shared && (!Ws1 || !Ws3 || !Ws2 || !dWs1 || !dWs3 || !dWs2)) return MOE_ERR_INVALID_ARG;
     for (const void* q : {x, W_r, W1, W3, W2, dy, (const void*)dx, (const void*)dW_r, (const void*)dW1,
                           (const void*)dW3, (const void*)dW2, (const void*)stats})
         if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
+    if (shared)
+        for (const void* q : {Ws1, Ws3, Ws2, (const void*)dWs1, (const void*)dWs3, (const void*)dWs2})
+            if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
     if (!std::isfinite(alpha) || !std::isfinite(beta)) return MOE_ERR_INVALID_ARG;
     const Layout L = make_layout(*p);
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -414,6 +433,12 @@ int moe_backward(const moe_problem* p, const void* x, const void* W_r, const voi
         CK(cudaMemsetAsync(dW1, 0, nw, st));
         CK(cudaMemsetAsync(dW3, 0, nw, st));
         CK(cudaMemsetAsync(dW2, 0, nw, st));
+        if (shared) {
+            const size_t ns = (size_t)p->d_ff_shared * p->d * sizeof(float);
+            CK(cudaMemsetAsync(dWs1, 0, ns, st));
+            CK(cudaMemsetAsync(dWs3, 0, ns, st));
+            CK(cudaMemsetAsync(dWs2, 0, ns, st));
+        }
         return MOE_OK;
     }
     struct PdlPass {
@@ -440,8 +465,35 @@ int moe_backward(const moe_problem* p, const void* x, const void* W_r, const voi
     CK(launch_bwd_gather(dy, ws + L.o, pos, gate, p->T, p->d, p->k, dO, dgate, st));
     g_pdl_after_first();
     CK(launch_pad_fill(p->dtype, indptr, stats, p->E, p->d, dO, nullptr, p->pad_rows, st));
-    CK(launch_router_bwd(logits, idx, gate, dgate, stats, p->T, p->E, p->k, p->gate_mode, alpha, beta, dz, st));
-    CK(launch_dwr(x, dz, p->T, p->d, p->E, reinterpret_cast<float*>(bw + B.dwr_part), dW_r, st));
+    // wide routers (E % 64 == 0) run both router GEMMs on the tensor cores
+    // with dz rounded to bf16: dW_r = x^T dz (one group of T rows, both
+    // operands MN-major) and the router term of dx, dz W_r^T (fp32 out)
+    const bool tc_router = p->E % 64 == 0;
+    void* dz16 = tc_router ? bw + B.dz16 : nullptr;
+    float* dxr = tc_router ? reinterpret_cast<float*>(bw + B.dxr) : nullptr;
+    int32_t* indptr_s = reinterpret_cast<int32_t*>(bw + B.indptr_s);
+    CK(launch_router_bwd(logits, idx, gate, dgate, stats, p->T, p->E, p->k, p->gate_mode, alpha, beta, dz, dz16,
+                         st));
+    if (tc_router) {
+        CK(launch_single_group(indptr_s, p->T, st));
+        BwdGemmArgs r = {};
+        r.mode = BW_DW2; r.indptr = indptr_s; r.tiles = nullptr; r.E = 1;
+        r.M = p->d; r.N = p->E; r.K = 0; r.d = p->d; r.d_ff = p->E;
+        r.A = x; r.a_rows = p->T; r.a_cols = p->d;
+        r.B0 = dz16; r.b_rows = p->T; r.b_cols = p->E;
+        r.out0 = dW_r; r.status = status;
+        CK(launch_bwd_gemm(r, st));
+        TcArgs a = {};
+        a.mode = TC_F32OUT; a.indptr = nullptr; a.tiles = nullptr; a.static_rows = p->T;
+        a.E = 1; a.has_shared = 0; a.T = p->T;
+        a.A[0] = dz16; a.a_rows[0] = p->T;
+        a.B[0][0] = W_r; a.B[0][1] = W_r; a.b_rows[0] = p->d; a.b_total_rows[0] = p->d;
+        a.N[0] = p->d; a.K[0] = p->E;
+        a.out[0] = dxr; a.status = status;
+        CK(launch_tc_gemm(a, st));
+    } else {
+        CK(launch_dwr(x, dz, p->T, p->d, p->E, reinterpret_cast<float*>(bw + B.dwr_part), dW_r, st));
+    }
     ScheduleSplit nosplit = {};
     CK(launch_schedule(indptr, p->E, p->T, 0, kTcTileM, ceil_div(p->d_ff, 256), ceil_div(p->d, 256), 0, 0,
                        tiles_dh, tiles_dx, nosplit, st));
@@ -475,7 +527,47 @@ int moe_backward(const moe_problem* p, const void* x, const void* W_r, const voi
     g.B0 = ws + L.xp; g.b_rows = Rmax; g.b_cols = p->d;
     g.out0 = dW1; g.out1 = dW3;
     CK(launch_bwd_gemm(g, st));
-    CK(launch_bwd_dx(dXp, pos, W_r, dz, p->T, p->d, p->E, p->k, dx, st));
+    void* dXs = nullptr;
+    if (shared) {
+        // the always-on expert: one group of all T rows, gate 1, so its output
+        // gradient is dy itself; rows are not padded (the tensor maps end at
+        // row T, so the last K-block of its weight gradients reads zeros)
+        const int dfs = p->d_ff_shared;
+        int32_t* ts_dh = reinterpret_cast<int32_t*>(bw + B.tiles_s_dh);
+        int32_t* ts_dx = reinterpret_cast<int32_t*>(bw + B.tiles_s_dx);
+        void* dABs = bw + B.dABs;
+        dXs = bw + B.dXs;
+        if (!tc_router) CK(launch_single_group(indptr_s, p->T, st));
+        CK(launch_schedule(indptr_s, 1, p->T, 0, kTcTileM, ceil_div(dfs, 256), ceil_div(p->d, 256), 0, 0, ts_dh,
+                           ts_dx, nosplit, st));
+        BwdGemmArgs s1 = {};
+        s1.indptr = indptr_s;
+        s1.E = 1;
+        s1.d = p->d;
+        s1.d_ff = dfs;
+        s1.status = status;
+        s1.mode = BW_DH; s1.tiles = ts_dh; s1.N = dfs; s1.K = p->d;
+        s1.A = dy; s1.a_rows = p->T; s1.a_cols = p->d;
+        s1.B0 = Ws2; s1.b_rows = p->d; s1.b_cols = dfs;
+        s1.ab = ws + L.abs; s1.out_bf16 = dABs;
+        CK(launch_bwd_gemm(s1, st));
+        s1.mode = BW_DX; s1.tiles = ts_dx; s1.N = p->d; s1.K = 2 * dfs;
+        s1.A = dABs; s1.a_rows = p->T; s1.a_cols = 2 * dfs;
+        s1.B0 = Ws1; s1.B1 = Ws3; s1.b_rows = dfs; s1.b_cols = p->d;
+        s1.ab = nullptr; s1.out_bf16 = dXs;
+        CK(launch_bwd_gemm(s1, st));
+        s1.mode = BW_DW2; s1.tiles = nullptr; s1.M = p->d; s1.N = dfs; s1.K = 0;
+        s1.A = dy; s1.a_rows = p->T; s1.a_cols = p->d;
+        s1.B0 = ws + L.hs; s1.B1 = nullptr; s1.b_rows = p->T; s1.b_cols = dfs;
+        s1.out_bf16 = nullptr; s1.out0 = dWs2; s1.out1 = nullptr;
+        CK(launch_bwd_gemm(s1, st));
+        s1.mode = BW_DW13; s1.M = 2 * dfs; s1.N = p->d;
+        s1.A = dABs; s1.a_rows = p->T; s1.a_cols = 2 * dfs;
+        s1.B0 = x; s1.b_rows = p->T; s1.b_cols = p->d;
+        s1.out0 = dWs1; s1.out1 = dWs3;
+        CK(launch_bwd_gemm(s1, st));
+    }
+    CK(launch_bwd_dx(dXp, pos, W_r, dz, dXs, dxr, p->T, p->d, p->E, p->k, dx, st));
     return MOE_OK;
 }
 
@@ -605,7 +697,8 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     // path writes it in the scan, two launches before
     rc = run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st, part13,
                      part2, sem, sem ? sem + L.sem13_n : nullptr, /*sched_early=*/!small,
-                     p->train ? wsp(workspace, L.ab) : nullptr);
+                     p->train ? wsp(workspace, L.ab) : nullptr,
+                     (p->train && shared) ? wsp(workspace, L.abs) : nullptr);
     if (rc != MOE_OK) return rc;
     CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st));
     return MOE_OK;

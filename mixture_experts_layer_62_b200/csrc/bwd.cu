@@ -90,7 +90,7 @@ constexpr int kMaxEPL = MOE_MAX_E / 32;   // experts per lane
 __global__ void __launch_bounds__(kWarps * 32)
 router_bwd_kernel(const float* __restrict__ logits, const int32_t* __restrict__ idx, const float* __restrict__ gate,
                   const float* __restrict__ dgate, const void* __restrict__ stats, int T, int E, int k,
-                  int gate_mode, float alpha, float beta, float* __restrict__ dz) {
+                  int gate_mode, float alpha, float beta, float* __restrict__ dz, __nv_bfloat16* __restrict__ dz16) {
     pdl_wait();
     pdl_launch();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -179,7 +179,10 @@ router_bwd_kernel(const float* __restrict__ logits, const int32_t* __restrict__ 
 #pragma unroll
     for (int i = 0; i < kMaxEPL; ++i) {
         const int e = lane + 32 * i;
-        if (i < epl && e < E) dz[static_cast<size_t>(t) * E + e] = g[i];
+        if (i < epl && e < E) {
+            dz[static_cast<size_t>(t) * E + e] = g[i];
+            if (dz16 != nullptr) dz16[static_cast<size_t>(t) * E + e] = __float2bfloat16_rn(g[i]);
+        }
     }
 }
 
@@ -243,70 +246,97 @@ dwr_reduce_kernel(const float* __restrict__ part, int nchunks, int d, int E, flo
     }
 }
 
-// dx_t = sum_j dXp[pos_{t,j}] + W_r dz_t. A thread owns 8 consecutive
-// columns of dx for a tile of kDxTok tokens; with E <= 16 its 8 rows of W_r
-// are loaded once into registers and reused across the tile (the rows of a
-// thread are contiguous but 128+ bytes apart from its neighbours', so
-// re-reading them per token was bound by L1 wavefronts); wider routers read
-// W_r per token. The tile's dz rows are staged in shared memory.
+// dx_t = sum_j dXp[pos_{t,j}] + W_r dz_t (+ the shared expert's dXs_t). A
+// thread owns 8 consecutive columns of dx for a tile of kDxTok tokens. The
+// router term reads the thread's 8 rows of W_r [d][E] once per tile: with
+// E <= 16 they are held in registers; wider routers walk the experts 8 at a
+// time (one 16-byte load per row) and accumulate the tile's tokens from each
+// load. (Rows of neighbouring threads are 8 E bytes apart, so reading them
+// per token was bound by L1 wavefronts.) The tile's dz rows are staged in
+// shared memory.
 constexpr int kDxTok = 16;
 
-template <int EG>   // EG = E / 8 uint4 per W_r row when staged in registers (1 or 2), 0: streamed
+template <int EG>   // E / 8 when E <= 16 (rows in registers), 0: E % 8 == 0, walked in groups of 8,
+                   // -1: the router term is given (dxr [T][d] fp32, from the tensor cores)
 __global__ void __launch_bounds__(256)
 bwd_dx_kernel(const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__ pos,
-              const __nv_bfloat16* __restrict__ W_r, const float* __restrict__ dz, int T, int d, int E, int k,
+              const __nv_bfloat16* __restrict__ W_r, const float* __restrict__ dz,
+              const __nv_bfloat16* __restrict__ dXs, const float* __restrict__ dxr, int T, int d, int E, int k,
               __nv_bfloat16* __restrict__ dx) {
-    extern __shared__ float dzs[];   // [kDxTok][E]
+    constexpr int TT = EG > 0 ? kDxTok : 8;   // tokens per tile
+    extern __shared__ float dzs[];             // [TT][E]
     pdl_wait();
     pdl_launch();
-    const int t0 = blockIdx.x * kDxTok;
-    const int nt = min(kDxTok, T - t0);
+    const int t0 = blockIdx.x * TT;
+    const int nt = min(TT, T - t0);
     for (int q = threadIdx.x; q < nt * E; q += blockDim.x) dzs[q] = dz[static_cast<size_t>(t0) * E + q];
     __syncthreads();
     const int v = blockIdx.y * blockDim.x + threadIdx.x;   // 8 consecutive columns
     if (v >= d / 8) return;
-    uint4 w[8][EG > 0 ? EG : 1];
-    if (EG > 0) {
+    // router term of every token of the tile, acc[tt][c]
+    float acc[TT][8];
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[tt][c] = 0.f;
+    const int groups = EG > 0 ? EG : (EG == 0 ? E / 8 : 0);
+    for (int g = 0; g < groups; ++g) {
+        float w[8][8];   // rows 8v .. 8v+7, experts 8g .. 8g+7
 #pragma unroll
         for (int c = 0; c < 8; ++c)
+            unpack8(reinterpret_cast<const uint4*>(W_r + static_cast<size_t>(8 * v + c) * E)[g], w[c]);
 #pragma unroll
-            for (int g = 0; g < EG; ++g)
-                w[c][g] = reinterpret_cast<const uint4*>(W_r + static_cast<size_t>(8 * v + c) * E)[g];
+        for (int tt = 0; tt < TT; ++tt) {
+            if (tt < nt) {
+                const float* zt = dzs + tt * E + 8 * g;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) acc[tt][c] = fmaf(w[c][q], zt[q], acc[tt][c]);
+            }
+        }
     }
-    for (int tt = 0; tt < nt; ++tt) {
-        const int t = t0 + tt;
-        const float* dzt = dzs + tt * E;
-        float acc[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    for (int tt = 0; tt < TT; ++tt) {
+        if (tt >= nt) break;
+        const int t = t0 + tt;
+        float sum[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) sum[c] = 0.f;
         for (int j = 0; j < k; ++j) {
             const int r = pos[static_cast<size_t>(t) * k + j];
             if (r < 0) continue;
             float a[8];
             unpack8(reinterpret_cast<const uint4*>(dXp + static_cast<size_t>(r) * d)[v], a);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc[c] += a[c];
+            for (int c = 0; c < 8; ++c) sum[c] += a[c];
         }
-        // router term, rows 8v .. 8v+7 of W_r [d][E], experts in order
+        if (EG >= 0) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            float s = 0.f;
-            if (EG > 0) {
+            for (int c = 0; c < 8; ++c) sum[c] += acc[tt][c];
+        } else {
+            const float4* pr = reinterpret_cast<const float4*>(dxr + static_cast<size_t>(t) * d + 8 * v);
+            const float4 r0 = pr[0], r1 = pr[1];
+            sum[0] += r0.x; sum[1] += r0.y; sum[2] += r0.z; sum[3] += r0.w;
+            sum[4] += r1.x; sum[5] += r1.y; sum[6] += r1.z; sum[7] += r1.w;
+        }
+        if (dXs != nullptr) {   // the shared expert's input gradient
+            float a[8];
+            unpack8(reinterpret_cast<const uint4*>(dXs + static_cast<size_t>(t) * d)[v], a);
 #pragma unroll
-                for (int g = 0; g < (EG > 0 ? EG : 1); ++g) {
-                    float wf[8];
-                    unpack8(w[c][g], wf);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) s = fmaf(wf[q], dzt[8 * g + q], s);
-                }
-            } else {
-                const __nv_bfloat16* wrow = W_r + static_cast<size_t>(8 * v + c) * E;
-                for (int e = 0; e < E; ++e) s = fmaf(__bfloat162float(wrow[e]), dzt[e], s);
-            }
-            acc[c] += s;
+            for (int c = 0; c < 8; ++c) sum[c] += a[c];
         }
         reinterpret_cast<uint4*>(dx + static_cast<size_t>(t) * d)[v] =
-            make_uint4(pack2(acc[0], acc[1]), pack2(acc[2], acc[3]), pack2(acc[4], acc[5]), pack2(acc[6], acc[7]));
+            make_uint4(pack2(sum[0], sum[1]), pack2(sum[2], sum[3]), pack2(sum[4], sum[5]), pack2(sum[6], sum[7]));
+    }
+}
+
+__global__ void single_group_kernel(int32_t* indptr, int T) {
+    pdl_wait();
+    pdl_launch();
+    if (threadIdx.x == 0) {
+        indptr[0] = 0;
+        indptr[1] = T;
     }
 }
 
@@ -336,10 +366,10 @@ cudaError_t launch_bwd_gather(const void* dy, const void* o, const int32_t* pos,
 
 cudaError_t launch_router_bwd(const float* logits, const int32_t* idx, const float* gate, const float* dgate,
                               const void* stats, int T, int E, int k, int gate_mode, float alpha, float beta,
-                              float* dz, cudaStream_t st) {
+                              float* dz, void* dz16, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     return launch_k(router_bwd_kernel, dim3(ceil_div(T, kWarps)), dim3(kWarps * 32), 0, st, logits, idx, gate, dgate,
-                    stats, T, E, k, gate_mode, alpha, beta, dz);
+                    stats, T, E, k, gate_mode, alpha, beta, dz, static_cast<__nv_bfloat16*>(dz16));
 }
 
 cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* part, float* dW_r,
@@ -358,18 +388,25 @@ cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, floa
                     dim3(256), 0, st, static_cast<const float*>(part), nchunks, d, E, dW_r);
 }
 
-cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, int T, int d,
-                          int E, int k, void* dx, cudaStream_t st) {
+cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, const void* dXs,
+                          const float* dxr, int T, int d, int E, int k, void* dx, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    const dim3 grid(ceil_div(T, kDxTok), ceil_div(d / 8, 256));
-    const size_t smem = sizeof(float) * kDxTok * E;
-    auto args = [&](auto kern) {
+    auto args = [&](auto kern, int tt) {
+        const dim3 grid(ceil_div(T, tt), ceil_div(d / 8, 256));
+        const size_t smem = sizeof(float) * tt * E;
         return launch_k(kern, grid, dim3(256), smem, st, static_cast<const __nv_bfloat16*>(dXp), pos,
-                        static_cast<const __nv_bfloat16*>(W_r), dz, T, d, E, k, static_cast<__nv_bfloat16*>(dx));
+                        static_cast<const __nv_bfloat16*>(W_r), dz, static_cast<const __nv_bfloat16*>(dXs), dxr, T,
+                        d, E, k, static_cast<__nv_bfloat16*>(dx));
     };
-    if (E == 8) return args(bwd_dx_kernel<1>);
-    if (E == 16) return args(bwd_dx_kernel<2>);
-    return args(bwd_dx_kernel<0>);
+    if (dxr != nullptr) return args(bwd_dx_kernel<-1>, 8);
+    if (E == 8) return args(bwd_dx_kernel<1>, kDxTok);
+    if (E == 16) return args(bwd_dx_kernel<2>, kDxTok);
+    if (E % 8 == 0) return args(bwd_dx_kernel<0>, 8);
+    return cudaErrorNotSupported;   // the backward requires E % 8 == 0
+}
+
+cudaError_t launch_single_group(int32_t* indptr, int T, cudaStream_t st) {
+    return launch_k(single_group_kernel, dim3(1), dim3(32), 0, st, indptr, T);
 }
 
 cudaError_t launch_bias_update(const void* stats, int T, int E, int k, float gamma, float* bias, cudaStream_t st) {

@@ -62,6 +62,7 @@ struct Layout {
     size_t blockcnt, blockoff, blockpsum, blockextra, tiles13, tiles2;
     size_t xp, h, o, hs, s;
     size_t ab;              // gate/up pre-activations kept for the backward (train)
+    size_t abs;             // the shared expert's, [T][2 d_ff_shared] (train)
     size_t part13, part2;   // fp32 split-K partials (small-T forward only)
     size_t sem;             // split-K arrival counters: [sem13_n] then [sem2_n]
     int sem13_n, sem2_n;
@@ -80,7 +81,10 @@ Layout make_layout(const moe_problem& p);
 long long permuted_rows(const moe_problem& p);
 // Byte offsets of the backward pass's own workspace.
 struct BwdLayout {
-    size_t dO, dAB, dXp, dz, dgate, tiles_dh, tiles_dx, dwr_part, total;
+    size_t dO, dAB, dXp, dz, dgate, tiles_dh, tiles_dx, dwr_part;
+    size_t dz16, dxr;   // wide routers (E % 64 == 0): bf16 dz and the router term of dx
+    size_t dABs, dXs, indptr_s, tiles_s_dh, tiles_s_dx;   // shared expert
+    size_t total;
 };
 BwdLayout make_bwd_layout(const moe_problem& p);
 
@@ -225,6 +229,7 @@ struct TcArgs {
     int32_t* sem;              // split-K arrival counters [tiles][kSemPerTile] (with partial)
     void* ab_out;              // SWIGLU, routed groups: also store the raw gate/up
                                // accumulators as bf16 [rows][2 N] (null: not kept)
+    void* ab_out_s;            // SWIGLU, the shared expert's rows: the same [T][2 N1]
     // the tile schedule (indptr, tiles) was written two or more launches
     // back, so the weight loads of the first stages may start before the
     // dependency wait
@@ -250,14 +255,19 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, cudaStream_t st);
 // Backward elementwise and reduction kernels: see bwd.cu.
 cudaError_t launch_bwd_gather(const void* dy, const void* o, const int32_t* pos, const float* gate, int T, int d,
                               int k, void* dO, float* dgate, cudaStream_t st);
+// dz16 (may be null): a bf16 copy of dz for the tensor-core router GEMMs
 cudaError_t launch_router_bwd(const float* logits, const int32_t* idx, const float* gate, const float* dgate,
                               const void* stats, int T, int E, int k, int gate_mode, float alpha, float beta,
-                              float* dz, cudaStream_t st);
+                              float* dz, void* dz16, cudaStream_t st);
 // dW_r = x^T dz via fp32 partials over 128-token chunks (part: ceil(T/128) * d * E floats)
 cudaError_t launch_dwr(const void* x, const float* dz, int T, int d, int E, float* part, float* dW_r,
                        cudaStream_t st);
-cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, int T, int d,
-                          int E, int k, void* dx, cudaStream_t st);
+// dx = sum_j dXp[pos] + W_r dz (+ dXs, the shared expert's input gradient, when not null);
+// dxr (may be null): the router term W_r dz already computed, fp32 [T][d]
+cudaError_t launch_bwd_dx(const void* dXp, const int32_t* pos, const void* W_r, const float* dz, const void* dXs,
+                          const float* dxr, int T, int d, int E, int k, void* dx, cudaStream_t st);
+// indptr = {0, T}: the shared expert as one group over all tokens
+cudaError_t launch_single_group(int32_t* indptr, int T, cudaStream_t st);
 cudaError_t launch_bias_update(const void* stats, int T, int E, int k, float gamma, float* bias, cudaStream_t st);
 
 // A cached 2-D bf16 tensor map over a row-major [rows, cols] matrix: box 64

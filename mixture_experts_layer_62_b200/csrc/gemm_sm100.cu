@@ -69,6 +69,7 @@ struct KParams {
     int partial_ld;            // elements per partial row
     int32_t* sem;              // split-K arrival counters [tile][kSemPerTile]
     __nv_bfloat16* ab_out;     // SWIGLU: raw gate/up accumulators of routed rows, or null
+    __nv_bfloat16* ab_out_s;   // SWIGLU: the same for the shared expert's rows, or null
     int b_before_wait;         // weight tiles of the first stages may load before the dependency wait
 };
 
@@ -451,8 +452,9 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
                 // training: the gate and up pre-activations of the tile, in the
                 // accumulator's own column order ([128 gate | 128 up] per tile)
-                __nv_bfloat16* abrow = (p.ab_out != nullptr && t.kind == 0)
-                                           ? p.ab_out + orow * (2 * static_cast<size_t>(N)) + t.n_blk * 256
+                __nv_bfloat16* abbase = t.kind == 0 ? p.ab_out : p.ab_out_s;
+                __nv_bfloat16* abrow = abbase != nullptr
+                                           ? abbase + orow * (2 * static_cast<size_t>(N)) + t.n_blk * 256
                                            : nullptr;
 #pragma unroll 1
                 for (int c = 0; c < 128; c += 32) {
@@ -670,6 +672,7 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     kp.partial_ld = a.partial_ld;
     kp.sem = a.sem;
     kp.ab_out = static_cast<__nv_bfloat16*>(a.ab_out);
+    kp.ab_out_s = static_cast<__nv_bfloat16*>(a.ab_out_s);
     kp.b_before_wait = a.b_before_wait;
     if (kp.partial != nullptr && kp.sem == nullptr) return cudaErrorInvalidValue;
     switch (a.mode) {

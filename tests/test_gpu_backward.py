@@ -45,12 +45,18 @@ def _layer(cfg, seed):
         L["bias"] = torch.linspace(0.5, -0.5, E)
     elif cfg.get("bias_mode", 0) == O.BIAS_PROB:
         L["bias"] = torch.rand((E,), generator=g) * 0.2 - 0.1
+    dfs = cfg.get("d_ff_shared", 0)
+    L["Ws1"] = L["Ws3"] = L["Ws2"] = None
+    if dfs:
+        L["Ws1"] = (torch.randn((dfs, d), generator=g) / math.sqrt(d)).to(bf)
+        L["Ws3"] = (torch.randn((dfs, d), generator=g) / math.sqrt(d)).to(bf)
+        L["Ws2"] = (torch.randn((d, dfs), generator=g) / math.sqrt(dfs)).to(bf)
     return L
 
 
 def _problem(cfg):
     return moe.problem(cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg.get("cf", 0.0), "bf16",
-                       cfg.get("bias_mode", 0), 0, cfg.get("gate", 0), cfg.get("drop", 0),
+                       cfg.get("bias_mode", 0), cfg.get("d_ff_shared", 0), cfg.get("gate", 0), cfg.get("drop", 0),
                        pad_rows=cfg["pad"], train=1)
 
 
@@ -61,15 +67,23 @@ def _gpu(cfg, L):
     ws = moe.alloc_workspace(p, DEV)
     st = moe.alloc_stats(E, DEV)
     out = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
-    moe.forward(p, D["x"], D["W_r"], D["W1"], D["W3"], D["W2"], out, st, ws, bias=D["bias"])
+    moe.forward(p, D["x"], D["W_r"], D["W1"], D["W3"], D["W2"], out, st, ws, bias=D["bias"], Ws1=D["Ws1"],
+                Ws3=D["Ws3"], Ws2=D["Ws2"])
     bws = moe.alloc_backward_workspace(p, DEV)
     G = dict(dx=torch.full((T, d), float("nan"), dtype=torch.bfloat16, device=DEV),
              dW_r=torch.full((d, E), float("nan"), device=DEV),
              dW1=torch.full((E, dff, d), float("nan"), device=DEV),
              dW3=torch.full((E, dff, d), float("nan"), device=DEV),
              dW2=torch.full((E, d, dff), float("nan"), device=DEV))
+    dfs = cfg.get("d_ff_shared", 0)
+    if dfs:
+        G.update(dWs1=torch.full((dfs, d), float("nan"), device=DEV),
+                 dWs3=torch.full((dfs, d), float("nan"), device=DEV),
+                 dWs2=torch.full((d, dfs), float("nan"), device=DEV))
     moe.backward(p, D["x"], D["W_r"], D["W1"], D["W3"], D["W2"], D["dy"], G["dx"], G["dW_r"], G["dW1"],
-                 G["dW3"], G["dW2"], st, ws, bws, alpha=cfg.get("alpha", 0.0), beta=cfg.get("beta", 0.0))
+                 G["dW3"], G["dW2"], st, ws, bws, alpha=cfg.get("alpha", 0.0), beta=cfg.get("beta", 0.0),
+                 Ws1=D["Ws1"], Ws3=D["Ws3"], Ws2=D["Ws2"], dWs1=G.get("dWs1"), dWs3=G.get("dWs3"),
+                 dWs2=G.get("dWs2"))
     torch.cuda.synchronize()
     assert moe.read_stats(st, E).status == moe.MOE_OK
     logits = moe.workspace_view(ws, p, "logits").cpu().numpy()
@@ -89,8 +103,9 @@ def _oracle(cfg, L, logits, idx):
     if exact:
         own = O.route(logits, cfg["k"], bias, cfg.get("bias_mode", 0), key_dtype=np.float32)
         assert np.array_equal(own.idx, idx)
+    sh = {n: (None if L[n] is None else f(L[n])) for n in ("Ws1", "Ws3", "Ws2")}
     return B.moe_backward(f(L["x"]), f(L["W_r"]), f(L["W1"]), f(L["W3"]), f(L["W2"]), cfg["k"], f(L["dy"]),
-                          cfg.get("cf", 0.0), bias, cfg.get("bias_mode", 0), alpha=cfg.get("alpha", 0.0),
+                          cfg.get("cf", 0.0), bias, cfg.get("bias_mode", 0), **sh, alpha=cfg.get("alpha", 0.0),
                           beta=cfg.get("beta", 0.0), gate_mode=cfg.get("gate", 0), drop_order=cfg.get("drop", 0),
                           logits=logits, key_dtype=np.float32 if exact else np.float64, idx=idx)
 
@@ -122,11 +137,16 @@ CASES = [
     dict(T=64, d=128, d_ff=128, E=32, k=2, pad=64, bias_mode=O.BIAS_PROB),
     # many tiles in every GEMM: 8 experts x ~512 rows, d = 1024, d_ff = 2048
     dict(T=2048, d=1024, d_ff=2048, E=8, k=2, cf=1.0, pad=128, alpha=0.01, beta=0.001),
+    # fine-grained experts with an always-on shared expert (T not a multiple of 64)
+    dict(T=300, d=256, d_ff=128, E=32, k=4, pad=64, bias_mode=O.BIAS_PROB, d_ff_shared=256, alpha=0.02),
+    # E % 64 == 0: both router GEMMs of the backward on the tensor cores
+    dict(T=260, d=512, d_ff=128, E=64, k=4, pad=64, d_ff_shared=128, alpha=0.05, beta=0.01),
+    dict(T=100, d=256, d_ff=256, E=128, k=2, cf=1.0, pad=128, bias_mode=O.BIAS_LOGIT, alpha=0.1),
 ]
 
 
 @pytest.mark.parametrize("cfg", CASES, ids=[f"T{c['T']}_d{c['d']}_f{c['d_ff']}_E{c['E']}_k{c['k']}_p{c['pad']}"
-                                            for c in CASES])
+                                            f"_s{c.get('d_ff_shared', 0)}" for c in CASES])
 def test_backward_matches_oracle(cfg):
     L = _layer(cfg, seed=cfg["T"] + cfg["E"])
     p, ws, st, G, logits = _gpu(cfg, L)
@@ -135,6 +155,9 @@ def test_backward_matches_oracle(cfg):
     _compare("dW_r", G["dW_r"][None], ref.dW_r[None], per_matrix=True)
     for n in ("dW1", "dW3", "dW2"):
         _compare(n, G[n], getattr(ref, n), per_matrix=True)
+    if cfg.get("d_ff_shared", 0):
+        for n in ("dWs1", "dWs3", "dWs2"):
+            _compare(n, G[n][None], getattr(ref, n)[None], per_matrix=True)
     # experts that received no rows get exactly zero weight gradients
     s = moe.read_stats(st, cfg["E"])
     for e, kept in enumerate(s.kept):
