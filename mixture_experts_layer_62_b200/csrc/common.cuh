@@ -274,6 +274,8 @@ cudaError_t launch_bias_update(const void* stats, int T, int E, int k, float gam
 // columns x box_rows rows, 128-byte swizzle, zeros outside (CUtensorMap is
 // the driver type; passed as void* so this header needs no driver header).
 bool make_tmap(void* map, const void* base, int rows, int cols, int box_rows);
+// A cached 2-D fp32 tensor map for bulk stores: box 32 x 32, 128-byte swizzle.
+bool make_tmap_f32_store(void* map, const float* base, int rows, int cols);
 
 int device_sm_count();
 

@@ -46,9 +46,10 @@ constexpr int MN_CHUNK = 64 * BK * 2;         // one 64-wide chunk of an MN-majo
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int NUM_THREADS = 192;
-constexpr int STAGE_PITCH = 33;               // floats per staged row (conflict-free banks)
-constexpr int STAGE_WARP_BYTES = 32 * STAGE_PITCH * 4;   // one epilogue warp's 32 x 32 fp32 block
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + 4 * STAGE_WARP_BYTES;
+constexpr int OUT_BLOCK = 32 * 32 * 4;        // one 32 x 32 fp32 block, 128-byte swizzled rows
+constexpr int OUT_WARP_BYTES = 2 * OUT_BLOCK;  // double-buffered per epilogue warp
+constexpr int CTL_BYTES = 1024;                // barriers; keeps the output blocks 1024-byte aligned
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + CTL_BYTES + 4 * OUT_WARP_BYTES;
 
 struct BParams {
     const int32_t* indptr;    // padded row offsets of the groups [E+1]
@@ -183,11 +184,13 @@ __device__ __forceinline__ void issue_stage(const BParams& p, const BTile& t, in
 template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
-            const __grid_constant__ CUtensorMap mB1, const BParams p) {
+            const __grid_constant__ CUtensorMap mB1, const __grid_constant__ CUtensorMap mO0,
+            const __grid_constant__ CUtensorMap mO1, const BParams p) {
     constexpr bool A_MN = (MODE == BW_DW2 || MODE == BW_DW13);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+    static_assert(sizeof(Ctl) <= CTL_BYTES, "barrier block");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -205,6 +208,8 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUte
         prefetch_map(&mA);
         prefetch_map(&mB0);
         prefetch_map(&mB1);
+        prefetch_map(&mO0);
+        prefetch_map(&mO1);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -287,7 +292,8 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUte
         const int r = q * 32 + lane;
         int acc = 0;
         uint32_t aph = 0;
-        float* stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256) + q * (32 * STAGE_PITCH);
+        uint8_t* outbuf = smem + STAGES * STAGE_BYTES + CTL_BYTES + q * OUT_WARP_BYTES;
+        int nstore = 0;   // bulk stores this warp has issued (buffer = nstore & 1)
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
             const BTile t = decode<MODE>(p, u);
             if (MODE == BW_DH) {
@@ -377,48 +383,48 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUte
                     }
                 }
             } else {
-                // weight gradients, fp32: BW_DW2 row m of dW2_e; BW_DW13 row of
+                // weight gradients, fp32: BW_DW2 rows of dW2_e; BW_DW13 rows of
                 // dW1_e (gate half of a 256-row AB group) or dW3_e (up half).
-                // Each 32 x 32 block of the warp goes through shared memory so
-                // that global stores cover whole 128-byte row segments.
+                // Each 32 x 32 block of the warp is written to shared memory in
+                // the 128-byte-swizzled layout of the output map and stored by
+                // one bulk tensor store; two buffers per warp let the next block
+                // be written while the previous store still reads.
                 if (!wait_b(&ctl->tfull[acc], aph, ctl, p)) break;
                 tc_fence_after();
                 const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                     static_cast<uint32_t>(acc * ACC_COLS);
                 const bool empty_k = t.num_kb == 0;   // an expert without rows: its gradient is 0
-                const int m0 = t.m_blk * BM + q * 32;  // first row of this warp's block
-                float* base;
-                int rows_ok;                           // valid rows of the block
+                const CUtensorMap* mo;
+                int orow;                              // first output row of this warp's block
                 if (MODE == BW_DW2) {
-                    base = p.out0 + (static_cast<size_t>(t.g) * p.M + m0) * static_cast<size_t>(p.N);
-                    rows_ok = min(32, p.M - m0);
+                    mo = &mO0;
+                    orow = t.g * p.M + t.m_blk * BM + q * 32;
                 } else {
-                    const int w0 = (t.m_blk >> 1) * 128 + q * 32;
-                    base = ((t.m_blk & 1) ? p.out1 : p.out0) +
-                           (static_cast<size_t>(t.g) * p.d_ff + w0) * static_cast<size_t>(p.N);
-                    rows_ok = min(32, p.d_ff - w0);
+                    mo = (t.m_blk & 1) ? &mO1 : &mO0;
+                    orow = t.g * p.d_ff + (t.m_blk >> 1) * 128 + q * 32;
                 }
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 32) {
                     uint32_t v[32];
                     if (!empty_k) tmem_ld32(tb + c, v);
                     const int col = t.n_blk * BN + c;
-                    if (col >= p.N) continue;         // the same for the whole warp
+                    if (col >= p.N) continue;          // the same for the whole warp
+                    uint8_t* buf = outbuf + (nstore & 1) * OUT_BLOCK;
+                    if (lane == 0) bulk_wait_read<1>();   // the store two blocks back has read `buf`
                     __syncwarp();
+                    uint8_t* rowp = buf + lane * 128;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) stage[lane * STAGE_PITCH + i] = empty_k ? 0.f : __uint_as_float(v[i]);
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+                            empty_k ? make_uint4(0u, 0u, 0u, 0u)
+                                    : make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    fence_proxy_async_smem();
                     __syncwarp();
-                    // lanes 8q..8q+7 write row 4 i + q's 32 columns (128 bytes)
-                    const int rl = lane >> 3, cl = (lane & 7) * 4;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int rr = 4 * i + rl;
-                        if (rr < rows_ok) {
-                            const float* sp = stage + rr * STAGE_PITCH + cl;
-                            *reinterpret_cast<float4*>(base + static_cast<size_t>(rr) * p.N + col + cl) =
-                                make_float4(sp[0], sp[1], sp[2], sp[3]);
-                        }
+                    if (lane == 0) {
+                        tma_store_2d(mo, smem_u32(buf), col, orow);
+                        bulk_commit();
                     }
+                    ++nstore;
                 }
             }
             tc_fence_before();
@@ -427,6 +433,7 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUte
             acc ^= 1;
             if (acc == 0) aph ^= 1u;
         }
+        if (lane == 0) bulk_wait_all();   // every bulk store of this warp has completed
     }
 
     tc_fence_before();
@@ -440,7 +447,7 @@ tc_bwd_gemm(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUte
 }
 
 template <int MODE>
-cudaError_t launch_bwd_mode(const CUtensorMap (&maps)[3], const BParams& bp, cudaStream_t st) {
+cudaError_t launch_bwd_mode(const CUtensorMap (&maps)[5], const BParams& bp, cudaStream_t st) {
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -453,18 +460,29 @@ cudaError_t launch_bwd_mode(const CUtensorMap (&maps)[3], const BParams& bp, cud
     const int grid = device_sm_count();
     if (grid <= 0) return cudaErrorInvalidDevice;
     return launch_k(tc_bwd_gemm<MODE>, dim3(grid), dim3(NUM_THREADS), (size_t)SMEM_BYTES, st, maps[0], maps[1],
-                    maps[2], bp);
+                    maps[2], maps[3], maps[4], bp);
 }
 
 }  // namespace
 
 cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, cudaStream_t st) {
-    CUtensorMap maps[3];
+    CUtensorMap maps[5];
     const bool a_mn = a.mode == BW_DW2 || a.mode == BW_DW13;
     // K-major operands: boxes of 64 K x 128 rows; MN-major: 64 columns x 64 K rows
     if (!make_tmap(&maps[0], a.A, a.a_rows, a.a_cols, a_mn ? 64 : 128)) return cudaErrorInvalidValue;
     if (!make_tmap(&maps[1], a.B0, a.b_rows, a.b_cols, 64)) return cudaErrorInvalidValue;
     if (!make_tmap(&maps[2], a.B1 != nullptr ? a.B1 : a.B0, a.b_rows, a.b_cols, 64)) return cudaErrorInvalidValue;
+    // weight-gradient outputs, fp32 [groups * rows][N] for bulk stores
+    if (a.mode == BW_DW2) {
+        if (!make_tmap_f32_store(&maps[3], a.out0, a.E * a.M, a.N)) return cudaErrorInvalidValue;
+        maps[4] = maps[3];
+    } else if (a.mode == BW_DW13) {
+        if (!make_tmap_f32_store(&maps[3], a.out0, a.E * a.d_ff, a.N)) return cudaErrorInvalidValue;
+        if (!make_tmap_f32_store(&maps[4], a.out1, a.E * a.d_ff, a.N)) return cudaErrorInvalidValue;
+    } else {
+        maps[3] = maps[0];
+        maps[4] = maps[0];
+    }
     BParams bp;
     bp.indptr = a.indptr;
     bp.tiles = a.tiles;

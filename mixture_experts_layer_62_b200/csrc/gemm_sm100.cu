@@ -599,11 +599,22 @@ bool make_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows
     return true;
 }
 
+// box_rows == kF32StoreBox: an fp32 matrix with 32 x 32 boxes (128-byte rows),
+// the layout of the weight-gradient stores
+constexpr int kF32StoreBox = -32;
+
 bool encode_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows > 0 ? rows : 1)};
+    cuuint32_t estr[2] = {1, 1};
+    if (box_rows == kF32StoreBox) {
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+        cuuint32_t box[2] = {32, 32};
+        return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
     cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -633,6 +644,10 @@ int tc_out_cols_per_tile(int mode) { return mode == TC_SWIGLU ? 128 : 256; }
 
 bool make_tmap(void* m, const void* base, int rows, int cols, int box_rows) {
     return get_encode() && make_map(static_cast<CUtensorMap*>(m), base, rows, cols, box_rows);
+}
+
+bool make_tmap_f32_store(void* m, const float* base, int rows, int cols) {
+    return get_encode() && make_map(static_cast<CUtensorMap*>(m), base, rows, cols, kF32StoreBox);
 }
 
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {

@@ -103,6 +103,21 @@ constexpr uint32_t make_idesc(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Bulk tensor store of a 2-D box from shared memory (the smem image in the
+// map's swizzled layout); completion is tracked by bulk async-groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(src) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N committed groups still read shared memory
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+// wait until every committed group has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// generic-proxy shared-memory writes become visible to the async proxy (TMA)
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // Shared-memory descriptor of an MN-major operand, 128-byte swizzle: the
 // operand is stored as 64-element (128-byte) runs along M or N, one run per
 // K index, 8 K rows per 1024-byte swizzle atom (stride byte offset 1024), and
