@@ -18,6 +18,10 @@ template <> struct VecTraits<float> {
         float4 a = *reinterpret_cast<const float4*>(p);
         v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     }
+    __device__ static void unpack(const uint4& u, float (&v)[4]) {
+        v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+        v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+    }
     __device__ static void store(void* p, const float (&v)[4]) {
         *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
     }
@@ -26,6 +30,9 @@ template <> struct VecTraits<__nv_bfloat16> {
     static constexpr int N = 8;
     __device__ static void load(const void* p, float (&v)[8]) {
         uint4 u = *reinterpret_cast<const uint4*>(p);
+        unpack(u, v);
+    }
+    __device__ static void unpack(const uint4& u, float (&v)[8]) {
         const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -57,40 +64,57 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const f
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long task = (long long)blockIdx.x * kCbWarps + warp;
     const int t = (int)(task / slices), sl = (int)(task % slices);
-    // pos and gate come from the routing, at least two launches back (both
-    // GEMMs run after it), so they are read before the dependency wait; the
-    // expert outputs are read after it
-    int p[MOE_MAX_K];
-    float g[MOE_MAX_K];
-    if (t < Tn) {
-#pragma unroll
-        for (int j = 0; j < MOE_MAX_K; ++j) {
-            if (j < k) {
-                p[j] = pos[(size_t)t * k + j];
-                g[j] = gate[(size_t)t * k + j];
-            }
-        }
+    if (t >= Tn) {
+        pdl_wait();
+        pdl_launch();
+        return;
+    }
+    // lane j holds the slot-j position and gate of the warp's token (k <= 32);
+    // they come from the routing, at least two launches back (both GEMMs run
+    // after it), so they are read before the dependency wait; the expert
+    // outputs are read after it
+    int p_l = -1;
+    float g_l = 0.f;
+    if (lane < k) {
+        p_l = pos[(size_t)t * k + lane];
+        g_l = gate[(size_t)t * k + lane];
     }
     pdl_wait();
     pdl_launch();
-    if (t >= Tn) return;
     const int nvec = d / VN;
-#pragma unroll 2
     for (int i = 0; i < vpl; ++i) {
-        const int v = (sl * vpl + i) * 32 + lane;
-        if (v >= nvec) break;
+        const int v0 = (sl * vpl + i) * 32;
+        if (v0 >= nvec) break;  // warp-uniform
+        const int v = v0 + lane;
+        const bool valid = v < nvec;
         float acc[VN];
 #pragma unroll
         for (int e = 0; e < VN; ++e) acc[e] = 0.f;
-#pragma unroll 4
-        for (int j = 0; j < MOE_MAX_K; ++j) {
-            if (j < k && p[j] >= 0) {
-                float ov[VN];
-                V::load(o + (size_t)p[j] * d + (size_t)v * VN, ov);
+        // slots in groups of 4: the group's rows are all requested before any
+        // is accumulated (slot order is kept)
+        for (int j0 = 0; j0 < k; j0 += 4) {
+            uint4 raw[4];
+            int pj[4];
+            float gj[4];
 #pragma unroll
-                for (int e = 0; e < VN; ++e) acc[e] = fmaf(g[j], ov[e], acc[e]);
+            for (int u = 0; u < 4; ++u) {
+                pj[u] = __shfl_sync(0xffffffffu, p_l, j0 + u);
+                gj[u] = __shfl_sync(0xffffffffu, g_l, j0 + u);
+                raw[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (j0 + u < k && pj[u] >= 0 && valid)
+                    raw[u] = *reinterpret_cast<const uint4*>(o + (size_t)pj[u] * d + (size_t)v * VN);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (j0 + u < k && pj[u] >= 0) {
+                    float ov[VN];
+                    V::unpack(raw[u], ov);
+#pragma unroll
+                    for (int e = 0; e < VN; ++e) acc[e] = fmaf(gj[u], ov[e], acc[e]);
+                }
             }
         }
+        if (!valid) continue;
         if (s != nullptr) {
             float sv[VN];
             V::load(s + (size_t)t * d + (size_t)v * VN, sv);
