@@ -273,36 +273,9 @@ bwd_dx_kernel(const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__
     __syncthreads();
     const int v = blockIdx.y * blockDim.x + threadIdx.x;   // 8 consecutive columns
     if (v >= d / 8) return;
-    // router term of every token of the tile, acc[tt][c]
-    float acc[TT][8];
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[tt][c] = 0.f;
-    const int groups = EG > 0 ? EG : (EG == 0 ? E / 8 : 0);
-    for (int g = 0; g < groups; ++g) {
-        float w[8][8];   // rows 8v .. 8v+7, experts 8g .. 8g+7
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            unpack8(reinterpret_cast<const uint4*>(W_r + static_cast<size_t>(8 * v + c) * E)[g], w[c]);
-#pragma unroll
-        for (int tt = 0; tt < TT; ++tt) {
-            if (tt < nt) {
-                const float* zt = dzs + tt * E + 8 * g;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) acc[tt][c] = fmaf(w[c][q], zt[q], acc[tt][c]);
-            }
-        }
-    }
-#pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-        if (tt >= nt) break;
-        const int t = t0 + tt;
-        float sum[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) sum[c] = 0.f;
+    // sum of the token's kept rows of dXp, plus the shared expert's input
+    // gradient when there is one
+    auto expert_terms = [&](int t, float (&sum)[8]) {
         for (int j = 0; j < k; ++j) {
             const int r = pos[static_cast<size_t>(t) * k + j];
             if (r < 0) continue;
@@ -311,23 +284,86 @@ bwd_dx_kernel(const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__
 #pragma unroll
             for (int c = 0; c < 8; ++c) sum[c] += a[c];
         }
-        if (EG >= 0) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) sum[c] += acc[tt][c];
-        } else {
-            const float4* pr = reinterpret_cast<const float4*>(dxr + static_cast<size_t>(t) * d + 8 * v);
-            const float4 r0 = pr[0], r1 = pr[1];
-            sum[0] += r0.x; sum[1] += r0.y; sum[2] += r0.z; sum[3] += r0.w;
-            sum[4] += r1.x; sum[5] += r1.y; sum[6] += r1.z; sum[7] += r1.w;
-        }
-        if (dXs != nullptr) {   // the shared expert's input gradient
+        if (dXs != nullptr) {
             float a[8];
             unpack8(reinterpret_cast<const uint4*>(dXs + static_cast<size_t>(t) * d)[v], a);
 #pragma unroll
             for (int c = 0; c < 8; ++c) sum[c] += a[c];
         }
+    };
+    auto store = [&](int t, const float (&sum)[8]) {
         reinterpret_cast<uint4*>(dx + static_cast<size_t>(t) * d)[v] =
             make_uint4(pack2(sum[0], sum[1]), pack2(sum[2], sum[3]), pack2(sum[4], sum[5]), pack2(sum[6], sum[7]));
+    };
+    if constexpr (EG > 0) {
+        // few experts: rows 8v .. 8v+7 of W_r stay packed in registers, the
+        // router term is formed token by token
+        uint4 w[8][EG > 0 ? EG : 1];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+            for (int g = 0; g < EG; ++g)
+                w[c][g] = reinterpret_cast<const uint4*>(W_r + static_cast<size_t>(8 * v + c) * E)[g];
+        for (int tt = 0; tt < nt; ++tt) {
+            const float* zt = dzs + tt * E;
+            float sum[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float acc = 0.f;
+#pragma unroll
+                for (int g = 0; g < EG; ++g) {
+                    float wf[8];
+                    unpack8(w[c][g], wf);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) acc = fmaf(wf[q], zt[8 * g + q], acc);
+                }
+                sum[c] = acc;
+            }
+            expert_terms(t0 + tt, sum);
+            store(t0 + tt, sum);
+        }
+    } else {
+        // router term of every token of the tile, acc[tt][c]: each group of
+        // 8 experts' W_r rows is loaded once for the TT tokens
+        float acc[TT][8];
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[tt][c] = 0.f;
+        const int groups = EG == 0 ? E / 8 : 0;
+        for (int g = 0; g < groups; ++g) {
+            float w[8][8];   // rows 8v .. 8v+7, experts 8g .. 8g+7
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                unpack8(reinterpret_cast<const uint4*>(W_r + static_cast<size_t>(8 * v + c) * E)[g], w[c]);
+#pragma unroll
+            for (int tt = 0; tt < TT; ++tt) {
+                if (tt < nt) {
+                    const float* zt = dzs + tt * E + 8 * g;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) acc[tt][c] = fmaf(w[c][q], zt[q], acc[tt][c]);
+                }
+            }
+        }
+#pragma unroll
+        for (int tt = 0; tt < TT; ++tt) {
+            if (tt >= nt) break;
+            const int t = t0 + tt;
+            float sum[8];
+            if (EG == 0) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) sum[c] = acc[tt][c];
+            } else {   // the router term comes from the tensor cores
+                const float4* pr = reinterpret_cast<const float4*>(dxr + static_cast<size_t>(t) * d + 8 * v);
+                const float4 r0 = pr[0], r1 = pr[1];
+                sum[0] = r0.x; sum[1] = r0.y; sum[2] = r0.z; sum[3] = r0.w;
+                sum[4] = r1.x; sum[5] = r1.y; sum[6] = r1.z; sum[7] = r1.w;
+            }
+            expert_terms(t, sum);
+            store(t, sum);
+        }
     }
 }
 
