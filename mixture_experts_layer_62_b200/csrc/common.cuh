@@ -189,6 +189,7 @@ struct SmallRouteArgs {
 };
 bool small_route_ok(const moe_problem& p);
 cudaError_t launch_route_small(const SmallRouteArgs& a, cudaStream_t st);
+int small_route_parts(int d);   // partial-logit blocks per token for row width d
 
 // fp32 grouped GEMM on CUDA cores (the fp32 path). Tile 64 x 64.
 constexpr int kSimtTileM = 64;

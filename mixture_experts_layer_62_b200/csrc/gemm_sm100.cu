@@ -15,7 +15,9 @@
 //    out group by group, and inside a group the 128-row M blocks vary
 //    fastest, so CTAs that run at the same time share one weight tile (read
 //    from HBM once, the others hit L2) and a group's activation rows stay in
-//    L2 across its N blocks;
+//    L2 across its N blocks; a group whose rows would not fit in L2 is cut
+//    into bands of M blocks (about 32 MB of rows each) that run one after
+//    the other, each over all N blocks;
 //  * warp 0: one thread issues TMA loads (A 128x64, B 2 x 128x64, 128-byte
 //    swizzle) into a 4-stage ring guarded by full/empty mbarriers;
 //  * warp 1: one thread issues tcgen05.mma (M=128, N=256, K=16, bf16 in,
@@ -31,6 +33,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -53,6 +56,9 @@ constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 2 * ACC_COLS;
 constexpr int NUM_THREADS = 192;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+#ifndef MOE_RASTER_BYTES
+#define MOE_RASTER_BYTES (32ll << 20)   // activation rows of one band of M blocks (0: no bands)
+#endif
 
 struct KParams {
     const int32_t* indptr;
@@ -71,6 +77,8 @@ struct KParams {
     __nv_bfloat16* ab_out;     // SWIGLU: raw gate/up accumulators of routed rows, or null
     __nv_bfloat16* ab_out_s;   // SWIGLU: the same for the shared expert's rows, or null
     int b_before_wait;         // weight tiles of the first stages may load before the dependency wait
+    int nt_blk[2];             // N blocks of a group (routed, shared)
+    int band_m[2];             // M blocks per band (0: the whole group is one band)
 };
 
 struct Tile {
@@ -100,8 +108,18 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, int tile) {
         tile -= p.tiles[lo];
     }
     const int mt = (t.rows + BM - 1) / BM;
-    t.n_blk = tile / mt;
-    t.m_blk = tile % mt;
+    // bands of band_m M blocks, each over all N blocks, M fastest inside a band
+    int h = mt, m0 = 0;
+    const int bm = p.band_m[t.kind];
+    if (bm > 0 && bm < mt) {
+        const int per_band = bm * p.nt_blk[t.kind];
+        const int band = tile / per_band;
+        tile -= band * per_band;
+        m0 = band * bm;
+        h = min(bm, mt - m0);
+    }
+    t.n_blk = tile / h;
+    t.m_blk = m0 + tile % h;
     t.num_kb = (p.K[t.kind] + BK - 1) / BK;
     return t;
 }
@@ -689,6 +707,12 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     kp.ab_out = static_cast<__nv_bfloat16*>(a.ab_out);
     kp.ab_out_s = static_cast<__nv_bfloat16*>(a.ab_out_s);
     kp.b_before_wait = a.b_before_wait;
+    const int cols = tc_out_cols_per_tile(a.mode);
+    for (int kd = 0; kd < 2; ++kd) {
+        kp.nt_blk[kd] = ceil_div(a.N[kd] > 0 ? a.N[kd] : 1, cols);
+        const long long row_bytes = static_cast<long long>(BM) * (a.K[kd] > 0 ? a.K[kd] : 1) * 2;
+        kp.band_m[kd] = MOE_RASTER_BYTES > 0 ? static_cast<int>(std::max(8ll, MOE_RASTER_BYTES / row_bytes)) : 0;
+    }
     if (kp.partial != nullptr && kp.sem == nullptr) return cudaErrorInvalidValue;
     switch (a.mode) {
         case TC_SWIGLU: return launch_mode<TC_SWIGLU>(a, kp, maps, st);

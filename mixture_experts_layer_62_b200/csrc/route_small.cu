@@ -14,22 +14,14 @@
 // Reductions run in a fixed order (the summation trees differ from the
 // general path's, so the two paths agree to fp32 rounding, not bit for bit).
 #include "common.cuh"
+#include "route_select.cuh"
 
 namespace moe {
 
 namespace {
 
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
+using small::warp_max;
+using small::warp_sum;
 __device__ __forceinline__ void bf16x8(const uint4& u, float (&v)[8]) {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -136,14 +128,7 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(const __gr
         for (int i = threadIdx.x; i < a.sem_n; i += blockDim.x) a.sem[i] = 0;
     for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
         const int t = i / E, e = i % E;
-        float pv[kSmallMaxParts];
-#pragma unroll
-        for (int part = 0; part < kSmallMaxParts; ++part)
-            pv[part] = part < P ? a.probs[((size_t)t * P + part) * E + e] : 0.f;
-        float v = 0.f;
-#pragma unroll
-        for (int part = 0; part < kSmallMaxParts; ++part)
-            if (part < P) v += pv[part];
+        const float v = small::sum_partials(a.probs, t, P, E, e);
         z[t][e] = v;
         if (writer) a.logits[i] = v;
     }
@@ -151,23 +136,12 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(const __gr
 
     float ex_z = 0.f, ex_h = 0.f, ex_g = 0.f;
     for (int t = warp; t < T; t += kFinWarps) {
-        float zz[2], key[2], ex[2];
-        unsigned valid = 0;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int e = lane + 32 * i;
-            zz[i] = e < E ? z[t][e] : -INFINITY;
-            if (e < E) valid |= 1u << i;
-        }
-        const float m = warp_max(fmaxf(zz[0], zz[1]));
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            ex[i] = ((valid >> i) & 1u) ? expf(zz[i] - m) : 0.f;
-            s += ex[i];
-        }
-        s = warp_sum(s);
-        const float inv_s = 1.f / s;
+        const small::TokenSoftmax ts =
+            small::token_softmax(lane < E ? z[t][lane] : 0.f, lane + 32 < E ? z[t][lane + 32] : 0.f, E, lane);
+        const float* zz = ts.zz;
+        const float* ex = ts.ex;
+        const unsigned valid = ts.valid;
+        const float m = ts.m, s = ts.s, inv_s = ts.inv_s;
         {   // router statistics of this token (z-loss, entropy, top-1/top-2 gap)
             float pz = 0.f, z1 = -INFINITY, z2 = -INFINITY;
 #pragma unroll
@@ -194,37 +168,11 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(const __gr
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int e = lane + 32 * i;
-            const float p = ex[i] * inv_s;
-            const float b = e < E ? bias_s[e] : 0.f;
-            if (e < E) psw[warp][e] += p;
-            key[i] = a.bias_mode == MOE_BIAS_NONE ? zz[i] : a.bias_mode == MOE_BIAS_LOGIT ? zz[i] + b : p + b;
+            if (e < E) psw[warp][e] += small::token_prob(ts, i);
         }
         // k rounds of a warp arg-max (the lowest index wins ties); the selected
         // logits and experts go to shared memory, lane j then finishes slot j
-        unsigned taken = 0;
-#pragma unroll 1
-        for (int j = 0; j < k; ++j) {
-            float bk = -INFINITY, bz = 0.f;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
-                if (ok && (key[i] > bk || be == 0x7fffffff)) { bk = key[i]; be = lane + 32 * i; bz = zz[i]; }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-                const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
-                if (better) { bk = ok_; be = oe; bz = oz; }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            if (lane == 0) {
-                zsel_s[warp][j] = bz;
-                esel_s[warp][j] = be;
-            }
-        }
+        small::token_topk(ts, bias_s, a.bias_mode, E, k, lane, zsel_s[warp], esel_s[warp]);
         __syncwarp();
         if (lane < k) {
             // gates: softmax over the k selected raw logits, summed in slot order
@@ -356,16 +304,8 @@ __global__ void __launch_bounds__(kFinWarps * 32) route_finish_kernel(const __gr
     }
     __syncthreads();
     for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-        const int t = i / k, j = i % k, e = sidx[i];
-        int rank = 0;
-        if (a.drop_slot) {   // earlier slots of every token, then this slot of earlier tokens
-            for (int q = 0; q < T * k; ++q) {
-                const int tq = q / k, jq = q % k;
-                rank += (sidx[q] == e) && (jq < j || (jq == j && tq < t));
-            }
-        } else {
-            for (int q = 0; q < t * k; ++q) rank += (sidx[q] == e);
-        }
+        const int t = i / k, e = sidx[i];
+        const int rank = small::pair_rank(sidx, i, T, k, a.drop_slot != 0);
         const int p = (a.capacity < 0 || rank < a.capacity) ? indptr_s[e] + rank : -1;
         spos[i] = p;
         if (writer) {
@@ -403,10 +343,15 @@ bool small_route_ok(const moe_problem& p) {
            p.E <= kSmallMaxE && p.E % 8 == 0 && p.d % 8 == 0;
 }
 
+int small_route_parts(int d) {
+    const int nchunk = d / 8;
+    const int P = (nchunk + 127) / 128;   // ~128 chunks (1 per lane of 4 warps) per block
+    return P < 1 ? 1 : (P > kSmallMaxParts ? kSmallMaxParts : P);
+}
+
 cudaError_t launch_route_small(const SmallRouteArgs& a, cudaStream_t st) {
     const int nchunk = a.d / 8;
-    int P = (nchunk + 127) / 128;   // ~128 chunks (1 per lane of 4 warps) per block
-    P = P < 1 ? 1 : (P > kSmallMaxParts ? kSmallMaxParts : P);
+    const int P = small_route_parts(a.d);
     cudaError_t e = launch_k(route_logits_kernel, dim3(a.T, P), dim3(kPartWarps * 32), 0, st, a, P);
     if (e != cudaSuccess) return e;
     g_pdl_after_first();

@@ -209,6 +209,11 @@ def test_padded_forward_equals_dense():
     ("bf16", 1024, 256, [300], 0, 10),                       # 16 k-blocks: ring wraps 4 times
     ("bf16", 128, 512, [5, 0, 0, 700, 3], 192, 257),         # shared width != routed width
     ("f32", 128, 256, [0, 70, 1, 129], 64, 50),
+    # groups wider than one band of M blocks (the GEMM runs a group's rows in
+    # bands of about 32 MB): GEMM 1/3 with K = 7168 (17 blocks a band) over 18
+    # blocks, GEMM 2 with K = 14336 (9 blocks a band) over 10 blocks
+    ("bf16", 7168, 256, [70, 2300], 0, 10),
+    ("bf16", 256, 14336, [1200, 3], 0, 10),
 ])
 def test_experts_stage(dtype, d, d_ff, counts, shared, T):
     E = len(counts)
@@ -311,6 +316,11 @@ SMALL = [
     dict(T=20, d=256, d_ff=256, E=64, k=2, cf=0.5, dtype="bf16", bias_mode=1, d_ff_shared=0),
     dict(T=8, d=512, d_ff=256, E=16, k=4, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=0),
     dict(T=3, d=128, d_ff=128, E=8, k=8, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    # T <= 8 on the small router: GEMM 1/3 derives the routing itself and reads x
+    dict(T=8, d=256, d_ff=256, E=8, k=2, cf=0.5, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=1, drop=1),
+    dict(T=7, d=256, d_ff=384, E=32, k=2, cf=0.75, dtype="bf16", bias_mode=1, d_ff_shared=0),
+    dict(T=6, d=128, d_ff=256, E=64, k=8, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    dict(T=4, d=192, d_ff=256, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     # routing variants: Switch full-softmax gates, GShard slot-priority drops
     dict(T=500, d=256, d_ff=256, E=8, k=1, cf=1.0, dtype="bf16", bias_mode=0, d_ff_shared=0, gate=1, drop=0),
     dict(T=700, d=128, d_ff=256, E=16, k=2, cf=0.7, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=0, drop=1),
