@@ -435,6 +435,12 @@ def main():
     rows = st.rows
     tflops = flops_per_step(cfg, rows) * world * args.steps / (job_ms / 1e3) / 1e12
 
+    # ---- per-stage breakdown (stage entry points, events between) ----
+    # (right after the timed steps, under the same flush-separated load: the
+    # end-to-end loop below keeps the GPU busy without gaps, and under the
+    # power cap the clock is lower after it)
+    stages = breakdown(moe, p, cfg, L, dev, stream, flush, iters=max(3, min(10, args.steps)))
+
     # ---- end to end through host buffers ----
     x_host = x.cpu().pin_memory()
     e2e_ms = e2e_pipelined(layer, x_host, dev, stream, args.steps, before_timed=barrier)
@@ -444,9 +450,6 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     e2e_value = tokens_total / (float(t.item()) / 1e3)
     nbytes = x.numel() * x.element_size()
-
-    # ---- per-stage breakdown (stage entry points, events between) ----
-    stages = breakdown(moe, p, cfg, L, dev, stream, flush, iters=max(3, min(10, args.steps)))
 
     peaks, peak_src = load_peaks()
     roofline = workload_roofline(cfg, args.workload, stages, st, peaks, peak_src)

@@ -73,25 +73,36 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const __grid_constan
 
     // 1. per expert row of chunk counts (expert-major order, chunk inner):
     //    exclusive prefix inside the row -> blockoff, row total -> start[e].
-    //    One warp per row, 32 consecutive entries per step (coalesced).
+    //    One warp per row, 32 consecutive entries per step (coalesced); the
+    //    loads of 8 steps are issued before their scans, so a row of a few
+    //    hundred chunks costs one or two memory round trips, not one a step.
     {
         const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
         const int len = a.kk * NB;   // (slot, chunk) entries of one expert
+        constexpr int U = 8;
         for (int e = warp; e < E; e += nw) {
             const int32_t* row = a.blockcnt + (size_t)e * len;
             int32_t* orow = a.blockoff + (size_t)e * len;
             int carry = 0;
-            for (int b0 = 0; b0 < len; b0 += 32) {
-                const int b = b0 + lane;
-                const int v = b < len ? row[b] : 0;
-                int incl = v;
+            for (int b0 = 0; b0 < len; b0 += 32 * U) {
+                int v[U];
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    int n_ = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += n_;
+                for (int u = 0; u < U; ++u) {
+                    const int b = b0 + 32 * u + lane;
+                    v[u] = b < len ? row[b] : 0;
                 }
-                if (b < len) orow[b] = carry + incl - v;
-                carry += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int b = b0 + 32 * u + lane;
+                    int incl = v[u];
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        int n_ = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += n_;
+                    }
+                    if (b < len) orow[b] = carry + incl - v[u];
+                    carry += __shfl_sync(0xffffffffu, incl, 31);
+                }
             }
             if (lane == 0) start[e] = carry;   // c_e (converted to a prefix below)
         }
@@ -136,21 +147,44 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const __grid_constan
         kept[e] = kp;
     }
 
-    // 4. P_e = mean router probability: one warp per expert, fixed order
+    // 4. P_e = mean router probability over the per-chunk sums [NB][E]: a
+    //    warp takes 32 consecutive experts (coalesced rows) and one of
+    //    `segs` contiguous ranges of chunks, summed in chunk order with 8
+    //    loads in flight; the ranges are then added in range order. Fixed
+    //    order throughout.
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __shared__ float psum_s[kScanThreads];
     if (a.blockpsum != nullptr) {
-        for (int ee = warp; ee < E; ee += kScanThreads / 32) {
+        const int groups = (E + 31) / 32;
+        const int segs = max(1, (kScanThreads / 32) / groups);
+        if (warp < groups * segs) {
+            const int g = warp % groups, sg = warp / groups;
+            const int ee = g * 32 + lane;
+            const int b_lo = (int)((long long)sg * NB / segs), b_hi = (int)((long long)(sg + 1) * NB / segs);
             float acc = 0.f;
-            for (int b = lane; b < NB; b += 32) acc += a.blockpsum[(size_t)b * E + ee];
+            if (ee < E) {
+                int b = b_lo;
+                for (; b + 8 <= b_hi; b += 8) {
+                    float v[8];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) {
-                float Pe = a.T > 0 ? acc / (float)a.T : 0.f;
-                float fe = a.T > 0 ? (float)(start[ee + 1] - start[ee]) / ((float)a.T * (float)a.k) : 0.f;
-                P[ee] = Pe;
-                f[ee] = fe;
-                fP[ee] = fe * Pe;
+                    for (int u = 0; u < 8; ++u) v[u] = a.blockpsum[(size_t)(b + u) * E + ee];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) acc += v[u];
+                }
+                for (; b < b_hi; ++b) acc += a.blockpsum[(size_t)b * E + ee];
+                psum_s[sg * E + ee] = acc;
             }
+        }
+        __syncthreads();
+        const int ee = threadIdx.x;
+        if (ee < E) {
+            float acc = 0.f;
+            for (int sg = 0; sg < segs; ++sg) acc += psum_s[sg * E + ee];
+            float Pe = a.T > 0 ? acc / (float)a.T : 0.f;
+            float fe = a.T > 0 ? (float)(start[ee + 1] - start[ee]) / ((float)a.T * (float)a.k) : 0.f;
+            P[ee] = Pe;
+            f[ee] = fe;
+            fP[ee] = fe * Pe;
         }
     }
     // router statistics: per-chunk sums of (z-loss, entropy, gap), one warp
@@ -158,7 +192,16 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const __grid_constan
     __shared__ float extra_s[3];
     if (a.blockextra != nullptr && warp < 3) {
         float acc = 0.f;
-        for (int b = lane; b < NB; b += 32) acc += a.blockextra[(size_t)b * 3 + warp];
+        for (int b0 = lane; b0 < NB; b0 += 32 * 4) {   // 4 loads in flight, summed in chunk order
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int b = b0 + 32 * u;
+                v[u] = b < NB ? a.blockextra[(size_t)b * 3 + warp] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc += v[u];
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (lane == 0) extra_s[warp] = a.T > 0 ? acc / (float)a.T : 0.f;
