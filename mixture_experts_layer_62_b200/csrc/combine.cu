@@ -2,11 +2,11 @@
 // "Week 2 Day 2: Mixture of Experts" §1.3, y = sum_{i in T} g_i f_i(x)),
 // plus the always-on shared expert (same page §4.1).
 //
-// One warp per token. Every lane owns 16-byte column vectors of the row and
-// accumulates in fp32: slot 0, 1, ..., k-1 (dropped slots skipped), then the
-// shared-expert row; the sum is rounded once on the store. Each output row is
-// written by exactly one warp, so no atomics are needed and the summation
-// order is fixed.
+// One warp per (token, slice of the row). Every lane owns 16-byte column
+// vectors of the slice and accumulates in fp32: slot 0, 1, ..., k-1 (dropped
+// slots skipped), then the shared-expert row; the sum is rounded once on the
+// store. Each output element is written by exactly one lane, so no atomics
+// are needed and the summation order is fixed.
 #include "common.cuh"
 
 namespace moe {
