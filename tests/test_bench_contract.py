@@ -1,0 +1,46 @@
+"""CPU checks of bench.py's arithmetic: the algorithmic FLOPs and bytes its
+throughput and roofline figures divide by, and the launch count it claims."""
+
+import types
+
+import bench
+from mixture_experts_layer_62_b200 import inputs
+
+
+def test_flops_of_the_prefill_workload():
+    # 2 T k 3 d d_ff for the experts + 2 T d E for the router
+    cfg = inputs.workload("mixtral_prefill")
+    want = 2 * 4096 * 2 * 3 * 4096 * 14336 + 2 * 4096 * 4096 * 8
+    assert bench.flops_per_step(cfg) == want
+    assert round(want / 1e12, 3) == 2.886
+    # GEMM 1/3 and GEMM 2 split the expert FLOPs 2 : 1
+    R = 4096 * 2
+    assert bench.up_flops(cfg, R) == 2 * R * 4096 * 2 * 14336
+    assert bench.down_flops(cfg, R) * 2 == bench.up_flops(cfg, R)
+    assert bench.up_flops(cfg, R) + bench.down_flops(cfg, R) + 2 * 4096 * 4096 * 8 == want
+
+
+def test_flops_with_the_shared_expert():
+    cfg = inputs.workload("deepseek_v3")
+    T, d, E, k, dff, dfs = 8192, 7168, 256, 8, 2048, 2048
+    want = 2 * T * k * 3 * d * dff + 2 * T * d * E + 2 * T * 3 * d * dfs
+    assert bench.flops_per_step(cfg) == want
+    assert round(want / 1e12, 2) == 6.52
+
+
+def test_decode_bytes_count_touched_experts_only():
+    cfg = inputs.workload("decode_t1")
+    st = types.SimpleNamespace(counts=[1, 0, 0, 1, 0, 0, 0, 0])
+    b = bench.decode_bytes(cfg, st)
+    # two experts' W1, W3, W2 in bf16, the router, one x row and one y row
+    assert b == 2 * 3 * 4096 * 14336 * 2 + 4096 * 8 * 2 + 2 * 4096 * 2
+    assert round(b / 1e6, 1) == 704.7
+
+
+def test_launch_counts():
+    assert bench.launches_per_forward(inputs.workload("decode_t1")) == 5
+    assert bench.launches_per_forward(inputs.workload("mixtral_prefill")) == 8
+    assert bench.launches_per_forward(inputs.workload("mixtral_prefill"), pad_rows=128) == 9
+    # the shared expert rules out the small-batch router
+    assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), d_ff_shared=2048)) == 8
+    assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), T=0)) == 1
