@@ -559,6 +559,40 @@ def test_forward_full_size(name, n_random, pad):
         assert s.capacity == 5120 and s.dropped > 0
 
 
+def test_decode_experts_touched_fraction():
+    # the decode sweep's routing, with a fresh router matrix per trial: the
+    # mean fraction of experts the GPU router touches matches
+    # 1 - (C(E-1, k) / C(E, k))^T within 3 sigma of the trials' mean
+    E, k, d, trials = 8, 2, 4096, 1000
+    g = torch.Generator(device=DEV)
+    g.manual_seed(1234)
+    for T in inputs.DECODE_TOKENS:
+        p = moe.problem(T, d, 14336, E, k, 0.0, "bf16", 0, 0)
+        ws = moe.alloc_workspace(p, DEV)
+        st = moe.alloc_stats(E, DEV)
+        x = torch.randn((T, d), generator=g, device=DEV).to(torch.bfloat16)
+        idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+        gate = torch.empty((T, k), dtype=torch.float32, device=DEV)
+        picks = torch.empty((trials, T, k), dtype=torch.int32, device=DEV)
+        for i in range(trials):
+            W_r = (torch.randn((d, E), generator=g, device=DEV) / math.sqrt(d)).to(torch.bfloat16)
+            moe.route(p, x, W_r, idx, gate, st, ws)
+            picks[i].copy_(idx)
+        torch.cuda.synchronize()
+        pk = picks.cpu().numpy().reshape(trials, T * k)
+        assert ((pk >= 0) & (pk < E)).all()
+        fr = np.array([len(set(row.tolist())) / E for row in pk])
+        expect = O.fraction_experts_touched(E, k, T)
+        # standard deviation of one trial's fraction under uniform k-subsets:
+        # N = experts touched, P(e missed) = q^T, P(e and e' missed) = r^T
+        q = math.comb(E - 1, k) / math.comb(E, k)
+        r = math.comb(E - 2, k) / math.comb(E, k)
+        pt = 1 - q ** T
+        var_n = E * pt * (1 - pt) + E * (E - 1) * (1 - 2 * q ** T + r ** T - pt * pt)
+        sigma = math.sqrt(max(var_n, 0.0)) / E / math.sqrt(trials)
+        assert abs(fr.mean() - expect) <= 3 * sigma + 1e-12, (T, fr.mean(), expect, sigma)
+
+
 @pytest.mark.parametrize("T", inputs.DECODE_TOKENS)
 def test_forward_decode(T):
     cfg = inputs.workload(f"decode_t{T}")
