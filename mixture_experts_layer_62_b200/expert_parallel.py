@@ -1,0 +1,114 @@
+"""Expert parallelism over W ranks: dispatch and combine as all-to-alls.
+
+Rank r owns the experts [r E/W, (r + 1) E/W) ("Lecture 21 · LLM:
+Mixture-of-Experts" §4, expert parallelism: every GPU holds E/W experts,
+tokens travel to their experts' GPU and back). Each rank routes and permutes
+its own tokens (``moe_route`` and ``moe_permute`` of the library, or the
+fused pass up to the permutation). The permutation is expert-major, so the
+rows bound for one owner form one contiguous slice of Xp, already in the
+owner's expert order; no packing step is needed. Then:
+
+1. ``plan``: an all-to-all of the per-expert row counts (E numbers a rank)
+   tells every owner how many rows of each of its experts each source sends.
+2. ``dispatch``: an all-to-all of the rows; the owner's buffer holds one
+   block per source, each block grouped by the owner's experts.
+3. ``run_local_experts``: the owner runs its experts over each source's block
+   (one grouped GEMM call per block, with the block's own offsets), so the
+   outputs stay in the order the rows came in.
+4. ``combine_back``: an all-to-all returns every block to its source, where
+   it lands exactly where the single-GPU pass puts its expert outputs (O, in
+   the permuted order), and the library's combine finishes the layer.
+
+Capacity is applied by each source on its own tokens (per-device capacity,
+as for the data-parallel replicas). This is the unfused form, with the
+collectives issued by torch.distributed (NCCL on GPUs, gloo on CPU tensors);
+the same functions serve both. Overlapping the transfers with the grouped
+GEMM tile by tile, over peer memory, is not built here.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Callable, List
+
+import torch
+import torch.distributed as dist
+
+
+def expert_range(E: int, world: int, rank: int):
+    """Experts [lo, hi) owned by `rank` (E must divide evenly)."""
+    if E % world:
+        raise ValueError(f"{E} experts do not split evenly over {world} ranks")
+    n = E // world
+    return rank * n, (rank + 1) * n
+
+
+@dataclass
+class EPPlan:
+    world: int
+    E: int
+    E_local: int
+    send_rows: List[int]        # rows this rank sends to each owner
+    recv_rows: List[int]        # rows this rank receives from each source
+    recv_counts: torch.Tensor   # [world, E_local] int64: rows per (source, local expert)
+
+    @property
+    def rows_out(self) -> int:
+        return sum(self.send_rows)
+
+    @property
+    def rows_in(self) -> int:
+        return sum(self.recv_rows)
+
+    def block_offsets(self, src: int) -> torch.Tensor:
+        """Row offsets [E_local + 1] of source `src`'s block, per local expert."""
+        c = self.recv_counts[src]
+        return torch.cat([torch.zeros(1, dtype=torch.int64), torch.cumsum(c, 0)])
+
+
+def plan(indptr: torch.Tensor, E: int, group=None) -> EPPlan:
+    """Exchange per-expert row counts. `indptr` [E + 1] is this rank's
+    permutation offsets (kept rows, expert-major)."""
+    world = dist.get_world_size(group)
+    lo, hi = expert_range(E, world, 0)
+    E_local = hi - lo
+    ip = indptr.to(torch.int64)
+    counts = ip[1:] - ip[:-1]                           # [E], owner-major
+    recv = torch.empty_like(counts)
+    dist.all_to_all_single(recv, counts, group=group)   # [world * E_local], source-major
+    send_rows = counts.view(world, E_local).sum(1).cpu().tolist()
+    recv_counts = recv.view(world, E_local).cpu()
+    recv_rows = recv_counts.sum(1).tolist()
+    return EPPlan(world, E, E_local, [int(v) for v in send_rows], [int(v) for v in recv_rows], recv_counts)
+
+
+def dispatch(xp: torch.Tensor, p: EPPlan, group=None) -> torch.Tensor:
+    """Send the permuted rows to their owners; returns the rows received,
+    one block per source in rank order."""
+    out = xp.new_empty((p.rows_in,) + tuple(xp.shape[1:]))
+    dist.all_to_all_single(out, xp[:p.rows_out].contiguous(), output_split_sizes=p.recv_rows,
+                           input_split_sizes=p.send_rows, group=group)
+    return out
+
+
+def run_local_experts(rows: torch.Tensor, p: EPPlan,
+                      experts_fn: Callable[[torch.Tensor, torch.Tensor], torch.Tensor], d_out: int) -> torch.Tensor:
+    """Apply the local experts block by block: experts_fn(block_rows,
+    offsets) returns the block's expert outputs [n, d_out], rows in the
+    block's order, offsets [E_local + 1] int64 on the host."""
+    out = rows.new_empty((p.rows_in, d_out))
+    at = 0
+    for src in range(p.world):
+        n = p.recv_rows[src]
+        if n:
+            out[at:at + n] = experts_fn(rows[at:at + n], p.block_offsets(src))
+        at += n
+    return out
+
+
+def combine_back(expert_out: torch.Tensor, p: EPPlan, o: torch.Tensor, group=None) -> torch.Tensor:
+    """Return every block to its source; fills o[:rows_out] (this rank's
+    expert outputs in its own permuted order) and returns o."""
+    dist.all_to_all_single(o[:p.rows_out], expert_out.contiguous(), output_split_sizes=p.send_rows,
+                           input_split_sizes=p.recv_rows, group=group)
+    return o

@@ -1,0 +1,107 @@
+"""Expert parallelism on CPU: world sizes 2 and 4 over gloo.
+
+Every rank routes and permutes its own token shard (with the oracle, on the
+CPU), then plan / dispatch / run_local_experts / combine_back move the rows
+to the ranks that own their experts and back. The local experts use only
+the owner's slice of the weights. Each rank's output must equal the oracle's
+single-process forward of its tokens with all the experts, drops included.
+"""
+
+import math
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from mixture_experts_layer_62_b200 import expert_parallel as ep
+from mixture_experts_layer_62_b200 import parallel
+from oracle import moe_oracle as O
+
+T, d, d_ff, E, k, CF = 157, 16, 24, 8, 2, 1.0
+
+
+def _layer():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((T, d))
+    W_r = rng.standard_normal((d, E)) / math.sqrt(d)
+    W1 = rng.standard_normal((E, d_ff, d)) / math.sqrt(d)
+    W3 = rng.standard_normal((E, d_ff, d)) / math.sqrt(d)
+    W2 = rng.standard_normal((E, d, d_ff)) / math.sqrt(d_ff)
+    return x, W_r, W1, W3, W2
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        x, W_r, W1, W3, W2 = _layer()
+        lo, hi = parallel.shard_range(T, world, rank)
+        xr = x[lo:hi]
+        e_lo, e_hi = ep.expert_range(E, world, rank)
+        W1l, W3l, W2l = W1[e_lo:e_hi], W3[e_lo:e_hi], W2[e_lo:e_hi]   # this rank's experts only
+
+        # routing and permutation of the rank's own tokens (per-rank capacity)
+        r = O.route(O.router_logits(xr, W_r), k)
+        perm = O.permute(r.idx, E, O.capacity(CF, hi - lo, k, E))
+        xp = torch.from_numpy(xr[perm.row_token])
+        p = ep.plan(torch.from_numpy(perm.indptr), E)
+        assert p.rows_out == int(perm.indptr[-1])
+
+        rows = ep.dispatch(xp, p)
+
+        def experts_fn(block, offsets):
+            b = block.numpy()
+            out = np.empty((b.shape[0], d))
+            for e in range(p.E_local):
+                s, t = int(offsets[e]), int(offsets[e + 1])
+                if t > s:
+                    out[s:t] = O.swiglu_expert(b[s:t], W1l[e], W3l[e], W2l[e])
+            return torch.from_numpy(out)
+
+        expert_out = ep.run_local_experts(rows, p, experts_fn, d)
+        o = torch.zeros((p.rows_out, d), dtype=torch.float64)
+        ep.combine_back(expert_out, p, o)
+        y = O.unpermute_combine(o.numpy(), perm.pos, r.gate)
+
+        ref = O.moe_forward(xr, W_r, W1, W3, W2, k, CF)
+        err = float(np.abs(y - ref.y).max() / max(1e-30, np.abs(ref.y).max()))
+        q.put((rank, err, int(perm.kept.sum()), int(ref.stats.dropped), p.rows_in))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_expert_parallel_matches_single_process(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    res.sort()
+    assert all(err < 1e-12 for _, err, _, _, _ in res), res
+    # some pairs were dropped by the per-rank capacity, and every kept row
+    # was computed by exactly one owner
+    assert sum(dr for _, _, _, dr, _ in res) > 0
+    assert sum(kept for _, _, kept, _, _ in res) == sum(n for _, _, _, _, n in res)
+
+
+def test_expert_range_requires_an_even_split():
+    assert ep.expert_range(8, 4, 3) == (6, 8)
+    with pytest.raises(ValueError):
+        ep.expert_range(8, 3, 0)
