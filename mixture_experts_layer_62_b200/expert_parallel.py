@@ -112,3 +112,29 @@ def combine_back(expert_out: torch.Tensor, p: EPPlan, o: torch.Tensor, group=Non
     dist.all_to_all_single(o[:p.rows_out], expert_out.contiguous(), output_split_sizes=p.send_rows,
                            input_split_sizes=p.recv_rows, group=group)
     return o
+
+
+def library_experts_fn(W1_local: torch.Tensor, W3_local: torch.Tensor, W2_local: torch.Tensor):
+    """An experts_fn for run_local_experts that runs the owner's experts with
+    the library's grouped GEMMs (moe_experts, GEMM 1/3 + SwiGLU then GEMM 2)
+    on the device of the weights: W1_local, W3_local [E_local, d_ff, d],
+    W2_local [E_local, d, d_ff]. A block of n rows is one call with a
+    problem of n tokens, one slot each, over the E_local experts; the
+    workspace of each block size is allocated once and kept."""
+    import mixture_experts_layer_62_b200 as moe
+
+    E_local, d_ff, d = W1_local.shape
+    workspaces = {}
+
+    def fn(block: torch.Tensor, offsets: torch.Tensor) -> torch.Tensor:
+        n = block.shape[0]
+        p = moe.problem(n, d, d_ff, E_local, 1, 0.0, block.dtype)
+        ws = workspaces.get(n)
+        if ws is None:
+            ws = workspaces[n] = moe.alloc_workspace(p, block.device)
+        indptr = offsets.to(device=block.device, dtype=torch.int32)
+        out = torch.empty((n, d), dtype=block.dtype, device=block.device)
+        moe.experts(p, block.contiguous(), indptr, W1_local, W3_local, W2_local, out, ws)
+        return out
+
+    return fn

@@ -105,3 +105,42 @@ def test_expert_range_requires_an_even_split():
     assert ep.expert_range(8, 4, 3) == (6, 8)
     with pytest.raises(ValueError):
         ep.expert_range(8, 3, 0)
+
+
+def test_library_experts_fn_wiring(monkeypatch):
+    # the library's expert stage stands in as a CPU fake that checks what it
+    # is handed (a problem of n tokens, one slot each, over the local
+    # experts; int32 offsets) and computes with the oracle
+    import mixture_experts_layer_62_b200 as moe
+    rng = np.random.default_rng(5)
+    E_l, dd, dff = 3, 8, 12
+    W1 = torch.from_numpy(rng.standard_normal((E_l, dff, dd)))
+    W3 = torch.from_numpy(rng.standard_normal((E_l, dff, dd)))
+    W2 = torch.from_numpy(rng.standard_normal((E_l, dd, dff)))
+    calls = []
+
+    def fake_experts(p, xp, indptr, w1, w3, w2, o, ws, **kw):
+        assert (p.T, p.d, p.d_ff, p.E, p.k) == (xp.shape[0], dd, dff, E_l, 1)
+        assert indptr.dtype == torch.int32 and indptr.shape == (E_l + 1,) and int(indptr[-1]) == xp.shape[0]
+        ip = indptr.tolist()
+        for e in range(E_l):
+            if ip[e + 1] > ip[e]:
+                o[ip[e]:ip[e + 1]] = torch.from_numpy(O.swiglu_expert(
+                    xp[ip[e]:ip[e + 1]].numpy(), w1[e].numpy(), w3[e].numpy(), w2[e].numpy()))
+        calls.append(xp.shape[0])
+
+    monkeypatch.setattr(moe, "experts", fake_experts)
+    monkeypatch.setattr(moe, "alloc_workspace", lambda p, device=None: torch.empty(1, dtype=torch.uint8))
+    monkeypatch.setattr(moe, "problem", lambda T, d, d_ff, E, k, cf, dtype: types_ns(T, d, d_ff, E, k))
+    fn = ep.library_experts_fn(W1, W3, W2)
+    block = torch.from_numpy(rng.standard_normal((7, dd)))
+    offsets = torch.tensor([0, 2, 2, 7], dtype=torch.int64)
+    got = fn(block, offsets).numpy()
+    want = np.concatenate([O.swiglu_expert(block[0:2].numpy(), W1[0].numpy(), W3[0].numpy(), W2[0].numpy()),
+                           O.swiglu_expert(block[2:7].numpy(), W1[2].numpy(), W3[2].numpy(), W2[2].numpy())])
+    assert np.allclose(got, want, rtol=0, atol=1e-12) and calls == [7]
+
+
+def types_ns(T, d, d_ff, E, k):
+    import types
+    return types.SimpleNamespace(T=T, d=d, d_ff=d_ff, E=E, k=k)
