@@ -847,10 +847,10 @@ int moe_experts(const moe_problem* p, const void* xp, const int32_t* indptr, con
                        sp.part13, sp.part2, sp.sem13, sp.sem2);
 }
 
-// Shared prologue of the expert-stage entry points: checks, status reset and
-// the tile schedules built from indptr.
+// Shared prologue of the expert-stage entry points: the workspace check and
+// the status word and tile schedule buffers.
 static int expert_stage_setup(const moe_problem* p, void* stats, void* workspace, size_t workspace_bytes,
-                              cudaStream_t st, int32_t** status, int32_t** tiles13, int32_t** tiles2) {
+                              int32_t** status, int32_t** tiles13, int32_t** tiles2) {
     const Layout L = make_layout(*p);
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return MOE_ERR_WORKSPACE;
@@ -875,7 +875,7 @@ int moe_expert_up(const moe_problem* p, const void* xp, const int32_t* indptr, c
             if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int32_t *status, *tiles13, *tiles2;
-    rc = expert_stage_setup(p, stats, workspace, workspace_bytes, st, &status, &tiles13, &tiles2);
+    rc = expert_stage_setup(p, stats, workspace, workspace_bytes, &status, &tiles13, &tiles2);
     if (rc != MOE_OK) return rc;
     if (p->T == 0) return MOE_OK;
     CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
@@ -903,7 +903,7 @@ int moe_expert_down(const moe_problem* p, const void* h, const int32_t* indptr, 
             if (!aligned16(q)) return MOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int32_t *status, *tiles13, *tiles2;
-    rc = expert_stage_setup(p, stats, workspace, workspace_bytes, st, &status, &tiles13, &tiles2);
+    rc = expert_stage_setup(p, stats, workspace, workspace_bytes, &status, &tiles13, &tiles2);
     if (rc != MOE_OK) return rc;
     if (p->T == 0) return MOE_OK;
     CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
