@@ -169,35 +169,43 @@ def blas_threads():
 
 def oracle_sample(cfg, L, n_tokens, seed=0, needed_experts=None):
     """Time the CPU oracle: routing of all tokens plus the expert math of a
-    seeded sample of n_tokens tokens. The weights of the experts the sample
-    can touch are copied to host numpy before the clock starts."""
+    seeded sample of n_tokens tokens. Every array the oracle reads is in
+    float64 on the host before the clock starts (the weights of the experts
+    the sample can touch, x, W_r), so the timed region holds the oracle's
+    own arithmetic only, not dtype conversions. Returns (tokens, seconds,
+    seconds of the routing-only pass over all tokens)."""
     from oracle import moe_oracle as O
-    x = L["x"].float().cpu().numpy()
-    W_r = L["W_r"].float().cpu().numpy()
-    bias = None if L["bias"] is None else L["bias"].float().cpu().numpy()
+    x = L["x"].double().cpu().numpy()
+    W_r = L["W_r"].double().cpu().numpy()
+    bias = None if L["bias"] is None else L["bias"].double().cpu().numpy()
     rng = np.random.default_rng(seed)
     tokens = np.sort(rng.choice(cfg["T"], size=min(n_tokens, cfg["T"]), replace=False))
     experts = range(cfg["E"]) if needed_experts is None else sorted(set(needed_experts(tokens)))
+
     class _Host(dict):
         # an expert the oracle's own routing picks beyond the prefetched set
         # (a near-tie) is copied on demand
         def __init__(self, W):
-            super().__init__({e: W[e].float().cpu().numpy() for e in experts})
+            super().__init__({e: W[e].double().cpu().numpy() for e in experts})
             self.W = W
 
         def __missing__(self, e):
-            v = self[e] = self.W[e].float().cpu().numpy()
+            v = self[e] = self.W[e].double().cpu().numpy()
             return v
 
     W1, W3, W2 = _Host(L["W1"]), _Host(L["W3"]), _Host(L["W2"])
     sh = {}
     if cfg["d_ff_shared"]:
-        sh = {n: L[n].float().cpu().numpy() for n in ("Ws1", "Ws3", "Ws2")}
+        sh = {n: L[n].double().cpu().numpy() for n in ("Ws1", "Ws3", "Ws2")}
+    args = (x, W_r, W1, W3, W2, cfg["k"], cfg["cf"], bias, cfg["bias_mode"], sh.get("Ws1"), sh.get("Ws3"),
+            sh.get("Ws2"))
     t0 = time.perf_counter()
-    O.moe_forward(x, W_r, W1, W3, W2, cfg["k"], cfg["cf"], bias, cfg["bias_mode"],
-                  sh.get("Ws1"), sh.get("Ws3"), sh.get("Ws2"), tokens=tokens)
+    O.moe_forward(*args, tokens=np.zeros(0, dtype=np.int64))     # routing, permutation, statistics only
+    t_route = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.moe_forward(*args, tokens=tokens)
     dt = time.perf_counter() - t0
-    return len(tokens), dt
+    return len(tokens), dt, t_route
 
 
 def touched_experts(st):
@@ -255,20 +263,25 @@ def run_reference(args, cfg, rank):
     n = args.ref_sample
     for i in range(args.warmup):
         oracle_sample(cfg, L, n, seed=1000 + i)
-    total_tok, total_t = 0, 0.0
+    total_tok, total_t, total_route = 0, 0.0, 0.0
     for i in range(args.steps):
-        nt, dt = oracle_sample(cfg, L, n, seed=i)
+        nt, dt, tr = oracle_sample(cfg, L, n, seed=i)
         total_tok += nt
         total_t += dt
+        total_route += tr
     value = total_tok / total_t
     cores = blas_threads()
-    sample = f"per step: routing of all {cfg['T']} tokens + expert math of {n} seeded random tokens"
+    sample = (f"per step: routing of all {cfg['T']} tokens + expert math of {n} seeded random tokens; "
+              f"routing alone {1e3 * total_route / args.steps:.0f} ms, expert math "
+              f"{1e3 * (total_t - total_route) / total_tok:.1f} ms per token")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(cfg, args),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+                         "route_ms": 1e3 * total_route / args.steps,
+                         "expert_ms_per_token": 1e3 * (total_t - total_route) / total_tok},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -314,6 +327,104 @@ def launches_per_forward(cfg, pad_rows=0):
     return 8 + (1 if pad_rows else 0)
 
 
+def time_steps(step, steps, warmup, dev, stream, flush, barrier, local_rank):
+    """Total device milliseconds of `steps` calls of step(): `warmup` untimed
+    calls, then each timed call bracketed by CUDA events on the launching
+    stream, with an L2 flush before it (outside the events); barrier and
+    synchronize on both sides. SM clocks are sampled during the timed calls."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    sampler = ClockSampler(gpu_index_for(local_rank))
+    sampler.start()
+    torch.cuda.synchronize(dev)
+    barrier()
+    evs = []
+    for _ in range(steps):
+        flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    return sum(a.elapsed_time(b) for a, b in evs), clocks
+
+
+def pass_roofline(cfg, st, ms_per_step, peaks):
+    """Roofline of the whole forward: the slower of its FLOPs (executed rows)
+    at the bf16 peak and its compulsory bytes (every touched expert's
+    weights, the router, x and y) at the HBM peak, over the measured step."""
+    fl = flops_per_step(cfg, st.rows)
+    by = decode_bytes(cfg, st)
+    t_c = fl / (peaks["bf16_tflops"] * 1e12)
+    t_m = by / (peaks["hbm_gbs"] * 1e9)
+    t = ms_per_step / 1e3
+    return {"bound": "tensor" if t_c >= t_m else "hbm", "flops": fl, "bytes": by,
+            "roofline_ms": 1e3 * max(t_c, t_m), "frac": max(t_c, t_m) / t,
+            "tflops": fl / t / 1e12, "hbm_gbs": by / t / 1e9}
+
+
+# The other configurations of the benchmark, measured in the same process
+# after the headline workload (one GPU): the decode sweep's batch sizes that
+# carry the HBM target, the DeepSeek-V3-shaped layer and the skewed layer
+# with capacity drops.
+EXTRA_WORKLOADS = ("decode_t1", "decode_t2", "decode_t4", "decode_t8", "skewed_capacity", "deepseek_v3")
+
+
+def measure_extra(name, args, moe, dev, stream, flush, peaks, peak_src, weight_cache):
+    """One more workload, timed like the headline (graph replay, L2 flushed
+    between steps, CUDA events); returns its summary."""
+    cfg = inputs.workload(name)
+    key = (cfg["d"], cfg["d_ff"], cfg["E"], cfg["dtype"], cfg["d_ff_shared"])
+    if key in weight_cache:
+        # same shapes and seed: the same weights, x and W_r drawn for this T
+        L = dict(weight_cache[key])
+        x, W_r, bias = inputs.make_routing_inputs(cfg, seed=0)
+        L.update(x=x.to(dev), W_r=W_r.to(dev), bias=None if bias is None else bias.to(dev))
+    else:
+        weight_cache.clear()
+        torch.cuda.empty_cache()
+        L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=dev)
+        L = {k_: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k_, v in L.items()}
+        weight_cache[key] = {n: L[n] for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2")}
+    p = moe.problem(cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg["cf"], cfg["dtype"], cfg["bias_mode"],
+                    cfg["d_ff_shared"])
+    layer = moe.MoELayer(p, L["W_r"], L["W1"], L["W3"], L["W2"], bias=L["bias"], Ws1=L["Ws1"], Ws3=L["Ws3"],
+                         Ws2=L["Ws2"])
+    x = L["x"]
+    for _ in range(args.warmup):
+        layer(x)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer(x)
+    torch.cuda.synchronize(dev)
+    total_ms, clocks = time_steps(graph.replay, args.steps, args.warmup, dev, stream, flush, lambda: None, 0)
+    st = layer.read_stats()
+    if st.status != moe.MOE_OK:
+        raise SystemExit(f"{name}: device status {st.status}: {moe.error_string(st.status)}")
+    ms = total_ms / args.steps
+    stages = breakdown(moe, p, cfg, L, dev, stream, flush, iters=max(3, min(10, args.steps)))
+    out = {"ms_per_step": ms, "tokens_per_s": cfg["T"] / (ms / 1e3), "T": cfg["T"],
+           "roofline": workload_roofline(cfg, name, stages, st, peaks, peak_src),
+           "pass_roofline": pass_roofline(cfg, st, ms, peaks), "stages_ms": stages, "clocks": clocks,
+           "routing": {"rows": st.rows, "dropped": st.dropped, "capacity": st.capacity, "l_aux": st.l_aux,
+                       "max_over_mean": st.max_over_mean, "experts_touched": touched_experts(st),
+                       "counts": st.counts if cfg["E"] <= 16 else None,
+                       "kept": st.kept if cfg["E"] <= 16 else None},
+           "gpu_launches": launches_per_forward(cfg) * args.steps}
+    if cfg["T"] <= 64:
+        out["forward_hbm_gbs"] = decode_bytes(cfg, st) / (ms / 1e3) / 1e9
+        out["forward_hbm_frac"] = out["forward_hbm_gbs"] / peaks["hbm_gbs"]
+    del graph, layer
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -322,8 +433,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral_prefill")
     ap.add_argument("--cpu-sample", type=int, default=1024, help="tokens of the timed CPU-oracle sample")
-    ap.add_argument("--ref-sample", type=int, default=16, help="tokens per step of the reference arm")
+    ap.add_argument("--ref-sample", type=int, default=64, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="measure the headline workload only (by default one GPU also measures " +
+                         ", ".join(EXTRA_WORKLOADS) + ")")
     ap.add_argument("--no-graph", action="store_true", help="launch the forward eagerly in the timed loop")
     ap.add_argument("--train", action="store_true",
                     help="time a training step (forward + backward) instead of the forward")
@@ -399,28 +513,7 @@ def main():
             dist.barrier()
 
     # ---- device-timed steps ----
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    barrier()
-    sampler = ClockSampler(gpu_index_for(local_rank))
-    sampler.start()
-    torch.cuda.synchronize(dev)
-    barrier()
-    evs = []
-    for _ in range(args.steps):
-        flush()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        step()
-        e1.record(stream)
-        evs.append((e0, e1))
-    torch.cuda.synchronize(dev)
-    barrier()
-    clocks = sampler.stop()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
+    total_ms, clocks = time_steps(step, args.steps, args.warmup, dev, stream, flush, barrier, local_rank)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -482,12 +575,21 @@ def main():
                                 "max_over_mean": gst.max_over_mean}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gidx = moe.workspace_view(layer.workspace, p, "idx").cpu().numpy()
-        n, dt = oracle_sample(cfg, L, args.cpu_sample, needed_experts=lambda toks: gidx[toks].reshape(-1).tolist())
+        n, dt, tr = oracle_sample(cfg, L, args.cpu_sample,
+                                  needed_experts=lambda toks: gidx[toks].reshape(-1).tolist())
         line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"routing of all {cfg['T']} tokens + expert math of {n} seeded random "
-                                          f"tokens ({dt:.1f} s)"}
+                                          f"tokens ({dt:.1f} s)",
+                                "route_ms": 1e3 * tr, "expert_ms_per_token": 1e3 * (dt - tr) / n}
+    line["pass_roofline"] = pass_roofline(cfg, st, ms_per_step, peaks)
     if not args.no_graph:
         del graph
+    if world == 1 and not args.no_extra and args.workload == "mixtral_prefill" and not args.pad_rows:
+        cache = {(cfg["d"], cfg["d_ff"], cfg["E"], cfg["dtype"], cfg["d_ff_shared"]):
+                 {n: L[n] for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2")}}
+        del layer
+        line["workloads"] = {name: measure_extra(name, args, moe, dev, stream, flush, peaks, peak_src, cache)
+                             for name in EXTRA_WORKLOADS}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

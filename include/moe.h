@@ -256,11 +256,15 @@ int moe_combine(const moe_problem* p, const void* o, const int32_t* pos, const f
  * expert counts and their scan) lives in a fixed 1 MiB array inside the
  * library, which every GPU that loads the library holds until the process
  * exits. Arguments, outputs and results are those of moe_permute.
- *  - Limit: E * ceil(T / 32) <= 131072 (e.g. T <= 16384 at E = 256);
- *    larger problems return MOE_ERR_UNSUPPORTED before anything is launched.
+ *  - Limit: E * kk * ceil(T / 32) <= 131072, with kk = k under
+ *    MOE_DROP_SLOT and 1 otherwise (e.g. T <= 16384 at E = 256 with the
+ *    token drop order); larger problems return MOE_ERR_UNSUPPORTED before
+ *    anything is launched. The problem checks and error codes are otherwise
+ *    those of moe_permute.
  *  - The first call on a device looks up the array's device address on that
  *    device (the device must be current); make that first call before any
- *    stream capture.
+ *    stream capture. If the lookup fails the call returns MOE_ERR_CUDA and
+ *    the next call on that device tries again.
  *  - All calls share the one array and it keeps the last call's contents
  *    (every entry a call reads is written earlier in the same call). Calls
  *    that overlap on the GPU (different streams, or different host threads,

@@ -152,14 +152,6 @@ int device_sm_count() {
     return cache[dev];
 }
 
-}  // namespace moe
-
-using namespace moe;
-
-namespace {
-
-bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
-
 int check_problem(const moe_problem* p) {
     if (p == nullptr) return MOE_ERR_INVALID_ARG;
     if (p->T < 0 || p->d <= 0 || p->d_ff <= 0 || p->E < 1 || p->E > MOE_MAX_E || p->k < 1 ||
@@ -193,6 +185,14 @@ int capacity_of(const moe_problem* p) {
     if (c > 2147483647.0) return -1;
     return (int)c;
 }
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 #define CK(expr)                                   \
     do {                                           \

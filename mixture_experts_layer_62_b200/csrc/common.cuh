@@ -280,4 +280,9 @@ bool make_tmap_f32_store(void* map, const float* base, int rows, int cols);
 
 int device_sm_count();
 
+// The problem checks every entry point shares (MOE_OK or an error code), and
+// the capacity C = ceil(cf T k / E) (-1 = no limit).
+int check_problem(const moe_problem* p);
+int capacity_of(const moe_problem* p);
+
 }  // namespace moe

@@ -14,7 +14,6 @@
 // only a host-side stand-in, not a device address, so the device address is
 // looked up with cudaGetSymbolAddress once per device, with that device
 // current, on the first call made on that device.
-#include <cmath>
 #include <mutex>
 
 #include "common.cuh"
@@ -28,57 +27,42 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) int32_t g_permute_scratch[2 * kMaxEntries];
 
-struct DeviceScratch {
-    std::once_flag once;
-    int32_t* ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-};
-DeviceScratch g_scratch[kMaxDevices];
+// Device address of the scratch array, per device. A successful lookup is
+// kept for the life of the process; a failed one is not, so a later call on
+// that device tries again instead of failing for the rest of the process.
+std::mutex g_scratch_mutex;
+int32_t* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once
-// per device); nullptr on failure.
+// Device address of the scratch array on the current device; nullptr if the
+// lookup failed.
 int32_t* scratch_on_current_device() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    DeviceScratch& s = g_scratch[dev];
-    std::call_once(s.once, [&s] {
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_ptr[dev] == nullptr) {
         void* ptr = nullptr;
-        s.err = cudaGetSymbolAddress(&ptr, g_permute_scratch);
-        if (s.err == cudaSuccess) s.ptr = static_cast<int32_t*>(ptr);
-    });
-    return s.err == cudaSuccess ? s.ptr : nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_permute_scratch) != cudaSuccess) {
+            cudaGetLastError();   // the failure is reported by the return code, not left pending
+            return nullptr;
+        }
+        g_scratch_ptr[dev] = static_cast<int32_t*>(ptr);
+    }
+    return g_scratch_ptr[dev];
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
-
-// The problem checks of the other entry points, restated for this one.
-int check(const moe_problem* p) {
-    if (p == nullptr) return MOE_ERR_INVALID_ARG;
-    if (p->T < 0 || p->d <= 0 || p->d_ff <= 0 || p->E < 1 || p->E > MOE_MAX_E || p->k < 1 || p->k > p->E ||
-        p->k > MOE_MAX_K || p->d_ff_shared < 0)
-        return MOE_ERR_INVALID_ARG;
-    if (p->dtype != MOE_DTYPE_F32 && p->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
-    if (p->bias_mode < MOE_BIAS_NONE || p->bias_mode > MOE_BIAS_PROB) return MOE_ERR_INVALID_ARG;
-    if (!(p->capacity_factor == p->capacity_factor)) return MOE_ERR_INVALID_ARG;
-    if ((long long)p->T * p->k >= (1LL << 30)) return MOE_ERR_UNSUPPORTED;
-    if (p->dtype == MOE_DTYPE_BF16 ? (p->d % 8 != 0) : (p->d % 4 != 0)) return MOE_ERR_UNSUPPORTED;
-    return MOE_OK;
-}
 
 }  // namespace
 
 extern "C" int moe_permute_noalloc(const moe_problem* p, const void* x, const int32_t* idx, int32_t* pos,
                                    int32_t* indptr, int32_t* row_token, void* xp, void* stats, void* stream) {
-    int rc = check(p);
+    int rc = moe::check_problem(p);   // the checks of moe_permute
     if (rc != MOE_OK) return rc;
     if (!idx || !pos || !indptr || !stats) return MOE_ERR_INVALID_ARG;
     if (xp && (!x || !aligned16(x) || !aligned16(xp))) return MOE_ERR_INVALID_ARG;
     if (!aligned16(stats)) return MOE_ERR_INVALID_ARG;
     const long long nb = (p->T + moe::kChunk - 1) / moe::kChunk;
-    if (p->gate_mode != MOE_GATE_SELECTED && p->gate_mode != MOE_GATE_FULL) return MOE_ERR_INVALID_ARG;
-    if (p->drop_order != MOE_DROP_TOKEN && p->drop_order != MOE_DROP_SLOT) return MOE_ERR_INVALID_ARG;
     const int kk = moe::count_slots(*p);
-    if (kk > 1 && p->E * p->k > moe::kMaxSlotCounts) return MOE_ERR_UNSUPPORTED;
     if ((long long)p->E * kk * nb > kMaxEntries) return MOE_ERR_UNSUPPORTED;   // beyond the static scratch
     if (p->pad_rows != 0) return MOE_ERR_UNSUPPORTED;                         // dense rows only
 
@@ -87,12 +71,7 @@ extern "C" int moe_permute_noalloc(const moe_problem* p, const void* x, const in
     int32_t* blockcnt = scratch;                 // written in full by the histogram
     int32_t* blockoff = scratch + kMaxEntries;   // written in full by the scan
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    double cf = (double)p->capacity_factor;
-    int C = -1;
-    if (cf > 0.0) {
-        double c = std::ceil(cf * (double)p->T * (double)p->k / (double)p->E);
-        C = c > 2147483647.0 ? -1 : (int)c;
-    }
+    const int C = moe::capacity_of(p);
     if (p->T == 0) {
         if (moe::launch_zero_stats(stats, p->E, C, st) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaMemsetAsync(indptr, 0, sizeof(int32_t) * (size_t)(p->E + 1), st) != cudaSuccess) return MOE_ERR_CUDA;

@@ -114,27 +114,46 @@ def combine_back(expert_out: torch.Tensor, p: EPPlan, o: torch.Tensor, group=Non
     return o
 
 
-def library_experts_fn(W1_local: torch.Tensor, W3_local: torch.Tensor, W2_local: torch.Tensor):
+def library_experts_fn(W1_local: torch.Tensor, W3_local: torch.Tensor, W2_local: torch.Tensor,
+                       max_rows: int | None = None):
     """An experts_fn for run_local_experts that runs the owner's experts with
     the library's grouped GEMMs (moe_experts, GEMM 1/3 + SwiGLU then GEMM 2)
     on the device of the weights: W1_local, W3_local [E_local, d_ff, d],
     W2_local [E_local, d, d_ff]. A block of n rows is one call with a
-    problem of n tokens, one slot each, over the E_local experts; the
-    workspace of each block size is allocated once and kept."""
+    problem of n tokens, one slot each, over the E_local experts.
+
+    The function holds one workspace. With ``max_rows`` (the largest block a
+    source can send, e.g. its tokens times k) it is sized once, up front;
+    without, it is replaced only when a block needs more than it holds, so
+    the memory held is that of the largest block seen, however the block
+    sizes vary from step to step. The calls share one statistics block,
+    ``fn.state["stats"]``, whose status word records a device-side error
+    (a bounded wait of a tensor-core kernel that gave up)."""
     import mixture_experts_layer_62_b200 as moe
 
     E_local, d_ff, d = W1_local.shape
-    workspaces = {}
+    dev = W1_local.device
+    state = {"ws": None, "stats": moe.alloc_stats(E_local, dev)}
+
+    def ensure(n, dtype):
+        need = moe.workspace_size(moe.problem(n, d, d_ff, E_local, 1, 0.0, dtype))
+        ws = state["ws"]
+        if ws is None or ws.numel() < need:
+            state["ws"] = None                      # release the old buffer before the new one
+            state["ws"] = torch.empty(need, dtype=torch.uint8, device=dev)
+        return state["ws"]
+
+    if max_rows is not None:
+        ensure(int(max_rows), W1_local.dtype)
 
     def fn(block: torch.Tensor, offsets: torch.Tensor) -> torch.Tensor:
         n = block.shape[0]
         p = moe.problem(n, d, d_ff, E_local, 1, 0.0, block.dtype)
-        ws = workspaces.get(n)
-        if ws is None:
-            ws = workspaces[n] = moe.alloc_workspace(p, block.device)
+        ws = ensure(n, block.dtype)
         indptr = offsets.to(device=block.device, dtype=torch.int32)
         out = torch.empty((n, d), dtype=block.dtype, device=block.device)
-        moe.experts(p, block.contiguous(), indptr, W1_local, W3_local, W2_local, out, ws)
+        moe.experts(p, block.contiguous(), indptr, W1_local, W3_local, W2_local, out, ws, stats=state["stats"])
         return out
 
+    fn.state = state
     return fn

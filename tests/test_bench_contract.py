@@ -44,3 +44,22 @@ def test_launch_counts():
     # the shared expert rules out the small-batch router
     assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), d_ff_shared=2048)) == 8
     assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), T=0)) == 1
+
+
+def test_pass_roofline_of_the_deepseek_shaped_layer():
+    # 6.52 TFLOP at the bf16 peak against 22.88 GB (all 256 experts touched,
+    # the shared expert, the router, x and y) at the HBM peak: compute-bound,
+    # 3.91 ms at this machine's measured peaks
+    cfg = inputs.workload("deepseek_v3")
+    st = types.SimpleNamespace(rows=8192 * 8, counts=[1] * 256)
+    peaks = {"bf16_tflops": 1667.2, "hbm_gbs": 6545.3}
+    r = bench.pass_roofline(cfg, st, 7.82, peaks)
+    assert round(r["flops"] / 1e12, 2) == 6.52
+    assert round(r["bytes"] / 1e9, 2) == 22.88
+    assert r["bound"] == "tensor" and round(r["roofline_ms"], 2) == 3.91
+    assert abs(r["frac"] - 3.91 / 7.82) < 1e-3
+
+
+def test_every_other_config_is_measured_by_default():
+    names = set(bench.EXTRA_WORKLOADS)
+    assert {"decode_t1", "decode_t2", "decode_t4", "decode_t8", "deepseek_v3", "skewed_capacity"} <= names

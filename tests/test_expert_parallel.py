@@ -107,21 +107,21 @@ def test_expert_range_requires_an_even_split():
         ep.expert_range(8, 3, 0)
 
 
-def test_library_experts_fn_wiring(monkeypatch):
-    # the library's expert stage stands in as a CPU fake that checks what it
-    # is handed (a problem of n tokens, one slot each, over the local
-    # experts; int32 offsets) and computes with the oracle
+def _fake_library(monkeypatch, E_l, dd, dff, calls, allocs):
+    """The library's expert stage as a CPU fake that checks what it is
+    handed (a problem of n tokens, one slot each, over the local experts;
+    int32 offsets; a workspace at least moe_workspace_size) and computes
+    with the oracle; workspace allocations are recorded."""
     import mixture_experts_layer_62_b200 as moe
-    rng = np.random.default_rng(5)
-    E_l, dd, dff = 3, 8, 12
-    W1 = torch.from_numpy(rng.standard_normal((E_l, dff, dd)))
-    W3 = torch.from_numpy(rng.standard_normal((E_l, dff, dd)))
-    W2 = torch.from_numpy(rng.standard_normal((E_l, dd, dff)))
-    calls = []
+
+    def ws_size(p):
+        return 1000 + 10 * p.T
 
     def fake_experts(p, xp, indptr, w1, w3, w2, o, ws, **kw):
         assert (p.T, p.d, p.d_ff, p.E, p.k) == (xp.shape[0], dd, dff, E_l, 1)
         assert indptr.dtype == torch.int32 and indptr.shape == (E_l + 1,) and int(indptr[-1]) == xp.shape[0]
+        assert ws.numel() >= ws_size(p)
+        assert kw.get("stats") is not None
         ip = indptr.tolist()
         for e in range(E_l):
             if ip[e + 1] > ip[e]:
@@ -129,9 +129,33 @@ def test_library_experts_fn_wiring(monkeypatch):
                     xp[ip[e]:ip[e + 1]].numpy(), w1[e].numpy(), w3[e].numpy(), w2[e].numpy()))
         calls.append(xp.shape[0])
 
+    real_empty = torch.empty
+
+    def counting_empty(*shape, dtype=None, device=None, **kw):
+        t = real_empty(*shape, dtype=dtype, **kw)
+        if dtype == torch.uint8:
+            allocs.append(t.numel())
+        return t
+
     monkeypatch.setattr(moe, "experts", fake_experts)
-    monkeypatch.setattr(moe, "alloc_workspace", lambda p, device=None: torch.empty(1, dtype=torch.uint8))
+    monkeypatch.setattr(moe, "workspace_size", ws_size)
+    monkeypatch.setattr(moe, "alloc_stats", lambda E, device=None: real_empty(64, dtype=torch.uint8))
     monkeypatch.setattr(moe, "problem", lambda T, d, d_ff, E, k, cf, dtype: types_ns(T, d, d_ff, E, k))
+    monkeypatch.setattr(ep.torch, "empty", counting_empty)
+
+
+def _weights(rng, E_l, dd, dff):
+    return (torch.from_numpy(rng.standard_normal((E_l, dff, dd))),
+            torch.from_numpy(rng.standard_normal((E_l, dff, dd))),
+            torch.from_numpy(rng.standard_normal((E_l, dd, dff))))
+
+
+def test_library_experts_fn_wiring(monkeypatch):
+    rng = np.random.default_rng(5)
+    E_l, dd, dff = 3, 8, 12
+    W1, W3, W2 = _weights(rng, E_l, dd, dff)
+    calls, allocs = [], []
+    _fake_library(monkeypatch, E_l, dd, dff, calls, allocs)
     fn = ep.library_experts_fn(W1, W3, W2)
     block = torch.from_numpy(rng.standard_normal((7, dd)))
     offsets = torch.tensor([0, 2, 2, 7], dtype=torch.int64)
@@ -139,6 +163,29 @@ def test_library_experts_fn_wiring(monkeypatch):
     want = np.concatenate([O.swiglu_expert(block[0:2].numpy(), W1[0].numpy(), W3[0].numpy(), W2[0].numpy()),
                            O.swiglu_expert(block[2:7].numpy(), W1[2].numpy(), W3[2].numpy(), W2[2].numpy())])
     assert np.allclose(got, want, rtol=0, atol=1e-12) and calls == [7]
+
+
+@pytest.mark.parametrize("max_rows", [None, 40])
+def test_library_experts_fn_keeps_one_workspace(monkeypatch, max_rows):
+    # block sizes change from step to step: one workspace is held, replaced
+    # only when a block needs more (or sized once from max_rows)
+    rng = np.random.default_rng(6)
+    E_l, dd, dff = 2, 8, 8
+    W1, W3, W2 = _weights(rng, E_l, dd, dff)
+    calls, allocs = [], []
+    _fake_library(monkeypatch, E_l, dd, dff, calls, allocs)
+    fn = ep.library_experts_fn(W1, W3, W2, max_rows=max_rows)
+    sizes = [7, 3, 12, 5, 12, 9, 30, 1, 30, 2]
+    for n in sizes:
+        block = torch.from_numpy(rng.standard_normal((n, dd)))
+        offsets = torch.tensor([0, n // 2, n], dtype=torch.int64)
+        fn(block, offsets)
+    assert calls == sizes
+    if max_rows is None:
+        assert allocs == [1000 + 10 * n for n in (7, 12, 30)]      # grows, never per size
+    else:
+        assert allocs == [1000 + 10 * max_rows]                   # once, up front
+    assert fn.state["ws"].numel() == allocs[-1]
 
 
 def types_ns(T, d, d_ff, E, k):
