@@ -322,9 +322,11 @@ def launches_per_forward(cfg, pad_rows=0):
     if small and not pad_rows:
         # partial router logits, routing finisher, grouped GEMM 1/3, grouped GEMM 2, combine
         return 5
-    # transpose W_r, logits (SIMT or tensor-core), select, scan, permute+gather,
+    # router: one fused kernel (logits and selection) up to 64 experts, else
+    # transpose W_r, tensor-core logits, select; then scan, permute+gather,
     # (padding fill,) grouped GEMM 1/3, grouped GEMM 2, combine
-    return 8 + (1 if pad_rows else 0)
+    wide = cfg["dtype"] == "bf16" and cfg["E"] >= 64 and cfg["E"] % 32 == 0
+    return (8 if wide else 6) + (1 if pad_rows else 0)
 
 
 def time_steps(step, steps, warmup, dev, stream, flush, barrier, local_rank):

@@ -320,6 +320,19 @@ const char* moe_error_string(int code);
  * on the current device, or -1 on error. */
 int moe_device_sm_count(void);
 
+/* Failure detection (no step of the notes): every mbarrier wait inside the
+ * tensor-core kernels gives up after `ns` nanoseconds of wall-clock time,
+ * records MOE_ERR_TIMEOUT in the status word of the call's statistics block,
+ * lets the copies and MMAs it already started land (a separate, fixed 2 s
+ * drain limit), frees its tensor memory and returns, so a stalled pipeline
+ * surfaces as an error the host reads instead of a hung GPU. ns <= 0 restores
+ * the default of 2 s. The setting is process-wide and applies to launches
+ * made after the call; the previous value is returned. A limit far below a
+ * kernel's normal run time makes its calls fail with MOE_ERR_TIMEOUT (their
+ * outputs are then unspecified); the next call with a normal limit is
+ * unaffected. */
+long long moe_set_wait_limit(long long ns);
+
 #ifdef __cplusplus
 }
 #endif

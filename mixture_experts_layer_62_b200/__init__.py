@@ -77,6 +77,8 @@ def _load():
     lib.moe_workspace_layout.restype = ctypes.c_int
     lib.moe_error_string.argtypes = [ctypes.c_int]
     lib.moe_error_string.restype = ctypes.c_char_p
+    lib.moe_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.moe_set_wait_limit.restype = ctypes.c_longlong
     lib.moe_device_sm_count.argtypes = []
     lib.moe_device_sm_count.restype = ctypes.c_int
     lib.moe_permuted_rows.argtypes = [P]
@@ -122,6 +124,13 @@ def __getattr__(name):
     if name == "lib":
         return _lib()
     raise AttributeError(name)
+
+
+def set_wait_limit(ns: int) -> int:
+    """Wall-clock limit (nanoseconds) of the device-side bounded waits of the
+    tensor-core kernels, process-wide; ns <= 0 restores the 2 s default.
+    Returns the previous limit (moe_set_wait_limit)."""
+    return int(_lib().moe_set_wait_limit(int(ns)))
 
 
 def error_string(code: int) -> str:

@@ -2,7 +2,9 @@
 // launch sequence of the forward pass (route -> scan -> permute/gather ->
 // grouped GEMM 1/3 + SwiGLU -> grouped GEMM 2 -> combine). Every launch is
 // asynchronous on the caller's stream; the host never waits on the device.
+#include <atomic>
 #include <cmath>
+#include <cstdlib>
 
 #include "common.cuh"
 
@@ -137,8 +139,22 @@ bool split_allowed(const moe_problem& p) {
            (long long)p.T * p.k <= kSplitMaxRows;
 }
 
+bool use_pair_tiles(const moe_problem& p) {
+    static const bool enabled = [] {
+        const char* v = std::getenv("MOE_CTA_PAIR");
+        return !(v != nullptr && v[0] == '0');
+    }();
+    return enabled && p.dtype == MOE_DTYPE_BF16 && p.T > 0 && p.pad_rows == 0 && !p.train && !split_allowed(p) &&
+           (long long)p.T * p.k >= 512LL * p.E;
+}
+
 thread_local bool g_pdl = false;
 thread_local bool g_pdl_pass = false;
+
+constexpr long long kDefaultWaitLimitNs = 2000000000LL;
+std::atomic<long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+
+long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 int device_sm_count() {
     static int cache[64] = {};
@@ -201,13 +217,22 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
 
 char* wsp(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
 
+// The general-path router: tensor cores for wide bf16 routers (a real GEMM),
+// otherwise one fused kernel (logits and selection) where it applies.
+bool router_on_tensor_cores(const moe_problem* p) {
+    return p->dtype == MOE_DTYPE_BF16 && p->E >= 64 && p->E % 32 == 0;
+}
+bool router_fused(const moe_problem* p) {
+    return !router_on_tensor_cores(p) && route_fused_ok(p->dtype, p->d, p->E);
+}
+
 // Router: logits (fp32) for all tokens into `logits`.
 int run_logits(const moe_problem* p, const void* x, const void* W_r, float* logits, const Layout& L,
                void* ws, int32_t* status, cudaStream_t st, bool reset_status = false) {
     void* wrt = wsp(ws, L.wrt);
     CK(launch_transpose_wr(p->dtype, W_r, wrt, p->d, p->E, st, reset_status ? status : nullptr));
     g_pdl_after_first();
-    if (p->dtype == MOE_DTYPE_BF16 && p->E >= 64 && p->E % 32 == 0) {
+    if (router_on_tensor_cores(p)) {
         // wide routers (e.g. 256 experts) are a real GEMM: tensor cores, fp32 out
         TcArgs a = {};
         a.mode = TC_F32OUT;
@@ -240,6 +265,7 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
     if (p->dtype == MOE_DTYPE_BF16) {
         TcArgs a = {};
         a.mode = TC_SWIGLU;
+        a.pair = use_pair_tiles(*p) ? 1 : 0;
         a.b_before_wait = sched_early ? 1 : 0;
         a.indptr = indptr; a.tiles = tiles13;
         a.E = p->E; a.has_shared = has_shared; a.T = p->T;
@@ -284,6 +310,7 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
     if (p->dtype == MOE_DTYPE_BF16) {
         TcArgs b = {};
         b.mode = TC_PLAIN;
+        b.pair = use_pair_tiles(*p) ? 1 : 0;
         b.b_before_wait = 1;   // the schedule comes from the router, two or more launches back
         b.indptr = indptr; b.tiles = tiles2;
         b.E = p->E; b.has_shared = has_shared; b.T = p->T;
@@ -330,7 +357,7 @@ int run_experts(const moe_problem* p, const void* xp, const int32_t* indptr, con
 
 void schedule_sizes(const moe_problem* p, int& tile_m, int& nt13, int& nt2, int& nt13s, int& nt2s) {
     if (p->dtype == MOE_DTYPE_BF16) {
-        tile_m = kTcTileM;
+        tile_m = use_pair_tiles(*p) ? kTcPairTileM : kTcTileM;
         int c13 = tc_out_cols_per_tile(TC_SWIGLU), c2 = tc_out_cols_per_tile(TC_PLAIN);
         nt13 = ceil_div(p->d_ff, c13);
         nt2 = ceil_div(p->d, c2);
@@ -393,6 +420,10 @@ int moe_workspace_layout(const moe_problem* p, moe_workspace_layout_t* out) {
 }
 
 int moe_device_sm_count(void) { return device_sm_count(); }
+
+long long moe_set_wait_limit(long long ns) {
+    return g_wait_limit_ns.exchange(ns > 0 ? ns : kDefaultWaitLimitNs);
+}
 
 // ---- backward ----------------------------------------------------------------
 
@@ -661,12 +692,18 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
         }
         CK(launch_route_small(sr, st));
     } else {
-    rc = run_logits(p, x, W_r, logits, L, workspace, status, st, /*reset_status=*/true);
-    if (rc != MOE_OK) return rc;
     float* blockextra = reinterpret_cast<float*>(wsp(workspace, L.blockextra));
     const int kk = count_slots(*p);
-    CK(launch_select(logits, bias, p->bias_mode, p->gate_mode, kk, p->T, p->E, p->k, idx, gate, blockcnt,
-                     blockpsum, blockextra, st));
+    if (router_fused(p)) {
+        CK(launch_route_fused(p->dtype, x, W_r, bias, p->bias_mode, p->gate_mode, kk, p->T, p->d, p->E, p->k,
+                              logits, idx, gate, blockcnt, blockpsum, blockextra, status, st));
+        g_pdl_after_first();
+    } else {
+        rc = run_logits(p, x, W_r, logits, L, workspace, status, st, /*reset_status=*/true);
+        if (rc != MOE_OK) return rc;
+        CK(launch_select(logits, bias, p->bias_mode, p->gate_mode, kk, p->T, p->E, p->k, idx, gate, blockcnt,
+                         blockpsum, blockextra, st));
+    }
     ScanArgs sa = {};
     sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C; sa.kk = kk;
     sa.blockcnt = blockcnt; sa.blockoff = blockoff; sa.blockpsum = blockpsum; sa.blockextra = blockextra;
@@ -725,14 +762,19 @@ int moe_route(const moe_problem* p, const void* x, const void* W_r, const float*
     int32_t* status = static_cast<int32_t*>(stats);
     CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
     float* lg = logits ? logits : reinterpret_cast<float*>(wsp(workspace, L.logits));
-    rc = run_logits(p, x, W_r, lg, L, workspace, status, st);
-    if (rc != MOE_OK) return rc;
     int32_t* blockcnt = reinterpret_cast<int32_t*>(wsp(workspace, L.blockcnt));
     float* blockpsum = reinterpret_cast<float*>(wsp(workspace, L.blockpsum));
     float* blockextra = reinterpret_cast<float*>(wsp(workspace, L.blockextra));
     const int kk = count_slots(*p);
-    CK(launch_select(lg, bias, p->bias_mode, p->gate_mode, kk, p->T, p->E, p->k, idx, gate, blockcnt, blockpsum,
-                     blockextra, st));
+    if (router_fused(p)) {
+        CK(launch_route_fused(p->dtype, x, W_r, bias, p->bias_mode, p->gate_mode, kk, p->T, p->d, p->E, p->k, lg,
+                              idx, gate, blockcnt, blockpsum, blockextra, nullptr, st));
+    } else {
+        rc = run_logits(p, x, W_r, lg, L, workspace, status, st);
+        if (rc != MOE_OK) return rc;
+        CK(launch_select(lg, bias, p->bias_mode, p->gate_mode, kk, p->T, p->E, p->k, idx, gate, blockcnt,
+                         blockpsum, blockextra, st));
+    }
     ScanArgs sa = {};
     sa.T = p->T; sa.k = p->k; sa.E = p->E; sa.capacity = C; sa.kk = kk;
     sa.blockcnt = blockcnt; sa.blockoff = reinterpret_cast<int32_t*>(wsp(workspace, L.blockoff));

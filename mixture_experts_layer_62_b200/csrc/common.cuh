@@ -121,6 +121,14 @@ cudaError_t launch_logits_simt(int dtype, const void* x, const void* wrt, float*
 // kk = k under the slot-priority drop order and kk = 1 otherwise.
 constexpr int kMaxSlotCounts = 4096;   // E * k limit of the slot-priority order
 inline int count_slots(const moe_problem& p) { return p.drop_order == MOE_DROP_SLOT ? p.k : 1; }
+// Logits and selection in one kernel (E <= 64, d % 8 == 0): the outputs of
+// launch_logits_simt followed by launch_select, from x and W_r [d, E] as
+// given; resets *status (if not null) to MOE_OK.
+bool route_fused_ok(int dtype, int d, int E);
+cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const float* bias, int bias_mode,
+                               int gate_mode, int kk, int T, int d, int E, int k, float* logits, int32_t* idx,
+                               float* gate, int32_t* blockcnt, float* blockpsum, float* blockextra, int32_t* status,
+                               cudaStream_t st);
 cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int gate_mode, int kk, int T,
                           int E, int k, int32_t* idx, float* gate, int32_t* blockcnt, float* blockpsum,
                           float* blockextra, cudaStream_t st);
@@ -209,6 +217,11 @@ cudaError_t launch_simt_gemm(bool swiglu, const GroupedArgs& a, cudaStream_t st)
 
 // bf16 grouped GEMM on tcgen05 tensor cores (sm_100a). Tile 128 x 256.
 constexpr int kTcTileM = 128;
+constexpr int kTcPairTileM = 256;   // rows of a CTA-pair tile
+// CTA-pair tiles for the prefill-sized grouped GEMMs of p (bf16, no split-K,
+// not the training forward, unpadded, at least 512 rows per expert on
+// average); the environment variable MOE_CTA_PAIR=0 turns them off.
+bool use_pair_tiles(const moe_problem& p);
 int tc_out_cols_per_tile(int mode);   // 128 for SWIGLU, 256 otherwise
 enum TcMode { TC_SWIGLU = 0, TC_PLAIN = 1, TC_F32OUT = 2 };
 struct TcArgs {
@@ -235,6 +248,9 @@ struct TcArgs {
     // back, so the weight loads of the first stages may start before the
     // dependency wait
     int b_before_wait;
+    // 1: CTA pairs with 256-row tiles (the schedule counts 256-row M blocks);
+    // SWIGLU or PLAIN, no split-K, no pre-activation output
+    int pair;
 };
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
 // Backward grouped GEMMs (tcgen05): see gemm_bwd_sm100.cu.
@@ -283,6 +299,13 @@ int device_sm_count();
 // The problem checks every entry point shares (MOE_OK or an error code), and
 // the capacity C = ceil(cf T k / E) (-1 = no limit).
 int check_problem(const moe_problem* p);
+// Wall-clock limit of every bounded mbarrier wait in the tensor-core kernels
+// (nanoseconds; moe_set_wait_limit sets it, 2 s by default), and the limit of
+// the drain that lets in-flight copies and MMAs land after a wait gave up
+// (fixed, long: a drain cut short would let a CTA exit with a copy still
+// landing in its shared memory).
+long long wait_limit_ns();
+constexpr long long kDrainLimitNs = 2000000000LL;
 int capacity_of(const moe_problem* p);
 
 }  // namespace moe

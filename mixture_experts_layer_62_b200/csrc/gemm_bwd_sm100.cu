@@ -63,7 +63,8 @@ struct BParams {
     float* out0;              // BW_DW2: dW2 [E][d][d_ff]; BW_DW13: dW1 [E][d_ff][d]
     float* out1;              // BW_DW13: dW3 [E][d_ff][d]
     int32_t* status;
-    long long timeout_ns;
+    long long timeout_ns;      // limit of every wait of the work itself
+    long long drain_ns;        // limit of the drain after a wait gave up
 };
 
 struct BTile {
@@ -125,10 +126,11 @@ __device__ __forceinline__ bool wait_b(uint64_t* bar, uint32_t parity, Ctl* ctl,
         }
     }
 }
+// drain after a wait gave up: its own long limit
 __device__ __forceinline__ void wait_d(uint64_t* bar, uint32_t parity, const BParams& p) {
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > static_cast<uint64_t>(p.timeout_ns)) {
+        if (global_timer_ns() - t0 > static_cast<uint64_t>(p.drain_ns)) {
             atomicExch(p.status, MOE_ERR_TIMEOUT);
             return;
         }
@@ -496,7 +498,8 @@ cudaError_t launch_bwd_gemm(const BwdGemmArgs& a, cudaStream_t st) {
     bp.out0 = a.out0;
     bp.out1 = a.out1;
     bp.status = a.status;
-    bp.timeout_ns = 2000000000LL;
+    bp.timeout_ns = wait_limit_ns();
+    bp.drain_ns = kDrainLimitNs;
     switch (a.mode) {
         case BW_DH: return launch_bwd_mode<BW_DH>(maps, bp, st);
         case BW_DX: return launch_bwd_mode<BW_DX>(maps, bp, st);

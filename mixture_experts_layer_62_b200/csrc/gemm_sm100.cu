@@ -69,7 +69,8 @@ struct KParams {
     int N[2], K[2];
     void* out[2];
     int32_t* status;
-    long long timeout_ns;
+    long long timeout_ns;      // limit of every wait of the work itself
+    long long drain_ns;        // limit of the drain after a wait gave up
     float* partial;            // split-K partial rows, or null
     long long partial_stride;  // elements between splits
     int partial_ld;            // elements per partial row
@@ -91,7 +92,8 @@ __device__ __forceinline__ int total_tiles(const KParams& p, int cols_per_tile) 
     return p.tiles[p.E + p.has_shared];
 }
 
-__device__ __forceinline__ Tile decode_tile(const KParams& p, int tile) {
+template <int TM>
+__device__ __forceinline__ Tile decode_tile_m(const KParams& p, int tile) {
     Tile t;
     if (p.indptr == nullptr) {
         t.kind = 0; t.g = 0; t.rows = p.static_rows; t.row0 = 0;
@@ -107,7 +109,7 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, int tile) {
         t.row0 = t.kind ? 0 : p.indptr[lo];
         tile -= p.tiles[lo];
     }
-    const int mt = (t.rows + BM - 1) / BM;
+    const int mt = (t.rows + TM - 1) / TM;
     // bands of band_m M blocks, each over all N blocks, M fastest inside a band
     int h = mt, m0 = 0;
     const int bm = p.band_m[t.kind];
@@ -123,6 +125,7 @@ __device__ __forceinline__ Tile decode_tile(const KParams& p, int tile) {
     t.num_kb = (p.K[t.kind] + BK - 1) / BK;
     return t;
 }
+__device__ __forceinline__ Tile decode_tile(const KParams& p, int tile) { return decode_tile_m<BM>(p, tile); }
 
 struct SharedCtl {
     uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
@@ -145,11 +148,12 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Sha
         }
     }
 }
-// Drain wait used on the abort path: ignores the abort flag, still bounded.
+// Drain wait used on the abort path: ignores the abort flag and has a limit
+// of its own, long, so that a short wait limit never cuts a drain short.
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, const KParams& p) {
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > static_cast<uint64_t>(p.timeout_ns)) {
+        if (global_timer_ns() - t0 > static_cast<uint64_t>(p.drain_ns)) {
             atomicExch(p.status, MOE_ERR_TIMEOUT);
             return;
         }
@@ -562,6 +566,309 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
     }
 }
 
+// ---- CTA-pair kernel (cta_group::2, M = 256) ---------------------------------
+//
+// The same grouped GEMM for groups large enough to fill 256-row tiles. The
+// grid is clusters of two CTAs on neighbouring SMs; a cluster takes one
+// 256 x 256 accumulator tile at a time: rank r loads the A rows [128 r,
+// 128 r + 128) of the tile and one 128-row half of the B tile (SWIGLU: the
+// W1 rows in rank 0 and the W3 rows of the same output columns in rank 1;
+// PLAIN: rows [128 r, 128 r + 128) of the 256), and the leader (rank 0)
+// issues M = 256 MMAs that read both CTAs' shared memory and write each
+// CTA's accumulator rows into that CTA's tensor memory, [gate | up] or the
+// 256 output columns, exactly as in the single-CTA kernel, so the epilogue
+// is the same. Per SM, a K step moves a third less data through shared
+// memory than the single-CTA tile of the same FLOPs (the B tile is read once
+// for both SMs), which is what lets the tensor pipe run without waiting on
+// shared-memory fill; 32 KB stages leave room for six of them.
+// Protocol: the leader's full barrier of a stage counts both CTAs' bytes
+// (each CTA's loads complete on it; only the leader arms it); MMA completion
+// is committed to both CTAs' empty and accumulator-full barriers (one
+// multicast commit); each CTA's four epilogue warps arrive on the leader's
+// accumulator-empty barrier. Waits are bounded as in the single-CTA kernel;
+// a wait that gives up also raises the other CTA's abort flag. No TMA
+// multicast: every CTA loads its own tiles.
+constexpr int PBM = 256;                               // rows of a pair tile
+constexpr int P_STAGES = 6;
+constexpr int P_STAGE_BYTES = A_BYTES + B_HALF_BYTES;  // 32 KB per CTA
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+struct PairCtl {
+    uint64_t full[P_STAGES], empty[P_STAGES], tfull[2], tempty[2], drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairCtl* ctl, uint32_t peer_abort,
+                                          const KParams& p) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) return false;
+        if (global_timer_ns() - t0 > static_cast<uint64_t>(p.timeout_ns)) {
+            *reinterpret_cast<volatile int*>(&ctl->abort_flag) = 1;
+            st_shared_remote_u32(peer_abort, 1u);
+            atomicExch(p.status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Epilogue of one accumulator tile for this thread's row (shared by nothing
+// else: the single-CTA kernel keeps its own, with the split-K and training
+// variants).
+template <int MODE>
+__device__ __forceinline__ void pair_store_row(const KParams& p, const Tile& t, uint32_t tb, bool valid,
+                                               size_t orow) {
+    const int N = p.N[t.kind];
+    if (MODE == TC_SWIGLU) {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+            uint32_t gv[32], uv[32];
+            tmem_ld32(tb + c, gv);
+            tmem_ld32(tb + 128 + c, uv);
+            const int col = t.n_blk * 128 + c;
+            if (valid && col < N) {
+                uint32_t packed[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
+                    const float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
+                    packed[i] = pack_bf16(silu(g0) * u0, silu(g1) * u1);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            }
+        }
+    } else {
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(tb + c, v);
+            const int col = t.n_blk * 256 + c;
+            if (valid && col < N) {
+                uint32_t packed[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    packed[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            }
+        }
+    }
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+             const __grid_constant__ CUtensorMap tmB00, const __grid_constant__ CUtensorMap tmB01,
+             const __grid_constant__ CUtensorMap tmB10, const __grid_constant__ CUtensorMap tmB11,
+             const KParams p) {
+    static_assert(MODE == TC_SWIGLU || MODE == TC_PLAIN, "pair tiles: SWIGLU or PLAIN");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PairCtl* ctl = reinterpret_cast<PairCtl*>(smem + P_STAGES * P_STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const uint32_t peer_abort = mapa_shared(smem_u32(&ctl->abort_flag), rank ^ 1u);
+    const int cluster = static_cast<int>(blockIdx.x >> 1), nclusters = static_cast<int>(gridDim.x >> 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(&ctl->full[s], 1);    // the leader's arming arrive (+ both CTAs' bytes)
+            mbar_init(&ctl->empty[s], 1);   // one multicast MMA commit
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&ctl->tfull[a], 1);   // one multicast MMA commit
+            mbar_init(&ctl->tempty[a], 8);  // four epilogue warps of each CTA (used in the leader)
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort_flag = 0;
+        fence_mbar_init();
+        prefetch_map(&tmA0); prefetch_map(&tmA1);
+        prefetch_map(&tmB00); prefetch_map(&tmB01);
+        prefetch_map(&tmB10); prefetch_map(&tmB11);
+    }
+    if (warp == 1) {
+        // one warp of each CTA, the same warp in both, allocates the pair's tensor memory
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&ctl->tmem_base)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();   // both CTAs' barriers initialised and tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+    const bool early = p.b_before_wait != 0;
+    if (!early) {
+        pdl_wait();
+        pdl_launch();
+    }
+    const int units = p.tiles[p.E + p.has_shared];
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs) ----------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t armed_mask = 0, armed_ph = 0;   // leader: stages whose full barrier it armed
+            bool aborted = false;
+            int pre = 0;
+            const CUtensorMap* mbh[2] = {MODE == TC_SWIGLU && rank ? &tmB01 : &tmB00,
+                                         MODE == TC_SWIGLU && rank ? &tmB11 : &tmB10};
+            auto b_row = [&](const Tile& t) {
+                const int eoff = t.kind ? 0 : t.g * p.b_rows[0];
+                return MODE == TC_SWIGLU ? eoff + t.n_blk * 128 : eoff + t.n_blk * 256 + static_cast<int>(rank) * 128;
+            };
+            auto full_of = [&](int st) { return mapa_shared(smem_u32(&ctl->full[st]), 0u); };
+            if (early) {
+                if (cluster < units) {
+                    const Tile t = decode_tile_m<PBM>(p, cluster);
+                    const int brow = b_row(t);
+                    for (int kb = 0; kb < t.num_kb && pre < P_STAGES; ++kb, ++pre) {
+                        const uint32_t sa = smem_u32(smem + pre * P_STAGE_BYTES);
+                        if (leader) {
+                            mbar_arrive_expect_tx(&ctl->full[pre], 2 * P_STAGE_BYTES);
+                            armed_mask |= 1u << pre;
+                        }
+                        tma_load_2d_pair(sa + A_BYTES, mbh[t.kind], full_of(pre), kb * BK, brow);
+                    }
+                }
+                pdl_wait();
+                pdl_launch();
+            }
+            for (int u = cluster; u < units && !aborted; u += nclusters) {
+                const Tile t = decode_tile_m<PBM>(p, u);
+                const CUtensorMap* ma = t.kind ? &tmA1 : &tmA0;
+                const int arow = t.row0 + t.m_blk * PBM + static_cast<int>(rank) * BM;
+                const int brow = b_row(t);
+                for (int kb = 0; kb < t.num_kb; ++kb) {
+                    const uint32_t sa = smem_u32(smem + s * P_STAGE_BYTES);
+                    if (u == cluster && kb < pre) {
+                        tma_load_2d_pair(sa, ma, full_of(s), kb * BK, arow);
+                    } else {
+                        if (!pair_wait(&ctl->empty[s], ph ^ 1u, ctl, peer_abort, p)) { aborted = true; break; }
+                        if (leader) {
+                            mbar_arrive_expect_tx(&ctl->full[s], 2 * P_STAGE_BYTES);
+                            armed_mask |= 1u << s;
+                            armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
+                        }
+                        tma_load_2d_pair(sa, ma, full_of(s), kb * BK, arow);
+                        tma_load_2d_pair(sa + A_BYTES, mbh[t.kind], full_of(s), kb * BK, brow);
+                    }
+                    if (++s == P_STAGES) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (aborted) {
+                // the leader's armed stages complete when both CTAs' bytes have
+                // landed; a load of the other CTA's that no armed phase counts
+                // is given a fixed time to land (it cannot be observed here)
+                if (leader) {
+                    for (int st = 0; st < P_STAGES; ++st)
+                        if ((armed_mask >> st) & 1u) wait_drain(&ctl->full[st], (armed_ph >> st) & 1u, p);
+                } else {
+                    const uint64_t t0 = global_timer_ns();
+                    while (global_timer_ns() - t0 < 50000ull) {}
+                }
+            }
+        } else if (early) {
+            pdl_wait();
+            pdl_launch();
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (the leader's) ----------------
+        if (early) {
+            pdl_wait();
+            pdl_launch();
+        }
+        if (lane == 0 && leader) {
+            constexpr uint32_t idesc = make_idesc(PBM, 256);
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t aph = 0;
+            bool aborted = false, issued_any = false;
+            for (int u = cluster; u < units && !aborted; u += nclusters) {
+                const Tile t = decode_tile_m<PBM>(p, u);
+                if (!pair_wait(&ctl->tempty[acc], aph ^ 1u, ctl, peer_abort, p)) { aborted = true; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
+                for (int kb = 0; kb < t.num_kb; ++kb) {
+                    if (!pair_wait(&ctl->full[s], ph, ctl, peer_abort, p)) { aborted = true; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + s * P_STAGE_BYTES);
+                    const uint64_t adesc = sw128_desc(sa);
+                    const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc_mma_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    issued_any = true;
+                    tc_commit_pair_mc(&ctl->empty[s], 0x3);
+                    if (++s == P_STAGES) { s = 0; ph ^= 1u; }
+                }
+                if (aborted) break;
+                tc_commit_pair_mc(&ctl->tfull[acc], 0x3);
+                acc ^= 1;
+                if (acc == 0) aph ^= 1u;
+            }
+            if (aborted && issued_any) {
+                // every MMA of this thread (both CTAs' memories) must finish
+                // before either CTA frees its tensor memory
+                tc_commit_pair(&ctl->drain);
+                wait_drain(&ctl->drain, 0, p);
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+        if (early) {
+            pdl_wait();
+            pdl_launch();
+        }
+        const int q = warp & 3;
+        const int r = static_cast<int>(rank) * BM + q * 32 + lane;   // row of this thread in the 256-row tile
+        const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&ctl->tempty[0]), 0u),
+                                           mapa_shared(smem_u32(&ctl->tempty[1]), 0u)};
+        int acc = 0;
+        uint32_t aph = 0;
+        for (int u = cluster; u < units; u += nclusters) {
+            const Tile t = decode_tile_m<PBM>(p, u);
+            if (!pair_wait(&ctl->tfull[acc], aph, ctl, peer_abort, p)) break;
+            tc_fence_after();
+            const int grow = t.m_blk * PBM + r;
+            const size_t orow = static_cast<size_t>(t.row0) + static_cast<size_t>(grow);
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_COLS);
+            pair_store_row<MODE>(p, t, tb, grow < t.rows, orow);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader) mbar_arrive(&ctl->tempty[acc]);
+                else mbar_arrive_remote(tempty_leader[acc]);
+            }
+            acc ^= 1;
+            if (acc == 0) aph ^= 1u;
+        }
+    }
+
+    // neither CTA leaves (or frees tensor memory) while the other may still
+    // use its shared memory, barriers or tensor memory
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
 // ---- host side --------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -640,6 +947,23 @@ bool encode_map(CUtensorMap* m, const void* base, int rows, int cols, int box_ro
 }
 
 template <int MODE>
+cudaError_t launch_pair_mode(const KParams& kp, const CUtensorMap (&maps)[6], cudaStream_t st) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(tc_pair_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             P_SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    const int sms = device_sm_count();
+    if (sms < 2) return cudaErrorInvalidDevice;
+    return launch_k(tc_pair_gemm<MODE>, dim3(sms & ~1), dim3(NUM_THREADS), (size_t)P_SMEM_BYTES, st, maps[0],
+                    maps[1], maps[2], maps[3], maps[4], maps[5], kp);
+}
+
+template <int MODE>
 cudaError_t launch_mode(const TcArgs& a, const KParams& kp, const CUtensorMap (&maps)[6], cudaStream_t st) {
     static bool attr_set[64] = {};
     int dev = 0;
@@ -699,7 +1023,8 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     kp.K[0] = a.K[0]; kp.K[1] = a.K[1];
     kp.out[0] = a.out[0]; kp.out[1] = a.out[1];
     kp.status = a.status;
-    kp.timeout_ns = a.timeout_ns > 0 ? a.timeout_ns : 2000000000LL;
+    kp.timeout_ns = a.timeout_ns > 0 ? a.timeout_ns : wait_limit_ns();
+    kp.drain_ns = kDrainLimitNs;
     kp.partial = a.partial;
     kp.partial_stride = a.partial_stride;
     kp.partial_ld = a.partial_ld;
@@ -708,12 +1033,18 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     kp.ab_out_s = static_cast<__nv_bfloat16*>(a.ab_out_s);
     kp.b_before_wait = a.b_before_wait;
     const int cols = tc_out_cols_per_tile(a.mode);
+    const bool pair = a.pair != 0;
+    if (pair && (a.mode == TC_F32OUT || a.partial != nullptr || a.ab_out != nullptr || a.ab_out_s != nullptr ||
+                 a.tiles == nullptr))
+        return cudaErrorInvalidValue;
     for (int kd = 0; kd < 2; ++kd) {
         kp.nt_blk[kd] = ceil_div(a.N[kd] > 0 ? a.N[kd] : 1, cols);
-        const long long row_bytes = static_cast<long long>(BM) * (a.K[kd] > 0 ? a.K[kd] : 1) * 2;
+        const long long row_bytes = static_cast<long long>(pair ? PBM : BM) * (a.K[kd] > 0 ? a.K[kd] : 1) * 2;
         kp.band_m[kd] = MOE_RASTER_BYTES > 0 ? static_cast<int>(std::max(8ll, MOE_RASTER_BYTES / row_bytes)) : 0;
     }
     if (kp.partial != nullptr && kp.sem == nullptr) return cudaErrorInvalidValue;
+    if (pair) return a.mode == TC_SWIGLU ? launch_pair_mode<TC_SWIGLU>(kp, maps, st)
+                                         : launch_pair_mode<TC_PLAIN>(kp, maps, st);
     switch (a.mode) {
         case TC_SWIGLU: return launch_mode<TC_SWIGLU>(a, kp, maps, st);
         case TC_PLAIN: return launch_mode<TC_PLAIN>(a, kp, maps, st);

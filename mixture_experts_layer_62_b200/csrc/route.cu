@@ -166,155 +166,157 @@ __device__ __forceinline__ float warp_sum(float v) {
 // the gap between the two largest probabilities, p_(1) - p_(2) =
 // (1 - exp(z_(2) - z_(1))) / sum_e exp(z_e - z_(1)).
 template <int EPL>
-__global__ void __launch_bounds__(kSelWarps * 32)
-select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int bias_mode, int gate_mode,
-              int kk, int Tn, int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
-              int32_t* __restrict__ blockcnt, float* __restrict__ blockpsum, float* __restrict__ blockextra) {
-    __shared__ int cnt[kMaxSlotCounts];
-    __shared__ float ps[kSelWarps][MOE_MAX_E];
-    __shared__ float ext[kSelWarps][3];
-    pdl_wait();
-    pdl_launch();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int chunk = blockIdx.x, NB = gridDim.x;
-    for (int e = threadIdx.x; e < E * kk; e += blockDim.x) cnt[e] = 0;
-    float ex_z = 0.f, ex_h = 0.f, ex_g = 0.f;
-    __syncthreads();
+struct SelAcc {
+    float b[EPL];      // selection bias of the lane's experts
+    float psum[EPL];   // sum of the warp's tokens' probabilities of the lane's experts
+    float ex_z, ex_h, ex_g;
+};
 
-    float b[EPL];
+template <int EPL>
+__device__ __forceinline__ void sel_init(SelAcc<EPL>& a, const float* __restrict__ bias, int bias_mode, int E,
+                                         int lane) {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        a.b[i] = (bias_mode != MOE_BIAS_NONE && e < E) ? bias[e] : 0.f;
+        a.psum[i] = 0.f;
+    }
+    a.ex_z = a.ex_h = a.ex_g = 0.f;
+}
+
+// One token t whose logits the warp holds (lane l: experts l + 32 i in
+// zin[i]): softmax, statistics, key, top-k, gates, and the chunk's counts.
+template <int EPL>
+__device__ __forceinline__ void sel_token(const float (&zin)[EPL], int t, int bias_mode, int gate_mode, int kk,
+                                          int E, int k, int lane, SelAcc<EPL>& a, int* cnt,
+                                          int32_t* __restrict__ idx_out, float* __restrict__ gate_out) {
+    float z[EPL], key[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         int e = lane + 32 * i;
-        b[i] = (bias_mode != MOE_BIAS_NONE && e < E) ? bias[e] : 0.f;
+        z[i] = e < E ? zin[i] : -INFINITY;
     }
-    float psum[EPL];
+    // full softmax over all E raw logits (for P and the PROB key)
+    float m = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) psum[i] = 0.f;
-
-    constexpr int kTokPerWarp = kChunk / kSelWarps;
-    for (int q = 0; q < kTokPerWarp; ++q) {
-        const int t = chunk * kChunk + warp * kTokPerWarp + q;
-        if (t >= Tn) break;
-        float z[EPL], key[EPL];
-        const float* zr = logits + (size_t)t * E;
+    for (int i = 0; i < EPL; ++i) m = fmaxf(m, z[i]);
+    m = warp_max(m);
+    float ex[EPL], s = 0.f;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            int e = lane + 32 * i;
-            z[i] = e < E ? zr[e] : -INFINITY;
-        }
-        // full softmax over all E raw logits (for P and the PROB key)
-        float m = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) m = fmaxf(m, z[i]);
-        m = warp_max(m);
-        float ex[EPL], s = 0.f;
+    for (int i = 0; i < EPL; ++i) {
+        int e = lane + 32 * i;
+        ex[i] = e < E ? expf(z[i] - m) : 0.f;
+        s += ex[i];
+    }
+    s = warp_sum(s);
+    const float inv_s = 1.f / s;
+    // router statistics of this token
+    {
+        float pz = 0.f, z1 = -INFINITY, z2 = -INFINITY;
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
-            int e = lane + 32 * i;
-            ex[i] = e < E ? expf(z[i] - m) : 0.f;
-            s += ex[i];
+            if (lane + 32 * i < E) {
+                pz += ex[i] * z[i];
+                if (z[i] > z1) { z2 = z1; z1 = z[i]; } else if (z[i] > z2) { z2 = z[i]; }
+            }
         }
-        s = warp_sum(s);
-        const float inv_s = 1.f / s;
-        // router statistics of this token
-        {
-            float pz = 0.f, z1 = -INFINITY, z2 = -INFINITY;
+        pz = warp_sum(pz) * inv_s;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float o1 = __shfl_xor_sync(0xffffffffu, z1, o);
+            const float o2 = __shfl_xor_sync(0xffffffffu, z2, o);
+            const float hi = fmaxf(z1, o1);
+            z2 = fmaxf(fminf(z1, o1), fmaxf(z2, o2));
+            z1 = hi;
+        }
+        const float lse = m + logf(s);
+        a.ex_z += lse * lse;
+        a.ex_h += lse - pz;
+        a.ex_g += (1.f - expf(z2 - m)) * inv_s;
+    }
+    unsigned valid = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        int e = lane + 32 * i;
+        float p = ex[i] * inv_s;
+        if (e < E) {
+            a.psum[i] += p;
+            valid |= 1u << i;
+        }
+        key[i] = bias_mode == MOE_BIAS_NONE ? z[i]
+               : bias_mode == MOE_BIAS_LOGIT ? z[i] + a.b[i]
+               : p + a.b[i];
+    }
+    // top-k: k rounds of a warp arg-max over (key desc, index asc)
+    unsigned taken = 0;
+    float zsel[MOE_MAX_K];
+    int esel[MOE_MAX_K];
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_K; ++j) {
+        if (j < k) {
+            float bk = -INFINITY, bz = 0.f;
+            int be = 0x7fffffff;
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
-                if (lane + 32 * i < E) {
-                    pz += ex[i] * z[i];
-                    if (z[i] > z1) { z2 = z1; z1 = z[i]; } else if (z[i] > z2) { z2 = z[i]; }
+                bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
+                if (ok && (key[i] > bk || be == 0x7fffffff)) {
+                    bk = key[i]; be = lane + 32 * i; bz = z[i];
                 }
             }
-            pz = warp_sum(pz) * inv_s;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
-                const float o1 = __shfl_xor_sync(0xffffffffu, z1, o);
-                const float o2 = __shfl_xor_sync(0xffffffffu, z2, o);
-                const float hi = fmaxf(z1, o1);
-                z2 = fmaxf(fminf(z1, o1), fmaxf(z2, o2));
-                z1 = hi;
+                float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
+                int oe = __shfl_xor_sync(0xffffffffu, be, o);
+                float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+                bool better = (oe != 0x7fffffff) &&
+                              (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
+                if (better) { bk = ok_; be = oe; bz = oz; }
             }
-            const float lse = m + logf(s);
-            ex_z += lse * lse;
-            ex_h += lse - pz;
-            ex_g += (1.f - expf(z2 - m)) * inv_s;
+            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            zsel[j] = bz;
+            esel[j] = be;
         }
-        unsigned valid = 0;
+    }
+    // gates: softmax over the selected raw logits, slot order
+    float zm = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            int e = lane + 32 * i;
-            float p = ex[i] * inv_s;
-            if (e < E) {
-                psum[i] += p;
-                valid |= 1u << i;
-            }
-            key[i] = bias_mode == MOE_BIAS_NONE ? z[i]
-                   : bias_mode == MOE_BIAS_LOGIT ? z[i] + b[i]
-                   : p + b[i];
-        }
-        // top-k: k rounds of a warp arg-max over (key desc, index asc)
-        unsigned taken = 0;
-        float zsel[MOE_MAX_K];
-        int esel[MOE_MAX_K];
+    for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) zm = fmaxf(zm, zsel[j]);
+    float gs = 0.f, ge[MOE_MAX_K];
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_K; ++j) {
+        if (j < k) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
+    }
+    const float inv_g = 1.f / gs;
+    if (lane == 0) {
 #pragma unroll
         for (int j = 0; j < MOE_MAX_K; ++j) {
             if (j < k) {
-                float bk = -INFINITY, bz = 0.f;
-                int be = 0x7fffffff;
-#pragma unroll
-                for (int i = 0; i < EPL; ++i) {
-                    bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
-                    if (ok && (key[i] > bk || be == 0x7fffffff)) {
-                        bk = key[i]; be = lane + 32 * i; bz = z[i];
-                    }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
-                    int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-                    bool better = (oe != 0x7fffffff) &&
-                                  (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
-                    if (better) { bk = ok_; be = oe; bz = oz; }
-                }
-                if ((be & 31) == lane) taken |= 1u << (be >> 5);
-                zsel[j] = bz;
-                esel[j] = be;
-            }
-        }
-        // gates: softmax over the selected raw logits, slot order
-        float zm = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) zm = fmaxf(zm, zsel[j]);
-        float gs = 0.f, ge[MOE_MAX_K];
-#pragma unroll
-        for (int j = 0; j < MOE_MAX_K; ++j) {
-            if (j < k) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
-        }
-        const float inv_g = 1.f / gs;
-        if (lane == 0) {
-#pragma unroll
-            for (int j = 0; j < MOE_MAX_K; ++j) {
-                if (j < k) {
-                    idx_out[(size_t)t * k + j] = esel[j];
-                    // selected softmax, or the full-softmax probability (Switch gate)
-                    gate_out[(size_t)t * k + j] =
-                        gate_mode == MOE_GATE_FULL ? expf(zsel[j] - m) * inv_s : ge[j] * inv_g;
-                    atomicAdd(&cnt[esel[j] * kk + (kk > 1 ? j : 0)], 1);   // integer: order does not matter
-                }
+                idx_out[(size_t)t * k + j] = esel[j];
+                // selected softmax, or the full-softmax probability (Switch gate)
+                gate_out[(size_t)t * k + j] =
+                    gate_mode == MOE_GATE_FULL ? expf(zsel[j] - m) * inv_s : ge[j] * inv_g;
+                atomicAdd(&cnt[esel[j] * kk + (kk > 1 ? j : 0)], 1);   // integer: order does not matter
             }
         }
     }
+}
+
+// The chunk's statistics: probability sums over warps in warp order, counts,
+// and the z-loss / entropy / gap sums.
+template <int EPL>
+__device__ __forceinline__ void sel_finish(const SelAcc<EPL>& a, int chunk, int NB, int E, int kk, int warp, int lane,
+                                           const int* cnt, float (*ps)[MOE_MAX_E], float (*ext)[3],
+                                           int32_t* __restrict__ blockcnt, float* __restrict__ blockpsum,
+                                           float* __restrict__ blockextra) {
     if (lane == 0) {
-        ext[warp][0] = ex_z;
-        ext[warp][1] = ex_h;
-        ext[warp][2] = ex_g;
+        ext[warp][0] = a.ex_z;
+        ext[warp][1] = a.ex_h;
+        ext[warp][2] = a.ex_g;
     }
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         int e = lane + 32 * i;
-        if (e < E) ps[warp][e] = psum[i];
+        if (e < E) ps[warp][e] = a.psum[i];
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -328,6 +330,216 @@ select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, 
         for (int w = 0; w < kSelWarps; ++w) acc += ext[w][threadIdx.x];
         blockextra[(size_t)chunk * 3 + threadIdx.x] = acc;
     }
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(kSelWarps * 32)
+select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int bias_mode, int gate_mode,
+              int kk, int Tn, int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+              int32_t* __restrict__ blockcnt, float* __restrict__ blockpsum, float* __restrict__ blockextra) {
+    __shared__ int cnt[kMaxSlotCounts];
+    __shared__ float ps[kSelWarps][MOE_MAX_E];
+    __shared__ float ext[kSelWarps][3];
+    pdl_wait();
+    pdl_launch();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunk = blockIdx.x, NB = gridDim.x;
+    for (int e = threadIdx.x; e < E * kk; e += blockDim.x) cnt[e] = 0;
+    SelAcc<EPL> a;
+    sel_init(a, bias, bias_mode, E, lane);
+    __syncthreads();
+
+    constexpr int kTokPerWarp = kChunk / kSelWarps;
+    for (int q = 0; q < kTokPerWarp; ++q) {
+        const int t = chunk * kChunk + warp * kTokPerWarp + q;
+        if (t >= Tn) break;
+        float z[EPL];
+        const float* zr = logits + (size_t)t * E;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            int e = lane + 32 * i;
+            z[i] = e < E ? zr[e] : -INFINITY;
+        }
+        sel_token<EPL>(z, t, bias_mode, gate_mode, kk, E, k, lane, a, cnt, idx_out, gate_out);
+    }
+    sel_finish<EPL>(a, chunk, NB, E, kk, warp, lane, cnt, ps, ext, blockcnt, blockpsum, blockextra);
+}
+
+// ---- fused router: logits and selection in one kernel ----------------------
+// One block per chunk of kChunk tokens, the same warp-to-token assignment as
+// select_kernel (warp w: tokens 4w .. 4w + 3 of the chunk). A warp computes
+// its four tokens' logits itself: lane l takes the 8-element chunks c = l,
+// l + 32, ... of the row (16-byte loads of x, four chunks in flight per
+// token), multiplies them with the matching rows of W_r [d, E] as given (no
+// transposed copy: a row of W_r holds the E weights of one input feature),
+// eight experts per pass, and an xor butterfly leaves every lane with the
+// sums, in a fixed order. The logits are written out (the workspace keeps
+// them) and, still in registers, go through the same per-token selection as
+// select_kernel. x is read once from HBM; W_r (d E elements) is re-read from
+// L1/L2 by each warp. E <= 64.
+template <typename T>
+struct RawVec8 {   // 8 elements of a row as loaded: one 16-byte vector (bf16) or two (fp32)
+    uint4 v[sizeof(T) == 2 ? 1 : 2];
+};
+template <typename T>
+__device__ __forceinline__ void raw_load8(const T* p, RawVec8<T>& r) {
+#pragma unroll
+    for (int i = 0; i < (sizeof(T) == 2 ? 1 : 2); ++i) r.v[i] = __ldg(reinterpret_cast<const uint4*>(p) + i);
+}
+__device__ __forceinline__ void unpack8(const RawVec8<__nv_bfloat16>& r, float (&v)[8]) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r.v[0]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x; v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void unpack8(const RawVec8<float>& r, float (&v)[8]) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        v[4 * i] = __uint_as_float(r.v[i].x); v[4 * i + 1] = __uint_as_float(r.v[i].y);
+        v[4 * i + 2] = __uint_as_float(r.v[i].z); v[4 * i + 3] = __uint_as_float(r.v[i].w);
+    }
+}
+
+template <typename T, int EPL>
+__global__ void __launch_bounds__(kSelWarps * 32)
+route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const float* __restrict__ bias,
+                   int bias_mode, int gate_mode, int kk, int Tn, int d, int E, int k, float* __restrict__ logits,
+                   int32_t* __restrict__ idx_out, float* __restrict__ gate_out, int32_t* __restrict__ blockcnt,
+                   float* __restrict__ blockpsum, float* __restrict__ blockextra, int32_t* __restrict__ status) {
+    static_assert(EPL <= 2, "fused router: E <= 64");
+    constexpr int kTokPerWarp = kChunk / kSelWarps;   // 4
+    constexpr int U = sizeof(T) == 2 ? 4 : 2;         // row chunks of x in flight per token
+    __shared__ int cnt[kMaxSlotCounts];
+    __shared__ float ps[kSelWarps][MOE_MAX_E];
+    __shared__ float ext[kSelWarps][3];
+    pdl_wait();
+    pdl_launch();
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = MOE_OK;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunk = blockIdx.x, NB = gridDim.x;
+    for (int e = threadIdx.x; e < E * kk; e += blockDim.x) cnt[e] = 0;
+    SelAcc<EPL> a;
+    sel_init(a, bias, bias_mode, E, lane);
+
+    const int t0 = chunk * kChunk + warp * kTokPerWarp;
+    const int nt = max(0, min(kTokPerWarp, Tn - t0));
+    const int nchunk = d / 8;
+    const bool wvec = (E % kExpPerPass) == 0;   // W_r rows start on 16-byte boundaries
+    float zt[kTokPerWarp][EPL];
+#pragma unroll
+    for (int q = 0; q < kTokPerWarp; ++q)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) zt[q][i] = -INFINITY;
+    for (int e0 = 0; e0 < E; e0 += kExpPerPass) {
+        float acc[kTokPerWarp][kExpPerPass];
+#pragma unroll
+        for (int q = 0; q < kTokPerWarp; ++q)
+#pragma unroll
+            for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = 0.f;
+        for (int cb = lane; cb < nchunk; cb += 32 * U) {
+            RawVec8<T> xr[U][kTokPerWarp];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = cb + 32 * u;
+#pragma unroll
+                for (int q = 0; q < kTokPerWarp; ++q) {
+                    if (q < nt && c < nchunk) {
+                        raw_load8(x + (size_t)(t0 + q) * d + (size_t)c * 8, xr[u][q]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < (sizeof(T) == 2 ? 1 : 2); ++i) xr[u][q].v[i] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = cb + 32 * u;
+                if (c < nchunk) {
+                    float xv[kTokPerWarp][8];
+#pragma unroll
+                    for (int q = 0; q < kTokPerWarp; ++q) unpack8(xr[u][q], xv[q]);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        // weights of input feature 8c + j for experts e0 .. e0 + 7
+                        const T* wrow = W_r + (size_t)(c * 8 + j) * E + e0;
+                        float wv[kExpPerPass];
+                        if (wvec) {
+                            load8(wrow, wv);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < kExpPerPass; ++e) wv[e] = e0 + e < E ? float(wrow[e]) : 0.f;
+                        }
+#pragma unroll
+                        for (int q = 0; q < kTokPerWarp; ++q)
+#pragma unroll
+                            for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = fmaf(xv[q][j], wv[e], acc[q][e]);
+                    }
+                }
+            }
+        }
+    // butterfly sums: every lane ends with the same bits
+#pragma unroll
+        for (int q = 0; q < kTokPerWarp; ++q)
+#pragma unroll
+            for (int e = 0; e < kExpPerPass; ++e) {
+                float v = acc[q][e];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                acc[q][e] = v;
+            }
+        // expert e0 + e belongs to lane (e0 + e) % 32, register (e0 + e) / 32
+        const int ir = e0 >> 5;
+#pragma unroll
+        for (int e = 0; e < kExpPerPass; ++e) {
+            if (lane == ((e0 + e) & 31) && e0 + e < E) {
+#pragma unroll
+                for (int q = 0; q < kTokPerWarp; ++q) {
+#pragma unroll
+                    for (int i = 0; i < EPL; ++i)
+                        if (i == ir) zt[q][i] = acc[q][e];
+                }
+            }
+        }
+    }
+    __syncthreads();   // the chunk's counters are zeroed
+#pragma unroll
+    for (int q = 0; q < kTokPerWarp; ++q) {
+        if (q < nt) {
+            const int t = t0 + q;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int e = lane + 32 * i;
+                if (e < E) logits[(size_t)t * E + e] = zt[q][i];
+            }
+            sel_token<EPL>(zt[q], t, bias_mode, gate_mode, kk, E, k, lane, a, cnt, idx_out, gate_out);
+        }
+    }
+    sel_finish<EPL>(a, chunk, NB, E, kk, warp, lane, cnt, ps, ext, blockcnt, blockpsum, blockextra);
+}
+
+bool route_fused_ok(int dtype, int d, int E) {
+    return E <= 64 && d % 8 == 0 && (dtype == MOE_DTYPE_F32 || dtype == MOE_DTYPE_BF16);
+}
+
+cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const float* bias, int bias_mode,
+                               int gate_mode, int kk, int T, int d, int E, int k, float* logits, int32_t* idx,
+                               float* gate, int32_t* blockcnt, float* blockpsum, float* blockextra, int32_t* status,
+                               cudaStream_t st) {
+    const int NB = ceil_div(T, kChunk);
+    if (NB == 0) return cudaSuccess;
+    dim3 grid(NB), block(kSelWarps * 32);
+#define MOE_FUSED(TYPE, EPLV)                                                                                     \
+    return launch_k(route_fused_kernel<TYPE, EPLV>, grid, block, 0, st, (const TYPE*)x, (const TYPE*)W_r, bias,   \
+                    bias_mode, gate_mode, kk, T, d, E, k, logits, idx, gate, blockcnt, blockpsum, blockextra, status)
+    if (dtype == MOE_DTYPE_BF16) {
+        if (E <= 32) MOE_FUSED(__nv_bfloat16, 1);
+        MOE_FUSED(__nv_bfloat16, 2);
+    }
+    if (E <= 32) MOE_FUSED(float, 1);
+    MOE_FUSED(float, 2);
+#undef MOE_FUSED
 }
 
 cudaError_t launch_select(const float* logits, const float* bias, int bias_mode, int gate_mode, int kk, int T,

@@ -17,7 +17,8 @@ HEADER = os.path.join(ROOT, "include", "moe.h")
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"^\s*(?:int|int32_t|size_t|const\s+char\s*\*)\s+(moe_\w+)\s*\(", src, flags=re.M)
+    names = re.findall(r"^\s*(?:int|int32_t|size_t|long\s+long|const\s+char\s*\*)\s+(moe_\w+)\s*\(", src,
+                       flags=re.M)
     assert names, "no declarations parsed"
     return sorted(set(names))
 
@@ -32,6 +33,20 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert set(names) <= exported
     # nothing exported under the moe_ prefix that the header does not declare
     assert exported <= set(names), exported - set(names)
+
+
+def test_wait_limit_is_settable_and_restorable():
+    # host-side setting only (nothing launched): the previous value comes back,
+    # and a non-positive value restores the 2 s default
+    prev = moe.set_wait_limit(12345)
+    try:
+        assert prev == 2_000_000_000
+        assert moe.set_wait_limit(777) == 12345
+        assert moe.set_wait_limit(0) == 777
+        assert moe.set_wait_limit(-5) == 2_000_000_000
+    finally:
+        moe.set_wait_limit(prev)
+    assert moe.set_wait_limit(0) == 2_000_000_000
 
 
 def test_error_strings():

@@ -39,10 +39,13 @@ def test_decode_bytes_count_touched_experts_only():
 
 def test_launch_counts():
     assert bench.launches_per_forward(inputs.workload("decode_t1")) == 5
-    assert bench.launches_per_forward(inputs.workload("mixtral_prefill")) == 8
-    assert bench.launches_per_forward(inputs.workload("mixtral_prefill"), pad_rows=128) == 9
+    # fused router up to 64 experts: router, scan, gather, GEMM 1/3, GEMM 2, combine
+    assert bench.launches_per_forward(inputs.workload("mixtral_prefill")) == 6
+    assert bench.launches_per_forward(inputs.workload("mixtral_prefill"), pad_rows=128) == 7
+    # wide routers run on the tensor cores: transpose, logits, select
+    assert bench.launches_per_forward(inputs.workload("deepseek_v3")) == 8
     # the shared expert rules out the small-batch router
-    assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), d_ff_shared=2048)) == 8
+    assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), d_ff_shared=2048)) == 6
     assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), T=0)) == 1
 
 

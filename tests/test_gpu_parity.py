@@ -214,6 +214,13 @@ def test_padded_forward_equals_dense():
     # blocks, GEMM 2 with K = 14336 (9 blocks a band) over 10 blocks
     ("bf16", 7168, 256, [70, 2300], 0, 10),
     ("bf16", 256, 14336, [1200, 3], 0, 10),
+    # at least 512 rows per expert on average: CTA-pair tiles of 256 rows
+    # (ragged, empty and single-row groups; the shared expert; a group of 11
+    # pair M blocks over a band of 8 at K = 14336)
+    ("bf16", 512, 384, [600, 0, 1300, 257], 0, 1100),
+    ("bf16", 256, 256, [700, 900], 128, 800),
+    ("bf16", 256, 14336, [2600, 3], 0, 10),
+    ("bf16", 128, 128, [1, 1023], 0, 512),
 ])
 def test_experts_stage(dtype, d, d_ff, counts, shared, T):
     E = len(counts)
@@ -324,6 +331,11 @@ SMALL = [
     dict(T=700, d=128, d_ff=256, E=16, k=2, cf=0.7, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=0, drop=1),
     dict(T=24, d=256, d_ff=128, E=8, k=2, cf=0.6, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=1, drop=1),
     dict(T=200, d=64, d_ff=64, E=6, k=3, cf=0.5, dtype="f32", bias_mode=0, d_ff_shared=0, gate=1, drop=1),
+    # at least 512 rows per expert on average: CTA-pair tiles of 256 rows
+    dict(T=2048, d=256, d_ff=384, E=4, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
+    dict(T=3000, d=128, d_ff=256, E=4, k=2, cf=0.9, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=1, drop=1),
+    dict(T=1024, d=128, d_ff=128, E=2, k=1, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=128),
+    dict(T=600, d=192, d_ff=320, E=1, k=1, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     # padded (MegaBlocks) layout: every expert's rows rounded up to 128 or 64
     dict(T=300, d=256, d_ff=384, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0, pad=128),
     dict(T=1000, d=256, d_ff=256, E=8, k=2, cf=0.6, dtype="bf16", bias_mode=1, d_ff_shared=0, pad=64),
