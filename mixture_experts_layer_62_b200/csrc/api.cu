@@ -42,8 +42,8 @@ Layout make_layout(const moe_problem& p) {
     // logits [T][parts][E] here
     L.blockpsum = take((small_route_ok(p) ? T * kSmallMaxParts : NB) * E * 4);
     L.blockextra = take(NB * 3 * 4);
-    L.tiles13 = take((E + 3) * 4);
-    L.tiles2 = take((E + 3) * 4);
+    L.tiles13 = take((size_t)schedule_ints(p.E) * 4);
+    L.tiles2 = take((size_t)schedule_ints(p.E) * 4);
     L.xp = take(Rmax * d * eb);
     L.h = take(Rmax * dff * eb);
     L.o = take(Rmax * d * eb);
@@ -146,6 +146,21 @@ bool use_pair_tiles(const moe_problem& p) {
     }();
     return enabled && p.dtype == MOE_DTYPE_BF16 && p.T > 0 && p.pad_rows == 0 && !p.train && !split_allowed(p) &&
            (long long)p.T * p.k >= 512LL * p.E;
+}
+
+GridSplit grid_split_of(const moe_problem& p) {
+    static const int forced = [] {
+        const char* v = std::getenv("MOE_SMALL_CTAS");
+        return v != nullptr ? std::atoi(v) : -1;
+    }();
+    GridSplit g = {};
+    g.on = forced != 0 && p.dtype == MOE_DTYPE_BF16 && p.T > 0 && p.pad_rows == 0 && !p.train && !split_allowed(p) &&
+           !use_pair_tiles(p) && p.E >= 32 && p.d % 64 == 0;
+    g.k13 = p.d; g.k2 = p.d_ff; g.k13s = p.d; g.k2s = p.d_ff_shared;
+    g.grid = device_sm_count();
+    g.force_ctas = forced > 0 ? forced : 0;
+    if (g.grid <= 1) g.on = 0;
+    return g;
 }
 
 thread_local bool g_pdl = false;
@@ -266,6 +281,7 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
         TcArgs a = {};
         a.mode = TC_SWIGLU;
         a.pair = use_pair_tiles(*p) ? 1 : 0;
+        a.split_grid = grid_split_of(*p).on;
         a.b_before_wait = sched_early ? 1 : 0;
         a.indptr = indptr; a.tiles = tiles13;
         a.E = p->E; a.has_shared = has_shared; a.T = p->T;
@@ -311,6 +327,7 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
         TcArgs b = {};
         b.mode = TC_PLAIN;
         b.pair = use_pair_tiles(*p) ? 1 : 0;
+        b.split_grid = grid_split_of(*p).on;
         b.b_before_wait = 1;   // the schedule comes from the router, two or more launches back
         b.indptr = indptr; b.tiles = tiles2;
         b.E = p->E; b.has_shared = has_shared; b.T = p->T;
@@ -382,6 +399,7 @@ struct StageSplit {
 };
 StageSplit stage_split(const moe_problem* p, const Layout& L, void* ws) {
     StageSplit s;
+    s.sched.gsplit = grid_split_of(*p);
     if (!split_allowed(*p)) return s;
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
@@ -710,6 +728,7 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     sa.indptr = indptr; sa.stats = stats;
     sa.tiles13 = tiles13; sa.tiles2 = tiles2; sa.has_shared = shared ? 1 : 0;
     schedule_sizes(p, sa.tile_m, sa.ntiles13, sa.ntiles2, sa.ntiles13_shared, sa.ntiles2_shared);
+    sa.gsplit = grid_split_of(*p);
     sa.split_on = split ? 1 : 0;
     if (split) {
         sa.sem = sem;

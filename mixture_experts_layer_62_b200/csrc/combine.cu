@@ -53,6 +53,7 @@ template <> struct VecTraits<__nv_bfloat16> {
 // vectors (vpl = 1 for small batches), so few tokens still spread over many
 // warps.
 constexpr int kCbVecPerLane = 2;
+constexpr int kCbSlotGroup = 2;   // slots whose rows are requested together
 constexpr int kCbWarps = 8;
 
 template <typename T>
@@ -82,46 +83,60 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const f
     pdl_wait();
     pdl_launch();
     const int nvec = d / VN;
-    for (int i = 0; i < vpl; ++i) {
-        const int v0 = (sl * vpl + i) * 32;
-        if (v0 >= nvec) break;  // warp-uniform
-        const int v = v0 + lane;
-        const bool valid = v < nvec;
-        float acc[VN];
+    // the warp's vpl vector columns are processed together: for each pair of
+    // slots, every row vector of the pair and of every column is requested
+    // before any is accumulated (2 vpl loads in flight per lane); the
+    // accumulation is still in slot order for each element
+    float acc[kCbVecPerLane][VN];
 #pragma unroll
-        for (int e = 0; e < VN; ++e) acc[e] = 0.f;
-        // slots in groups of 4: the group's rows are all requested before any
-        // is accumulated (slot order is kept)
-        for (int j0 = 0; j0 < k; j0 += 4) {
-            uint4 raw[4];
-            int pj[4];
-            float gj[4];
+    for (int i = 0; i < kCbVecPerLane; ++i)
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                pj[u] = __shfl_sync(0xffffffffu, p_l, j0 + u);
-                gj[u] = __shfl_sync(0xffffffffu, g_l, j0 + u);
-                raw[u] = make_uint4(0u, 0u, 0u, 0u);
-                if (j0 + u < k && pj[u] >= 0 && valid)
-                    raw[u] = *reinterpret_cast<const uint4*>(o + (size_t)pj[u] * d + (size_t)v * VN);
+        for (int e = 0; e < VN; ++e) acc[i][e] = 0.f;
+    int vv[kCbVecPerLane];
+    bool valid[kCbVecPerLane];
+#pragma unroll
+    for (int i = 0; i < kCbVecPerLane; ++i) {
+        vv[i] = (sl * vpl + i) * 32 + lane;
+        valid[i] = i < vpl && vv[i] < nvec;
+    }
+    for (int j0 = 0; j0 < k; j0 += kCbSlotGroup) {
+        uint4 raw[kCbSlotGroup][kCbVecPerLane];
+        int pj[kCbSlotGroup];
+        float gj[kCbSlotGroup];
+#pragma unroll
+        for (int u = 0; u < kCbSlotGroup; ++u) {
+            pj[u] = __shfl_sync(0xffffffffu, p_l, j0 + u);
+            gj[u] = __shfl_sync(0xffffffffu, g_l, j0 + u);
+#pragma unroll
+            for (int i = 0; i < kCbVecPerLane; ++i) {
+                raw[u][i] = make_uint4(0u, 0u, 0u, 0u);
+                if (j0 + u < k && pj[u] >= 0 && valid[i])
+                    raw[u][i] = *reinterpret_cast<const uint4*>(o + (size_t)pj[u] * d + (size_t)vv[i] * VN);
             }
+        }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (j0 + u < k && pj[u] >= 0) {
+        for (int u = 0; u < kCbSlotGroup; ++u) {
+            if (j0 + u < k && pj[u] >= 0) {
+#pragma unroll
+                for (int i = 0; i < kCbVecPerLane; ++i) {
                     float ov[VN];
-                    V::unpack(raw[u], ov);
+                    V::unpack(raw[u][i], ov);
 #pragma unroll
-                    for (int e = 0; e < VN; ++e) acc[e] = fmaf(gj[u], ov[e], acc[e]);
+                    for (int e = 0; e < VN; ++e) acc[i][e] = fmaf(gj[u], ov[e], acc[i][e]);
                 }
             }
         }
-        if (!valid) continue;
+    }
+#pragma unroll
+    for (int i = 0; i < kCbVecPerLane; ++i) {
+        if (!valid[i]) continue;
         if (s != nullptr) {
             float sv[VN];
-            V::load(s + (size_t)t * d + (size_t)v * VN, sv);
+            V::load(s + (size_t)t * d + (size_t)vv[i] * VN, sv);
 #pragma unroll
-            for (int e = 0; e < VN; ++e) acc[e] += sv[e];
+            for (int e = 0; e < VN; ++e) acc[i][e] += sv[e];
         }
-        V::store(out + (size_t)t * d + (size_t)v * VN, acc);
+        V::store(out + (size_t)t * d + (size_t)vv[i] * VN, acc[i]);
     }
 }
 

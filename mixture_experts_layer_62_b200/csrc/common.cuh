@@ -137,6 +137,25 @@ cudaError_t launch_hist(const int32_t* idx, int T, int k, int kk, int E, int32_t
 // Scan over per-chunk expert counts: per-expert totals, capacity, indptr,
 // chunk rank bases, statistics and (optionally) the tile schedules of the
 // two grouped GEMMs.
+// Grid split of the single-CTA grouped GEMMs for fine-grained experts: the
+// groups of at most kSmallRows rows run as operand-swapped tiles (the
+// weights as the 128-row MMA operand, the group's rows as N = 32..128, so a
+// 7-row group costs little tensor work and its time is its weight stream) on
+// the first S CTAs, while the other CTAs run the larger groups' ordinary
+// tiles; the schedule writer picks S so that both classes end together.
+// Schedule array of one GEMM with the split: [0..G] cumulative tiles of the
+// large class, [G+1] split-K factor (1), [G+2] S, [G+3 .. 2G+3] cumulative
+// tiles of the small class (one M block per group); without the split only
+// [0..G+1] are used and [G+2] is 0.
+constexpr int kSmallRows = 128;
+struct GridSplit {
+    int on;
+    int k13, k2, k13s, k2s;   // K of the routed and shared GEMM 1/3 and GEMM 2
+    int grid;                 // CTAs of the GEMM launches
+    int force_ctas;           // > 0: S from the environment (tuning), else the cost model
+};
+inline int schedule_ints(int E) { return 2 * (E + 1) + 6; }
+
 struct ScanArgs {
     int T, k, E, capacity;       // capacity < 0: unlimited
     int kk;                      // count slots per expert (k for slot priority, else 1)
@@ -153,6 +172,7 @@ struct ScanArgs {
     int32_t* sem; int sem_n;     // split-K counters to zero (sem_n ints), or null
     SplitTable split;
     int pad;                     // > 0: indptr over kept rows rounded up to a multiple of pad
+    GridSplit gsplit;            // small/large tile classes of the single-CTA GEMMs
 };
 cudaError_t launch_scan(const ScanArgs& a, cudaStream_t st);
 // Padding rows of a padded permutation: rows [indptr[e] + kept[e], indptr[e+1])
@@ -165,6 +185,7 @@ struct ScheduleSplit {
     int split_on;
     int32_t* sem; int sem_n;
     SplitTable split;
+    GridSplit gsplit;
 };
 cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
                             int ntiles13, int ntiles2, int ntiles13_shared, int ntiles2_shared,
@@ -222,6 +243,10 @@ constexpr int kTcPairTileM = 256;   // rows of a CTA-pair tile
 // not the training forward, unpadded, at least 512 rows per expert on
 // average); the environment variable MOE_CTA_PAIR=0 turns them off.
 bool use_pair_tiles(const moe_problem& p);
+// The small/large grid split for p (bf16 inference, no split-K, no pairs,
+// at least 32 experts); MOE_SMALL_CTAS=n forces S = n (n = 0 turns the split
+// off).
+GridSplit grid_split_of(const moe_problem& p);
 int tc_out_cols_per_tile(int mode);   // 128 for SWIGLU, 256 otherwise
 enum TcMode { TC_SWIGLU = 0, TC_PLAIN = 1, TC_F32OUT = 2 };
 struct TcArgs {
@@ -251,6 +276,9 @@ struct TcArgs {
     // 1: CTA pairs with 256-row tiles (the schedule counts 256-row M blocks);
     // SWIGLU or PLAIN, no split-K, no pre-activation output
     int pair;
+    // 1: the schedule carries the small/large grid split (GridSplit); SWIGLU
+    // or PLAIN, no split-K, no pre-activation output
+    int split_grid;
 };
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
 // Backward grouped GEMMs (tcgen05): see gemm_bwd_sm100.cu.

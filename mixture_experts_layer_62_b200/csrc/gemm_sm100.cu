@@ -80,6 +80,7 @@ struct KParams {
     int b_before_wait;         // weight tiles of the first stages may load before the dependency wait
     int nt_blk[2];             // N blocks of a group (routed, shared)
     int band_m[2];             // M blocks per band (0: the whole group is one band)
+    int split_grid;            // the schedule carries the small/large grid split
 };
 
 struct Tile {
@@ -126,6 +127,49 @@ __device__ __forceinline__ Tile decode_tile_m(const KParams& p, int tile) {
     return t;
 }
 __device__ __forceinline__ Tile decode_tile(const KParams& p, int tile) { return decode_tile_m<BM>(p, tile); }
+
+// The units a CTA runs: first, first + step, ... below count. With the grid
+// split, CTAs [0, S) run the small class (operand-swapped tiles of the
+// groups of at most kSmallRows rows) and the others the large class.
+struct Units {
+    int first, step, count;
+    bool small;
+};
+__device__ __forceinline__ Units cta_units(const KParams& p, int total, int nsplit) {
+    Units r;
+    if (p.split_grid) {
+        const int G = p.E + p.has_shared;
+        const int S = p.tiles[G + 2];
+        if (static_cast<int>(blockIdx.x) < S) {
+            r.first = blockIdx.x; r.step = S; r.count = p.tiles[2 * G + 3]; r.small = true;
+        } else {
+            r.first = blockIdx.x - S; r.step = gridDim.x - S; r.count = total; r.small = false;
+        }
+        return r;
+    }
+    r.first = blockIdx.x; r.step = gridDim.x; r.count = total * nsplit; r.small = false;
+    return r;
+}
+// Tile u of the small class: one M block of a routed group of 1..128 rows.
+__device__ __forceinline__ Tile decode_small_tile(const KParams& p, int u) {
+    const int G = p.E + p.has_shared;
+    const int32_t* cum = p.tiles + G + 3;
+    int lo = 0, hi = G;   // cum[lo] <= u < cum[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cum[mid] <= u) lo = mid; else hi = mid;
+    }
+    Tile t;
+    t.g = lo;
+    t.kind = 0;
+    t.row0 = p.indptr[lo];
+    t.rows = p.indptr[lo + 1] - t.row0;
+    t.m_blk = 0;
+    t.n_blk = u - cum[lo];
+    t.num_kb = (p.K[0] + BK - 1) / BK;
+    return t;
+}
+__device__ __forceinline__ int small_boxes(const Tile& t) { return (t.rows + 31) / 32; }   // 32-row A boxes
 
 struct SharedCtl {
     uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
@@ -274,7 +318,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                 const __grid_constant__ CUtensorMap tmB00, const __grid_constant__ CUtensorMap tmB01,
                 const __grid_constant__ CUtensorMap tmB10, const __grid_constant__ CUtensorMap tmB11,
-                const KParams p) {
+                const __grid_constant__ CUtensorMap tmA0s, const KParams p) {
     constexpr int COLS_PER_TILE = MODE == TC_SWIGLU ? 128 : 256;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -296,6 +340,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
         prefetch_map(&tmA0); prefetch_map(&tmA1);
         prefetch_map(&tmB00); prefetch_map(&tmB01);
         prefetch_map(&tmB10); prefetch_map(&tmB11);
+        if (p.split_grid) prefetch_map(&tmA0s);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -322,7 +367,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
     // CTAs running at the same time read different K ranges of the weights
     // (spreading the traffic over all DRAM channels)
     const int nsplit = (p.partial != nullptr && p.tiles != nullptr) ? p.tiles[p.E + p.has_shared + 1] : 1;
-    const int units = total * nsplit;
+    const Units un = cta_units(p, total, nsplit);
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -332,16 +377,39 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             uint32_t issued_mask = 0, issued_ph = 0;
             bool aborted = false;
             int pre = 0;   // stages of the first unit whose weight tiles were requested before the wait
+            // the unit's tile and K-block range (a split of it with split-K)
+            auto unit_tile = [&](int u, int& kb0, int& kb1) {
+                if (un.small) {
+                    const Tile t = decode_small_tile(p, u);
+                    kb0 = 0; kb1 = t.num_kb;
+                    return t;
+                }
+                const int sp = u % nsplit;
+                const Tile t = decode_tile(p, u / nsplit);
+                kb0 = sp * t.num_kb / nsplit; kb1 = (sp + 1) * t.num_kb / nsplit;
+                return t;
+            };
+            // bytes of one stage: small tiles load only the group's 32-row boxes of A
+            auto stage_tx = [&](const Tile& t) {
+                return un.small ? static_cast<uint32_t>(B_BYTES + small_boxes(t) * 4096) : static_cast<uint32_t>(STAGE_BYTES);
+            };
+            auto load_a = [&](uint32_t sa, const Tile& t, const TileLoads& l, int kb, uint64_t* bar) {
+                if (un.small) {
+                    const int nb = small_boxes(t);
+                    for (int j = 0; j < nb; ++j) tma_load_2d(sa + j * 4096, &tmA0s, bar, kb * BK, t.row0 + 32 * j);
+                } else {
+                    tma_load_2d(sa, l.ma, bar, kb * BK, l.arow);
+                }
+            };
             if (early) {
-                if (static_cast<int>(blockIdx.x) < units) {
-                    const int sp = blockIdx.x % nsplit;
-                    const Tile t = decode_tile(p, blockIdx.x / nsplit);
-                    const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
+                if (un.first < un.count) {
+                    int kb0, kb1;
+                    const Tile t = unit_tile(un.first, kb0, kb1);
                     const TileLoads l = tile_loads<MODE>(p, t, &tmA0, &tmA1, &tmB00, &tmB01, &tmB10, &tmB11);
                     for (int kb = kb0; kb < kb1 && pre < STAGES; ++kb, ++pre) {
                         // every stage is free at the start: no empty-barrier wait
                         const uint32_t sa = smem_u32(smem + pre * STAGE_BYTES);
-                        mbar_arrive_expect_tx(&ctl->full[pre], STAGE_BYTES);
+                        mbar_arrive_expect_tx(&ctl->full[pre], stage_tx(t));
                         tma_load_2d(sa + A_BYTES, l.mlo, &ctl->full[pre], kb * BK, l.brow0);
                         tma_load_2d(sa + A_BYTES + B_HALF_BYTES, l.mhi, &ctl->full[pre], kb * BK, l.brow1);
                         issued_mask |= 1u << pre;
@@ -350,20 +418,19 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                 pdl_wait();
                 pdl_launch();
             }
-            for (int u = blockIdx.x; u < units && !aborted; u += gridDim.x) {
-                const int sp = u % nsplit;
-                const Tile t = decode_tile(p, u / nsplit);
-                const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
+            for (int u = un.first; u < un.count && !aborted; u += un.step) {
+                int kb0, kb1;
+                const Tile t = unit_tile(u, kb0, kb1);
                 const TileLoads l = tile_loads<MODE>(p, t, &tmA0, &tmA1, &tmB00, &tmB01, &tmB10, &tmB11);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-                    if (u == static_cast<int>(blockIdx.x) && kb - kb0 < pre) {
+                    if (u == un.first && kb - kb0 < pre) {
                         // weights already requested: the A rows complete the stage
-                        tma_load_2d(sa, l.ma, &ctl->full[s], kb * BK, l.arow);
+                        load_a(sa, t, l, kb, &ctl->full[s]);
                     } else {
                         if (!wait_bounded(&ctl->empty[s], ph ^ 1u, ctl, p)) { aborted = true; break; }
-                        mbar_arrive_expect_tx(&ctl->full[s], STAGE_BYTES);
-                        tma_load_2d(sa, l.ma, &ctl->full[s], kb * BK, l.arow);
+                        mbar_arrive_expect_tx(&ctl->full[s], stage_tx(t));
+                        load_a(sa, t, l, kb, &ctl->full[s]);
                         tma_load_2d(sa + A_BYTES, l.mlo, &ctl->full[s], kb * BK, l.brow0);
                         tma_load_2d(sa + A_BYTES + B_HALF_BYTES, l.mhi, &ctl->full[s], kb * BK, l.brow1);
                     }
@@ -396,10 +463,21 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             int acc = 0;
             uint32_t aph = 0;
             bool aborted = false, issued_any = false;
-            for (int u = blockIdx.x; u < units && !aborted; u += gridDim.x) {
-                const int sp = u % nsplit;
-                const Tile t = decode_tile(p, u / nsplit);
-                const int kb0 = sp * t.num_kb / nsplit, kb1 = (sp + 1) * t.num_kb / nsplit;
+            for (int u = un.first; u < un.count && !aborted; u += un.step) {
+                int kb0 = 0, kb1;
+                Tile t;
+                if (un.small) {
+                    t = decode_small_tile(p, u);
+                    kb1 = t.num_kb;
+                } else {
+                    const int sp = u % nsplit;
+                    t = decode_tile(p, u / nsplit);
+                    kb0 = sp * t.num_kb / nsplit; kb1 = (sp + 1) * t.num_kb / nsplit;
+                }
+                // operand-swapped small tile: the two 128-row halves of the
+                // weight tile are the M operands, the group's rows (N = 32 per
+                // A box) the N operand; D columns [0, N) and [128, 128 + N)
+                const uint32_t idesc_s = un.small ? make_idesc(BM, 32 * small_boxes(t)) : 0u;
                 if (!wait_bounded(&ctl->tempty[acc], aph ^ 1u, ctl, p)) { aborted = true; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
@@ -409,9 +487,19 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                     const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
                     const uint64_t adesc = sw128_desc(sa);
                     const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+                    if (un.small) {
+                        const uint64_t wlo = bdesc, whi = sw128_desc(sa + A_BYTES + B_HALF_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        tc_mma(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint32_t accum = (kb != kb0 || kk != 0) ? 1u : 0u;
+                            tc_mma(d_tmem, wlo + 2u * kk, adesc + 2u * kk, idesc_s, accum);
+                            tc_mma(d_tmem + 128u, whi + 2u * kk, adesc + 2u * kk, idesc_s, accum);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            tc_mma(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                    }
                     issued_any = true;
                     tc_commit(&ctl->empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -437,9 +525,9 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
         const int r = q * 32 + lane;            // accumulator row of this thread
         int acc = 0;
         uint32_t aph = 0;
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const int sp = u % nsplit;
-            const Tile t = decode_tile(p, u / nsplit);
+        for (int u = un.first; u < un.count; u += un.step) {
+            const int sp = un.small ? 0 : u % nsplit;
+            const Tile t = un.small ? decode_small_tile(p, u) : decode_tile(p, u / nsplit);
             if (!wait_bounded(&ctl->tfull[acc], aph, ctl, p)) break;
             tc_fence_after();
             const int grow = t.m_blk * BM + r;
@@ -449,7 +537,33 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                 static_cast<uint32_t>(acc * ACC_COLS);
             bool released = false;
-            if (MODE != TC_F32OUT && nsplit > 1) {
+            if (MODE != TC_F32OUT && un.small) {
+                // operand-swapped tile: this thread's TMEM lane is output
+                // column m of the tile, its columns are the group's rows
+                __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(p.out[0]);
+                const int ncol = 32 * small_boxes(t);
+                const int col0 = MODE == TC_SWIGLU ? t.n_blk * 128 + r : t.n_blk * 256 + r;
+#pragma unroll 1
+                for (int c = 0; c < ncol; c += 32) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(tb + c, v0);
+                    tmem_ld32(tb + 128 + c, v1);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int n = c + i;
+                        if (n < t.rows) {
+                            __nv_bfloat16* orow_p = outp + (static_cast<size_t>(t.row0) + n) * N;
+                            const float a = __uint_as_float(v0[i]), b = __uint_as_float(v1[i]);
+                            if (MODE == TC_SWIGLU) {
+                                if (col0 < N) orow_p[col0] = __float2bfloat16_rn(silu(a) * b);
+                            } else {
+                                if (col0 < N) orow_p[col0] = __float2bfloat16_rn(a);
+                                if (col0 + 128 < N) orow_p[col0 + 128] = __float2bfloat16_rn(b);
+                            }
+                        }
+                    }
+                }
+            } else if (MODE != TC_F32OUT && nsplit > 1) {
                 // fp32 partial of this split: the raw 256 accumulator columns
                 float* out = p.partial + static_cast<size_t>(sp) * p.partial_stride + orow * p.partial_ld;
 #pragma unroll 1
@@ -947,7 +1061,7 @@ bool encode_map(CUtensorMap* m, const void* base, int rows, int cols, int box_ro
 }
 
 template <int MODE>
-cudaError_t launch_pair_mode(const KParams& kp, const CUtensorMap (&maps)[6], cudaStream_t st) {
+cudaError_t launch_pair_mode(const KParams& kp, const CUtensorMap (&maps)[7], cudaStream_t st) {
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -964,7 +1078,7 @@ cudaError_t launch_pair_mode(const KParams& kp, const CUtensorMap (&maps)[6], cu
 }
 
 template <int MODE>
-cudaError_t launch_mode(const TcArgs& a, const KParams& kp, const CUtensorMap (&maps)[6], cudaStream_t st) {
+cudaError_t launch_mode(const TcArgs& a, const KParams& kp, const CUtensorMap (&maps)[7], cudaStream_t st) {
     static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -977,7 +1091,7 @@ cudaError_t launch_mode(const TcArgs& a, const KParams& kp, const CUtensorMap (&
     int grid = device_sm_count();
     if (grid <= 0) return cudaErrorInvalidDevice;
     return launch_k(tc_grouped_gemm<MODE>, dim3(grid), dim3(NUM_THREADS), (size_t)SMEM_BYTES, st, maps[0], maps[1],
-                    maps[2], maps[3], maps[4], maps[5], kp);
+                    maps[2], maps[3], maps[4], maps[5], maps[6], kp);
 }
 
 }  // namespace
@@ -994,8 +1108,9 @@ bool make_tmap_f32_store(void* m, const float* base, int rows, int cols) {
 
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     if (!get_encode()) return cudaErrorNotSupported;
-    CUtensorMap maps[6];
-    // A maps: [rows, K]; B maps: [total rows, K]. Unused slots reuse slot 0.
+    CUtensorMap maps[7];
+    // A maps: [rows, K]; B maps: [total rows, K]; slot 6: the routed A rows
+    // in 32-row boxes (operand-swapped small tiles). Unused slots reuse slot 0.
     const int has1 = a.has_shared && a.A[1] != nullptr;
     if (!make_map(&maps[0], a.A[0], a.a_rows[0], a.K[0])) return cudaErrorInvalidValue;
     if (!make_map(&maps[1], has1 ? a.A[1] : a.A[0], has1 ? a.a_rows[1] : a.a_rows[0], has1 ? a.K[1] : a.K[0]))
@@ -1011,7 +1126,13 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
         maps[4] = maps[2];
         maps[5] = maps[3];
     }
+    if (a.split_grid) {
+        if (!make_map(&maps[6], a.A[0], a.a_rows[0], a.K[0], 32)) return cudaErrorInvalidValue;
+    } else {
+        maps[6] = maps[0];
+    }
     KParams kp;
+    kp.split_grid = a.split_grid;
     kp.indptr = a.indptr;
     kp.tiles = a.tiles;
     kp.static_rows = a.static_rows;
@@ -1034,9 +1155,10 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     kp.b_before_wait = a.b_before_wait;
     const int cols = tc_out_cols_per_tile(a.mode);
     const bool pair = a.pair != 0;
-    if (pair && (a.mode == TC_F32OUT || a.partial != nullptr || a.ab_out != nullptr || a.ab_out_s != nullptr ||
-                 a.tiles == nullptr))
+    if ((pair || a.split_grid) && (a.mode == TC_F32OUT || a.partial != nullptr || a.ab_out != nullptr ||
+                                   a.ab_out_s != nullptr || a.tiles == nullptr || a.indptr == nullptr))
         return cudaErrorInvalidValue;
+    if (pair && a.split_grid) return cudaErrorInvalidValue;
     for (int kd = 0; kd < 2; ++kd) {
         kp.nt_blk[kd] = ceil_div(a.N[kd] > 0 ? a.N[kd] : 1, cols);
         const long long row_bytes = static_cast<long long>(pair ? PBM : BM) * (a.K[kd] > 0 ? a.K[kd] : 1) * 2;

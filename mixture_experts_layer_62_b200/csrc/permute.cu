@@ -62,6 +62,89 @@ __device__ void build_schedule(const int* rows, int G, int E, int tile_m, int nt
     if (threadIdx.x == 0) tiles[G] = carry;
 }
 
+// CTAs of the small class (the first S of the grid) for one GEMM with the
+// grid split: the S minimising the later of the two classes' end times,
+// with a large tile's K block of MMAs taken as kLargeKbSec and the small
+// tiles as weight streams of kSmallCtaBw per CTA, kSmallHbmShare at most in
+// all (the large class keeps the rest of the memory bandwidth).
+constexpr double kLargeKbSec = 0.44e-6;
+constexpr double kSmallCtaBw = 150e9;
+constexpr double kSmallHbmShare = 4.5e12;
+
+__device__ int choose_small_ctas(double large_kb, double small_bytes, int grid) {
+    if (small_bytes <= 0.0) return 0;
+    if (large_kb <= 0.0) return grid;
+    int best = 1;
+    double best_t = 1e30;
+    for (int S = 1; S < grid; ++S) {
+        const double tl = large_kb * kLargeKbSec / (double)(grid - S);
+        const double bw = fmin((double)S * kSmallCtaBw, kSmallHbmShare);
+        const double ts = small_bytes / bw;
+        const double t = fmax(tl, ts);
+        if (t < best_t) { best_t = t; best = S; }
+    }
+    return best;
+}
+
+// The schedules of GEMM 1/3 and GEMM 2 from the rows per group (rows[E] =
+// T for the shared expert): one class of tiles, or with gs.on the large
+// class (groups of more than kSmallRows rows, the shared expert), the small
+// class and S. Block-wide; ends synchronised.
+__device__ void build_gemm_schedules(int* rows, int G, int E, int tile_m, int nt13, int nt13s, int nt2, int nt2s,
+                                     int32_t* tiles13, int32_t* tiles2, const GridSplit& gs, int* warp_tot,
+                                     int* srows) {
+    if (!gs.on) {
+        build_schedule(rows, G, E, tile_m, nt13, nt13s, tiles13, warp_tot);
+        __syncthreads();
+        build_schedule(rows, G, E, tile_m, nt2, nt2s, tiles2, warp_tot);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            tiles13[G + 2] = 0;
+            tiles2[G + 2] = 0;
+        }
+        return;
+    }
+    // small class: one (operand-swapped) M block per group of 1..kSmallRows rows
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+        const bool small = g < E && rows[g] > 0 && rows[g] <= kSmallRows;
+        srows[g] = small ? rows[g] : 0;
+    }
+    __syncthreads();
+    for (int g = threadIdx.x; g < G; g += blockDim.x)
+        if (srows[g] > 0) rows[g] = 0;   // the large class skips them
+    __syncthreads();
+    build_schedule(rows, G, E, tile_m, nt13, nt13s, tiles13, warp_tot);
+    __syncthreads();
+    build_schedule(rows, G, E, tile_m, nt2, nt2s, tiles2, warp_tot);
+    __syncthreads();
+    build_schedule(srows, G, E, kSmallRows, nt13, nt13s, tiles13 + G + 3, warp_tot);
+    __syncthreads();
+    build_schedule(srows, G, E, kSmallRows, nt2, nt2s, tiles2 + G + 3, warp_tot);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int kb13 = (gs.k13 + 63) / 64, kb2 = (gs.k2 + 63) / 64;
+        const int kb13s = (gs.k13s + 63) / 64, kb2s = (gs.k2s + 63) / 64;
+        double l13 = 0, l2 = 0, s13 = 0, s2 = 0;
+        for (int g = 0; g < G; ++g) {
+            if (rows[g] > 0) {
+                const double mt = (double)((rows[g] + tile_m - 1) / tile_m);
+                l13 += mt * (g < E ? (double)nt13 * kb13 : (double)nt13s * kb13s);
+                l2 += mt * (g < E ? (double)nt2 * kb2 : (double)nt2s * kb2s);
+            }
+            if (srows[g] > 0) {
+                // per K block: the 256 weight rows (32 KB) and the group's 32-row boxes of A
+                const double xb = (double)((srows[g] + 31) / 32) * 4096.0;
+                s13 += (double)nt13 * kb13 * (32768.0 + xb);
+                s2 += (double)nt2 * kb2 * (32768.0 + xb);
+            }
+        }
+        const int f = gs.force_ctas > 0 ? min(gs.force_ctas, gs.grid) : -1;
+        tiles13[G + 2] = f > 0 ? (s13 > 0 ? f : 0) : choose_small_ctas(l13, s13, gs.grid);
+        tiles2[G + 2] = f > 0 ? (s2 > 0 ? f : 0) : choose_small_ctas(l2, s2, gs.grid);
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kScanThreads) scan_kernel(const __grid_constant__ ScanArgs a, int NB) {
     __shared__ int warp_tot[33];
     __shared__ int start[MOE_MAX_E + 1];
@@ -243,9 +326,9 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const __grid_constan
         if (threadIdx.x == 0) rows[E] = a.T;
         __syncthreads();
         const int G = E + a.has_shared;
-        build_schedule(rows, G, E, a.tile_m, a.ntiles13, a.ntiles13_shared, a.tiles13, warp_tot);
-        __syncthreads();
-        build_schedule(rows, G, E, a.tile_m, a.ntiles2, a.ntiles2_shared, a.tiles2, warp_tot);
+        __shared__ int srows[MOE_MAX_E + 1];
+        build_gemm_schedules(rows, G, E, a.tile_m, a.ntiles13, a.ntiles13_shared, a.ntiles2, a.ntiles2_shared,
+                             a.tiles13, a.tiles2, a.gsplit, warp_tot, srows);
         // split factors: with split-K on, every active expert is one M-block,
         // so the host-built table indexed by the active-expert count applies
         int n_active;
@@ -279,11 +362,10 @@ schedule_kernel(const int32_t* __restrict__ indptr, int E, int T, int has_shared
     if (threadIdx.x == 0) rows[E] = T;
     __syncthreads();
     const int G = E + has_shared;
-    build_schedule(rows, G, E, tile_m, nt13, nt13s, tiles13, warp_tot);
-    __syncthreads();
-    build_schedule(rows, G, E, tile_m, nt2, nt2s, tiles2, warp_tot);
     int n_active;
     block_exclusive_scan(threadIdx.x < E && rows[threadIdx.x] > 0 ? 1 : 0, warp_tot, n_active);
+    __shared__ int srows[MOE_MAX_E + 1];
+    build_gemm_schedules(rows, G, E, tile_m, nt13, nt13s, nt2, nt2s, tiles13, tiles2, sp.gsplit, warp_tot, srows);
     if (threadIdx.x == 0) {
         const int n = n_active < kSplitMaxRows ? n_active : kSplitMaxRows;
         tiles13[G + 1] = sp.split_on ? sp.split.s13[n] : 1;
@@ -361,9 +443,17 @@ permute_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ i
         for (int j = 0; j < k; ++j)
             if (spos[q][j] >= 0) dst[nd++] = spos[q][j];
         if (nd == 0) continue;
-        for (int v = v_lo + lane; v < v_hi; v += 32) {
-            uint4 val = src[v];
-            for (int j = 0; j < nd; ++j) xp[(size_t)dst[j] * nvec + v] = val;
+        // four vectors of the row in flight per lane before any is written
+        for (int v0 = v_lo + lane; v0 < v_hi; v0 += 32 * 4) {
+            uint4 val[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (v0 + 32 * u < v_hi) val[u] = src[v0 + 32 * u];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (v0 + 32 * u < v_hi)
+                    for (int j = 0; j < nd; ++j) xp[(size_t)dst[j] * nvec + v0 + 32 * u] = val[u];
+            }
         }
     }
 }
