@@ -223,7 +223,17 @@ def decode_bytes(cfg, st):
     return b
 
 
-def workload_roofline(cfg, workload, stages, st, peaks, peak_src):
+KERNEL_NAMES = {
+    "pair": ("tc_pair_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU, CTA pairs)", "tc_pair_gemm_swiglu"),
+    "grid_split": ("tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU, small groups on their own CTAs)",
+                   "tc_grouped_gemm_swiglu"),
+    "single": ("tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU)", "tc_grouped_gemm_swiglu"),
+    "split_k": ("tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU, split-K)", "tc_grouped_gemm_swiglu"),
+    "simt": ("simt_gemm_kernel<true> (grouped GEMM 1/3 + SwiGLU, CUDA cores)", "simt_gemm_swiglu"),
+}
+
+
+def workload_roofline(cfg, workload, stages, st, peaks, peak_src, variant="single"):
     """Roofline of the dominant kernel, grouped GEMM 1/3 + SwiGLU."""
     rows = st.rows
     up_ms = stages["expert_up"]
@@ -239,11 +249,12 @@ def workload_roofline(cfg, workload, stages, st, peaks, peak_src):
     tflops, gbs = fl / t / 1e12, up_bytes / t / 1e9
     peak_tf, peak_bw = peaks["bf16_tflops"], peaks["hbm_gbs"]
     t_compute, t_memory = fl / (peak_tf * 1e12), up_bytes / (peak_bw * 1e9)
-    common = {"kernel": "tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU)", "ms_per_launch": up_ms,
+    kname, tkey = KERNEL_NAMES[variant]
+    common = {"kernel": kname, "gemm_variant": variant, "ms_per_launch": up_ms,
               "flops_per_launch": fl, "bytes_per_launch": up_bytes,
               "roofline_time_ms": 1e3 * max(t_compute, t_memory),
               "frac_of_roofline_time": max(t_compute, t_memory) / t,
-              "traffic": traffic_for("tc_grouped_gemm_swiglu", workload),
+              "traffic": traffic_for(tkey, workload),
               "down_proj": {"ms_per_launch": down_ms, "tflops": down_flops(cfg, rows) / (down_ms / 1e3) / 1e12}}
     if t_memory > t_compute:
         return {"bound": "hbm", "achieved": gbs, "peak": peak_bw, "unit": "GB/s", "frac": gbs / peak_bw,
@@ -413,7 +424,7 @@ def measure_extra(name, args, moe, dev, stream, flush, peaks, peak_src, weight_c
     ms = total_ms / args.steps
     stages = breakdown(moe, p, cfg, L, dev, stream, flush, iters=max(3, min(10, args.steps)))
     out = {"ms_per_step": ms, "tokens_per_s": cfg["T"] / (ms / 1e3), "T": cfg["T"],
-           "roofline": workload_roofline(cfg, name, stages, st, peaks, peak_src),
+           "roofline": workload_roofline(cfg, name, stages, st, peaks, peak_src, moe.gemm_variant(p)),
            "pass_roofline": pass_roofline(cfg, st, ms, peaks), "stages_ms": stages, "clocks": clocks,
            "routing": {"rows": st.rows, "dropped": st.dropped, "capacity": st.capacity, "l_aux": st.l_aux,
                        "max_over_mean": st.max_over_mean, "experts_touched": touched_experts(st),
@@ -547,7 +558,7 @@ def main():
     nbytes = x.numel() * x.element_size()
 
     peaks, peak_src = load_peaks()
-    roofline = workload_roofline(cfg, args.workload, stages, st, peaks, peak_src)
+    roofline = workload_roofline(cfg, args.workload, stages, st, peaks, peak_src, moe.gemm_variant(p))
     if cfg["T"] <= 64:
         # decode: weight-read bound; the headline figure is HBM bandwidth
         roofline["forward_hbm_gbs"] = decode_bytes(cfg, st) / (ms_per_step / 1e3) / 1e9

@@ -333,6 +333,30 @@ int moe_device_sm_count(void);
  * unaffected. */
 long long moe_set_wait_limit(long long ns);
 
+/* Which grouped-GEMM kernel moe_forward and the expert stages use for p:
+ * MOE_GEMM_SINGLE (one CTA per 128-row tile), MOE_GEMM_PAIR (CTA pairs,
+ * 256-row tiles), MOE_GEMM_GRID_SPLIT (single-CTA tiles, groups of at most
+ * 128 rows as operand-swapped tiles on their own CTAs), MOE_GEMM_SPLIT_K
+ * (decode-sized batches: K split over CTAs), MOE_GEMM_SIMT (fp32, CUDA
+ * cores); a negative MOE_ERR_* code if p is invalid. Host only. */
+#define MOE_GEMM_SINGLE      0
+#define MOE_GEMM_PAIR        1
+#define MOE_GEMM_GRID_SPLIT  2
+#define MOE_GEMM_SPLIT_K     3
+#define MOE_GEMM_SIMT        4
+int moe_gemm_variant(const moe_problem* p);
+
+/* Kernel-selection overrides, read once per process from the environment
+ * (for measurement and tests; results are the same either way, up to the
+ * summation order inside one MMA):
+ *   MOE_CTA_PAIR=0   the grouped GEMMs never use CTA pairs (256-row tiles on
+ *                    two SMs); by default they do when the experts average
+ *                    at least 512 rows (bf16 inference, no split-K).
+ *   MOE_SMALL_CTAS=n with 32 or more experts and fewer than 512 rows per
+ *                    expert on average, the first n CTAs run the groups of
+ *                    at most 128 rows as operand-swapped tiles; n = 0 turns
+ *                    this grid split off; unset, n comes from a cost model. */
+
 #ifdef __cplusplus
 }
 #endif

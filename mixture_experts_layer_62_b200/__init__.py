@@ -77,6 +77,8 @@ def _load():
     lib.moe_workspace_layout.restype = ctypes.c_int
     lib.moe_error_string.argtypes = [ctypes.c_int]
     lib.moe_error_string.restype = ctypes.c_char_p
+    lib.moe_gemm_variant.argtypes = [P]
+    lib.moe_gemm_variant.restype = ctypes.c_int
     lib.moe_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.moe_set_wait_limit.restype = ctypes.c_longlong
     lib.moe_device_sm_count.argtypes = []
@@ -124,6 +126,17 @@ def __getattr__(name):
     if name == "lib":
         return _lib()
     raise AttributeError(name)
+
+
+GEMM_VARIANTS = {0: "single", 1: "pair", 2: "grid_split", 3: "split_k", 4: "simt"}
+
+
+def gemm_variant(p: Problem) -> str:
+    """Name of the grouped-GEMM kernel the library uses for p (moe_gemm_variant)."""
+    v = int(_lib().moe_gemm_variant(ctypes.byref(p)))
+    if v < 0:
+        raise MoEError(-v, "moe_gemm_variant")
+    return GEMM_VARIANTS[v]
 
 
 def set_wait_limit(ns: int) -> int:

@@ -439,6 +439,16 @@ int moe_workspace_layout(const moe_problem* p, moe_workspace_layout_t* out) {
 
 int moe_device_sm_count(void) { return device_sm_count(); }
 
+int moe_gemm_variant(const moe_problem* p) {
+    const int rc = check_problem(p);
+    if (rc != MOE_OK) return -rc;
+    if (p->dtype != MOE_DTYPE_BF16) return MOE_GEMM_SIMT;
+    if (split_allowed(*p)) return MOE_GEMM_SPLIT_K;
+    if (use_pair_tiles(*p)) return MOE_GEMM_PAIR;
+    if (grid_split_of(*p).on) return MOE_GEMM_GRID_SPLIT;
+    return MOE_GEMM_SINGLE;
+}
+
 long long moe_set_wait_limit(long long ns) {
     return g_wait_limit_ns.exchange(ns > 0 ? ns : kDefaultWaitLimitNs);
 }

@@ -169,3 +169,23 @@ def test_binding_refuses_cpu_tensors():
     t = torch.zeros(4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         moe.combine(p, t, t, t, t)
+
+
+def test_gemm_variant_follows_the_shape():
+    # host-side selection only (no launch): CTA pairs for prefill-sized
+    # experts, split-K for decode-sized batches, CUDA cores for fp32
+    from mixture_experts_layer_62_b200 import inputs
+
+    def variant(name, **kw):
+        c = dict(inputs.workload(name), **kw)
+        return moe.gemm_variant(moe.problem(c["T"], c["d"], c["d_ff"], c["E"], c["k"], c["cf"], c["dtype"],
+                                            c["bias_mode"], c["d_ff_shared"], train=kw.get("train", 0)))
+    assert variant("mixtral_prefill") == "pair"
+    assert variant("skewed_capacity") == "pair"
+    assert variant("decode_t1") == "split_k"
+    assert variant("toy_fp32") == "simt"
+    assert variant("mixtral_prefill", T=1000) == "single"          # 250 rows per expert
+    assert variant("mixtral_prefill", d_ff=14336, train=1) == "single"
+    assert variant("deepseek_v3") in ("grid_split", "single")      # grid_split on a GPU (needs the SM count)
+    with pytest.raises(moe.MoEError):
+        moe.gemm_variant(moe.problem(16, 256, 64, 4, 5))            # k > E

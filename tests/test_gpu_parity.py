@@ -445,9 +445,18 @@ def _check_forward(cfg, L_cpu, tokens=None, check_own_routing=True):
         res64 = O.moe_forward(x_np, W_r64, W["W1"], W["W3"], W["W2"], k, cfg["cf"], bias, cfg["bias_mode"],
                               W["Ws1"], W["Ws3"], W["Ws2"], tokens=toks, gate_mode=cfg.get("gate", 0),
                               drop_order=cfg.get("drop", 0), pad=cfg.get("pad") or None)
-        same = far[toks] & (g_idx[toks] == res64.routing.idx[toks]).all(axis=1) \
-            & ((g_pos[toks] >= 0) == (res64.perm.pos[toks] >= 0)).all(axis=1)
-        assert same.mean() >= 0.9, same.mean()
+        # the same experts, kept the same way (slot order may differ where
+        # keys inside the selected set are within rounding of each other: the
+        # output is a sum over slots)
+        def kept_sets(idx, pos):
+            return np.sort(np.where(pos >= 0, idx, -1), axis=1)
+        o_idx, o_pos = res64.routing.idx[toks], res64.perm.pos[toks]
+        same = far[toks] & (np.sort(g_idx[toks], axis=1) == np.sort(o_idx, axis=1)).all(axis=1) \
+            & (kept_sets(g_idx[toks], g_pos[toks]) == kept_sets(o_idx, o_pos)).all(axis=1)
+        # away from near-ties the selections agree everywhere; the kept sets
+        # differ only where another token's flipped near-tie moved a pair across
+        # the capacity boundary
+        assert same[far[toks]].mean() >= 0.9, (same[far[toks]].mean(), far.mean())
         assert_rows_close(got[same], res64.y[same], tol, "oracle on its own fp64 routing")
     return rel
 
