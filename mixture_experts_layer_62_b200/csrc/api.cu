@@ -79,8 +79,8 @@ BwdLayout make_bwd_layout(const moe_problem& p) {
     B.dXp = take(Rmax * d * eb);
     B.dz = take(T * E * 4);
     B.dgate = take(T * k * 4);
-    B.tiles_dh = take((E + 3) * 4);
-    B.tiles_dx = take((E + 3) * 4);
+    B.tiles_dh = take((size_t)schedule_ints(p.E) * 4);
+    B.tiles_dx = take((size_t)schedule_ints(p.E) * 4);
     const bool tc_router = E % 64 == 0;
     B.dwr_part = take(tc_router ? 0 : (size_t)ceil_div((int)T, 128) * d * E * 4);
     B.dz16 = take(tc_router ? T * E * 2 : 0);

@@ -12,6 +12,7 @@ tokens (routing over all tokens), determinism, and stage composition.
 """
 
 import math
+import os
 
 import numpy as np
 import pytest
@@ -589,6 +590,10 @@ def _sample_tokens(pos, indptr, rng, n_random):
                                                ("deepseek_v3", 6, 0), ("mixtral_prefill", 8, 128)])
 def test_forward_full_size(name, n_random, pad):
     cfg = dict(inputs.workload(name), pad=pad)
+    # the kernel each full-size workload exercises
+    want = {"mixtral_prefill": "single" if pad else "pair", "skewed_capacity": "pair", "deepseek_v3": "grid_split"}
+    if os.environ.get("MOE_CTA_PAIR", "1") != "0" and os.environ.get("MOE_SMALL_CTAS", "1") != "0":
+        assert moe.gemm_variant(problem_of(cfg)) == want[name]
     L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=DEV)
     Ld = to_device(L)
     p, out, st, ws = gpu_forward(cfg, Ld)
