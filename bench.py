@@ -446,7 +446,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mixtral_prefill")
     ap.add_argument("--cpu-sample", type=int, default=1024, help="tokens of the timed CPU-oracle sample")
-    ap.add_argument("--ref-sample", type=int, default=64, help="tokens per step of the reference arm")
+    ap.add_argument("--ref-sample", type=int, default=256, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="measure the headline workload only (by default one GPU also measures " +

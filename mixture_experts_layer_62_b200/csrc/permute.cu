@@ -66,9 +66,13 @@ __device__ void build_schedule(const int* rows, int G, int E, int tile_m, int nt
 // grid split: the S minimising the later of the two classes' end times,
 // with a large tile's K block of MMAs taken as kLargeKbSec and the small
 // tiles as weight streams of kSmallCtaBw per CTA, kSmallHbmShare at most in
-// all (the large class keeps the rest of the memory bandwidth).
+// all (the large class keeps the rest of the memory bandwidth). Both rates
+// are measured on B200: a large tile's K block in the Mixtral-shaped GEMM
+// 1/3 (1.44 ms for 3293 K blocks per CTA), and the small class's stream per
+// CTA from a sweep of S on the DeepSeek-shaped layer (about 55 GB/s: four
+// stages in flight per CTA bound it).
 constexpr double kLargeKbSec = 0.44e-6;
-constexpr double kSmallCtaBw = 150e9;
+constexpr double kSmallCtaBw = 55e9;
 constexpr double kSmallHbmShare = 4.5e12;
 
 __device__ int choose_small_ctas(double large_kb, double small_bytes, int grid) {

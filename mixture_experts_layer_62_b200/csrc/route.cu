@@ -402,6 +402,11 @@ __device__ __forceinline__ void unpack8(const RawVec8<float>& r, float (&v)[8]) 
     }
 }
 
+// Rows of W_r a block stages in shared memory at a time, for eight experts:
+// 32 KB of W_r^T.
+template <typename T>
+constexpr int fused_slab() { return 32768 / (kExpPerPass * (int)sizeof(T)); }
+
 template <typename T, int EPL>
 __global__ void __launch_bounds__(kSelWarps * 32)
 route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const float* __restrict__ bias,
@@ -411,9 +416,12 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
     static_assert(EPL <= 2, "fused router: E <= 64");
     constexpr int kTokPerWarp = kChunk / kSelWarps;   // 4
     constexpr int U = sizeof(T) == 2 ? 4 : 2;         // row chunks of x in flight per token
+    constexpr int SLAB = fused_slab<T>();             // rows of W_r per staged slab
     __shared__ int cnt[kMaxSlotCounts];
     __shared__ float ps[kSelWarps][MOE_MAX_E];
     __shared__ float ext[kSelWarps][3];
+    extern __shared__ __align__(16) uint8_t fused_dsm[];
+    T* wt = reinterpret_cast<T*>(fused_dsm);          // [kExpPerPass][SLAB]: W_r^T of the slab
     pdl_wait();
     pdl_launch();
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = MOE_OK;
@@ -425,8 +433,6 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
 
     const int t0 = chunk * kChunk + warp * kTokPerWarp;
     const int nt = max(0, min(kTokPerWarp, Tn - t0));
-    const int nchunk = d / 8;
-    const bool wvec = (E % kExpPerPass) == 0;   // W_r rows start on 16-byte boundaries
     float zt[kTokPerWarp][EPL];
 #pragma unroll
     for (int q = 0; q < kTokPerWarp; ++q)
@@ -438,43 +444,52 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
         for (int q = 0; q < kTokPerWarp; ++q)
 #pragma unroll
             for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = 0.f;
-        for (int cb = lane; cb < nchunk; cb += 32 * U) {
-            RawVec8<T> xr[U][kTokPerWarp];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = cb + 32 * u;
-#pragma unroll
-                for (int q = 0; q < kTokPerWarp; ++q) {
-                    if (q < nt && c < nchunk) {
-                        raw_load8(x + (size_t)(t0 + q) * d + (size_t)c * 8, xr[u][q]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < (sizeof(T) == 2 ? 1 : 2); ++i) xr[u][q].v[i] = make_uint4(0, 0, 0, 0);
-                    }
-                }
+        for (int d0 = 0; d0 < d; d0 += SLAB) {
+            const int ns = min(SLAB, d - d0);
+            // stage W_r^T [e0 .. e0 + 7][d0 .. d0 + ns) (zeros past E): reads
+            // of W_r follow its rows, writes go to the transposed slab
+            __syncthreads();
+            for (int i = threadIdx.x; i < ns * kExpPerPass; i += blockDim.x) {
+                const int r = i / kExpPerPass, e = i % kExpPerPass;
+                wt[e * SLAB + r] = e0 + e < E ? W_r[(size_t)(d0 + r) * E + e0 + e] : T(0.f);
             }
+            __syncthreads();
+            // lane l takes the slab's 8-element chunks l, l + 32, ...: x from
+            // global memory (U chunks of each token in flight), the weights of
+            // the chunk's 8 input features from the staged slab
+            const int nchunk = ns / 8;
+            for (int cb = lane; cb < nchunk; cb += 32 * U) {
+                RawVec8<T> xr[U][kTokPerWarp];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = cb + 32 * u;
-                if (c < nchunk) {
-                    float xv[kTokPerWarp][8];
+                for (int u = 0; u < U; ++u) {
+                    const int c = cb + 32 * u;
 #pragma unroll
-                    for (int q = 0; q < kTokPerWarp; ++q) unpack8(xr[u][q], xv[q]);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        // weights of input feature 8c + j for experts e0 .. e0 + 7
-                        const T* wrow = W_r + (size_t)(c * 8 + j) * E + e0;
-                        float wv[kExpPerPass];
-                        if (wvec) {
-                            load8(wrow, wv);
+                    for (int q = 0; q < kTokPerWarp; ++q) {
+                        if (q < nt && c < nchunk) {
+                            raw_load8(x + (size_t)(t0 + q) * d + (size_t)d0 + (size_t)c * 8, xr[u][q]);
                         } else {
 #pragma unroll
-                            for (int e = 0; e < kExpPerPass; ++e) wv[e] = e0 + e < E ? float(wrow[e]) : 0.f;
+                            for (int i = 0; i < (sizeof(T) == 2 ? 1 : 2); ++i)
+                                xr[u][q].v[i] = make_uint4(0, 0, 0, 0);
                         }
+                    }
+                }
 #pragma unroll
-                        for (int q = 0; q < kTokPerWarp; ++q)
+                for (int u = 0; u < U; ++u) {
+                    const int c = cb + 32 * u;
+                    if (c < nchunk) {
+                        float xv[kTokPerWarp][8];
 #pragma unroll
-                            for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = fmaf(xv[q][j], wv[e], acc[q][e]);
+                        for (int q = 0; q < kTokPerWarp; ++q) unpack8(xr[u][q], xv[q]);
+#pragma unroll
+                        for (int e = 0; e < kExpPerPass; ++e) {
+                            float wv[8];
+                            load8(wt + e * SLAB + c * 8, wv);
+#pragma unroll
+                            for (int q = 0; q < kTokPerWarp; ++q)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) acc[q][e] = fmaf(xv[q][j], wv[j], acc[q][e]);
+                        }
                     }
                 }
             }
@@ -530,15 +545,30 @@ cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const 
     const int NB = ceil_div(T, kChunk);
     if (NB == 0) return cudaSuccess;
     dim3 grid(NB), block(kSelWarps * 32);
-#define MOE_FUSED(TYPE, EPLV)                                                                                     \
-    return launch_k(route_fused_kernel<TYPE, EPLV>, grid, block, 0, st, (const TYPE*)x, (const TYPE*)W_r, bias,   \
-                    bias_mode, gate_mode, kk, T, d, E, k, logits, idx, gate, blockcnt, blockpsum, blockextra, status)
+    // the staged W_r slab (32 KB) is dynamic shared memory beside the
+    // selection's static arrays: above the default 48 KB, so opted in once
+    // per device and variant
+    static bool attr_set[64][4] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+#define MOE_FUSED(TYPE, EPLV, SLOT)                                                                                  \
+    do {                                                                                                             \
+        if (!attr_set[dev][SLOT]) {                                                                                  \
+            cudaError_t e_ = cudaFuncSetAttribute(route_fused_kernel<TYPE, EPLV>,                                    \
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 32768);               \
+            if (e_ != cudaSuccess) return e_;                                                                        \
+            attr_set[dev][SLOT] = true;                                                                              \
+        }                                                                                                            \
+        return launch_k(route_fused_kernel<TYPE, EPLV>, grid, block, 32768, st, (const TYPE*)x, (const TYPE*)W_r,   \
+                        bias, bias_mode, gate_mode, kk, T, d, E, k, logits, idx, gate, blockcnt, blockpsum,         \
+                        blockextra, status);                                                                         \
+    } while (0)
     if (dtype == MOE_DTYPE_BF16) {
-        if (E <= 32) MOE_FUSED(__nv_bfloat16, 1);
-        MOE_FUSED(__nv_bfloat16, 2);
+        if (E <= 32) MOE_FUSED(__nv_bfloat16, 1, 0);
+        MOE_FUSED(__nv_bfloat16, 2, 1);
     }
-    if (E <= 32) MOE_FUSED(float, 1);
-    MOE_FUSED(float, 2);
+    if (E <= 32) MOE_FUSED(float, 1, 2);
+    MOE_FUSED(float, 2, 3);
 #undef MOE_FUSED
 }
 
