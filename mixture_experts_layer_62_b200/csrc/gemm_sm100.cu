@@ -779,6 +779,77 @@ __device__ __forceinline__ void pair_store_row(const KParams& p, const Tile& t, 
     }
 }
 
+// Epilogue of a half-width tail tile (N = 128 pair MMA over half of each
+// CTA's B rows): accumulator columns [0, 64) come from rank 0's B rows
+// [64 h, 64 h + 64), columns [64, 128) from rank 1's. SWIGLU: gate and up of
+// the 64 output columns [n_blk 128 + 64 h, + 64); PLAIN: output columns
+// n_blk 256 + 64 h + [0, 64) and n_blk 256 + 128 + 64 h + [0, 64).
+template <int MODE>
+__device__ __forceinline__ void pair_store_half_row(const KParams& p, const Tile& t, uint32_t tb, bool valid,
+                                                    size_t orow, int half) {
+    const int N = p.N[t.kind];
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[t.kind]) + orow * N;
+#pragma unroll 1
+    for (int c = 0; c < 64; c += 32) {
+        uint32_t lo[32], hi[32];
+        tmem_ld32(tb + c, lo);
+        tmem_ld32(tb + 64 + c, hi);
+        if (!valid) continue;
+        uint32_t pk_lo[16], pk_hi[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float a0 = __uint_as_float(lo[2 * i]), a1 = __uint_as_float(lo[2 * i + 1]);
+            const float b0 = __uint_as_float(hi[2 * i]), b1 = __uint_as_float(hi[2 * i + 1]);
+            if (MODE == TC_SWIGLU) {
+                pk_lo[i] = pack_bf16(silu(a0) * b0, silu(a1) * b1);
+            } else {
+                pk_lo[i] = pack_bf16(a0, a1);
+                pk_hi[i] = pack_bf16(b0, b1);
+            }
+        }
+        if (MODE == TC_SWIGLU) {
+            const int col = t.n_blk * 128 + 64 * half + c;
+            if (col < N) {
+                uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk_lo[4 * i], pk_lo[4 * i + 1], pk_lo[4 * i + 2], pk_lo[4 * i + 3]);
+            }
+        } else {
+            const int col0 = t.n_blk * 256 + 64 * half + c, col1 = col0 + 128;
+            if (col0 < N) {
+                uint4* dst = reinterpret_cast<uint4*>(out + col0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk_lo[4 * i], pk_lo[4 * i + 1], pk_lo[4 * i + 2], pk_lo[4 * i + 3]);
+            }
+            if (col1 < N) {
+                uint4* dst = reinterpret_cast<uint4*>(out + col1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk_hi[4 * i], pk_hi[4 * i + 1], pk_hi[4 * i + 2], pk_hi[4 * i + 3]);
+            }
+        }
+    }
+}
+
+// Work items of the pair kernel: the tiles that fill whole waves of the
+// grid, then the remaining (tail) tiles as two half-width items each, so the
+// last wave is as short as a half tile. Item v -> tile, and half (-1: whole).
+struct PairWork {
+    int full, items;
+};
+__device__ __forceinline__ PairWork pair_work(int units, int nclusters) {
+    PairWork w;
+    w.full = (units / nclusters) * nclusters;
+    const int tail = units - w.full;
+    w.items = (tail > 0 && 2 * tail <= nclusters) ? w.full + 2 * tail : units;
+    if (w.items == units) w.full = units;
+    return w;
+}
+__device__ __forceinline__ int pair_item_tile(const PairWork& w, int v, int& half) {
+    if (v < w.full) { half = -1; return v; }
+    half = (v - w.full) & 1;
+    return w.full + ((v - w.full) >> 1);
+}
+
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -827,6 +898,7 @@ tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ C
         pdl_launch();
     }
     const int units = p.tiles[p.E + p.has_shared];
+    const PairWork work = pair_work(units, nclusters);
 
     if (warp == 0) {
         // ---------------- TMA producer (both CTAs) ----------------
@@ -844,8 +916,9 @@ tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ C
             };
             auto full_of = [&](int st) { return mapa_shared(smem_u32(&ctl->full[st]), 0u); };
             if (early) {
-                if (cluster < units) {
-                    const Tile t = decode_tile_m<PBM>(p, cluster);
+                if (cluster < work.items) {
+                    int hf;
+                    const Tile t = decode_tile_m<PBM>(p, pair_item_tile(work, cluster, hf));
                     const int brow = b_row(t);
                     for (int kb = 0; kb < t.num_kb && pre < P_STAGES; ++kb, ++pre) {
                         const uint32_t sa = smem_u32(smem + pre * P_STAGE_BYTES);
@@ -859,8 +932,9 @@ tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ C
                 pdl_wait();
                 pdl_launch();
             }
-            for (int u = cluster; u < units && !aborted; u += nclusters) {
-                const Tile t = decode_tile_m<PBM>(p, u);
+            for (int u = cluster; u < work.items && !aborted; u += nclusters) {
+                int hf;
+                const Tile t = decode_tile_m<PBM>(p, pair_item_tile(work, u, hf));
                 const CUtensorMap* ma = t.kind ? &tmA1 : &tmA0;
                 const int arow = t.row0 + t.m_blk * PBM + static_cast<int>(rank) * BM;
                 const int brow = b_row(t);
@@ -910,8 +984,13 @@ tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ C
             int acc = 0;
             uint32_t aph = 0;
             bool aborted = false, issued_any = false;
-            for (int u = cluster; u < units && !aborted; u += nclusters) {
-                const Tile t = decode_tile_m<PBM>(p, u);
+            constexpr uint32_t idesc_half = make_idesc(PBM, 128);
+            for (int u = cluster; u < work.items && !aborted; u += nclusters) {
+                int hf;
+                const Tile t = decode_tile_m<PBM>(p, pair_item_tile(work, u, hf));
+                // a half-width item multiplies half of each CTA's B rows (N = 128)
+                const uint32_t id = hf < 0 ? idesc : idesc_half;
+                const uint32_t boff = hf > 0 ? 64u * 128u : 0u;
                 if (!pair_wait(&ctl->tempty[acc], aph ^ 1u, ctl, peer_abort, p)) { aborted = true; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
@@ -920,10 +999,10 @@ tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ C
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + s * P_STAGE_BYTES);
                     const uint64_t adesc = sw128_desc(sa);
-                    const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+                    const uint64_t bdesc = sw128_desc(sa + A_BYTES + boff);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        tc_mma_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma_pair(d_tmem, adesc + 2u * kk, bdesc + 2u * kk, id, (kb | kk) != 0 ? 1u : 0u);
                     issued_any = true;
                     tc_commit_pair_mc(&ctl->empty[s], 0x3);
                     if (++s == P_STAGES) { s = 0; ph ^= 1u; }
@@ -952,14 +1031,16 @@ tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ C
                                            mapa_shared(smem_u32(&ctl->tempty[1]), 0u)};
         int acc = 0;
         uint32_t aph = 0;
-        for (int u = cluster; u < units; u += nclusters) {
-            const Tile t = decode_tile_m<PBM>(p, u);
+        for (int u = cluster; u < work.items; u += nclusters) {
+            int hf;
+            const Tile t = decode_tile_m<PBM>(p, pair_item_tile(work, u, hf));
             if (!pair_wait(&ctl->tfull[acc], aph, ctl, peer_abort, p)) break;
             tc_fence_after();
             const int grow = t.m_blk * PBM + r;
             const size_t orow = static_cast<size_t>(t.row0) + static_cast<size_t>(grow);
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_COLS);
-            pair_store_row<MODE>(p, t, tb, grow < t.rows, orow);
+            if (hf < 0) pair_store_row<MODE>(p, t, tb, grow < t.rows, orow);
+            else pair_store_half_row<MODE>(p, t, tb, grow < t.rows, orow, hf);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
