@@ -446,12 +446,39 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
             for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = 0.f;
         for (int d0 = 0; d0 < d; d0 += SLAB) {
             const int ns = min(SLAB, d - d0);
-            // stage W_r^T [e0 .. e0 + 7][d0 .. d0 + ns) (zeros past E): reads
-            // of W_r follow its rows, writes go to the transposed slab
+            // stage W_r^T [e0 .. e0 + 7][d0 .. d0 + ns) (zeros past E). The rows
+            // [d0, d0 + ns) of W_r are one contiguous run of ns E elements: every
+            // thread requests eight 8-element vectors of it before it writes
+            // any, transposed, into the slab
             __syncthreads();
-            for (int i = threadIdx.x; i < ns * kExpPerPass; i += blockDim.x) {
-                const int r = i / kExpPerPass, e = i % kExpPerPass;
-                wt[e * SLAB + r] = e0 + e < E ? W_r[(size_t)(d0 + r) * E + e0 + e] : T(0.f);
+            if (e0 + kExpPerPass > E) {
+                for (int i = threadIdx.x; i < kExpPerPass * ns; i += blockDim.x) wt[(i / ns) * SLAB + i % ns] = T(0.f);
+                __syncthreads();
+            }
+            {
+                const T* src = W_r + (size_t)d0 * E;
+                const int ng = ns * E / 8;
+                for (int g0 = threadIdx.x; g0 < ng; g0 += blockDim.x * 8) {
+                    RawVec8<T> wr[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int g = g0 + (int)blockDim.x * j;
+                        if (g < ng) raw_load8(src + (size_t)g * 8, wr[j]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int g = g0 + (int)blockDim.x * j;
+                        if (g < ng) {
+                            float v[8];
+                            unpack8(wr[j], v);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int idx = g * 8 + i, r = idx / E, e = idx - r * E - e0;
+                                if (e >= 0 && e < kExpPerPass) wt[e * SLAB + r] = T(v[i]);
+                            }
+                        }
+                    }
+                }
             }
             __syncthreads();
             // lane l takes the slab's 8-element chunks l, l + 32, ...: x from
