@@ -7,6 +7,7 @@
 // 04" §2.3.3c (bias added to the softmax score). Router arithmetic is fp32
 // ("Lecture 21 · LLM: Mixture-of-Experts" §7.1: the router runs in fp32).
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace moe {
 
@@ -402,10 +403,15 @@ __device__ __forceinline__ void unpack8(const RawVec8<float>& r, float (&v)[8]) 
     }
 }
 
-// Rows of W_r a block stages in shared memory at a time, for eight experts:
-// 32 KB of W_r^T.
+// Rows of W_r (input features) a block stages at a time: 4 KB of x per token
+// for the chunk's 32 tokens (128 KB; a whole Mixtral-sized row block would
+// not fit), and W_r^T of those rows for eight experts (32 KB for bf16).
 template <typename T>
-constexpr int fused_slab() { return 32768 / (kExpPerPass * (int)sizeof(T)); }
+constexpr int fused_slab() { return 4096 / (int)sizeof(T); }
+template <typename T>
+constexpr size_t fused_smem_bytes() {
+    return (size_t)kChunk * fused_slab<T>() * sizeof(T) + (size_t)kExpPerPass * fused_slab<T>() * sizeof(T) + 64;
+}
 
 template <typename T, int EPL>
 __global__ void __launch_bounds__(kSelWarps * 32)
@@ -415,29 +421,36 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
                    float* __restrict__ blockpsum, float* __restrict__ blockextra, int32_t* __restrict__ status) {
     static_assert(EPL <= 2, "fused router: E <= 64");
     constexpr int kTokPerWarp = kChunk / kSelWarps;   // 4
-    constexpr int U = sizeof(T) == 2 ? 4 : 2;         // row chunks of x in flight per token
-    constexpr int SLAB = fused_slab<T>();             // rows of W_r per staged slab
+    constexpr int SLAB = fused_slab<T>();             // rows of W_r (columns of x) per slab
     __shared__ int cnt[kMaxSlotCounts];
     __shared__ float ps[kSelWarps][MOE_MAX_E];
     __shared__ float ext[kSelWarps][3];
-    extern __shared__ __align__(16) uint8_t fused_dsm[];
-    T* wt = reinterpret_cast<T*>(fused_dsm);          // [kExpPerPass][SLAB]: W_r^T of the slab
+    extern __shared__ __align__(128) uint8_t fused_dsm[];
+    T* xs = reinterpret_cast<T*>(fused_dsm);                      // [kChunk][SLAB]: x of the slab
+    T* wt = xs + (size_t)kChunk * SLAB;                           // [kExpPerPass][SLAB]: W_r^T of the slab
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(wt + (size_t)kExpPerPass * SLAB);
     pdl_wait();
     pdl_launch();
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = MOE_OK;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunk = blockIdx.x, NB = gridDim.x;
     for (int e = threadIdx.x; e < E * kk; e += blockDim.x) cnt[e] = 0;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(xbar, 1);
+        tc::fence_mbar_init();
+    }
     SelAcc<EPL> a;
     sel_init(a, bias, bias_mode, E, lane);
-
-    const int t0 = chunk * kChunk + warp * kTokPerWarp;
-    const int nt = max(0, min(kTokPerWarp, Tn - t0));
+    const int c0tok = chunk * kChunk;
+    const int ntok = min(kChunk, Tn - c0tok);                     // tokens of the block
+    const int q0 = warp * kTokPerWarp;                            // the warp's first token in the block
+    const int nt = max(0, min(kTokPerWarp, ntok - q0));
     float zt[kTokPerWarp][EPL];
 #pragma unroll
     for (int q = 0; q < kTokPerWarp; ++q)
 #pragma unroll
         for (int i = 0; i < EPL; ++i) zt[q][i] = -INFINITY;
+    uint32_t xph = 0;
     for (int e0 = 0; e0 < E; e0 += kExpPerPass) {
         float acc[kTokPerWarp][kExpPerPass];
 #pragma unroll
@@ -446,15 +459,23 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
             for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = 0.f;
         for (int d0 = 0; d0 < d; d0 += SLAB) {
             const int ns = min(SLAB, d - d0);
-            // stage W_r^T [e0 .. e0 + 7][d0 .. d0 + ns) (zeros past E). The rows
-            // [d0, d0 + ns) of W_r are one contiguous run of ns E elements: every
-            // thread requests eight 8-element vectors of it before it writes
-            // any, transposed, into the slab
-            __syncthreads();
-            if (e0 + kExpPerPass > E) {
-                for (int i = threadIdx.x; i < kExpPerPass * ns; i += blockDim.x) wt[(i / ns) * SLAB + i % ns] = T(0.f);
-                __syncthreads();
+            __syncthreads();   // the previous slab is consumed (and the barrier initialised)
+            // x of the block's tokens, columns [d0, d0 + ns): one bulk copy per
+            // token row into the slab
+            if (threadIdx.x == 0) {
+                tc::fence_proxy_async_smem();   // the slab's earlier generic reads precede the copies
+                tc::mbar_arrive_expect_tx(xbar, (uint32_t)(ntok * ns * (int)sizeof(T)));
+                for (int q = 0; q < ntok; ++q)
+                    tc::bulk_load(tc::smem_u32(xs + (size_t)q * SLAB), x + (size_t)(c0tok + q) * d + d0,
+                                  (uint32_t)(ns * (int)sizeof(T)), xbar);
             }
+            // W_r^T [e0 .. e0 + 7][d0 .. d0 + ns) (zeros past E): the rows
+            // [d0, d0 + ns) of W_r are one contiguous run of ns E elements,
+            // requested as 16-byte vectors, eight per thread, before any is
+            // written, transposed, into the slab
+            if (e0 + kExpPerPass > E)
+                for (int i = threadIdx.x; i < kExpPerPass * ns; i += blockDim.x) wt[(i / ns) * SLAB + i % ns] = T(0.f);
+            __syncthreads();
             {
                 const T* src = W_r + (size_t)d0 * E;
                 const int ng = ns * E / 8;
@@ -480,44 +501,43 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
                     }
                 }
             }
-            __syncthreads();
-            // lane l takes the slab's 8-element chunks l, l + 32, ...: x from
-            // global memory (U chunks of each token in flight), the weights of
-            // the chunk's 8 input features from the staged slab
+            __syncthreads();   // W_r^T slab written
+            // the x slab has landed (bulk copies of this block's own rows, which
+            // complete on their own; the wait is still bounded)
+            if (!tc::mbar_try_wait(xbar, xph)) {
+                const uint64_t t0 = tc::global_timer_ns();
+                while (!tc::mbar_try_wait(xbar, xph)) {
+                    if (tc::global_timer_ns() - t0 > static_cast<uint64_t>(kDrainLimitNs)) {
+                        if (status != nullptr) atomicExch(status, MOE_ERR_TIMEOUT);
+                        break;
+                    }
+                }
+            }
+            xph ^= 1u;
+            // lane l takes the slab's 8-element chunks l, l + 32, ...: the four
+            // tokens' x and the eight experts' weights of the chunk's 8 input
+            // features, all from shared memory
             const int nchunk = ns / 8;
-            for (int cb = lane; cb < nchunk; cb += 32 * U) {
-                RawVec8<T> xr[U][kTokPerWarp];
+#pragma unroll 1
+            for (int c = lane; c < nchunk; c += 32) {
+                float xv[kTokPerWarp][8];
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int c = cb + 32 * u;
+                for (int q = 0; q < kTokPerWarp; ++q) {
+                    if (q < nt) {
+                        load8(xs + (size_t)(q0 + q) * SLAB + c * 8, xv[q]);
+                    } else {
 #pragma unroll
-                    for (int q = 0; q < kTokPerWarp; ++q) {
-                        if (q < nt && c < nchunk) {
-                            raw_load8(x + (size_t)(t0 + q) * d + (size_t)d0 + (size_t)c * 8, xr[u][q]);
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < (sizeof(T) == 2 ? 1 : 2); ++i)
-                                xr[u][q].v[i] = make_uint4(0, 0, 0, 0);
-                        }
+                        for (int j = 0; j < 8; ++j) xv[q][j] = 0.f;
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int c = cb + 32 * u;
-                    if (c < nchunk) {
-                        float xv[kTokPerWarp][8];
+                for (int e = 0; e < kExpPerPass; ++e) {
+                    float wv[8];
+                    load8(wt + e * SLAB + c * 8, wv);
 #pragma unroll
-                        for (int q = 0; q < kTokPerWarp; ++q) unpack8(xr[u][q], xv[q]);
+                    for (int q = 0; q < kTokPerWarp; ++q)
 #pragma unroll
-                        for (int e = 0; e < kExpPerPass; ++e) {
-                            float wv[8];
-                            load8(wt + e * SLAB + c * 8, wv);
-#pragma unroll
-                            for (int q = 0; q < kTokPerWarp; ++q)
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) acc[q][e] = fmaf(xv[q][j], wv[j], acc[q][e]);
-                        }
-                    }
+                        for (int j = 0; j < 8; ++j) acc[q][e] = fmaf(xv[q][j], wv[j], acc[q][e]);
                 }
             }
         }
@@ -549,7 +569,7 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
 #pragma unroll
     for (int q = 0; q < kTokPerWarp; ++q) {
         if (q < nt) {
-            const int t = t0 + q;
+            const int t = c0tok + q0 + q;
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const int e = lane + 32 * i;
@@ -572,9 +592,8 @@ cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const 
     const int NB = ceil_div(T, kChunk);
     if (NB == 0) return cudaSuccess;
     dim3 grid(NB), block(kSelWarps * 32);
-    // the staged W_r slab (32 KB) is dynamic shared memory beside the
-    // selection's static arrays: above the default 48 KB, so opted in once
-    // per device and variant
+    // the staged x and W_r slabs (160 KB) are dynamic shared memory beside
+    // the selection's static arrays: opted in once per device and variant
     static bool attr_set[64][4] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -582,11 +601,13 @@ cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const 
     do {                                                                                                             \
         if (!attr_set[dev][SLOT]) {                                                                                  \
             cudaError_t e_ = cudaFuncSetAttribute(route_fused_kernel<TYPE, EPLV>,                                    \
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 32768);               \
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,                       \
+                                                  (int)fused_smem_bytes<TYPE>());                                    \
             if (e_ != cudaSuccess) return e_;                                                                        \
             attr_set[dev][SLOT] = true;                                                                              \
         }                                                                                                            \
-        return launch_k(route_fused_kernel<TYPE, EPLV>, grid, block, 32768, st, (const TYPE*)x, (const TYPE*)W_r,   \
+        return launch_k(route_fused_kernel<TYPE, EPLV>, grid, block, fused_smem_bytes<TYPE>(), st, (const TYPE*)x,  \
+                        (const TYPE*)W_r,                                                                            \
                         bias, bias_mode, gate_mode, kk, T, d, E, k, logits, idx, gate, blockcnt, blockpsum,         \
                         blockextra, status);                                                                         \
     } while (0)
