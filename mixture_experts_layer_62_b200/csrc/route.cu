@@ -187,7 +187,7 @@ __device__ __forceinline__ void sel_init(SelAcc<EPL>& a, const float* __restrict
 
 // One token t whose logits the warp holds (lane l: experts l + 32 i in
 // zin[i]): softmax, statistics, key, top-k, gates, and the chunk's counts.
-template <int EPL>
+template <int EPL, bool COMPACT = false>
 __device__ __forceinline__ void sel_token(const float (&zin)[EPL], int t, int bias_mode, int gate_mode, int kk,
                                           int E, int k, int lane, SelAcc<EPL>& a, int* cnt,
                                           int32_t* __restrict__ idx_out, float* __restrict__ gate_out) {
@@ -248,56 +248,71 @@ __device__ __forceinline__ void sel_token(const float (&zin)[EPL], int t, int bi
                : bias_mode == MOE_BIAS_LOGIT ? z[i] + a.b[i]
                : p + a.b[i];
     }
-    // top-k: k rounds of a warp arg-max over (key desc, index asc)
+    // top-k: k rounds of a warp arg-max over (key desc, index asc); the
+    // compact form keeps the rounds a loop (small code for kernels that run
+    // the selection beside other work), the other unrolls them
     unsigned taken = 0;
     float zsel[MOE_MAX_K];
     int esel[MOE_MAX_K];
+    auto round = [&](int j) {
+        float bk = -INFINITY, bz = 0.f;
+        int be = 0x7fffffff;
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j) {
-        if (j < k) {
-            float bk = -INFINITY, bz = 0.f;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) {
-                bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
-                if (ok && (key[i] > bk || be == 0x7fffffff)) {
-                    bk = key[i]; be = lane + 32 * i; bz = z[i];
-                }
+        for (int i = 0; i < EPL; ++i) {
+            bool ok = ((valid >> i) & 1u) && !((taken >> i) & 1u);
+            if (ok && (key[i] > bk || be == 0x7fffffff)) {
+                bk = key[i]; be = lane + 32 * i; bz = z[i];
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
-                int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-                bool better = (oe != 0x7fffffff) &&
-                              (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
-                if (better) { bk = ok_; be = oe; bz = oz; }
-            }
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            zsel[j] = bz;
-            esel[j] = be;
         }
-    }
-    // gates: softmax over the selected raw logits, slot order
-    float zm = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) zm = fmaxf(zm, zsel[j]);
-    float gs = 0.f, ge[MOE_MAX_K];
+        for (int o = 16; o > 0; o >>= 1) {
+            float ok_ = __shfl_xor_sync(0xffffffffu, bk, o);
+            int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            float oz = __shfl_xor_sync(0xffffffffu, bz, o);
+            bool better = (oe != 0x7fffffff) &&
+                          (be == 0x7fffffff || ok_ > bk || (ok_ == bk && oe < be));
+            if (better) { bk = ok_; be = oe; bz = oz; }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        zsel[j] = bz;
+        esel[j] = be;
+    };
+    float zm = -INFINITY, gs = 0.f, ge[MOE_MAX_K];
+    if constexpr (COMPACT) {
+#pragma unroll 1
+        for (int j = 0; j < k; ++j) round(j);
+        // gates: softmax over the selected raw logits, slot order
+#pragma unroll 1
+        for (int j = 0; j < k; ++j) zm = fmaxf(zm, zsel[j]);
+#pragma unroll 1
+        for (int j = 0; j < k; ++j) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
+    } else {
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_K; ++j) {
-        if (j < k) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
+        for (int j = 0; j < MOE_MAX_K; ++j)
+            if (j < k) round(j);
+        // gates: softmax over the selected raw logits, slot order
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) if (j < k) zm = fmaxf(zm, zsel[j]);
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_K; ++j) {
+            if (j < k) { ge[j] = expf(zsel[j] - zm); gs += ge[j]; }
+        }
     }
     const float inv_g = 1.f / gs;
     if (lane == 0) {
+        auto emit = [&](int j) {
+            idx_out[(size_t)t * k + j] = esel[j];
+            // selected softmax, or the full-softmax probability (Switch gate)
+            gate_out[(size_t)t * k + j] = gate_mode == MOE_GATE_FULL ? expf(zsel[j] - m) * inv_s : ge[j] * inv_g;
+            atomicAdd(&cnt[esel[j] * kk + (kk > 1 ? j : 0)], 1);   // integer: order does not matter
+        };
+        if constexpr (COMPACT) {
+#pragma unroll 1
+            for (int j = 0; j < k; ++j) emit(j);
+        } else {
 #pragma unroll
-        for (int j = 0; j < MOE_MAX_K; ++j) {
-            if (j < k) {
-                idx_out[(size_t)t * k + j] = esel[j];
-                // selected softmax, or the full-softmax probability (Switch gate)
-                gate_out[(size_t)t * k + j] =
-                    gate_mode == MOE_GATE_FULL ? expf(zsel[j] - m) * inv_s : ge[j] * inv_g;
-                atomicAdd(&cnt[esel[j] * kk + (kk > 1 ? j : 0)], 1);   // integer: order does not matter
-            }
+            for (int j = 0; j < MOE_MAX_K; ++j)
+                if (j < k) emit(j);
         }
     }
 }
@@ -486,13 +501,21 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
                         const int g = g0 + (int)blockDim.x * j;
                         if (g < ng) raw_load8(src + (size_t)g * 8, wr[j]);
                     }
-#pragma unroll
+#pragma unroll 1
                     for (int j = 0; j < 8; ++j) {
                         const int g = g0 + (int)blockDim.x * j;
-                        if (g < ng) {
-                            float v[8];
-                            unpack8(wr[j], v);
+                        if (g >= ng) break;
+                        float v[8];
+                        unpack8(wr[j], v);
+                        if (E % kExpPerPass == 0) {
+                            // the group is experts [eb, eb + 8) of one input feature r
+                            const int r = (g * 8) / E, eb = g * 8 - r * E;
+                            if (eb == e0) {
 #pragma unroll
+                                for (int i = 0; i < 8; ++i) wt[i * SLAB + r] = T(v[i]);
+                            }
+                        } else {
+#pragma unroll 1
                             for (int i = 0; i < 8; ++i) {
                                 const int idx = g * 8 + i, r = idx / E, e = idx - r * E - e0;
                                 if (e >= 0 && e < kExpPerPass) wt[e * SLAB + r] = T(v[i]);
@@ -575,7 +598,7 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
                 const int e = lane + 32 * i;
                 if (e < E) logits[(size_t)t * E + e] = zt[q][i];
             }
-            sel_token<EPL>(zt[q], t, bias_mode, gate_mode, kk, E, k, lane, a, cnt, idx_out, gate_out);
+            sel_token<EPL, true>(zt[q], t, bias_mode, gate_mode, kk, E, k, lane, a, cnt, idx_out, gate_out);
         }
     }
     sel_finish<EPL>(a, chunk, NB, E, kk, warp, lane, cnt, ps, ext, blockcnt, blockpsum, blockextra);
