@@ -336,7 +336,8 @@ long long moe_set_wait_limit(long long ns);
 /* Which grouped-GEMM kernel moe_forward and the expert stages use for p:
  * MOE_GEMM_SINGLE (one CTA per 128-row tile), MOE_GEMM_PAIR (CTA pairs,
  * 256-row tiles), MOE_GEMM_GRID_SPLIT (single-CTA tiles, groups of at most
- * 128 rows as operand-swapped tiles on their own CTAs), MOE_GEMM_SPLIT_K
+ * 128 rows as operand-swapped tiles on their own CTAs; MOE_SMALL_CTAS
+ * below), MOE_GEMM_SPLIT_K
  * (decode-sized batches: K split over CTAs), MOE_GEMM_SIMT (fp32, CUDA
  * cores); a negative MOE_ERR_* code if p is invalid. Host only. */
 #define MOE_GEMM_SINGLE      0
@@ -353,9 +354,11 @@ int moe_gemm_variant(const moe_problem* p);
  *                    two SMs); by default they do when the experts average
  *                    at least 512 rows (bf16 inference, no split-K).
  *   MOE_SMALL_CTAS=n with 32 or more experts and fewer than 512 rows per
- *                    expert on average, the first n CTAs run the groups of
- *                    at most 128 rows as operand-swapped tiles; n = 0 turns
- *                    this grid split off; unset, n comes from a cost model. */
+ *                    expert on average, the first n > 0 CTAs run the groups
+ *                    of at most 128 rows as operand-swapped tiles beside the
+ *                    larger groups (a grid split); unset or 0, no split (the
+ *                    default: measured no faster on the DeepSeek-shaped
+ *                    layer). */
 
 #ifdef __cplusplus
 }

@@ -222,10 +222,10 @@ def test_padded_forward_equals_dense():
     ("bf16", 256, 256, [700, 900], 128, 800),
     ("bf16", 256, 14336, [2600, 3], 0, 10),
     ("bf16", 128, 128, [1, 1023], 0, 512),
-    # at least 32 experts: groups of 1..128 rows run as operand-swapped tiles
-    # on their own CTAs beside the larger groups (every A-box boundary: 1, 32,
+    # at least 32 experts, mixed group sizes (every 32-row boundary: 1, 32,
     # 33, 64, 65, 96, 97, 128 rows), with and without the shared expert, and a
-    # large group over several bands of M blocks at K = 14336
+    # large group over several bands of M blocks at K = 14336 (the grid-split
+    # run of the same cases is in test_gpu_grid_split.py)
     ("bf16", 256, 384, [0, 1, 5, 31, 32, 33, 64, 65, 96, 97, 128, 129, 200, 300, 0, 7] + [3] * 16, 128, 800),
     ("bf16", 512, 256, [2, 40, 129, 700, 17, 0, 1, 90] * 4, 0, 2000),
     ("bf16", 256, 14336, [2500, 3, 7] + [1] * 29, 0, 10),
@@ -344,7 +344,7 @@ SMALL = [
     dict(T=3000, d=128, d_ff=256, E=4, k=2, cf=0.9, dtype="bf16", bias_mode=1, d_ff_shared=0, gate=1, drop=1),
     dict(T=1024, d=128, d_ff=128, E=2, k=1, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=128),
     dict(T=600, d=192, d_ff=320, E=1, k=1, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
-    # 32 or more experts: small groups on their own CTAs (operand-swapped tiles)
+    # 32 or more experts, many small groups
     dict(T=400, d=256, d_ff=256, E=32, k=4, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=0),
     dict(T=900, d=128, d_ff=384, E=64, k=6, cf=0.8, dtype="bf16", bias_mode=1, d_ff_shared=128, gate=1),
     # padded (MegaBlocks) layout: every expert's rows rounded up to 128 or 64
@@ -591,8 +591,8 @@ def _sample_tokens(pos, indptr, rng, n_random):
 def test_forward_full_size(name, n_random, pad):
     cfg = dict(inputs.workload(name), pad=pad)
     # the kernel each full-size workload exercises
-    want = {"mixtral_prefill": "single" if pad else "pair", "skewed_capacity": "pair", "deepseek_v3": "grid_split"}
-    if os.environ.get("MOE_CTA_PAIR", "1") != "0" and os.environ.get("MOE_SMALL_CTAS", "1") != "0":
+    want = {"mixtral_prefill": "single" if pad else "pair", "skewed_capacity": "pair", "deepseek_v3": "single"}
+    if os.environ.get("MOE_CTA_PAIR", "1") != "0" and "MOE_SMALL_CTAS" not in os.environ:
         assert moe.gemm_variant(problem_of(cfg)) == want[name]
     L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=DEV)
     Ld = to_device(L)
