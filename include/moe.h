@@ -48,6 +48,8 @@ extern "C" {
 #define MOE_ERR_WORKSPACE   3  /* workspace missing or smaller than moe_workspace_size() */
 #define MOE_ERR_CUDA        4  /* a CUDA launch or driver call failed */
 #define MOE_ERR_TIMEOUT     5  /* device status only: a bounded wait gave up */
+#define MOE_ERR_BOUNDS      6  /* device status only, debug build (libmoe_debug.so): an index
+                                  out of its buffer was found and the access skipped */
 
 /* ---- enums -------------------------------------------------------------- */
 #define MOE_DTYPE_F32  0
@@ -346,6 +348,16 @@ long long moe_set_wait_limit(long long ns);
 #define MOE_GEMM_SPLIT_K     3
 #define MOE_GEMM_SIMT        4
 int moe_gemm_variant(const moe_problem* p);
+
+/* Debug build. The library also builds as libmoe_debug.so (compiled with
+ * MOE_DEBUG), with the same entry points and results, plus device-side bounds
+ * checks that record MOE_ERR_BOUNDS in the call's status word and skip the
+ * access instead of faulting: the group offsets handed to the expert stages
+ * (non-decreasing, within the permuted rows; a violation empties the tile
+ * schedule, so no tile runs), every output row a grouped GEMM stores, and
+ * every permuted row the combine reads (moe_forward's status word; the
+ * standalone moe_combine has none, so it only skips). The Python binding
+ * loads it when MOE_LIBRARY=debug. */
 
 /* Kernel-selection overrides, read once per process from the environment
  * (for measurement and tests; results are the same either way, up to the

@@ -18,7 +18,8 @@ from typing import Optional
 import torch
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG_DIR, "libmoe.so")
+# MOE_LIBRARY=debug selects the build with device-side bounds checks
+LIB_PATH = os.path.join(_PKG_DIR, "libmoe_debug.so" if os.environ.get("MOE_LIBRARY") == "debug" else "libmoe.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -26,6 +27,7 @@ MOE_ERR_UNSUPPORTED = 2
 MOE_ERR_WORKSPACE = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_TIMEOUT = 5
+MOE_ERR_BOUNDS = 6
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1

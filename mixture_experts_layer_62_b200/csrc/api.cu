@@ -400,9 +400,11 @@ struct StageSplit {
     int32_t* sem13 = nullptr;
     int32_t* sem2 = nullptr;
 };
-StageSplit stage_split(const moe_problem* p, const Layout& L, void* ws) {
+StageSplit stage_split(const moe_problem* p, const Layout& L, void* ws, int32_t* status) {
     StageSplit s;
     s.sched.gsplit = grid_split_of(*p);
+    s.sched.rows_max = (int)permuted_rows(*p);
+    s.sched.status = status;
     if (!split_allowed(*p)) return s;
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
@@ -654,6 +656,7 @@ const char* moe_error_string(int code) {
         case MOE_ERR_WORKSPACE: return "workspace missing or too small";
         case MOE_ERR_CUDA: return "CUDA launch or driver error";
         case MOE_ERR_TIMEOUT: return "device-side bounded wait timed out";
+        case MOE_ERR_BOUNDS: return "device-side bounds check failed (debug build)";
         default: return "unknown error";
     }
 }
@@ -769,7 +772,7 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
                      p->train ? wsp(workspace, L.ab) : nullptr,
                      (p->train && shared) ? wsp(workspace, L.abs) : nullptr);
     if (rc != MOE_OK) return rc;
-    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st));
+    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, (int)permuted_rows(*p), status, st));
     return MOE_OK;
 }
 
@@ -912,7 +915,7 @@ int moe_experts(const moe_problem* p, const void* xp, const int32_t* indptr, con
     int32_t* tiles2 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles2));
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
-    const StageSplit sp = stage_split(p, L, workspace);
+    const StageSplit sp = stage_split(p, L, workspace, status);
     CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2,
                        sp.sched, st));
     void* h = wsp(workspace, L.h);
@@ -955,7 +958,7 @@ int moe_expert_up(const moe_problem* p, const void* xp, const int32_t* indptr, c
     CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
-    const StageSplit sp = stage_split(p, make_layout(*p), workspace);
+    const StageSplit sp = stage_split(p, make_layout(*p), workspace, status);
     CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2,
                        sp.sched, st));
     return run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, shared ? hs : nullptr, status, st, sp.part13,
@@ -983,7 +986,7 @@ int moe_expert_down(const moe_problem* p, const void* h, const int32_t* indptr, 
     CK(cudaMemsetAsync(status, 0, sizeof(int32_t), st));
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
-    const StageSplit sp = stage_split(p, make_layout(*p), workspace);
+    const StageSplit sp = stage_split(p, make_layout(*p), workspace, status);
     CK(launch_schedule(indptr, p->E, p->T, shared ? 1 : 0, tile_m, nt13, nt2, nt13s, nt2s, tiles13, tiles2,
                        sp.sched, st));
     return run_down(p, h, indptr, tiles2, W2, shared ? hs : nullptr, Ws2, o, shared ? s : nullptr, status, st,
@@ -997,7 +1000,7 @@ int moe_combine(const moe_problem* p, const void* o, const int32_t* pos, const f
     if (!o || !pos || !gate || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(o) || !aligned16(out) || (s && !aligned16(s))) return MOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, st));
+    CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, (int)permuted_rows(*p), nullptr, st));
     return MOE_OK;
 }
 

@@ -59,7 +59,8 @@ constexpr int kCbWarps = 8;
 template <typename T>
 __global__ void __launch_bounds__(kCbWarps * 32, 4)
 combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const float* __restrict__ gate,
-               const T* __restrict__ s, T* __restrict__ out, int Tn, int d, int k, int slices, int vpl) {
+               const T* __restrict__ s, T* __restrict__ out, int Tn, int d, int k, int slices, int vpl, int rows,
+               int32_t* __restrict__ status) {
     using V = VecTraits<T>;
     constexpr int VN = V::N;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -79,6 +80,10 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const f
     if (lane < k) {
         p_l = pos[(size_t)t * k + lane];
         g_l = gate[(size_t)t * k + lane];
+        if (kDebugChecks && p_l >= rows) {   // a position past o: recorded, the slot skipped
+            if (sl == 0) debug_record_bounds(status);
+            p_l = -1;
+        }
     }
     pdl_wait();
     pdl_launch();
@@ -141,7 +146,8 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ pos, const f
 }
 
 cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const float* gate,
-                           const void* s, void* out, int T, int d, int k, cudaStream_t st) {
+                           const void* s, void* out, int T, int d, int k, int rows, int32_t* status,
+                           cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int vn = dtype == MOE_DTYPE_BF16 ? 8 : 4;
     // small batches: one vector per lane per warp, so the few rows are spread
@@ -153,9 +159,9 @@ cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const f
     if (dtype == MOE_DTYPE_BF16)
         return launch_k(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(kCbWarps * 32), 0, st,
                         (const __nv_bfloat16*)o, pos, gate, (const __nv_bfloat16*)s, (__nv_bfloat16*)out, T, d, k,
-                        slices, vpl);
+                        slices, vpl, rows, status);
     return launch_k(combine_kernel<float>, dim3(grid), dim3(kCbWarps * 32), 0, st, (const float*)o, pos, gate,
-                    (const float*)s, (float*)out, T, d, k, slices, vpl);
+                    (const float*)s, (float*)out, T, d, k, slices, vpl, rows, status);
 }
 
 }  // namespace moe

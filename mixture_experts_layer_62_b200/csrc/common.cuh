@@ -16,6 +16,17 @@ namespace moe {
 // gather all work on chunks of this many consecutive tokens.
 constexpr int kChunk = 32;
 
+// Debug build (compiled with MOE_DEBUG): device-side bounds checks record
+// MOE_ERR_BOUNDS in a status word and skip the access.
+#ifdef MOE_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ void debug_record_bounds(int32_t* status) {
+    if (status != nullptr) atomicCAS(status, MOE_OK, MOE_ERR_BOUNDS);
+}
+
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Programmatic dependent launch. moe_forward launches every kernel after its
@@ -186,6 +197,10 @@ struct ScheduleSplit {
     int32_t* sem; int sem_n;
     SplitTable split;
     GridSplit gsplit;
+    // debug build: the given group offsets are checked against rows_max and
+    // a violation is recorded in *status (when not null)
+    int rows_max;
+    int32_t* status;
 };
 cudaError_t launch_schedule(const int32_t* indptr, int E, int T, int has_shared, int tile_m,
                             int ntiles13, int ntiles2, int ntiles13_shared, int ntiles2_shared,
@@ -194,8 +209,11 @@ cudaError_t launch_permute_gather(int dtype, const void* x, const int32_t* idx,
                                   const int32_t* blockoff, const int32_t* indptr,
                                   int T, int d, int E, int k, int kk, int capacity,
                                   int32_t* pos, int32_t* row_token, void* xp, cudaStream_t st);
+// rows: rows of o (permuted rows); status: where a debug build records an
+// out-of-range position (may be null)
 cudaError_t launch_combine(int dtype, const void* o, const int32_t* pos, const float* gate,
-                           const void* s, void* out, int T, int d, int k, cudaStream_t st);
+                           const void* s, void* out, int T, int d, int k, int rows, int32_t* status,
+                           cudaStream_t st);
 cudaError_t launch_zero_stats(void* stats, int E, int capacity, cudaStream_t st);
 
 // Small-batch router (T*k <= kSmallMaxPairs, E <= kSmallMaxE, E % 8 == 0,

@@ -81,6 +81,7 @@ struct KParams {
     int nt_blk[2];             // N blocks of a group (routed, shared)
     int band_m[2];             // M blocks per band (0: the whole group is one band)
     int split_grid;            // the schedule carries the small/large grid split
+    int out_rows[2];           // rows of the output buffers (debug-build bounds checks)
 };
 
 struct Tile {
@@ -531,8 +532,12 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             if (!wait_bounded(&ctl->tfull[acc], aph, ctl, p)) break;
             tc_fence_after();
             const int grow = t.m_blk * BM + r;
-            const bool valid = grow < t.rows;
+            bool valid = grow < t.rows;
             const size_t orow = static_cast<size_t>(t.row0) + static_cast<size_t>(grow);
+            if (kDebugChecks && valid && orow >= static_cast<size_t>(p.out_rows[t.kind])) {
+                debug_record_bounds(p.status);   // an output row past its buffer: not stored
+                valid = false;
+            }
             const int N = p.N[t.kind];
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                 static_cast<uint32_t>(acc * ACC_COLS);
@@ -551,7 +556,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int n = c + i;
-                        if (n < t.rows) {
+                        if (n < t.rows && (!kDebugChecks || t.row0 + n < p.out_rows[0])) {
                             __nv_bfloat16* orow_p = outp + (static_cast<size_t>(t.row0) + n) * N;
                             const float a = __uint_as_float(v0[i]), b = __uint_as_float(v1[i]);
                             if (MODE == TC_SWIGLU) {
@@ -1039,8 +1044,13 @@ tc_pair_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ C
             const int grow = t.m_blk * PBM + r;
             const size_t orow = static_cast<size_t>(t.row0) + static_cast<size_t>(grow);
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_COLS);
-            if (hf < 0) pair_store_row<MODE>(p, t, tb, grow < t.rows, orow);
-            else pair_store_half_row<MODE>(p, t, tb, grow < t.rows, orow, hf);
+            bool valid = grow < t.rows;
+            if (kDebugChecks && valid && orow >= static_cast<size_t>(p.out_rows[t.kind])) {
+                debug_record_bounds(p.status);   // an output row past its buffer: not stored
+                valid = false;
+            }
+            if (hf < 0) pair_store_row<MODE>(p, t, tb, valid, orow);
+            else pair_store_half_row<MODE>(p, t, tb, valid, orow, hf);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -1214,6 +1224,8 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
     }
     KParams kp;
     kp.split_grid = a.split_grid;
+    kp.out_rows[0] = a.a_rows[0];
+    kp.out_rows[1] = a.T;
     kp.indptr = a.indptr;
     kp.tiles = a.tiles;
     kp.static_rows = a.static_rows;

@@ -365,6 +365,21 @@ schedule_kernel(const int32_t* __restrict__ indptr, int E, int T, int has_shared
     for (int g = threadIdx.x; g < E; g += blockDim.x) rows[g] = indptr[g + 1] - indptr[g];
     if (threadIdx.x == 0) rows[E] = T;
     __syncthreads();
+    if (kDebugChecks) {
+        // the given offsets must start at 0 or above, never decrease and end
+        // within the permuted rows; otherwise no tile is scheduled
+        __shared__ int bad;
+        if (threadIdx.x == 0) bad = 0;
+        __syncthreads();
+        for (int g = threadIdx.x; g < E; g += blockDim.x)
+            if (indptr[g] < 0 || indptr[g + 1] < indptr[g] || indptr[g + 1] > sp.rows_max) bad = 1;
+        __syncthreads();
+        if (bad) {
+            for (int g = threadIdx.x; g <= E; g += blockDim.x) rows[g] = 0;
+            if (threadIdx.x == 0) debug_record_bounds(sp.status);
+        }
+        __syncthreads();
+    }
     const int G = E + has_shared;
     int n_active;
     block_exclusive_scan(threadIdx.x < E && rows[threadIdx.x] > 0 ? 1 : 0, warp_tot, n_active);

@@ -51,7 +51,7 @@ def test_wait_limit_is_settable_and_restorable():
 
 def test_error_strings():
     assert moe.error_string(0) == "ok"
-    for code in range(1, 6):
+    for code in range(1, 7):
         assert moe.error_string(code) not in ("ok", "unknown error")
     assert moe.error_string(99) == "unknown error"
 
@@ -189,3 +189,16 @@ def test_gemm_variant_follows_the_shape():
     assert variant("deepseek_v3") == "single"                      # the grid split is opt-in
     with pytest.raises(moe.MoEError):
         moe.gemm_variant(moe.problem(16, 256, 64, 4, 5))            # k > E
+
+
+def test_debug_library_exports_the_same_entry_points():
+    # libmoe_debug.so (device-side bounds checks) is a drop-in for libmoe.so
+    from mixture_experts_layer_62_b200 import build as mb
+    assert os.path.exists(mb.DEBUG_LIB_PATH), "build() makes the debug library too"
+    out = subprocess.run(["nm", "-D", "--defined-only", mb.DEBUG_LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(moe_\w+)", out))
+    assert exported == set(declared_functions())
+    dbg = ctypes.CDLL(mb.DEBUG_LIB_PATH)
+    dbg.moe_error_string.restype = ctypes.c_char_p
+    assert dbg.moe_error_string(6).decode() == "device-side bounds check failed (debug build)"
+    assert moe.error_string(6) == "device-side bounds check failed (debug build)"
