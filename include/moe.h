@@ -341,12 +341,17 @@ long long moe_set_wait_limit(long long ns);
  * 128 rows as operand-swapped tiles on their own CTAs; MOE_SMALL_CTAS
  * below), MOE_GEMM_SPLIT_K
  * (decode-sized batches: K split over CTAs), MOE_GEMM_SIMT (fp32, CUDA
- * cores); a negative MOE_ERR_* code if p is invalid. Host only. */
+ * cores), MOE_GEMM_INTERLEAVED (single-CTA tiles; with 32 or more experts
+ * averaging fewer than 512 rows, the tiles of the groups of at most 128
+ * rows are spread evenly through the others' and load their weights with an
+ * evict-first L2 policy); a negative MOE_ERR_* code if p is invalid. Host
+ * only. */
 #define MOE_GEMM_SINGLE      0
 #define MOE_GEMM_PAIR        1
 #define MOE_GEMM_GRID_SPLIT  2
 #define MOE_GEMM_SPLIT_K     3
 #define MOE_GEMM_SIMT        4
+#define MOE_GEMM_INTERLEAVED 5
 int moe_gemm_variant(const moe_problem* p);
 
 /* Debug build. The library also builds as libmoe_debug.so (compiled with
@@ -368,9 +373,11 @@ int moe_gemm_variant(const moe_problem* p);
  *   MOE_SMALL_CTAS=n with 32 or more experts and fewer than 512 rows per
  *                    expert on average, the first n > 0 CTAs run the groups
  *                    of at most 128 rows as operand-swapped tiles beside the
- *                    larger groups (a grid split); unset or 0, no split (the
- *                    default: measured no faster on the DeepSeek-shaped
- *                    layer). */
+ *                    larger groups (a grid split; measured no faster on the
+ *                    DeepSeek-shaped layer); 0 turns the two-class schedule
+ *                    off altogether.
+ *   MOE_INTERLEAVE=0 no interleaved two-class schedule (the default for such
+ *                    shapes, MOE_GEMM_INTERLEAVED above). */
 
 #ifdef __cplusplus
 }

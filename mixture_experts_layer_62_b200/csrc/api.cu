@@ -156,13 +156,18 @@ GridSplit grid_split_of(const moe_problem& p) {
     // measured on the DeepSeek-shaped layer (alternating runs on one box):
     // 7.43-7.49 ms per step with the split against 7.39-7.44 ms without, so
     // the split is opt-in (MOE_SMALL_CTAS=n > 0), not the default
+    static const bool interleave = [] {
+        const char* v = std::getenv("MOE_INTERLEAVE");
+        return !(v != nullptr && v[0] == '0');
+    }();
     GridSplit g = {};
-    g.on = forced > 0 && p.dtype == MOE_DTYPE_BF16 && p.T > 0 && p.pad_rows == 0 && !p.train && !split_allowed(p) &&
-           !use_pair_tiles(p) && p.E >= 32 && p.d % 64 == 0;
+    g.interleave = forced > 0 ? 0 : 1;
+    g.on = (forced > 0 || (forced != 0 && interleave)) && p.dtype == MOE_DTYPE_BF16 && p.T > 0 && p.pad_rows == 0 &&
+           !p.train && !split_allowed(p) && !use_pair_tiles(p) && p.E >= 32 && p.d % 64 == 0;
     g.k13 = p.d; g.k2 = p.d_ff; g.k13s = p.d; g.k2s = p.d_ff_shared;
     g.grid = device_sm_count();
     g.force_ctas = forced > 0 ? forced : 0;
-    if (g.grid <= 1) g.on = 0;
+    if (g.grid <= 1 && !g.interleave) g.on = 0;
     return g;
 }
 
@@ -284,7 +289,11 @@ int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const in
         TcArgs a = {};
         a.mode = TC_SWIGLU;
         a.pair = use_pair_tiles(*p) ? 1 : 0;
-        a.split_grid = grid_split_of(*p).on;
+        {
+            const GridSplit gs = grid_split_of(*p);
+            a.split_grid = gs.on;
+            a.interleave = gs.on && gs.interleave;
+        }
         a.b_before_wait = sched_early ? 1 : 0;
         a.indptr = indptr; a.tiles = tiles13;
         a.E = p->E; a.has_shared = has_shared; a.T = p->T;
@@ -330,7 +339,11 @@ int run_down(const moe_problem* p, const void* h, const int32_t* indptr, const i
         TcArgs b = {};
         b.mode = TC_PLAIN;
         b.pair = use_pair_tiles(*p) ? 1 : 0;
-        b.split_grid = grid_split_of(*p).on;
+        {
+            const GridSplit gs = grid_split_of(*p);
+            b.split_grid = gs.on;
+            b.interleave = gs.on && gs.interleave;
+        }
         b.b_before_wait = 1;   // the schedule comes from the router, two or more launches back
         b.indptr = indptr; b.tiles = tiles2;
         b.E = p->E; b.has_shared = has_shared; b.T = p->T;
@@ -450,7 +463,10 @@ int moe_gemm_variant(const moe_problem* p) {
     if (p->dtype != MOE_DTYPE_BF16) return MOE_GEMM_SIMT;
     if (split_allowed(*p)) return MOE_GEMM_SPLIT_K;
     if (use_pair_tiles(*p)) return MOE_GEMM_PAIR;
-    if (grid_split_of(*p).on) return MOE_GEMM_GRID_SPLIT;
+    {
+        const GridSplit gs = grid_split_of(*p);
+        if (gs.on) return gs.interleave ? MOE_GEMM_INTERLEAVED : MOE_GEMM_GRID_SPLIT;
+    }
     return MOE_GEMM_SINGLE;
 }
 

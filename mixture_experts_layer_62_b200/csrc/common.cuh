@@ -161,6 +161,8 @@ cudaError_t launch_hist(const int32_t* idx, int T, int k, int kk, int E, int32_t
 constexpr int kSmallRows = 128;
 struct GridSplit {
     int on;
+    int interleave;           // 1: no CTA split; the small groups' tiles are spread through the large
+                              // groups' in the order all CTAs take them (S written as 0)
     int k13, k2, k13s, k2s;   // K of the routed and shared GEMM 1/3 and GEMM 2
     int grid;                 // CTAs of the GEMM launches
     int force_ctas;           // > 0: S from the environment (tuning), else the cost model
@@ -261,9 +263,9 @@ constexpr int kTcPairTileM = 256;   // rows of a CTA-pair tile
 // not the training forward, unpadded, at least 512 rows per expert on
 // average); the environment variable MOE_CTA_PAIR=0 turns them off.
 bool use_pair_tiles(const moe_problem& p);
-// The small/large grid split for p (bf16 inference, no split-K, no pairs,
-// at least 32 experts); MOE_SMALL_CTAS=n forces S = n (n = 0 turns the split
-// off).
+// The two-class schedule for p (bf16 inference, no split-K, no pairs, at
+// least 32 experts): interleaved by default (MOE_INTERLEAVE=0 turns it off);
+// MOE_SMALL_CTAS=n > 0 splits the grid instead, n CTAs for the small class.
 GridSplit grid_split_of(const moe_problem& p);
 int tc_out_cols_per_tile(int mode);   // 128 for SWIGLU, 256 otherwise
 enum TcMode { TC_SWIGLU = 0, TC_PLAIN = 1, TC_F32OUT = 2 };
@@ -297,6 +299,10 @@ struct TcArgs {
     // 1: the schedule carries the small/large grid split (GridSplit); SWIGLU
     // or PLAIN, no split-K, no pre-activation output
     int split_grid;
+    // with split_grid: the two classes are interleaved in one order over all
+    // CTAs, the small groups as ordinary tiles whose weights are loaded with
+    // an evict-first L2 policy
+    int interleave;
 };
 cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st);
 // Backward grouped GEMMs (tcgen05): see gemm_bwd_sm100.cu.

@@ -82,6 +82,7 @@ struct KParams {
     int band_m[2];             // M blocks per band (0: the whole group is one band)
     int split_grid;            // the schedule carries the small/large grid split
     int out_rows[2];           // rows of the output buffers (debug-build bounds checks)
+    int interleave;            // with split_grid: both classes in one interleaved order
 };
 
 struct Tile {
@@ -138,6 +139,11 @@ struct Units {
 };
 __device__ __forceinline__ Units cta_units(const KParams& p, int total, int nsplit) {
     Units r;
+    if (p.split_grid && p.interleave) {
+        const int G = p.E + p.has_shared;
+        r.first = blockIdx.x; r.step = gridDim.x; r.count = total + p.tiles[2 * G + 3]; r.small = false;
+        return r;
+    }
     if (p.split_grid) {
         const int G = p.E + p.has_shared;
         const int S = p.tiles[G + 2];
@@ -171,6 +177,20 @@ __device__ __forceinline__ Tile decode_small_tile(const KParams& p, int u) {
     return t;
 }
 __device__ __forceinline__ int small_boxes(const Tile& t) { return (t.rows + 31) / 32; }   // 32-row A boxes
+
+// Unit u of the interleaved two-class order: the S tiles of the small class
+// (groups of at most 128 rows, run as ordinary tiles) are spread evenly
+// through the L tiles of the large class. Position u holds small tile
+// floor(u S / (L + S)) when floor((u + 1) S / (L + S)) exceeds it, else large
+// tile u - floor(u S / (L + S)) (the large tiles keep their order, so the
+// CTAs that share a weight tile still run together).
+__device__ __forceinline__ Tile decode_mixed(const KParams& p, int u, bool& small_class) {
+    const int G = p.E + p.has_shared;
+    const long long L = p.tiles[G], S = p.tiles[2 * G + 3], N = L + S;
+    const long long a = (long long)u * S / N, b = (long long)(u + 1) * S / N;
+    small_class = b > a;
+    return small_class ? decode_small_tile(p, static_cast<int>(a)) : decode_tile(p, u - static_cast<int>(a));
+}
 
 struct SharedCtl {
     uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
@@ -379,9 +399,17 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             bool aborted = false;
             int pre = 0;   // stages of the first unit whose weight tiles were requested before the wait
             // the unit's tile and K-block range (a split of it with split-K)
+            bool cls_small = false;   // interleaved order: the unit is a small-class tile
+            const uint64_t evict_first = l2_evict_first_policy();
             auto unit_tile = [&](int u, int& kb0, int& kb1) {
+                cls_small = false;
                 if (un.small) {
                     const Tile t = decode_small_tile(p, u);
+                    kb0 = 0; kb1 = t.num_kb;
+                    return t;
+                }
+                if (p.split_grid && p.interleave) {
+                    const Tile t = decode_mixed(p, u, cls_small);
                     kb0 = 0; kb1 = t.num_kb;
                     return t;
                 }
@@ -393,6 +421,17 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
             // bytes of one stage: small tiles load only the group's 32-row boxes of A
             auto stage_tx = [&](const Tile& t) {
                 return un.small ? static_cast<uint32_t>(B_BYTES + small_boxes(t) * 4096) : static_cast<uint32_t>(STAGE_BYTES);
+            };
+            // the weight rows of a tile; a small-class tile's are read by that tile
+            // alone, so they go to L2 as evict-first
+            auto load_b = [&](uint32_t sa, const TileLoads& l, int kb, uint64_t* bar) {
+                if (cls_small) {
+                    tma_load_2d_hint(sa + A_BYTES, l.mlo, bar, kb * BK, l.brow0, evict_first);
+                    tma_load_2d_hint(sa + A_BYTES + B_HALF_BYTES, l.mhi, bar, kb * BK, l.brow1, evict_first);
+                } else {
+                    tma_load_2d(sa + A_BYTES, l.mlo, bar, kb * BK, l.brow0);
+                    tma_load_2d(sa + A_BYTES + B_HALF_BYTES, l.mhi, bar, kb * BK, l.brow1);
+                }
             };
             auto load_a = [&](uint32_t sa, const Tile& t, const TileLoads& l, int kb, uint64_t* bar) {
                 if (un.small) {
@@ -411,8 +450,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                         // every stage is free at the start: no empty-barrier wait
                         const uint32_t sa = smem_u32(smem + pre * STAGE_BYTES);
                         mbar_arrive_expect_tx(&ctl->full[pre], stage_tx(t));
-                        tma_load_2d(sa + A_BYTES, l.mlo, &ctl->full[pre], kb * BK, l.brow0);
-                        tma_load_2d(sa + A_BYTES + B_HALF_BYTES, l.mhi, &ctl->full[pre], kb * BK, l.brow1);
+                        load_b(sa, l, kb, &ctl->full[pre]);
                         issued_mask |= 1u << pre;
                     }
                 }
@@ -432,8 +470,7 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                         if (!wait_bounded(&ctl->empty[s], ph ^ 1u, ctl, p)) { aborted = true; break; }
                         mbar_arrive_expect_tx(&ctl->full[s], stage_tx(t));
                         load_a(sa, t, l, kb, &ctl->full[s]);
-                        tma_load_2d(sa + A_BYTES, l.mlo, &ctl->full[s], kb * BK, l.brow0);
-                        tma_load_2d(sa + A_BYTES + B_HALF_BYTES, l.mhi, &ctl->full[s], kb * BK, l.brow1);
+                        load_b(sa, l, kb, &ctl->full[s]);
                     }
                     issued_mask |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
@@ -469,6 +506,10 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
                 Tile t;
                 if (un.small) {
                     t = decode_small_tile(p, u);
+                    kb1 = t.num_kb;
+                } else if (p.split_grid && p.interleave) {
+                    bool cs;
+                    t = decode_mixed(p, u, cs);
                     kb1 = t.num_kb;
                 } else {
                     const int sp = u % nsplit;
@@ -528,7 +569,9 @@ tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA0, const __grid_constant_
         uint32_t aph = 0;
         for (int u = un.first; u < un.count; u += un.step) {
             const int sp = un.small ? 0 : u % nsplit;
-            const Tile t = un.small ? decode_small_tile(p, u) : decode_tile(p, u / nsplit);
+            bool cs;
+            const Tile t = un.small ? decode_small_tile(p, u)
+                         : (p.split_grid && p.interleave) ? decode_mixed(p, u, cs) : decode_tile(p, u / nsplit);
             if (!wait_bounded(&ctl->tfull[acc], aph, ctl, p)) break;
             tc_fence_after();
             const int grow = t.m_blk * BM + r;
@@ -1217,13 +1260,14 @@ cudaError_t launch_tc_gemm(const TcArgs& a, cudaStream_t st) {
         maps[4] = maps[2];
         maps[5] = maps[3];
     }
-    if (a.split_grid) {
+    if (a.split_grid && !a.interleave) {
         if (!make_map(&maps[6], a.A[0], a.a_rows[0], a.K[0], 32)) return cudaErrorInvalidValue;
     } else {
         maps[6] = maps[0];
     }
     KParams kp;
     kp.split_grid = a.split_grid;
+    kp.interleave = a.interleave;
     kp.out_rows[0] = a.a_rows[0];
     kp.out_rows[1] = a.T;
     kp.indptr = a.indptr;

@@ -143,8 +143,8 @@ __device__ void build_gemm_schedules(int* rows, int G, int E, int tile_m, int nt
             }
         }
         const int f = gs.force_ctas > 0 ? min(gs.force_ctas, gs.grid) : -1;
-        tiles13[G + 2] = f > 0 ? (s13 > 0 ? f : 0) : choose_small_ctas(l13, s13, gs.grid);
-        tiles2[G + 2] = f > 0 ? (s2 > 0 ? f : 0) : choose_small_ctas(l2, s2, gs.grid);
+        tiles13[G + 2] = gs.interleave ? 0 : f > 0 ? (s13 > 0 ? f : 0) : choose_small_ctas(l13, s13, gs.grid);
+        tiles2[G + 2] = gs.interleave ? 0 : f > 0 ? (s2 > 0 ? f : 0) : choose_small_ctas(l2, s2, gs.grid);
     }
     __syncthreads();
 }
