@@ -229,6 +229,8 @@ KERNEL_NAMES = {
                    "tc_grouped_gemm_swiglu"),
     "single": ("tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU)", "tc_grouped_gemm_swiglu"),
     "split_k": ("tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU, split-K)", "tc_grouped_gemm_swiglu"),
+    "interleaved": ("tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU, small groups interleaved)",
+                    "tc_grouped_gemm_swiglu"),
     "simt": ("simt_gemm_kernel<true> (grouped GEMM 1/3 + SwiGLU, CUDA cores)", "simt_gemm_swiglu"),
 }
 

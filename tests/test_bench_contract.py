@@ -66,3 +66,8 @@ def test_pass_roofline_of_the_deepseek_shaped_layer():
 def test_every_other_config_is_measured_by_default():
     names = set(bench.EXTRA_WORKLOADS)
     assert {"decode_t1", "decode_t2", "decode_t4", "decode_t8", "deepseek_v3", "skewed_capacity"} <= names
+
+
+def test_every_gemm_variant_has_a_kernel_name():
+    from mixture_experts_layer_62_b200 import GEMM_VARIANTS
+    assert set(GEMM_VARIANTS.values()) <= set(bench.KERNEL_NAMES)
