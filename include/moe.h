@@ -374,10 +374,10 @@ int moe_gemm_variant(const moe_problem* p);
  *                    expert on average, the first n > 0 CTAs run the groups
  *                    of at most 128 rows as operand-swapped tiles beside the
  *                    larger groups (a grid split; measured no faster on the
- *                    DeepSeek-shaped layer); 0 turns the two-class schedule
- *                    off altogether.
- *   MOE_INTERLEAVE=0 no interleaved two-class schedule (the default for such
- *                    shapes, MOE_GEMM_INTERLEAVED above). */
+ *                    DeepSeek-shaped layer).
+ *   MOE_INTERLEAVE=1 for the same shapes, the interleaved two-class order
+ *                    (MOE_GEMM_INTERLEAVED above; also measured no faster
+ *                    there). Without either, one order in expert order. */
 
 #ifdef __cplusplus
 }

@@ -156,9 +156,12 @@ GridSplit grid_split_of(const moe_problem& p) {
     // measured on the DeepSeek-shaped layer (alternating runs on one box):
     // 7.43-7.49 ms per step with the split against 7.39-7.44 ms without, so
     // the split is opt-in (MOE_SMALL_CTAS=n > 0), not the default
+    // both two-class schedules measured no faster than the single order on
+    // the DeepSeek-shaped layer (alternating runs on one box: 7.82 / 7.75 ms
+    // without, 7.89 / 7.86 ms interleaved), so both are opt-in
     static const bool interleave = [] {
         const char* v = std::getenv("MOE_INTERLEAVE");
-        return !(v != nullptr && v[0] == '0');
+        return v != nullptr && v[0] == '1';
     }();
     GridSplit g = {};
     g.interleave = forced > 0 ? 0 : 1;

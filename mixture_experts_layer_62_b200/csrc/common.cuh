@@ -264,8 +264,8 @@ constexpr int kTcPairTileM = 256;   // rows of a CTA-pair tile
 // average); the environment variable MOE_CTA_PAIR=0 turns them off.
 bool use_pair_tiles(const moe_problem& p);
 // The two-class schedule for p (bf16 inference, no split-K, no pairs, at
-// least 32 experts): interleaved by default (MOE_INTERLEAVE=0 turns it off);
-// MOE_SMALL_CTAS=n > 0 splits the grid instead, n CTAs for the small class.
+// least 32 experts), opt-in: MOE_INTERLEAVE=1 interleaves the classes,
+// MOE_SMALL_CTAS=n > 0 splits the grid, n CTAs for the small class.
 GridSplit grid_split_of(const moe_problem& p);
 int tc_out_cols_per_tile(int mode);   // 128 for SWIGLU, 256 otherwise
 enum TcMode { TC_SWIGLU = 0, TC_PLAIN = 1, TC_F32OUT = 2 };

@@ -186,7 +186,7 @@ def test_gemm_variant_follows_the_shape():
     assert variant("toy_fp32") == "simt"
     assert variant("mixtral_prefill", T=1000) == "single"          # 250 rows per expert
     assert variant("mixtral_prefill", d_ff=14336, train=1) == "single"
-    assert variant("deepseek_v3") == "interleaved"                 # small groups spread through the large
+    assert variant("deepseek_v3") == "single"                      # the two-class schedules are opt-in
     with pytest.raises(moe.MoEError):
         moe.gemm_variant(moe.problem(16, 256, 64, 4, 5))            # k > E
 

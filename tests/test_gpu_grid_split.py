@@ -1,13 +1,16 @@
-"""The opt-in grid split of the single-CTA grouped GEMMs (MOE_SMALL_CTAS=n).
+"""The opt-in two-class schedules of the single-CTA grouped GEMMs.
 
-With 32 or more experts and fewer than 512 rows per expert on average, the
-split runs the groups of at most 128 rows as operand-swapped tiles (the
-weight rows as the MMA's M operand, the group's rows in 32-row boxes as its
-N operand) on the first n CTAs, and the other groups on the rest. The
-override is read once per process, so the runs with it set happen in a
-child process; its outputs are checked here against the oracle, element by
-element, at the bf16 bar, over groups of every size around the 32-row box
-boundaries, with and without the shared expert, and in a whole forward.
+With 32 or more experts and fewer than 512 rows per expert on average:
+  * MOE_SMALL_CTAS=n (grid split) runs the groups of at most 128 rows as
+    operand-swapped tiles (the weight rows as the MMA's M operand, the
+    group's rows in 32-row boxes as its N operand) on the first n CTAs, and
+    the other groups on the rest;
+  * MOE_INTERLEAVE=1 spreads those groups' ordinary tiles evenly through the
+    others' in one order, their weights loaded with an evict-first L2 policy.
+The overrides are read once per process, so each runs in a child process;
+its outputs are checked here against the oracle, element by element, at the
+bf16 bar, over groups of every size around the 32-row boundaries, with and
+without the shared expert, and in a whole forward.
 """
 
 import math
@@ -62,7 +65,7 @@ for i, (d, d_ff, counts, dfs, T) in enumerate(CASES):
     E = len(counts)
     xp, W1, W3, W2, x, sh = _inputs(i, d, d_ff, counts, dfs, T)
     p = moe.problem(T, d, d_ff, E, 2, 0.0, "bf16", 0, dfs)
-    assert moe.gemm_variant(p) == "grid_split"
+    assert moe.gemm_variant(p) == sys.argv[3]
     ws = moe.alloc_workspace(p, DEV)
     st = moe.alloc_stats(E, DEV)
     o = torch.zeros((2 * T, d), dtype=torch.bfloat16, device=DEV)
@@ -80,7 +83,7 @@ from test_gpu_grid_split import _forward_layer, FWD
 T, d, d_ff, E, k, cf = FWD
 L = _forward_layer()
 p = moe.problem(T, d, d_ff, E, k, cf, "bf16", 1, 0)
-assert moe.gemm_variant(p) == "grid_split"
+assert moe.gemm_variant(p) == sys.argv[3]
 ws = moe.alloc_workspace(p, DEV)
 st = moe.alloc_stats(E, DEV)
 y = torch.empty((T, d), dtype=torch.bfloat16, device=DEV)
@@ -108,11 +111,13 @@ def _forward_layer():
                 bias=torch.linspace(0.5, -0.5, E))
 
 
-def test_grid_split_expert_stages_match_the_oracle(tmp_path):
+@pytest.mark.parametrize("env_var,value,variant", [("MOE_SMALL_CTAS", "24", "grid_split"),
+                                                 ("MOE_INTERLEAVE", "1", "interleaved")])
+def test_two_class_schedules_match_the_oracle(tmp_path, env_var, value, variant):
     path = tmp_path / "split.npz"
-    env = dict(os.environ, MOE_SMALL_CTAS="24")
-    r = subprocess.run([sys.executable, "-c", SCRIPT, str(path), ROOT], env=env, capture_output=True, text=True,
-                       timeout=900)
+    env = dict(os.environ, **{env_var: value})
+    r = subprocess.run([sys.executable, "-c", SCRIPT, str(path), ROOT, variant], env=env, capture_output=True,
+                       text=True, timeout=900)
     assert r.returncode == 0, r.stdout + r.stderr
     got = dict(np.load(path))
     for i, (d, d_ff, counts, dfs, T) in enumerate(CASES):

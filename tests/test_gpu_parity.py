@@ -224,9 +224,8 @@ def test_padded_forward_equals_dense():
     ("bf16", 128, 128, [1, 1023], 0, 512),
     # at least 32 experts, mixed group sizes (every 32-row boundary: 1, 32,
     # 33, 64, 65, 96, 97, 128 rows), with and without the shared expert, and a
-    # large group over several bands of M blocks at K = 14336: the groups of
-    # at most 128 rows interleaved through the others' tiles (the grid-split
-    # run of the same cases is in test_gpu_grid_split.py)
+    # large group over several bands of M blocks at K = 14336 (the runs of the
+    # same cases with the two-class schedules are in test_gpu_grid_split.py)
     ("bf16", 256, 384, [0, 1, 5, 31, 32, 33, 64, 65, 96, 97, 128, 129, 200, 300, 0, 7] + [3] * 16, 128, 800),
     ("bf16", 512, 256, [2, 40, 129, 700, 17, 0, 1, 90] * 4, 0, 2000),
     ("bf16", 256, 14336, [2500, 3, 7] + [1] * 29, 0, 10),
@@ -592,7 +591,7 @@ def _sample_tokens(pos, indptr, rng, n_random):
 def test_forward_full_size(name, n_random, pad):
     cfg = dict(inputs.workload(name), pad=pad)
     # the kernel each full-size workload exercises
-    want = {"mixtral_prefill": "single" if pad else "pair", "skewed_capacity": "pair", "deepseek_v3": "interleaved"}
+    want = {"mixtral_prefill": "single" if pad else "pair", "skewed_capacity": "pair", "deepseek_v3": "single"}
     if not any(v in os.environ for v in ("MOE_CTA_PAIR", "MOE_SMALL_CTAS", "MOE_INTERLEAVE")):
         assert moe.gemm_variant(problem_of(cfg)) == want[name]
     L = inputs.make_layer(cfg, seed=0, device="cpu", weights_device=DEV)
