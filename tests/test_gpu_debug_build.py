@@ -3,7 +3,8 @@ checks that turn an out-of-range index into MOE_ERR_BOUNDS instead of a fault.
 
 The debug library is loaded in a child process (MOE_LIBRARY=debug). There:
   * whole forwards on valid inputs (the CTA-pair and single-CTA kernels, the
-    split-K decode path) give the release library's bits and MOE_OK;
+    split-K decode path after either router) give the release library's bits
+    and MOE_OK;
   * the expert stage handed group offsets that decrease, or that end past
     the permuted rows, records MOE_ERR_BOUNDS, schedules no tile and writes
     nothing: every row of the output keeps its sentinel value.
@@ -29,7 +30,8 @@ DEV = "cuda"
 
 FORWARDS = [dict(T=2048, d=256, d_ff=384, E=4, k=2, cf=0.0),      # CTA pairs
             dict(T=300, d=256, d_ff=384, E=8, k=2, cf=0.6),       # single-CTA tiles, capacity drops
-            dict(T=4, d=512, d_ff=512, E=8, k=2, cf=0.0)]         # decode path, split-K
+            dict(T=40, d=512, d_ff=512, E=8, k=2, cf=0.0),        # split-K, general router
+            dict(T=4, d=512, d_ff=512, E=8, k=2, cf=0.0)]         # split-K, small-batch router
 
 
 def _layer(c, seed):
