@@ -19,11 +19,17 @@ owner's expert order; no packing step is needed. Then:
    it lands exactly where the single-GPU pass puts its expert outputs (O, in
    the permuted order), and the library's combine finishes the layer.
 
+``forward_overlapped`` does steps 2-4 in rounds of paired sends and
+receives (rank r exchanges with r + i and r - i in round i), so the grouped
+GEMMs of one source's block run while the next block's rows, and the
+previous block's outputs, are on the wire.
+
 Capacity is applied by each source on its own tokens (per-device capacity,
-as for the data-parallel replicas). This is the unfused form, with the
-collectives issued by torch.distributed (NCCL on GPUs, gloo on CPU tensors);
-the same functions serve both. Overlapping the transfers with the grouped
-GEMM tile by tile, over peer memory, is not built here.
+as for the data-parallel replicas). The collectives and point-to-point
+transfers are issued by torch.distributed (NCCL on GPUs, gloo on CPU
+tensors); the same functions serve both. The overlap is per block; a single
+kernel that moves tiles over peer memory while it multiplies is not built
+here.
 """
 
 from __future__ import annotations
@@ -111,6 +117,82 @@ def combine_back(expert_out: torch.Tensor, p: EPPlan, o: torch.Tensor, group=Non
     expert outputs in its own permuted order) and returns o."""
     dist.all_to_all_single(o[:p.rows_out], expert_out.contiguous(), output_split_sizes=p.send_rows,
                            input_split_sizes=p.recv_rows, group=group)
+    return o
+
+
+def _peer(rank: int, group) -> int:
+    return rank if group is None else dist.get_global_rank(group, rank)
+
+
+def forward_overlapped(xp: torch.Tensor, p: EPPlan,
+                       experts_fn: Callable[[torch.Tensor, torch.Tensor], torch.Tensor], o: torch.Tensor,
+                       group=None) -> torch.Tensor:
+    """dispatch + run_local_experts + combine_back with the transfers
+    overlapping the grouped GEMMs.
+
+    The exchange runs in rounds. In round r (1 <= r < W) this rank sends its
+    rows for owner (rank + r) mod W and receives the rows of source
+    (rank - r) mod W; the return of round r sends that source its outputs
+    and receives this rank's outputs from owner (rank + r) mod W. The
+    rank's own rows (round 0) are computed first, while round 1's dispatch
+    is in flight; after that, the block of round r is computed while round
+    r + 1's dispatch and round r - 1's return are in flight. Every rank
+    posts the same sequence of paired send/receive groups (D1, D2, R1, D3,
+    R2, ...), so on a backend that runs one rank's transfers in order (NCCL)
+    every send meets its receive. Each block goes through experts_fn exactly
+    as in run_local_experts, so o[:rows_out] gets the same values as
+    dispatch, run_local_experts and combine_back give. Returns o."""
+    world = p.world
+    rank = dist.get_rank(group)
+    d = xp.shape[1]
+    send_off = [0]
+    for n in p.send_rows:
+        send_off.append(send_off[-1] + n)
+    keep = []   # tensors in flight must outlive their transfers
+
+    def src_of(r):
+        return (rank - r) % world
+
+    def dst_of(r):
+        return (rank + r) % world
+
+    def exchange(send_t, send_to, n_send, recv_t, recv_from, n_recv):
+        ops = []
+        if n_send:
+            ops.append(dist.P2POp(dist.isend, send_t, _peer(send_to, group), group))
+        if n_recv:
+            ops.append(dist.P2POp(dist.irecv, recv_t, _peer(recv_from, group), group))
+        keep.append((send_t, recv_t))
+        return dist.batch_isend_irecv(ops) if ops else []
+
+    recv_buf = {}
+
+    def post_dispatch(r):
+        dst, src = dst_of(r), src_of(r)
+        recv_buf[src] = xp.new_empty((p.recv_rows[src], d))
+        return exchange(xp[send_off[dst]:send_off[dst + 1]].contiguous(), dst, p.send_rows[dst],
+                        recv_buf[src], src, p.recv_rows[src])
+
+    def wait(works):
+        for w in works:
+            w.wait()
+
+    pending_d = post_dispatch(1) if world > 1 else []
+    # round 0: this rank's rows for its own experts
+    if p.send_rows[rank]:
+        o[send_off[rank]:send_off[rank + 1]] = experts_fn(xp[send_off[rank]:send_off[rank + 1]],
+                                                          p.block_offsets(rank))
+    pending_r = []
+    for r in range(1, world):
+        wait(pending_d)
+        pending_d = post_dispatch(r + 1) if r + 1 < world else []
+        src, dst = src_of(r), dst_of(r)
+        rows = recv_buf.pop(src)
+        out_blk = experts_fn(rows, p.block_offsets(src)) if p.recv_rows[src] else rows.new_empty((0, o.shape[1]))
+        recv_t = o[send_off[dst]:send_off[dst + 1]]
+        pending_r.append(exchange(out_blk.contiguous(), src, p.recv_rows[src], recv_t, dst, p.send_rows[dst]))
+    for works in pending_r:
+        wait(works)
     return o
 
 

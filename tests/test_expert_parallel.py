@@ -2,7 +2,8 @@
 
 Every rank routes and permutes its own token shard (with the oracle, on the
 CPU), then plan / dispatch / run_local_experts / combine_back move the rows
-to the ranks that own their experts and back. The local experts use only
+to the ranks that own their experts and back, and forward_overlapped does
+the same exchange in rounds that overlap the local experts. The local experts use only
 the owner's slice of the weights. Each rank's output must equal the oracle's
 single-process forward of its tokens with all the experts, drops included.
 """
@@ -74,9 +75,16 @@ def _worker(rank, world, port, q):
         ep.combine_back(expert_out, p, o)
         y = O.unpermute_combine(o.numpy(), perm.pos, r.gate)
 
+        # the overlapped exchange (rounds of paired sends and receives, one
+        # block's experts running while the next block moves) gives the same
+        # rows in the same places
+        o2 = torch.full((p.rows_out, d), float("nan"), dtype=torch.float64)
+        ep.forward_overlapped(xp, p, experts_fn, o2)
+        same = bool(torch.equal(o, o2))
+
         ref = O.moe_forward(xr, W_r, W1, W3, W2, k, CF)
         err = float(np.abs(y - ref.y).max() / max(1e-30, np.abs(ref.y).max()))
-        q.put((rank, err, int(perm.kept.sum()), int(ref.stats.dropped), p.rows_in))
+        q.put((rank, err, int(perm.kept.sum()), int(ref.stats.dropped), p.rows_in, same))
     finally:
         dist.destroy_process_group()
 
@@ -94,11 +102,12 @@ def test_expert_parallel_matches_single_process(world):
         pr.join(timeout=60)
         assert pr.exitcode == 0
     res.sort()
-    assert all(err < 1e-12 for _, err, _, _, _ in res), res
+    assert all(err < 1e-12 for _, err, _, _, _, _ in res), res
+    assert all(same for *_, same in res), res
     # some pairs were dropped by the per-rank capacity, and every kept row
     # was computed by exactly one owner
-    assert sum(dr for _, _, _, dr, _ in res) > 0
-    assert sum(kept for _, _, kept, _, _ in res) == sum(n for _, _, _, _, n in res)
+    assert sum(dr for _, _, _, dr, _, _ in res) > 0
+    assert sum(kept for _, _, kept, _, _, _ in res) == sum(n for _, _, _, _, n, _ in res)
 
 
 def test_expert_range_requires_an_even_split():
@@ -191,3 +200,56 @@ def test_library_experts_fn_keeps_one_workspace(monkeypatch, max_rows):
 def types_ns(T, d, d_ff, E, k):
     import types
     return types.SimpleNamespace(T=T, d=d, d_ff=d_ff, E=E, k=k)
+
+
+# rows per (source rank, expert) with empty pairs: rank 2 sends nothing,
+# owner 1 gets nothing from ranks 0 and 3, rank 3 keeps everything local
+_COUNTS = {0: [3, 0, 0, 0, 1, 2, 0, 0],
+           1: [0, 1, 0, 0, 0, 0, 2, 1],
+           2: [0, 0, 0, 0, 0, 0, 0, 0],
+           3: [0, 0, 0, 0, 0, 0, 4, 0]}
+
+
+def _edge_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        counts = _COUNTS[rank]
+        indptr = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int64)
+        n = int(indptr[-1])
+        xp = torch.arange(n * 4, dtype=torch.float64).reshape(n, 4) + 100.0 * rank
+        p = ep.plan(indptr, 8)
+        e_lo, _ = ep.expert_range(8, world, rank)
+
+        def experts_fn(block, offsets):
+            # expert e of this owner scales its rows by (global expert id + 1)
+            out = torch.empty_like(block)
+            for e in range(p.E_local):
+                s, t = int(offsets[e]), int(offsets[e + 1])
+                out[s:t] = block[s:t] * (e_lo + e + 1)
+            return out
+
+        o = torch.zeros((n, 4), dtype=torch.float64)
+        ep.combine_back(ep.run_local_experts(ep.dispatch(xp, p), p, experts_fn, 4), p, o)
+        o2 = torch.full((n, 4), float("nan"), dtype=torch.float64)
+        ep.forward_overlapped(xp, p, experts_fn, o2)
+        scale = torch.repeat_interleave(torch.arange(1, 9, dtype=torch.float64), torch.tensor(counts))
+        q.put((rank, bool(torch.equal(o, o2)), bool(torch.equal(o2, xp * scale[:, None]))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_overlapped_exchange_with_empty_pairs():
+    world = 4
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_edge_worker, args=(r, world, port, q)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    assert all(a and b for _, a, b in res), res

@@ -17,7 +17,9 @@ each owner's experts run by the library's grouped GEMMs.
   library_experts_fn (moe_experts on the owner's weight slice), combine_back
   returns them and moe_combine finishes the layer. Each rank's output must
   match, element by element, the oracle's single-process forward of its
-  tokens with all the experts, capacity drops included.
+  tokens with all the experts, capacity drops included; forward_overlapped
+  (the same exchange in rounds that overlap the experts) must put the same
+  expert outputs in the same rows.
 """
 
 import math
@@ -119,10 +121,15 @@ def _ep_worker(rank, world, port, q):
         y = torch.empty((Tr, d), dtype=torch.bfloat16, device=dev)
         moe.combine(p, o.to(dev), pos, gate, y)
         torch.cuda.synchronize()
+        # the overlapped exchange: each block's experts run on the GPU while
+        # the next block's rows move; the same rows in the same places
+        o2 = torch.full((Tr * k, d), float("nan"), dtype=torch.bfloat16)
+        ep.forward_overlapped(xp.cpu(), plan, lambda blk, offs: fn(blk.to(dev), offs).cpu(), o2)
+        same = bool(torch.equal(o[:plan.rows_out], o2[:plan.rows_out]))
         q.put((rank, y.float().cpu().numpy(), logits.cpu().numpy(), idx.cpu().numpy(), status,
-               plan.rows_in, int(indptr[-1].item()), None))
+               plan.rows_in, int(indptr[-1].item()), same, None))
     except Exception as e:
-        q.put((rank, None, None, None, None, None, None, repr(e)))
+        q.put((rank, None, None, None, None, None, None, None, repr(e)))
     finally:
         dist.destroy_process_group()
 
@@ -179,8 +186,9 @@ def test_expert_parallel_forward_with_library_experts():
     x, W_r, W1, W3, W2 = _layer()
     W = {n: {e: w[e].float().numpy() for e in range(E)} for n, w in (("W1", W1), ("W3", W3), ("W2", W2))}
     total_in, total_out, drops = 0, 0, 0
-    for rank, y, logits, idx, status, rows_in, rows_out, _ in res:
+    for rank, y, logits, idx, status, rows_in, rows_out, same, _ in res:
         assert status == 0
+        assert same, f"rank {rank}: the overlapped exchange differs from dispatch / combine_back"
         lo, hi = parallel.shard_range(T, 2, rank)
         ref = O.moe_forward(x[lo:hi].float().numpy(), None, W["W1"], W["W3"], W["W2"], k, CF, logits=logits,
                             key_dtype=np.float32)
