@@ -153,12 +153,10 @@ GridSplit grid_split_of(const moe_problem& p) {
         const char* v = std::getenv("MOE_SMALL_CTAS");
         return v != nullptr ? std::atoi(v) : -1;
     }();
-    // measured on the DeepSeek-shaped layer (alternating runs on one box):
-    // 7.43-7.49 ms per step with the split against 7.39-7.44 ms without, so
-    // the split is opt-in (MOE_SMALL_CTAS=n > 0), not the default
-    // both two-class schedules measured no faster than the single order on
-    // the DeepSeek-shaped layer (alternating runs on one box: 7.82 / 7.75 ms
-    // without, 7.89 / 7.86 ms interleaved), so both are opt-in
+    // Both two-class schedules are opt-in: on the DeepSeek-shaped layer
+    // (alternating runs on one box) the grid split (MOE_SMALL_CTAS=n > 0)
+    // measured 7.43-7.49 ms per step against 7.39-7.44 ms without, the
+    // interleaved order (MOE_INTERLEAVE=1) 7.86-7.89 ms against 7.75-7.82 ms.
     static const bool interleave = [] {
         const char* v = std::getenv("MOE_INTERLEAVE");
         return v != nullptr && v[0] == '1';
