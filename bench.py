@@ -26,6 +26,7 @@ and (rank 0, N = 1) the CPU oracle timed on a bounded token sample.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -74,9 +75,14 @@ def down_flops(cfg, rows):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """nvidia-smi samples of SM clock and throttle reasons while running.
 
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+    Each sample carries nvidia-smi's own timestamp; mark() and stop() take
+    the host time at the two ends of the timed region, and only the samples
+    inside it are summarised (the sampler starts before the region and
+    stops after it, and an idle GPU's clock says nothing about the work)."""
+
+    FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
               "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
               "clocks_event_reasons.sw_power_cap"]
     REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -86,12 +92,13 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.thread = None
+        self.t0 = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
-                 "-lms", "50", "-i", str(self.gpu_index)],
+                 "-lms", "20", "-i", str(self.gpu_index)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -104,9 +111,16 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def mark(self):
+        """The timed region starts now."""
+        self.t0 = time.time()
+
     def stop(self):
+        """Summary of the samples taken since mark() (all samples when mark()
+        was not called)."""
         if self.proc is None:
             return None
+        t1 = time.time()
         time.sleep(0.1)
         self.proc.terminate()
         try:
@@ -115,21 +129,31 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
-        sm, mx, reasons = [], None, set()
-        for ln in self.lines:
+        return self.summarise(self.lines, self.t0, t1)
+
+    @classmethod
+    def summarise(cls, lines, t0=None, t1=None):
+        sm, mx, reasons, outside = [], None, set(), 0
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != len(self.FIELDS):
+            if len(parts) != len(cls.FIELDS):
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk = float(parts[1])
+                mx = float(parts[2])
             except ValueError:
                 continue
-            for name, val in zip(self.REASONS, parts[3:]):
+            if t0 is not None and not (t0 <= ts <= t1):
+                outside += 1
+                continue
+            sm.append(clk)
+            for name, val in zip(cls.REASONS, parts[4:]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
         if not sm:
-            return None
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0,
+                    "note": "no nvidia-smi sample fell inside the timed region"}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
@@ -355,6 +379,7 @@ def time_steps(step, steps, warmup, dev, stream, flush, barrier, local_rank):
     sampler.start()
     torch.cuda.synchronize(dev)
     barrier()
+    sampler.mark()
     evs = []
     for _ in range(steps):
         flush()
@@ -551,7 +576,10 @@ def main():
 
     # ---- end to end through host buffers ----
     x_host = x.cpu().pin_memory()
-    e2e_ms = e2e_pipelined(layer, x_host, dev, stream, args.steps, before_timed=barrier)
+    e2e_sampler = ClockSampler(gpu_index_for(local_rank))
+    e2e_sampler.start()
+    e2e_ms = e2e_pipelined(layer, x_host, dev, stream, args.steps, before_timed=barrier, sampler=e2e_sampler)
+    e2e_clocks = e2e_sampler.stop()
     barrier()
     t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -577,7 +605,8 @@ def main():
                 "d2h_bytes_per_step": nbytes, "ms_per_step": float(t.item()) / args.steps,
                 "schedule": "double-buffered: the copy-in of step i+1 and the copy-out of step i-1 run on "
                             "their own streams beside the forward of step i; one timed region from the "
-                            "first copy-in to the last copy-out; no L2 flush (the weights exceed L2)"},
+                            "first copy-in to the last copy-out; no L2 flush (the weights exceed L2)",
+                "clocks": e2e_clocks},
         "gpu_launches": launches_per_forward(cfg, args.pad_rows) * args.steps,
         "clocks": clocks,
         "stages_ms": stages,
@@ -612,7 +641,7 @@ def main():
         print(json.dumps(line), flush=True)
 
 
-def e2e_pipelined(layer, x_host, dev, stream, steps, before_timed=None):
+def e2e_pipelined(layer, x_host, dev, stream, steps, before_timed=None, sampler=None):
     """Milliseconds for `steps` forwards through host buffers, as a serving
     loop runs them: each step copies its input rows from pinned host memory
     and its output rows back to pinned host memory; the copy-in of step i+1
@@ -667,6 +696,8 @@ def e2e_pipelined(layer, x_host, dev, stream, steps, before_timed=None):
     run(3)
     if before_timed is not None:
         before_timed()
+    if sampler is not None:
+        sampler.mark()
     return run(steps)
 
 
@@ -731,6 +762,7 @@ def run_train(args, cfg, moe, L, dev, stream, flush):
         graphs["step"].replay()
     sampler = ClockSampler(gpu_index_for(0))
     sampler.start()
+    sampler.mark()
     step_ms = timed(graphs["step"], args.steps)
     clocks = sampler.stop()
     fwd_ms = timed(graphs["fwd"], max(3, args.steps // 3))

@@ -71,3 +71,22 @@ def test_every_other_config_is_measured_by_default():
 def test_every_gemm_variant_has_a_kernel_name():
     from mixture_experts_layer_62_b200 import GEMM_VARIANTS
     assert set(GEMM_VARIANTS.values()) <= set(bench.KERNEL_NAMES)
+
+
+def test_clock_samples_are_taken_inside_the_timed_region_only():
+    # nvidia-smi lines (timestamp first) before, inside and after the timed
+    # region: only the ones inside count, so idle samples around the region
+    # cannot hide a power-capped clock under load
+    import datetime
+    t = datetime.datetime(2026, 1, 2, 3, 4, 5)
+    rows = [(1965, "Not Active"), (1965, "Not Active"), (1500, "Active"), (1440, "Active"), (1965, "Not Active")]
+    lines = []
+    for i, (clk, cap) in enumerate(rows):
+        ts = (t + datetime.timedelta(milliseconds=20 * i)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        lines.append(f"{ts}, {clk}, 1965, 900.0, Not Active, Not Active, Not Active, {cap}")
+    at = lambda ms: (t + datetime.timedelta(milliseconds=ms)).timestamp()
+    inside = bench.ClockSampler.summarise(lines, at(30), at(70))
+    assert inside["samples"] == 2 and inside["sm_mhz"] == 1470.0 and inside["reasons"] == ["sw_power_cap"]
+    assert bench.ClockSampler.summarise(lines)["samples"] == 5
+    none = bench.ClockSampler.summarise(lines, at(200), at(300))
+    assert none["samples"] == 0 and none["sm_mhz"] is None
