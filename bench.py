@@ -29,6 +29,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -444,20 +445,30 @@ def measure_extra(name, args, moe, dev, stream, flush, peaks, peak_src, weight_c
     with torch.cuda.graph(graph):
         layer(x)
     torch.cuda.synchronize(dev)
-    total_ms, clocks = time_steps(graph.replay, args.steps, args.warmup, dev, stream, flush, lambda: None, 0)
+    # at least about 100 ms of timed steps, so that the 20 ms clock samples
+    # fall inside the timed region even for a decode step of a tenth of a ms
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(3):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    est_ms = max(e0.elapsed_time(e1) / 3, 1e-3)
+    steps = min(2000, max(args.steps, int(math.ceil(100.0 / est_ms))))
+    total_ms, clocks = time_steps(graph.replay, steps, args.warmup, dev, stream, flush, lambda: None, 0)
     st = layer.read_stats()
     if st.status != moe.MOE_OK:
         raise SystemExit(f"{name}: device status {st.status}: {moe.error_string(st.status)}")
-    ms = total_ms / args.steps
+    ms = total_ms / steps
     stages = breakdown(moe, p, cfg, L, dev, stream, flush, iters=max(3, min(10, args.steps)))
-    out = {"ms_per_step": ms, "tokens_per_s": cfg["T"] / (ms / 1e3), "T": cfg["T"],
+    out = {"ms_per_step": ms, "steps": steps, "tokens_per_s": cfg["T"] / (ms / 1e3), "T": cfg["T"],
            "roofline": workload_roofline(cfg, name, stages, st, peaks, peak_src, moe.gemm_variant(p)),
            "pass_roofline": pass_roofline(cfg, st, ms, peaks), "stages_ms": stages, "clocks": clocks,
            "routing": {"rows": st.rows, "dropped": st.dropped, "capacity": st.capacity, "l_aux": st.l_aux,
                        "max_over_mean": st.max_over_mean, "experts_touched": touched_experts(st),
                        "counts": st.counts if cfg["E"] <= 16 else None,
                        "kept": st.kept if cfg["E"] <= 16 else None},
-           "gpu_launches": launches_per_forward(cfg) * args.steps}
+           "gpu_launches": launches_per_forward(cfg) * steps}
     if cfg["T"] <= 64:
         out["forward_hbm_gbs"] = decode_bytes(cfg, st) / (ms / 1e3) / 1e9
         out["forward_hbm_frac"] = out["forward_hbm_gbs"] / peaks["hbm_gbs"]
