@@ -353,6 +353,10 @@ SMALL = [
     dict(T=600, d=192, d_ff=320, E=1, k=1, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     # 32 or more experts, many small groups
     dict(T=400, d=256, d_ff=256, E=32, k=4, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=0),
+    # the largest expert count (MOE_MAX_E: tensor-core router, 512 groups)
+    # and the largest k (MOE_MAX_K)
+    dict(T=300, d=256, d_ff=128, E=512, k=8, cf=0.0, dtype="bf16", bias_mode=2, d_ff_shared=128),
+    dict(T=100, d=128, d_ff=128, E=64, k=16, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     dict(T=900, d=128, d_ff=384, E=64, k=6, cf=0.8, dtype="bf16", bias_mode=1, d_ff_shared=128, gate=1),
     # padded (MegaBlocks) layout: every expert's rows rounded up to 128 or 64
     dict(T=300, d=256, d_ff=384, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0, pad=128),
