@@ -48,7 +48,9 @@ from mixture_experts_layer_62_b200 import inputs  # noqa: E402
 METRIC = "MoE-layer fwd tokens/s & TFLOP/s vs bf16 peak; small-batch decode HBM GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-GEMM_SRC = os.path.join(ROOT, "mixture_experts_layer_62_b200", "csrc", "gemm_sm100.cu")
+CSRC = os.path.join(ROOT, "mixture_experts_layer_62_b200", "csrc")
+GEMM_SRC = os.path.join(CSRC, "gemm_sm100.cu")
+GEMV_SRC = os.path.join(CSRC, "gemv_sm100.cu")
 
 
 def load_peaks():
@@ -174,7 +176,8 @@ def traffic_for(kernel, workload):
         return None
     with open(TRAFFIC_FILE) as fh:
         d = json.load(fh)
-    src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
+    src = GEMV_SRC if kernel.startswith("gemv") else GEMM_SRC
+    src_hash = hashlib.sha256(open(src, "rb").read()).hexdigest()
     ent = d.get(kernel, {}).get(workload)
     if not ent or ent.get("source_sha256") != src_hash:
         return None
@@ -257,6 +260,7 @@ KERNEL_NAMES = {
     "interleaved": ("tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU, small groups interleaved)",
                     "tc_grouped_gemm_swiglu"),
     "simt": ("simt_gemm_kernel<true> (grouped GEMM 1/3 + SwiGLU, CUDA cores)", "simt_gemm_swiglu"),
+    "gemv": ("gemv_swiglu_kernel (grouped GEMM 1/3 + SwiGLU as weight-streaming GEMVs)", "gemv_swiglu"),
 }
 
 

@@ -344,14 +344,19 @@ long long moe_set_wait_limit(long long ns);
  * cores), MOE_GEMM_INTERLEAVED (single-CTA tiles; with 32 or more experts
  * averaging fewer than 512 rows, the tiles of the groups of at most 128
  * rows are spread evenly through the others' and load their weights with an
- * evict-first L2 policy); a negative MOE_ERR_* code if p is invalid. Host
- * only. */
+ * evict-first L2 policy), MOE_GEMM_GEMV (bf16 batches of at most 8
+ * permuted rows and no shared expert: GEMM 1/3 + SwiGLU as weight-streaming
+ * GEMVs, the weights copied through shared memory, the K range split over
+ * the warps of each CTA, each CTA one equal, contiguous range of 8-column
+ * output groups; GEMM 2 as split-K tiles); a negative MOE_ERR_* code if p is
+ * invalid. Host only. */
 #define MOE_GEMM_SINGLE      0
 #define MOE_GEMM_PAIR        1
 #define MOE_GEMM_GRID_SPLIT  2
 #define MOE_GEMM_SPLIT_K     3
 #define MOE_GEMM_SIMT        4
 #define MOE_GEMM_INTERLEAVED 5
+#define MOE_GEMM_GEMV        6
 int moe_gemm_variant(const moe_problem* p);
 
 /* Debug build. The library also builds as libmoe_debug.so (compiled with
@@ -359,14 +364,16 @@ int moe_gemm_variant(const moe_problem* p);
  * checks that record MOE_ERR_BOUNDS in the call's status word and skip the
  * access instead of faulting: the group offsets handed to the expert stages
  * (non-decreasing, within the permuted rows; a violation empties the tile
- * schedule, so no tile runs), every output row a grouped GEMM stores, and
+ * schedule, so no tile runs; the GEMV kernel skips the groups whose offsets
+ * are out of range, and so does the release build), every output row a
+ * grouped GEMM stores, and
  * every permuted row the combine reads (moe_forward's status word; the
  * standalone moe_combine has none, so it only skips). The Python binding
  * loads it when MOE_LIBRARY=debug. */
 
 /* Kernel-selection overrides, read once per process from the environment
  * (for measurement and tests; results are the same either way, up to the
- * summation order inside one MMA):
+ * order of the fp32 sums):
  *   MOE_CTA_PAIR=0   the grouped GEMMs never use CTA pairs (256-row tiles on
  *                    two SMs); by default they do when the experts average
  *                    at least 512 rows (bf16 inference, no split-K).
@@ -377,7 +384,11 @@ int moe_gemm_variant(const moe_problem* p);
  *                    DeepSeek-shaped layer).
  *   MOE_INTERLEAVE=1 for the same shapes, the interleaved two-class order
  *                    (MOE_GEMM_INTERLEAVED above; also measured no faster
- *                    there). Without either, one order in expert order. */
+ *                    there). Without either, one order in expert order.
+ *   MOE_GEMV=0       decode-sized batches use the split-K tensor-core tiles
+ *                    (MOE_GEMM_SPLIT_K) for GEMM 1/3 too.
+ *   MOE_GEMV_ROWS=n  the GEMV path takes batches of at most n permuted rows
+ *                    (default and largest 8). */
 
 #ifdef __cplusplus
 }

@@ -130,7 +130,7 @@ def __getattr__(name):
     raise AttributeError(name)
 
 
-GEMM_VARIANTS = {0: "single", 1: "pair", 2: "grid_split", 3: "split_k", 4: "simt", 5: "interleaved"}
+GEMM_VARIANTS = {0: "single", 1: "pair", 2: "grid_split", 3: "split_k", 4: "simt", 5: "interleaved", 6: "gemv"}
 
 
 def gemm_variant(p: Problem) -> str:

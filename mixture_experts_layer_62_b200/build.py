@@ -30,7 +30,8 @@ DEBUG_BUILD_DIR = os.path.join(ROOT, "_build_debug")
 DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libmoe_debug.so")
 
 SOURCES = ["api.cu", "route.cu", "permute.cu", "combine.cu", "gemm_simt.cu", "gemm_sm100.cu",
-           "permute_noalloc.cu", "route_small.cu", "gemm_bwd_sm100.cu", "bwd.cu"]
+           "permute_noalloc.cu", "route_small.cu", "gemm_bwd_sm100.cu", "bwd.cu",
+           "gemv_sm100.cu"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
           "--expt-relaxed-constexpr"]

@@ -139,6 +139,29 @@ bool split_allowed(const moe_problem& p) {
            (long long)p.T * p.k <= kSplitMaxRows;
 }
 
+// Decode-sized batches (at most 8 permuted rows by default, bf16, no shared
+// expert) run GEMM 1/3 as weight-streaming GEMVs; GEMM 2 keeps the split-K
+// tensor-core tiles. Measured against split-K tiles for both (decode at
+// d = 4096, d_ff = 14336, top-2 of 8): 3 % faster per step at one token,
+// 1.4 % at two, 0.5 % at four, 2.7 % slower at eight. MOE_GEMV=0 keeps the
+// split-K tiles; MOE_GEMV_ROWS=n lowers the row limit (measurement; n <= 8).
+bool gemv_on(const moe_problem& p) {
+    static const bool enabled = [] {
+        const char* v = std::getenv("MOE_GEMV");
+        return !(v != nullptr && v[0] == '0');
+    }();
+    static const int rows = [] {
+        const char* v = std::getenv("MOE_GEMV_ROWS");
+        const int n = v != nullptr ? std::atoi(v) : 8;
+        return n < 0 ? 0 : (n > kGemvMaxRows ? kGemvMaxRows : n);
+    }();
+    return enabled && split_allowed(p) && (long long)p.T * p.k <= rows;
+}
+
+// Split-K tensor-core tiles (GEMM 2 of every small batch; GEMM 1/3 where the
+// GEMVs do not take it).
+bool split_k_on(const moe_problem& p) { return split_allowed(p); }
+
 bool use_pair_tiles(const moe_problem& p) {
     static const bool enabled = [] {
         const char* v = std::getenv("MOE_CTA_PAIR");
@@ -278,14 +301,39 @@ int run_logits(const moe_problem* p, const void* x, const void* W_r, float* logi
     return MOE_OK;
 }
 
+// Arguments of a GEMV launch. group_rows: the most rows one expert can
+// hold (T when the offsets come from the router, which picks distinct experts
+// per token; 0: any split of the T*k rows).
+GemvLaunch gemv_launch(const moe_problem* p, const int32_t* indptr, const void* A, const void* B0, const void* B1,
+                       void* out, int N, int K, int group_rows, int32_t* status) {
+    GemvLaunch g = {};
+    g.indptr = indptr;
+    g.E = p->E;
+    g.A = A;
+    g.B0 = B0;
+    g.B1 = B1;
+    g.out = out;
+    g.N = N;
+    g.K = K;
+    g.rows_max = (int)permuted_rows(*p);
+    g.max_group_rows = group_rows > 0 && group_rows < g.rows_max ? group_rows : g.rows_max;
+    g.grid = device_sm_count();
+    g.status = status;
+    return g;
+}
+
 // Grouped GEMM 1/3 with the SwiGLU epilogue (and the shared expert's).
 int run_up(const moe_problem* p, const void* xp, const int32_t* indptr, const int32_t* tiles13, const void* W1,
            const void* W3, const void* x, const void* Ws1, const void* Ws3, void* h, void* hs, int32_t* status,
            cudaStream_t st, float* part13 = nullptr, int32_t* sem13 = nullptr, bool sched_early = true,
-           void* ab = nullptr, void* ab_s = nullptr) {
+           void* ab = nullptr, void* ab_s = nullptr, int group_rows = 0) {
     const int has_shared = p->d_ff_shared > 0 ? 1 : 0;
     const int rows = p->T * p->k;
     const int arows = (int)permuted_rows(*p);   // rows of the permuted buffers
+    if (gemv_on(*p)) {
+        CK(launch_gemv_swiglu(gemv_launch(p, indptr, xp, W1, W3, h, p->d_ff, p->d, group_rows, status), st));
+        return MOE_OK;
+    }
     if (p->dtype == MOE_DTYPE_BF16) {
         TcArgs a = {};
         a.mode = TC_SWIGLU;
@@ -382,9 +430,9 @@ int run_experts(const moe_problem* p, const void* xp, const int32_t* indptr, con
                 const void* Ws1, const void* Ws3, const void* Ws2, void* h, void* hs, void* o, void* s,
                 int32_t* status, cudaStream_t st, float* part13 = nullptr, float* part2 = nullptr,
                 int32_t* sem13 = nullptr, int32_t* sem2 = nullptr, bool sched_early = true, void* ab = nullptr,
-                void* ab_s = nullptr) {
+                void* ab_s = nullptr, int group_rows = 0) {
     int rc = run_up(p, xp, indptr, tiles13, W1, W3, x, Ws1, Ws3, h, hs, status, st, part13, sem13, sched_early, ab,
-                    ab_s);
+                    ab_s, group_rows);
     if (rc != MOE_OK) return rc;
     return run_down(p, h, indptr, tiles2, W2, hs, Ws2, o, s, status, st, part2, sem2);
 }
@@ -419,7 +467,7 @@ StageSplit stage_split(const moe_problem* p, const Layout& L, void* ws, int32_t*
     s.sched.gsplit = grid_split_of(*p);
     s.sched.rows_max = (int)permuted_rows(*p);
     s.sched.status = status;
-    if (!split_allowed(*p)) return s;
+    if (!split_k_on(*p)) return s;
     int tile_m, nt13, nt2, nt13s, nt2s;
     schedule_sizes(p, tile_m, nt13, nt2, nt13s, nt2s);
     s.sched.split_on = 1;
@@ -462,6 +510,7 @@ int moe_gemm_variant(const moe_problem* p) {
     const int rc = check_problem(p);
     if (rc != MOE_OK) return -rc;
     if (p->dtype != MOE_DTYPE_BF16) return MOE_GEMM_SIMT;
+    if (gemv_on(*p)) return MOE_GEMM_GEMV;
     if (split_allowed(*p)) return MOE_GEMM_SPLIT_K;
     if (use_pair_tiles(*p)) return MOE_GEMM_PAIR;
     {
@@ -720,7 +769,7 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     int32_t* tiles13 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles13));
     int32_t* tiles2 = reinterpret_cast<int32_t*>(wsp(workspace, L.tiles2));
 
-    const bool split = split_allowed(*p);
+    const bool split = split_k_on(*p);
     int32_t* sem = split ? reinterpret_cast<int32_t*>(wsp(workspace, L.sem)) : nullptr;
     void* xp = wsp(workspace, L.xp);
     const bool small = small_route_ok(*p);
@@ -787,7 +836,7 @@ int moe_forward(const moe_problem* p, const void* x, const void* W_r, const floa
     rc = run_experts(p, xp, indptr, tiles13, tiles2, W1, W3, W2, x, Ws1, Ws3, Ws2, h, hs, o, s, status, st, part13,
                      part2, sem, sem ? sem + L.sem13_n : nullptr, /*sched_early=*/!small,
                      p->train ? wsp(workspace, L.ab) : nullptr,
-                     (p->train && shared) ? wsp(workspace, L.abs) : nullptr);
+                     (p->train && shared) ? wsp(workspace, L.abs) : nullptr, /*group_rows=*/p->T);
     if (rc != MOE_OK) return rc;
     CK(launch_combine(p->dtype, o, pos, gate, s, out, p->T, p->d, p->k, (int)permuted_rows(*p), status, st));
     return MOE_OK;

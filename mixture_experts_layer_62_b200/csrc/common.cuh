@@ -256,6 +256,24 @@ struct GroupedArgs {
 };
 cudaError_t launch_simt_gemm(bool swiglu, const GroupedArgs& a, cudaStream_t st);
 
+// Decode-sized bf16 grouped GEMM 1/3 + SwiGLU as weight-streaming GEMVs
+// (groups of at most kGemvMaxRows rows, no shared expert): one contiguous
+// range of 8-column output groups per CTA, K split over the CTA's warps.
+constexpr int kGemvMaxRows = 8;
+struct GemvLaunch {
+    const int32_t* indptr;   // [E+1] (device)
+    int E;
+    const void* A;           // [rows_max, K] bf16: the permuted rows
+    const void* B0;          // [E, N, K] bf16: W1
+    const void* B1;          // [E, N, K] bf16: W3
+    void* out;               // [rows_max, N] bf16: H
+    int N, K, rows_max;
+    int max_group_rows;      // largest group the offsets can hold (<= kGemvMaxRows)
+    int grid;                // CTAs (the SM count)
+    int32_t* status;
+};
+cudaError_t launch_gemv_swiglu(const GemvLaunch& a, cudaStream_t st);
+
 // bf16 grouped GEMM on tcgen05 tensor cores (sm_100a). Tile 128 x 256.
 constexpr int kTcTileM = 128;
 constexpr int kTcPairTileM = 256;   // rows of a CTA-pair tile

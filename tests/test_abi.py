@@ -173,7 +173,8 @@ def test_binding_refuses_cpu_tensors():
 
 def test_gemm_variant_follows_the_shape():
     # host-side selection only (no launch): CTA pairs for prefill-sized
-    # experts, split-K for decode-sized batches, CUDA cores for fp32
+    # experts, GEMVs for GEMM 1/3 of decode batches of at most 8 rows, split-K
+    # up to 128 rows, CUDA cores for fp32
     from mixture_experts_layer_62_b200 import inputs
 
     def variant(name, **kw):
@@ -182,7 +183,10 @@ def test_gemm_variant_follows_the_shape():
                                             c["bias_mode"], c["d_ff_shared"], train=kw.get("train", 0)))
     assert variant("mixtral_prefill") == "pair"
     assert variant("skewed_capacity") == "pair"
-    assert variant("decode_t1") == "split_k"
+    assert variant("decode_t1") == "gemv"
+    assert variant("decode_t4") == "gemv"                          # 8 rows
+    assert variant("decode_t8") == "split_k"                       # 16 rows
+    assert variant("decode_t1", d_ff_shared=1024) == "single"      # a shared expert: ordinary tiles
     assert variant("toy_fp32") == "simt"
     assert variant("mixtral_prefill", T=1000) == "single"          # 250 rows per expert
     assert variant("mixtral_prefill", d_ff=14336, train=1) == "single"

@@ -3,8 +3,7 @@ checks that turn an out-of-range index into MOE_ERR_BOUNDS instead of a fault.
 
 The debug library is loaded in a child process (MOE_LIBRARY=debug). There:
   * whole forwards on valid inputs (the CTA-pair and single-CTA kernels, the
-    split-K decode path after either router) give the release library's bits
-    and MOE_OK;
+    split-K and GEMV decode paths) give the release library's bits and MOE_OK;
   * the expert stage handed group offsets that decrease, or that end past
     the permuted rows, records MOE_ERR_BOUNDS, schedules no tile and writes
     nothing: every row of the output keeps its sentinel value.
@@ -31,7 +30,7 @@ DEV = "cuda"
 FORWARDS = [dict(T=2048, d=256, d_ff=384, E=4, k=2, cf=0.0),      # CTA pairs
             dict(T=300, d=256, d_ff=384, E=8, k=2, cf=0.6),       # single-CTA tiles, capacity drops
             dict(T=40, d=512, d_ff=512, E=8, k=2, cf=0.0),        # split-K, general router
-            dict(T=4, d=512, d_ff=512, E=8, k=2, cf=0.0)]         # split-K, small-batch router
+            dict(T=4, d=512, d_ff=512, E=8, k=2, cf=0.0)]         # GEMVs, small-batch router
 
 
 def _layer(c, seed):
@@ -108,7 +107,7 @@ def test_debug_build_matches_release_and_catches_bad_offsets(tmp_path):
         assert int(dbg[f"status{i}"][0]) == moe.MOE_OK
         assert str(dbg[f"variant{i}"][0]) == str(rel[f"variant{i}"][0])
         assert np.array_equal(dbg[f"y{i}"], rel[f"y{i}"]), i
-    assert {str(rel[f"variant{i}"][0]) for i in range(len(FORWARDS))} == {"pair", "single", "split_k"}
+    assert {str(rel[f"variant{i}"][0]) for i in range(len(FORWARDS))} == {"pair", "single", "split_k", "gemv"}
     for name in ("decreasing", "past_rows"):
         assert int(dbg[f"status_{name}"][0]) == moe.MOE_ERR_BOUNDS, name
         assert bool(dbg[f"untouched_{name}"][0]), name

@@ -229,9 +229,10 @@ def test_padded_forward_equals_dense():
     ("bf16", 256, 384, [0, 1, 5, 31, 32, 33, 64, 65, 96, 97, 128, 129, 200, 300, 0, 7] + [3] * 16, 128, 800),
     ("bf16", 512, 256, [2, 40, 129, 700, 17, 0, 1, 90] * 4, 0, 2000),
     ("bf16", 256, 14336, [2500, 3, 7] + [1] * 29, 0, 10),
-    # at most 16 permuted rows, no shared expert (split K over CTAs): one- to
-    # sixteen-row groups, empty groups, K = 64 (a single K-block to split),
-    # N = 64 (fewer output tiles than CTAs)
+    # at most 16 permuted rows, no shared expert: GEMM 1/3 as weight-streaming
+    # GEMVs up to 8 rows (one- to eight-row groups, empty groups, K = 64: one
+    # half-size item per row and fewer items than K warps, N = 64: fewer
+    # output groups than CTAs), split-K tiles above
     ("bf16", 512, 384, [0, 3, 0, 5], 0, 4),
     ("bf16", 256, 512, [16], 0, 16),
     ("bf16", 64, 128, [3, 0, 9, 4], 0, 8),
@@ -548,7 +549,7 @@ def test_stages_compose_to_forward():
     dict(T=4, d=512, d_ff=512, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     dict(T=40, d=512, d_ff=512, E=8, k=2, cf=0.0, dtype="bf16", bias_mode=0, d_ff_shared=0),
     dict(T=600, d=256, d_ff=384, E=16, k=4, cf=0.8, dtype="bf16", bias_mode=1, d_ff_shared=128),
-], ids=["decode_split_t4_pdl", "decode_split_t40_pdl", "general_pdl"])
+], ids=["decode_gemv_pdl", "decode_split_pdl", "general_pdl"])
 def test_forward_captures_in_a_cuda_graph(cfg):
     # moe_forward is asynchronous and allocation-free: captured once and
     # replayed, it gives the eager call's bits
