@@ -388,7 +388,11 @@ int moe_gemm_variant(const moe_problem* p);
  *   MOE_GEMV=0       decode-sized batches use the split-K tensor-core tiles
  *                    (MOE_GEMM_SPLIT_K) for GEMM 1/3 too.
  *   MOE_GEMV_ROWS=n  the GEMV path takes batches of at most n permuted rows
- *                    (default and largest 8). */
+ *                    (default and largest 8).
+ *   MOE_ROUTER_MMA=0 the fused bf16 router (up to 63 experts) forms its
+ *                    logits with fp32 FMAs instead of the warp-level MMA
+ *                    (bf16 products, fp32 sums; the default where W_r^T of
+ *                    eight experts fits its shared memory, d <= 5344). */
 
 #ifdef __cplusplus
 }

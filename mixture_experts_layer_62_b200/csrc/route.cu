@@ -6,8 +6,12 @@
 // the raw z), §3.2 (f_i and P_i of the balance loss); "Stanford CS336 Lecture
 // 04" §2.3.3c (bias added to the softmax score). Router arithmetic is fp32
 // ("Lecture 21 · LLM: Mixture-of-Experts" §7.1: the router runs in fp32).
+#include <algorithm>
+#include <cstdlib>
+
 #include "common.cuh"
 #include "tc_common.cuh"
+#include "warp_mma.cuh"
 
 namespace moe {
 
@@ -317,6 +321,168 @@ __device__ __forceinline__ void sel_token(const float (&zin)[EPL], int t, int bi
     }
 }
 
+// Q tokens at once (lane l holds the logits of experts l + 32 i of each):
+// per token the same arithmetic as sel_token (compact form) in the same
+// order, with the Q tokens' steps interleaved so that their shuffle chains
+// overlap instead of running one token after another. Only tokens q < nt
+// are counted and emitted (the others run on zeros); the statistics take
+// the tokens in order, so the bits are those of sel_token called token by
+// token.
+template <int EPL, int Q>
+__device__ __forceinline__ void sel_tokens(const float (&zin)[Q][EPL], int nt, int t0, int bias_mode, int gate_mode,
+                                           int kk, int E, int k, int lane, SelAcc<EPL>& a, int* cnt,
+                                           int32_t* __restrict__ idx_out, float* __restrict__ gate_out) {
+    float z[Q][EPL], ex[Q][EPL], key[Q][EPL], m[Q], s[Q], inv_s[Q];
+#pragma unroll
+    for (int q = 0; q < Q; ++q)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            z[q][i] = e < E ? (q < nt ? zin[q][i] : 0.f) : -INFINITY;
+        }
+    // full softmax over all E raw logits
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+        m[q] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) m[q] = fmaxf(m[q], z[q][i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int q = 0; q < Q; ++q) m[q] = fmaxf(m[q], __shfl_xor_sync(0xffffffffu, m[q], o));
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+        s[q] = 0.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            ex[q][i] = e < E ? expf(z[q][i] - m[q]) : 0.f;
+            s[q] += ex[q][i];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int q = 0; q < Q; ++q) s[q] += __shfl_xor_sync(0xffffffffu, s[q], o);
+#pragma unroll
+    for (int q = 0; q < Q; ++q) inv_s[q] = 1.f / s[q];
+    // router statistics
+    {
+        float pz[Q], z1[Q], z2[Q];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            pz[q] = 0.f; z1[q] = -INFINITY; z2[q] = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                if (lane + 32 * i < E) {
+                    pz[q] += ex[q][i] * z[q][i];
+                    if (z[q][i] > z1[q]) { z2[q] = z1[q]; z1[q] = z[q][i]; } else if (z[q][i] > z2[q]) { z2[q] = z[q][i]; }
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int q = 0; q < Q; ++q) pz[q] += __shfl_xor_sync(0xffffffffu, pz[q], o);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+                const float o1 = __shfl_xor_sync(0xffffffffu, z1[q], o);
+                const float o2 = __shfl_xor_sync(0xffffffffu, z2[q], o);
+                const float hi = fmaxf(z1[q], o1);
+                z2[q] = fmaxf(fminf(z1[q], o1), fmaxf(z2[q], o2));
+                z1[q] = hi;
+            }
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            if (q < nt) {
+                const float pzq = pz[q] * inv_s[q];
+                const float lse = m[q] + logf(s[q]);
+                a.ex_z += lse * lse;
+                a.ex_h += lse - pzq;
+                a.ex_g += (1.f - expf(z2[q] - m[q])) * inv_s[q];
+            }
+        }
+    }
+    unsigned valid = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i < E) valid |= 1u << i;
+#pragma unroll
+    for (int q = 0; q < Q; ++q)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const float p = ex[q][i] * inv_s[q];
+            if (q < nt && ((valid >> i) & 1u)) a.psum[i] += p;
+            key[q][i] = bias_mode == MOE_BIAS_NONE ? z[q][i]
+                      : bias_mode == MOE_BIAS_LOGIT ? z[q][i] + a.b[i]
+                      : p + a.b[i];
+        }
+    // top-k: k rounds of a warp arg-max over (key desc, index asc)
+    unsigned taken[Q];
+    float zsel[Q][MOE_MAX_K];
+    int esel[Q][MOE_MAX_K];
+#pragma unroll
+    for (int q = 0; q < Q; ++q) taken[q] = 0;
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) {
+        float bk[Q], bz[Q];
+        int be[Q];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            bk[q] = -INFINITY; bz[q] = 0.f; be[q] = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const bool ok = ((valid >> i) & 1u) && !((taken[q] >> i) & 1u);
+                if (ok && (key[q][i] > bk[q] || be[q] == 0x7fffffff)) {
+                    bk[q] = key[q][i]; be[q] = lane + 32 * i; bz[q] = z[q][i];
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int q = 0; q < Q; ++q) {
+                const float ok_ = __shfl_xor_sync(0xffffffffu, bk[q], o);
+                const int oe = __shfl_xor_sync(0xffffffffu, be[q], o);
+                const float oz = __shfl_xor_sync(0xffffffffu, bz[q], o);
+                const bool better = (oe != 0x7fffffff) &&
+                                    (be[q] == 0x7fffffff || ok_ > bk[q] || (ok_ == bk[q] && oe < be[q]));
+                if (better) { bk[q] = ok_; be[q] = oe; bz[q] = oz; }
+            }
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            if ((be[q] & 31) == lane) taken[q] |= 1u << (be[q] >> 5);
+            zsel[q][j] = bz[q];
+            esel[q][j] = be[q];
+        }
+    }
+    // gates: softmax over the selected raw logits, slot order
+    if (lane == 0) {
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+            if (q >= nt) break;
+            float zm = -INFINITY, gs = 0.f;
+#pragma unroll 1
+            for (int j = 0; j < k; ++j) zm = fmaxf(zm, zsel[q][j]);
+#pragma unroll 1
+            for (int j = 0; j < k; ++j) gs += expf(zsel[q][j] - zm);
+            const float inv_g = 1.f / gs;
+            const int t = t0 + q;
+#pragma unroll 1
+            for (int j = 0; j < k; ++j) {
+                idx_out[(size_t)t * k + j] = esel[q][j];
+                // selected softmax, or the full-softmax probability (Switch gate)
+                gate_out[(size_t)t * k + j] =
+                    gate_mode == MOE_GATE_FULL ? expf(zsel[q][j] - m[q]) * inv_s[q] : expf(zsel[q][j] - zm) * inv_g;
+                atomicAdd(&cnt[esel[q][j] * kk + (kk > 1 ? j : 0)], 1);   // integer: order does not matter
+            }
+        }
+    }
+}
+
 // The chunk's statistics: probability sums over warps in warp order, counts,
 // and the z-loss / entropy / gap sums.
 template <int EPL>
@@ -383,16 +549,18 @@ select_kernel(const float* __restrict__ logits, const float* __restrict__ bias, 
 
 // ---- fused router: logits and selection in one kernel ----------------------
 // One block per chunk of kChunk tokens, the same warp-to-token assignment as
-// select_kernel (warp w: tokens 4w .. 4w + 3 of the chunk). A warp computes
-// its four tokens' logits itself: lane l takes the 8-element chunks c = l,
-// l + 32, ... of the row (16-byte loads of x, four chunks in flight per
-// token), multiplies them with the matching rows of W_r [d, E] as given (no
-// transposed copy: a row of W_r holds the E weights of one input feature),
-// eight experts per pass, and an xor butterfly leaves every lane with the
-// sums, in a fixed order. The logits are written out (the workspace keeps
-// them) and, still in registers, go through the same per-token selection as
-// select_kernel. x is read once from HBM; W_r (d E elements) is re-read from
-// L1/L2 by each warp. E <= 64.
+// select_kernel (warp w: tokens 4w .. 4w + 3 of the chunk). Experts are taken
+// eight per pass: the block first copies W_r^T of the pass's experts into
+// shared memory (W_r [d, E] as given: a row holds the E weights of one input
+// feature). A warp then computes its four tokens' logits itself: lane l
+// takes the 8-element chunks c = l, l + 32, ... of the row (16-byte loads of
+// x straight from global memory, several chunks of every token in flight),
+// multiplies them with the pass's W_r^T from shared memory in fp32 FMAs, and
+// an xor butterfly leaves every lane with the sums, in a fixed order. The
+// logits are written out (the workspace keeps them) and, still in registers,
+// go through the same per-token selection as select_kernel. E <= 64. This
+// is the fp32 router, and the bf16 one where the MMA form below does not
+// fit; its speed is set by FMA issue (8 FMAs per element of x per pass).
 template <typename T>
 struct RawVec8 {   // 8 elements of a row as loaded: one 16-byte vector (bf16) or two (fp32)
     uint4 v[sizeof(T) == 2 ? 1 : 2];
@@ -418,14 +586,34 @@ __device__ __forceinline__ void unpack8(const RawVec8<float>& r, float (&v)[8]) 
     }
 }
 
-// Rows of W_r (input features) a block stages at a time: 4 KB of x per token
-// for the chunk's 32 tokens (128 KB; a whole Mixtral-sized row block would
-// not fit), and W_r^T of those rows for eight experts (32 KB for bf16).
+// The selection half of both fused routers: the warp's nt tokens t0, t0 + 1,
+// ... (lane l holds the logits of experts l + 32 i) are written out and go
+// through the per-token selection.
+template <int EPL>
+__device__ __forceinline__ void fused_select(const float (&zt)[kChunk / kSelWarps][EPL], int nt, int t0,
+                                             int bias_mode, int gate_mode, int kk, int E, int k, int lane,
+                                             SelAcc<EPL>& a, int* cnt, float* __restrict__ logits,
+                                             int32_t* __restrict__ idx_out, float* __restrict__ gate_out) {
+#pragma unroll
+    for (int q = 0; q < kChunk / kSelWarps; ++q) {
+        if (q < nt) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const int e = lane + 32 * i;
+                if (e < E) logits[(size_t)(t0 + q) * E + e] = zt[q][i];
+            }
+        }
+    }
+    sel_tokens<EPL, kChunk / kSelWarps>(zt, nt, t0, bias_mode, gate_mode, kk, E, k, lane, a, cnt, idx_out, gate_out);
+}
+
+// Shared memory of the fused router: W_r^T of one pass's eight experts over
+// the whole row (64 KB for bf16 at d = 4096); wider rows take the
+// three-kernel router.
+constexpr size_t kFusedWtMaxBytes = 160 * 1024;
 template <typename T>
-constexpr int fused_slab() { return 4096 / (int)sizeof(T); }
-template <typename T>
-constexpr size_t fused_smem_bytes() {
-    return (size_t)kChunk * fused_slab<T>() * sizeof(T) + (size_t)kExpPerPass * fused_slab<T>() * sizeof(T) + 64;
+size_t fused_smem_bytes(int d) {
+    return (size_t)kExpPerPass * (size_t)d * sizeof(T);
 }
 
 template <typename T, int EPL>
@@ -436,24 +624,17 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
                    float* __restrict__ blockpsum, float* __restrict__ blockextra, int32_t* __restrict__ status) {
     static_assert(EPL <= 2, "fused router: E <= 64");
     constexpr int kTokPerWarp = kChunk / kSelWarps;   // 4
-    constexpr int SLAB = fused_slab<T>();             // rows of W_r (columns of x) per slab
     __shared__ int cnt[kMaxSlotCounts];
     __shared__ float ps[kSelWarps][MOE_MAX_E];
     __shared__ float ext[kSelWarps][3];
     extern __shared__ __align__(128) uint8_t fused_dsm[];
-    T* xs = reinterpret_cast<T*>(fused_dsm);                      // [kChunk][SLAB]: x of the slab
-    T* wt = xs + (size_t)kChunk * SLAB;                           // [kExpPerPass][SLAB]: W_r^T of the slab
-    uint64_t* xbar = reinterpret_cast<uint64_t*>(wt + (size_t)kExpPerPass * SLAB);
+    T* wt = reinterpret_cast<T*>(fused_dsm);                      // [kExpPerPass][d]: W_r^T of the pass
     pdl_wait();
     pdl_launch();
     if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = MOE_OK;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunk = blockIdx.x, NB = gridDim.x;
     for (int e = threadIdx.x; e < E * kk; e += blockDim.x) cnt[e] = 0;
-    if (threadIdx.x == 0) {
-        tc::mbar_init(xbar, 1);
-        tc::fence_mbar_init();
-    }
     SelAcc<EPL> a;
     sel_init(a, bias, bias_mode, E, lane);
     const int c0tok = chunk * kChunk;
@@ -465,89 +646,77 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
     for (int q = 0; q < kTokPerWarp; ++q)
 #pragma unroll
         for (int i = 0; i < EPL; ++i) zt[q][i] = -INFINITY;
-    uint32_t xph = 0;
+    const int nchunk = d / 8;                                     // 8-element chunks of a row
     for (int e0 = 0; e0 < E; e0 += kExpPerPass) {
+        __syncthreads();   // the previous pass's W_r^T is consumed
+        // W_r^T [e0 .. e0 + 7][0 .. d) (zeros past E): the rows of W_r are one
+        // contiguous run of d E elements, requested as 16-byte vectors, eight
+        // per thread, before any is written, transposed, into shared memory
+        if (e0 + kExpPerPass > E)
+            for (int i = threadIdx.x; i < kExpPerPass * d; i += blockDim.x) wt[i] = T(0.f);
+        __syncthreads();
+        {
+            const int ng = d * E / 8;
+            for (int g0 = threadIdx.x; g0 < ng; g0 += blockDim.x * 8) {
+                RawVec8<T> wr[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int g = g0 + (int)blockDim.x * j;
+                    if (g < ng) raw_load8(W_r + (size_t)g * 8, wr[j]);
+                }
+#pragma unroll 1
+                for (int j = 0; j < 8; ++j) {
+                    const int g = g0 + (int)blockDim.x * j;
+                    if (g >= ng) break;
+                    float v[8];
+                    unpack8(wr[j], v);
+                    if (E % kExpPerPass == 0) {
+                        // the group is experts [eb, eb + 8) of one input feature r
+                        const int r = (g * 8) / E, eb = g * 8 - r * E;
+                        if (eb == e0) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) wt[i * d + r] = T(v[i]);
+                        }
+                    } else {
+#pragma unroll 1
+                        for (int i = 0; i < 8; ++i) {
+                            const int idx = g * 8 + i, r = idx / E, e = idx - r * E - e0;
+                            if (e >= 0 && e < kExpPerPass) wt[e * d + r] = T(v[i]);
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();   // W_r^T written
+        // lane l takes the row's 8-element chunks l, l + 32, ...: the warp's
+        // tokens' x straight from global memory (512 contiguous bytes a row
+        // per warp load, kXUnroll chunks of every token in flight), the eight
+        // experts' weights of the chunk's input features from shared memory
         float acc[kTokPerWarp][kExpPerPass];
 #pragma unroll
         for (int q = 0; q < kTokPerWarp; ++q)
 #pragma unroll
             for (int e = 0; e < kExpPerPass; ++e) acc[q][e] = 0.f;
-        for (int d0 = 0; d0 < d; d0 += SLAB) {
-            const int ns = min(SLAB, d - d0);
-            __syncthreads();   // the previous slab is consumed (and the barrier initialised)
-            // x of the block's tokens, columns [d0, d0 + ns): one bulk copy per
-            // token row into the slab
-            if (threadIdx.x == 0) {
-                tc::fence_proxy_async_smem();   // the slab's earlier generic reads precede the copies
-                tc::mbar_arrive_expect_tx(xbar, (uint32_t)(ntok * ns * (int)sizeof(T)));
-                for (int q = 0; q < ntok; ++q)
-                    tc::bulk_load(tc::smem_u32(xs + (size_t)q * SLAB), x + (size_t)(c0tok + q) * d + d0,
-                                  (uint32_t)(ns * (int)sizeof(T)), xbar);
-            }
-            // W_r^T [e0 .. e0 + 7][d0 .. d0 + ns) (zeros past E): the rows
-            // [d0, d0 + ns) of W_r are one contiguous run of ns E elements,
-            // requested as 16-byte vectors, eight per thread, before any is
-            // written, transposed, into the slab
-            if (e0 + kExpPerPass > E)
-                for (int i = threadIdx.x; i < kExpPerPass * ns; i += blockDim.x) wt[(i / ns) * SLAB + i % ns] = T(0.f);
-            __syncthreads();
-            {
-                const T* src = W_r + (size_t)d0 * E;
-                const int ng = ns * E / 8;
-                for (int g0 = threadIdx.x; g0 < ng; g0 += blockDim.x * 8) {
-                    RawVec8<T> wr[8];
+        constexpr int kXUnroll = sizeof(T) == 2 ? 4 : 2;
+#pragma unroll 1
+        for (int cb = lane; cb < nchunk; cb += 32 * kXUnroll) {
+            RawVec8<T> xr[kXUnroll][kTokPerWarp];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int g = g0 + (int)blockDim.x * j;
-                        if (g < ng) raw_load8(src + (size_t)g * 8, wr[j]);
-                    }
-#pragma unroll 1
-                    for (int j = 0; j < 8; ++j) {
-                        const int g = g0 + (int)blockDim.x * j;
-                        if (g >= ng) break;
-                        float v[8];
-                        unpack8(wr[j], v);
-                        if (E % kExpPerPass == 0) {
-                            // the group is experts [eb, eb + 8) of one input feature r
-                            const int r = (g * 8) / E, eb = g * 8 - r * E;
-                            if (eb == e0) {
+            for (int u = 0; u < kXUnroll; ++u) {
+                const int c = cb + 32 * u;
 #pragma unroll
-                                for (int i = 0; i < 8; ++i) wt[i * SLAB + r] = T(v[i]);
-                            }
-                        } else {
-#pragma unroll 1
-                            for (int i = 0; i < 8; ++i) {
-                                const int idx = g * 8 + i, r = idx / E, e = idx - r * E - e0;
-                                if (e >= 0 && e < kExpPerPass) wt[e * SLAB + r] = T(v[i]);
-                            }
-                        }
-                    }
-                }
+                for (int q = 0; q < kTokPerWarp; ++q)
+                    if (c < nchunk && q < nt) raw_load8(x + (size_t)(c0tok + q0 + q) * d + (size_t)c * 8, xr[u][q]);
             }
-            __syncthreads();   // W_r^T slab written
-            // the x slab has landed (bulk copies of this block's own rows, which
-            // complete on their own; the wait is still bounded)
-            if (!tc::mbar_try_wait(xbar, xph)) {
-                const uint64_t t0 = tc::global_timer_ns();
-                while (!tc::mbar_try_wait(xbar, xph)) {
-                    if (tc::global_timer_ns() - t0 > static_cast<uint64_t>(kDrainLimitNs)) {
-                        if (status != nullptr) atomicExch(status, MOE_ERR_TIMEOUT);
-                        break;
-                    }
-                }
-            }
-            xph ^= 1u;
-            // lane l takes the slab's 8-element chunks l, l + 32, ...: the four
-            // tokens' x and the eight experts' weights of the chunk's 8 input
-            // features, all from shared memory
-            const int nchunk = ns / 8;
-#pragma unroll 1
-            for (int c = lane; c < nchunk; c += 32) {
+#pragma unroll
+            for (int u = 0; u < kXUnroll; ++u) {
+                const int c = cb + 32 * u;
+                if (c >= nchunk) break;
                 float xv[kTokPerWarp][8];
 #pragma unroll
                 for (int q = 0; q < kTokPerWarp; ++q) {
                     if (q < nt) {
-                        load8(xs + (size_t)(q0 + q) * SLAB + c * 8, xv[q]);
+                        unpack8(xr[u][q], xv[q]);
                     } else {
 #pragma unroll
                         for (int j = 0; j < 8; ++j) xv[q][j] = 0.f;
@@ -556,7 +725,7 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
 #pragma unroll
                 for (int e = 0; e < kExpPerPass; ++e) {
                     float wv[8];
-                    load8(wt + e * SLAB + c * 8, wv);
+                    load8(wt + (size_t)e * d + (size_t)c * 8, wv);
 #pragma unroll
                     for (int q = 0; q < kTokPerWarp; ++q)
 #pragma unroll
@@ -589,23 +758,272 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
         }
     }
     __syncthreads();   // the chunk's counters are zeroed
+    fused_select<EPL>(zt, nt, c0tok + q0, bias_mode, gate_mode, kk, E, k, lane, a, cnt, logits, idx_out, gate_out);
+    sel_finish<EPL>(a, chunk, NB, E, kk, warp, lane, cnt, ps, ext, blockcnt, blockpsum, blockextra);
+}
+
+// ---- fused router, bf16: the logits on the warp-level MMA ------------------
+// The same block and selection as route_fused_kernel (one block of 8 warps
+// per chunk of kChunk tokens), with the dot products of the logits done by
+// mma.sync (m16n8k16, bf16 products exact in fp32, fp32 accumulate) instead
+// of fp32 FMAs, so the block is bound by its stream of x rather than by
+// instruction issue.
+//
+// Operands. A is W_r^T of the pass's experts (16 expert rows per MMA; rows
+// past the pass's experts are fed as zeros), kept in shared memory for the
+// whole pass. B is 8 token rows of x. Warp w takes token octet w % 4 of the
+// chunk and the 128-element items h, h + 2, h + 4, ... of the row, h = w / 4;
+// each warp streams its items through its own ring of kRmStages shared-memory
+// buffers with 16-byte cp.async copies (a half-warp copies 256 contiguous
+// bytes of one row). For a 32-element chunk at kb, lane (g, t) takes the 8
+// values at kb + 8t of A row g (and g + 8) and of token row g: values 0-3 feed
+// one MMA, 4-7 a second, so each k of the chunk is multiplied once (the order
+// of k inside an MMA is not memory order; a dot product does not see it).
+// Piece p of staged token row r sits at position p ^ sw(r) in its 256-byte
+// row, W_r^T rows are 2d + 64 bytes apart: the fragment reads of a quarter
+// warp fall in eight different bank groups.
+//
+// The two K halves of each octet meet in shared memory: half 1 stores its
+// partial logits, half 0 adds its own (a fixed order), and the selection
+// reads the chunk's logits from there. Passes of P experts (P a multiple of
+// 8, W_r^T of P experts within kRmWtMaxBytes) cover E <= 64; each pass reads
+// x again (from L2 after the first).
+constexpr int kRmItemK = 128;                                        // K elements per staged item
+constexpr int kRmItemBytes = 8 * kRmItemK * 2;                       // 8 token rows of it
+constexpr int kRmStages = 6;                                         // items in each warp's ring
+constexpr int kRmZStride = 64;                                       // logits tile: up to 64 experts a token
+constexpr size_t kRmRingBytes = (size_t)kSelWarps * kRmStages * kRmItemBytes;   // 96 KB
+constexpr size_t kRmZBytes = (size_t)kChunk * kRmZStride * sizeof(float);         // 8 KB
+constexpr size_t kRmWtMaxBytes = 84 * 1024;
+constexpr size_t kRmSmemMax = kRmRingBytes + kRmZBytes + kRmWtMaxBytes;
+
+int rm_row_bytes(int d) { return 2 * d + 64; }
+// experts per pass (0: not even eight rows of W_r^T fit)
+int rm_pass_experts(int d, int E) {
+    const int fit = (int)(kRmWtMaxBytes / (size_t)rm_row_bytes(d)) / 8 * 8;
+    return std::min(fit, std::min(64, ceil_div(E, 8) * 8));
+}
+bool route_fused_mma_ok(int d, int E) {
+    static const bool enabled = [] {
+        const char* v = std::getenv("MOE_ROUTER_MMA");
+        return !(v != nullptr && v[0] == '0');
+    }();
+    return enabled && E <= 64 && d % 8 == 0 && rm_pass_experts(d, E) >= 8;
+}
+
+__device__ __forceinline__ int rm_swz(int r) { return ((r & 1) << 2) | ((r >> 1) & 3); }
+
+template <int EPL>
+__global__ void __launch_bounds__(kSelWarps * 32, 1)
+route_fused_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ W_r,
+                       const float* __restrict__ bias, int bias_mode, int gate_mode, int kk, int Tn, int d, int E,
+                       int k, int P, float* __restrict__ logits, int32_t* __restrict__ idx_out,
+                       float* __restrict__ gate_out, int32_t* __restrict__ blockcnt, float* __restrict__ blockpsum,
+                       float* __restrict__ blockextra, int32_t* __restrict__ status) {
+    static_assert(EPL <= 2, "fused router: E <= 64");
+    constexpr int kTokPerWarp = kChunk / kSelWarps;   // 4
+    constexpr int NS = kRmStages;
+    __shared__ int cnt[kMaxSlotCounts];
+    __shared__ float ps[kSelWarps][MOE_MAX_E];
+    __shared__ float ext[kSelWarps][3];
+    extern __shared__ __align__(128) uint8_t rm_smem[];
+    // [kSelWarps][NS] item buffers, the chunk's logits [kChunk][kRmZStride],
+    // then W_r^T of the pass [P][2d + 64 bytes]
+    float* zl = reinterpret_cast<float*>(rm_smem + kRmRingBytes);
+    const uint32_t wt = smem_addr(rm_smem + kRmRingBytes + kRmZBytes);
+    pdl_wait();
+    pdl_launch();
+    if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = MOE_OK;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunk = blockIdx.x, NB = gridDim.x;
+    for (int e = threadIdx.x; e < E * kk; e += blockDim.x) cnt[e] = 0;
+    SelAcc<EPL> a;
+    sel_init(a, bias, bias_mode, E, lane);
+    const int c0tok = chunk * kChunk;
+    const int ntok = min(kChunk, Tn - c0tok);
+    const int rs = 2 * d + 64;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int oct = warp & 3, half = warp >> 2;
+    const int S = (d + kRmItemK - 1) / kRmItemK;
+    const int nmine = (S - half + 1) / 2;                 // this warp's items: half, half + 2, ...
+    const uint32_t ring = smem_addr(rm_smem + (size_t)warp * NS * kRmItemBytes);
+    const bool tok_ok = oct * 8 + gid < ntok;             // the lane's token row (B column)
+
+    // the lane's four copies of an item: piece lane % 16 of rows 2i + lane / 16
+    const int pc = lane & 15;
+    const __nv_bfloat16* xsrc[4];
+    uint32_t xdst[4];
+    bool xrow[4];
 #pragma unroll
-    for (int q = 0; q < kTokPerWarp; ++q) {
-        if (q < nt) {
-            const int t = c0tok + q0 + q;
+    for (int i = 0; i < 4; ++i) {
+        const int r = 2 * i + (lane >> 4);
+        xrow[i] = oct * 8 + r < ntok;
+        xsrc[i] = x + (size_t)(xrow[i] ? c0tok + oct * 8 + r : c0tok) * d + pc * 8;
+        xdst[i] = (uint32_t)(r * (kRmItemK * 2) + ((pc ^ rm_swz(r)) << 4));
+    }
+    // copy this warp's item m into ring slot `slot`; always one commit group
+    // (empty past the end), so the wait counts stay aligned
+    auto issue = [&](int slot, int m) {
+        if (m < nmine) {
+            const int k0 = (half + 2 * m) * kRmItemK;
+            const bool pin = pc * 8 < d - k0;   // the piece lies inside the row
+            const uint32_t dst = ring + (uint32_t)slot * kRmItemBytes;
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) {
-                const int e = lane + 32 * i;
-                if (e < E) logits[(size_t)t * E + e] = zt[q][i];
+            for (int i = 0; i < 4; ++i)
+                if (pin && xrow[i]) cp_async16(dst + xdst[i], xsrc[i] + k0);
+        }
+        cp_async_commit();
+    };
+
+    for (int e0 = 0; e0 < E; e0 += P) {
+        const int pe = min(P, E - e0);
+#pragma unroll
+        for (int s = 0; s < NS - 1; ++s) issue(s, s);
+        __syncthreads();   // the previous pass's W_r^T and logits are consumed
+        // W_r^T [e0, e0 + pe) x [0, d): the rows of W_r hold the E weights of
+        // one input feature each
+        if (E % 8 == 0) {
+            // features (r, r + 1) x 8 experts: two 16-byte loads, eight
+            // 4-byte stores of (feature r, feature r + 1) pairs
+            // (kStage pairs of loads in flight per thread)
+            constexpr int kStage = 8;
+            const int hd = d / 2;
+            const int n = hd * (pe / 8);
+            for (int it0 = threadIdx.x; it0 < n; it0 += kStage * blockDim.x) {
+                uint4 u0[kStage], u1[kStage];
+#pragma unroll
+                for (int b = 0; b < kStage; ++b) {
+                    const int it = it0 + b * (int)blockDim.x;
+                    if (it < n) {
+                        const int c = it / hd, r = 2 * (it - c * hd);
+                        const __nv_bfloat16* src = W_r + (size_t)r * E + e0 + 8 * c;
+                        u0[b] = __ldg(reinterpret_cast<const uint4*>(src));
+                        u1[b] = __ldg(reinterpret_cast<const uint4*>(src + E));
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < kStage; ++b) {
+                    const int it = it0 + b * (int)blockDim.x;
+                    if (it < n) {
+                        const int c = it / hd, r = 2 * (it - c * hd);
+                        const uint32_t w0[4] = {u0[b].x, u0[b].y, u0[b].z, u0[b].w};
+                        const uint32_t w1[4] = {u1[b].x, u1[b].y, u1[b].z, u1[b].w};
+                        const uint32_t base = wt + (uint32_t)(8 * c) * rs + (uint32_t)r * 2;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            sts32(base + (uint32_t)(2 * i) * rs, __byte_perm(w0[i], w1[i], 0x5410));
+                            sts32(base + (uint32_t)(2 * i + 1) * rs, __byte_perm(w0[i], w1[i], 0x7632));
+                        }
+                    }
+                }
             }
-            sel_token<EPL, true>(zt[q], t, bias_mode, gate_mode, kk, E, k, lane, a, cnt, idx_out, gate_out);
+        } else {
+            __nv_bfloat16* wtp = reinterpret_cast<__nv_bfloat16*>(rm_smem + kRmRingBytes + kRmZBytes);
+            for (int it = threadIdx.x; it < pe * d; it += blockDim.x) {
+                const int e = it / d, r = it - e * d;
+                wtp[(size_t)e * (rs / 2) + r] = W_r[(size_t)r * E + e0 + e];
+            }
+        }
+        __syncthreads();   // W_r^T written
+
+        // one accumulator set per 32-element chunk of an item, so that
+        // consecutive MMAs are independent; the sets are summed in a fixed
+        // order at the end of the pass
+        float accu[4][kRmItemK / 32][4];
+#pragma unroll
+        for (int G = 0; G < 4; ++G)
+#pragma unroll
+            for (int u = 0; u < kRmItemK / 32; ++u) accu[G][u][0] = accu[G][u][1] = accu[G][u][2] = accu[G][u][3] = 0.f;
+        const int g16 = (pe + 15) / 16;
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        for (int m = 0; m < nmine; ++m) {
+            issue((m + NS - 1) % NS, m + NS - 1);
+            cp_async_wait<NS - 1>();
+            __syncwarp();
+            const uint32_t buf = ring + (uint32_t)(m % NS) * kRmItemBytes;
+            const int k0 = (half + 2 * m) * kRmItemK;
+            // the lane's 8 elements of chunk u start at kb(u) = k0 + 32u + 8t
+            // (d % 8 == 0: all inside the row or all outside)
+            uint4 xb[kRmItemK / 32];
+#pragma unroll
+            for (int u = 0; u < kRmItemK / 32; ++u) {
+                const bool kin = k0 + 32 * u + 8 * tig < d;
+                xb[u] = (kin && tok_ok)
+                            ? lds128(buf + (uint32_t)(gid * (kRmItemK * 2) + (((4 * u + tig) ^ rm_swz(gid)) << 4)))
+                            : z4;
+            }
+#pragma unroll
+            for (int G = 0; G < 4; ++G) {
+                if (G < g16) {
+                    const int ea = 16 * G + gid, eb = ea + 8;
+                    uint4 wa[kRmItemK / 32], wb[kRmItemK / 32];
+#pragma unroll
+                    for (int u = 0; u < kRmItemK / 32; ++u) {
+                        const int kb = k0 + 32 * u + 8 * tig;
+                        const bool kin = kb < d;
+                        wa[u] = (kin && ea < pe) ? lds128(wt + (uint32_t)ea * rs + (uint32_t)kb * 2) : z4;
+                        wb[u] = (kin && eb < pe) ? lds128(wt + (uint32_t)eb * rs + (uint32_t)kb * 2) : z4;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kRmItemK / 32; ++u)
+                        mma_bf16(accu[G][u], wa[u].x, wb[u].x, wa[u].y, wb[u].y, xb[u].x, xb[u].y);
+#pragma unroll
+                    for (int u = 0; u < kRmItemK / 32; ++u)
+                        mma_bf16(accu[G][u], wa[u].z, wb[u].z, wa[u].w, wb[u].w, xb[u].z, xb[u].w);
+                }
+            }
+            __syncwarp();   // the buffer is refilled by a later issue()
+        }
+        cp_async_wait<0>();
+        float acc[4][4];
+#pragma unroll
+        for (int G = 0; G < 4; ++G)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[G][c] = ((accu[G][0][c] + accu[G][1][c]) + accu[G][2][c]) + accu[G][3][c];
+        // D element (expert e0 + 16G + g (+ 8), token 8 oct + 2t (+ 1)):
+        // half 1 stores its partial sums, half 0 adds its own to them
+        auto zat = [&](int G, int c) -> float* {
+            const int e = 16 * G + gid + ((c & 2) ? 8 : 0);
+            const int tok = oct * 8 + 2 * tig + (c & 1);
+            return zl + tok * kRmZStride + e0 + e;
+        };
+        if (half == 1) {
+#pragma unroll
+            for (int G = 0; G < 4; ++G)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (G < g16 && 16 * G + gid + ((c & 2) ? 8 : 0) < pe) *zat(G, c) = acc[G][c];
+        }
+        __syncthreads();
+        if (half == 0) {
+#pragma unroll
+            for (int G = 0; G < 4; ++G)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (G < g16 && 16 * G + gid + ((c & 2) ? 8 : 0) < pe) {
+                        float* q = zat(G, c);
+                        *q = acc[G][c] + *q;
+                    }
         }
     }
+    __syncthreads();   // the chunk's logits are complete (and its counters zeroed)
+    const int q0 = warp * kTokPerWarp;
+    const int nt = max(0, min(kTokPerWarp, ntok - q0));
+    float zt[kTokPerWarp][EPL];
+#pragma unroll
+    for (int q = 0; q < kTokPerWarp; ++q)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            zt[q][i] = e < E ? zl[(q0 + q) * kRmZStride + e] : -INFINITY;
+        }
+    fused_select<EPL>(zt, nt, c0tok + q0, bias_mode, gate_mode, kk, E, k, lane, a, cnt, logits, idx_out, gate_out);
     sel_finish<EPL>(a, chunk, NB, E, kk, warp, lane, cnt, ps, ext, blockcnt, blockpsum, blockextra);
 }
 
 bool route_fused_ok(int dtype, int d, int E) {
-    return E <= 64 && d % 8 == 0 && (dtype == MOE_DTYPE_F32 || dtype == MOE_DTYPE_BF16);
+    return E <= 64 && d % 8 == 0 && (dtype == MOE_DTYPE_F32 || dtype == MOE_DTYPE_BF16) &&
+           fused_smem_bytes<float>(d) / (dtype == MOE_DTYPE_BF16 ? 2 : 1) <= kFusedWtMaxBytes;
 }
 
 cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const float* bias, int bias_mode,
@@ -615,21 +1033,41 @@ cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const 
     const int NB = ceil_div(T, kChunk);
     if (NB == 0) return cudaSuccess;
     dim3 grid(NB), block(kSelWarps * 32);
-    // the staged x and W_r slabs (160 KB) are dynamic shared memory beside
-    // the selection's static arrays: opted in once per device and variant
-    static bool attr_set[64][4] = {};
+    // the staged operands (up to 160 KB; 188 KB for the MMA form) are dynamic
+    // shared memory beside the selection's static arrays: opted in once per
+    // device and variant
+    static bool attr_set[64][6] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (dtype == MOE_DTYPE_BF16 && route_fused_mma_ok(d, E)) {
+        const int P = rm_pass_experts(d, E);
+        const size_t smem = kRmRingBytes + kRmZBytes + (size_t)P * rm_row_bytes(d);
+#define MOE_FUSED_MMA(EPLV, SLOT)                                                                                    \
+    do {                                                                                                             \
+        if (!attr_set[dev][SLOT]) {                                                                                  \
+            cudaError_t e_ = cudaFuncSetAttribute(route_fused_mma_kernel<EPLV>,                                      \
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRmSmemMax);     \
+            if (e_ != cudaSuccess) return e_;                                                                        \
+            attr_set[dev][SLOT] = true;                                                                              \
+        }                                                                                                            \
+        return launch_k(route_fused_mma_kernel<EPLV>, grid, block, smem, st, (const __nv_bfloat16*)x,                \
+                        (const __nv_bfloat16*)W_r, bias, bias_mode, gate_mode, kk, T, d, E, k, P, logits, idx, gate, \
+                        blockcnt, blockpsum, blockextra, status);                                                    \
+    } while (0)
+        if (E <= 32) MOE_FUSED_MMA(1, 4);
+        MOE_FUSED_MMA(2, 5);
+#undef MOE_FUSED_MMA
+    }
 #define MOE_FUSED(TYPE, EPLV, SLOT)                                                                                  \
     do {                                                                                                             \
         if (!attr_set[dev][SLOT]) {                                                                                  \
             cudaError_t e_ = cudaFuncSetAttribute(route_fused_kernel<TYPE, EPLV>,                                    \
                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,                       \
-                                                  (int)fused_smem_bytes<TYPE>());                                    \
+                                                  (int)kFusedWtMaxBytes);                                            \
             if (e_ != cudaSuccess) return e_;                                                                        \
             attr_set[dev][SLOT] = true;                                                                              \
         }                                                                                                            \
-        return launch_k(route_fused_kernel<TYPE, EPLV>, grid, block, fused_smem_bytes<TYPE>(), st, (const TYPE*)x,  \
+        return launch_k(route_fused_kernel<TYPE, EPLV>, grid, block, fused_smem_bytes<TYPE>(d), st, (const TYPE*)x, \
                         (const TYPE*)W_r,                                                                            \
                         bias, bias_mode, gate_mode, kk, T, d, E, k, logits, idx, gate, blockcnt, blockpsum,         \
                         blockextra, status);                                                                         \
