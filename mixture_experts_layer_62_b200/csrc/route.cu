@@ -420,24 +420,30 @@ __device__ __forceinline__ void sel_tokens(const float (&zin)[Q][EPL], int nt, i
                       : bias_mode == MOE_BIAS_LOGIT ? z[q][i] + a.b[i]
                       : p + a.b[i];
         }
-    // top-k: k rounds of a warp arg-max over (key desc, index asc)
+    // top-k: k rounds of a warp arg-max over (key desc, index asc), on one
+    // 64-bit value per candidate: the key mapped to an unsigned integer of
+    // the same order (-0 taken as +0, as a float compare does) above the
+    // complemented index, so the larger value is the larger key and, among
+    // equal keys, the lower index; 0 stands for no candidate. Lane j keeps
+    // the winner of round j (its raw logit and index) in registers.
     unsigned taken[Q];
-    float zsel[Q][MOE_MAX_K];
-    int esel[Q][MOE_MAX_K];
+    float zmine[Q];
+    int emine[Q];
 #pragma unroll
-    for (int q = 0; q < Q; ++q) taken[q] = 0;
+    for (int q = 0; q < Q; ++q) { taken[q] = 0; zmine[q] = 0.f; emine[q] = 0; }
 #pragma unroll 1
     for (int j = 0; j < k; ++j) {
-        float bk[Q], bz[Q];
-        int be[Q];
+        unsigned long long best[Q];
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
-            bk[q] = -INFINITY; bz[q] = 0.f; be[q] = 0x7fffffff;
+            best[q] = 0ull;
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
-                const bool ok = ((valid >> i) & 1u) && !((taken[q] >> i) & 1u);
-                if (ok && (key[q][i] > bk[q] || be[q] == 0x7fffffff)) {
-                    bk[q] = key[q][i]; be[q] = lane + 32 * i; bz[q] = z[q][i];
+                if (((valid >> i) & 1u) && !((taken[q] >> i) & 1u)) {
+                    const uint32_t b = __float_as_uint(key[q][i] + 0.f);
+                    const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+                    const unsigned long long c = ((unsigned long long)o << 32) | (uint32_t)(~(lane + 32 * i));
+                    best[q] = c > best[q] ? c : best[q];
                 }
             }
         }
@@ -445,39 +451,44 @@ __device__ __forceinline__ void sel_tokens(const float (&zin)[Q][EPL], int nt, i
         for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
             for (int q = 0; q < Q; ++q) {
-                const float ok_ = __shfl_xor_sync(0xffffffffu, bk[q], o);
-                const int oe = __shfl_xor_sync(0xffffffffu, be[q], o);
-                const float oz = __shfl_xor_sync(0xffffffffu, bz[q], o);
-                const bool better = (oe != 0x7fffffff) &&
-                                    (be[q] == 0x7fffffff || ok_ > bk[q] || (ok_ == bk[q] && oe < be[q]));
-                if (better) { bk[q] = ok_; be[q] = oe; bz[q] = oz; }
+                const unsigned long long c = __shfl_xor_sync(0xffffffffu, best[q], o);
+                best[q] = c > best[q] ? c : best[q];
             }
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
-            if ((be[q] & 31) == lane) taken[q] |= 1u << (be[q] >> 5);
-            zsel[q][j] = bz[q];
-            esel[q][j] = be[q];
+            const int be = (int)(~(uint32_t)best[q]);
+            float zc = z[q][0];
+#pragma unroll
+            for (int i = 1; i < EPL; ++i)
+                if ((be >> 5) == i) zc = z[q][i];
+            const float bz = __shfl_sync(0xffffffffu, zc, be & 31);   // the raw logit, from its lane
+            if ((be & 31) == lane) taken[q] |= 1u << (be >> 5);
+            if (lane == j) { zmine[q] = bz; emine[q] = be; }
         }
     }
-    // gates: softmax over the selected raw logits, slot order
-    if (lane == 0) {
+    // gates: softmax over the selected raw logits, slot order (every lane
+    // reads slot j from lane j, in order); lane j < k emits slot j
+    float zm[Q], gs[Q];
+#pragma unroll
+    for (int q = 0; q < Q; ++q) { zm[q] = -INFINITY; gs[q] = 0.f; }
+#pragma unroll 1
+    for (int j = 0; j < k; ++j)
+#pragma unroll
+        for (int q = 0; q < Q; ++q) zm[q] = fmaxf(zm[q], __shfl_sync(0xffffffffu, zmine[q], j));
+#pragma unroll 1
+    for (int j = 0; j < k; ++j)
+#pragma unroll
+        for (int q = 0; q < Q; ++q) gs[q] += expf(__shfl_sync(0xffffffffu, zmine[q], j) - zm[q]);
+    if (lane < k) {
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
-            if (q >= nt) break;
-            float zm = -INFINITY, gs = 0.f;
-#pragma unroll 1
-            for (int j = 0; j < k; ++j) zm = fmaxf(zm, zsel[q][j]);
-#pragma unroll 1
-            for (int j = 0; j < k; ++j) gs += expf(zsel[q][j] - zm);
-            const float inv_g = 1.f / gs;
-            const int t = t0 + q;
-#pragma unroll 1
-            for (int j = 0; j < k; ++j) {
-                idx_out[(size_t)t * k + j] = esel[q][j];
+            if (q < nt) {
+                const size_t o = (size_t)(t0 + q) * k + lane;
+                idx_out[o] = emine[q];
                 // selected softmax, or the full-softmax probability (Switch gate)
-                gate_out[(size_t)t * k + j] =
-                    gate_mode == MOE_GATE_FULL ? expf(zsel[q][j] - m[q]) * inv_s[q] : expf(zsel[q][j] - zm) * inv_g;
-                atomicAdd(&cnt[esel[q][j] * kk + (kk > 1 ? j : 0)], 1);   // integer: order does not matter
+                gate_out[o] = gate_mode == MOE_GATE_FULL ? expf(zmine[q] - m[q]) * inv_s[q]
+                                                         : expf(zmine[q] - zm[q]) * (1.f / gs[q]);
+                atomicAdd(&cnt[emine[q] * kk + (kk > 1 ? lane : 0)], 1);   // integer: order does not matter
             }
         }
     }
@@ -769,9 +780,9 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
 // of fp32 FMAs, so the block is bound by its stream of x rather than by
 // instruction issue.
 //
-// Operands. A is W_r^T of the pass's experts (16 expert rows per MMA; rows
-// past the pass's experts are fed as zeros), kept in shared memory for the
-// whole pass. B is 8 token rows of x. Warp w takes token octet w % 4 of the
+// Operands. A is W_r^T of the pass's experts (16 expert rows per MMA; an
+// 8-row half past the pass's experts is fed as zeros, and the rows of a
+// partial half are zero-filled), kept in shared memory for the whole pass. B is 8 token rows of x. Warp w takes token octet w % 4 of the
 // chunk and the 128-element items h, h + 2, h + 4, ... of the row, h = w / 4;
 // each warp streams its items through its own ring of kRmStages shared-memory
 // buffers with 16-byte cp.async copies (a half-warp copies 256 contiguous
@@ -813,7 +824,7 @@ bool route_fused_mma_ok(int d, int E) {
 
 __device__ __forceinline__ int rm_swz(int r) { return ((r & 1) << 2) | ((r >> 1) & 3); }
 
-template <int EPL>
+template <int EPL, int GM>
 __global__ void __launch_bounds__(kSelWarps * 32, 1)
 route_fused_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ W_r,
                        const float* __restrict__ bias, int bias_mode, int gate_mode, int kk, int Tn, int d, int E,
@@ -842,12 +853,12 @@ route_fused_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16*
     const int c0tok = chunk * kChunk;
     const int ntok = min(kChunk, Tn - c0tok);
     const int rs = 2 * d + 64;
+
     const int gid = lane >> 2, tig = lane & 3;
     const int oct = warp & 3, half = warp >> 2;
     const int S = (d + kRmItemK - 1) / kRmItemK;
     const int nmine = (S - half + 1) / 2;                 // this warp's items: half, half + 2, ...
     const uint32_t ring = smem_addr(rm_smem + (size_t)warp * NS * kRmItemBytes);
-    const bool tok_ok = oct * 8 + gid < ntok;             // the lane's token row (B column)
 
     // the lane's four copies of an item: piece lane % 16 of rows 2i + lane / 16
     const int pc = lane & 15;
@@ -918,23 +929,28 @@ route_fused_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16*
                 }
             }
         } else {
+            // rows pe .. pe8 - 1 are zeros, so that 8-row halves are whole
             __nv_bfloat16* wtp = reinterpret_cast<__nv_bfloat16*>(rm_smem + kRmRingBytes + kRmZBytes);
-            for (int it = threadIdx.x; it < pe * d; it += blockDim.x) {
+            const int pe8 = (pe + 7) / 8 * 8;
+            for (int it = threadIdx.x; it < pe8 * d; it += blockDim.x) {
                 const int e = it / d, r = it - e * d;
-                wtp[(size_t)e * (rs / 2) + r] = W_r[(size_t)r * E + e0 + e];
+                wtp[(size_t)e * (rs / 2) + r] = e < pe ? W_r[(size_t)r * E + e0 + e] : __float2bfloat16(0.f);
             }
         }
         __syncthreads();   // W_r^T written
 
-        // one accumulator set per 32-element chunk of an item, so that
-        // consecutive MMAs are independent; the sets are summed in a fixed
-        // order at the end of the pass
-        float accu[4][kRmItemK / 32][4];
+        // independent accumulator sets (with one 16-row group, one per MMA of
+        // an item: 8; otherwise one per 32-element chunk: 4), so that no MMA
+        // waits for the one before it; the sets are summed in a fixed order
+        // at the end of the pass
+        constexpr int NSET = GM == 1 ? 2 * (kRmItemK / 32) : kRmItemK / 32;
+        float accu[GM][NSET][4];
 #pragma unroll
-        for (int G = 0; G < 4; ++G)
+        for (int G = 0; G < GM; ++G)
 #pragma unroll
-            for (int u = 0; u < kRmItemK / 32; ++u) accu[G][u][0] = accu[G][u][1] = accu[G][u][2] = accu[G][u][3] = 0.f;
+            for (int u = 0; u < NSET; ++u) accu[G][u][0] = accu[G][u][1] = accu[G][u][2] = accu[G][u][3] = 0.f;
         const int g16 = (pe + 15) / 16;
+        const int pe8 = (pe + 7) / 8 * 8;   // W^T rows present (zeros past pe)
         const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
         for (int m = 0; m < nmine; ++m) {
             issue((m + NS - 1) % NS, m + NS - 1);
@@ -943,43 +959,52 @@ route_fused_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16*
             const uint32_t buf = ring + (uint32_t)(m % NS) * kRmItemBytes;
             const int k0 = (half + 2 * m) * kRmItemK;
             // the lane's 8 elements of chunk u start at kb(u) = k0 + 32u + 8t
-            // (d % 8 == 0: all inside the row or all outside)
+            // (d % 8 == 0: all inside the row or all outside); a whole item
+            // needs no checks. Rows of the item past the chunk's tokens hold
+            // stale data: they only feed their own columns of D, which are
+            // never read. Expert halves are whole (8 rows, zeros past pe).
+            const bool full = k0 + kRmItemK <= d;
             uint4 xb[kRmItemK / 32];
 #pragma unroll
             for (int u = 0; u < kRmItemK / 32; ++u) {
-                const bool kin = k0 + 32 * u + 8 * tig < d;
-                xb[u] = (kin && tok_ok)
-                            ? lds128(buf + (uint32_t)(gid * (kRmItemK * 2) + (((4 * u + tig) ^ rm_swz(gid)) << 4)))
-                            : z4;
+                const uint32_t a = buf + (uint32_t)(gid * (kRmItemK * 2) + (((4 * u + tig) ^ rm_swz(gid)) << 4));
+                xb[u] = (full || k0 + 32 * u + 8 * tig < d) ? lds128(a) : z4;
             }
 #pragma unroll
-            for (int G = 0; G < 4; ++G) {
+            for (int G = 0; G < GM; ++G) {
                 if (G < g16) {
                     const int ea = 16 * G + gid, eb = ea + 8;
+                    const bool hi = 16 * G + 8 < pe8;   // the upper 8-row half holds experts
                     uint4 wa[kRmItemK / 32], wb[kRmItemK / 32];
 #pragma unroll
                     for (int u = 0; u < kRmItemK / 32; ++u) {
                         const int kb = k0 + 32 * u + 8 * tig;
-                        const bool kin = kb < d;
-                        wa[u] = (kin && ea < pe) ? lds128(wt + (uint32_t)ea * rs + (uint32_t)kb * 2) : z4;
-                        wb[u] = (kin && eb < pe) ? lds128(wt + (uint32_t)eb * rs + (uint32_t)kb * 2) : z4;
+                        const bool kin = full || kb < d;
+                        wa[u] = kin ? lds128(wt + (uint32_t)ea * rs + (uint32_t)kb * 2) : z4;
+                        wb[u] = (hi && kin) ? lds128(wt + (uint32_t)eb * rs + (uint32_t)kb * 2) : z4;
                     }
 #pragma unroll
                     for (int u = 0; u < kRmItemK / 32; ++u)
                         mma_bf16(accu[G][u], wa[u].x, wb[u].x, wa[u].y, wb[u].y, xb[u].x, xb[u].y);
 #pragma unroll
                     for (int u = 0; u < kRmItemK / 32; ++u)
-                        mma_bf16(accu[G][u], wa[u].z, wb[u].z, wa[u].w, wb[u].w, xb[u].z, xb[u].w);
+                        mma_bf16(accu[G][(u + kRmItemK / 32) % NSET], wa[u].z, wb[u].z, wa[u].w, wb[u].w, xb[u].z,
+                                 xb[u].w);
                 }
             }
             __syncwarp();   // the buffer is refilled by a later issue()
         }
         cp_async_wait<0>();
-        float acc[4][4];
+        float acc[GM][4];
 #pragma unroll
-        for (int G = 0; G < 4; ++G)
+        for (int G = 0; G < GM; ++G)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[G][c] = ((accu[G][0][c] + accu[G][1][c]) + accu[G][2][c]) + accu[G][3][c];
+            for (int c = 0; c < 4; ++c) {
+                float v = accu[G][0][c];
+#pragma unroll
+                for (int u = 1; u < NSET; ++u) v += accu[G][u][c];
+                acc[G][c] = v;
+            }
         // D element (expert e0 + 16G + g (+ 8), token 8 oct + 2t (+ 1)):
         // half 1 stores its partial sums, half 0 adds its own to them
         auto zat = [&](int G, int c) -> float* {
@@ -989,7 +1014,7 @@ route_fused_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16*
         };
         if (half == 1) {
 #pragma unroll
-            for (int G = 0; G < 4; ++G)
+            for (int G = 0; G < GM; ++G)
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     if (G < g16 && 16 * G + gid + ((c & 2) ? 8 : 0) < pe) *zat(G, c) = acc[G][c];
@@ -997,7 +1022,7 @@ route_fused_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16*
         __syncthreads();
         if (half == 0) {
 #pragma unroll
-            for (int G = 0; G < 4; ++G)
+            for (int G = 0; G < GM; ++G)
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     if (G < g16 && 16 * G + gid + ((c & 2) ? 8 : 0) < pe) {
@@ -1036,26 +1061,31 @@ cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const 
     // the staged operands (up to 160 KB; 188 KB for the MMA form) are dynamic
     // shared memory beside the selection's static arrays: opted in once per
     // device and variant
-    static bool attr_set[64][6] = {};
+    static bool attr_set[64][8] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (dtype == MOE_DTYPE_BF16 && route_fused_mma_ok(d, E)) {
         const int P = rm_pass_experts(d, E);
         const size_t smem = kRmRingBytes + kRmZBytes + (size_t)P * rm_row_bytes(d);
-#define MOE_FUSED_MMA(EPLV, SLOT)                                                                                    \
+#define MOE_FUSED_MMA(EPLV, GMV, SLOT)                                                                               \
     do {                                                                                                             \
         if (!attr_set[dev][SLOT]) {                                                                                  \
-            cudaError_t e_ = cudaFuncSetAttribute(route_fused_mma_kernel<EPLV>,                                      \
+            cudaError_t e_ = cudaFuncSetAttribute(route_fused_mma_kernel<EPLV, GMV>,                                 \
                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRmSmemMax);     \
             if (e_ != cudaSuccess) return e_;                                                                        \
             attr_set[dev][SLOT] = true;                                                                              \
         }                                                                                                            \
-        return launch_k(route_fused_mma_kernel<EPLV>, grid, block, smem, st, (const __nv_bfloat16*)x,                \
+        return launch_k(route_fused_mma_kernel<EPLV, GMV>, grid, block, smem, st, (const __nv_bfloat16*)x,           \
                         (const __nv_bfloat16*)W_r, bias, bias_mode, gate_mode, kk, T, d, E, k, P, logits, idx, gate, \
                         blockcnt, blockpsum, blockextra, status);                                                    \
     } while (0)
-        if (E <= 32) MOE_FUSED_MMA(1, 4);
-        MOE_FUSED_MMA(2, 5);
+        // GM: 16-row expert groups a pass needs (one up to 16 experts a pass)
+        if (E <= 32) {
+            if (P <= 16) MOE_FUSED_MMA(1, 1, 4);
+            MOE_FUSED_MMA(1, 4, 5);
+        }
+        if (P <= 16) MOE_FUSED_MMA(2, 1, 6);
+        MOE_FUSED_MMA(2, 4, 7);
 #undef MOE_FUSED_MMA
     }
 #define MOE_FUSED(TYPE, EPLV, SLOT)                                                                                  \

@@ -48,6 +48,7 @@ CASES = {
     "E40_partial_groups": (300, 512, 40, 4, 0, "bf16"),
     "E56_d1024": (257, 1024, 56, 8, 1, "bf16"),
     "E16_two_passes_d4992": (129, 4992, 16, 2, 0, "bf16"),
+    "E40_five_passes_d4992": (70, 4992, 40, 4, 1, "bf16"),
     "d6016_fma_form": (64, 6016, 8, 2, 0, "bf16"),
     "f32_E12": (100, 200, 12, 3, 1, "f32"),
     "T1": (1, 4096, 8, 2, 0, "bf16"),
