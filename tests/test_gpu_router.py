@@ -18,8 +18,8 @@ For every token of each case:
   * counts exact, P and L_aux against the oracle's statistics.
 The shapes cover the ragged edges of the MMA form: rows that end inside a
 staged 128-element item (bf16 rows are a multiple of 64), chunks of fewer
-than 32 tokens, expert counts that are not a multiple of 8 or 16, and two
-passes over x.
+than 32 tokens, expert counts that are not a multiple of 8 or 16 (one
+expert; 20 in passes of 8, 8 and 4), and up to five passes over x.
 """
 
 import math
@@ -49,6 +49,8 @@ CASES = {
     "E56_d1024": (257, 1024, 56, 8, 1, "bf16"),
     "E16_two_passes_d4992": (129, 4992, 16, 2, 0, "bf16"),
     "E40_five_passes_d4992": (70, 4992, 40, 4, 1, "bf16"),
+    "E20_three_passes_d4992": (50, 4992, 20, 3, 1, "bf16"),
+    "E1_k1": (100, 256, 1, 1, 0, "bf16"),
     "d6016_fma_form": (64, 6016, 8, 2, 0, "bf16"),
     "f32_E12": (100, 200, 12, 3, 1, "f32"),
     "T1": (1, 4096, 8, 2, 0, "bf16"),
