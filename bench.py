@@ -355,20 +355,22 @@ def config_of(cfg, args):
             "pad_rows": getattr(args, "pad_rows", 0)}
 
 
-def launches_per_forward(cfg, pad_rows=0):
-    """Kernels one moe_forward launches (the library's own choice of path)."""
+def launches_per_forward(cfg, pad_rows=0, train=0):
+    """Kernels one moe_forward launches, from the library's own choice of
+    router (moe_router_variant)."""
     if cfg["T"] == 0:
         return 1
-    small = (cfg["dtype"] == "bf16" and cfg["d_ff_shared"] == 0 and cfg["T"] * cfg["k"] <= 64
-             and cfg["E"] <= 64 and cfg["E"] % 8 == 0 and cfg["d"] % 8 == 0)
-    if small and not pad_rows:
+    import mixture_experts_layer_62_b200 as moe
+    p = moe.problem(cfg["T"], cfg["d"], cfg["d_ff"], cfg["E"], cfg["k"], cfg.get("cf", 0.0), cfg["dtype"],
+                    cfg.get("bias_mode", 0), cfg["d_ff_shared"], pad_rows=pad_rows, train=train)
+    router = moe.router_variant(p)
+    if router == "small":
         # partial router logits, routing finisher, grouped GEMM 1/3, grouped GEMM 2, combine
         return 5
-    # router: one fused kernel (logits and selection) up to 64 experts, else
-    # transpose W_r, tensor-core logits, select; then scan, permute+gather,
+    # router: one fused kernel (logits and selection), or transpose W_r,
+    # logits (tensor or CUDA cores), select; then scan, permute+gather,
     # (padding fill,) grouped GEMM 1/3, grouped GEMM 2, combine
-    wide = cfg["dtype"] == "bf16" and cfg["E"] >= 64 and cfg["E"] % 32 == 0
-    return (8 if wide else 6) + (1 if pad_rows else 0)
+    return (6 if router.startswith("fused") else 8) + (1 if pad_rows else 0)
 
 
 def time_steps(step, steps, warmup, dev, stream, flush, barrier, local_rank):
@@ -467,6 +469,7 @@ def measure_extra(name, args, moe, dev, stream, flush, peaks, peak_src, weight_c
     stages = breakdown(moe, p, cfg, L, dev, stream, flush, iters=max(3, min(10, args.steps)))
     out = {"ms_per_step": ms, "steps": steps, "tokens_per_s": cfg["T"] / (ms / 1e3), "T": cfg["T"],
            "roofline": workload_roofline(cfg, name, stages, st, peaks, peak_src, moe.gemm_variant(p)),
+           "router_variant": moe.router_variant(p),
            "pass_roofline": pass_roofline(cfg, st, ms, peaks), "stages_ms": stages, "clocks": clocks,
            "routing": {"rows": st.rows, "dropped": st.dropped, "capacity": st.capacity, "l_aux": st.l_aux,
                        "max_over_mean": st.max_over_mean, "experts_touched": touched_experts(st),
@@ -623,6 +626,7 @@ def main():
                             "first copy-in to the last copy-out; no L2 flush (the weights exceed L2)",
                 "clocks": e2e_clocks},
         "gpu_launches": launches_per_forward(cfg, args.pad_rows) * args.steps,
+        "router_variant": moe.router_variant(p),
         "clocks": clocks,
         "stages_ms": stages,
         "routing": {"rows": rows, "dropped": st.dropped, "l_aux": st.l_aux, "max_over_mean": st.max_over_mean,
@@ -813,7 +817,7 @@ def run_train(args, cfg, moe, L, dev, stream, flush):
                      "frac_of_sustained": tf_bwd / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                      "flops_per_launch": fl_bwd, "traffic": None},
         "cpu_baseline": cpu,
-        "gpu_launches": (launches_per_forward(cfg, pad) + 10 + (6 if dfs else 0)) * args.steps,
+        "gpu_launches": (launches_per_forward(cfg, pad, train=1) + 10 + (6 if dfs else 0)) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

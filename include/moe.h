@@ -359,6 +359,33 @@ long long moe_set_wait_limit(long long ns);
 #define MOE_GEMM_GEMV        6
 int moe_gemm_variant(const moe_problem* p);
 
+/* Which router a call uses for p ("Week 2 Day 2: Mixture of Experts" §1.3:
+ * z = W_r^T x, top-k, gates; the forms differ in kernels, not in results
+ * beyond the order of the fp32 sums). forward != 0: the router moe_forward
+ * uses; forward == 0: the one moe_route uses (never MOE_ROUTER_SMALL).
+ *   MOE_ROUTER_SMALL      decode-sized batches in moe_forward: partial
+ *                         logits, then one block that selects, counts,
+ *                         ranks and gathers;
+ *   MOE_ROUTER_FUSED_MMA  bf16, at most 63 experts, W_r^T of eight experts
+ *                         within the kernel's shared memory (d <= 5344):
+ *                         logits on the warp-level MMA (bf16 products, fp32
+ *                         sums) and the selection in one kernel;
+ *   MOE_ROUTER_FUSED_FMA  the same kernel layout with fp32 FMAs: fp32 up to
+ *                         64 experts and d <= 5120, bf16 rows past the MMA
+ *                         form's budget (d <= 10240), or MOE_ROUTER_MMA=0;
+ *   MOE_ROUTER_TENSOR     wide bf16 routers (E >= 64, E % 32 == 0): W_r
+ *                         transposed, logits as a tensor-core GEMM (fp32
+ *                         out), then the selection kernel;
+ *   MOE_ROUTER_SIMT       everything else: W_r transposed, logits on CUDA
+ *                         cores, then the selection kernel.
+ * A negative MOE_ERR_* code if p is invalid. Host only. */
+#define MOE_ROUTER_SMALL     0
+#define MOE_ROUTER_FUSED_MMA 1
+#define MOE_ROUTER_FUSED_FMA 2
+#define MOE_ROUTER_TENSOR    3
+#define MOE_ROUTER_SIMT      4
+int moe_router_variant(const moe_problem* p, int forward);
+
 /* Debug build. The library also builds as libmoe_debug.so (compiled with
  * MOE_DEBUG), with the same entry points and results, plus device-side bounds
  * checks that record MOE_ERR_BOUNDS in the call's status word and skip the

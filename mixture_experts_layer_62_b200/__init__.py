@@ -81,6 +81,8 @@ def _load():
     lib.moe_error_string.restype = ctypes.c_char_p
     lib.moe_gemm_variant.argtypes = [P]
     lib.moe_gemm_variant.restype = ctypes.c_int
+    lib.moe_router_variant.argtypes = [P, ctypes.c_int]
+    lib.moe_router_variant.restype = ctypes.c_int
     lib.moe_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.moe_set_wait_limit.restype = ctypes.c_longlong
     lib.moe_device_sm_count.argtypes = []
@@ -139,6 +141,18 @@ def gemm_variant(p: Problem) -> str:
     if v < 0:
         raise MoEError(-v, "moe_gemm_variant")
     return GEMM_VARIANTS[v]
+
+
+ROUTER_VARIANTS = {0: "small", 1: "fused_mma", 2: "fused_fma", 3: "tensor", 4: "simt"}
+
+
+def router_variant(p: Problem, forward: bool = True) -> str:
+    """Name of the router the library uses for p: moe_forward's (forward=True)
+    or moe_route's (moe_router_variant)."""
+    v = int(_lib().moe_router_variant(ctypes.byref(p), 1 if forward else 0))
+    if v < 0:
+        raise MoEError(-v, "moe_router_variant")
+    return ROUTER_VARIANTS[v]
 
 
 def set_wait_limit(ns: int) -> int:

@@ -520,6 +520,16 @@ int moe_gemm_variant(const moe_problem* p) {
     return MOE_GEMM_SINGLE;
 }
 
+int moe_router_variant(const moe_problem* p, int forward) {
+    const int rc = check_problem(p);
+    if (rc != MOE_OK) return -rc;
+    if (forward && small_route_ok(*p)) return MOE_ROUTER_SMALL;
+    if (router_fused(p))
+        return p->dtype == MOE_DTYPE_BF16 && route_fused_mma_ok(p->d, p->E) ? MOE_ROUTER_FUSED_MMA
+                                                                            : MOE_ROUTER_FUSED_FMA;
+    return router_on_tensor_cores(p) ? MOE_ROUTER_TENSOR : MOE_ROUTER_SIMT;
+}
+
 long long moe_set_wait_limit(long long ns) {
     return g_wait_limit_ns.exchange(ns > 0 ? ns : kDefaultWaitLimitNs);
 }

@@ -136,6 +136,7 @@ inline int count_slots(const moe_problem& p) { return p.drop_order == MOE_DROP_S
 // launch_logits_simt followed by launch_select, from x and W_r [d, E] as
 // given; resets *status (if not null) to MOE_OK.
 bool route_fused_ok(int dtype, int d, int E);
+bool route_fused_mma_ok(int d, int E);   // the bf16 fused router runs its MMA form
 cudaError_t launch_route_fused(int dtype, const void* x, const void* W_r, const float* bias, int bias_mode,
                                int gate_mode, int kk, int T, int d, int E, int k, float* logits, int32_t* idx,
                                float* gate, int32_t* blockcnt, float* blockpsum, float* blockextra, int32_t* status,

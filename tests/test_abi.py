@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -193,6 +194,41 @@ def test_gemm_variant_follows_the_shape():
     assert variant("deepseek_v3") == "single"                      # the two-class schedules are opt-in
     with pytest.raises(moe.MoEError):
         moe.gemm_variant(moe.problem(16, 256, 64, 4, 5))            # k > E
+
+
+def test_router_variant_follows_the_shape():
+    # host-side selection only (no launch): the fused router's MMA form for
+    # bf16 rows within its shared-memory budget, its FMA form for fp32 and
+    # wider rows, tensor cores for wide bf16 routers, the small-batch router
+    # in moe_forward for decode-sized batches
+    from mixture_experts_layer_62_b200 import inputs
+
+    def variant(name, forward=True, **kw):
+        c = dict(inputs.workload(name), **kw)
+        return moe.router_variant(moe.problem(c["T"], c["d"], c["d_ff"], c["E"], c["k"], c["cf"], c["dtype"],
+                                              c["bias_mode"], c["d_ff_shared"]), forward)
+    assert variant("mixtral_prefill") == "fused_mma"
+    assert variant("skewed_capacity") == "fused_mma"
+    assert variant("decode_t1") == "small"
+    assert variant("decode_t1", forward=False) == "fused_mma"      # moe_route has no small-batch path
+    assert variant("deepseek_v3") == "tensor"                      # 256 experts
+    assert variant("toy_fp32") == "fused_fma"
+    assert variant("mixtral_prefill", d=5312) == "fused_mma"       # W_r^T of 8 experts: 84.5 KB
+    assert variant("mixtral_prefill", d=5376) == "fused_fma"       # 85.5 KB: past the MMA form's budget
+    assert variant("mixtral_prefill", E=72) == "simt"              # wide, but E % 32 != 0
+    assert variant("toy_fp32", E=72) == "simt"
+    with pytest.raises(moe.MoEError):
+        moe.router_variant(moe.problem(16, 256, 64, 4, 5))          # k > E
+
+
+def test_router_mma_switch_selects_the_fma_form():
+    # MOE_ROUTER_MMA=0 is read once per process: checked in a child
+    code = ("import mixture_experts_layer_62_b200 as moe; "
+            "print(moe.router_variant(moe.problem(4096, 4096, 14336, 8, 2, 0.0, 'bf16'), False))")
+    env = dict(os.environ, MOE_ROUTER_MMA="0")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == "fused_fma"
 
 
 def test_debug_library_exports_the_same_entry_points():

@@ -47,6 +47,8 @@ def test_launch_counts():
     # the shared expert rules out the small-batch router
     assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), d_ff_shared=2048)) == 6
     assert bench.launches_per_forward(dict(inputs.workload("decode_t1"), T=0)) == 1
+    # fp32 past 64 experts: transpose, CUDA-core logits, select
+    assert bench.launches_per_forward(dict(inputs.workload("toy_fp32"), E=72)) == 8
 
 
 def test_pass_roofline_of_the_deepseek_shaped_layer():

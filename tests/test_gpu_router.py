@@ -56,6 +56,8 @@ CASES = {
     "T1": (1, 4096, 8, 2, 0, "bf16"),
 }
 FORCED_FMA = ["mixtral_4096x4096_E8", "d192_ragged_item", "E40_partial_groups"]
+# the form moe_route takes for each case (moe_router_variant)
+FMA_CASES = {"d6016_fma_form", "f32_E12"}
 
 
 def _inputs(name):
@@ -68,11 +70,15 @@ def _inputs(name):
     return x, W_r, bias
 
 
-def check_case(name):
-    """Runs moe_route on one case and checks it against the oracle."""
+def check_case(name, form=None):
+    """Runs moe_route on one case and checks it against the oracle; the
+    router form moe_route takes must be `form` (by default the one the case
+    is listed for)."""
     T, d, E, k, bm, dt = CASES[name]
     x, W_r, bias = _inputs(name)
     p = moe.problem(T, d, 64, E, k, 0.0, dt, bm)
+    want = form or ("fused_fma" if name in FMA_CASES else "fused_mma")
+    assert moe.router_variant(p, forward=False) == want, name
     ws = moe.alloc_workspace(p, DEV)
     st = moe.alloc_stats(E, DEV)
     idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
@@ -118,7 +124,7 @@ sys.path.insert(0, sys.argv[1])
 sys.path.insert(0, sys.argv[1] + "/tests")
 from test_gpu_router import check_case
 for name in sys.argv[2:]:
-    check_case(name)
+    check_case(name, form="fused_fma")
 print("ok")
 """
 
