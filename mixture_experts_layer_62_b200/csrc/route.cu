@@ -777,13 +777,15 @@ route_fused_kernel(const T* __restrict__ x, const T* __restrict__ W_r, const flo
 // The same block and selection as route_fused_kernel (one block of 8 warps
 // per chunk of kChunk tokens), with the dot products of the logits done by
 // mma.sync (m16n8k16, bf16 products exact in fp32, fp32 accumulate) instead
-// of fp32 FMAs, so the block is bound by its stream of x rather than by
-// instruction issue.
+// of fp32 FMAs: less than half the instructions. With one block of 8 warps
+// per SM, its time goes to three latency-bound phases in turn: staging
+// W_r^T, streaming x through the MMAs, and the selection.
 //
 // Operands. A is W_r^T of the pass's experts (16 expert rows per MMA; an
 // 8-row half past the pass's experts is fed as zeros, and the rows of a
-// partial half are zero-filled), kept in shared memory for the whole pass. B is 8 token rows of x. Warp w takes token octet w % 4 of the
-// chunk and the 128-element items h, h + 2, h + 4, ... of the row, h = w / 4;
+// partial half are zero-filled), kept in shared memory for the whole pass.
+// B is 8 token rows of x. Warp w takes token octet w % 4 of the chunk and
+// the 128-element items h, h + 2, h + 4, ... of the row, h = w / 4;
 // each warp streams its items through its own ring of kRmStages shared-memory
 // buffers with 16-byte cp.async copies (a half-warp copies 256 contiguous
 // bytes of one row). For a 32-element chunk at kb, lane (g, t) takes the 8
