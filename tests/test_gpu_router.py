@@ -53,11 +53,13 @@ CASES = {
     "E1_k1": (100, 256, 1, 1, 0, "bf16"),
     "d6016_fma_form": (64, 6016, 8, 2, 0, "bf16"),
     "f32_E12": (100, 200, 12, 3, 1, "f32"),
+    "f32_E40": (90, 128, 40, 4, 1, "f32"),
+    "d6016_E48_fma_form": (70, 6016, 48, 6, 0, "bf16"),
     "T1": (1, 4096, 8, 2, 0, "bf16"),
 }
 FORCED_FMA = ["mixtral_4096x4096_E8", "d192_ragged_item", "E40_partial_groups"]
 # the form moe_route takes for each case (moe_router_variant)
-FMA_CASES = {"d6016_fma_form", "f32_E12"}
+FMA_CASES = {"d6016_fma_form", "f32_E12", "f32_E40", "d6016_E48_fma_form"}
 
 
 def _inputs(name):
