@@ -251,6 +251,34 @@ def decode_bytes(cfg, st):
     return b
 
 
+def stage_bytes(cfg, rows):
+    """Algorithmic bytes of the HBM-bound stages, as their stage entry points
+    run them: route reads x and W_r and writes the fp32 logits, idx and
+    gates; permute reads x and writes the `rows` kept rows of Xp, pos and
+    row_token; combine reads those rows of O (and the shared expert's rows)
+    and writes y."""
+    T, d, E, k = cfg["T"], cfg["d"], cfg["E"], cfg["k"]
+    eb = 2 if cfg["dtype"] == "bf16" else 4
+    route = T * d * eb + d * E * eb + T * E * 4 + T * k * 8
+    permute = T * d * eb + rows * d * eb + T * k * 4 + rows * 4
+    combine = rows * d * eb + T * k * 8 + T * d * eb + (T * d * eb if cfg["d_ff_shared"] else 0)
+    return {"route": route, "permute": permute, "combine": combine}
+
+
+def hbm_stages(cfg, rows, stages_ms, peaks):
+    """Achieved HBM bandwidth of route, permute and combine: their
+    algorithmic bytes over their stage times (CUDA events around each stage
+    entry point, L2 cleared between iterations)."""
+    out = {}
+    for name, b in stage_bytes(cfg, rows).items():
+        ms = stages_ms.get(name)
+        if not ms:
+            continue
+        gbs = b / (ms / 1e3) / 1e9
+        out[name] = {"bytes": b, "ms": ms, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
+    return out
+
+
 KERNEL_NAMES = {
     "pair": ("tc_pair_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU, CTA pairs)", "tc_pair_gemm_swiglu"),
     "grid_split": ("tc_grouped_gemm<SWIGLU> (grouped GEMM 1/3 + SwiGLU, small groups on their own CTAs)",
@@ -470,7 +498,8 @@ def measure_extra(name, args, moe, dev, stream, flush, peaks, peak_src, weight_c
     out = {"ms_per_step": ms, "steps": steps, "tokens_per_s": cfg["T"] / (ms / 1e3), "T": cfg["T"],
            "roofline": workload_roofline(cfg, name, stages, st, peaks, peak_src, moe.gemm_variant(p)),
            "router_variant": moe.router_variant(p),
-           "pass_roofline": pass_roofline(cfg, st, ms, peaks), "stages_ms": stages, "clocks": clocks,
+           "pass_roofline": pass_roofline(cfg, st, ms, peaks), "stages_ms": stages,
+           "hbm_stages": hbm_stages(cfg, st.rows, stages, peaks), "clocks": clocks,
            "routing": {"rows": st.rows, "dropped": st.dropped, "capacity": st.capacity, "l_aux": st.l_aux,
                        "max_over_mean": st.max_over_mean, "experts_touched": touched_experts(st),
                        "counts": st.counts if cfg["E"] <= 16 else None,
@@ -629,6 +658,7 @@ def main():
         "router_variant": moe.router_variant(p),
         "clocks": clocks,
         "stages_ms": stages,
+        "hbm_stages": hbm_stages(cfg, rows, stages, peaks),
         "routing": {"rows": rows, "dropped": st.dropped, "l_aux": st.l_aux, "max_over_mean": st.max_over_mean,
                     "experts_touched": touched_experts(st), "counts": st.counts if E <= 16 else None,
                     "kept": st.kept if E <= 16 else None},

@@ -37,6 +37,19 @@ def test_decode_bytes_count_touched_experts_only():
     assert round(b / 1e6, 1) == 704.7
 
 
+def test_stage_bytes_of_the_mixtral_shaped_layer():
+    # route: x + W_r + fp32 logits + idx/gate; permute: x + 8192 rows of Xp
+    # + pos + row_token; combine: 8192 rows of O + idx/gate + y
+    cfg = inputs.workload("mixtral_prefill")
+    b = bench.stage_bytes(cfg, 8192)
+    assert b["route"] == 4096 * 4096 * 2 + 4096 * 8 * 2 + 4096 * 8 * 4 + 4096 * 2 * 8
+    assert b["permute"] == 4096 * 4096 * 2 + 8192 * 4096 * 2 + 4096 * 2 * 4 + 8192 * 4
+    assert b["combine"] == 8192 * 4096 * 2 + 4096 * 2 * 8 + 4096 * 4096 * 2
+    h = bench.hbm_stages(cfg, 8192, {"route": 0.02, "permute": 0.04, "combine": 0.03}, {"hbm_gbs": 6500.0})
+    assert abs(h["combine"]["gbs"] - b["combine"] / 30e-6 / 1e9) < 1e-6
+    assert abs(h["combine"]["frac"] - h["combine"]["gbs"] / 6500.0) < 1e-12
+
+
 def test_launch_counts():
     assert bench.launches_per_forward(inputs.workload("decode_t1")) == 5
     # fused router up to 64 experts: router, scan, gather, GEMM 1/3, GEMM 2, combine
